@@ -1,0 +1,92 @@
+"""UniGist prefill layout (oracle; test infrastructure only).
+
+Source: "UniGist: Towards General and Hardware-aligned Sequence-level Long
+Context Compression" (AI summary page): Approach (one-pass training with a
+unified sparse pattern of sink tokens, gist tokens and a local window; the gist
+shift trick that moves gists to the right so kernels skip non-visible blocks),
+Measured effects table (128 sink tokens; local window 128). Interleaved
+fine-grained gists and the compression ratio come from "A Silver Bullet or a
+Compromise for Full Attention? A Comprehensive Study of Gist Token-based
+Context Compression" (section 2, Preliminaries).
+
+Readings taken where the pages are silent:
+* positions 0..sinks-1 are raw sink tokens with no gists among them;
+* after the sinks a gist follows every ``ratio`` raw tokens (R..RG repeated),
+  so position p >= sinks is a gist iff (p - sinks) mod (ratio + 1) == ratio;
+* the window is a distance in logical positions: i - j < window (self
+  included); gist queries use the same rule as raw queries;
+* the gist shift acts inside each tile of ``tile`` positions: the tile's raw
+  tokens keep their order and come first, its gists follow in order.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+FULL, MASKED, TAIL = 0, 1, 2
+
+
+def gist_flags(N: int, sinks: int, ratio: int) -> np.ndarray:
+    p = np.arange(N)
+    return (p >= sinks) & ((p - sinks) % (ratio + 1) == ratio)
+
+
+def visibility(is_gist, sinks: int, window: int, rows=None) -> np.ndarray:
+    """vis[i, j] = j <= i and (j < sinks or gist(j) or i - j < window), in
+    logical positions (dense bool, optionally for some query rows only)."""
+    g = np.asarray(is_gist, bool)
+    N = len(g)
+    i = (np.arange(N) if rows is None else np.asarray(rows))[:, None]
+    j = np.arange(N)[None, :]
+    return (j <= i) & ((j < sinks) | g[None, :] | (i - j < window))
+
+
+def visible_keys(is_gist, sinks: int, window: int, i: int) -> np.ndarray:
+    """Logical key positions visible from query i (one row of visibility)."""
+    g = np.asarray(is_gist, bool)
+    j = np.arange(i + 1)
+    return j[(j < sinks) | g[: i + 1] | (i - j < window)]
+
+
+def shift_permutation(is_gist, tile: int) -> np.ndarray:
+    """perm[physical index] = logical position stored there."""
+    g = np.asarray(is_gist, bool)
+    N = len(g)
+    perm = []
+    for t0 in range(0, N, tile):
+        idx = np.arange(t0, min(N, t0 + tile))
+        perm.extend(idx[~g[idx]].tolist())
+        perm.extend(idx[g[idx]].tolist())
+    return np.asarray(perm, dtype=np.int32)
+
+
+def tile_lists(vis_phys: np.ndarray, tile: int, tail: int):
+    """Per query tile, the key tiles that hold at least one visible pair.
+
+    ``vis_phys`` is the visibility matrix in physical (shifted) order. Each
+    entry is (key tile, kind): FULL if every pair of the tile block is
+    visible, TAIL if every visible column lies in the key tile's last ``tail``
+    columns (the shifted gists), MASKED otherwise. Returned as
+    (row_ptr [T+1], key_tile [nnz], kind [nnz]) int32 with key tiles ascending.
+    """
+    N = vis_phys.shape[0]
+    T = (N + tile - 1) // tile
+    row_ptr, keys, kinds = [0], [], []
+    for I in range(T):
+        r = slice(I * tile, min(N, (I + 1) * tile))
+        for J in range(T):
+            c0, c1 = J * tile, min(N, (J + 1) * tile)
+            blk = vis_phys[r, c0:c1]
+            if not blk.any():
+                continue
+            cols = np.nonzero(blk.any(axis=0))[0]
+            if blk.all():
+                kind = FULL
+            elif cols.min() >= (c1 - c0) - tail:
+                kind = TAIL
+            else:
+                kind = MASKED
+            keys.append(J)
+            kinds.append(kind)
+        row_ptr.append(len(keys))
+    return (np.asarray(row_ptr, np.int32), np.asarray(keys, np.int32),
+            np.asarray(kinds, np.int32))

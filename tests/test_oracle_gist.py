@@ -1,0 +1,97 @@
+"""Pins for the oracle's UniGist layout (CPU only): gist counts in closed
+form, the page's compression ratio and 75% memory figure, visible-key counts,
+reductions to dense causal and self-only attention, the shift permutation
+against NumPy's stable sort, and the tile lists' closed-form structure."""
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import attention as A
+from oracle import gist as Gi
+
+GOLD = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "page_values.json")))
+
+
+def test_gist_count_and_ratio():
+    g = Gi.gist_flags(32768, 128, 4)
+    assert g.sum() == 6528 and (~g).sum() == 26240
+    assert not g[:128].any()
+    gold = GOLD["kv_reduction_at_ratio_4"]
+    body = Gi.gist_flags(4000, 0, gold["ratio"])
+    raw_per_gist = (~body).sum() / body.sum()
+    assert raw_per_gist == gold["ratio"]
+    assert 1 - 1 / raw_per_gist == gold["reduction"]
+
+
+def test_visible_key_count_closed_form():
+    S, W, N = GOLD["unigist_sinks_and_window"]["sinks"], GOLD["unigist_sinks_and_window"]["window"], 3000
+    g = Gi.gist_flags(N, S, 4)
+    for i in (255, 256, 700, 1234, 2999):
+        n_gist = (i - 128 - 128 + 1) // 5
+        assert len(Gi.visible_keys(g, S, W, i)) == S + n_gist + W
+    vis = Gi.visibility(g, S, W, rows=[300, 2999])
+    assert vis.sum(1).tolist() == [len(Gi.visible_keys(g, S, W, i)) for i in (300, 2999)]
+
+
+def test_wide_window_is_dense_causal_and_unit_window_is_self():
+    N = 200
+    g = Gi.gist_flags(N, 16, 4)
+    assert np.array_equal(Gi.visibility(g, 16, N), np.tril(np.ones((N, N), bool)))
+    g0 = Gi.gist_flags(N, 0, N)  # no gists at all
+    assert not g0.any()
+    vis = Gi.visibility(g0, 0, 1)
+    assert np.array_equal(vis, np.eye(N, dtype=bool))
+    rng = np.random.default_rng(0)
+    q, k, v = rng.standard_normal((3, N, 8))
+    assert np.array_equal(A.forward(q, k, v, vis)[0], v)
+
+
+def test_gist_attention_matches_torch_sdpa():
+    N, d = 300, 16
+    g = Gi.gist_flags(N, 8, 4)
+    vis = Gi.visibility(g, 8, 16)
+    rng = np.random.default_rng(1)
+    q, k, v = rng.standard_normal((3, N, d))
+    o, _ = A.forward(q, k, v, vis)
+    t = lambda x: torch.from_numpy(x)[None, None]
+    ref = torch.nn.functional.scaled_dot_product_attention(t(q), t(k), t(v),
+                                                           attn_mask=torch.from_numpy(vis)[None, None])
+    np.testing.assert_allclose(o, ref[0, 0].numpy(), atol=1e-12)
+
+
+@pytest.mark.parametrize("N,tile", [(32768, 128), (1000, 128), (77, 16)])
+def test_shift_permutation_is_stable_partition_per_tile(N, tile):
+    g = Gi.gist_flags(N, 128 if N > 1000 else 5, 4)
+    perm = Gi.shift_permutation(g, tile)
+    assert sorted(perm.tolist()) == list(range(N))
+    for t0 in range(0, N, tile):
+        idx = np.arange(t0, min(N, t0 + tile))
+        want = idx[np.argsort(g[idx].astype(np.int8), kind="stable")]
+        assert np.array_equal(perm[idx], want)
+
+
+def test_tile_lists_structure():
+    # tiles of 128 positions, 128 sinks, ratio 4, window 128, 32-wide tail
+    N, tile = 128 * 12 + 77, 128
+    g = Gi.gist_flags(N, 128, 4)
+    perm = Gi.shift_permutation(g, tile)
+    vis = Gi.visibility(g, 128, 128)[np.ix_(perm, perm)]
+    rp, kt, kd = Gi.tile_lists(vis, tile, 32)
+    T = (N + tile - 1) // tile
+    for I in range(T):
+        got = list(zip(kt[rp[I]:rp[I + 1]].tolist(), kd[rp[I]:rp[I + 1]].tolist()))
+        if I == 0:
+            want = [(0, Gi.MASKED)]
+        elif I == 1:
+            want = [(0, Gi.FULL), (1, Gi.MASKED)]
+        else:
+            want = [(0, Gi.FULL)] + [(J, Gi.TAIL) for J in range(1, I - 1)] + \
+                   [(I - 1, Gi.MASKED), (I, Gi.MASKED)]
+        assert got == want, I
+    # every gist of a full tile sits in its last 32 columns after the shift
+    for t0 in range(tile, N - tile, tile):
+        gp = g[perm[t0:t0 + tile]]
+        assert gp[-32:].sum() == gp.sum() and gp.sum() in (25, 26)
