@@ -124,3 +124,45 @@ def forward_rows(q, k, v, keys_of_row, rows, scale=None):
         o[n] = np.exp(s - l) @ np.asarray(v[keys], np.float64)
         lse[n] = l
     return o, lse
+
+
+def _row_terms(q, k, v, do, keys, p, scale):
+    """Softmax row p over `keys`: (P, O_p, D_p) in float64."""
+    kk = np.asarray(k[keys], np.float64)
+    s = (kk @ np.asarray(q[p], np.float64)) * scale
+    m = s.max()
+    P = np.exp(s - (m + np.log(np.exp(s - m).sum())))
+    o = P @ np.asarray(v[keys], np.float64)
+    return P, o, float(np.asarray(do[p], np.float64) @ o)
+
+
+def backward_rows(q, k, v, do, keys_of_row, rows, scale=None):
+    """dQ for selected query rows only: dQ_p = sum_j dS_pj k_j * scale with
+    dS_pj = P_pj (dO_p . v_j - D_p) over the keys row p may attend."""
+    scale = 1.0 / np.sqrt(q.shape[1]) if scale is None else float(scale)
+    out = np.empty((len(rows), k.shape[1]), np.float64)
+    for n, p in enumerate(rows):
+        keys = np.asarray(keys_of_row(int(p)))
+        P, _, D = _row_terms(q, k, v, do, keys, p, scale)
+        dP = np.asarray(v[keys], np.float64) @ np.asarray(do[p], np.float64)
+        out[n] = ((P * (dP - D)) @ np.asarray(k[keys], np.float64)) * scale
+    return out
+
+
+def backward_cols(q, k, v, do, keys_of_row, rows_of_key, cols, scale=None):
+    """dK and dV for selected keys only: sums over the query rows that attend
+    key j of dS_pj q_p * scale and P_pj dO_p."""
+    scale = 1.0 / np.sqrt(q.shape[1]) if scale is None else float(scale)
+    dk = np.zeros((len(cols), k.shape[1]))
+    dv = np.zeros((len(cols), v.shape[1]))
+    vj_all = np.asarray(v, np.float64)
+    for n, j in enumerate(cols):
+        for p in rows_of_key(int(j)):
+            keys = np.asarray(keys_of_row(int(p)))
+            P, _, D = _row_terms(q, k, v, do, keys, p, scale)
+            pj = P[np.searchsorted(keys, j)]
+            dop = np.asarray(do[p], np.float64)
+            ds = pj * (dop @ vj_all[j] - D)
+            dk[n] += ds * np.asarray(q[p], np.float64) * scale
+            dv[n] += pj * dop
+    return dk, dv

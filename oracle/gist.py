@@ -59,29 +59,33 @@ def shift_permutation(is_gist, tile: int) -> np.ndarray:
     return np.asarray(perm, dtype=np.int32)
 
 
-def tile_lists(vis_phys: np.ndarray, tile: int, tail: int):
+def tile_lists(vis_phys, tile: int, tail: int, N: int | None = None):
     """Per query tile, the key tiles that hold at least one visible pair.
 
     ``vis_phys`` is the visibility matrix in physical (shifted) order. Each
     entry is (key tile, kind): FULL if every pair of the tile block is
-    visible, TAIL if every visible column lies in the key tile's last ``tail``
-    columns (the shifted gists), MASKED otherwise. Returned as
+    visible, TAIL if every visible column lies in the last ``tail`` of the
+    tile's ``tile`` nominal columns (where the shift puts a full tile's
+    gists), MASKED otherwise. Returned as
     (row_ptr [T+1], key_tile [nnz], kind [nnz]) int32 with key tiles ascending.
+    ``vis_phys`` may also be a callable rows -> bool [len(rows), N] (then N
+    must be given), evaluated one query tile at a time.
     """
-    N = vis_phys.shape[0]
+    N = vis_phys.shape[0] if N is None else N
     T = (N + tile - 1) // tile
     row_ptr, keys, kinds = [0], [], []
     for I in range(T):
-        r = slice(I * tile, min(N, (I + 1) * tile))
+        rows = np.arange(I * tile, min(N, (I + 1) * tile))
+        vrows = vis_phys(rows) if callable(vis_phys) else vis_phys[rows]
         for J in range(T):
             c0, c1 = J * tile, min(N, (J + 1) * tile)
-            blk = vis_phys[r, c0:c1]
+            blk = vrows[:, c0:c1]
             if not blk.any():
                 continue
             cols = np.nonzero(blk.any(axis=0))[0]
             if blk.all():
                 kind = FULL
-            elif cols.min() >= (c1 - c0) - tail:
+            elif cols.min() >= tile - tail:
                 kind = TAIL
             else:
                 kind = MASKED

@@ -124,3 +124,38 @@ def bitmask(mask: np.ndarray) -> np.ndarray:
         for j in np.nonzero(mask[i])[0]:
             out[i, j // 32] |= np.uint32(1) << np.uint32(j % 32)
     return out
+
+
+def tile_lists(block_mask: np.ndarray, b: int, tile: int = 128):
+    """Tile-level lists of the token mask: for every query tile I (rows
+    [tile*I, tile*I + tile)), the key tiles J holding at least one allowed
+    pair, ascending, with kind 0 (every pair of the tile block allowed) or
+    1 (some pair not allowed). Returned as (row_ptr [T+1], key_tile [nnz],
+    kind [nnz]) int32 and computed from the dense token mask one query tile
+    at a time."""
+    N = block_mask.shape[0] * b
+    T = (N + tile - 1) // tile
+    row_ptr, keys, kinds = [0], [], []
+    for I in range(T):
+        tm = token_mask(block_mask, b, rows=np.arange(I * tile, min(N, I * tile + tile)))
+        for J in range(T):
+            blk = tm[:, J * tile:min(N, J * tile + tile)]
+            if blk.any():
+                keys.append(J)
+                kinds.append(0 if blk.all() else 1)
+        row_ptr.append(len(keys))
+    return (np.asarray(row_ptr, np.int32), np.asarray(keys, np.int32),
+            np.asarray(kinds, np.int32))
+
+
+def transpose_lists(row_ptr, cols, kinds, n_cols):
+    """CSR (row -> ascending cols, kind) to CSC (col -> ascending rows, kind)."""
+    ent = []
+    for r in range(len(row_ptr) - 1):
+        for e in range(row_ptr[r], row_ptr[r + 1]):
+            ent.append((int(cols[e]), r, int(kinds[e])))
+    ent.sort()
+    counts = np.bincount([c for c, _, _ in ent], minlength=n_cols)
+    ptr = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    return (ptr, np.asarray([r for _, r, _ in ent], np.int32),
+            np.asarray([k for _, _, k in ent], np.int32))

@@ -114,3 +114,18 @@ def test_backward_matches_torch_autograd_and_invariants():
     P = A.probabilities(q, k, allowed)
     dP = do @ v.T
     np.testing.assert_allclose((P * dP).sum(1), (do * o).sum(1), atol=1e-12)
+
+
+def test_row_and_column_forms_of_backward_agree_with_dense():
+    N, b, d = 64, 8, 16
+    flags = (np.random.default_rng(22).random(N // b) < 0.5).astype(np.uint8)
+    allowed = G.token_mask(G.block_masks(flags, 1)[G.HYBRID], b)
+    q, k, v, do = (_rand(s, N, d) for s in (23, 24, 25, 26))
+    dq, dk, dv, _, _ = A.backward(q, k, v, do, allowed)
+    keys_of = lambda p: np.nonzero(allowed[p])[0]
+    rows_of = lambda j: np.nonzero(allowed[:, j])[0]
+    sel = [0, 9, 40, 63]
+    np.testing.assert_allclose(A.backward_rows(q, k, v, do, keys_of, sel), dq[sel], atol=1e-12)
+    dk2, dv2 = A.backward_cols(q, k, v, do, keys_of, rows_of, sel)
+    np.testing.assert_allclose(dk2, dk[sel], atol=1e-12)
+    np.testing.assert_allclose(dv2, dv[sel], atol=1e-12)

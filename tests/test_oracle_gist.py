@@ -95,3 +95,13 @@ def test_tile_lists_structure():
     for t0 in range(tile, N - tile, tile):
         gp = g[perm[t0:t0 + tile]]
         assert gp[-32:].sum() == gp.sum() and gp.sum() in (25, 26)
+
+
+def test_tile_lists_row_callable_matches_dense():
+    N = 600
+    g = Gi.gist_flags(N, 16, 4)
+    perm = Gi.shift_permutation(g, 128)
+    dense = Gi.visibility(g, 16, 40)[np.ix_(perm, perm)]
+    fn = lambda rows: Gi.visibility(g, 16, 40, rows=perm[rows])[:, perm]
+    for a, b in zip(Gi.tile_lists(dense, 128, 32), Gi.tile_lists(fn, 128, 32, N=N)):
+        assert np.array_equal(a, b)

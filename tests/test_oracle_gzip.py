@@ -153,3 +153,29 @@ def test_lists_and_bits():
         assert ri[cp[i]:cp[i + 1]].tolist() == [r for r in range(70) if m[r, i]]
         for j in range(70):
             assert bool((int(bits[i, j // 32]) >> (j % 32)) & 1) == bool(m[i, j])
+
+
+def test_tile_lists_closed_forms():
+    # b = 128: tile lists equal block lists, diagonal masked, others full
+    flags = (np.random.default_rng(12).random(20) < 0.3).astype(np.uint8)
+    m = G.block_masks(flags, 2)[G.HYBRID]
+    rp, kt, kd = G.tile_lists(m, 128)
+    brp, bci = G.csr(m)
+    assert np.array_equal(rp, brp) and np.array_equal(kt, bci)
+    assert all(kd[e] == (1 if kt[e] == i else 0) for i in range(20) for e in range(rp[i], rp[i + 1]))
+    # b = 64, local class, w = 2: query tile I covers blocks 2I, 2I+1 whose union
+    # reaches back to block 2I-2 -> key tiles I-1 (not all pairs) and I (diag)
+    m = G.block_masks(np.zeros(16, np.uint8), 2)[G.LOCAL]
+    rp, kt, kd = G.tile_lists(m, 64)
+    for I in range(8):
+        got = list(zip(kt[rp[I]:rp[I + 1]].tolist(), kd[rp[I]:rp[I + 1]].tolist()))
+        assert got == ([(I - 1, 1)] if I else []) + [(I, 1)]
+    # b = 256: two tiles per block; all-literal -> dense causal at tile level
+    m = G.block_masks(np.ones(4, np.uint8), 0)[G.LITERAL]
+    rp, kt, kd = G.tile_lists(m, 256)
+    for I in range(8):
+        assert kt[rp[I]:rp[I + 1]].tolist() == list(range(I + 1))
+        assert kd[rp[I]:rp[I + 1]].tolist() == [0] * I + [1]
+    cp, ri, rk = G.transpose_lists(rp, kt, kd, 8)
+    for J in range(8):
+        assert ri[cp[J]:cp[J + 1]].tolist() == list(range(J, 8))
