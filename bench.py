@@ -1,0 +1,516 @@
+#!/usr/bin/env python
+"""Benchmark of the block-sparse attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one pass of the workload's hot path over one batch of synthetic,
+seeded input already resident in HBM:
+  gzip_8k            mask build + forward      (default; batch 8, N=8192, b=64)
+  gzip_64k_fwdbwd    mask build + forward + backward (batch 2, N=65536, b=128)
+  gist_prefill_32k   layout build + forward    (N=32768, 32q/8kv heads)
+  gist_decode_128k   one decode step           (16 seqs, 131072-token caches)
+Prefill/backward workloads report visited-tile TFLOP/s (every visited block
+pair counted as a full b x b tile: 4*d*b^2 forward, 10*d*b^2 backward); the
+decode workload reports algorithmic HBM GB/s. Inputs are larger than the
+126 MB L2, so no flush is needed between steps. Under torchrun each rank runs
+its own independent copy of the workload (weak scaling, no collective on the
+data path); the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import sa_workloads as W  # noqa: E402
+
+METRIC = "visited-tile attn TFLOP/s & % bf16 tensor peak; gist-decode HBM GB/s"
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d["hbm_gbs"], d["bf16_tflops"], "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+# --------------------------------------------------------------- clocks
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index, self.proc, self.lines = index, None, []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            threading.Thread(target=self._read, daemon=True).start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        self.proc.wait(timeout=5)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, val in zip(names, f[5:9]):
+                if val.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------- workloads
+_host_out = {}
+
+
+def copy_out(tensors):
+    """Device -> pinned host copies of a step's results (reused buffers)."""
+    outs = []
+    for t in tensors:
+        key = (t.data_ptr(), t.numel(), t.dtype)
+        if key not in _host_out:
+            _host_out[key] = t.new_empty(t.shape, device="cpu").pin_memory()
+        _host_out[key].copy_(t, non_blocking=True)
+        outs.append(_host_out[key])
+    return outs
+
+class GzipWorkload:
+    def __init__(self, sa, torch, name, backward, rank):
+        self.sa, self.torch, self.backward = sa, torch, backward
+        w = dict(W.WORKLOADS[name])
+        if rank:
+            w["index"] = w["index"] + 1000 * rank  # an independent copy per rank
+        self.w = w
+        Bt, N, H, d, b = w["batch"], w["seq_len"], w["heads"], w["head_dim"], w["block"]
+        if w.get("flags_from") == "bernoulli":
+            flags = W.bernoulli_flags(w)
+        else:
+            flags = np.stack([sa.literal_flags(W.workload_bytes(w, i), b) for i in range(Bt)])
+        self.h_flags = torch.from_numpy(flags).pin_memory()
+        mk = lambda t: torch.from_numpy(np.stack([W.qkv(w, t, i) for i in range(Bt)])).to(torch.bfloat16)
+        self.h_in = {t: mk(t).pin_memory() for t in (["q", "k", "v"] + (["do"] if backward else []))}
+        dev = {t: x.cuda() for t, x in self.h_in.items()}
+        self.q, self.k, self.v = dev["q"], dev["k"], dev["v"]
+        self.do = dev.get("do")
+        self.flags = self.h_flags.cuda()
+        self.md = sa.gzip_mask(Bt, N, b, w["window"], H)
+        self.lists = sa.BlockLists(self.md)
+        self.build_ws = sa._workspace(256, "cuda")
+        self.o = torch.empty_like(self.q)
+        self.lse = torch.empty(Bt, H, N, dtype=torch.float32, device="cuda")
+        self.ad = sa.attn_desc(self.q, self.k, self.v, self.o)
+        self.fws = sa.forward_workspace(self.ad, self.md)
+        if backward:
+            self.dq = torch.empty(self.q.shape, dtype=torch.float32, device="cuda")
+            self.dk = torch.empty_like(self.dq)
+            self.dv = torch.empty_like(self.dq)
+            self.bws = sa.backward_workspace(self.ad, self.md)
+        self.step()
+        torch.cuda.synchronize()
+        # visited block pairs per (batch, class) from the lists just built
+        B = N // b
+        rp = self.lists.row_ptr.cpu().numpy().reshape(Bt * 3, B + 1)
+        nnz = rp[:, -1] - rp[:, 0]
+        cls = [0] * (H // 2) + [1] * (H // 4) + [2] * (H - H // 2 - H // 4)
+        pairs = sum(int(nnz[bt * 3 + c]) for bt in range(Bt) for c in cls)
+        self.pairs = pairs
+        self.flops_fwd = 4.0 * d * b * b * pairs
+        self.flops = self.flops_fwd * (1 + (2.5 if backward else 0))
+        self.kernels_per_step = 2 + (3 if backward else 0)
+        self.unit = "TFLOP/s"
+
+    def fwd_only(self):
+        self.sa.sa_forward(self.ad, self.md, self.q, self.k, self.v, self.lists, self.o, self.lse,
+                           self.fws)
+
+    def step(self, ev=None):
+        sa = self.sa
+        sa.sa_build_block_mask(self.md, self.flags, self.lists, self.build_ws)
+        if ev is not None:
+            ev[0].record()
+        self.fwd_only()
+        if ev is not None:
+            ev[1].record()
+        if self.backward:
+            sa.sa_backward(self.ad, self.md, self.q, self.k, self.v, self.o, self.lse, self.do,
+                           self.lists, self.dq, self.dk, self.dv, self.bws)
+
+    def e2e_step(self):
+        """Host buffers in, result out: the public API with H2D/D2H copies."""
+        for t, h in self.h_in.items():
+            getattr(self, t).copy_(h, non_blocking=True)
+        self.flags.copy_(self.h_flags, non_blocking=True)
+        self.step()
+        out = [self.o, self.lse] + ([self.dq, self.dk, self.dv] if self.backward else [])
+        return copy_out(out)
+
+    def io_bytes(self):
+        h2d = sum(x.numel() * x.element_size() for x in self.h_in.values()) + self.h_flags.numel()
+        d2h = self.o.numel() * 2 + self.lse.numel() * 4
+        if self.backward:
+            d2h += 3 * self.dq.numel() * 4
+        return h2d, d2h
+
+    def cpu_baseline(self, heads=None):
+        """The oracle on batch row 0, one head of each class (whole heads)."""
+        from oracle import attention as A
+        from oracle import gzip_mask as G
+        w, b = self.w, self.w["block"]
+        flags = G.literal_flags(W.workload_bytes(w, 0), b) if w.get("flags_from") != "bernoulli" \
+            else W.bernoulli_flags(w)[0]
+        masks = G.block_masks(flags, w["window"])
+        H = w["heads"]
+        heads = [0, H // 2, H - 1] if heads is None else heads
+        cls = G.head_classes(H)
+        t0 = time.perf_counter()
+        flops = 0.0
+        for h in heads:
+            bm = masks[cls[h]]
+            q, k, v = (W.qkv(w, t, 0, head=h) for t in ("q", "k", "v"))
+            mask = lambda rows: G.token_mask(bm, b, rows=rows)
+            if self.backward:
+                do = W.qkv(w, "do", 0, head=h)
+                A.backward(q, k, v, do, mask)
+            else:
+                A.forward(q, k, v, mask)
+            flops += (4.0 + (10.0 if self.backward else 0.0)) * w["head_dim"] * b * b * int(bm.sum())
+        dt = time.perf_counter() - t0
+        return flops / dt / 1e12, f"batch row 0, heads {heads} (one per class), whole heads, fp64", dt
+
+
+class GistWorkload(GzipWorkload):
+    def __init__(self, sa, torch, name, rank):
+        self.sa, self.torch, self.backward = sa, torch, False
+        w = dict(W.WORKLOADS[name])
+        if rank:
+            w["index"] = w["index"] + 1000 * rank
+        self.w = w
+        N, H, Hkv, d = w["seq_len"], w["heads"], w["kv_heads"], w["head_dim"]
+        self.h_in = {t: torch.from_numpy(W.qkv(w, t, 0)[None]).to(torch.bfloat16).pin_memory()
+                     for t in ("q", "k", "v")}
+        self.q, self.k, self.v = (self.h_in[t].cuda() for t in ("q", "k", "v"))
+        self.md = sa.gist_mask(N, H, w["sinks"], w["ratio"], w["window"], gist_tail=w["gist_tail"])
+        self.lists = sa.BlockLists(self.md)
+        self.flags = None
+        self.h_flags = torch.zeros(1, dtype=torch.uint8)
+        self.build_ws = sa._workspace(256, "cuda")
+        self.o = torch.empty_like(self.q)
+        self.lse = torch.empty(1, H, N, dtype=torch.float32, device="cuda")
+        self.ad = sa.attn_desc(self.q, self.k, self.v, self.o)
+        self.fws = sa.forward_workspace(self.ad, self.md)
+        self.step()
+        torch.cuda.synchronize()
+        T = (N + 127) // 128
+        rp = self.lists.tile_row_ptr.cpu().numpy()
+        kinds = self.lists.tile_kind.cpu().numpy()[: rp[-1]]
+        width = np.where(kinds == 2, w["gist_tail"], 128)
+        self.flops_fwd = 4.0 * d * H * 128 * float(width.sum())
+        self.flops = self.flops_fwd
+        self.kernels_per_step = 2
+        self.unit = "TFLOP/s"
+
+    def e2e_step(self):
+        for t, h in self.h_in.items():
+            getattr(self, t).copy_(h, non_blocking=True)
+        self.step()
+        return copy_out([self.o, self.lse])
+
+    def cpu_baseline(self):
+        from oracle import attention as A
+        from oracle import gist as Gi
+        w = self.w
+        N = w["seq_len"]
+        g = Gi.gist_flags(N, w["sinks"], w["ratio"])
+        perm = Gi.shift_permutation(g, 128)
+        inv = np.empty_like(perm)
+        inv[perm] = np.arange(N)
+        rows = np.arange(N - 2048, N)  # the last 2048 logical query rows of head 0
+        q = W.qkv(w, "q", 0, head=0)[inv]
+        k = W.qkv(w, "k", 0, head=0)[inv]
+        v = W.qkv(w, "v", 0, head=0)[inv]
+        t0 = time.perf_counter()
+        A.forward(q[rows], k, v, lambda r: Gi.visibility(g, w["sinks"], w["window"], rows=rows[r]))
+        dt = time.perf_counter() - t0
+        # algorithmic FLOPs of those rows: exact visible pairs x 4d
+        n_vis = int(Gi.visibility(g, w["sinks"], w["window"], rows=rows).sum())
+        return 4.0 * w["head_dim"] * n_vis / dt / 1e12, \
+            "head 0, last 2048 query rows, exact visible pairs, fp64", dt
+
+
+class DecodeWorkload:
+    def __init__(self, sa, torch, name, rank):
+        self.sa, self.torch = sa, torch
+        w = dict(W.WORKLOADS[name])
+        if rank:
+            w["index"] = w["index"] + 1000 * rank
+        self.w = w
+        n, Hkv, L, d, G = w["n_seq"], w["kv_heads"], w["cache_len"], w["head_dim"], w["n_gists"]
+        self.kc = torch.empty(n, Hkv, L, d, dtype=torch.bfloat16, device="cuda")
+        self.vc = torch.empty_like(self.kc)
+        from concurrent.futures import ThreadPoolExecutor
+
+        def one(i):
+            s, g = divmod(i, Hkv)
+            return i, W.decode_raw(w, s, g, "k"), W.decode_raw(w, s, g, "v")
+
+        with ThreadPoolExecutor(8) as ex:
+            for i, rk, rv in ex.map(one, range(n * Hkv)):
+                s, g = divmod(i, Hkv)
+                self.kc[s, g] = torch.from_numpy(rk).to("cuda", torch.bfloat16)
+                self.vc[s, g] = torch.from_numpy(rv).to("cuda", torch.bfloat16)
+        bf = lambda a: torch.from_numpy(a).to(torch.bfloat16)
+        self.h_q = bf(W.decode_query(w)).pin_memory()
+        self.h_gk = bf(np.stack([W.decode_gists(w, s, "k") for s in range(n)])).pin_memory()
+        self.h_gv = bf(np.stack([W.decode_gists(w, s, "v") for s in range(n)])).pin_memory()
+        self.q, self.gk, self.gv = self.h_q.cuda(), self.h_gk.cuda(), self.h_gv.cuda()
+        self.o = torch.empty_like(self.q)
+        self.lse = torch.empty(n, w["heads"], dtype=torch.float32, device="cuda")
+        self.sel = torch.empty(n, Hkv, w["top_k"], dtype=torch.int32, device="cuda")
+        self.dd = sa.decode_desc(self.q, self.gk, self.kc, self.o, w["chunk"], w["top_k"], w["window"])
+        self.ws = sa.decode_workspace(self.dd)
+        self.step()
+        torch.cuda.synchronize()
+        per = (G + w["top_k"] * w["chunk"] + w["window"]) * d * 2 * 2
+        self.bytes = float(n * Hkv * per + 2 * self.q.numel() * 2 + self.lse.numel() * 4
+                           + self.sel.numel() * 4)
+        self.kernels_per_step = 4
+        self.unit = "GB/s"
+
+    def step(self, ev=None):
+        if ev is not None:
+            ev[0].record()
+        self.sa.sa_gist_decode(self.dd, self.q, self.gk, self.gv, self.kc, self.vc, self.sel, self.o,
+                               self.lse, self.ws)
+        if ev is not None:
+            ev[1].record()
+
+    def e2e_step(self):
+        # the new token's query and the sequence's gist K/V come from the host
+        self.q.copy_(self.h_q, non_blocking=True)
+        self.gk.copy_(self.h_gk, non_blocking=True)
+        self.gv.copy_(self.h_gv, non_blocking=True)
+        self.step()
+        return copy_out([self.o, self.lse, self.sel])
+
+    def io_bytes(self):
+        h2d = sum(x.numel() * 2 for x in (self.h_q, self.h_gk, self.h_gv))
+        return h2d, self.o.numel() * 2 + self.lse.numel() * 4 + self.sel.numel() * 4
+
+    def cpu_baseline(self):
+        from oracle import decode as D
+        w = self.w
+        q = W.decode_query(w)[0]
+        gk, gv = W.decode_gists(w, 0, "k"), W.decode_gists(w, 0, "v")
+        rk = [W.decode_raw(w, 0, g, "k") for g in range(w["kv_heads"])]
+        rv = [W.decode_raw(w, 0, g, "v") for g in range(w["kv_heads"])]
+        raw_k, raw_v = (lambda g: rk[g]), (lambda g: rv[g])
+        t0 = time.perf_counter()
+        D.decode_one(q, gk, gv, raw_k, raw_v, w["chunk"], w["window"], w["top_k"])
+        dt = time.perf_counter() - t0
+        per = (w["n_gists"] + w["top_k"] * w["chunk"] + w["window"]) * w["head_dim"] * 2 * 2
+        return w["kv_heads"] * per / dt / 1e9, \
+            "sequence 0, all kv heads (raw cache generation excluded), fp64", dt
+
+
+def make(sa, torch, name, rank):
+    if name.startswith("gzip"):
+        return GzipWorkload(sa, torch, name, name.endswith("fwdbwd"), rank)
+    if name.startswith("gist_prefill"):
+        return GistWorkload(sa, torch, name, rank)
+    return DecodeWorkload(sa, torch, name, rank)
+
+
+# ----------------------------------------------------------------- main
+def run_reference(args):
+    """The oracle on the host cores, on a bounded sample of the workload."""
+    import torch
+
+    class Stub:
+        pass
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    torch.set_num_threads(len(os.sched_getaffinity(0)))
+    wl = Stub()
+    wl.w = dict(W.WORKLOADS[args.workload])
+    wl.backward = args.workload.endswith("fwdbwd")
+    cls = {"gzip": GzipWorkload, "gist": GistWorkload, "deco": DecodeWorkload}
+    fn = cls[args.workload[:4]].cpu_baseline
+    vals = []
+    H = wl.w["heads"]
+    for i in range(args.warmup + args.steps):
+        if args.workload.startswith("gzip"):
+            # one whole head per step, cycling through the three classes
+            v, sample, dt = fn(wl, heads=[(0, H // 2, H - 1)[i % 3]])
+            sample = "batch row 0, one whole head per step cycling local/literal/hybrid, fp64"
+        else:
+            v, sample, dt = fn(wl)
+        if i >= args.warmup:
+            vals.append((v, dt))
+    value = float(np.mean([v for v, _ in vals]))
+    unit = "GB/s" if args.workload.startswith("gist_decode") else "TFLOP/s"
+    cores = len(os.sched_getaffinity(0))
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": unit, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": float(np.mean([dt for _, dt in vals]) * 1e3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": args.workload},
+        "cpu_baseline": {"value": value, "unit": unit, "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}))
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="gzip_8k",
+                    choices=["gzip_8k", "gzip_64k_fwdbwd", "gist_prefill_32k", "gist_decode_128k"])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+
+    import content_adaptive_block_sa_b200 as sa
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], device="cuda", dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    wl = make(sa, torch, args.workload, rank)
+    for _ in range(args.warmup):
+        wl.step()
+    torch.cuda.synchronize()
+
+    # ---- device-timed region: K steps, inputs resident
+    fwd_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for i in range(args.steps):
+        wl.step(fwd_ev[i])
+    t1.record()
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    ms = max_over_ranks(t0.elapsed_time(t1)) / args.steps
+    kern_ms = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in fwd_ev])))
+
+    # ---- end-to-end through the public API with host buffers
+    for _ in range(2):
+        wl.e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        outs = wl.e2e_step()
+    e1.record()
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1)) / args.steps
+    h2d, d2h = wl.io_bytes()
+
+    hbm, bf16, src = peaks()
+    if wl.unit == "GB/s":
+        units = wl.bytes
+        value = units * world / (ms * 1e-3) / 1e9
+        e2e_value = units * world / (e2e_ms * 1e-3) / 1e9
+        ach = wl.bytes / (kern_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
+                "traffic": None, "peak_source": src, "kernel": "sa_gist_decode (4 launches)"}
+    else:
+        value = wl.flops * world / (ms * 1e-3) / 1e12
+        e2e_value = wl.flops * world / (e2e_ms * 1e-3) / 1e12
+        ach = wl.flops_fwd / (kern_ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": ach, "peak": bf16, "unit": "TFLOP/s",
+                "frac": ach / bf16, "traffic": None, "peak_source": src, "kernel": "sa_forward"}
+    if rank != 0:
+        if world > 1:
+            dist.destroy_process_group()
+        return
+    line = {
+        "metric": METRIC, "value": value, "unit": wl.unit, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "fp32" if wl.w.get("dtype") == "fp32" else "bf16",
+        "data": "synthetic (seeded generators in sa_workloads)",
+        "config": {"workload": args.workload, "l2": "inputs larger than L2, no flush",
+                   "parallelism": f"independent replica per rank x{world}"},
+        "roofline": roof, "clocks": clk,
+        "e2e": {"value": e2e_value, "unit": wl.unit, "h2d_bytes_per_step": int(h2d),
+                "d2h_bytes_per_step": int(d2h)},
+        "gpu_launches": int(wl.kernels_per_step * args.steps),
+        "kernel_ms": kern_ms,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        torch.set_num_threads(len(os.sched_getaffinity(0)))
+        v, sample, dt = wl.cpu_baseline()
+        line["cpu_baseline"] = {"value": v, "unit": wl.unit, "cores": len(os.sched_getaffinity(0)),
+                                "kind": "oracle", "sample": sample, "seconds": dt}
+    print(json.dumps(line))
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,355 @@
+// Gist-scored selective unfolding at decode.
+//
+// "Simplified Sparse Attention via Gist Tokens" (abstract): the current query
+// is scored against the small set of gist keys only, the top-k chunks are
+// unfolded by bringing back their raw tokens, and attention runs over them;
+// "Forget, Then Recall: ... Gist Sparse Attention" (abstract): compress into
+// gists, select the most relevant gists, restore the corresponding raw chunks.
+//
+// Per (sequence, KV head g) with query heads h in the group:
+//   1. gist pass (split over gist slices): s_h,c = q_h . gk_c * scale for
+//      every gist c; the selection score sum_h s_h,c goes to the workspace and
+//      the same logits feed the gist part of the attention as a partial
+//      (max m, sum l, unnormalised o) per head and slice. Gist K and V are
+//      streamed once.
+//   2. select: top_k eligible chunks (wholly before the window) by score,
+//      ties to the lower index, written ascending (-1 padded).
+//   3. raw pass (split over the unfolded keys): the same partials over the
+//      raw tokens of the selected chunks followed by the last `window`
+//      tokens.
+//   4. combine the partials of every slice into O (bf16) and LSE (fp32).
+// Keys and values are read with 16-byte loads, 16 lanes per 256-byte row.
+#include "sa_common.cuh"
+
+namespace sa {
+
+constexpr int kDecD = 128;
+constexpr int kDecMaxRep = 8;   // query heads per KV head
+constexpr int kGistSlice = 256;
+constexpr int kRawSlice = 256;
+constexpr int kDecThreads = 128;
+
+struct DecodeArgs {
+  const __nv_bfloat16 *q, *gk, *gv, *kc, *vc;
+  int32_t* sel;
+  __nv_bfloat16* o;
+  float* lse;
+  float* scores;   // [n_seq, Hkv, G]
+  float* part;     // [n_seq, Hq, n_part, 2 + D]
+  int n_seq, cache_len, chunk, G, top_k, window, Hq, Hkv, rep;
+  int n_gslices, n_rslices, n_part;
+  float scale;
+  int64_t qs[2], gs[3], cs[3], os[2];
+};
+
+__device__ __forceinline__ void bf16x8_to_float(const uint4& u, float* f) {
+  const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 t = __bfloat1622float2(b[i]);
+    f[2 * i] = t.x;
+    f[2 * i + 1] = t.y;
+  }
+}
+
+// Online-softmax state of one half-warp for the group's heads; each lane
+// holds 8 of the 128 output dimensions.
+template <int REP>
+struct HalfState {
+  float m[REP], l[REP], o[REP][8];
+  __device__ void init() {
+#pragma unroll
+    for (int h = 0; h < REP; ++h) {
+      m[h] = -INFINITY;
+      l[h] = 0.f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) o[h][i] = 0.f;
+    }
+  }
+};
+
+// Processes keys [e0, e1) of a key list given by `row` (returns k/v row
+// pointers) and writes one partial per head to `out` (slot `slot`).
+template <int REP, typename RowFn>
+__device__ void attend_slice(const DecodeArgs& a, const float (*qf)[kDecD], int e0, int e1,
+                             RowFn row, float* score_out, int seq, int g, int slot) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int half = lane >> 4, hl = lane & 15;  // 16 lanes per key row
+  HalfState<REP> st;
+  st.init();
+  float qreg[REP][8];
+#pragma unroll
+  for (int h = 0; h < REP; ++h)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) qreg[h][i] = qf[h][hl * 8 + i];
+  const int nw = blockDim.x >> 5;
+  for (int base = e0 + warp * 2; base < e1; base += nw * 2) {
+    const int e = base + half;
+    const bool valid = e < e1;
+    float kf[8], vf[8];
+    if (valid) {
+      const __nv_bfloat16 *kr, *vr;
+      row(e, kr, vr);
+      bf16x8_to_float(*reinterpret_cast<const uint4*>(kr + hl * 8), kf);
+      bf16x8_to_float(*reinterpret_cast<const uint4*>(vr + hl * 8), vf);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) kf[i] = vf[i] = 0.f;
+    }
+    float s[REP];
+    float ssum = 0.f;
+#pragma unroll
+    for (int h = 0; h < REP; ++h) {
+      float t = 0.f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) t = fmaf(qreg[h][i], kf[i], t);
+#pragma unroll
+      for (int off = 8; off > 0; off >>= 1) t += __shfl_xor_sync(0xffffffffu, t, off);
+      s[h] = t * a.scale;
+      ssum += s[h];
+    }
+    if (valid && score_out != nullptr && hl == 0) score_out[e] = ssum;
+    if (!valid) continue;
+#pragma unroll
+    for (int h = 0; h < REP; ++h) {
+      const float mnew = fmaxf(st.m[h], s[h]);
+      const float alpha = expf(st.m[h] - mnew);
+      const float p = expf(s[h] - mnew);
+      st.l[h] = st.l[h] * alpha + p;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) st.o[h][i] = fmaf(p, vf[i], st.o[h][i] * alpha);
+      st.m[h] = mnew;
+    }
+  }
+  // combine the 2 * nwarps half-warp states through shared memory
+  __shared__ float red_m[8][kDecMaxRep], red_l[8][kDecMaxRep];
+  __shared__ float red_o[kDecMaxRep][kDecD];
+  const int hw = warp * 2 + half;  // 0..7
+  if (hl == 0)
+#pragma unroll
+    for (int h = 0; h < REP; ++h) { red_m[hw][h] = st.m[h]; red_l[hw][h] = st.l[h]; }
+  for (int x = threadIdx.x; x < REP * kDecD; x += blockDim.x) red_o[x / kDecD][x % kDecD] = 0.f;
+  __syncthreads();
+  float M[REP], scale_me[REP];
+#pragma unroll
+  for (int h = 0; h < REP; ++h) {
+    M[h] = -INFINITY;
+    for (int t = 0; t < 2 * nw; ++t) M[h] = fmaxf(M[h], red_m[t][h]);
+    scale_me[h] = (st.m[h] == -INFINITY) ? 0.f : expf(st.m[h] - M[h]);
+  }
+#pragma unroll
+  for (int h = 0; h < REP; ++h)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) atomicAdd(&red_o[h][hl * 8 + i], st.o[h][i] * scale_me[h]);
+  __syncthreads();
+  for (int x = threadIdx.x; x < REP * kDecD; x += blockDim.x) {
+    const int h = x / kDecD, c = x % kDecD;
+    float* dst = a.part + (((int64_t)seq * a.Hq + g * a.rep + h) * a.n_part + slot) * (2 + kDecD);
+    dst[2 + c] = red_o[h][c];
+    if (c == 0) {
+      float L = 0.f;
+      for (int t = 0; t < 2 * nw; ++t)
+        if (red_m[t][h] != -INFINITY) L += red_l[t][h] * expf(red_m[t][h] - M[h]);
+      dst[0] = M[h];
+      dst[1] = L;
+    }
+  }
+}
+
+__device__ void load_group_q(const DecodeArgs& a, int seq, int g, float (*qf)[kDecD]) {
+  for (int x = threadIdx.x; x < a.rep * kDecD; x += blockDim.x) {
+    const int h = x / kDecD, c = x % kDecD;
+    qf[h][c] = __bfloat162float(a.q[seq * a.qs[0] + (int64_t)(g * a.rep + h) * a.qs[1] + c]);
+  }
+  __syncthreads();
+}
+
+template <int REP>
+__global__ void __launch_bounds__(kDecThreads) decode_gist_kernel(DecodeArgs a) {
+  __shared__ float qf[kDecMaxRep][kDecD];
+  const int slice = blockIdx.x, g = blockIdx.y, seq = blockIdx.z;
+  load_group_q(a, seq, g, qf);
+  const __nv_bfloat16* gk = a.gk + seq * a.gs[0] + (int64_t)g * a.gs[1];
+  const __nv_bfloat16* gv = a.gv + seq * a.gs[0] + (int64_t)g * a.gs[1];
+  const int64_t rs = a.gs[2];
+  auto row = [&](int e, const __nv_bfloat16*& kr, const __nv_bfloat16*& vr) {
+    kr = gk + e * rs;
+    vr = gv + e * rs;
+  };
+  const int e0 = slice * kGistSlice, e1 = min(a.G, e0 + kGistSlice);
+  float* sc = a.scores + ((int64_t)seq * a.Hkv + g) * a.G;
+  attend_slice<REP>(a, qf, e0, e1, row, sc, seq, g, slice);
+}
+
+// Order-preserving map of a float to an unsigned key.
+__device__ __forceinline__ uint32_t float_key(float f) {
+  const uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__global__ void __launch_bounds__(1024) decode_select_kernel(DecodeArgs a, int pow2) {
+  extern __shared__ unsigned long long keys[];
+  __shared__ int chosen[256];
+  const int g = blockIdx.x, seq = blockIdx.y;
+  const float* sc = a.scores + ((int64_t)seq * a.Hkv + g) * a.G;
+  const int last_ok = a.cache_len - a.window;  // chunk c eligible iff (c+1)*chunk <= last_ok
+  for (int i = threadIdx.x; i < pow2; i += blockDim.x) {
+    unsigned long long kk = 0ull;
+    if (i < a.G && (int64_t)(i + 1) * a.chunk <= last_ok)
+      kk = ((unsigned long long)float_key(sc[i]) << 32) | (0xFFFFFFFFu - (uint32_t)i);
+    keys[i] = kk;
+  }
+  __syncthreads();
+  // bitonic sort, descending
+  for (int size = 2; size <= pow2; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int i = threadIdx.x; i < pow2; i += blockDim.x) {
+        const int j = i ^ stride;
+        if (j > i) {
+          const bool desc = (i & size) == 0;
+          const unsigned long long x = keys[i], y = keys[j];
+          if ((x < y) == desc) { keys[i] = y; keys[j] = x; }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  const int k = a.top_k;
+  for (int t = threadIdx.x; t < k; t += blockDim.x)
+    chosen[t] = (t < pow2 && keys[t] != 0ull) ? (int)(0xFFFFFFFFu - (uint32_t)(keys[t] & 0xFFFFFFFFull))
+                                              : 0x7FFFFFFF;
+  __syncthreads();
+  int32_t* out = a.sel + ((int64_t)seq * a.Hkv + g) * k;
+  for (int t = threadIdx.x; t < k; t += blockDim.x) {
+    const int v = chosen[t];
+    int rank = 0;
+    for (int u = 0; u < k; ++u) rank += chosen[u] < v || (chosen[u] == v && u < t);
+    out[rank] = (v == 0x7FFFFFFF) ? -1 : v;
+  }
+}
+
+template <int REP>
+__global__ void __launch_bounds__(kDecThreads) decode_raw_kernel(DecodeArgs a) {
+  __shared__ float qf[kDecMaxRep][kDecD];
+  __shared__ int sel_s[256];
+  __shared__ int n_sel_s;
+  const int slice = blockIdx.x, g = blockIdx.y, seq = blockIdx.z;
+  const int32_t* sel = a.sel + ((int64_t)seq * a.Hkv + g) * a.top_k;
+  for (int t = threadIdx.x; t < a.top_k; t += blockDim.x) sel_s[t] = sel[t];
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int n = 0;
+    for (int t = 0; t < a.top_k; ++t) n += sel_s[t] >= 0;
+    n_sel_s = n;
+  }
+  load_group_q(a, seq, g, qf);
+  const int n_chunk_keys = n_sel_s * a.chunk;
+  const int total = n_chunk_keys + a.window;
+  const __nv_bfloat16* kc = a.kc + seq * a.cs[0] + (int64_t)g * a.cs[1];
+  const __nv_bfloat16* vc = a.vc + seq * a.cs[0] + (int64_t)g * a.cs[1];
+  const int64_t rs = a.cs[2];
+  const int chunk = a.chunk, wstart = a.cache_len - a.window;
+  auto row = [&](int e, const __nv_bfloat16*& kr, const __nv_bfloat16*& vr) {
+    const int pos = e < n_chunk_keys ? sel_s[e / chunk] * chunk + e % chunk
+                                     : wstart + (e - n_chunk_keys);
+    kr = kc + pos * rs;
+    vr = vc + pos * rs;
+  };
+  const int e0 = min(total, slice * kRawSlice), e1 = min(total, e0 + kRawSlice);
+  attend_slice<REP>(a, qf, e0, e1, row, nullptr, seq, g, a.n_gslices + slice);
+}
+
+__global__ void decode_combine_kernel(DecodeArgs a) {
+  const int h = blockIdx.x, seq = blockIdx.y, c = threadIdx.x;  // 128 threads
+  const float* p = a.part + ((int64_t)seq * a.Hq + h) * a.n_part * (2 + kDecD);
+  float M = -INFINITY;
+  for (int t = 0; t < a.n_part; ++t) M = fmaxf(M, p[t * (2 + kDecD)]);
+  float L = 0.f, acc = 0.f;
+  for (int t = 0; t < a.n_part; ++t) {
+    const float* q = p + t * (2 + kDecD);
+    if (q[0] == -INFINITY) continue;
+    const float w = expf(q[0] - M);
+    L += q[1] * w;
+    acc += q[2 + c] * w;
+  }
+  a.o[seq * a.os[0] + (int64_t)h * a.os[1] + c] = __float2bfloat16_rn(acc / L);
+  if (c == 0) a.lse[(int64_t)seq * a.Hq + h] = M + logf(L);
+}
+
+// ------------------------------------------------------------- host side
+struct DecodePlan {
+  int n_gslices, n_rslices, n_part, pow2;
+  size_t scores_off, part_off, bytes;
+};
+
+DecodePlan decode_plan(const sa_decode_desc& d) {
+  DecodePlan p{};
+  p.n_gslices = (d.n_gists + kGistSlice - 1) / kGistSlice;
+  const int max_raw = d.top_k * d.chunk + d.window;
+  p.n_rslices = max(1, (max_raw + kRawSlice - 1) / kRawSlice);
+  p.n_part = p.n_gslices + p.n_rslices;
+  p.pow2 = 1;
+  while (p.pow2 < d.n_gists) p.pow2 <<= 1;
+  p.scores_off = kStatusBytes;
+  size_t sb = (size_t)d.n_seq * d.num_kv_heads * d.n_gists * sizeof(float);
+  p.part_off = p.scores_off + ((sb + 255) / 256) * 256;
+  size_t pb = (size_t)d.n_seq * d.num_q_heads * p.n_part * (2 + kDecD) * sizeof(float);
+  p.bytes = p.part_off + pb;
+  return p;
+}
+
+template <int REP>
+static cudaError_t decode_launch_rep(const DecodeArgs& a, const DecodePlan& pl, cudaStream_t s) {
+  decode_gist_kernel<REP><<<dim3(pl.n_gslices, a.Hkv, a.n_seq), kDecThreads, 0, s>>>(a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const size_t smem = (size_t)pl.pow2 * sizeof(unsigned long long);
+  if (smem > 48 * 1024) {
+    e = cudaFuncSetAttribute(decode_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  decode_select_kernel<<<dim3(a.Hkv, a.n_seq), 1024, smem, s>>>(a, pl.pow2);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  decode_raw_kernel<REP><<<dim3(pl.n_rslices, a.Hkv, a.n_seq), kDecThreads, 0, s>>>(a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  decode_combine_kernel<<<dim3(a.Hq, a.n_seq), kDecD, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_decode(const sa_decode_desc& d, const void* q, const void* gk, const void* gv,
+                          const void* kc, const void* vc, int32_t* sel, void* o, float* lse,
+                          void* ws, cudaStream_t s) {
+  const DecodePlan pl = decode_plan(d);
+  DecodeArgs a{};
+  a.q = (const __nv_bfloat16*)q;
+  a.gk = (const __nv_bfloat16*)gk;
+  a.gv = (const __nv_bfloat16*)gv;
+  a.kc = (const __nv_bfloat16*)kc;
+  a.vc = (const __nv_bfloat16*)vc;
+  a.sel = sel;
+  a.o = (__nv_bfloat16*)o;
+  a.lse = lse;
+  a.scores = (float*)((char*)ws + pl.scores_off);
+  a.part = (float*)((char*)ws + pl.part_off);
+  a.n_seq = d.n_seq; a.cache_len = d.cache_len; a.chunk = d.chunk; a.G = d.n_gists;
+  a.top_k = d.top_k; a.window = d.window; a.Hq = d.num_q_heads; a.Hkv = d.num_kv_heads;
+  a.rep = d.num_q_heads / d.num_kv_heads;
+  a.n_gslices = pl.n_gslices; a.n_rslices = pl.n_rslices; a.n_part = pl.n_part;
+  a.scale = d.softmax_scale > 0.f ? d.softmax_scale : 1.f / sqrtf((float)d.head_dim);
+  for (int i = 0; i < 2; ++i) { a.qs[i] = d.q_strides[i]; a.os[i] = d.o_strides[i]; }
+  for (int i = 0; i < 3; ++i) { a.gs[i] = d.gist_strides[i]; a.cs[i] = d.cache_strides[i]; }
+  switch (a.rep) {
+    case 1: return decode_launch_rep<1>(a, pl, s);
+    case 2: return decode_launch_rep<2>(a, pl, s);
+    case 4: return decode_launch_rep<4>(a, pl, s);
+    case 8: return decode_launch_rep<8>(a, pl, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+size_t decode_workspace_bytes(const sa_decode_desc& d) { return decode_plan(d).bytes; }
+
+}  // namespace sa

@@ -1,0 +1,81 @@
+"""sa_backward vs the oracle: dQ, dK, dV element by element on small cases;
+at the 64K workload sampled dQ rows, sampled dK/dV keys, and the identities
+sum_j dK_j = 0 and sum_j dV_j = sum_p dO_p that hold at any size."""
+import numpy as np
+import pytest
+import torch
+
+import sa_workloads as W
+from oracle import attention as A
+from oracle import gzip_mask as G
+
+from _cases import check_close, gzip_flags_oracle, gzip_flags_product, gzip_inputs, to_dev, to_np
+
+pytestmark = pytest.mark.gpu
+
+
+def run(sa, w, q, k, v, do, flags):
+    dt = w["dtype"]
+    md = sa.gzip_mask(w["batch"], w["seq_len"], w["block"], w["window"], w["heads"])
+    lists = sa.build_block_mask(md, flags)
+    tq, tk, tv, tdo = (to_dev(x, dt) for x in (q, k, v, do))
+    o, lse = sa.forward(tq, tk, tv, md, lists)
+    dq, dk, dv = sa.backward(tq, tk, tv, o, lse, tdo, md, lists)
+    torch.cuda.synchronize()
+    return to_np(o), to_np(dq), to_np(dk), to_np(dv)
+
+
+@pytest.mark.parametrize("w", [
+    W.scaled("gzip_8k", index=301, batch=2, seq_len=16 * 24, block=16, window=1, heads=4,
+             kv_heads=4, head_dim=32, dtype="fp32"),
+    W.scaled("gzip_8k", index=302, batch=1, seq_len=64 * 11, block=64, window=2, heads=4,
+             kv_heads=4, head_dim=64, dtype="bf16"),
+    W.scaled("gzip_8k", index=303, batch=1, seq_len=128 * 6, block=128, window=1, heads=4,
+             kv_heads=4, head_dim=128, dtype="bf16", p_literal=0.5),
+], ids=["b16_fp32", "b64_ragged_bf16", "b128_bf16"])
+def test_backward_small(sa, w):
+    q, k, v, do = gzip_inputs(w, with_do=True)
+    fp, fo = gzip_flags_product(sa, w), gzip_flags_oracle(w)
+    o, dq, dk, dv = run(sa, w, q, k, v, do, fp)
+    cls = G.head_classes(w["heads"])
+    for bt in range(w["batch"]):
+        masks = G.block_masks(fo[bt], w["window"])
+        for h in range(w["heads"]):
+            allowed = G.token_mask(masks[cls[h]], w["block"])
+            # the oracle's upstream gradient is the one the kernel was given
+            rq, rk, rv, _, _ = A.backward(q[bt, :, h], k[bt, :, h], v[bt, :, h], do[bt, :, h], allowed)
+            check_close(dq[bt, :, h], rq, w["dtype"], f"dQ b{bt} h{h}")
+            check_close(dk[bt, :, h], rk, w["dtype"], f"dK b{bt} h{h}")
+            check_close(dv[bt, :, h], rv, w["dtype"], f"dV b{bt} h{h}")
+
+
+def test_backward_full_size(sa):
+    w = W.WORKLOADS["gzip_64k_fwdbwd"]
+    q, k, v, do = gzip_inputs(w, with_do=True)
+    fp, fo = gzip_flags_product(sa, w), gzip_flags_oracle(w)
+    o, dq, dk, dv = run(sa, w, q, k, v, do, fp)
+    assert all(np.isfinite(x).all() for x in (dq, dk, dv))
+    b, B = w["block"], w["seq_len"] // w["block"]
+    cls = G.head_classes(w["heads"])
+    rng = np.random.default_rng(0)
+    for bt in range(w["batch"]):
+        masks = G.block_masks(fo[bt], w["window"])
+        # identities over all keys of every head (any size)
+        np.testing.assert_allclose(dk[bt].sum(0), 0, atol=0.5)
+        np.testing.assert_allclose(dv[bt].sum(0), do[bt].astype(np.float64).sum(0), rtol=1e-3, atol=0.5)
+        for h in (0, w["heads"] // 2, w["heads"] - 1):
+            bm = masks[cls[h]]
+            keys_of = lambda p: np.nonzero(G.token_mask(bm, b, rows=[p])[0])[0]
+            rows = np.unique(np.concatenate([[0, 127, 128, w["seq_len"] - 1], rng.choice(w["seq_len"], 6)]))
+            rq = A.backward_rows(q[bt, :, h], k[bt, :, h], v[bt, :, h], do[bt, :, h], keys_of, rows)
+            check_close(dq[bt, rows, h], rq, "bf16", f"dQ rows b{bt} h{h}")
+            # keys whose block is seen only by nearby query blocks (cheap to sum)
+            lit = fo[bt].astype(bool)
+            cheap = [j for j in range(B) if not (lit[j] and cls[h] != G.LOCAL) or
+                     lit[j] and not lit[j + 1:].any()]
+            jb = [cheap[0], cheap[len(cheap) // 2], cheap[-1]]
+            cols = np.array([x * b + o_ for x in jb for o_ in (0, 77)])
+            rows_of = lambda j: np.nonzero(G.token_mask(bm, b, rows=np.arange(j, min(w["seq_len"], j + (w["window"] + 2) * b)))[:, j])[0] + j
+            rk, rv = A.backward_cols(q[bt, :, h], k[bt, :, h], v[bt, :, h], do[bt, :, h], keys_of, rows_of, cols)
+            check_close(dk[bt, cols, h], rk, "bf16", f"dK cols b{bt} h{h}")
+            check_close(dv[bt, cols, h], rv, "bf16", f"dV cols b{bt} h{h}")

@@ -1,0 +1,83 @@
+"""sa_gist_decode vs the oracle: the selected chunks (exact, except where the
+oracle's k-th and (k+1)-th scores are closer than float32 rounding can
+resolve), and O / LSE over the selected key set."""
+import numpy as np
+import pytest
+import torch
+from concurrent.futures import ThreadPoolExecutor
+
+import sa_workloads as W
+from oracle import decode as D
+
+from _cases import check_close, to_np
+
+pytestmark = pytest.mark.gpu
+
+
+def upload_workload(w):
+    """Device tensors [n_seq, Hkv, L, d] for raw K/V, [n_seq, Hkv, G, d] gists."""
+    n, Hkv, L, d = w["n_seq"], w["kv_heads"], w["cache_len"], w["head_dim"]
+    kc = torch.empty(n, Hkv, L, d, dtype=torch.bfloat16, device="cuda")
+    vc = torch.empty_like(kc)
+
+    def one(i):
+        s, g = divmod(i, Hkv)
+        return i, W.decode_raw(w, s, g, "k"), W.decode_raw(w, s, g, "v")
+
+    with ThreadPoolExecutor(8) as ex:
+        for i, rk, rv in ex.map(one, range(n * Hkv)):
+            s, g = divmod(i, Hkv)
+            kc[s, g] = torch.from_numpy(rk).to("cuda", torch.bfloat16)
+            vc[s, g] = torch.from_numpy(rv).to("cuda", torch.bfloat16)
+    gk = np.stack([W.decode_gists(w, s, "k") for s in range(n)])
+    gv = np.stack([W.decode_gists(w, s, "v") for s in range(n)])
+    q = W.decode_query(w)
+    dev = lambda x: torch.from_numpy(x).to("cuda", torch.bfloat16)
+    return q, gk, gv, dev(q), dev(gk), dev(gv), kc, vc
+
+
+def check(sa, w, seqs=None):
+    q, gk, gv, tq, tgk, tgv, kc, vc = upload_workload(w)
+    sel, o, lse = sa.gist_decode(tq, tgk, tgv, kc, vc, w["chunk"], w["top_k"], w["window"])
+    torch.cuda.synchronize()
+    sel, o, lse = sel.cpu().numpy(), to_np(o), to_np(lse)
+    rep = w["heads"] // w["kv_heads"]
+    for s in (range(w["n_seq"]) if seqs is None else seqs):
+        raw_k = lambda g: to_np(kc[s, g])
+        raw_v = lambda g: to_np(vc[s, g])
+        osel, oo, ol, scores = D.decode_one(q[s], gk[s], gv[s], raw_k, raw_v, w["chunk"],
+                                            w["window"], w["top_k"])
+        for g in range(w["kv_heads"]):
+            if not np.array_equal(sel[s, g], osel[g]):
+                # accept a different set only across a float32-level near tie
+                elig = D.eligible_chunks(w["n_gists"], w["chunk"], w["cache_len"], w["window"])
+                sc = np.where(elig, scores[g], -np.inf)
+                kth = np.sort(sc)[::-1][[w["top_k"] - 1, w["top_k"]]]
+                assert abs(kth[0] - kth[1]) < 1e-5 * max(1.0, abs(kth[0])), (s, g, sel[s, g], osel[g])
+                # O must then match the oracle evaluated on the GPU's own set
+                pos = D.raw_key_positions(sel[s, g], w["chunk"], w["cache_len"], w["window"])
+                keys = np.concatenate([gk[s, g], raw_k(g)[pos]])
+                vals = np.concatenate([gv[s, g], raw_v(g)[pos]])
+                for h in range(g * rep, (g + 1) * rep):
+                    oo[h], ol[h] = D.attend(q[s, h], keys, vals, 1 / np.sqrt(w["head_dim"]))
+        check_close(o[s], oo, "bf16", f"O seq {s}")
+        check_close(lse[s], ol, "bf16", f"LSE seq {s}")
+
+
+@pytest.mark.parametrize("top_k,window,chunk,G", [(8, 64, 16, 64), (0, 64, 16, 64), (60, 64, 16, 64),
+                                                  (5, 0, 32, 40), (3, 100, 8, 300)])
+def test_decode_small(sa, top_k, window, chunk, G):
+    w = W.scaled("gist_decode_128k", index=400 + top_k + G, n_seq=3, cache_len=chunk * G,
+                 chunk=chunk, n_gists=G, top_k=top_k, window=window, heads=8, kv_heads=2)
+    check(sa, w)
+
+
+@pytest.mark.parametrize("rep", [1, 8])
+def test_decode_group_sizes(sa, rep):
+    w = W.scaled("gist_decode_128k", index=450 + rep, n_seq=2, cache_len=32 * 128, chunk=32,
+                 n_gists=128, top_k=16, window=128, heads=2 * rep, kv_heads=2)
+    check(sa, w)
+
+
+def test_decode_full_size(sa):
+    check(sa, W.WORKLOADS["gist_decode_128k"], seqs=[0, 7, 15])
