@@ -167,7 +167,7 @@ def _dtype_code(t: torch.Tensor) -> int:
     raise TypeError(f"unsupported dtype {t.dtype}")
 
 
-def attn_desc(q, k, v, o, softmax_scale: float = 0.0) -> _abi.sa_attn_desc:
+def attn_desc(q, k, v, o, softmax_scale: float = 0.0, impl: int = 0) -> _abi.sa_attn_desc:
     """Descriptor from [Bt, N, H, d] tensors (any strides, last dim contiguous)."""
     Bt, N, Hq, d = q.shape
     st = lambda t: (i64 * 3)(t.stride(0), t.stride(1), t.stride(2))
@@ -176,7 +176,8 @@ def attn_desc(q, k, v, o, softmax_scale: float = 0.0) -> _abi.sa_attn_desc:
             raise ValueError("head_dim must be contiguous")
     return _abi.sa_attn_desc(dtype=_dtype_code(q), batch=Bt, seq_len=N, num_q_heads=Hq,
                              num_kv_heads=k.shape[2], head_dim=d, softmax_scale=softmax_scale,
-                             q_strides=st(q), k_strides=st(k), v_strides=st(v), o_strides=st(o))
+                             q_strides=st(q), k_strides=st(k), v_strides=st(v), o_strides=st(o),
+                             impl=impl)
 
 
 i64 = C.c_int64
@@ -195,11 +196,12 @@ def forward_workspace(adesc, mdesc, device="cuda") -> torch.Tensor:
     return _workspace(n.value, device)
 
 
-def forward(q, k, v, mdesc, lists: BlockLists, softmax_scale: float = 0.0, stream=None):
+def forward(q, k, v, mdesc, lists: BlockLists, softmax_scale: float = 0.0, stream=None,
+            impl: int = 0):
     """O [Bt, N, Hq, d] (dtype of q) and LSE fp32 [Bt, Hq, N]."""
     o = torch.empty_like(q)
     lse = torch.empty(q.shape[0], q.shape[2], q.shape[1], dtype=torch.float32, device=q.device)
-    ad = attn_desc(q, k, v, o, softmax_scale)
+    ad = attn_desc(q, k, v, o, softmax_scale, impl)
     ws = forward_workspace(ad, mdesc, q.device)
     sa_forward(ad, mdesc, q, k, v, lists, o, lse, ws, stream)
     return o, lse
@@ -218,14 +220,15 @@ def backward_workspace(adesc, mdesc, device="cuda") -> torch.Tensor:
     return _workspace(n.value, device)
 
 
-def backward(q, k, v, o, lse, dout, mdesc, lists, softmax_scale: float = 0.0, stream=None):
+def backward(q, k, v, o, lse, dout, mdesc, lists, softmax_scale: float = 0.0, stream=None,
+             impl: int = 0):
     """fp32 dQ [Bt, N, Hq, d], dK and dV [Bt, N, Hkv, d]. dout has o's strides."""
     if dout.stride() != o.stride():
         raise ValueError("dout must have the same strides as o")
     dq = torch.empty(q.shape, dtype=torch.float32, device=q.device)
     dk = torch.empty(k.shape, dtype=torch.float32, device=q.device)
     dv = torch.empty(v.shape, dtype=torch.float32, device=q.device)
-    ad = attn_desc(q, k, v, o, softmax_scale)
+    ad = attn_desc(q, k, v, o, softmax_scale, impl)
     ws = backward_workspace(ad, mdesc, q.device)
     sa_backward(ad, mdesc, q, k, v, o, lse, dout, lists, dq, dk, dv, ws, stream)
     return dq, dk, dv

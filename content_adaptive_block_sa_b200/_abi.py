@@ -16,6 +16,7 @@ SA_CLASS_LOCAL, SA_CLASS_LITERAL, SA_CLASS_HYBRID = 0, 1, 2
 SA_DTYPE_BF16, SA_DTYPE_FP32 = 0, 1
 SA_TILE_FULL, SA_TILE_MASKED, SA_TILE_TAIL = 0, 1, 2
 SA_SELECT_SUM_LOGITS_PER_GROUP = 0
+SA_IMPL_AUTO, SA_IMPL_CUDA_CORES, SA_IMPL_TENSOR_CORES = 0, 1, 2
 SA_TILE = 128
 
 i32, i64, f32, vp = C.c_int32, C.c_int64, C.c_float, C.c_void_p
@@ -43,7 +44,7 @@ class sa_attn_desc(C.Structure):
     _fields_ = [("dtype", i32), ("batch", i32), ("seq_len", i64), ("num_q_heads", i32),
                 ("num_kv_heads", i32), ("head_dim", i32), ("softmax_scale", f32),
                 ("q_strides", i64 * 3), ("k_strides", i64 * 3), ("v_strides", i64 * 3),
-                ("o_strides", i64 * 3)]
+                ("o_strides", i64 * 3), ("impl", i32)]
 
 
 class sa_decode_desc(C.Structure):

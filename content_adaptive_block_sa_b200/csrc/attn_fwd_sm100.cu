@@ -1,0 +1,386 @@
+// Block-sparse attention forward on the 5th-generation tensor cores (sm_100a).
+//
+// For one (128-query tile, head, sequence) per CTA, the listed 128-key tiles
+// are visited in order; everything else is skipped ("UniGist ...", Approach:
+// skipping non-visible blocks is what makes the sparse layout fast; "Gzip-
+// guided sparse attention ...", Scope: dense-then-mask gives no speed-up).
+//
+// Roles (192 threads):
+//   warp 0      TMA producer: Q once, then K_j / V_j into a 2-stage ring
+//               (128-byte swizzled, 64-column atoms), and TMEM allocation.
+//   warp 1      one thread issues tcgen05.mma: S_j = Q K_j^T into one of two
+//               TMEM S buffers, then O += P_j V_j into the TMEM O accumulator.
+//               Completion is signalled with tcgen05.commit on mbarriers.
+//   warps 2-5   softmax: thread t owns query row t (TMEM lane t). It reads its
+//               S row, applies the element mask on MASKED/TAIL tiles, keeps a
+//               running max in the log2 domain and rescales its O row only
+//               when the max grew by more than 2^8 (the reference max is kept
+//               otherwise, so P <= 256), writes P (bf16) into a swizzled
+//               shared tile and hands it to the MMA thread. The epilogue
+//               divides O by the row sum and writes O (bf16) and LSE (fp32).
+// S is double-buffered so that S_{j+1} = Q K_{j+1}^T runs on the tensor core
+// while the softmax of tile j runs. Every wait is bounded; on timeout the
+// device status word is set and all roles leave after draining their copies
+// and MMAs, freeing TMEM.
+#include <cuda.h>
+
+#include "attn_mask.cuh"
+#include "sm100.cuh"
+
+namespace sa {
+
+using namespace sm100;
+
+struct FwdTcParams {
+  CUtensorMap tmq, tmk, tmv;
+  AttnArgs a;
+  MaskArgs m;
+};
+
+template <int D>
+struct FwdLayout {
+  static constexpr uint32_t kQ = 128 * D * 2;       // Q tile
+  static constexpr uint32_t kKV = 128 * D * 2;      // one K or V tile
+  static constexpr uint32_t kP = 128 * 128 * 2;     // one P tile
+  static constexpr uint32_t kAtom = 128 * 128;      // [128 rows][64 bf16] swizzle atom
+  static constexpr uint32_t q = 0;
+  static constexpr uint32_t k0 = kQ;
+  static constexpr uint32_t v0 = kQ + 2 * kKV;
+  static constexpr uint32_t p0 = kQ + 4 * kKV;
+  static constexpr uint32_t bars = p0 + 2 * kP;
+  static constexpr uint32_t bytes = bars + 256 + 1024;  // + alignment slack
+};
+
+enum { B_Q = 0, B_KVF = 1, B_KVE = 3, B_SF = 5, B_SE = 7, B_PF = 9, B_OD = 11, B_DRAIN = 13 };
+
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kTmemO = 256;
+
+template <int D>
+__global__ void __launch_bounds__(192, 1) fwd_tc_kernel(const __grid_constant__ FwdTcParams P) {
+  using L = FwdLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  const uint32_t sb = smem_u32(smem);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + L::bars);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 16);
+  volatile int* abort = reinterpret_cast<volatile int*>(bar + 16) + 1;
+
+  const AttnArgs& a = P.a;
+  const MaskArgs& m = P.m;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int T = m.T;
+  const int I = T - 1 - (int)blockIdx.x;  // long lists (late tiles) first
+  const int h = blockIdx.y, bt = blockIdx.z;
+  const int hk = h / (a.Hq / a.Hkv);
+  const int list = list_of(m, bt, h);
+  const int e0 = m.trp[list * (T + 1) + I];
+  const int n = m.trp[list * (T + 1) + I + 1] - e0;
+  const int q0 = I * kTile;
+  DeviceStatus* st = a.status;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bar[B_Q], 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bar[B_KVF + s], 1);
+      mbar_init(&bar[B_KVE + s], 1);
+      mbar_init(&bar[B_SF + s], 1);
+      mbar_init(&bar[B_SE + s], 128);
+      mbar_init(&bar[B_PF + s], 128);
+      mbar_init(&bar[B_OD + s], 1);
+    }
+    mbar_init(&bar[B_DRAIN], 1);
+    *abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------ TMA producer
+      prefetch_tmap(&P.tmq);
+      prefetch_tmap(&P.tmk);
+      prefetch_tmap(&P.tmv);
+      mbar_arrive_expect_tx(&bar[B_Q], L::kQ);
+      for (int at = 0; at < D / 64; ++at)
+        tma_load_4d(smem + L::q + at * L::kAtom, &P.tmq, &bar[B_Q], at * 64, h, q0, bt);
+      int last[2] = {-1, -1};
+      for (int it = 0; it < n; ++it) {
+        const int s = it & 1;
+        if (!mbar_wait(&bar[B_KVE + s], ((it >> 1) & 1) ^ 1, abort, st, 1)) break;
+        const int k0 = m.tcol[e0 + it] * kTile;
+        mbar_arrive_expect_tx(&bar[B_KVF + s], 2 * L::kKV);
+        for (int at = 0; at < D / 64; ++at) {
+          tma_load_4d(smem + L::k0 + s * L::kKV + at * L::kAtom, &P.tmk, &bar[B_KVF + s],
+                      at * 64, hk, k0, bt);
+          tma_load_4d(smem + L::v0 + s * L::kKV + at * L::kAtom, &P.tmv, &bar[B_KVF + s],
+                      at * 64, hk, k0, bt);
+        }
+        last[s] = it;
+      }
+      // every copy this CTA started must land before the CTA may exit
+      volatile int no_abort = 0;
+      mbar_wait(&bar[B_Q], 0, &no_abort, nullptr, 2);
+      for (int s = 0; s < 2; ++s)
+        if (last[s] >= 0) mbar_wait(&bar[B_KVF + s], (last[s] >> 1) & 1, &no_abort, nullptr, 3);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // --------------------------------------------------------- MMA issuer
+      constexpr uint32_t kIdQK = idesc_bf16_f32(128, 128, false, false);
+      constexpr uint32_t kIdPV = idesc_bf16_f32(128, D, false, true);
+      bool ok = mbar_wait(&bar[B_Q], 0, abort, st, 10);
+      for (int it = 0; ok && it <= n; ++it) {
+        if (it < n) {
+          const int s = it & 1;
+          if (!mbar_wait(&bar[B_KVF + s], (it >> 1) & 1, abort, st, 11)) break;
+          if (!mbar_wait(&bar[B_SE + s], ((it >> 1) & 1) ^ 1, abort, st, 12)) break;
+          tc_fence_after();
+          const uint32_t kbase = sb + L::k0 + s * L::kKV;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * L::kAtom + (kk & 3) * 32;
+            mma_bf16(tmem + s * 128, smem_desc_sw128(sb + L::q + off, 16, 1024),
+                     smem_desc_sw128(kbase + off, 16, 1024), kIdQK, kk > 0);
+          }
+          mma_commit(&bar[B_SF + s]);
+        }
+        if (it >= 1) {
+          const int j = it - 1, s = j & 1;
+          if (!mbar_wait(&bar[B_PF + s], (j >> 1) & 1, abort, st, 13)) break;
+          tc_fence_after();
+          const uint32_t pbase = sb + L::p0 + s * L::kP;
+          const uint32_t vbase = sb + L::v0 + s * L::kKV;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint64_t ad = smem_desc_sw128(pbase + (kk >> 2) * L::kAtom + (kk & 3) * 32, 16, 1024);
+            const uint64_t bd = smem_desc_sw128(vbase + kk * 2048, L::kAtom, 1024);
+            mma_bf16(tmem + kTmemO, ad, bd, kIdPV, (j > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(&bar[B_OD + s]);
+          mma_commit(&bar[B_KVE + s]);
+        }
+      }
+      // drain: every MMA issued above has completed
+      mma_commit(&bar[B_DRAIN]);
+      volatile int no_abort = 0;
+      mbar_wait(&bar[B_DRAIN], 0, &no_abort, nullptr, 14);
+    }
+  } else {
+    // --------------------------------------------------------------- softmax
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const int p = q0 + r;
+    const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
+    const float sl2 = a.scale * 1.4426950408889634f;
+    float m_run = -INFINITY, l_run = 0.f;
+    const int gzip = m.kind == SA_MASK_GZIP;
+    const uint32_t* rowbits = nullptr;
+    int li = 0;
+    if (gzip && p < a.N) rowbits = m.bits + ((int64_t)list * m.B + p / m.b) * m.words;
+    if (!gzip && p < a.N) li = m.perm[p];
+    // Every tcgen05.ld/st below is warp-collective: the branches around them
+    // are made warp-uniform with __all_sync / __any_sync.
+    bool ok = true;
+    for (int it = 0; it < n; ++it) {
+      const int s = it & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(&bar[B_SF + s], (it >> 1) & 1, abort, st, 20))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      float x[128];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(lane_addr + s * 128 + c * 32, x + c * 32);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(&bar[B_SE + s]);
+
+      const int J = m.tcol[e0 + it];
+      const int kbase = J * kTile;
+      const bool full = m.tkind[e0 + it] == SA_TILE_FULL && kbase + kTile <= a.N && p < a.N;
+      if (full) {
+#pragma unroll
+        for (int c = 0; c < 128; ++c) x[c] *= sl2;
+      } else {
+#pragma unroll
+        for (int c = 0; c < 128; ++c) {
+          const int kq = kbase + c;
+          bool vis = p < a.N && kq < a.N;
+          if (vis) {
+            if (gzip) {
+              const int jb = kq / m.b;
+              vis = kq <= p && ((rowbits[jb >> 5] >> (jb & 31)) & 1u);
+            } else {
+              const int lj = m.perm[kq];
+              const bool g = (m.gist_bits[lj >> 5] >> (lj & 31)) & 1u;
+              vis = lj <= li && (lj < m.sinks || g || (li - lj) < m.window);
+            }
+          }
+          x[c] = vis ? x[c] * sl2 : -INFINITY;
+        }
+      }
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 128; ++c) mx = fmaxf(mx, x[c]);
+      const float m_new = fmaxf(m_run, mx);
+      const bool resc = m_new > m_run + 8.f;  // true on the first finite max
+      const float m_use = resc ? m_new : m_run;
+      float rowsum = 0.f;
+      uint32_t pk[64];
+      if (m_use == -INFINITY) {
+#pragma unroll
+        for (int c = 0; c < 64; ++c) pk[c] = 0u;
+      } else {
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          const float p0 = ex2(x[2 * c] - m_use), p1 = ex2(x[2 * c + 1] - m_use);
+          __nv_bfloat162 v = __floats2bfloat162_rn(p0, p1);
+          const float2 f = __bfloat1622float2(v);
+          rowsum += f.x + f.y;
+          pk[c] = *reinterpret_cast<uint32_t*>(&v);
+        }
+      }
+      const float alpha = !resc ? 1.f : (m_run == -INFINITY ? 0.f : ex2(m_run - m_use));
+      // P tile s was last read by PV(it - 2)
+      if (it >= 2 &&
+          !__all_sync(0xffffffffu, mbar_wait(&bar[B_OD + s], ((it - 2) >> 1) & 1, abort, st, 21))) {
+        ok = false;
+        break;
+      }
+      if (it >= 1 && __any_sync(0xffffffffu, resc)) {
+        // O must not be accumulated while it is rescaled: wait for PV(it-1).
+        // The whole warp takes part; rows that keep their max use alpha = 1.
+        if (!__all_sync(0xffffffffu, mbar_wait(&bar[B_OD + ((it - 1) & 1)], ((it - 1) >> 1) & 1,
+                                                abort, st, 22))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          float o[32];
+          tmem_ld32(lane_addr + kTmemO + c * 32, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] *= alpha;
+          tmem_st32(lane_addr + kTmemO + c * 32, o);
+        }
+        tmem_wait_st();
+      }
+      l_run = l_run * alpha + rowsum;
+      m_run = m_use;
+      const uint32_t prow = sb + L::p0 + s * L::kP;
+#pragma unroll
+      for (int ch = 0; ch < 16; ++ch) {  // 16 chunks of 8 columns
+        const int col = ch * 8;
+        const uint32_t addr = prow + (col >> 6) * L::kAtom + sw128_offset(r, col & 63);
+        st_shared_v4(addr, pk[ch * 4], pk[ch * 4 + 1], pk[ch * 4 + 2], pk[ch * 4 + 3]);
+      }
+      fence_async_shared();
+      tc_fence_before();
+      mbar_arrive(&bar[B_PF + s]);
+    }
+    // ---------------------------------------------------------------- epilogue
+    if (ok && n > 0 &&
+        __all_sync(0xffffffffu,
+                   mbar_wait(&bar[B_OD + ((n - 1) & 1)], ((n - 1) >> 1) & 1, abort, st, 23))) {
+      tc_fence_after();
+      const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+      __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.o) + bt * a.os[0] +
+                            (int64_t)p * a.os[1] + (int64_t)h * a.os[2];
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        float o[32];
+        tmem_ld32(lane_addr + kTmemO + c * 32, o);  // all lanes: collective
+        tmem_wait_ld();
+        if (p < a.N) {
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            uint4 w;
+            w.x = pack_bf16(o[v * 8 + 0] * inv, o[v * 8 + 1] * inv);
+            w.y = pack_bf16(o[v * 8 + 2] * inv, o[v * 8 + 3] * inv);
+            w.z = pack_bf16(o[v * 8 + 4] * inv, o[v * 8 + 5] * inv);
+            w.w = pack_bf16(o[v * 8 + 6] * inv, o[v * 8 + 7] * inv);
+            *reinterpret_cast<uint4*>(orow + c * 32 + v * 8) = w;
+          }
+        }
+      }
+      if (p < a.N)
+        a.lse[((int64_t)bt * a.Hq + h) * a.N + p] =
+            l_run > 0.f ? (m_run + __log2f(l_run)) * 0.6931471805599453f : -INFINITY;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tmem, kTmemCols);
+}
+
+// -------------------------------------------------------------- host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// [Bt, N, H, d] bf16 with element strides {batch, seq, head}; box 64 x 1 x 128 x 1.
+static bool make_map(CUtensorMap* map, const void* base, int d, int H, int N, int Bt,
+                     const int64_t* s) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const int64_t sh = s[2] > 0 ? s[2] : d, sn = s[1];
+  const int64_t sbat = (Bt > 1) ? s[0] : sn * N;
+  cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)N, (cuuint64_t)Bt};
+  cuuint64_t strides[3] = {(cuuint64_t)(sh * 2), (cuuint64_t)(sn * 2), (cuuint64_t)(sbat * 2)};
+  cuuint32_t box[4] = {64, 1, 128, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D>
+static cudaError_t fwd_tc_launch(const AttnArgs& a, const MaskArgs& m, cudaStream_t s) {
+  FwdTcParams P;
+  memset(&P, 0, sizeof(P));
+  if (!make_map(&P.tmq, a.q, D, a.Hq, a.N, a.Bt, a.qs) ||
+      !make_map(&P.tmk, a.k, D, a.Hkv, a.N, a.Bt, a.ks) ||
+      !make_map(&P.tmv, a.v, D, a.Hkv, a.N, a.Bt, a.vs))
+    return cudaErrorInvalidValue;
+  P.a = a;
+  P.m = m;
+  const int bytes = (int)FwdLayout<D>::bytes;
+  cudaError_t e = cudaFuncSetAttribute(fwd_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       bytes);
+  if (e != cudaSuccess) return e;
+  fwd_tc_kernel<D><<<dim3(m.T, a.Hq, a.Bt), 192, bytes, s>>>(P);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fwd_tc(int d, const AttnArgs& a, const MaskArgs& m, cudaStream_t s) {
+  if (d == 64) return fwd_tc_launch<64>(a, m, s);
+  if (d == 128) return fwd_tc_launch<128>(a, m, s);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace sa

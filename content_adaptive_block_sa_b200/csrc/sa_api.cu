@@ -13,6 +13,7 @@ cudaError_t launch_gist_build(const sa_mask_desc&, const uint8_t*, const sa_bloc
                               cudaStream_t);
 cudaError_t launch_fwd_simt(int dtype, int d, const AttnArgs&, const MaskArgs&, cudaStream_t);
 cudaError_t launch_bwd_simt(int dtype, int d, const AttnArgs&, const MaskArgs&, cudaStream_t);
+cudaError_t launch_fwd_tc(int d, const AttnArgs&, const MaskArgs&, cudaStream_t);
 cudaError_t launch_decode(const sa_decode_desc&, const void*, const void*, const void*,
                           const void*, const void*, int32_t*, void*, float*, void*,
                           cudaStream_t);
@@ -125,6 +126,7 @@ sa_status check_attn(const sa_attn_desc* a, const sa_mask_desc* m) {
   SA_CHECK(a->num_kv_heads >= 1 && a->num_q_heads % a->num_kv_heads == 0, SA_ERR_INVALID_ARG);
   SA_CHECK(a->head_dim == 32 || a->head_dim == 64 || a->head_dim == 128, SA_ERR_UNSUPPORTED);
   SA_CHECK(a->softmax_scale >= 0.f && isfinite(a->softmax_scale), SA_ERR_INVALID_ARG);
+  SA_CHECK(a->impl >= SA_IMPL_AUTO && a->impl <= SA_IMPL_TENSOR_CORES, SA_ERR_INVALID_ARG);
   const int64_t* all[4] = {a->q_strides, a->k_strides, a->v_strides, a->o_strides};
   for (auto s : all) {
     SA_CHECK(s[0] >= 0 && s[2] >= 0 && s[1] >= a->head_dim, SA_ERR_INVALID_ARG);
@@ -179,6 +181,25 @@ AttnArgs make_attn_args(const sa_attn_desc& a) {
 }
 
 size_t round256(size_t x) { return (x + 255) / 256 * 256; }
+
+// Can the TMA + tcgen05 kernels read these tensors?
+bool tensor_core_ok(const sa_attn_desc& a, const void* const* ptrs, int nptr) {
+  if (a.dtype != SA_DTYPE_BF16 || (a.head_dim != 64 && a.head_dim != 128)) return false;
+  for (int i = 0; i < nptr; ++i)
+    if (!aligned(ptrs[i], 16)) return false;
+  const int64_t* all[4] = {a.q_strides, a.k_strides, a.v_strides, a.o_strides};
+  for (auto s : all)
+    for (int i = 0; i < 3; ++i)
+      if (s[i] % 8 != 0) return false;
+  return true;
+}
+
+// Resolves SA_IMPL_AUTO; -1 if the request cannot be served.
+int pick_impl(const sa_attn_desc& a, bool tc_ok) {
+  if (a.impl == SA_IMPL_AUTO) return tc_ok ? SA_IMPL_TENSOR_CORES : SA_IMPL_CUDA_CORES;
+  if (a.impl == SA_IMPL_TENSOR_CORES && !tc_ok) return -1;
+  return a.impl;
+}
 
 }  // namespace
 
@@ -274,12 +295,17 @@ sa_status sa_forward(const sa_attn_desc* attn, const sa_mask_desc* mask, const v
   if (st != SA_OK) return st;
   st = check_ws(ws, ws_bytes, kStatusBytes);
   if (st != SA_OK) return st;
-  st = clear_status(ws, stream);
-  if (st != SA_OK) return st;
   AttnArgs a = make_attn_args(*attn);
   a.q = q; a.k = k; a.v = v; a.o = o; a.lse = lse;
   a.status = (DeviceStatus*)ws;
+  const void* ptrs[4] = {q, k, v, o};
+  const int impl = pick_impl(*attn, tensor_core_ok(*attn, ptrs, 4));
+  if (impl < 0) return SA_ERR_UNSUPPORTED;
+  st = clear_status(ws, stream);
+  if (st != SA_OK) return st;
   const MaskArgs m = make_mask_args(*mask, *lists);
+  if (impl == SA_IMPL_TENSOR_CORES)
+    return cuda_status(launch_fwd_tc(attn->head_dim, a, m, stream));
   return cuda_status(launch_fwd_simt(attn->dtype, attn->head_dim, a, m, stream));
 }
 

@@ -189,7 +189,18 @@ typedef struct sa_block_lists_sizes {
  *               [Bt, Hq, N] array.
  *  softmax_scale  0 selects 1/sqrt(d). Scores are q.k * scale; LSE uses the
  *               natural log.
+ *  impl         SA_IMPL_AUTO picks the tensor-core kernels when dtype is bf16,
+ *               head_dim is 64 or 128, every base pointer is 16-byte aligned
+ *               and every stride is a multiple of 8 elements (TMA); otherwise
+ *               the CUDA-core kernels. SA_IMPL_TENSOR_CORES on an input that
+ *               does not meet those conditions returns SA_ERR_UNSUPPORTED.
  */
+typedef enum {
+  SA_IMPL_AUTO = 0,
+  SA_IMPL_CUDA_CORES = 1,    /* fp32 FMA path (fp32 or bf16 inputs) */
+  SA_IMPL_TENSOR_CORES = 2,  /* tcgen05 + TMA path (bf16 only)      */
+} sa_impl;
+
 typedef struct sa_attn_desc {
   int32_t dtype;
   int32_t batch;
@@ -202,6 +213,7 @@ typedef struct sa_attn_desc {
   int64_t k_strides[3];
   int64_t v_strides[3];
   int64_t o_strides[3];
+  int32_t impl;
 } sa_attn_desc;
 
 typedef enum { SA_SELECT_SUM_LOGITS_PER_GROUP = 0 } sa_select_rule;

@@ -131,3 +131,21 @@ def test_calls_reject_null_and_small_workspace_without_a_device(sa):
     assert sa.lib().sa_gist_decode_workspace_size(C.byref(dd), C.byref(n)) == 2
     dd.top_k, dd.n_gists = 64, 4095
     assert sa.lib().sa_gist_decode_workspace_size(C.byref(dd), C.byref(n)) == 1
+
+
+def test_tensor_core_request_on_fp32_is_unsupported_before_any_launch(sa):
+    L = sa._abi
+    md = sa.gzip_mask(1, 1024, 128, 1, 4)
+    fake = C.c_void_p(1 << 20)  # never dereferenced: validation fails first
+    caps = L.sa_block_lists_sizes()
+    sa.lib().sa_block_lists_capacity(C.byref(md), C.byref(caps))
+    lists = L.sa_block_lists(*([fake.value] * 13), caps.nnz, caps.tile_nnz)
+    st = (C.c_int64 * 3)(1024 * 4 * 64, 4 * 64, 64)
+    ad = L.sa_attn_desc(dtype=L.SA_DTYPE_FP32, batch=1, seq_len=1024, num_q_heads=4, num_kv_heads=4,
+                        head_dim=64, q_strides=st, k_strides=st, v_strides=st, o_strides=st,
+                        impl=L.SA_IMPL_TENSOR_CORES)
+    assert sa.lib().sa_forward(C.byref(ad), C.byref(md), fake, fake, fake, C.byref(lists), fake,
+                               fake, fake, 4096, None) == L.SA_ERR_UNSUPPORTED
+    ad.impl = 7
+    assert sa.lib().sa_forward(C.byref(ad), C.byref(md), fake, fake, fake, C.byref(lists), fake,
+                               fake, fake, 4096, None) == L.SA_ERR_INVALID_ARG

@@ -15,10 +15,14 @@ from _cases import (check_close, gist_layout, gzip_flags_oracle, gzip_flags_prod
 pytestmark = pytest.mark.gpu
 
 
-def run_gzip(sa, w, q, k, v, flags):
+IMPLS = {"cuda_cores": 1, "tensor_cores": 2}
+
+
+def run_gzip(sa, w, q, k, v, flags, impl=0):
     md = sa.gzip_mask(w["batch"], w["seq_len"], w["block"], w["window"], w["heads"])
     lists = sa.build_block_mask(md, flags)
-    o, lse = sa.forward(to_dev(q, w["dtype"]), to_dev(k, w["dtype"]), to_dev(v, w["dtype"]), md, lists)
+    o, lse = sa.forward(to_dev(q, w["dtype"]), to_dev(k, w["dtype"]), to_dev(v, w["dtype"]), md, lists,
+                        impl=impl)
     torch.cuda.synchronize()
     return to_np(o), to_np(lse)
 
@@ -35,11 +39,17 @@ def gzip_case(index, batch, N, b, w, H, d, dtype, p=0.3):
     gzip_case(103, 2, 16 * 50, 16, 3, 4, 32, "fp32"),
     gzip_case(104, 1, 256 * 3, 256, 0, 4, 128, "bf16", p=0.6),
     gzip_case(105, 1, 64 * 12, 64, 20, 4, 64, "fp32"),
-], ids=["tiny_fp32", "b64_ragged_bf16", "b128_h6_bf16", "b16_fp32", "b256_bf16", "wide_w_fp32"])
-def test_gzip_forward_small(sa, w):
+    gzip_case(106, 2, 32 * 40, 32, 1, 8, 128, "bf16", p=0.5),
+    gzip_case(107, 1, 16 * 72, 16, 4, 4, 64, "bf16", p=0.4),
+], ids=["tiny_fp32", "b64_ragged_bf16", "b128_h6_bf16", "b16_fp32", "b256_bf16", "wide_w_fp32",
+        "b32_d128_bf16", "b16_d64_bf16"])
+@pytest.mark.parametrize("impl", list(IMPLS))
+def test_gzip_forward_small(sa, w, impl):
+    if w["dtype"] == "fp32" and impl == "tensor_cores":
+        pytest.skip("tensor cores take bf16 only")
     q, k, v, _ = gzip_inputs(w)
     fp, fo = gzip_flags_product(sa, w), gzip_flags_oracle(w)
-    o, lse = run_gzip(sa, w, q, k, v, fp)
+    o, lse = run_gzip(sa, w, q, k, v, fp, IMPLS[impl])
     cls = G.head_classes(w["heads"])
     for bt in range(w["batch"]):
         masks = G.block_masks(fo[bt], w["window"])
@@ -69,21 +79,23 @@ def test_gzip_forward_full_size_sampled(sa, name):
     assert np.isfinite(o).all() and np.isfinite(lse).all()
 
 
-def run_gist(sa, w, q, k, v):
+def run_gist(sa, w, q, k, v, impl=0):
     md = sa.gist_mask(w["seq_len"], w["heads"], w["sinks"], w["ratio"], w["window"],
                       gist_tail=w.get("gist_tail", 32))
     lists = sa.build_block_mask(md, None)
-    o, lse = sa.forward(to_dev(q, "bf16"), to_dev(k, "bf16"), to_dev(v, "bf16"), md, lists)
+    o, lse = sa.forward(to_dev(q, "bf16"), to_dev(k, "bf16"), to_dev(v, "bf16"), md, lists,
+                        impl=impl)
     torch.cuda.synchronize()
     return to_np(o), to_np(lse)
 
 
 @pytest.mark.parametrize("N,sinks,window", [(1000, 16, 32), (128 * 6, 128, 128), (2000, 130, 200)])
-def test_gist_forward_small(sa, N, sinks, window):
+@pytest.mark.parametrize("impl", list(IMPLS))
+def test_gist_forward_small(sa, N, sinks, window, impl):
     w = W.scaled("gist_prefill_32k", index=200 + N, seq_len=N, sinks=sinks, window=window,
                  heads=4, kv_heads=2)
     q, k, v = (W.qkv(w, t, 0)[None] for t in ("q", "k", "v"))  # physical order
-    o, lse = run_gist(sa, w, q, k, v)
+    o, lse = run_gist(sa, w, q, k, v, IMPLS[impl])
     g, perm, inv = gist_layout(N, sinks, w["ratio"])
     vis = Gi.visibility(g, sinks, window)
     for h in range(4):
@@ -108,3 +120,19 @@ def test_gist_forward_full_size_sampled(sa):
         check_close(o[0, rows, h], ro, "bf16", f"O h{h}")
         check_close(lse[0, h, rows], rl, "bf16", f"LSE h{h}")
     assert np.isfinite(o).all() and np.isfinite(lse).all()
+
+
+def test_tensor_cores_agree_with_cuda_cores_on_strided_inputs(sa):
+    # q/k/v as slices of one packed [Bt, N, 3, H, d] buffer (non-contiguous heads)
+    w = gzip_case(108, 2, 128 * 4, 128, 1, 4, 64, "bf16")
+    q, k, v, _ = gzip_inputs(w)
+    packed = torch.from_numpy(np.stack([q, k, v], axis=2)).to("cuda", torch.bfloat16)
+    tq, tk, tv = packed[:, :, 0], packed[:, :, 1], packed[:, :, 2]
+    fp = gzip_flags_product(sa, w)
+    md = sa.gzip_mask(2, w["seq_len"], 128, 1, 4)
+    lists = sa.build_block_mask(md, fp)
+    o1, l1 = sa.forward(tq, tk, tv, md, lists, impl=1)
+    o2, l2 = sa.forward(tq, tk, tv, md, lists, impl=2)
+    torch.cuda.synchronize()
+    check_close(to_np(o2), to_np(o1), "bf16", "O tc vs cuda cores")
+    check_close(to_np(l2), to_np(l1), "bf16", "LSE tc vs cuda cores")
