@@ -73,6 +73,7 @@ PROTOTYPES = {
     "sa_gist_decode_workspace_size": (C.c_int, [P(sa_decode_desc), P(C.c_size_t)]),
     "sa_gist_decode": (C.c_int, [P(sa_decode_desc), vp, vp, vp, vp, vp, vp, vp, vp, vp,
                                  C.c_size_t, vp]),
+    "sa_gist_decode_noalloc": (C.c_int, [P(sa_decode_desc), vp, vp, vp, vp, vp, vp, vp, vp, vp]),
 }
 
 

@@ -19,6 +19,8 @@
 //      tokens.
 //   4. combine the partials of every slice into O (bf16) and LSE (fp32).
 // Keys and values are read with 16-byte loads, 16 lanes per 256-byte row.
+#include <mutex>
+
 #include "sa_common.cuh"
 
 namespace sa {
@@ -353,3 +355,60 @@ cudaError_t launch_decode(const sa_decode_desc& d, const void* q, const void* gk
 size_t decode_workspace_bytes(const sa_decode_desc& d) { return decode_plan(d).bytes; }
 
 }  // namespace sa
+
+// ---------------------------------------------------- allocation-free variant
+// Scratch for sa_gist_decode_noalloc: a file-scope device array that every GPU
+// loading this library holds until the process exits. All calls share it.
+namespace sa {
+constexpr size_t kStaticDecodeScratch = size_t(16) << 20;  // 16 MiB
+static __device__ __align__(256) unsigned char g_decode_scratch[kStaticDecodeScratch];
+
+constexpr int kMaxDevices = 64;
+static std::mutex g_scratch_mutex;
+static void* g_scratch_addr[kMaxDevices];
+
+// Device address of the array on the current device. In host code the
+// array's name is only a stand-in, so the address is looked up once per
+// device (with that device current) and cached.
+static cudaError_t decode_scratch_address(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (g_scratch_addr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_decode_scratch);
+    if (e != cudaSuccess) return e;
+    g_scratch_addr[dev] = p;
+  }
+  *out = g_scratch_addr[dev];
+  return cudaSuccess;
+}
+}  // namespace sa
+
+extern "C" sa_status sa_gist_decode_noalloc(const sa_decode_desc* desc, const void* q,
+                                            const void* gist_k, const void* gist_v,
+                                            const void* k_cache, const void* v_cache,
+                                            int32_t* sel_chunks, void* o, float* lse,
+                                            sa_stream_t stream) {
+  size_t need = 0;
+  sa_status st = sa_gist_decode_workspace_size(desc, &need);  // validates the shapes
+  if (st != SA_OK) return st;
+  if (!(q && gist_k && gist_v && k_cache && v_cache && o && lse)) return SA_ERR_INVALID_ARG;
+  if (sel_chunks == nullptr && desc->top_k != 0) return SA_ERR_INVALID_ARG;
+  auto al = [](const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; };
+  if (!(al(gist_k, 16) && al(gist_v, 16) && al(k_cache, 16) && al(v_cache, 16) && al(q, 2) &&
+        al(o, 2)))
+    return SA_ERR_INVALID_ARG;
+  if (need > sa::kStaticDecodeScratch) return SA_ERR_WORKSPACE;
+  void* ws = nullptr;
+  if (sa::decode_scratch_address(&ws) != cudaSuccess) return SA_ERR_CUDA;
+  // the array keeps the previous call's contents: the status word must start at zero
+  // (every score and partial slot is written before it is read)
+  if (cudaMemsetAsync(ws, 0, sa::kStatusBytes, stream) != cudaSuccess) return SA_ERR_CUDA;
+  return sa::launch_decode(*desc, q, gist_k, gist_v, k_cache, v_cache, sel_chunks, o, lse, ws,
+                           stream) == cudaSuccess
+             ? SA_OK
+             : SA_ERR_CUDA;
+}

@@ -340,6 +340,33 @@ sa_status sa_gist_decode(const sa_decode_desc* desc, const void* q,
                          int32_t* sel_chunks, void* o, float* lse,
                          void* ws, size_t ws_bytes, sa_stream_t stream);
 
+/* Allocation-free variant of sa_gist_decode (the method's pages have no
+ * counterpart; this is a deployment convenience).
+ *
+ * Some callers cannot allocate device memory: a serving engine that reserves
+ * all free memory for its KV cache at start-up and forbids later allocations,
+ * a plugin that a host framework only hands raw pointers, or a decode loop
+ * in which cudaMalloc's implicit device synchronisation would stall the other
+ * streams. This entry point takes the same inputs and outputs as
+ * sa_gist_decode but no workspace: its scratch is a fixed 16 MiB array in
+ * device memory that every GPU loading the library holds until the process
+ * exits. It calls no cudaMalloc or cudaFree.
+ *  - Sizes whose workspace (sa_gist_decode_workspace_size) exceeds 16 MiB
+ *    return SA_ERR_WORKSPACE; use sa_gist_decode for them.
+ *  - The first call on a device looks up the array's device address (with
+ *    that device current) and caches it; make that first call before any
+ *    stream capture.
+ *  - Every call on a device shares the one array, which keeps the last call's
+ *    contents (its status word is cleared by each call). Calls that overlap on
+ *    the GPU - on different streams, or from different host threads without
+ *    ordering - race on it; serialise them.
+ *  - sa_get_device_status cannot read this array's status word. */
+sa_status sa_gist_decode_noalloc(const sa_decode_desc* desc, const void* q,
+                                 const void* gist_k, const void* gist_v,
+                                 const void* k_cache, const void* v_cache,
+                                 int32_t* sel_chunks, void* o, float* lse,
+                                 sa_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
