@@ -94,3 +94,28 @@ def tile_lists(vis_phys, tile: int, tail: int, N: int | None = None):
         row_ptr.append(len(keys))
     return (np.asarray(row_ptr, np.int32), np.asarray(keys, np.int32),
             np.asarray(kinds, np.int32))
+
+
+def always_visible_keys(is_gist, sinks: int, perm, tile: int):
+    """Keys every later query sees whatever its window: sinks and gists.
+
+    Returns (far_idx, far_ptr): far_idx[f] is the PHYSICAL index of the f-th
+    such key in logical order, far_ptr[J] the number of them at logical
+    positions below tile * J (J = 0..T). A query tile I whose window cannot
+    reach below key tile J sees, among keys below tile * J, exactly
+    far_idx[:far_ptr[J]].
+    """
+    g = np.asarray(is_gist, bool)
+    N = len(g)
+    inv = np.empty(N, np.int64)
+    inv[np.asarray(perm)] = np.arange(N)
+    pos = np.nonzero((np.arange(N) < sinks) | g)[0]
+    T = (N + tile - 1) // tile
+    far_ptr = np.array([np.count_nonzero(pos < tile * J) for J in range(T + 1)], np.int32)
+    return inv[pos].astype(np.int32), far_ptr
+
+
+def near_tile_start(I: int, window: int, tile: int) -> int:
+    """First key tile that query tile I must visit with the element rule: for
+    every key below tile * Jlo and query at or above tile * I, i - j >= window."""
+    return max(0, I - (window - 1 + tile - 1) // tile)

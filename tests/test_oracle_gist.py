@@ -105,3 +105,20 @@ def test_tile_lists_row_callable_matches_dense():
     fn = lambda rows: Gi.visibility(g, 16, 40, rows=perm[rows])[:, perm]
     for a, b in zip(Gi.tile_lists(dense, 128, 32), Gi.tile_lists(fn, 128, 32, N=N)):
         assert np.array_equal(a, b)
+
+
+@pytest.mark.parametrize("N,sinks,window", [(2000, 128, 128), (1500, 5, 300), (777, 0, 1)])
+def test_far_prefix_covers_exactly_the_visible_keys_outside_the_near_tiles(N, sinks, window):
+    g = Gi.gist_flags(N, sinks, 4)
+    perm = Gi.shift_permutation(g, 128)
+    far_idx, far_ptr = Gi.always_visible_keys(g, sinks, perm, 128)
+    T = (N + 127) // 128
+    for I in range(T):
+        Jlo = Gi.near_tile_start(I, window, 128)
+        rows = np.arange(I * 128, min(N, I * 128 + 128))
+        vis = Gi.visibility(g, sinks, window, rows=rows)[:, : 128 * Jlo]
+        # every key below the near tiles is visible to all rows of the tile or to none
+        cols = np.nonzero(vis.any(axis=0))[0]
+        assert vis[:, cols].all()
+        assert np.array_equal(np.sort(perm[far_idx[: far_ptr[Jlo]]]), cols)
+    assert far_ptr[-1] == len(far_idx) == sinks + g[sinks:].sum()
