@@ -109,11 +109,8 @@ def copy_out(tensors):
     return outs
 
 class GzipWorkload:
-    def __init__(self, sa, torch, name, backward, rank):
+    def __init__(self, sa, torch, w, backward):
         self.sa, self.torch, self.backward = sa, torch, backward
-        w = dict(W.WORKLOADS[name])
-        if rank:
-            w["index"] = w["index"] + 1000 * rank  # an independent copy per rank
         self.w = w
         Bt, N, H, d, b = w["batch"], w["seq_len"], w["heads"], w["head_dim"], w["block"]
         if w.get("flags_from") == "bernoulli":
@@ -196,28 +193,30 @@ class GzipWorkload:
         H = w["heads"]
         heads = [0, H // 2, H - 1] if heads is None else heads
         cls = G.head_classes(H)
+        N = w["seq_len"]
+        R = min(N, max(b, 2048 // b * b))  # the last R query rows (whole blocks)
+        rows = np.arange(N - R, N)
+        data = {h: [W.qkv(w, t, 0, head=h) for t in ("q", "k", "v", "do")] for h in heads}
         t0 = time.perf_counter()
         flops = 0.0
         for h in heads:
             bm = masks[cls[h]]
-            q, k, v = (W.qkv(w, t, 0, head=h) for t in ("q", "k", "v"))
-            mask = lambda rows: G.token_mask(bm, b, rows=rows)
+            q, k, v, do = data[h]
+            mask = lambda r: G.token_mask(bm, b, rows=rows[r])
             if self.backward:
-                do = W.qkv(w, "do", 0, head=h)
-                A.backward(q, k, v, do, mask)
+                A.backward(q[rows], k, v, do[rows], mask)
             else:
-                A.forward(q, k, v, mask)
-            flops += (4.0 + (10.0 if self.backward else 0.0)) * w["head_dim"] * b * b * int(bm.sum())
+                A.forward(q[rows], k, v, mask)
+            pairs = int(bm[(N - R) // b:].sum())
+            flops += (4.0 + (10.0 if self.backward else 0.0)) * w["head_dim"] * b * b * pairs
         dt = time.perf_counter() - t0
-        return flops / dt / 1e12, f"batch row 0, heads {heads} (one per class), whole heads, fp64", dt
+        return flops / dt / 1e12, (f"batch row 0, heads {heads} (one per class), last {R} query "
+                                   "rows each, fp64"), dt
 
 
 class GistWorkload(GzipWorkload):
-    def __init__(self, sa, torch, name, rank):
+    def __init__(self, sa, torch, w):
         self.sa, self.torch, self.backward = sa, torch, False
-        w = dict(W.WORKLOADS[name])
-        if rank:
-            w["index"] = w["index"] + 1000 * rank
         self.w = w
         N, H, Hkv, d = w["seq_len"], w["heads"], w["kv_heads"], w["head_dim"]
         self.h_in = {t: torch.from_numpy(W.qkv(w, t, 0)[None]).to(torch.bfloat16).pin_memory()
@@ -272,11 +271,8 @@ class GistWorkload(GzipWorkload):
 
 
 class DecodeWorkload:
-    def __init__(self, sa, torch, name, rank):
+    def __init__(self, sa, torch, w):
         self.sa, self.torch = sa, torch
-        w = dict(W.WORKLOADS[name])
-        if rank:
-            w["index"] = w["index"] + 1000 * rank
         self.w = w
         n, Hkv, L, d, G = w["n_seq"], w["kv_heads"], w["cache_len"], w["head_dim"], w["n_gists"]
         self.kc = torch.empty(n, Hkv, L, d, dtype=torch.bfloat16, device="cuda")
@@ -319,16 +315,13 @@ class DecodeWorkload:
             ev[1].record()
 
     def e2e_step(self):
-        # the new token's query and the sequence's gist K/V come from the host
+        # a decode step's input is the new token's query; the caches are resident
         self.q.copy_(self.h_q, non_blocking=True)
-        self.gk.copy_(self.h_gk, non_blocking=True)
-        self.gv.copy_(self.h_gv, non_blocking=True)
         self.step()
         return copy_out([self.o, self.lse, self.sel])
 
     def io_bytes(self):
-        h2d = sum(x.numel() * 2 for x in (self.h_q, self.h_gk, self.h_gv))
-        return h2d, self.o.numel() * 2 + self.lse.numel() * 4 + self.sel.numel() * 4
+        return self.h_q.numel() * 2, self.o.numel() * 2 + self.lse.numel() * 4 + self.sel.numel() * 4
 
     def cpu_baseline(self):
         from oracle import decode as D
@@ -346,12 +339,26 @@ class DecodeWorkload:
             "sequence 0, all kv heads (raw cache generation excluded), fp64", dt
 
 
-def make(sa, torch, name, rank):
+SMALL = {"gzip_8k": dict(batch=8), "gzip_64k_fwdbwd": dict(batch=1, heads=4, kv_heads=4),
+         "gist_prefill_32k": dict(heads=8, kv_heads=2), "gist_decode_128k": dict(n_seq=4)}
+
+
+def workload_params(name, rank, size):
+    w = dict(W.WORKLOADS[name])
+    if size == "small":
+        w.update(SMALL[name])
+    if rank:
+        w["index"] = w["index"] + 1000 * rank  # an independent copy per rank
+    return w
+
+
+def make(sa, torch, name, rank, size="full"):
+    w = workload_params(name, rank, size)
     if name.startswith("gzip"):
-        return GzipWorkload(sa, torch, name, name.endswith("fwdbwd"), rank)
+        return GzipWorkload(sa, torch, w, name.endswith("fwdbwd"))
     if name.startswith("gist_prefill"):
-        return GistWorkload(sa, torch, name, rank)
-    return DecodeWorkload(sa, torch, name, rank)
+        return GistWorkload(sa, torch, w)
+    return DecodeWorkload(sa, torch, w)
 
 
 # ----------------------------------------------------------------- main
@@ -403,6 +410,8 @@ def main():
     ap.add_argument("--workload", default="gzip_8k",
                     choices=["gzip_8k", "gzip_64k_fwdbwd", "gist_prefill_32k", "gist_decode_128k"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--size", default="full", choices=["full", "small"],
+                    help="small: fewer heads/sequences (inputs still larger than L2), for profiling")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -433,7 +442,7 @@ def main():
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         return float(t.item())
 
-    wl = make(sa, torch, args.workload, rank)
+    wl = make(sa, torch, args.workload, rank, args.size)
     for _ in range(args.warmup):
         wl.step()
     torch.cuda.synchronize()

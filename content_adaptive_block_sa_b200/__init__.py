@@ -122,11 +122,13 @@ class BlockLists:
         self.tile_kind_t = mk(caps.tile_nnz, torch.int8)
         self.perm = mk(caps.perm, torch.int32)
         self.gist_bits = mk(caps.gist_bits, torch.int32)
+        self.far_idx = mk(caps.far_idx, torch.int32)
+        self.far_ptr = mk(caps.far_ptr, torch.int32)
         self.struct = _abi.sa_block_lists(
             *[_ptr(getattr(self, n)) for n in ("row_ptr", "col_idx", "col_ptr", "row_idx", "bits",
                                                 "tile_row_ptr", "tile_col", "tile_kind",
                                                 "tile_col_ptr", "tile_row", "tile_kind_t",
-                                                "perm", "gist_bits")],
+                                                "perm", "gist_bits", "far_idx", "far_ptr")],
             int(caps.nnz), int(caps.tile_nnz))
 
 

@@ -31,13 +31,14 @@ class sa_mask_desc(C.Structure):
 class sa_block_lists(C.Structure):
     _fields_ = [(n, vp) for n in ("row_ptr", "col_idx", "col_ptr", "row_idx", "bits",
                                   "tile_row_ptr", "tile_col", "tile_kind", "tile_col_ptr",
-                                  "tile_row", "tile_kind_t", "perm", "gist_bits")] + \
+                                  "tile_row", "tile_kind_t", "perm", "gist_bits", "far_idx",
+                                  "far_ptr")] + \
                [("cap_nnz", i64), ("cap_tile_nnz", i64)]
 
 
 class sa_block_lists_sizes(C.Structure):
     _fields_ = [(n, i64) for n in ("row_ptr", "nnz", "bits", "tile_row_ptr", "tile_nnz",
-                                   "perm", "gist_bits")]
+                                   "perm", "gist_bits", "far_idx", "far_ptr")]
 
 
 class sa_attn_desc(C.Structure):

@@ -33,8 +33,56 @@ using namespace sm100;
 
 struct FwdTcParams {
   CUtensorMap tmq, tmk, tmv;
+  CUtensorMap tmkc, tmvc;  // gist mode: sinks + gists compacted in logical order
   AttnArgs a;
   MaskArgs m;
+};
+
+// Internal tile kind: only the first `cnt` columns hold keys (the last tile of
+// the compacted sink/gist keys).
+constexpr int kTileCount = 3;
+
+// The CTA's visit list, the same in every role. Gzip mode: the tile list of
+// (sequence, head class, query tile). Gist mode: the dense prefix of the
+// compacted sink/gist keys that lie below the near tiles, then the near tiles
+// Jlo..I of the physical sequence, which take the element rule.
+struct WorkList {
+  int gist, e0, n, nft, nf, jlo;
+  __device__ void init(const MaskArgs& m, int list, int I) {
+    gist = m.kind == SA_MASK_GIST;
+    if (gist) {
+      jlo = max(0, I - (m.window - 1 + kTile - 1) / kTile);
+      nf = m.far_ptr[jlo];
+      nft = (nf + kTile - 1) / kTile;
+      n = nft + (I - jlo + 1);
+      e0 = 0;
+    } else {
+      e0 = m.trp[list * (m.T + 1) + I];
+      n = m.trp[list * (m.T + 1) + I + 1] - e0;
+      nft = nf = jlo = 0;
+    }
+  }
+  // source (0 = sequence, 1 = compacted keys), first key row, kind, valid columns
+  __device__ void entry(const MaskArgs& m, int it, int& src, int& k0, int& kind, int& cnt) const {
+    if (gist) {
+      if (it < nft) {
+        src = 1;
+        k0 = it * kTile;
+        cnt = min(kTile, nf - k0);
+        kind = cnt == kTile ? SA_TILE_FULL : kTileCount;
+      } else {
+        src = 0;
+        k0 = (jlo + it - nft) * kTile;
+        kind = SA_TILE_MASKED;
+        cnt = kTile;
+      }
+    } else {
+      src = 0;
+      k0 = m.tcol[e0 + it] * kTile;
+      kind = m.tkind[e0 + it] == SA_TILE_FULL ? SA_TILE_FULL : SA_TILE_MASKED;
+      cnt = kTile;
+    }
+  }
 };
 
 template <int D>
@@ -47,7 +95,7 @@ struct FwdLayout {
   static constexpr uint32_t k0 = kQ;
   static constexpr uint32_t v0 = kQ + 2 * kKV;
   static constexpr uint32_t p0 = kQ + 4 * kKV;
-  static constexpr uint32_t bars = p0 + 2 * kP;
+  static constexpr uint32_t bars = p0 + 2 * kP;    // 16 mbarriers + TMEM slot + flags
   static constexpr uint32_t bytes = bars + 256 + 1024;  // + alignment slack
 };
 
@@ -74,8 +122,9 @@ __global__ void __launch_bounds__(192, 1) fwd_tc_kernel(const __grid_constant__ 
   const int h = blockIdx.y, bt = blockIdx.z;
   const int hk = h / (a.Hq / a.Hkv);
   const int list = list_of(m, bt, h);
-  const int e0 = m.trp[list * (T + 1) + I];
-  const int n = m.trp[list * (T + 1) + I + 1] - e0;
+  WorkList wl;
+  wl.init(m, list, I);
+  const int n = wl.n;
   const int q0 = I * kTile;
   DeviceStatus* st = a.status;
 
@@ -108,6 +157,10 @@ __global__ void __launch_bounds__(192, 1) fwd_tc_kernel(const __grid_constant__ 
       prefetch_tmap(&P.tmq);
       prefetch_tmap(&P.tmk);
       prefetch_tmap(&P.tmv);
+      if (wl.gist) {
+        prefetch_tmap(&P.tmkc);
+        prefetch_tmap(&P.tmvc);
+      }
       mbar_arrive_expect_tx(&bar[B_Q], L::kQ);
       for (int at = 0; at < D / 64; ++at)
         tma_load_4d(smem + L::q + at * L::kAtom, &P.tmq, &bar[B_Q], at * 64, h, q0, bt);
@@ -115,13 +168,16 @@ __global__ void __launch_bounds__(192, 1) fwd_tc_kernel(const __grid_constant__ 
       for (int it = 0; it < n; ++it) {
         const int s = it & 1;
         if (!mbar_wait(&bar[B_KVE + s], ((it >> 1) & 1) ^ 1, abort, st, 1)) break;
-        const int k0 = m.tcol[e0 + it] * kTile;
+        int src, k0, kind, cnt;
+        wl.entry(m, it, src, k0, kind, cnt);
+        const CUtensorMap* mk = src ? &P.tmkc : &P.tmk;
+        const CUtensorMap* mv = src ? &P.tmvc : &P.tmv;
         mbar_arrive_expect_tx(&bar[B_KVF + s], 2 * L::kKV);
         for (int at = 0; at < D / 64; ++at) {
-          tma_load_4d(smem + L::k0 + s * L::kKV + at * L::kAtom, &P.tmk, &bar[B_KVF + s],
-                      at * 64, hk, k0, bt);
-          tma_load_4d(smem + L::v0 + s * L::kKV + at * L::kAtom, &P.tmv, &bar[B_KVF + s],
-                      at * 64, hk, k0, bt);
+          tma_load_4d(smem + L::k0 + s * L::kKV + at * L::kAtom, mk, &bar[B_KVF + s], at * 64, hk,
+                      k0, bt);
+          tma_load_4d(smem + L::v0 + s * L::kKV + at * L::kAtom, mv, &bar[B_KVF + s], at * 64, hk,
+                      k0, bt);
         }
         last[s] = it;
       }
@@ -186,6 +242,7 @@ __global__ void __launch_bounds__(192, 1) fwd_tc_kernel(const __grid_constant__ 
     int li = 0;
     if (gzip && p < a.N) rowbits = m.bits + ((int64_t)list * m.B + p / m.b) * m.words;
     if (!gzip && p < a.N) li = m.perm[p];
+    const int lb = (gzip && m.b < kTile) ? __ffs(m.b) - 1 : 0;  // b < 128 is a power of two
     // Every tcgen05.ld/st below is warp-collective: the branches around them
     // are made warp-uniform with __all_sync / __any_sync.
     bool ok = true;
@@ -203,28 +260,62 @@ __global__ void __launch_bounds__(192, 1) fwd_tc_kernel(const __grid_constant__ 
       tc_fence_before();
       mbar_arrive(&bar[B_SE + s]);
 
-      const int J = m.tcol[e0 + it];
-      const int kbase = J * kTile;
-      const bool full = m.tkind[e0 + it] == SA_TILE_FULL && kbase + kTile <= a.N && p < a.N;
-      if (full) {
+      int src, kbase, kind, cnt;
+      wl.entry(m, it, src, kbase, kind, cnt);
+      // The branch taken depends only on CTA-uniform values (kind, src,
+      // kbase); rows past the end of the sequence are handled inside each.
+      const bool row_ok = p < a.N;
+      if (kind == SA_TILE_FULL && (src || kbase + kTile <= a.N)) {
 #pragma unroll
-        for (int c = 0; c < 128; ++c) x[c] *= sl2;
+        for (int c = 0; c < 128; ++c) x[c] = row_ok ? x[c] * sl2 : -INFINITY;
+      } else if (kind == kTileCount) {
+        // compacted sink/gist keys, all visible: only the first cnt columns exist
+#pragma unroll
+        for (int c = 0; c < 128; ++c) x[c] = (c < cnt && row_ok) ? x[c] * sl2 : -INFINITY;
+      } else if (gzip) {
+        // this row's block bits over the key tile, then the causal cut
+        if (m.b >= kTile) {
+          const int jb = kbase / m.b;  // the whole key tile lies in one block
+          const bool blk = row_ok && ((rowbits[jb >> 5] >> (jb & 31)) & 1u);
+#pragma unroll
+          for (int c = 0; c < 128; ++c)
+            x[c] = (blk && kbase + c <= p && kbase + c < a.N) ? x[c] * sl2 : -INFINITY;
+        } else if (lb >= 2) {
+          const int kb0 = kbase >> lb;  // 128 / b <= 32 blocks, inside one word
+          const uint32_t bb = row_ok ? (rowbits[kb0 >> 5] >> (kb0 & 31)) : 0u;
+#pragma unroll
+          for (int c = 0; c < 128; ++c)
+            x[c] = (((bb >> (c >> lb)) & 1u) && kbase + c <= p && kbase + c < a.N) ? x[c] * sl2
+                                                                                   : -INFINITY;
+        } else {
+#pragma unroll
+          for (int c = 0; c < 128; ++c) {
+            const int kq = kbase + c, jb = kq >> lb;
+            const bool v = row_ok && kq <= p && kq < a.N && ((rowbits[jb >> 5] >> (jb & 31)) & 1u);
+            x[c] = v ? x[c] * sl2 : -INFINITY;
+          }
+        }
       } else {
+        // gist near tile: each lane fetches 4 column codes (logical position |
+        // always-visible bit), shared across the warp with shuffles
+        int32_t cw[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int kq = kbase + 32 * j + lane;
+          int32_t code = 0x3FFFFFFF;  // no key: never visible
+          if (kq < a.N) {
+            const int lj = m.perm[kq];
+            const bool always = lj < m.sinks || ((m.gist_bits[lj >> 5] >> (lj & 31)) & 1u);
+            code = lj | (always ? 0x40000000 : 0);
+          }
+          cw[j] = code;
+        }
 #pragma unroll
         for (int c = 0; c < 128; ++c) {
-          const int kq = kbase + c;
-          bool vis = p < a.N && kq < a.N;
-          if (vis) {
-            if (gzip) {
-              const int jb = kq / m.b;
-              vis = kq <= p && ((rowbits[jb >> 5] >> (jb & 31)) & 1u);
-            } else {
-              const int lj = m.perm[kq];
-              const bool g = (m.gist_bits[lj >> 5] >> (lj & 31)) & 1u;
-              vis = lj <= li && (lj < m.sinks || g || (li - lj) < m.window);
-            }
-          }
-          x[c] = vis ? x[c] * sl2 : -INFINITY;
+          const int code = __shfl_sync(0xffffffffu, cw[c >> 5], c & 31);
+          const int lj = code & 0x3FFFFFFF;
+          const bool v = row_ok && lj <= li && ((code & 0x40000000) || li - lj < m.window);
+          x[c] = v ? x[c] * sl2 : -INFINITY;
         }
       }
       float mx = -INFINITY;
@@ -359,14 +450,57 @@ static bool make_map(CUtensorMap* map, const void* base, int d, int H, int N, in
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Gist mode: copies the K and V rows of every sink / gist (far_idx, logical
+// order) into dense [Bt, N, Hkv, D] buffers, and zero-fills the rest of the
+// last 128-row tile so that masked columns multiply finite values.
 template <int D>
-static cudaError_t fwd_tc_launch(const AttnArgs& a, const MaskArgs& m, cudaStream_t s) {
+__global__ void __launch_bounds__(256) gist_gather_kernel(AttnArgs a, MaskArgs m,
+                                                          __nv_bfloat16* kc, __nv_bfloat16* vc) {
+  const int f = blockIdx.x * 8 + (threadIdx.x >> 5), bt = blockIdx.y, lane = threadIdx.x & 31;
+  const int nf = m.far_ptr[m.T];
+  const int nf_pad = (nf + kTile - 1) / kTile * kTile;
+  if (f >= nf_pad || f >= a.N) return;
+  const int64_t row = (int64_t)a.Hkv * D;  // elements per compacted row
+  __nv_bfloat16* dk = kc + ((int64_t)bt * a.N + f) * row;
+  __nv_bfloat16* dv = vc + ((int64_t)bt * a.N + f) * row;
+  for (int x = lane * 8; x < row; x += 32 * 8) {
+    const int hh = x / D, c = x % D;
+    uint4 kv = make_uint4(0, 0, 0, 0), vv = make_uint4(0, 0, 0, 0);
+    if (f < nf) {
+      const int src = m.far_idx[f];
+      kv = *reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(a.k) +
+                                           bt * a.ks[0] + (int64_t)src * a.ks[1] + hh * a.ks[2] + c);
+      vv = *reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(a.v) +
+                                           bt * a.vs[0] + (int64_t)src * a.vs[1] + hh * a.vs[2] + c);
+    }
+    *reinterpret_cast<uint4*>(dk + x) = kv;
+    *reinterpret_cast<uint4*>(dv + x) = vv;
+  }
+}
+
+template <int D>
+static cudaError_t fwd_tc_launch(const AttnArgs& a, const MaskArgs& m, void* compact,
+                                 cudaStream_t s) {
   FwdTcParams P;
   memset(&P, 0, sizeof(P));
   if (!make_map(&P.tmq, a.q, D, a.Hq, a.N, a.Bt, a.qs) ||
       !make_map(&P.tmk, a.k, D, a.Hkv, a.N, a.Bt, a.ks) ||
       !make_map(&P.tmv, a.v, D, a.Hkv, a.N, a.Bt, a.vs))
     return cudaErrorInvalidValue;
+  P.tmkc = P.tmk;
+  P.tmvc = P.tmv;
+  if (m.kind == SA_MASK_GIST) {
+    const int64_t row = (int64_t)a.Hkv * D;
+    __nv_bfloat16* kc = static_cast<__nv_bfloat16*>(compact);
+    __nv_bfloat16* vc = kc + (int64_t)a.Bt * a.N * row;
+    const int64_t cs[3] = {(int64_t)a.N * row, row, D};
+    if (!make_map(&P.tmkc, kc, D, a.Hkv, a.N, a.Bt, cs) ||
+        !make_map(&P.tmvc, vc, D, a.Hkv, a.N, a.Bt, cs))
+      return cudaErrorInvalidValue;
+    gist_gather_kernel<D><<<dim3((a.N + 7) / 8, a.Bt), 256, 0, s>>>(a, m, kc, vc);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
   P.a = a;
   P.m = m;
   const int bytes = (int)FwdLayout<D>::bytes;
@@ -377,9 +511,11 @@ static cudaError_t fwd_tc_launch(const AttnArgs& a, const MaskArgs& m, cudaStrea
   return cudaGetLastError();
 }
 
-cudaError_t launch_fwd_tc(int d, const AttnArgs& a, const MaskArgs& m, cudaStream_t s) {
-  if (d == 64) return fwd_tc_launch<64>(a, m, s);
-  if (d == 128) return fwd_tc_launch<128>(a, m, s);
+// `compact`: gist mode only, 2 * Bt * N * Hkv * d bf16 of workspace.
+cudaError_t launch_fwd_tc(int d, const AttnArgs& a, const MaskArgs& m, void* compact,
+                          cudaStream_t s) {
+  if (d == 64) return fwd_tc_launch<64>(a, m, compact, s);
+  if (d == 128) return fwd_tc_launch<128>(a, m, compact, s);
   return cudaErrorInvalidValue;
 }
 

@@ -24,6 +24,8 @@ struct MaskArgs {
   // gist
   const int32_t* perm;      // physical -> logical
   const uint32_t* gist_bits;
+  const int32_t* far_idx;   // sinks + gists in logical order (physical indices)
+  const int32_t* far_ptr;   // [T+1] far keys below each key tile
   int sinks, window;
   uint8_t head_class[kMaxHeads];  // gzip: class of each query head
 };

@@ -186,6 +186,7 @@ struct GistBuild {
   int64_t tregion;
   uint32_t* gist_bits;
   int32_t* perm;
+  int32_t *far_idx, *far_ptr;
   int32_t *trp, *tcol, *tcp, *trow;
   int8_t *tkind, *tkind_t;
 };
@@ -275,6 +276,37 @@ __global__ void __launch_bounds__(1024) gist_build_kernel(GistBuild p) {
       }
       before += __popc(gw);
     }
+    // keys visible to every later query: sinks and gists of this tile
+    int nf = 0;
+    for (int c = 0; c < kTile / 32; ++c) {
+      const int pos = j0 + c * 32 + lane;
+      nf += __popc(__ballot_sync(0xffffffffu, pos < N && (pos < p.sinks || is_gist(p.gist_bits, pos))));
+    }
+    if (lane == 0) p.far_ptr[J + 1] = nf;
+  }
+  if (threadIdx.x == 0) p.far_ptr[0] = 0;
+  __syncthreads();
+  block_inclusive_scan(p.far_ptr + 1, T, 0);
+  // far_idx: the physical index of every sink / gist, in logical order
+  for (int J = warp; J < T; J += nwarps) {
+    const int j0 = J * kTile, n = min(kTile, N - j0);
+    const int ng = count_gists(p.gist_bits, j0, j0 + n);
+    int f = p.far_ptr[J], gbefore = 0;
+    for (int c = 0; c < kTile / 32; ++c) {
+      const int off = c * 32 + lane, pos = j0 + off;
+      const bool ok = pos < N;
+      const bool g = ok && is_gist(p.gist_bits, pos);
+      const bool far = ok && (pos < p.sinks || g);
+      const uint32_t gmask = __ballot_sync(0xffffffffu, g);
+      const uint32_t fmask = __ballot_sync(0xffffffffu, far);
+      const uint32_t below = (1u << lane) - 1u;
+      if (far) {
+        const int gb = gbefore + __popc(gmask & below);
+        p.far_idx[f + __popc(fmask & below)] = j0 + (g ? (n - ng) + gb : off - gb);
+      }
+      f += __popc(fmask);
+      gbefore += __popc(gmask);
+    }
   }
   __syncthreads();
   for (int I = threadIdx.x; I < T; I += blockDim.x) {
@@ -349,6 +381,8 @@ cudaError_t launch_gist_build(const sa_mask_desc& d, const uint8_t* flags,
   p.tregion = (int64_t)p.T * (p.T + 1) / 2;
   p.gist_bits = L.gist_bits;
   p.perm = L.perm;
+  p.far_idx = L.far_idx;
+  p.far_ptr = L.far_ptr;
   p.trp = L.tile_row_ptr; p.tcol = L.tile_col; p.tkind = L.tile_kind;
   p.tcp = L.tile_col_ptr; p.trow = L.tile_row; p.tkind_t = L.tile_kind_t;
   gist_build_kernel<<<1, 1024, 0, s>>>(p);

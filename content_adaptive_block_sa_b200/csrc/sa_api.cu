@@ -13,7 +13,7 @@ cudaError_t launch_gist_build(const sa_mask_desc&, const uint8_t*, const sa_bloc
                               cudaStream_t);
 cudaError_t launch_fwd_simt(int dtype, int d, const AttnArgs&, const MaskArgs&, cudaStream_t);
 cudaError_t launch_bwd_simt(int dtype, int d, const AttnArgs&, const MaskArgs&, cudaStream_t);
-cudaError_t launch_fwd_tc(int d, const AttnArgs&, const MaskArgs&, cudaStream_t);
+cudaError_t launch_fwd_tc(int d, const AttnArgs&, const MaskArgs&, void* compact, cudaStream_t);
 cudaError_t launch_decode(const sa_decode_desc&, const void*, const void*, const void*,
                           const void*, const void*, int32_t*, void*, float*, void*,
                           cudaStream_t);
@@ -83,6 +83,8 @@ sa_block_lists_sizes capacity(const sa_mask_desc& d) {
   } else {
     c.perm = d.seq_len;
     c.gist_bits = (d.seq_len + 31) / 32;
+    c.far_idx = d.seq_len;
+    c.far_ptr = T + 1;
   }
   return c;
 }
@@ -98,7 +100,7 @@ sa_status check_lists(const sa_mask_desc& d, const sa_block_lists* L) {
     SA_CHECK(L->row_ptr && L->col_idx && L->col_ptr && L->row_idx && L->bits, SA_ERR_INVALID_ARG);
     SA_CHECK(L->cap_nnz >= c.nnz, SA_ERR_WORKSPACE);
   } else {
-    SA_CHECK(L->perm && L->gist_bits, SA_ERR_INVALID_ARG);
+    SA_CHECK(L->perm && L->gist_bits && L->far_idx && L->far_ptr, SA_ERR_INVALID_ARG);
   }
   return SA_OK;
 }
@@ -158,6 +160,8 @@ MaskArgs make_mask_args(const sa_mask_desc& d, const sa_block_lists& L) {
   } else {
     m.perm = L.perm;
     m.gist_bits = L.gist_bits;
+    m.far_idx = L.far_idx;
+    m.far_ptr = L.far_ptr;
     m.sinks = d.sinks;
     m.window = d.window;
   }
@@ -278,6 +282,9 @@ sa_status sa_forward_workspace_size(const sa_attn_desc* attn, const sa_mask_desc
   if (st != SA_OK) return st;
   SA_CHECK(bytes != nullptr, SA_ERR_INVALID_ARG);
   *bytes = kStatusBytes;
+  if (mask->kind == SA_MASK_GIST)  // compacted sink/gist K and V (tensor-core path)
+    *bytes += 2 * round256((size_t)attn->batch * attn->seq_len * attn->num_kv_heads *
+                           attn->head_dim * 2);
   return SA_OK;
 }
 
@@ -293,7 +300,9 @@ sa_status sa_forward(const sa_attn_desc* attn, const sa_mask_desc* mask, const v
            SA_ERR_INVALID_ARG);
   st = check_lists(*mask, lists);
   if (st != SA_OK) return st;
-  st = check_ws(ws, ws_bytes, kStatusBytes);
+  size_t need = 0;
+  sa_forward_workspace_size(attn, mask, &need);
+  st = check_ws(ws, ws_bytes, need);
   if (st != SA_OK) return st;
   AttnArgs a = make_attn_args(*attn);
   a.q = q; a.k = k; a.v = v; a.o = o; a.lse = lse;
@@ -305,7 +314,7 @@ sa_status sa_forward(const sa_attn_desc* attn, const sa_mask_desc* mask, const v
   if (st != SA_OK) return st;
   const MaskArgs m = make_mask_args(*mask, *lists);
   if (impl == SA_IMPL_TENSOR_CORES)
-    return cuda_status(launch_fwd_tc(attn->head_dim, a, m, stream));
+    return cuda_status(launch_fwd_tc(attn->head_dim, a, m, (char*)ws + kStatusBytes, stream));
   return cuda_status(launch_fwd_simt(attn->dtype, attn->head_dim, a, m, stream));
 }
 

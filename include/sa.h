@@ -152,6 +152,12 @@ typedef struct sa_mask_desc {
  *             order).
  *  gist_bits  uint32 [ceil(N/32)]: bit p%32 of word p/32 is 1 iff LOGICAL
  *             position p is a gist.
+ *  far_idx    int32 [N]: the keys every later query sees whatever its window
+ *             (sinks and gists), in logical order, as PHYSICAL indices.
+ *  far_ptr    int32 [T+1]: far_ptr[J] = number of those keys at logical
+ *             positions below 128*J. Query tile I's window cannot reach below
+ *             key tile Jlo = max(0, I - ceil((W-1)/128)), so the keys it sees
+ *             there are exactly far_idx[0 .. far_ptr[Jlo]).
  */
 typedef struct sa_block_lists {
   int32_t* row_ptr;
@@ -167,6 +173,8 @@ typedef struct sa_block_lists {
   int8_t* tile_kind_t;
   int32_t* perm;
   uint32_t* gist_bits;
+  int32_t* far_idx;
+  int32_t* far_ptr;
   int64_t cap_nnz;       /* elements of col_idx and row_idx      */
   int64_t cap_tile_nnz;  /* elements of tile_col/_kind/_row/_kind_t */
 } sa_block_lists;
@@ -175,7 +183,7 @@ typedef struct sa_block_lists {
 typedef struct sa_block_lists_sizes {
   int64_t row_ptr, nnz, bits;
   int64_t tile_row_ptr, tile_nnz;
-  int64_t perm, gist_bits;
+  int64_t perm, gist_bits, far_idx, far_ptr;
 } sa_block_lists_sizes;
 
 /* Attention shapes.

@@ -90,6 +90,7 @@ def test_capacity_and_validation(sa):
     assert caps.tile_nnz == 6 * 512 * 513 // 2 and caps.bits == 6 * 512 * 16
     st, caps = _caps(sa, sa.gist_mask(32768, 32, 128, 4, 128))
     assert st == 0 and caps.perm == 32768 and caps.gist_bits == 1024 and caps.tile_row_ptr == 257
+    assert caps.far_idx == 32768 and caps.far_ptr == 257
     bad = [sa.gzip_mask(1, 1000, 64, 1, 4),      # N % b != 0
            sa.gzip_mask(1, 960, 96, 1, 4),       # b neither divides nor is a multiple of 128
            sa.gzip_mask(1, 1024, 64, -1, 4),     # negative window
@@ -139,7 +140,7 @@ def test_tensor_core_request_on_fp32_is_unsupported_before_any_launch(sa):
     fake = C.c_void_p(1 << 20)  # never dereferenced: validation fails first
     caps = L.sa_block_lists_sizes()
     sa.lib().sa_block_lists_capacity(C.byref(md), C.byref(caps))
-    lists = L.sa_block_lists(*([fake.value] * 13), caps.nnz, caps.tile_nnz)
+    lists = L.sa_block_lists(*([fake.value] * 15), caps.nnz, caps.tile_nnz)
     st = (C.c_int64 * 3)(1024 * 4 * 64, 4 * 64, 64)
     ad = L.sa_attn_desc(dtype=L.SA_DTYPE_FP32, batch=1, seq_len=1024, num_q_heads=4, num_kv_heads=4,
                         head_dim=64, q_strides=st, k_strides=st, v_strides=st, o_strides=st,

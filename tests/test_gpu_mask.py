@@ -100,6 +100,9 @@ def check_gist(sa, lists, N, sinks, ratio, window, tail, flags=None):
     assert np.array_equal(_np(lists.tile_col_ptr), otcp)
     assert np.array_equal(_np(lists.tile_row)[:otcp[-1]], otr)
     assert np.array_equal(_np(lists.tile_kind_t)[:otcp[-1]], otkt)
+    far_idx, far_ptr = Gi.always_visible_keys(g, sinks, perm, 128)
+    assert np.array_equal(_np(lists.far_ptr), far_ptr)
+    assert np.array_equal(_np(lists.far_idx)[:far_ptr[-1]], far_idx)
 
 
 @pytest.mark.parametrize("N,sinks,ratio,window,tail", [
