@@ -118,8 +118,10 @@ __global__ void __launch_bounds__(192, 1) fwd_tc_kernel(const __grid_constant__ 
   const MaskArgs& m = P.m;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int T = m.T;
-  const int I = T - 1 - (int)blockIdx.x;  // long lists (late tiles) first
-  const int h = blockIdx.y, bt = blockIdx.z;
+  // late query tiles (long lists) of every head and sequence first
+  const int hb = a.Hq * a.Bt;
+  const int I = T - 1 - (int)(blockIdx.x / hb);
+  const int h = (int)(blockIdx.x % hb) % a.Hq, bt = (int)(blockIdx.x % hb) / a.Hq;
   const int hk = h / (a.Hq / a.Hkv);
   const int list = list_of(m, bt, h);
   WorkList wl;
@@ -265,13 +267,16 @@ __global__ void __launch_bounds__(192, 1) fwd_tc_kernel(const __grid_constant__ 
       // The branch taken depends only on CTA-uniform values (kind, src,
       // kbase); rows past the end of the sequence are handled inside each.
       const bool row_ok = p < a.N;
+      // scores stay unscaled here; the scale is folded into the exponent
       if (kind == SA_TILE_FULL && (src || kbase + kTile <= a.N)) {
+        if (!row_ok) {
 #pragma unroll
-        for (int c = 0; c < 128; ++c) x[c] = row_ok ? x[c] * sl2 : -INFINITY;
+          for (int c = 0; c < 128; ++c) x[c] = -INFINITY;
+        }
       } else if (kind == kTileCount) {
         // compacted sink/gist keys, all visible: only the first cnt columns exist
 #pragma unroll
-        for (int c = 0; c < 128; ++c) x[c] = (c < cnt && row_ok) ? x[c] * sl2 : -INFINITY;
+        for (int c = 0; c < 128; ++c) x[c] = (c < cnt && row_ok) ? x[c] : -INFINITY;
       } else if (gzip) {
         // this row's block bits over the key tile, then the causal cut
         if (m.b >= kTile) {
@@ -279,20 +284,20 @@ __global__ void __launch_bounds__(192, 1) fwd_tc_kernel(const __grid_constant__ 
           const bool blk = row_ok && ((rowbits[jb >> 5] >> (jb & 31)) & 1u);
 #pragma unroll
           for (int c = 0; c < 128; ++c)
-            x[c] = (blk && kbase + c <= p && kbase + c < a.N) ? x[c] * sl2 : -INFINITY;
+            x[c] = (blk && kbase + c <= p && kbase + c < a.N) ? x[c] : -INFINITY;
         } else if (lb >= 2) {
           const int kb0 = kbase >> lb;  // 128 / b <= 32 blocks, inside one word
           const uint32_t bb = row_ok ? (rowbits[kb0 >> 5] >> (kb0 & 31)) : 0u;
 #pragma unroll
           for (int c = 0; c < 128; ++c)
-            x[c] = (((bb >> (c >> lb)) & 1u) && kbase + c <= p && kbase + c < a.N) ? x[c] * sl2
+            x[c] = (((bb >> (c >> lb)) & 1u) && kbase + c <= p && kbase + c < a.N) ? x[c]
                                                                                    : -INFINITY;
         } else {
 #pragma unroll
           for (int c = 0; c < 128; ++c) {
             const int kq = kbase + c, jb = kq >> lb;
             const bool v = row_ok && kq <= p && kq < a.N && ((rowbits[jb >> 5] >> (jb & 31)) & 1u);
-            x[c] = v ? x[c] * sl2 : -INFINITY;
+            x[c] = v ? x[c] : -INFINITY;
           }
         }
       } else {
@@ -315,13 +320,13 @@ __global__ void __launch_bounds__(192, 1) fwd_tc_kernel(const __grid_constant__ 
           const int code = __shfl_sync(0xffffffffu, cw[c >> 5], c & 31);
           const int lj = code & 0x3FFFFFFF;
           const bool v = row_ok && lj <= li && ((code & 0x40000000) || li - lj < m.window);
-          x[c] = v ? x[c] * sl2 : -INFINITY;
+          x[c] = v ? x[c] : -INFINITY;
         }
       }
       float mx = -INFINITY;
 #pragma unroll
       for (int c = 0; c < 128; ++c) mx = fmaxf(mx, x[c]);
-      const float m_new = fmaxf(m_run, mx);
+      const float m_new = fmaxf(m_run, mx * sl2);  // scale > 0 keeps the order
       const bool resc = m_new > m_run + 8.f;  // true on the first finite max
       const float m_use = resc ? m_new : m_run;
       float rowsum = 0.f;
@@ -332,11 +337,10 @@ __global__ void __launch_bounds__(192, 1) fwd_tc_kernel(const __grid_constant__ 
       } else {
 #pragma unroll
         for (int c = 0; c < 64; ++c) {
-          const float p0 = ex2(x[2 * c] - m_use), p1 = ex2(x[2 * c + 1] - m_use);
-          __nv_bfloat162 v = __floats2bfloat162_rn(p0, p1);
-          const float2 f = __bfloat1622float2(v);
-          rowsum += f.x + f.y;
-          pk[c] = *reinterpret_cast<uint32_t*>(&v);
+          const float p0 = ex2(fmaf(x[2 * c], sl2, -m_use));
+          const float p1 = ex2(fmaf(x[2 * c + 1], sl2, -m_use));
+          rowsum += p0 + p1;
+          pk[c] = pack_bf16(p0, p1);
         }
       }
       const float alpha = !resc ? 1.f : (m_run == -INFINITY ? 0.f : ex2(m_run - m_use));
@@ -435,7 +439,7 @@ static EncodeTiledFn encode_fn() {
 }
 
 // [Bt, N, H, d] bf16 with element strides {batch, seq, head}; box 64 x 1 x 128 x 1.
-static bool make_map(CUtensorMap* map, const void* base, int d, int H, int N, int Bt,
+bool make_tile_map(CUtensorMap* map, const void* base, int d, int H, int N, int Bt,
                      const int64_t* s) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
@@ -483,9 +487,9 @@ static cudaError_t fwd_tc_launch(const AttnArgs& a, const MaskArgs& m, void* com
                                  cudaStream_t s) {
   FwdTcParams P;
   memset(&P, 0, sizeof(P));
-  if (!make_map(&P.tmq, a.q, D, a.Hq, a.N, a.Bt, a.qs) ||
-      !make_map(&P.tmk, a.k, D, a.Hkv, a.N, a.Bt, a.ks) ||
-      !make_map(&P.tmv, a.v, D, a.Hkv, a.N, a.Bt, a.vs))
+  if (!make_tile_map(&P.tmq, a.q, D, a.Hq, a.N, a.Bt, a.qs) ||
+      !make_tile_map(&P.tmk, a.k, D, a.Hkv, a.N, a.Bt, a.ks) ||
+      !make_tile_map(&P.tmv, a.v, D, a.Hkv, a.N, a.Bt, a.vs))
     return cudaErrorInvalidValue;
   P.tmkc = P.tmk;
   P.tmvc = P.tmv;
@@ -494,8 +498,8 @@ static cudaError_t fwd_tc_launch(const AttnArgs& a, const MaskArgs& m, void* com
     __nv_bfloat16* kc = static_cast<__nv_bfloat16*>(compact);
     __nv_bfloat16* vc = kc + (int64_t)a.Bt * a.N * row;
     const int64_t cs[3] = {(int64_t)a.N * row, row, D};
-    if (!make_map(&P.tmkc, kc, D, a.Hkv, a.N, a.Bt, cs) ||
-        !make_map(&P.tmvc, vc, D, a.Hkv, a.N, a.Bt, cs))
+    if (!make_tile_map(&P.tmkc, kc, D, a.Hkv, a.N, a.Bt, cs) ||
+        !make_tile_map(&P.tmvc, vc, D, a.Hkv, a.N, a.Bt, cs))
       return cudaErrorInvalidValue;
     gist_gather_kernel<D><<<dim3((a.N + 7) / 8, a.Bt), 256, 0, s>>>(a, m, kc, vc);
     cudaError_t e = cudaGetLastError();
@@ -507,7 +511,7 @@ static cudaError_t fwd_tc_launch(const AttnArgs& a, const MaskArgs& m, void* com
   cudaError_t e = cudaFuncSetAttribute(fwd_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        bytes);
   if (e != cudaSuccess) return e;
-  fwd_tc_kernel<D><<<dim3(m.T, a.Hq, a.Bt), 192, bytes, s>>>(P);
+  fwd_tc_kernel<D><<<dim3(m.T * a.Hq * a.Bt), 192, bytes, s>>>(P);
   return cudaGetLastError();
 }
 

@@ -41,13 +41,14 @@ __device__ __forceinline__ bool block_visible(int cls, const uint8_t* f, int w, 
   return cls == SA_CLASS_LOCAL ? loc : cls == SA_CLASS_LITERAL ? lit : (loc || lit);
 }
 
-// Kind of tile pair (I, J), or -1 when it holds no visible token pair.
-__device__ int gzip_tile_kind(const GzipBuild& p, int cls, const uint8_t* f, int I, int J) {
+// Kind of tile pair (I, J), or -1 when it holds no visible token pair
+// (b < 128, a power of two: lb = log2 b).
+__device__ int gzip_tile_kind(const GzipBuild& p, int lb, int cls, const uint8_t* f, int I, int J) {
   if (J > I) return -1;
   const int q_end = min(p.N, (I + 1) * kTile);
   if (J == I) return (q_end - I * kTile == 1) ? SA_TILE_FULL : SA_TILE_MASKED;
-  const int qb0 = (I * kTile) / p.b, qb1 = (q_end - 1) / p.b;
-  const int kb0 = (J * kTile) / p.b, kb1 = (min(p.N, (J + 1) * kTile) - 1) / p.b;
+  const int qb0 = (I * kTile) >> lb, qb1 = (q_end - 1) >> lb;
+  const int kb0 = (J * kTile) >> lb, kb1 = (min(p.N, (J + 1) * kTile) - 1) >> lb;
   bool any = false, all = true;
   for (int i = qb0; i <= qb1; ++i)
     for (int j = kb0; j <= kb1; ++j) {
@@ -144,11 +145,59 @@ __global__ void __launch_bounds__(1024) gzip_build_kernel(GzipBuild p) {
   }
 
   // ---- tile lists (CSR) and their transpose (CSC)
+  __syncthreads();  // the block lists above are read below
   const int T = p.T;
   int32_t* trp = p.trp + (int64_t)bc * (T + 1);
+  int32_t* tcp = p.tcp + (int64_t)bc * (T + 1);
+  if (p.b >= kTile) {
+    // r whole tiles per block: key tile J of a visited block kb is FULL,
+    // except the diagonal tile; tiles of the diagonal block past I are skipped
+    const int r = p.b / kTile;
+    for (int I = threadIdx.x; I < T; I += blockDim.x) {
+      const int i = I / r;
+      trp[I + 1] = (rp[i + 1] - rp[i] - 1) * r + (I - i * r + 1);
+    }
+    if (threadIdx.x == 0) trp[0] = (int32_t)(bc * p.tregion);
+    __syncthreads();
+    block_inclusive_scan(trp + 1, T, (int32_t)(bc * p.tregion));
+    for (int I = threadIdx.x; I < T; I += blockDim.x) {
+      const int i = I / r;
+      int n = trp[I];
+      for (int e = rp[i]; e < rp[i + 1]; ++e) {
+        const int kb = p.col_idx[e];
+        const int last = kb < i ? kb * r + r - 1 : I;
+        for (int J = kb * r; J <= last; ++J) {
+          p.tcol[n] = J;
+          p.tkind[n] = (int8_t)(J == I ? SA_TILE_MASKED : SA_TILE_FULL);
+          ++n;
+        }
+      }
+    }
+    for (int J = threadIdx.x; J < T; J += blockDim.x) {
+      const int j = J / r;
+      tcp[J + 1] = (cp[j + 1] - cp[j] - 1) * r + (j * r + r - J);
+    }
+    if (threadIdx.x == 0) tcp[0] = (int32_t)(bc * p.tregion);
+    __syncthreads();
+    block_inclusive_scan(tcp + 1, T, (int32_t)(bc * p.tregion));
+    for (int J = threadIdx.x; J < T; J += blockDim.x) {
+      const int j = J / r;
+      int n = tcp[J];
+      for (int e = cp[j]; e < cp[j + 1]; ++e) {
+        const int qb = p.row_idx[e];
+        for (int I = qb == j ? J : qb * r; I < qb * r + r; ++I) {
+          p.trow[n] = I;
+          p.tkind_t[n] = (int8_t)(I == J ? SA_TILE_MASKED : SA_TILE_FULL);
+          ++n;
+        }
+      }
+    }
+    return;
+  }
+  const int lb = __ffs(p.b) - 1;  // b divides 128: a power of two
   for (int I = threadIdx.x; I < T; I += blockDim.x) {
     int cnt = 0;
-    for (int J = 0; J <= I; ++J) cnt += gzip_tile_kind(p, cls, f, I, J) >= 0;
+    for (int J = 0; J <= I; ++J) cnt += gzip_tile_kind(p, lb, cls, f, I, J) >= 0;
     trp[I + 1] = cnt;
   }
   if (threadIdx.x == 0) trp[0] = (int32_t)(bc * p.tregion);
@@ -157,14 +206,13 @@ __global__ void __launch_bounds__(1024) gzip_build_kernel(GzipBuild p) {
   for (int I = threadIdx.x; I < T; I += blockDim.x) {
     int n = trp[I];
     for (int J = 0; J <= I; ++J) {
-      const int k = gzip_tile_kind(p, cls, f, I, J);
+      const int k = gzip_tile_kind(p, lb, cls, f, I, J);
       if (k >= 0) { p.tcol[n] = J; p.tkind[n] = (int8_t)k; ++n; }
     }
   }
-  int32_t* tcp = p.tcp + (int64_t)bc * (T + 1);
   for (int J = threadIdx.x; J < T; J += blockDim.x) {
     int cnt = 0;
-    for (int I = J; I < T; ++I) cnt += gzip_tile_kind(p, cls, f, I, J) >= 0;
+    for (int I = J; I < T; ++I) cnt += gzip_tile_kind(p, lb, cls, f, I, J) >= 0;
     tcp[J + 1] = cnt;
   }
   if (threadIdx.x == 0) tcp[0] = (int32_t)(bc * p.tregion);
@@ -173,7 +221,7 @@ __global__ void __launch_bounds__(1024) gzip_build_kernel(GzipBuild p) {
   for (int J = threadIdx.x; J < T; J += blockDim.x) {
     int n = tcp[J];
     for (int I = J; I < T; ++I) {
-      const int k = gzip_tile_kind(p, cls, f, I, J);
+      const int k = gzip_tile_kind(p, lb, cls, f, I, J);
       if (k >= 0) { p.trow[n] = I; p.tkind_t[n] = (int8_t)k; ++n; }
     }
   }
@@ -209,10 +257,16 @@ __device__ int count_gists(const uint32_t* gb, int a, int b) {
   return n;
 }
 
-// first raw (non-gist) position in [a, b), or -1
+// first raw (non-gist) position in [a, b), or -1 (one 32-bit word at a time)
 __device__ int first_raw(const uint32_t* gb, int a, int b) {
-  for (int p = a; p < b; ++p)
-    if (!is_gist(gb, p)) return p;
+  for (int p = a; p < b;) {
+    const int lo = p & 31;
+    const int span = min(32 - lo, b - p);
+    uint32_t m = ~gb[p >> 5] >> lo;
+    if (span < 32) m &= (1u << span) - 1u;
+    if (m) return p + __ffs(m) - 1;
+    p += span;
+  }
   return -1;
 }
 

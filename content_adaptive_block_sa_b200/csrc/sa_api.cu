@@ -14,6 +14,8 @@ cudaError_t launch_gist_build(const sa_mask_desc&, const uint8_t*, const sa_bloc
 cudaError_t launch_fwd_simt(int dtype, int d, const AttnArgs&, const MaskArgs&, cudaStream_t);
 cudaError_t launch_bwd_simt(int dtype, int d, const AttnArgs&, const MaskArgs&, cudaStream_t);
 cudaError_t launch_fwd_tc(int d, const AttnArgs&, const MaskArgs&, void* compact, cudaStream_t);
+cudaError_t launch_bwd_tc(int d, const AttnArgs&, const MaskArgs&, void* ws, cudaStream_t);
+size_t bwd_tc_workspace(int Bt, int Hq, int T);
 cudaError_t launch_decode(const sa_decode_desc&, const void*, const void*, const void*,
                           const void*, const void*, int32_t*, void*, float*, void*,
                           cudaStream_t);
@@ -323,8 +325,9 @@ sa_status sa_backward_workspace_size(const sa_attn_desc* attn, const sa_mask_des
   sa_status st = check_attn(attn, mask);
   if (st != SA_OK) return st;
   SA_CHECK(bytes != nullptr, SA_ERR_INVALID_ARG);
-  *bytes = kStatusBytes +
-           round256((size_t)attn->batch * attn->num_q_heads * attn->seq_len * sizeof(float));
+  const size_t simt = (size_t)attn->batch * attn->num_q_heads * attn->seq_len * sizeof(float);
+  const size_t tc = bwd_tc_workspace(attn->batch, attn->num_q_heads, tiles_of(attn->seq_len));
+  *bytes = kStatusBytes + round256(simt > tc ? simt : tc);
   return SA_OK;
 }
 
@@ -341,6 +344,14 @@ sa_status sa_backward(const sa_attn_desc* attn, const sa_mask_desc* mask, const 
   if (st != SA_OK) return st;
   st = check_ws(ws, ws_bytes, need);
   if (st != SA_OK) return st;
+  // tensor cores: bf16, gzip masks with b >= 4 (gist-mode gradients and fp32
+  // inputs use the CUDA-core kernels)
+  const void* ptrs[5] = {q, k, v, o, dout};
+  const bool tc_ok = tensor_core_ok(*attn, ptrs, 5) && mask->kind == SA_MASK_GZIP &&
+                     mask->block_size >= 4 && aligned(dq, 16) && aligned(dk, 16) &&
+                     aligned(dv, 16);
+  const int impl = pick_impl(*attn, tc_ok);
+  if (impl < 0) return SA_ERR_UNSUPPORTED;
   st = clear_status(ws, stream);
   if (st != SA_OK) return st;
   AttnArgs a = make_attn_args(*attn);
@@ -349,6 +360,8 @@ sa_status sa_backward(const sa_attn_desc* attn, const sa_mask_desc* mask, const 
   a.delta = (float*)((char*)ws + kStatusBytes);
   a.status = (DeviceStatus*)ws;
   const MaskArgs m = make_mask_args(*mask, *lists);
+  if (impl == SA_IMPL_TENSOR_CORES)
+    return cuda_status(launch_bwd_tc(attn->head_dim, a, m, (char*)ws + kStatusBytes, stream));
   return cuda_status(launch_bwd_simt(attn->dtype, attn->head_dim, a, m, stream));
 }
 

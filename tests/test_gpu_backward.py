@@ -14,13 +14,16 @@ from _cases import check_close, gzip_flags_oracle, gzip_flags_product, gzip_inpu
 pytestmark = pytest.mark.gpu
 
 
-def run(sa, w, q, k, v, do, flags):
+IMPLS = {"cuda_cores": 1, "tensor_cores": 2}
+
+
+def run(sa, w, q, k, v, do, flags, impl=0):
     dt = w["dtype"]
     md = sa.gzip_mask(w["batch"], w["seq_len"], w["block"], w["window"], w["heads"])
     lists = sa.build_block_mask(md, flags)
     tq, tk, tv, tdo = (to_dev(x, dt) for x in (q, k, v, do))
     o, lse = sa.forward(tq, tk, tv, md, lists)
-    dq, dk, dv = sa.backward(tq, tk, tv, o, lse, tdo, md, lists)
+    dq, dk, dv = sa.backward(tq, tk, tv, o, lse, tdo, md, lists, impl=impl)
     torch.cuda.synchronize()
     return to_np(o), to_np(dq), to_np(dk), to_np(dv)
 
@@ -32,11 +35,18 @@ def run(sa, w, q, k, v, do, flags):
              kv_heads=4, head_dim=64, dtype="bf16"),
     W.scaled("gzip_8k", index=303, batch=1, seq_len=128 * 6, block=128, window=1, heads=4,
              kv_heads=4, head_dim=128, dtype="bf16", p_literal=0.5),
-], ids=["b16_fp32", "b64_ragged_bf16", "b128_bf16"])
-def test_backward_small(sa, w):
+    W.scaled("gzip_8k", index=304, batch=2, seq_len=16 * 40, block=16, window=3, heads=4,
+             kv_heads=4, head_dim=64, dtype="bf16", p_literal=0.4),
+    W.scaled("gzip_8k", index=305, batch=1, seq_len=256 * 4, block=256, window=1, heads=6,
+             kv_heads=6, head_dim=128, dtype="bf16", p_literal=0.5),
+], ids=["b16_fp32", "b64_ragged_bf16", "b128_bf16", "b16_bf16", "b256_h6_bf16"])
+@pytest.mark.parametrize("impl", list(IMPLS))
+def test_backward_small(sa, w, impl):
+    if w["dtype"] == "fp32" and impl == "tensor_cores":
+        pytest.skip("tensor cores take bf16 only")
     q, k, v, do = gzip_inputs(w, with_do=True)
     fp, fo = gzip_flags_product(sa, w), gzip_flags_oracle(w)
-    o, dq, dk, dv = run(sa, w, q, k, v, do, fp)
+    o, dq, dk, dv = run(sa, w, q, k, v, do, fp, IMPLS[impl])
     cls = G.head_classes(w["heads"])
     for bt in range(w["batch"]):
         masks = G.block_masks(fo[bt], w["window"])
