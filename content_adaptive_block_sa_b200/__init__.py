@@ -278,6 +278,7 @@ def gist_decode(q, gist_k, gist_v, k_cache, v_cache, chunk: int, top_k: int, win
     dd = decode_desc(q, gist_k, k_cache, o, chunk, top_k, window, softmax_scale)
     ws = decode_workspace(dd, q.device)
     sa_gist_decode(dd, q, gist_k, gist_v, k_cache, v_cache, sel, o, lse, ws, stream)
+    gist_decode.last_workspace = ws
     return sel[:, :, :top_k], o, lse
 
 

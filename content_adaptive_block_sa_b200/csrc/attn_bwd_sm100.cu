@@ -245,6 +245,7 @@ __global__ void __launch_bounds__(192, 1) bwd_tc_kernel(const __grid_constant__ 
         }
       }
       uint32_t pk[64], dk[64];
+      __syncwarp();  // the TMEM loads below are warp-collective (.sync.aligned)
 #pragma unroll
       for (int c4 = 0; c4 < 4; ++c4) {
         float sv[32], dv[32];
@@ -286,6 +287,7 @@ __global__ void __launch_bounds__(192, 1) bwd_tc_kernel(const __grid_constant__ 
         break;
       }
       tc_fence_after();
+      __syncwarp();
       const int qrow = q0 + j;
       float* dq = a.dq + (((int64_t)bt * a.N + qrow) * a.Hq + h) * D;
 #pragma unroll
@@ -307,6 +309,7 @@ __global__ void __launch_bounds__(192, 1) bwd_tc_kernel(const __grid_constant__ 
     if (ok && n > 0) {
       // the last dQ commit follows every dV / dK MMA
       tc_fence_after();
+      __syncwarp();
       float* dkr = a.dk + (((int64_t)bt * a.N + kq) * a.Hkv + hk) * D;
       float* dvr = a.dv + (((int64_t)bt * a.N + kq) * a.Hkv + hk) * D;
 #pragma unroll

@@ -255,6 +255,7 @@ __global__ void __launch_bounds__(192, 1) fwd_tc_kernel(const __grid_constant__ 
         break;
       }
       tc_fence_after();
+      __syncwarp();  // tcgen05.ld is warp-collective (.sync.aligned)
       float x[128];
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_ld32(lane_addr + s * 128 + c * 32, x + c * 32);
@@ -359,6 +360,7 @@ __global__ void __launch_bounds__(192, 1) fwd_tc_kernel(const __grid_constant__ 
           break;
         }
         tc_fence_after();
+        __syncwarp();
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           float o[32];
@@ -388,6 +390,7 @@ __global__ void __launch_bounds__(192, 1) fwd_tc_kernel(const __grid_constant__ 
         __all_sync(0xffffffffu,
                    mbar_wait(&bar[B_OD + ((n - 1) & 1)], ((n - 1) >> 1) & 1, abort, st, 23))) {
       tc_fence_after();
+      __syncwarp();
       const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
       __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.o) + bt * a.os[0] +
                             (int64_t)p * a.os[1] + (int64_t)h * a.os[2];
