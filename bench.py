@@ -361,6 +361,30 @@ def make(sa, torch, name, rank, size="full"):
     return DecodeWorkload(sa, torch, w)
 
 
+# ----------------------------------------------------------------- ranks
+def rank_barrier(world: int) -> None:
+    """Barrier across ranks (no-op on one process)."""
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def rank_max(x: float, world: int, device: str = "cuda") -> float:
+    """Max of a per-rank number over all ranks (the timing reduction only)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_value(units_per_rank: float, world: int, ms_per_step: float, scale: float) -> float:
+    """Whole-job throughput: every rank's units over the slowest rank's time."""
+    return units_per_rank * world / (ms_per_step * 1e-3) / scale
+
+
 # ----------------------------------------------------------------- main
 def run_reference(args):
     """The oracle on the host cores, on a bounded sample of the workload."""
@@ -431,16 +455,8 @@ def main():
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
 
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
-    def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    barrier = lambda: rank_barrier(world)
+    max_over_ranks = lambda x: rank_max(x, world, "cuda")
 
     wl = make(sa, torch, args.workload, rank, args.size)
     for _ in range(args.warmup):
@@ -483,14 +499,14 @@ def main():
     hbm, bf16, src = peaks()
     if wl.unit == "GB/s":
         units = wl.bytes
-        value = units * world / (ms * 1e-3) / 1e9
-        e2e_value = units * world / (e2e_ms * 1e-3) / 1e9
+        value = weak_scaling_value(units, world, ms, 1e9)
+        e2e_value = weak_scaling_value(units, world, e2e_ms, 1e9)
         ach = wl.bytes / (kern_ms * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
                 "traffic": None, "peak_source": src, "kernel": "sa_gist_decode (4 launches)"}
     else:
-        value = wl.flops * world / (ms * 1e-3) / 1e12
-        e2e_value = wl.flops * world / (e2e_ms * 1e-3) / 1e12
+        value = weak_scaling_value(wl.flops, world, ms, 1e12)
+        e2e_value = weak_scaling_value(wl.flops, world, e2e_ms, 1e12)
         ach = wl.flops_fwd / (kern_ms * 1e-3) / 1e12
         roof = {"bound": "tensor", "achieved": ach, "peak": bf16, "unit": "TFLOP/s",
                 "frac": ach / bf16, "traffic": None, "peak_source": src, "kernel": "sa_forward"}
