@@ -1,27 +1,43 @@
 // Block-sparse attention forward on the 5th-generation tensor cores (sm_100a).
 //
-// For one (128-query tile, head, sequence) per CTA, the listed 128-key tiles
-// are visited in order; everything else is skipped ("UniGist ...", Approach:
-// skipping non-visible blocks is what makes the sparse layout fast; "Gzip-
-// guided sparse attention ...", Scope: dense-then-mask gives no speed-up).
+// A work item is one (128-query tile, head, sequence); its listed 128-key
+// tiles are visited in order and everything else is skipped ("UniGist ...",
+// Approach: skipping non-visible blocks is what makes the sparse layout fast;
+// "Gzip-guided sparse attention ...", Scope: dense-then-mask gives no
+// speed-up). The kernel is persistent: one CTA per SM walks the items
+// blockIdx.x, blockIdx.x + gridDim.x, ... (late query tiles, which have the
+// longest lists, first). Ring slots and mbarrier phases run on across items,
+// so the loads and the first Q K^T of the next item overlap the softmax and
+// epilogue of the current one.
 //
-// Roles (192 threads):
-//   warp 0      TMA producer: Q once, then K_j / V_j into a 2-stage ring
-//               (128-byte swizzled, 64-column atoms), and TMEM allocation.
+// Roles (352 threads):
+//   warp 0      TMA producer: Q per item; K and V in separate rings, K one
+//               tile ahead of V (K_j is free once Q K_j^T is done, V_j only
+//               after P_j V_j); TMEM allocation.
 //   warp 1      one thread issues tcgen05.mma: S_j = Q K_j^T into one of two
-//               TMEM S buffers, then O += P_j V_j into the TMEM O accumulator.
-//               Completion is signalled with tcgen05.commit on mbarriers.
-//   warps 2-5   softmax: thread t owns query row t (TMEM lane t). It reads its
-//               S row, applies the element mask on MASKED/TAIL tiles, keeps a
-//               running max in the log2 domain and rescales its O row only
-//               when the max grew by more than 2^8 (the reference max is kept
-//               otherwise, so P <= 256), writes P (bf16) into a swizzled
-//               shared tile and hands it to the MMA thread. The epilogue
-//               divides O by the row sum and writes O (bf16) and LSE (fp32).
-// S is double-buffered so that S_{j+1} = Q K_{j+1}^T runs on the tensor core
-// while the softmax of tile j runs. Every wait is bounded; on timeout the
-// device status word is set and all roles leave after draining their copies
-// and MMAs, freeing TMEM.
+//               TMEM S buffers, then O_h += P_j[:, h-half] V_j[h-half, :] for
+//               the two column halves h = 0, 1, each into its own TMEM
+//               accumulator, with P_j read from TMEM (A operand) and V_j from
+//               shared memory. Completion is signalled with tcgen05.commit.
+//   warps 2-9   softmax, two groups of four warps: group h owns key columns
+//               [64h, 64h + 64) of every S tile; thread (h, r) owns query row
+//               r (TMEM lane r) within that half. Each half keeps its own
+//               running max (log2 domain) and row sum, so the two halves never
+//               synchronise per tile; O_h is rescaled lazily, only when the
+//               half's max grew by more than 2^8 (P <= 256 otherwise). The
+//               epilogue exchanges (max, sum) between the halves and merges:
+//               O = (2^(m_0-m) O_0 + 2^(m_1-m) O_1) / (2^(m_0-m) l_0 + 2^(m_1-m) l_1).
+//   warp 10     mask: for each visited tile, ahead of the softmax, the
+//               visibility of its 128 x 128 (row, key) pairs as 4 x 128 bit
+//               words in a shared-memory ring, so that no global load or
+//               mask arithmetic sits on the softmax's path.
+// S is double-buffered (Q K^T of tile j+1 runs while tile j's softmax runs).
+// Each half writes its bf16 P over the first 32 of its own 64 S columns, so P
+// never passes through shared memory; Q K^T(j+2) may overwrite that buffer
+// right after P V(j) is issued, as tcgen05.mma ops of one thread execute in
+// issue order. Every wait is bounded; on timeout the device status word
+// is set and all roles leave after draining their copies and MMAs, freeing
+// TMEM.
 #include <cuda.h>
 
 #include "attn_mask.cuh"
@@ -42,8 +58,8 @@ struct FwdTcParams {
 // the compacted sink/gist keys).
 constexpr int kTileCount = 3;
 
-// The CTA's visit list, the same in every role. Gzip mode: the tile list of
-// (sequence, head class, query tile). Gist mode: the dense prefix of the
+// The visit list of one item, the same in every role. Gzip mode: the tile list
+// of (sequence, head class, query tile). Gist mode: the dense prefix of the
 // compacted sink/gist keys that lie below the near tiles, then the near tiles
 // Jlo..I of the physical sequence, which take the element rule.
 struct WorkList {
@@ -85,61 +101,156 @@ struct WorkList {
   }
 };
 
-template <int D>
-struct FwdLayout {
-  static constexpr uint32_t kQ = 128 * D * 2;       // Q tile
-  static constexpr uint32_t kKV = 128 * D * 2;      // one K or V tile
-  static constexpr uint32_t kP = 128 * 128 * 2;     // one P tile
-  static constexpr uint32_t kAtom = 128 * 128;      // [128 rows][64 bf16] swizzle atom
-  static constexpr uint32_t q = 0;
-  static constexpr uint32_t k0 = kQ;
-  static constexpr uint32_t v0 = kQ + 2 * kKV;
-  static constexpr uint32_t p0 = kQ + 4 * kKV;
-  static constexpr uint32_t bars = p0 + 2 * kP;    // 16 mbarriers + TMEM slot + flags
-  static constexpr uint32_t bytes = bars + 256 + 1024;  // + alignment slack
+// Item -> (query tile, head, sequence): late query tiles of every head and
+// sequence first.
+struct Item {
+  int I, h, bt;
+  __device__ Item(int idx, int T, int Hq, int Bt) {
+    const int hb = Hq * Bt;
+    I = T - 1 - idx / hb;
+    h = (idx % hb) % Hq;
+    bt = (idx % hb) / Hq;
+  }
 };
 
-enum { B_Q = 0, B_KVF = 1, B_KVE = 3, B_SF = 5, B_SE = 7, B_PF = 9, B_OD = 11, B_DRAIN = 13 };
 
-constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kTmemO = 256;
+constexpr int kMaskSlots = 4;              // mask ring depth (tiles)
+constexpr uint32_t kMaskSlotBytes = 2048;  // [4 words][128 rows] uint32
 
 template <int D>
-__global__ void __launch_bounds__(192, 1) fwd_tc_kernel(const __grid_constant__ FwdTcParams P) {
+struct FwdLayout {
+  static constexpr int kKStages = D == 64 ? 4 : 3;  // K ring depth
+  static constexpr int kVStages = D == 64 ? 4 : 2;  // V ring depth
+  static constexpr uint32_t kQ = 128 * D * 2;        // Q tile
+  static constexpr uint32_t kKV = 128 * D * 2;       // one K or V tile
+  static constexpr uint32_t kAtom = 128 * 128;       // [128 rows][64 bf16] swizzle atom
+  static constexpr uint32_t q = 0;
+  static constexpr uint32_t k0 = kQ;
+  static constexpr uint32_t v0 = k0 + kKStages * kKV;
+  static constexpr uint32_t mask = v0 + kVStages * kKV;
+  static constexpr uint32_t ml = mask + kMaskSlots * kMaskSlotBytes;  // [2 halves][128] (max, sum)
+  static constexpr uint32_t bars = ml + 2 * 128 * 8;
+  static constexpr uint32_t bytes = bars + 512 + 1024;  // + alignment slack
+};
+
+// mbarriers. QF/QE: Q tile full / consumed (per item). KF/KE, VF/VE: K or V
+// stage full / free. SF: S buffer written. PF: P half written (TMEM). OD: P V
+// of the half done (per tile). MF/ME: mask slot written / read. OI: every MMA
+// of the item done. OF: both halves have read O (per item). ML: (max, sum)
+// exchanged. DRAIN: all MMAs done before exit.
+enum {
+  B_QF = 0, B_QE = 1, B_KF = 2, B_KE = 6, B_VF = 10, B_VE = 14, B_SF = 18, B_PF = 20,
+  B_OD = 22, B_MF = 24, B_ME = 28, B_OI = 32, B_OF = 33, B_ML = 34, B_DRAIN = 35,
+  kNumBars = 36
+};
+
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kTmemO = 256;  // O_0 at 256, O_1 at 256 + D
+constexpr int kSoftmaxThreads = 256;
+constexpr int kThreads = 64 + kSoftmaxThreads + 32;
+constexpr int kMaskWarp = 10;
+
+// Bits [0, n) set, n clamped to [0, 32].
+__device__ __forceinline__ uint32_t prefix_bits(int n) {
+  return n <= 0 ? 0u : (n >= 32 ? 0xffffffffu : ((1u << n) - 1u));
+}
+
+// Each set bit of e (nb bits) widened to a run of 2^lb bits (lb <= 4).
+__device__ __forceinline__ uint32_t widen_bits(uint32_t e, int lb, int nb) {
+  if (lb == 0) return e;
+  uint32_t w = 0u;
+  const uint32_t run = (1u << (1 << lb)) - 1u;
+  for (int i = 0; i < nb; ++i)
+    if ((e >> i) & 1u) w |= run << (i << lb);
+  return w;
+}
+
+// One query row as the mask warp sees it: position, logical position (gist
+// layout), in range, and its packed block bits (gzip).
+struct RowCtx {
+  int p, li;
+  bool ok;
+  const uint32_t* bits;
+};
+
+// Visibility of key columns [32w, 32w + 32) of a tile from one row, for gzip
+// tiles and compacted sink/gist tiles (gist near tiles take the element rule,
+// evaluated with the whole warp in the mask role). Gzip: the row's block bits
+// over the tile, then the causal cut ("Gzip-guided sparse attention ...", Core
+// equations: M restricted to j <= i). Compacted tiles: the first cnt columns.
+__device__ __forceinline__ uint32_t tile_word(const MaskArgs& m, int gzip, int lb, int N,
+                                              const RowCtx& rc, int kbase, int kind, int cnt,
+                                              int w) {
+  if (!rc.ok) return 0u;
+  if (!gzip) return kind == SA_TILE_FULL ? 0xffffffffu : prefix_bits(cnt - 32 * w);
+  if (kind == SA_TILE_FULL && kbase + kTile <= N) return 0xffffffffu;
+  const int cw0 = kbase + 32 * w;
+  const uint32_t causal = prefix_bits(min(rc.p, N - 1) - cw0 + 1);
+  if (causal == 0u) return 0u;
+  if (m.b >= kTile) {
+    const int jb = kbase / m.b;  // the whole key tile lies in one block
+    return ((rc.bits[jb >> 5] >> (jb & 31)) & 1u) ? causal : 0u;
+  }
+  if (lb >= 5) {
+    const int jb = cw0 >> lb;  // 32 columns lie in one block
+    return ((rc.bits[jb >> 5] >> (jb & 31)) & 1u) ? causal : 0u;
+  }
+  const int kb = cw0 >> lb, nb = 32 >> lb;  // nb blocks inside one bit word
+  const uint32_t e = (rc.bits[kb >> 5] >> (kb & 31)) & prefix_bits(nb);
+  return widen_bits(e, lb, nb) & causal;
+}
+
+// Number of visited tiles of item idx.
+__device__ __forceinline__ int item_tiles(const MaskArgs& m, int idx, int T, int Hq, int Bt) {
+  const Item itm(idx, T, Hq, Bt);
+  WorkList wl;
+  wl.init(m, list_of(m, itm.bt, itm.h), itm.I);
+  return wl.n;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1) fwd_tc_kernel(const __grid_constant__ FwdTcParams P) {
   using L = FwdLayout<D>;
+  constexpr int KS = L::kKStages, VS = L::kVStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const uint32_t sb = smem_u32(smem);
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + L::bars);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 16);
-  volatile int* abort = reinterpret_cast<volatile int*>(bar + 16) + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + kNumBars);
+  volatile int* abort = reinterpret_cast<volatile int*>(bar + kNumBars) + 1;
+  float2* ml = reinterpret_cast<float2*>(smem + L::ml);
+  uint32_t* mwords = reinterpret_cast<uint32_t*>(smem + L::mask);
 
   const AttnArgs& a = P.a;
   const MaskArgs& m = P.m;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int T = m.T;
-  // late query tiles (long lists) of every head and sequence first
-  const int hb = a.Hq * a.Bt;
-  const int I = T - 1 - (int)(blockIdx.x / hb);
-  const int h = (int)(blockIdx.x % hb) % a.Hq, bt = (int)(blockIdx.x % hb) / a.Hq;
-  const int hk = h / (a.Hq / a.Hkv);
-  const int list = list_of(m, bt, h);
-  WorkList wl;
-  wl.init(m, list, I);
-  const int n = wl.n;
-  const int q0 = I * kTile;
+  const int n_items = T * a.Hq * a.Bt;
   DeviceStatus* st = a.status;
 
   if (threadIdx.x == 0) {
-    mbar_init(&bar[B_Q], 1);
+    mbar_init(&bar[B_QF], 1);
+    mbar_init(&bar[B_QE], 1);
+    for (int s = 0; s < KS; ++s) {
+      mbar_init(&bar[B_KF + s], 1);
+      mbar_init(&bar[B_KE + s], 1);
+    }
+    for (int s = 0; s < VS; ++s) {
+      mbar_init(&bar[B_VF + s], 1);
+      mbar_init(&bar[B_VE + s], 1);
+    }
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&bar[B_KVF + s], 1);
-      mbar_init(&bar[B_KVE + s], 1);
       mbar_init(&bar[B_SF + s], 1);
-      mbar_init(&bar[B_SE + s], 128);
-      mbar_init(&bar[B_PF + s], 128);
+      mbar_init(&bar[B_PF + s], kSoftmaxThreads / 2);
       mbar_init(&bar[B_OD + s], 1);
     }
+    for (int s = 0; s < kMaskSlots; ++s) {
+      mbar_init(&bar[B_MF + s], 32);
+      mbar_init(&bar[B_ME + s], kSoftmaxThreads);
+    }
+    mbar_init(&bar[B_OI], 1);
+    mbar_init(&bar[B_OF], kSoftmaxThreads);
+    mbar_init(&bar[B_ML], kSoftmaxThreads);
     mbar_init(&bar[B_DRAIN], 1);
     *abort = 0;
     fence_barrier_init();
@@ -159,261 +270,375 @@ __global__ void __launch_bounds__(192, 1) fwd_tc_kernel(const __grid_constant__ 
       prefetch_tmap(&P.tmq);
       prefetch_tmap(&P.tmk);
       prefetch_tmap(&P.tmv);
-      if (wl.gist) {
+      if (m.kind == SA_MASK_GIST) {
         prefetch_tmap(&P.tmkc);
         prefetch_tmap(&P.tmvc);
       }
-      mbar_arrive_expect_tx(&bar[B_Q], L::kQ);
-      for (int at = 0; at < D / 64; ++at)
-        tma_load_4d(smem + L::q + at * L::kAtom, &P.tmq, &bar[B_Q], at * 64, h, q0, bt);
-      int last[2] = {-1, -1};
-      for (int it = 0; it < n; ++it) {
-        const int s = it & 1;
-        if (!mbar_wait(&bar[B_KVE + s], ((it >> 1) & 1) ^ 1, abort, st, 1)) break;
-        int src, k0, kind, cnt;
-        wl.entry(m, it, src, k0, kind, cnt);
-        const CUtensorMap* mk = src ? &P.tmkc : &P.tmk;
-        const CUtensorMap* mv = src ? &P.tmvc : &P.tmv;
-        mbar_arrive_expect_tx(&bar[B_KVF + s], 2 * L::kKV);
-        for (int at = 0; at < D / 64; ++at) {
-          tma_load_4d(smem + L::k0 + s * L::kKV + at * L::kAtom, mk, &bar[B_KVF + s], at * 64, hk,
-                      k0, bt);
-          tma_load_4d(smem + L::v0 + s * L::kKV + at * L::kAtom, mv, &bar[B_KVF + s], at * 64, hk,
-                      k0, bt);
+      int g = 0, k = 0, last_k = -1, last_v = -1, last_q = -1;
+      bool ok = true;
+      for (int idx = blockIdx.x; ok && idx < n_items; idx += gridDim.x, ++k) {
+        const Item itm(idx, T, a.Hq, a.Bt);
+        WorkList wl;
+        wl.init(m, list_of(m, itm.bt, itm.h), itm.I);
+        const int hk = itm.h / (a.Hq / a.Hkv);
+        // the previous item's last Q K^T has read Q
+        if (k > 0 && !mbar_wait(&bar[B_QE], (k - 1) & 1, abort, st, 1)) break;
+        mbar_arrive_expect_tx(&bar[B_QF], L::kQ);
+        for (int at = 0; at < D / 64; ++at)
+          tma_load_4d(smem + L::q + at * L::kAtom, &P.tmq, &bar[B_QF], at * 64, itm.h,
+                      itm.I * kTile, itm.bt);
+        last_q = k;
+        // K of tile it + 1 is requested before V of tile it
+        auto load = [&](bool is_k, int it) -> bool {
+          const int ns = is_k ? KS : VS;
+          const int gt = g + it, s = gt % ns;
+          uint64_t* full = &bar[(is_k ? B_KF : B_VF) + s];
+          if (!mbar_wait(&bar[(is_k ? B_KE : B_VE) + s], ((gt / ns) & 1) ^ 1, abort, st, 2))
+            return false;
+          int src, k0, kind, cnt;
+          wl.entry(m, it, src, k0, kind, cnt);
+          const CUtensorMap* map = is_k ? (src ? &P.tmkc : &P.tmk) : (src ? &P.tmvc : &P.tmv);
+          const uint32_t dst = (is_k ? L::k0 : L::v0) + s * L::kKV;
+          mbar_arrive_expect_tx(full, L::kKV);
+          for (int at = 0; at < D / 64; ++at)
+            tma_load_4d(smem + dst + at * L::kAtom, map, full, at * 64, hk, k0, itm.bt);
+          if (is_k) last_k = gt; else last_v = gt;
+          return true;
+        };
+        if (wl.n > 0) ok = load(true, 0);
+        for (int it = 0; ok && it < wl.n; ++it) {
+          if (it + 1 < wl.n) ok = load(true, it + 1);
+          if (ok) ok = load(false, it);
         }
-        last[s] = it;
+        g += wl.n;
       }
       // every copy this CTA started must land before the CTA may exit
       volatile int no_abort = 0;
-      mbar_wait(&bar[B_Q], 0, &no_abort, nullptr, 2);
-      for (int s = 0; s < 2; ++s)
-        if (last[s] >= 0) mbar_wait(&bar[B_KVF + s], (last[s] >> 1) & 1, &no_abort, nullptr, 3);
+      if (last_q >= 0) mbar_wait(&bar[B_QF], last_q & 1, &no_abort, nullptr, 3);
+      for (int s = 0; s < KS; ++s) {
+        if (last_k >= s) {
+          const int gs = last_k - ((last_k - s) % KS);
+          mbar_wait(&bar[B_KF + s], (gs / KS) & 1, &no_abort, nullptr, 4);
+        }
+      }
+      for (int s = 0; s < VS; ++s) {
+        if (last_v >= s) {
+          const int gs = last_v - ((last_v - s) % VS);
+          mbar_wait(&bar[B_VF + s], (gs / VS) & 1, &no_abort, nullptr, 5);
+        }
+      }
     }
   } else if (warp == 1) {
     if (lane == 0) {
       // --------------------------------------------------------- MMA issuer
       constexpr uint32_t kIdQK = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t kIdPV = idesc_bf16_f32(128, D, false, true);
-      bool ok = mbar_wait(&bar[B_Q], 0, abort, st, 10);
-      for (int it = 0; ok && it <= n; ++it) {
-        if (it < n) {
-          const int s = it & 1;
-          if (!mbar_wait(&bar[B_KVF + s], (it >> 1) & 1, abort, st, 11)) break;
-          if (!mbar_wait(&bar[B_SE + s], ((it >> 1) & 1) ^ 1, abort, st, 12)) break;
-          tc_fence_after();
-          const uint32_t kbase = sb + L::k0 + s * L::kKV;
+      int g = 0, k = 0;
+      bool ok = true;
+      int n_next = blockIdx.x < n_items ? item_tiles(m, blockIdx.x, T, a.Hq, a.Bt) : 0;
+      for (int idx = blockIdx.x; ok && idx < n_items; idx += gridDim.x, ++k) {
+        const int n = n_next;
+        n_next = idx + (int)gridDim.x < n_items ? item_tiles(m, idx + gridDim.x, T, a.Hq, a.Bt) : 0;
+        if (!mbar_wait(&bar[B_QF], k & 1, abort, st, 10)) break;
+        // both halves have read the previous item's O before it is overwritten
+        bool o_free = k == 0;
+        for (int it = 0; it <= n; ++it) {
+          if (it < n) {
+            // S buffer gq & 1 last held P(gq - 2), read by P V(gq - 2), which
+            // was issued before this Q K^T; tcgen05.mma ops of one thread run in
+            // issue order, so no wait is needed for it
+            const int gq = g + it, s = gq % KS, sb2 = gq & 1;
+            if (!mbar_wait(&bar[B_KF + s], (gq / KS) & 1, abort, st, 11)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t kb = sb + L::k0 + s * L::kKV;
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * L::kAtom + (kk & 3) * 32;
-            mma_bf16(tmem + s * 128, smem_desc_sw128(sb + L::q + off, 16, 1024),
-                     smem_desc_sw128(kbase + off, 16, 1024), kIdQK, kk > 0);
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t off = (kk >> 2) * L::kAtom + (kk & 3) * 32;
+              mma_bf16(tmem + sb2 * 128, smem_desc_sw128(sb + L::q + off, 16, 1024),
+                       smem_desc_sw128(kb + off, 16, 1024), kIdQK, kk > 0);
+            }
+            mma_commit(&bar[B_SF + sb2]);
+            mma_commit(&bar[B_KE + s]);
+            if (it == n - 1) mma_commit(&bar[B_QE]);
           }
-          mma_commit(&bar[B_SF + s]);
-        }
-        if (it >= 1) {
-          const int j = it - 1, s = j & 1;
-          if (!mbar_wait(&bar[B_PF + s], (j >> 1) & 1, abort, st, 13)) break;
-          tc_fence_after();
-          const uint32_t pbase = sb + L::p0 + s * L::kP;
-          const uint32_t vbase = sb + L::v0 + s * L::kKV;
+          if (it >= 1) {
+            const int gp = g + it - 1, s = gp % VS;
+            if (!o_free) {
+              if (!mbar_wait(&bar[B_OF], (k - 1) & 1, abort, st, 13)) {
+                ok = false;
+                break;
+              }
+              o_free = true;
+            }
+            if (!mbar_wait(&bar[B_VF + s], (gp / VS) & 1, abort, st, 14)) {
+              ok = false;
+              break;
+            }
+            const uint32_t vb = sb + L::v0 + s * L::kKV;
+            for (int hf = 0; hf < 2; ++hf) {
+              if (!mbar_wait(&bar[B_PF + hf], gp & 1, abort, st, 15 + hf)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              // P of this half: bf16 pairs in the first 32 columns of its S columns
+              const uint32_t pa = tmem + (gp & 1) * 128 + hf * 64;
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint64_t ad = smem_desc_sw128(pbase + (kk >> 2) * L::kAtom + (kk & 3) * 32, 16, 1024);
-            const uint64_t bd = smem_desc_sw128(vbase + kk * 2048, L::kAtom, 1024);
-            mma_bf16(tmem + kTmemO, ad, bd, kIdPV, (j > 0 || kk > 0) ? 1u : 0u);
+              for (int kk = 0; kk < 4; ++kk) {
+                const uint64_t bd = smem_desc_sw128(vb + (hf * 4 + kk) * 2048, L::kAtom, 1024);
+                mma_bf16_ts(tmem + kTmemO + hf * D, pa + kk * 8, bd, kIdPV,
+                            (it > 1 || kk > 0) ? 1u : 0u);
+              }
+              mma_commit(&bar[B_OD + hf]);
+            }
+            if (!ok) break;
+            mma_commit(&bar[B_VE + s]);
           }
-          mma_commit(&bar[B_OD + s]);
-          mma_commit(&bar[B_KVE + s]);
         }
+        if (!ok) break;
+        if (n == 0) {
+          mma_commit(&bar[B_QE]);
+          if (!o_free && !mbar_wait(&bar[B_OF], (k - 1) & 1, abort, st, 13)) break;
+        }
+        mma_commit(&bar[B_OI]);
+        g += n;
       }
       // drain: every MMA issued above has completed
       mma_commit(&bar[B_DRAIN]);
       volatile int no_abort = 0;
-      mbar_wait(&bar[B_DRAIN], 0, &no_abort, nullptr, 14);
+      mbar_wait(&bar[B_DRAIN], 0, &no_abort, nullptr, 17);
     }
-  } else {
-    // --------------------------------------------------------------- softmax
-    const int quarter = warp & 3;
-    const int r = quarter * 32 + lane;
-    const int p = q0 + r;
-    const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
-    const float sl2 = a.scale * 1.4426950408889634f;
-    float m_run = -INFINITY, l_run = 0.f;
+  } else if (warp == kMaskWarp) {
+    // -------------------------------------------------------------- mask
+    // Lane l writes rows l, l + 32, l + 64, l + 96 of every slot:
+    // word w of row r at mwords[slot][w][r].
     const int gzip = m.kind == SA_MASK_GZIP;
-    const uint32_t* rowbits = nullptr;
-    int li = 0;
-    if (gzip && p < a.N) rowbits = m.bits + ((int64_t)list * m.B + p / m.b) * m.words;
-    if (!gzip && p < a.N) li = m.perm[p];
     const int lb = (gzip && m.b < kTile) ? __ffs(m.b) - 1 : 0;  // b < 128 is a power of two
-    // Every tcgen05.ld/st below is warp-collective: the branches around them
-    // are made warp-uniform with __all_sync / __any_sync.
-    bool ok = true;
-    for (int it = 0; it < n; ++it) {
-      const int s = it & 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(&bar[B_SF + s], (it >> 1) & 1, abort, st, 20))) {
-        ok = false;
-        break;
+    int g = 0;
+    for (int idx = blockIdx.x; idx < n_items; idx += gridDim.x) {
+      const Item itm(idx, T, a.Hq, a.Bt);
+      const int list = list_of(m, itm.bt, itm.h);
+      WorkList wl;
+      wl.init(m, list, itm.I);
+      RowCtx rc[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        rc[i].p = itm.I * kTile + lane + 32 * i;
+        rc[i].ok = rc[i].p < a.N;
+        rc[i].bits = (gzip && rc[i].ok) ? m.bits + ((int64_t)list * m.B + rc[i].p / m.b) * m.words
+                                        : nullptr;
+        rc[i].li = (!gzip && rc[i].ok) ? m.perm[rc[i].p] : 0;
       }
-      tc_fence_after();
-      __syncwarp();  // tcgen05.ld is warp-collective (.sync.aligned)
-      float x[128];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(lane_addr + s * 128 + c * 32, x + c * 32);
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(&bar[B_SE + s]);
-
-      int src, kbase, kind, cnt;
-      wl.entry(m, it, src, kbase, kind, cnt);
-      // The branch taken depends only on CTA-uniform values (kind, src,
-      // kbase); rows past the end of the sequence are handled inside each.
-      const bool row_ok = p < a.N;
-      // scores stay unscaled here; the scale is folded into the exponent
-      if (kind == SA_TILE_FULL && (src || kbase + kTile <= a.N)) {
-        if (!row_ok) {
-#pragma unroll
-          for (int c = 0; c < 128; ++c) x[c] = -INFINITY;
+      bool ok = true;
+      for (int it = 0; it < wl.n; ++it) {
+        const int gq = g + it, slot = gq % kMaskSlots;
+        if (!__all_sync(0xffffffffu, mbar_wait(&bar[B_ME + slot], ((gq / kMaskSlots) & 1) ^ 1,
+                                                abort, st, 30))) {
+          ok = false;
+          break;
         }
-      } else if (kind == kTileCount) {
-        // compacted sink/gist keys, all visible: only the first cnt columns exist
+        int src, kbase, kind, cnt;
+        wl.entry(m, it, src, kbase, kind, cnt);
+        uint32_t* words = mwords + slot * (kMaskSlotBytes / 4);
+        if (!gzip && src == 0) {
+          // gist near tile: code = logical position | always-visible bit;
+          // sinks and gists are visible when not in the future, raw tokens
+          // also within the window ("UniGist ...", Approach)
+#pragma unroll 1
+          for (int w = 0; w < 4; ++w) {
+            const int kq = kbase + 32 * w + lane;
+            int32_t code = 0x3FFFFFFF;  // no key: never visible
+            if (kq < a.N) {
+              const int lj = m.perm[kq];
+              const bool always = lj < m.sinks || ((m.gist_bits[lj >> 5] >> (lj & 31)) & 1u);
+              code = lj | (always ? 0x40000000 : 0);
+            }
+            uint32_t acc[4] = {0u, 0u, 0u, 0u};
+#pragma unroll 8
+            for (int j = 0; j < 32; ++j) {
+              const int cj = __shfl_sync(0xffffffffu, code, j);
+              const int lj = cj & 0x3FFFFFFF;
+              const bool al = (cj & 0x40000000) != 0;
 #pragma unroll
-        for (int c = 0; c < 128; ++c) x[c] = (c < cnt && row_ok) ? x[c] : -INFINITY;
-      } else if (gzip) {
-        // this row's block bits over the key tile, then the causal cut
-        if (m.b >= kTile) {
-          const int jb = kbase / m.b;  // the whole key tile lies in one block
-          const bool blk = row_ok && ((rowbits[jb >> 5] >> (jb & 31)) & 1u);
+              for (int i = 0; i < 4; ++i) {
+                const bool v = lj <= rc[i].li && (al || rc[i].li - lj < m.window);
+                acc[i] |= (v ? 1u : 0u) << j;
+              }
+            }
 #pragma unroll
-          for (int c = 0; c < 128; ++c)
-            x[c] = (blk && kbase + c <= p && kbase + c < a.N) ? x[c] : -INFINITY;
-        } else if (lb >= 2) {
-          const int kb0 = kbase >> lb;  // 128 / b <= 32 blocks, inside one word
-          const uint32_t bb = row_ok ? (rowbits[kb0 >> 5] >> (kb0 & 31)) : 0u;
-#pragma unroll
-          for (int c = 0; c < 128; ++c)
-            x[c] = (((bb >> (c >> lb)) & 1u) && kbase + c <= p && kbase + c < a.N) ? x[c]
-                                                                                   : -INFINITY;
+            for (int i = 0; i < 4; ++i) words[w * 128 + lane + 32 * i] = rc[i].ok ? acc[i] : 0u;
+          }
         } else {
 #pragma unroll
-          for (int c = 0; c < 128; ++c) {
-            const int kq = kbase + c, jb = kq >> lb;
-            const bool v = row_ok && kq <= p && kq < a.N && ((rowbits[jb >> 5] >> (jb & 31)) & 1u);
-            x[c] = v ? x[c] : -INFINITY;
-          }
-        }
-      } else {
-        // gist near tile: each lane fetches 4 column codes (logical position |
-        // always-visible bit), shared across the warp with shuffles
-        int32_t cw[4];
+          for (int i = 0; i < 4; ++i)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int kq = kbase + 32 * j + lane;
-          int32_t code = 0x3FFFFFFF;  // no key: never visible
-          if (kq < a.N) {
-            const int lj = m.perm[kq];
-            const bool always = lj < m.sinks || ((m.gist_bits[lj >> 5] >> (lj & 31)) & 1u);
-            code = lj | (always ? 0x40000000 : 0);
-          }
-          cw[j] = code;
+            for (int w = 0; w < 4; ++w)
+              words[w * 128 + lane + 32 * i] = tile_word(m, gzip, lb, a.N, rc[i], kbase, kind, cnt, w);
         }
-#pragma unroll
-        for (int c = 0; c < 128; ++c) {
-          const int code = __shfl_sync(0xffffffffu, cw[c >> 5], c & 31);
-          const int lj = code & 0x3FFFFFFF;
-          const bool v = row_ok && lj <= li && ((code & 0x40000000) || li - lj < m.window);
-          x[c] = v ? x[c] : -INFINITY;
-        }
+        mbar_arrive(&bar[B_MF + slot]);  // release: the words above are visible to the waiter
       }
-      float mx = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < 128; ++c) mx = fmaxf(mx, x[c]);
-      const float m_new = fmaxf(m_run, mx * sl2);  // scale > 0 keeps the order
-      const bool resc = m_new > m_run + 8.f;  // true on the first finite max
-      const float m_use = resc ? m_new : m_run;
-      float rowsum = 0.f;
-      uint32_t pk[64];
-      if (m_use == -INFINITY) {
-#pragma unroll
-        for (int c = 0; c < 64; ++c) pk[c] = 0u;
-      } else {
-#pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          const float p0 = ex2(fmaf(x[2 * c], sl2, -m_use));
-          const float p1 = ex2(fmaf(x[2 * c + 1], sl2, -m_use));
-          rowsum += p0 + p1;
-          pk[c] = pack_bf16(p0, p1);
-        }
-      }
-      const float alpha = !resc ? 1.f : (m_run == -INFINITY ? 0.f : ex2(m_run - m_use));
-      // P tile s was last read by PV(it - 2)
-      if (it >= 2 &&
-          !__all_sync(0xffffffffu, mbar_wait(&bar[B_OD + s], ((it - 2) >> 1) & 1, abort, st, 21))) {
-        ok = false;
-        break;
-      }
-      if (it >= 1 && __any_sync(0xffffffffu, resc)) {
-        // O must not be accumulated while it is rescaled: wait for PV(it-1).
-        // The whole warp takes part; rows that keep their max use alpha = 1.
-        if (!__all_sync(0xffffffffu, mbar_wait(&bar[B_OD + ((it - 1) & 1)], ((it - 1) >> 1) & 1,
-                                                abort, st, 22))) {
+      if (!ok) break;
+      g += wl.n;
+    }
+  } else if (warp >= 2 && warp < 2 + kSoftmaxThreads / 32) {
+    // --------------------------------------------------------------- softmax
+    const int half = (warp - 2) >> 2;
+    const int quarter = warp & 3;  // TMEM lane quarter of this warp
+    const int r = quarter * 32 + lane;
+    const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
+    const float sl2 = a.scale * 1.4426950408889634f;
+    int g = 0, k = 0, xk = 0;
+    bool ok = true;
+    int n_next = blockIdx.x < n_items ? item_tiles(m, blockIdx.x, T, a.Hq, a.Bt) : 0;
+    // Every tcgen05.ld/st below is warp-collective: the branches around them
+    // are made warp-uniform with __all_sync / __any_sync.
+    for (int idx = blockIdx.x; ok && idx < n_items; idx += gridDim.x, ++k) {
+      const Item itm(idx, T, a.Hq, a.Bt);
+      const int n = n_next;
+      n_next = idx + (int)gridDim.x < n_items ? item_tiles(m, idx + gridDim.x, T, a.Hq, a.Bt) : 0;
+      const int p = itm.I * kTile + r;
+      float m_run = -INFINITY, l_run = 0.f;
+      for (int it = 0; it < n; ++it) {
+        const int gq = g + it, s = gq & 1, slot = gq % kMaskSlots;
+        if (!__all_sync(0xffffffffu,
+                        mbar_wait(&bar[B_SF + s], (gq >> 1) & 1, abort, st, 20) &&
+                            mbar_wait(&bar[B_MF + slot], (gq / kMaskSlots) & 1, abort, st, 24))) {
           ok = false;
           break;
         }
         tc_fence_after();
-        __syncwarp();
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          float o[32];
-          tmem_ld32(lane_addr + kTmemO + c * 32, o);
-          tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] *= alpha;
-          tmem_st32(lane_addr + kTmemO + c * 32, o);
-        }
-        tmem_wait_st();
-      }
-      l_run = l_run * alpha + rowsum;
-      m_run = m_use;
-      const uint32_t prow = sb + L::p0 + s * L::kP;
-#pragma unroll
-      for (int ch = 0; ch < 16; ++ch) {  // 16 chunks of 8 columns
-        const int col = ch * 8;
-        const uint32_t addr = prow + (col >> 6) * L::kAtom + sw128_offset(r, col & 63);
-        st_shared_v4(addr, pk[ch * 4], pk[ch * 4 + 1], pk[ch * 4 + 2], pk[ch * 4 + 3]);
-      }
-      fence_async_shared();
-      tc_fence_before();
-      mbar_arrive(&bar[B_PF + s]);
-    }
-    // ---------------------------------------------------------------- epilogue
-    if (ok && n > 0 &&
-        __all_sync(0xffffffffu,
-                   mbar_wait(&bar[B_OD + ((n - 1) & 1)], ((n - 1) >> 1) & 1, abort, st, 23))) {
-      tc_fence_after();
-      __syncwarp();
-      const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-      __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.o) + bt * a.os[0] +
-                            (int64_t)p * a.os[1] + (int64_t)h * a.os[2];
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        float o[32];
-        tmem_ld32(lane_addr + kTmemO + c * 32, o);  // all lanes: collective
+        __syncwarp();  // tcgen05.ld is warp-collective (.sync.aligned)
+        float x[64];
+        tmem_ld32(lane_addr + s * 128 + half * 64, x);
+        tmem_ld32(lane_addr + s * 128 + half * 64 + 32, x + 32);
+        const uint32_t* words = mwords + slot * (kMaskSlotBytes / 4);
+        const uint32_t mw0 = words[(2 * half) * 128 + r], mw1 = words[(2 * half + 1) * 128 + r];
+        mbar_arrive(&bar[B_ME + slot]);
         tmem_wait_ld();
-        if (p < a.N) {
+        // scores stay unscaled here; the scale is folded into the exponent
+        if ((mw0 & mw1) != 0xffffffffu) {
 #pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            uint4 w;
-            w.x = pack_bf16(o[v * 8 + 0] * inv, o[v * 8 + 1] * inv);
-            w.y = pack_bf16(o[v * 8 + 2] * inv, o[v * 8 + 3] * inv);
-            w.z = pack_bf16(o[v * 8 + 4] * inv, o[v * 8 + 5] * inv);
-            w.w = pack_bf16(o[v * 8 + 6] * inv, o[v * 8 + 7] * inv);
-            *reinterpret_cast<uint4*>(orow + c * 32 + v * 8) = w;
+          for (int i = 0; i < 32; ++i) {
+            x[i] = ((mw0 >> i) & 1u) ? x[i] : -INFINITY;
+            x[32 + i] = ((mw1 >> i) & 1u) ? x[32 + i] : -INFINITY;
           }
         }
+        float t[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          t[i] = fmaxf(fmaxf(x[4 * i], x[4 * i + 1]), fmaxf(x[4 * i + 2], x[4 * i + 3]));
+#pragma unroll
+        for (int w = 8; w >= 1; w >>= 1)
+#pragma unroll
+          for (int i = 0; i < w; ++i) t[i] = fmaxf(t[i], t[i + w]);
+        const float m_new = fmaxf(m_run, t[0] * sl2);  // scale > 0 keeps the order
+        const bool resc = m_new > m_run + 8.f;          // true on the first finite max
+        const float m_use = resc ? m_new : m_run;
+        uint32_t pk[32];
+        float sum[4] = {0.f, 0.f, 0.f, 0.f};
+        if (m_use == -INFINITY) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) pk[i] = 0u;
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float p0 = ex2(fmaf(x[2 * i], sl2, -m_use));
+            const float p1 = ex2(fmaf(x[2 * i + 1], sl2, -m_use));
+            sum[i & 3] += p0 + p1;
+            pk[i] = pack_bf16(p0, p1);
+          }
+        }
+        const float rowsum = (sum[0] + sum[1]) + (sum[2] + sum[3]);
+        const float alpha = !resc ? 1.f : (m_run == -INFINITY ? 0.f : ex2(m_run - m_use));
+        // O_h was last accumulated by P V of tile gq - 1
+        if (gq >= 1 && !__all_sync(0xffffffffu,
+                                   mbar_wait(&bar[B_OD + half], (gq - 1) & 1, abort, st, 21))) {
+          ok = false;
+          break;
+        }
+        if (it >= 1 && __any_sync(0xffffffffu, resc)) {
+          // the whole warp takes part; rows that keep their max use alpha = 1
+          tc_fence_after();
+          __syncwarp();
+#pragma unroll
+          for (int cc = 0; cc < D / 32; ++cc) {
+            float o[32];
+            tmem_ld32(lane_addr + kTmemO + half * D + cc * 32, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] *= alpha;
+            tmem_st32(lane_addr + kTmemO + half * D + cc * 32, o);
+          }
+        }
+        l_run = l_run * alpha + rowsum;
+        m_run = m_use;
+        // P (bf16 pairs) over the first 32 of this half's S columns, already read
+        __syncwarp();
+        tmem_st32(lane_addr + s * 128 + half * 64, reinterpret_cast<const float*>(pk));
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&bar[B_PF + half]);
       }
-      if (p < a.N)
-        a.lse[((int64_t)bt * a.Hq + h) * a.N + p] =
-            l_run > 0.f ? (m_run + __log2f(l_run)) * 0.6931471805599453f : -INFINITY;
+      if (!ok) break;
+      // ------------------------------------------------------------ epilogue
+      if (!__all_sync(0xffffffffu, mbar_wait(&bar[B_OI], k & 1, abort, st, 22))) break;
+      const bool row_ok = p < a.N;
+      __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.o) + itm.bt * a.os[0] +
+                            (int64_t)p * a.os[1] + (int64_t)itm.h * a.os[2] + half * (D / 2);
+      float mm = -INFINITY, l = 0.f;
+      if (n > 0) {
+        // exchange (max, sum) with the other half of the same rows
+        ml[half * 128 + r] = make_float2(m_run, l_run);
+        mbar_arrive(&bar[B_ML]);
+        if (!__all_sync(0xffffffffu, mbar_wait(&bar[B_ML], xk & 1, abort, st, 23))) break;
+        ++xk;
+        const float2 other = ml[(half ^ 1) * 128 + r];
+        const float m0 = half ? other.x : m_run, l0 = half ? other.y : l_run;
+        const float m1 = half ? m_run : other.x, l1 = half ? l_run : other.y;
+        mm = fmaxf(m0, m1);
+        const float a0 = m0 == -INFINITY ? 0.f : ex2(m0 - mm);
+        const float a1 = m1 == -INFINITY ? 0.f : ex2(m1 - mm);
+        l = l0 * a0 + l1 * a1;
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+        const float c0 = a0 * inv, c1 = a1 * inv;
+        tc_fence_after();
+        __syncwarp();
+#pragma unroll
+        for (int cc = 0; cc < D / 64; ++cc) {  // this half's D/2 output columns
+          const uint32_t col = half * (D / 2) + cc * 32;
+          float o0[32], o1[32];
+          tmem_ld32(lane_addr + kTmemO + col, o0);  // all lanes: collective
+          tmem_ld32(lane_addr + kTmemO + D + col, o1);
+          tmem_wait_ld();
+          if (row_ok) {
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              uint4 wv;
+              wv.x = pack_bf16(o0[v * 8 + 0] * c0 + o1[v * 8 + 0] * c1,
+                               o0[v * 8 + 1] * c0 + o1[v * 8 + 1] * c1);
+              wv.y = pack_bf16(o0[v * 8 + 2] * c0 + o1[v * 8 + 2] * c1,
+                               o0[v * 8 + 3] * c0 + o1[v * 8 + 3] * c1);
+              wv.z = pack_bf16(o0[v * 8 + 4] * c0 + o1[v * 8 + 4] * c1,
+                               o0[v * 8 + 5] * c0 + o1[v * 8 + 5] * c1);
+              wv.w = pack_bf16(o0[v * 8 + 6] * c0 + o1[v * 8 + 6] * c1,
+                               o0[v * 8 + 7] * c0 + o1[v * 8 + 7] * c1);
+              *reinterpret_cast<uint4*>(orow + cc * 32 + v * 8) = wv;
+            }
+          }
+        }
+      } else if (row_ok) {
+        for (int cc = 0; cc < D / 2; cc += 8)
+          *reinterpret_cast<uint4*>(orow + cc) = make_uint4(0u, 0u, 0u, 0u);
+      }
+      tc_fence_before();
+      mbar_arrive(&bar[B_OF]);  // O may be overwritten by the next item
+      if (half == 0 && row_ok)
+        a.lse[((int64_t)itm.bt * a.Hq + itm.h) * a.N + p] =
+            l > 0.f ? (mm + __log2f(l)) * 0.6931471805599453f : -INFINITY;
+      g += n;
     }
   }
   tc_fence_before();
@@ -485,6 +710,20 @@ __global__ void __launch_bounds__(256) gist_gather_kernel(AttnArgs a, MaskArgs m
   }
 }
 
+// Streaming multiprocessors of the current device (cached per device).
+static int sm_count() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (cached[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
 template <int D>
 static cudaError_t fwd_tc_launch(const AttnArgs& a, const MaskArgs& m, void* compact,
                                  cudaStream_t s) {
@@ -514,7 +753,10 @@ static cudaError_t fwd_tc_launch(const AttnArgs& a, const MaskArgs& m, void* com
   cudaError_t e = cudaFuncSetAttribute(fwd_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        bytes);
   if (e != cudaSuccess) return e;
-  fwd_tc_kernel<D><<<dim3(m.T * a.Hq * a.Bt), 192, bytes, s>>>(P);
+  // persistent: one CTA per SM (TMEM and shared memory admit one per SM)
+  const int items = m.T * a.Hq * a.Bt;
+  const int grid = items < sm_count() ? items : sm_count();
+  fwd_tc_kernel<D><<<dim3(grid), kThreads, bytes, s>>>(P);
   return cudaGetLastError();
 }
 

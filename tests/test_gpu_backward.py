@@ -70,8 +70,12 @@ def test_backward_full_size(sa):
     rng = np.random.default_rng(0)
     for bt in range(w["batch"]):
         masks = G.block_masks(fo[bt], w["window"])
-        # identities over all keys of every head (any size)
-        np.testing.assert_allclose(dk[bt].sum(0), 0, atol=0.5)
+        # identity over all keys of every head (any size): sum_j dV_j = sum_i dO_i,
+        # since every row of P sums to one. (The companion identity sum_j dK_j = 0
+        # is not checked here: it holds only up to the bf16 rounding of O inside
+        # Delta = rowsum(dO * O) and of dS, which over 65536 rows grows to the
+        # size of any fixed bound; the sampled rows and columns below are compared
+        # with the oracle instead.)
         np.testing.assert_allclose(dv[bt].sum(0), do[bt].astype(np.float64).sum(0), rtol=1e-3, atol=0.5)
         for h in (0, w["heads"] // 2, w["heads"] - 1):
             bm = masks[cls[h]]
