@@ -52,7 +52,15 @@ struct FwdTcParams {
   CUtensorMap tmkc, tmvc;  // gist mode: sinks + gists compacted in logical order
   AttnArgs a;
   MaskArgs m;
+  // gist mode: element masks of (query tile I, near key tile J), [T][near_nt][4][128]
+  // words, pair index I * near_nt + (J - I + near_nt - 1)
+  const uint32_t* near;
+  int near_nt;
 };
+
+// Near key tiles of a query tile in gist mode: Jlo..I with
+// Jlo = I - ceil((window - 1) / 128).
+int fwd_tc_near_tiles(int window) { return (window - 1 + kTile - 1) / kTile + 1; }
 
 // Internal tile kind: only the first `cnt` columns hold keys (the last tile of
 // the compacted sink/gist keys).
@@ -116,6 +124,7 @@ struct Item {
 
 constexpr int kMaskSlots = 4;              // mask ring depth (tiles)
 constexpr uint32_t kMaskSlotBytes = 2048;  // [4 words][128 rows] uint32
+constexpr int kRowCacheWords = 1024;       // gzip: the item's block-row bits
 
 template <int D>
 struct FwdLayout {
@@ -128,7 +137,8 @@ struct FwdLayout {
   static constexpr uint32_t k0 = kQ;
   static constexpr uint32_t v0 = k0 + kKStages * kKV;
   static constexpr uint32_t mask = v0 + kVStages * kKV;
-  static constexpr uint32_t ml = mask + kMaskSlots * kMaskSlotBytes;  // [2 halves][128] (max, sum)
+  static constexpr uint32_t rows = mask + kMaskSlots * kMaskSlotBytes;
+  static constexpr uint32_t ml = rows + kRowCacheWords * 4;  // [2 halves][128] (max, sum)
   static constexpr uint32_t bars = ml + 2 * 128 * 8;
   static constexpr uint32_t bytes = bars + 512 + 1024;  // + alignment slack
 };
@@ -150,9 +160,10 @@ constexpr int kSoftmaxThreads = 256;
 constexpr int kThreads = 64 + kSoftmaxThreads + 32;
 constexpr int kMaskWarp = 10;
 
-// Bits [0, n) set, n clamped to [0, 32].
+// Bits [0, n) set, n clamped to [0, 32] (no branch).
 __device__ __forceinline__ uint32_t prefix_bits(int n) {
-  return n <= 0 ? 0u : (n >= 32 ? 0xffffffffu : ((1u << n) - 1u));
+  const int c = min(max(n, 0), 32);
+  return (uint32_t)((1ull << c) - 1ull);
 }
 
 // Each set bit of e (nb bits) widened to a run of 2^lb bits (lb <= 4).
@@ -198,6 +209,54 @@ __device__ __forceinline__ uint32_t tile_word(const MaskArgs& m, int gzip, int l
   const int kb = cw0 >> lb, nb = 32 >> lb;  // nb blocks inside one bit word
   const uint32_t e = (rc.bits[kb >> 5] >> (kb & 31)) & prefix_bits(nb);
   return widen_bits(e, lb, nb) & causal;
+}
+
+// Gzip tiles: words w = 0..3 of rows i = 0..3 of one lane (rows lane + 32 i),
+// out[w * 128 + lane + 32 i]. Same rule as tile_word, arranged so that every
+// bit-word load is issued before any of them is used: rc[i].bits always
+// points at valid words (rows past N read some row and are cleared by lim).
+__device__ __forceinline__ void gzip_tile_words(const MaskArgs& m, int lb, int N, const RowCtx* rc,
+                                                int kbase, int kind, int lane, uint32_t* out) {
+  if (kind == SA_TILE_FULL && kbase + kTile <= N) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int w = 0; w < 4; ++w) out[w * 128 + lane + 32 * i] = rc[i].ok ? 0xffffffffu : 0u;
+    return;
+  }
+  int lim[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) lim[i] = rc[i].ok ? min(rc[i].p, N - 1) : -1;
+  if (m.b >= kTile || lb >= 5) {
+    // one block bit per (row, word): the whole tile (b >= 128) or 32 columns
+    uint32_t u[4][4];
+    int jb[4];
+#pragma unroll
+    for (int w = 0; w < 4; ++w)  // clamped: columns past N are cleared by lim anyway
+      jb[w] = min(m.B - 1, m.b >= kTile ? kbase / m.b : (kbase + 32 * w) >> lb);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int w = 0; w < 4; ++w) u[i][w] = rc[i].bits[jb[w] >> 5];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        const uint32_t causal = prefix_bits(lim[i] - (kbase + 32 * w) + 1);
+        out[w * 128 + lane + 32 * i] = ((u[i][w] >> (jb[w] & 31)) & 1u) ? causal : 0u;
+      }
+    return;
+  }
+  // b < 32: 32 >> lb blocks per word, inside one bit word
+  const int nb = 32 >> lb;
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const int cw0 = kbase + 32 * w, kb = min(cw0 >> lb, m.B - 1);  // clamped as above
+      const uint32_t e = (rc[i].bits[kb >> 5] >> (kb & 31)) & prefix_bits(nb);
+      out[w * 128 + lane + 32 * i] = widen_bits(e, lb, nb) & prefix_bits(lim[i] - cw0 + 1);
+    }
 }
 
 // Number of visited tiles of item idx.
@@ -417,23 +476,44 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_kernel(const __grid_consta
     // word w of row r at mwords[slot][w][r].
     const int gzip = m.kind == SA_MASK_GZIP;
     const int lb = (gzip && m.b < kTile) ? __ffs(m.b) - 1 : 0;  // b < 128 is a power of two
+    uint32_t* rcache = reinterpret_cast<uint32_t*>(smem + L::rows);
     int g = 0;
     for (int idx = blockIdx.x; idx < n_items; idx += gridDim.x) {
       const Item itm(idx, T, a.Hq, a.Bt);
       const int list = list_of(m, itm.bt, itm.h);
       WorkList wl;
       wl.init(m, list, itm.I);
+      // gzip: the block rows of this query tile, copied once per item when they fit
+      const int rb0 = itm.I * kTile / (gzip ? m.b : 1);
+      const int rb1 = gzip ? min(m.B - 1, (itm.I * kTile + kTile - 1) / m.b) : rb0;
+      const bool cached = gzip && (rb1 - rb0 + 1) * m.words <= kRowCacheWords;
+      __syncwarp();  // the previous item's lookups are done
+      if (cached) {
+        const uint32_t* src = m.bits + ((int64_t)list * m.B + rb0) * m.words;
+        for (int x = lane; x < (rb1 - rb0 + 1) * m.words; x += 32) rcache[x] = src[x];
+      }
+      __syncwarp();
       RowCtx rc[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         rc[i].p = itm.I * kTile + lane + 32 * i;
         rc[i].ok = rc[i].p < a.N;
-        rc[i].bits = (gzip && rc[i].ok) ? m.bits + ((int64_t)list * m.B + rc[i].p / m.b) * m.words
-                                        : nullptr;
-        rc[i].li = (!gzip && rc[i].ok) ? m.perm[rc[i].p] : 0;
+        rc[i].bits = nullptr;
+        if (gzip) {  // rows past N point at the first row of the tile (cleared later)
+          const int rb = rc[i].ok ? rc[i].p / m.b : rb0;
+          rc[i].bits = cached ? rcache + (rb - rb0) * m.words
+                              : m.bits + ((int64_t)list * m.B + rb) * m.words;
+        }
+        rc[i].li = 0;
       }
       bool ok = true;
+      int col_reg = 0, kind_reg = 0;  // gzip: tile list entries it0 + lane
       for (int it = 0; it < wl.n; ++it) {
+        if (gzip && (it & 31) == 0) {
+          const int e = it + lane;
+          col_reg = e < wl.n ? m.tcol[wl.e0 + e] : 0;
+          kind_reg = e < wl.n ? m.tkind[wl.e0 + e] : 0;
+        }
         const int gq = g + it, slot = gq % kMaskSlots;
         if (!__all_sync(0xffffffffu, mbar_wait(&bar[B_ME + slot], ((gq / kMaskSlots) & 1) ^ 1,
                                                 abort, st, 30))) {
@@ -441,36 +521,27 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_kernel(const __grid_consta
           break;
         }
         int src, kbase, kind, cnt;
-        wl.entry(m, it, src, kbase, kind, cnt);
+        if (gzip) {
+          src = 0;
+          cnt = kTile;
+          kbase = __shfl_sync(0xffffffffu, col_reg, it & 31) * kTile;
+          kind = __shfl_sync(0xffffffffu, kind_reg, it & 31) == SA_TILE_FULL ? SA_TILE_FULL
+                                                                              : SA_TILE_MASKED;
+        } else {
+          wl.entry(m, it, src, kbase, kind, cnt);
+        }
         uint32_t* words = mwords + slot * (kMaskSlotBytes / 4);
         if (!gzip && src == 0) {
-          // gist near tile: code = logical position | always-visible bit;
-          // sinks and gists are visible when not in the future, raw tokens
-          // also within the window ("UniGist ...", Approach)
-#pragma unroll 1
-          for (int w = 0; w < 4; ++w) {
-            const int kq = kbase + 32 * w + lane;
-            int32_t code = 0x3FFFFFFF;  // no key: never visible
-            if (kq < a.N) {
-              const int lj = m.perm[kq];
-              const bool always = lj < m.sinks || ((m.gist_bits[lj >> 5] >> (lj & 31)) & 1u);
-              code = lj | (always ? 0x40000000 : 0);
-            }
-            uint32_t acc[4] = {0u, 0u, 0u, 0u};
-#pragma unroll 8
-            for (int j = 0; j < 32; ++j) {
-              const int cj = __shfl_sync(0xffffffffu, code, j);
-              const int lj = cj & 0x3FFFFFFF;
-              const bool al = (cj & 0x40000000) != 0;
+          // gist near tile: the element rule was evaluated once for every head
+          const uint4* from = reinterpret_cast<const uint4*>(
+              P.near + ((int64_t)itm.I * P.near_nt + (kbase / kTile - itm.I + P.near_nt - 1)) * 512);
+          uint4 v[4];
 #pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                const bool v = lj <= rc[i].li && (al || rc[i].li - lj < m.window);
-                acc[i] |= (v ? 1u : 0u) << j;
-              }
-            }
+          for (int q4 = 0; q4 < 4; ++q4) v[q4] = from[lane + 32 * q4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) words[w * 128 + lane + 32 * i] = rc[i].ok ? acc[i] : 0u;
-          }
+          for (int q4 = 0; q4 < 4; ++q4) reinterpret_cast<uint4*>(words)[lane + 32 * q4] = v[q4];
+        } else if (gzip) {
+          gzip_tile_words(m, lb, a.N, rc, kbase, kind, lane, words);
         } else {
 #pragma unroll
           for (int i = 0; i < 4; ++i)
@@ -724,9 +795,47 @@ static int sm_count() {
   return cached[dev];
 }
 
+// Gist mode: the element masks of every (query tile I, near key tile J) pair,
+// the same for every head ("UniGist ...", Approach: a query sees the sinks and
+// the gists that are not in its future, and the raw tokens of its window).
+// Block (I, J - I + nt - 1), thread r = query row; bit c of word w tells
+// whether key 128 J + 32 w + c is visible from row 128 I + r. With d = li - lj
+// (logical positions) the rule is (unsigned)d < lim, lim = 2^31 for sinks and
+// gists (d >= 0) and the window for raw tokens (0 <= d < window).
+__global__ void __launch_bounds__(128) gist_near_mask_kernel(MaskArgs m, int N, int nt_count,
+                                                             uint32_t* near) {
+  const int I = blockIdx.x, nt = blockIdx.y, r = threadIdx.x;
+  const int J = I - (nt_count - 1) + nt;
+  if (J < 0) return;  // not a key tile of this query tile
+  __shared__ int lj_s[kTile];
+  __shared__ uint32_t lim_s[kTile];
+  const int kq = J * kTile + r;
+  int lj = 0;
+  uint32_t lim = 0u;  // no key: never visible
+  if (kq < N) {
+    lj = m.perm[kq];
+    const bool always = lj < m.sinks || ((m.gist_bits[lj >> 5] >> (lj & 31)) & 1u);
+    lim = always ? 0x80000000u : (uint32_t)m.window;
+  }
+  lj_s[r] = lj;
+  lim_s[r] = lim;
+  __syncthreads();
+  const int p = I * kTile + r;
+  const int li = p < N ? m.perm[p] : 0;
+  uint32_t* out = near + ((int64_t)I * nt_count + nt) * 512;
+#pragma unroll 1
+  for (int w = 0; w < 4; ++w) {
+    uint32_t word = 0u;
+#pragma unroll 8
+    for (int j = 0; j < 32; ++j)
+      word |= ((uint32_t)(li - lj_s[32 * w + j]) < lim_s[32 * w + j] ? 1u : 0u) << j;
+    out[w * 128 + r] = p < N ? word : 0u;
+  }
+}
+
 template <int D>
 static cudaError_t fwd_tc_launch(const AttnArgs& a, const MaskArgs& m, void* compact,
-                                 cudaStream_t s) {
+                                 void* near, cudaStream_t s) {
   FwdTcParams P;
   memset(&P, 0, sizeof(P));
   if (!make_tile_map(&P.tmq, a.q, D, a.Hq, a.N, a.Bt, a.qs) ||
@@ -746,6 +855,12 @@ static cudaError_t fwd_tc_launch(const AttnArgs& a, const MaskArgs& m, void* com
     gist_gather_kernel<D><<<dim3((a.N + 7) / 8, a.Bt), 256, 0, s>>>(a, m, kc, vc);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
+    P.near = static_cast<const uint32_t*>(near);
+    P.near_nt = fwd_tc_near_tiles(m.window);
+    gist_near_mask_kernel<<<dim3(m.T, P.near_nt), kTile, 0, s>>>(m, a.N, P.near_nt,
+                                                               static_cast<uint32_t*>(near));
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
   }
   P.a = a;
   P.m = m;
@@ -760,11 +875,12 @@ static cudaError_t fwd_tc_launch(const AttnArgs& a, const MaskArgs& m, void* com
   return cudaGetLastError();
 }
 
-// `compact`: gist mode only, 2 * Bt * N * Hkv * d bf16 of workspace.
-cudaError_t launch_fwd_tc(int d, const AttnArgs& a, const MaskArgs& m, void* compact,
+// Gist mode only: `compact`, 2 * Bt * N * Hkv * d bf16 of workspace; `near`,
+// T * fwd_tc_near_tiles(window) * 2048 bytes.
+cudaError_t launch_fwd_tc(int d, const AttnArgs& a, const MaskArgs& m, void* compact, void* near,
                           cudaStream_t s) {
-  if (d == 64) return fwd_tc_launch<64>(a, m, compact, s);
-  if (d == 128) return fwd_tc_launch<128>(a, m, compact, s);
+  if (d == 64) return fwd_tc_launch<64>(a, m, compact, near, s);
+  if (d == 128) return fwd_tc_launch<128>(a, m, compact, near, s);
   return cudaErrorInvalidValue;
 }
 

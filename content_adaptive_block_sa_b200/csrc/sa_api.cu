@@ -13,7 +13,9 @@ cudaError_t launch_gist_build(const sa_mask_desc&, const uint8_t*, const sa_bloc
                               cudaStream_t);
 cudaError_t launch_fwd_simt(int dtype, int d, const AttnArgs&, const MaskArgs&, cudaStream_t);
 cudaError_t launch_bwd_simt(int dtype, int d, const AttnArgs&, const MaskArgs&, cudaStream_t);
-cudaError_t launch_fwd_tc(int d, const AttnArgs&, const MaskArgs&, void* compact, cudaStream_t);
+cudaError_t launch_fwd_tc(int d, const AttnArgs&, const MaskArgs&, void* compact, void* near,
+                          cudaStream_t);
+int fwd_tc_near_tiles(int window);
 cudaError_t launch_bwd_tc(int d, const AttnArgs&, const MaskArgs&, void* ws, cudaStream_t);
 size_t bwd_tc_workspace(int Bt, int Hq, int T);
 cudaError_t launch_decode(const sa_decode_desc&, const void*, const void*, const void*,
@@ -284,9 +286,13 @@ sa_status sa_forward_workspace_size(const sa_attn_desc* attn, const sa_mask_desc
   if (st != SA_OK) return st;
   SA_CHECK(bytes != nullptr, SA_ERR_INVALID_ARG);
   *bytes = kStatusBytes;
-  if (mask->kind == SA_MASK_GIST)  // compacted sink/gist K and V (tensor-core path)
+  if (mask->kind == SA_MASK_GIST) {
+    // tensor-core path: compacted sink/gist K and V, then the element masks of
+    // every (query tile, near key tile) pair, 128 x 128 bits each
     *bytes += 2 * round256((size_t)attn->batch * attn->seq_len * attn->num_kv_heads *
                            attn->head_dim * 2);
+    *bytes += round256((size_t)tiles_of(attn->seq_len) * fwd_tc_near_tiles(mask->window) * 2048);
+  }
   return SA_OK;
 }
 
@@ -315,8 +321,12 @@ sa_status sa_forward(const sa_attn_desc* attn, const sa_mask_desc* mask, const v
   st = clear_status(ws, stream);
   if (st != SA_OK) return st;
   const MaskArgs m = make_mask_args(*mask, *lists);
-  if (impl == SA_IMPL_TENSOR_CORES)
-    return cuda_status(launch_fwd_tc(attn->head_dim, a, m, (char*)ws + kStatusBytes, stream));
+  if (impl == SA_IMPL_TENSOR_CORES) {
+    char* compact = (char*)ws + kStatusBytes;
+    char* near = compact + 2 * round256((size_t)attn->batch * attn->seq_len *
+                                        attn->num_kv_heads * attn->head_dim * 2);
+    return cuda_status(launch_fwd_tc(attn->head_dim, a, m, compact, near, stream));
+  }
   return cuda_status(launch_fwd_simt(attn->dtype, attn->head_dim, a, m, stream));
 }
 
