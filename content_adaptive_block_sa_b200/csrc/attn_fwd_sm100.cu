@@ -737,20 +737,26 @@ static EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// [Bt, N, H, d] bf16 with element strides {batch, seq, head}; box 64 x 1 x 128 x 1.
-bool make_tile_map(CUtensorMap* map, const void* base, int d, int H, int N, int Bt,
-                     const int64_t* s) {
+// [Bt, N, H, d] bf16 with element strides {batch, seq, head}; box 64 x 1 x rows x 1,
+// 128-byte swizzle.
+bool make_tile_map_box(CUtensorMap* map, const void* base, int d, int H, int N, int Bt,
+                       const int64_t* s, int rows) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   const int64_t sh = s[2] > 0 ? s[2] : d, sn = s[1];
   const int64_t sbat = (Bt > 1) ? s[0] : sn * N;
   cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)N, (cuuint64_t)Bt};
   cuuint64_t strides[3] = {(cuuint64_t)(sh * 2), (cuuint64_t)(sn * 2), (cuuint64_t)(sbat * 2)};
-  cuuint32_t box[4] = {64, 1, 128, 1};
+  cuuint32_t box[4] = {64, 1, (cuuint32_t)rows, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_tile_map(CUtensorMap* map, const void* base, int d, int H, int N, int Bt,
+                   const int64_t* s) {
+  return make_tile_map_box(map, base, d, H, N, Bt, s, kTile);
 }
 
 // Gist mode: copies the K and V rows of every sink / gist (far_idx, logical

@@ -321,9 +321,18 @@ static cudaError_t decode_launch_rep(const DecodeArgs& a, const DecodePlan& pl, 
   return cudaGetLastError();
 }
 
+bool decode_tc_supported(const sa_decode_desc& d);
+cudaError_t launch_decode_tc(const sa_decode_desc& d, const void* q, const void* gk,
+                             const void* gv, const void* kc, const void* vc, int32_t* sel, void* o,
+                             float* lse, void* ws, cudaStream_t s);
+
+// The tensor-core kernel (one CTA per sequence and KV head) takes the shapes it
+// supports; the four-pass CUDA-core kernels below take the rest.
 cudaError_t launch_decode(const sa_decode_desc& d, const void* q, const void* gk, const void* gv,
                           const void* kc, const void* vc, int32_t* sel, void* o, float* lse,
                           void* ws, cudaStream_t s) {
+  if (decode_tc_supported(d))
+    return launch_decode_tc(d, q, gk, gv, kc, vc, sel, o, lse, ws, s);
   const DecodePlan pl = decode_plan(d);
   DecodeArgs a{};
   a.q = (const __nv_bfloat16*)q;

@@ -1,0 +1,594 @@
+// Gist-scored selective unfolding at decode, one CTA per (sequence, KV head),
+// on the 5th-generation tensor cores.
+//
+// "Simplified Sparse Attention via Gist Tokens" (abstract) and "Forget, Then
+// Recall: ... Gist Sparse Attention" (abstract): the new query is scored
+// against the gist keys, the top-k chunks are unfolded into their raw tokens,
+// and attention runs over the gists, the unfolded chunks and the recent
+// window. Everything of one (sequence, KV head g) happens in one CTA, in one
+// online softmax over 128-key blocks:
+//   1. gist blocks: S^T = K_blk Q_g^T (keys on TMEM lanes, the group's query
+//      heads on columns); the selection score of gist j, sum_h s_hj, goes to
+//      shared memory; O^T += V_blk^T P with the same logits.
+//   2. window blocks: the last `window` positions of the raw cache (these are
+//      loaded while step 3 runs).
+//   3. top-k selection over the eligible chunks (wholly before the window) by
+//      a 4-pass radix select on the order-preserving 32-bit key of the score,
+//      ties to the lower chunk index, written ascending (-1 padded).
+//   4. chunk blocks: 128 / chunk selected chunks per block, each brought in
+//      by its own TMA box.
+// The output O = O^T / l and LSE follow from the single softmax state; no
+// partial results leave the CTA.
+//
+// Roles (192 threads): warp 0 issues the TMA loads (K and V blocks into a
+// 2-stage ring) and owns the TMEM allocation; one thread of warp 1 issues
+// tcgen05.mma (S^T = K Q^T, M = 128 keys, N = 16 head columns; O^T += V^T P,
+// M = 128 dims, N = 16) with completion on mbarriers; warps 2-5 (thread = key
+// row of the block for the softmax, = output dimension for O^T) run the
+// softmax, the selection and the epilogue. The block maximum per head is
+// exchanged between the four softmax warps through shared memory; O^T is
+// rescaled only when a head's maximum grew by more than 2^8. Every wait is
+// bounded; on timeout the device status word is set and all roles leave
+// after draining their copies and MMAs.
+#include <cuda.h>
+
+#include "sa_common.cuh"
+#include "sm100.cuh"
+
+namespace sa {
+
+using namespace sm100;
+
+bool make_tile_map_box(CUtensorMap* map, const void* base, int d, int H, int N, int Bt,
+                       const int64_t* s, int rows);
+
+namespace dec {
+
+constexpr int kD = 128;        // head dim
+constexpr int kBlk = 128;      // keys per block
+constexpr int kN = 16;         // MMA N: query-head columns (rep <= 8 used)
+constexpr int kMaxG = 8192;    // gists held in shared memory for the selection
+constexpr int kMaxTopK = 256;
+constexpr int kThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2-5 softmax
+
+struct Params {
+  CUtensorMap gk, gv;    // gists, box 128 rows
+  CUtensorMap ck, cv;    // raw cache, box 128 rows (window)
+  CUtensorMap ckc, cvc;  // raw cache, box `chunk` rows (unfolded chunks)
+  const __nv_bfloat16* q;
+  __nv_bfloat16* o;
+  float* lse;
+  int32_t* sel;
+  DeviceStatus* status;
+  int n_seq, Hkv, rep, G, cache_len, chunk, top_k, window;
+  int nG, nW, nC;        // gist, window and chunk blocks
+  float scale;
+  int64_t qs[2], os[2];
+};
+
+// Shared memory (offsets from a 1024-aligned base).
+constexpr uint32_t kAtom = kBlk * 128;          // [128 rows][64 bf16]
+constexpr uint32_t kTileBytes = 2 * kAtom;      // one K or V block, 2 atoms
+constexpr uint32_t kStage = 2 * kTileBytes;     // K + V
+constexpr uint32_t kQtAtom = kN * 128;          // [16 rows][64 bf16]
+constexpr uint32_t OFF_KV = 0;                  // 2 stages
+constexpr uint32_t OFF_QT = 2 * kStage;         // Q^T [16][128], 2 atoms
+constexpr uint32_t OFF_PT = OFF_QT + 2 * kQtAtom;  // P^T [2 buffers][16][128], 2 atoms each
+constexpr uint32_t OFF_SCORE = OFF_PT + 2 * 2 * kQtAtom;  // float [kMaxG]
+constexpr uint32_t OFF_HIST = OFF_SCORE + kMaxG * 4;     // uint32 [256]
+constexpr uint32_t OFF_SEL = OFF_HIST + 256 * 4;         // int32 [kMaxTopK]
+constexpr uint32_t OFF_RED = OFF_SEL + kMaxTopK * 4;     // float [2][4 warps][kN]
+constexpr uint32_t OFF_SCAN = OFF_RED + 2 * 4 * kN * 4;  // uint32 [8] + misc
+constexpr uint32_t OFF_BARS = OFF_SCAN + 64;
+constexpr uint32_t kSmemBytes = OFF_BARS + 256 + 1024;
+
+enum {
+  B_KVF = 0, B_KVE = 2, B_SF = 4, B_SE = 6, B_PF = 8, B_PD = 10, B_MX = 11, B_GS = 12,
+  B_QR = 13, B_SELD = 14, B_DRAIN = 15, kNumBars = 16
+};
+
+constexpr uint32_t kTmemCols = 64;  // S^T buffers at 0 and 16, O^T at 32
+constexpr uint32_t kTmemO = 32;
+
+// Order-preserving map of a float to an unsigned key (0 is below every float).
+__device__ __forceinline__ uint32_t float_key(float f) {
+  const uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Arrive-and-wait of the 128 softmax threads on one mbarrier (bounded).
+struct GroupSync {
+  uint64_t* bar;
+  uint32_t phase;
+  volatile int* abort;
+  DeviceStatus* st;
+  __device__ bool operator()(int where) {
+    mbar_arrive(bar);
+    const bool ok = mbar_wait(bar, phase & 1u, abort, st, where);
+    ++phase;
+    return ok;
+  }
+};
+
+// Block-wide exclusive prefix sum over the 128 softmax threads (t = 0..127);
+// returns the exclusive prefix, *total the sum.
+__device__ __forceinline__ uint32_t group_exclusive_scan(uint32_t v, int t, uint32_t* buf,
+                                                         GroupSync& gs, bool& ok,
+                                                         uint32_t* total) {
+  const int lane = t & 31, w = t >> 5;
+  uint32_t x = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, x, off);
+    if (lane >= off) x += y;
+  }
+  if (lane == 31) buf[w] = x;
+  ok = ok && gs(40);
+  uint32_t before = 0, sum = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t tw = buf[i];
+    if (i < w) before += tw;
+    sum += tw;
+  }
+  ok = ok && gs(41);  // buf may be reused after this
+  *total = sum;
+  return before + x - v;
+}
+
+}  // namespace dec
+
+using namespace dec;
+
+template <int REP>
+__global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_constant__ Params P) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  const uint32_t sb = smem_u32(smem);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + OFF_BARS);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + kNumBars);
+  volatile int* abort = reinterpret_cast<volatile int*>(bar + kNumBars) + 1;
+  int32_t* sel_s = reinterpret_cast<int32_t*>(smem + OFF_SEL);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = blockIdx.x % P.Hkv, seq = blockIdx.x / P.Hkv;
+  const int nb = P.nG + P.nW + P.nC;
+  DeviceStatus* st = P.status;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bar[B_KVF + s], 1);
+      mbar_init(&bar[B_KVE + s], 1);
+      mbar_init(&bar[B_SF + s], 1);
+      mbar_init(&bar[B_SE + s], 128);
+      mbar_init(&bar[B_PF + s], 128);
+    }
+    mbar_init(&bar[B_PD], 1);
+    mbar_init(&bar[B_MX], 128);
+    mbar_init(&bar[B_GS], 128);
+    mbar_init(&bar[B_QR], 128);
+    mbar_init(&bar[B_SELD], 128);
+    mbar_init(&bar[B_DRAIN], 1);
+    *abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------ TMA producer
+      prefetch_tmap(&P.gk);
+      prefetch_tmap(&P.gv);
+      prefetch_tmap(&P.ck);
+      prefetch_tmap(&P.cv);
+      prefetch_tmap(&P.ckc);
+      prefetch_tmap(&P.cvc);
+      const int ws = P.cache_len - P.window;
+      const int cpb = kBlk / P.chunk;  // chunks per block
+      int last = -1;
+      for (int b = 0; b < nb; ++b) {
+        const int s = b & 1;
+        if (!mbar_wait(&bar[B_KVE + s], ((b >> 1) & 1) ^ 1, abort, st, 1)) break;
+        // the chunks are known once the selection is done
+        if (b == P.nG + P.nW && !mbar_wait(&bar[B_SELD], 0, abort, st, 2)) break;
+        uint8_t* kdst = smem + OFF_KV + s * kStage;
+        uint8_t* vdst = kdst + kTileBytes;
+        mbar_arrive_expect_tx(&bar[B_KVF + s], kStage);
+        if (b < P.nG + P.nW) {  // a gist block or a window block
+          const bool gist = b < P.nG;
+          const int row0 = gist ? b * kBlk : ws + (b - P.nG) * kBlk;
+          const CUtensorMap* mk = gist ? &P.gk : &P.ck;
+          const CUtensorMap* mv = gist ? &P.gv : &P.cv;
+          for (int at = 0; at < 2; ++at) {
+            tma_load_4d(kdst + at * kAtom, mk, &bar[B_KVF + s], at * 64, g, row0, seq);
+            tma_load_4d(vdst + at * kAtom, mv, &bar[B_KVF + s], at * 64, g, row0, seq);
+          }
+        } else {
+          const int cb = b - P.nG - P.nW;
+          for (int i = 0; i < cpb; ++i) {
+            const int slot = cb * cpb + i;
+            // an empty slot loads chunk 0 (finite values; its keys are masked)
+            const int c = (slot < P.top_k && sel_s[slot] >= 0) ? sel_s[slot] : 0;
+            const uint32_t roff = (uint32_t)(i * P.chunk) * 128u;
+            for (int at = 0; at < 2; ++at) {
+              tma_load_4d(kdst + at * kAtom + roff, &P.ckc, &bar[B_KVF + s], at * 64, g,
+                          c * P.chunk, seq);
+              tma_load_4d(vdst + at * kAtom + roff, &P.cvc, &bar[B_KVF + s], at * 64, g,
+                          c * P.chunk, seq);
+            }
+          }
+        }
+        last = b;
+      }
+      // every copy this CTA started must land before the CTA may exit
+      volatile int no_abort = 0;
+      for (int s = 0; s < 2; ++s) {
+        if (last >= s) {
+          const int bs = last - ((last - s) & 1);
+          mbar_wait(&bar[B_KVF + s], (bs >> 1) & 1, &no_abort, nullptr, 3);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // --------------------------------------------------------- MMA issuer
+      constexpr uint32_t kIdQK = idesc_bf16_f32(kBlk, kN, false, false);
+      constexpr uint32_t kIdPV = idesc_bf16_f32(kD, kN, true, false);
+      bool ok = mbar_wait(&bar[B_QR], 0, abort, st, 10);
+      for (int b = 0; ok && b <= nb; ++b) {
+        if (b < nb) {
+          const int s = b & 1;
+          if (!mbar_wait(&bar[B_KVF + s], (b >> 1) & 1, abort, st, 11) ||
+              !mbar_wait(&bar[B_SE + s], ((b >> 1) & 1) ^ 1, abort, st, 12))
+            break;
+          tc_fence_after();
+          const uint32_t kb = sb + OFF_KV + s * kStage;
+#pragma unroll
+          for (int kk = 0; kk < kD / 16; ++kk) {
+            const uint64_t ad = smem_desc_sw128(kb + (kk >> 2) * kAtom + (kk & 3) * 32, 16, 1024);
+            const uint64_t bd =
+                smem_desc_sw128(sb + OFF_QT + (kk >> 2) * kQtAtom + (kk & 3) * 32, 16, 1024);
+            mma_bf16(tmem + s * kN, ad, bd, kIdQK, kk > 0);
+          }
+          mma_commit(&bar[B_SF + s]);
+        }
+        if (b >= 1) {
+          const int bp = b - 1, s = bp & 1;
+          if (!mbar_wait(&bar[B_PF + s], (bp >> 1) & 1, abort, st, 13)) break;
+          tc_fence_after();
+          const uint32_t vb = sb + OFF_KV + s * kStage + kTileBytes;
+          const uint32_t pb = sb + OFF_PT + s * 2 * kQtAtom;
+#pragma unroll
+          for (int kk = 0; kk < kBlk / 16; ++kk) {
+            // A = V^T (dims x keys, dims contiguous), B = P^T (heads x keys, keys contiguous)
+            const uint64_t ad = smem_desc_sw128(vb + kk * 2048, kAtom, 1024);
+            const uint64_t bd = smem_desc_sw128(pb + (kk >> 2) * kQtAtom + (kk & 3) * 32, 16, 1024);
+            mma_bf16(tmem + kTmemO, ad, bd, kIdPV, (bp > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(&bar[B_PD]);
+          mma_commit(&bar[B_KVE + s]);
+        }
+      }
+      mma_commit(&bar[B_DRAIN]);
+      volatile int no_abort = 0;
+      mbar_wait(&bar[B_DRAIN], 0, &no_abort, nullptr, 14);
+    }
+  } else {
+    // ------------------------------------------- softmax, selection, epilogue
+    const int sw = warp - 2;                // softmax warp 0..3
+    const int quarter = warp & 3;           // TMEM lane quarter of this warp
+    const int r = quarter * 32 + lane;      // key row of a block / output dimension
+    const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
+    GroupSync gs{&bar[B_GS], 0u, abort, st};
+    float* scores = reinterpret_cast<float*>(smem + OFF_SCORE);
+    float* red = reinterpret_cast<float*>(smem + OFF_RED);  // [2][4][kN]
+    uint32_t* hist = reinterpret_cast<uint32_t*>(smem + OFF_HIST);
+    uint32_t* scan = reinterpret_cast<uint32_t*>(smem + OFF_SCAN);
+
+    // Q^T of the group (rows >= REP zero) and zeroed P^T buffers
+    for (int x = r; x < kN * (kD / 8); x += 128) {
+      const int h = x >> 4, c0 = (x & 15) * 8;
+      uint32_t w4[4] = {0u, 0u, 0u, 0u};
+      if (h < REP) {
+        const __nv_bfloat16* qp = P.q + seq * P.qs[0] + (int64_t)(g * REP + h) * P.qs[1] + c0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          w4[i] = pack_bf16(__bfloat162float(qp[2 * i]), __bfloat162float(qp[2 * i + 1]));
+      }
+      st_shared_v4(sb + OFF_QT + (c0 >> 6) * kQtAtom + sw128_offset(h, c0 & 63), w4[0], w4[1],
+                   w4[2], w4[3]);
+    }
+    for (int x = r; x < (int)(2 * 2 * kQtAtom / 16); x += 128)
+      st_shared_v4(sb + OFF_PT + x * 16, 0u, 0u, 0u, 0u);
+    fence_async_shared();
+    mbar_arrive(&bar[B_QR]);
+
+    const float sl2 = P.scale * 1.4426950408889634f;
+    float m_run[REP], l_part[REP];
+#pragma unroll
+    for (int h = 0; h < REP; ++h) {
+      m_run[h] = -INFINITY;
+      l_part[h] = 0.f;
+    }
+    const int wstart = P.cache_len - P.window, cpb = kBlk / P.chunk;
+    bool ok = true;
+    for (int b = 0; b < nb; ++b) {
+      const int s = b & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(&bar[B_SF + s], (b >> 1) & 1, abort, st, 20))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      __syncwarp();
+      float sv[kN];
+      tmem_ld16(lane_addr + s * kN, sv);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(&bar[B_SE + s]);
+      bool valid;
+      if (b < P.nG) {
+        const int key = b * kBlk + r;
+        valid = key < P.G;
+        if (valid) {  // selection score: sum over the group's heads of q_h . k * scale
+          float sum = 0.f;
+#pragma unroll
+          for (int h = 0; h < REP; ++h) sum += sv[h];
+          scores[key] = sum * P.scale;
+        }
+      } else if (b < P.nG + P.nW) {
+        valid = wstart + (b - P.nG) * kBlk + r < P.cache_len;
+      } else {
+        const int slot = (b - P.nG - P.nW) * cpb + r / P.chunk;
+        valid = slot < P.top_k && sel_s[slot] >= 0;
+      }
+      // block maximum per head over the four softmax warps
+      float* rb = red + s * 4 * kN;
+#pragma unroll
+      for (int h = 0; h < REP; ++h) {
+        float v = valid ? sv[h] : -INFINITY;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
+        if (lane == 0) rb[sw * kN + h] = v;
+      }
+      mbar_arrive(&bar[B_MX]);
+      if (!__all_sync(0xffffffffu, mbar_wait(&bar[B_MX], b & 1, abort, st, 21))) {
+        ok = false;
+        break;
+      }
+      float alpha[REP], pv[REP];
+      bool any_resc = false;
+#pragma unroll
+      for (int h = 0; h < REP; ++h) {
+        const float M = fmaxf(fmaxf(rb[h], rb[kN + h]), fmaxf(rb[2 * kN + h], rb[3 * kN + h]));
+        const float m_new = fmaxf(m_run[h], M * sl2);  // scale > 0 keeps the order
+        const bool resc = m_new > m_run[h] + 8.f;       // the same in every thread
+        const float m_use = resc ? m_new : m_run[h];
+        alpha[h] = !resc ? 1.f : (m_run[h] == -INFINITY ? 0.f : ex2(m_run[h] - m_use));
+        pv[h] = (valid && m_use != -INFINITY) ? ex2(fmaf(sv[h], sl2, -m_use)) : 0.f;
+        l_part[h] = l_part[h] * alpha[h] + pv[h];
+        m_run[h] = m_use;
+        any_resc = any_resc || resc;
+      }
+      // P V(b - 1) is done: P^T buffer s (read by P V(b - 2)) is free, O^T is quiet
+      if (b >= 1 &&
+          !__all_sync(0xffffffffu, mbar_wait(&bar[B_PD], (b - 1) & 1, abort, st, 22))) {
+        ok = false;
+        break;
+      }
+      if (any_resc && b >= 1) {
+        tc_fence_after();
+        __syncwarp();
+        float o[kN];
+        tmem_ld16(lane_addr + kTmemO, o);
+        tmem_wait_ld();
+#pragma unroll
+        for (int h = 0; h < REP; ++h) o[h] *= alpha[h];
+        tmem_st16(lane_addr + kTmemO, o);
+        tmem_wait_st();
+      }
+      uint8_t* pt = smem + OFF_PT + s * 2 * kQtAtom + (r >> 6) * kQtAtom;
+#pragma unroll
+      for (int h = 0; h < REP; ++h)
+        *reinterpret_cast<__nv_bfloat16*>(pt + sw128_offset(h, r & 63)) = __float2bfloat16_rn(pv[h]);
+      fence_async_shared();
+      tc_fence_before();
+      mbar_arrive(&bar[B_PF + s]);
+
+      if (b == P.nG - 1 && P.top_k > 0) {
+        // ---------------------------------------------------- top-k select
+        // thread r owns gists [r * per, r * per + per): ascending index order
+        // across threads, so an exclusive scan keeps the output ascending
+        ok = ok && gs(30);  // every score is written
+        const int per = (P.G + 127) / 128, j0 = r * per, j1 = min(P.G, j0 + per);
+        const int64_t last_ok = (int64_t)P.cache_len - P.window;
+        auto key_of = [&](int j) -> uint32_t {
+          return ((int64_t)(j + 1) * P.chunk <= last_ok) ? float_key(scores[j]) : 0u;
+        };
+        uint32_t n_elig = 0;
+        for (int j = j0; j < j1; ++j) n_elig += key_of(j) != 0u;
+        uint32_t E = 0;
+        group_exclusive_scan(n_elig, r, scan, gs, ok, &E);
+        // threshold T and the number of keys equal to T to take (lowest indices)
+        uint32_t T = 0u, want = 0u;
+        if (E > (uint32_t)P.top_k) {
+          uint32_t prefix = 0u, pmask = 0u;
+          want = (uint32_t)P.top_k;
+          for (int pass = 0; pass < 4 && ok; ++pass) {
+            const int shift = 24 - 8 * pass;
+            hist[r] = 0u;
+            hist[r + 128] = 0u;
+            ok = ok && gs(31);
+            for (int j = j0; j < j1; ++j) {
+              const uint32_t k = key_of(j);
+              if (k != 0u && (k & pmask) == prefix) atomicAdd(&hist[(k >> shift) & 255u], 1u);
+            }
+            ok = ok && gs(32);
+            if (sw == 0) {
+              // lane l sums bins [8l, 8l + 8); suffix over lanes from the top
+              uint32_t c8 = 0u;
+#pragma unroll
+              for (int i = 0; i < 8; ++i) c8 += hist[8 * lane + i];
+              uint32_t suf = c8;
+#pragma unroll
+              for (int off = 1; off < 32; off <<= 1) {
+                const uint32_t y = __shfl_down_sync(0xffffffffu, suf, off);
+                if (lane + off < 32) suf += y;
+              }
+              const uint32_t mask = __ballot_sync(0xffffffffu, suf >= want);
+              const int L = 31 - __clz(mask);  // highest lane whose suffix reaches want
+              if (lane == L) {
+                uint32_t above = suf - c8;  // keys in bins above this lane's
+                int B = 8 * lane;
+                for (int bb = 8 * lane + 7; bb >= 8 * lane; --bb) {
+                  if (above + hist[bb] >= want) {
+                    B = bb;
+                    break;
+                  }
+                  above += hist[bb];
+                }
+                scan[4] = (uint32_t)B;
+                scan[5] = want - above;
+              }
+            }
+            ok = ok && gs(33);
+            prefix |= scan[4] << shift;
+            pmask |= 0xFFu << shift;
+            want = scan[5];
+            ok = ok && gs(34);  // scan[4..5] and hist are rewritten by the next pass
+          }
+          T = prefix;
+        }
+        // take key > T, and the first `want` keys equal to T in index order
+        uint32_t n_gt = 0u, n_eq = 0u;
+        for (int j = j0; j < j1; ++j) {
+          const uint32_t k = key_of(j);
+          n_gt += k > T;
+          n_eq += (k == T && k != 0u);
+        }
+        uint32_t eq_total = 0u, sel_total = 0u;
+        const uint32_t eq_before = group_exclusive_scan(n_eq, r, scan, gs, ok, &eq_total);
+        const uint32_t take_eq = want > eq_before ? min(n_eq, want - eq_before) : 0u;
+        uint32_t off = group_exclusive_scan(n_gt + take_eq, r, scan, gs, ok, &sel_total);
+        uint32_t eq_seen = 0u;
+        for (int j = j0; j < j1; ++j) {
+          const uint32_t k = key_of(j);
+          const bool take = k > T || (k == T && k != 0u && eq_seen++ < take_eq);
+          if (take && off < (uint32_t)P.top_k) sel_s[off++] = j;
+        }
+        for (int x = r; x < P.top_k; x += 128)
+          if (x >= (int)sel_total) sel_s[x] = -1;
+        ok = ok && gs(35);
+        int32_t* sel_out = P.sel + ((int64_t)seq * P.Hkv + g) * P.top_k;
+        for (int x = r; x < P.top_k; x += 128) sel_out[x] = sel_s[x];
+        mbar_arrive(&bar[B_SELD]);  // release: sel_s is complete
+        if (!__all_sync(0xffffffffu, ok)) break;
+      }
+    }
+    // -------------------------------------------------------------- epilogue
+    if (ok && nb > 0 &&
+        __all_sync(0xffffffffu, mbar_wait(&bar[B_PD], (nb - 1) & 1, abort, st, 23))) {
+      float* lr = red + (nb & 1) * 4 * kN;  // the slot no thread reads any more
+#pragma unroll
+      for (int h = 0; h < REP; ++h) {
+        float v = l_part[h];
+#pragma unroll
+        for (int off2 = 16; off2 > 0; off2 >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off2);
+        if (lane == 0) lr[sw * kN + h] = v;
+      }
+      if (gs(36)) {
+        tc_fence_after();
+        __syncwarp();
+        float o[kN];
+        tmem_ld16(lane_addr + kTmemO, o);  // lane = output dimension r
+        tmem_wait_ld();
+#pragma unroll
+        for (int h = 0; h < REP; ++h) {
+          const float l = (lr[h] + lr[kN + h]) + (lr[2 * kN + h] + lr[3 * kN + h]);
+          const int hq = g * REP + h;
+          P.o[seq * P.os[0] + (int64_t)hq * P.os[1] + r] =
+              __float2bfloat16_rn(l > 0.f ? o[h] / l : 0.f);
+          if (r == 0)
+            P.lse[(int64_t)seq * P.Hkv * REP + hq] =
+                l > 0.f ? (m_run[h] + __log2f(l)) * 0.6931471805599453f : -INFINITY;
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tmem, kTmemCols);
+}
+
+// --------------------------------------------------------------- host side
+// Shapes this kernel takes: 8 <= chunk <= 128 dividing 128 (a chunk is whole
+// 8-row swizzle groups of a block), at least one full block of gists and of
+// cache positions (TMA boxes of 128 rows), and whatever check_decode admits.
+bool decode_tc_supported(const sa_decode_desc& d) {
+  return d.head_dim == kD && d.chunk >= 8 && d.chunk <= kBlk && kBlk % d.chunk == 0 &&
+         d.n_gists >= kBlk && d.n_gists <= kMaxG && d.cache_len >= kBlk &&
+         d.top_k <= kMaxTopK && d.num_q_heads / d.num_kv_heads <= 8;
+}
+
+template <int REP>
+static cudaError_t decode_tc_launch(const Params& P, cudaStream_t s) {
+  cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel<REP>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  if (e != cudaSuccess) return e;
+  decode_tc_kernel<REP><<<dim3(P.n_seq * P.Hkv), kThreads, kSmemBytes, s>>>(P);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_decode_tc(const sa_decode_desc& d, const void* q, const void* gk,
+                             const void* gv, const void* kc, const void* vc, int32_t* sel, void* o,
+                             float* lse, void* ws, cudaStream_t s) {
+  Params P;
+  memset(&P, 0, sizeof(P));
+  const int64_t gstr[3] = {d.gist_strides[0], d.gist_strides[2], d.gist_strides[1]};
+  const int64_t cstr[3] = {d.cache_strides[0], d.cache_strides[2], d.cache_strides[1]};
+  if (!make_tile_map_box(&P.gk, gk, kD, d.num_kv_heads, d.n_gists, d.n_seq, gstr, kBlk) ||
+      !make_tile_map_box(&P.gv, gv, kD, d.num_kv_heads, d.n_gists, d.n_seq, gstr, kBlk) ||
+      !make_tile_map_box(&P.ck, kc, kD, d.num_kv_heads, d.cache_len, d.n_seq, cstr, kBlk) ||
+      !make_tile_map_box(&P.cv, vc, kD, d.num_kv_heads, d.cache_len, d.n_seq, cstr, kBlk) ||
+      !make_tile_map_box(&P.ckc, kc, kD, d.num_kv_heads, d.cache_len, d.n_seq, cstr, d.chunk) ||
+      !make_tile_map_box(&P.cvc, vc, kD, d.num_kv_heads, d.cache_len, d.n_seq, cstr, d.chunk))
+    return cudaErrorInvalidValue;
+  P.q = static_cast<const __nv_bfloat16*>(q);
+  P.o = static_cast<__nv_bfloat16*>(o);
+  P.lse = lse;
+  P.sel = sel;
+  P.status = static_cast<DeviceStatus*>(ws);
+  P.n_seq = d.n_seq;
+  P.Hkv = d.num_kv_heads;
+  P.rep = d.num_q_heads / d.num_kv_heads;
+  P.G = d.n_gists;
+  P.cache_len = d.cache_len;
+  P.chunk = d.chunk;
+  P.top_k = d.top_k;
+  P.window = d.window;
+  P.nG = (d.n_gists + kBlk - 1) / kBlk;
+  P.nW = (d.window + kBlk - 1) / kBlk;
+  const int cpb = kBlk / d.chunk;
+  P.nC = (d.top_k + cpb - 1) / cpb;
+  P.scale = d.softmax_scale > 0.f ? d.softmax_scale : 1.f / sqrtf((float)d.head_dim);
+  for (int i = 0; i < 2; ++i) {
+    P.qs[i] = d.q_strides[i];
+    P.os[i] = d.o_strides[i];
+  }
+  switch (P.rep) {
+    case 1: return decode_tc_launch<1>(P, s);
+    case 2: return decode_tc_launch<2>(P, s);
+    case 4: return decode_tc_launch<4>(P, s);
+    case 8: return decode_tc_launch<8>(P, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace sa

@@ -95,3 +95,18 @@ def test_decode_group_sizes(sa, rep):
 
 def test_decode_full_size(sa):
     check(sa, W.WORKLOADS["gist_decode_128k"], seqs=[0, 7, 15])
+
+
+@pytest.mark.parametrize("top_k,window,chunk,G", [
+    (0, 256, 16, 256),     # nothing unfolded
+    (40, 0, 32, 256),      # no window: chunk blocks follow the gist blocks
+    (256, 128, 8, 200),    # fewer eligible chunks than top_k: -1 padding
+    (17, 1000, 128, 130),  # one chunk per block, ragged window and gist blocks
+    (33, 300, 64, 777),    # two chunks per block, ragged everywhere
+])
+def test_decode_tensor_core_shapes(sa, top_k, window, chunk, G):
+    """Shapes of the one-CTA-per-(sequence, KV head) tensor-core kernel
+    (G >= 128, 8 <= chunk <= 128 dividing 128)."""
+    w = W.scaled("gist_decode_128k", index=500 + top_k + G, n_seq=2, cache_len=chunk * G,
+                 chunk=chunk, n_gists=G, top_k=top_k, window=window, heads=8, kv_heads=2)
+    check(sa, w)
