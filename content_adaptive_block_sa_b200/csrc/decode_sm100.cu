@@ -20,8 +20,9 @@
 // The output O = O^T / l and LSE follow from the single softmax state; no
 // partial results leave the CTA.
 //
-// Roles (192 threads): warp 0 issues the TMA loads (K and V blocks into a
-// 2-stage ring) and owns the TMEM allocation; one thread of warp 1 issues
+// Roles (192 threads): warp 0 issues the TMA loads (K blocks into a 3-stage
+// ring, up to two blocks ahead, freed once Q K^T has read them; V blocks into
+// a 2-stage ring, freed after P V) and owns the TMEM allocation; one thread of warp 1 issues
 // tcgen05.mma (S^T = K Q^T, M = 128 keys, N = 16 head columns; O^T += V^T P,
 // M = 128 dims, N = 16) with completion on mbarriers; warps 2-5 (thread = key
 // row of the block for the softmax, = output dimension for O^T) run the
@@ -69,10 +70,12 @@ struct Params {
 // Shared memory (offsets from a 1024-aligned base).
 constexpr uint32_t kAtom = kBlk * 128;          // [128 rows][64 bf16]
 constexpr uint32_t kTileBytes = 2 * kAtom;      // one K or V block, 2 atoms
-constexpr uint32_t kStage = 2 * kTileBytes;     // K + V
+constexpr int kKStages = 3, kVStages = 2;
+constexpr int kKAhead = 2;                      // K blocks requested ahead of V
 constexpr uint32_t kQtAtom = kN * 128;          // [16 rows][64 bf16]
-constexpr uint32_t OFF_KV = 0;                  // 2 stages
-constexpr uint32_t OFF_QT = 2 * kStage;         // Q^T [16][128], 2 atoms
+constexpr uint32_t OFF_K = 0;
+constexpr uint32_t OFF_V = OFF_K + kKStages * kTileBytes;
+constexpr uint32_t OFF_QT = OFF_V + kVStages * kTileBytes;  // Q^T [16][128], 2 atoms
 constexpr uint32_t OFF_PT = OFF_QT + 2 * kQtAtom;  // P^T [2 buffers][16][128], 2 atoms each
 constexpr uint32_t OFF_SCORE = OFF_PT + 2 * 2 * kQtAtom;  // float [kMaxG]
 constexpr uint32_t OFF_HIST = OFF_SCORE + kMaxG * 4;     // uint32 [256]
@@ -83,8 +86,8 @@ constexpr uint32_t OFF_BARS = OFF_SCAN + 64;
 constexpr uint32_t kSmemBytes = OFF_BARS + 256 + 1024;
 
 enum {
-  B_KVF = 0, B_KVE = 2, B_SF = 4, B_SE = 6, B_PF = 8, B_PD = 10, B_MX = 11, B_GS = 12,
-  B_QR = 13, B_SELD = 14, B_DRAIN = 15, kNumBars = 16
+  B_KF = 0, B_KE = 3, B_VF = 6, B_VE = 8, B_SF = 10, B_SE = 12, B_PF = 14, B_PD = 16, B_MX = 17,
+  B_GS = 18, B_QR = 19, B_SELD = 20, B_DRAIN = 21, kNumBars = 22
 };
 
 constexpr uint32_t kTmemCols = 64;  // S^T buffers at 0 and 16, O^T at 32
@@ -156,9 +159,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
   DeviceStatus* st = P.status;
 
   if (threadIdx.x == 0) {
+    for (int s = 0; s < kKStages; ++s) {
+      mbar_init(&bar[B_KF + s], 1);
+      mbar_init(&bar[B_KE + s], 1);
+    }
+    for (int s = 0; s < kVStages; ++s) {
+      mbar_init(&bar[B_VF + s], 1);
+      mbar_init(&bar[B_VE + s], 1);
+    }
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&bar[B_KVF + s], 1);
-      mbar_init(&bar[B_KVE + s], 1);
       mbar_init(&bar[B_SF + s], 1);
       mbar_init(&bar[B_SE + s], 128);
       mbar_init(&bar[B_PF + s], 128);
@@ -192,49 +201,67 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
       prefetch_tmap(&P.cvc);
       const int ws = P.cache_len - P.window;
       const int cpb = kBlk / P.chunk;  // chunks per block
-      int last = -1;
-      for (int b = 0; b < nb; ++b) {
-        const int s = b & 1;
-        if (!mbar_wait(&bar[B_KVE + s], ((b >> 1) & 1) ^ 1, abort, st, 1)) break;
-        // the chunks are known once the selection is done
-        if (b == P.nG + P.nW && !mbar_wait(&bar[B_SELD], 0, abort, st, 2)) break;
-        uint8_t* kdst = smem + OFF_KV + s * kStage;
-        uint8_t* vdst = kdst + kTileBytes;
-        mbar_arrive_expect_tx(&bar[B_KVF + s], kStage);
+      int last_k = -1, last_v = -1;
+      // block b of K (is_k) or V into its ring slot; false on timeout
+      auto load = [&](bool is_k, int b) -> bool {
+        const int ns = is_k ? kKStages : kVStages, s = b % ns;
+        if (!mbar_wait(&bar[(is_k ? B_KE : B_VE) + s], ((b / ns) & 1) ^ 1, abort, st, 1))
+          return false;
+        uint8_t* dst = smem + (is_k ? OFF_K : OFF_V) + s * kTileBytes;
+        uint64_t* full = &bar[(is_k ? B_KF : B_VF) + s];
+        mbar_arrive_expect_tx(full, kTileBytes);
         if (b < P.nG + P.nW) {  // a gist block or a window block
           const bool gist = b < P.nG;
           const int row0 = gist ? b * kBlk : ws + (b - P.nG) * kBlk;
-          const CUtensorMap* mk = gist ? &P.gk : &P.ck;
-          const CUtensorMap* mv = gist ? &P.gv : &P.cv;
-          for (int at = 0; at < 2; ++at) {
-            tma_load_4d(kdst + at * kAtom, mk, &bar[B_KVF + s], at * 64, g, row0, seq);
-            tma_load_4d(vdst + at * kAtom, mv, &bar[B_KVF + s], at * 64, g, row0, seq);
-          }
+          const CUtensorMap* map = gist ? (is_k ? &P.gk : &P.gv) : (is_k ? &P.ck : &P.cv);
+          for (int at = 0; at < 2; ++at) tma_load_4d(dst + at * kAtom, map, full, at * 64, g, row0, seq);
         } else {
           const int cb = b - P.nG - P.nW;
+          const CUtensorMap* map = is_k ? &P.ckc : &P.cvc;
           for (int i = 0; i < cpb; ++i) {
             const int slot = cb * cpb + i;
             // an empty slot loads chunk 0 (finite values; its keys are masked)
             const int c = (slot < P.top_k && sel_s[slot] >= 0) ? sel_s[slot] : 0;
             const uint32_t roff = (uint32_t)(i * P.chunk) * 128u;
-            for (int at = 0; at < 2; ++at) {
-              tma_load_4d(kdst + at * kAtom + roff, &P.ckc, &bar[B_KVF + s], at * 64, g,
-                          c * P.chunk, seq);
-              tma_load_4d(vdst + at * kAtom + roff, &P.cvc, &bar[B_KVF + s], at * 64, g,
-                          c * P.chunk, seq);
-            }
+            for (int at = 0; at < 2; ++at)
+              tma_load_4d(dst + at * kAtom + roff, map, full, at * 64, g, c * P.chunk, seq);
           }
         }
-        last = b;
+        if (is_k) last_k = b; else last_v = b;
+        return true;
+      };
+      // K runs up to kKAhead blocks ahead of V. A chunk block's K needs the
+      // selection: it is prefetched only once the selection is known, and
+      // waited for only when it is the K of the current block (by then every
+      // earlier V has been requested, so the softmax can reach the selection).
+      bool ok = true, seld = P.nC == 0;
+      int nk = 0;
+      for (int b = 0; ok && b < nb; ++b) {
+        while (ok && nk < nb && nk <= b + kKAhead) {
+          if (nk >= P.nG + P.nW && !seld) {
+            if (nk > b) break;
+            if (!mbar_wait(&bar[B_SELD], 0, abort, st, 2)) {
+              ok = false;
+              break;
+            }
+            seld = true;
+          }
+          ok = load(true, nk++);
+        }
+        if (ok) ok = load(false, b);
       }
       // every copy this CTA started must land before the CTA may exit
       volatile int no_abort = 0;
-      for (int s = 0; s < 2; ++s) {
-        if (last >= s) {
-          const int bs = last - ((last - s) & 1);
-          mbar_wait(&bar[B_KVF + s], (bs >> 1) & 1, &no_abort, nullptr, 3);
+      for (int s = 0; s < kKStages; ++s)
+        if (last_k >= s) {
+          const int bs = last_k - ((last_k - s) % kKStages);
+          mbar_wait(&bar[B_KF + s], (bs / kKStages) & 1, &no_abort, nullptr, 3);
         }
-      }
+      for (int s = 0; s < kVStages; ++s)
+        if (last_v >= s) {
+          const int bs = last_v - ((last_v - s) % kVStages);
+          mbar_wait(&bar[B_VF + s], (bs / kVStages) & 1, &no_abort, nullptr, 4);
+        }
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -244,12 +271,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
       bool ok = mbar_wait(&bar[B_QR], 0, abort, st, 10);
       for (int b = 0; ok && b <= nb; ++b) {
         if (b < nb) {
-          const int s = b & 1;
-          if (!mbar_wait(&bar[B_KVF + s], (b >> 1) & 1, abort, st, 11) ||
+          const int s = b & 1, sk = b % kKStages;
+          if (!mbar_wait(&bar[B_KF + sk], (b / kKStages) & 1, abort, st, 11) ||
               !mbar_wait(&bar[B_SE + s], ((b >> 1) & 1) ^ 1, abort, st, 12))
             break;
           tc_fence_after();
-          const uint32_t kb = sb + OFF_KV + s * kStage;
+          const uint32_t kb = sb + OFF_K + sk * kTileBytes;
 #pragma unroll
           for (int kk = 0; kk < kD / 16; ++kk) {
             const uint64_t ad = smem_desc_sw128(kb + (kk >> 2) * kAtom + (kk & 3) * 32, 16, 1024);
@@ -258,12 +285,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
             mma_bf16(tmem + s * kN, ad, bd, kIdQK, kk > 0);
           }
           mma_commit(&bar[B_SF + s]);
+          mma_commit(&bar[B_KE + sk]);
         }
         if (b >= 1) {
-          const int bp = b - 1, s = bp & 1;
-          if (!mbar_wait(&bar[B_PF + s], (bp >> 1) & 1, abort, st, 13)) break;
+          const int bp = b - 1, s = bp & 1, sv = bp % kVStages;
+          if (!mbar_wait(&bar[B_VF + sv], (bp / kVStages) & 1, abort, st, 15) ||
+              !mbar_wait(&bar[B_PF + s], (bp >> 1) & 1, abort, st, 13))
+            break;
           tc_fence_after();
-          const uint32_t vb = sb + OFF_KV + s * kStage + kTileBytes;
+          const uint32_t vb = sb + OFF_V + sv * kTileBytes;
           const uint32_t pb = sb + OFF_PT + s * 2 * kQtAtom;
 #pragma unroll
           for (int kk = 0; kk < kBlk / 16; ++kk) {
@@ -273,7 +303,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
             mma_bf16(tmem + kTmemO, ad, bd, kIdPV, (bp > 0 || kk > 0) ? 1u : 0u);
           }
           mma_commit(&bar[B_PD]);
-          mma_commit(&bar[B_KVE + s]);
+          mma_commit(&bar[B_VE + sv]);
         }
       }
       mma_commit(&bar[B_DRAIN]);
