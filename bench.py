@@ -97,6 +97,34 @@ class ClockSampler:
 _host_out = {}
 
 
+KERNEL_SOURCES = {"fwd_tc_kernel": "attn_fwd_sm100.cu", "bwd_tc_kernel": "attn_bwd_sm100.cu",
+                  "decode_tc_kernel": "decode_sm100.cu"}
+
+
+def kernel_digest(kernel):
+    """SHA-256 (16 hex digits) of a kernel's .cu file and the shared headers."""
+    import hashlib
+    csrc = os.path.join(ROOT, "content_adaptive_block_sa_b200", "csrc")
+    m = hashlib.sha256()
+    for f in [KERNEL_SOURCES[kernel], "sm100.cuh", "attn_mask.cuh", "sa_common.cuh"]:
+        with open(os.path.join(csrc, f), "rb") as fh:
+            m.update(fh.read())
+    return m.hexdigest()[:16]
+
+
+def recorded_traffic(workload, kernel):
+    """DRAM bytes per launch from profiles/traffic.md, or None when no row
+    exists or the kernel's sources changed since the counters were taken."""
+    path = os.path.join(ROOT, "profiles", "traffic.md")
+    if kernel not in KERNEL_SOURCES or not os.path.exists(path):
+        return None
+    for line in open(path):
+        cells = [c.strip() for c in line.strip().strip("|").split("|")]
+        if len(cells) == 8 and cells[0] == workload and cells[1] == kernel:
+            return int(cells[5]) if cells[2] == kernel_digest(kernel) else None
+    return None
+
+
 def copy_out(tensors):
     """Device -> pinned host copies of a step's results (reused buffers)."""
     outs = []
@@ -147,7 +175,9 @@ class GzipWorkload:
         self.pairs = pairs
         self.flops_fwd = 4.0 * d * b * b * pairs
         self.flops = self.flops_fwd * (1 + (2.5 if backward else 0))
-        self.kernels_per_step = 2 + (3 if backward else 0)
+        # builder + forward (+ backward: row prep + key-major kernel)
+        self.kernels_per_step = 2 + (2 if backward else 0)
+        self.kernel = "fwd_tc_kernel"
         self.unit = "TFLOP/s"
 
     def fwd_only(self):
@@ -165,6 +195,8 @@ class GzipWorkload:
         if self.backward:
             sa.sa_backward(self.ad, self.md, self.q, self.k, self.v, self.o, self.lse, self.do,
                            self.lists, self.dq, self.dk, self.dv, self.bws)
+            if ev is not None:
+                ev[2].record()
 
     def e2e_step(self):
         """Host buffers in, result out: the public API with H2D/D2H copies."""
@@ -239,7 +271,9 @@ class GistWorkload(GzipWorkload):
         width = np.where(kinds == 2, w["gist_tail"], 128)
         self.flops_fwd = 4.0 * d * H * 128 * float(width.sum())
         self.flops = self.flops_fwd
-        self.kernels_per_step = 2
+        # builder + sink/gist gather + near-tile masks + forward
+        self.kernels_per_step = 4
+        self.kernel = "fwd_tc_kernel"
         self.unit = "TFLOP/s"
 
     def e2e_step(self):
@@ -303,7 +337,11 @@ class DecodeWorkload:
         per = (G + w["top_k"] * w["chunk"] + w["window"]) * d * 2 * 2
         self.bytes = float(n * Hkv * per + 2 * self.q.numel() * 2 + self.lse.numel() * 4
                            + self.sel.numel() * 4)
-        self.kernels_per_step = 4
+        # one tensor-core kernel for these shapes, else the four CUDA-core passes
+        c = w["chunk"]
+        tc = 8 <= c <= 128 and 128 % c == 0 and 128 <= G <= 8192 and L >= 128
+        self.kernels_per_step = 1 if tc else 4
+        self.kernel = "decode_tc_kernel" if tc else "decode (4 CUDA-core passes)"
         self.unit = "GB/s"
 
     def step(self, ev=None):
@@ -464,7 +502,8 @@ def main():
     torch.cuda.synchronize()
 
     # ---- device-timed region: K steps, inputs resident
-    fwd_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+    # per step: before the timed kernel, after it (and after the backward)
+    fwd_ev = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3))
               for _ in range(args.steps)]
     clocks = ClockSampler(local)
     clocks.start()
@@ -479,7 +518,9 @@ def main():
     barrier()
     clk = clocks.stop()
     ms = max_over_ranks(t0.elapsed_time(t1)) / args.steps
-    kern_ms = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in fwd_ev])))
+    kern_ms = max_over_ranks(float(np.mean([e[0].elapsed_time(e[1]) for e in fwd_ev])))
+    bwd_ms = (max_over_ranks(float(np.mean([e[1].elapsed_time(e[2]) for e in fwd_ev])))
+              if getattr(wl, "backward", False) else None)
 
     # ---- end-to-end through the public API with host buffers
     for _ in range(2):
@@ -503,13 +544,22 @@ def main():
         e2e_value = weak_scaling_value(units, world, e2e_ms, 1e9)
         ach = wl.bytes / (kern_ms * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
-                "traffic": None, "peak_source": src, "kernel": "sa_gist_decode (4 launches)"}
+                "traffic": None, "peak_source": src, "kernel": wl.kernel}
     else:
         value = weak_scaling_value(wl.flops, world, ms, 1e12)
         e2e_value = weak_scaling_value(wl.flops, world, e2e_ms, 1e12)
-        ach = wl.flops_fwd / (kern_ms * 1e-3) / 1e12
+        fwd_ach = wl.flops_fwd / (kern_ms * 1e-3) / 1e12
+        if bwd_ms is not None and bwd_ms > kern_ms:  # the backward dominates the step
+            ach = (wl.flops - wl.flops_fwd) / (bwd_ms * 1e-3) / 1e12
+            kname = "bwd_tc_kernel"
+        else:
+            ach, kname = fwd_ach, wl.kernel
         roof = {"bound": "tensor", "achieved": ach, "peak": bf16, "unit": "TFLOP/s",
-                "frac": ach / bf16, "traffic": None, "peak_source": src, "kernel": "sa_forward"}
+                "frac": ach / bf16, "traffic": None, "peak_source": src, "kernel": kname}
+        if bwd_ms is not None:
+            roof["forward_tflops"] = fwd_ach
+            roof["backward_ms"] = bwd_ms
+    roof["traffic"] = recorded_traffic(args.workload if args.size == "full" else "", roof["kernel"])
     if rank != 0:
         if world > 1:
             dist.destroy_process_group()
