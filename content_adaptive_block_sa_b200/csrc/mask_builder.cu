@@ -16,10 +16,12 @@
 //   vis(i, j) = j <= i and (j < sinks or gist(j) or i - j < window)
 // with FULL / MASKED / TAIL kinds.
 //
-// One CTA builds one (sequence, class) pair (gzip) or the whole layout
-// (gist); counts are turned into absolute offsets with a block-wide scan into
-// fixed per-pair regions, so no global scratch and no second launch is
-// needed.
+// Gzip: one CTA builds one (sequence, class) pair; counts become absolute
+// offsets with a block-wide scan into fixed per-pair regions, and every list
+// is filled by one warp per row (column) with its lanes over the entries.
+// Gist: four launches, one warp per 128-position tile in each (bits and
+// permutation; row and column counts; one-CTA scans; list fills), so no
+// global scratch beyond the output lists is needed.
 #include "sa_common.cuh"
 
 namespace sa {
@@ -78,7 +80,11 @@ __global__ void __launch_bounds__(1024) gzip_build_kernel(GzipBuild p) {
   __syncthreads();
   const int L = lp[B], w = p.w;
 
-  // ---- CSR: query block i -> ascending key blocks
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+
+  // ---- CSR: query block i -> ascending key blocks (literal blocks below the
+  // window first, then the window lo..i; the literal class: literal blocks
+  // up to i, or i alone)
   int32_t* rp = p.row_ptr + (int64_t)bc * (B + 1);
   for (int i = threadIdx.x; i < B; i += blockDim.x) {
     const int lo = max(0, i - w);
@@ -91,21 +97,17 @@ __global__ void __launch_bounds__(1024) gzip_build_kernel(GzipBuild p) {
   if (threadIdx.x == 0) rp[0] = (int32_t)(bc * p.region);
   __syncthreads();
   block_inclusive_scan(rp + 1, B, (int32_t)(bc * p.region));
-  for (int i = threadIdx.x; i < B; i += blockDim.x) {
+  for (int i = warp; i < B; i += nwarps) {  // one warp per row, lanes over entries
     int32_t* out = p.col_idx + rp[i];
-    const int lo = max(0, i - w);
-    int n = 0;
-    if (cls == SA_CLASS_LITERAL) {
-      if (f[i]) for (int t = 0; t < lp[i + 1]; ++t) out[n++] = lit_idx[t];
-      else out[n++] = i;
-    } else {
-      if (cls == SA_CLASS_HYBRID && f[i])
-        for (int t = 0; t < lp[lo]; ++t) out[n++] = lit_idx[t];
-      for (int j = lo; j <= i; ++j) out[n++] = j;
-    }
+    const int lo = max(0, i - w), n = rp[i + 1] - rp[i];
+    const int nlit = cls == SA_CLASS_LITERAL ? (f[i] ? n : 0)
+                     : (cls == SA_CLASS_HYBRID && f[i] ? lp[lo] : 0);
+    for (int t = lane; t < n; t += 32)
+      out[t] = t < nlit ? lit_idx[t] : (cls == SA_CLASS_LITERAL ? i : lo + (t - nlit));
   }
 
-  // ---- CSC: key block j -> ascending query blocks
+  // ---- CSC: key block j -> ascending query blocks (the window j..hi, then
+  // literal blocks above it; the literal class: literal blocks from j, or j)
   int32_t* cp = p.col_ptr + (int64_t)bc * (B + 1);
   for (int j = threadIdx.x; j < B; j += blockDim.x) {
     const int hi = min(B - 1, j + w);
@@ -118,17 +120,14 @@ __global__ void __launch_bounds__(1024) gzip_build_kernel(GzipBuild p) {
   if (threadIdx.x == 0) cp[0] = (int32_t)(bc * p.region);
   __syncthreads();
   block_inclusive_scan(cp + 1, B, (int32_t)(bc * p.region));
-  for (int j = threadIdx.x; j < B; j += blockDim.x) {
+  for (int j = warp; j < B; j += nwarps) {
     int32_t* out = p.row_idx + cp[j];
-    const int hi = min(B - 1, j + w);
-    int n = 0;
-    if (cls == SA_CLASS_LITERAL) {
-      if (f[j]) for (int t = lp[j]; t < L; ++t) out[n++] = lit_idx[t];
-      else out[n++] = j;
-    } else {
-      for (int i = j; i <= hi; ++i) out[n++] = i;
-      if (cls == SA_CLASS_HYBRID && f[j])
-        for (int t = lp[hi + 1]; t < L; ++t) out[n++] = lit_idx[t];
+    const int hi = min(B - 1, j + w), n = cp[j + 1] - cp[j];
+    for (int t = lane; t < n; t += 32) {
+      int v;
+      if (cls == SA_CLASS_LITERAL) v = f[j] ? lit_idx[lp[j] + t] : j;
+      else v = t <= hi - j ? j + t : lit_idx[lp[hi + 1] + (t - (hi - j + 1))];
+      out[t] = v;
     }
   }
 
@@ -160,17 +159,15 @@ __global__ void __launch_bounds__(1024) gzip_build_kernel(GzipBuild p) {
     if (threadIdx.x == 0) trp[0] = (int32_t)(bc * p.tregion);
     __syncthreads();
     block_inclusive_scan(trp + 1, T, (int32_t)(bc * p.tregion));
-    for (int I = threadIdx.x; I < T; I += blockDim.x) {
-      const int i = I / r;
-      int n = trp[I];
-      for (int e = rp[i]; e < rp[i + 1]; ++e) {
-        const int kb = p.col_idx[e];
-        const int last = kb < i ? kb * r + r - 1 : I;
-        for (int J = kb * r; J <= last; ++J) {
-          p.tcol[n] = J;
-          p.tkind[n] = (int8_t)(J == I ? SA_TILE_MASKED : SA_TILE_FULL);
-          ++n;
-        }
+    for (int I = warp; I < T; I += nwarps) {
+      // entry x of the row: block entry x / r (the diagonal block, last in
+      // the list, contributes the tiles i r .. I)
+      const int i = I / r, e0 = rp[i], ne = rp[i + 1] - e0, n = trp[I + 1] - trp[I];
+      for (int x = lane; x < n; x += 32) {
+        const int k = min(x / r, ne - 1);
+        const int J = k < ne - 1 ? p.col_idx[e0 + k] * r + (x % r) : i * r + (x - (ne - 1) * r);
+        p.tcol[trp[I] + x] = J;
+        p.tkind[trp[I] + x] = (int8_t)(J == I ? SA_TILE_MASKED : SA_TILE_FULL);
       }
     }
     for (int J = threadIdx.x; J < T; J += blockDim.x) {
@@ -180,49 +177,69 @@ __global__ void __launch_bounds__(1024) gzip_build_kernel(GzipBuild p) {
     if (threadIdx.x == 0) tcp[0] = (int32_t)(bc * p.tregion);
     __syncthreads();
     block_inclusive_scan(tcp + 1, T, (int32_t)(bc * p.tregion));
-    for (int J = threadIdx.x; J < T; J += blockDim.x) {
-      const int j = J / r;
-      int n = tcp[J];
-      for (int e = cp[j]; e < cp[j + 1]; ++e) {
-        const int qb = p.row_idx[e];
-        for (int I = qb == j ? J : qb * r; I < qb * r + r; ++I) {
-          p.trow[n] = I;
-          p.tkind_t[n] = (int8_t)(I == J ? SA_TILE_MASKED : SA_TILE_FULL);
-          ++n;
-        }
+    for (int J = warp; J < T; J += nwarps) {
+      // the diagonal block, first in the column list, contributes J .. j r + r - 1
+      const int j = J / r, e0 = cp[j], n = tcp[J + 1] - tcp[J], nd = j * r + r - J;
+      for (int x = lane; x < n; x += 32) {
+        const int I = x < nd ? J + x : p.row_idx[e0 + 1 + (x - nd) / r] * r + (x - nd) % r;
+        p.trow[tcp[J] + x] = I;
+        p.tkind_t[tcp[J] + x] = (int8_t)(I == J ? SA_TILE_MASKED : SA_TILE_FULL);
       }
     }
     return;
   }
-  const int lb = __ffs(p.b) - 1;  // b divides 128: a power of two
-  for (int I = threadIdx.x; I < T; I += blockDim.x) {
+  // b < 128 (a power of two): the kind of every tile pair from the block
+  // bits; one warp per row (column), lanes over 32 candidate tiles at a time,
+  // compacted with ballots
+  const int lb = __ffs(p.b) - 1;
+  for (int I = warp; I < T; I += nwarps) {
     int cnt = 0;
-    for (int J = 0; J <= I; ++J) cnt += gzip_tile_kind(p, lb, cls, f, I, J) >= 0;
-    trp[I + 1] = cnt;
+    for (int J0 = 0; J0 <= I; J0 += 32) {
+      const int J = J0 + lane;
+      cnt += __popc(__ballot_sync(0xffffffffu, J <= I && gzip_tile_kind(p, lb, cls, f, I, J) >= 0));
+    }
+    if (lane == 0) trp[I + 1] = cnt;
   }
-  if (threadIdx.x == 0) trp[0] = (int32_t)(bc * p.tregion);
+  for (int J = warp; J < T; J += nwarps) {
+    int cnt = 0;
+    for (int I0 = J; I0 < T; I0 += 32) {
+      const int I = I0 + lane;
+      cnt += __popc(__ballot_sync(0xffffffffu, I < T && gzip_tile_kind(p, lb, cls, f, I, J) >= 0));
+    }
+    if (lane == 0) tcp[J + 1] = cnt;
+  }
+  if (threadIdx.x == 0) {
+    trp[0] = (int32_t)(bc * p.tregion);
+    tcp[0] = (int32_t)(bc * p.tregion);
+  }
   __syncthreads();
   block_inclusive_scan(trp + 1, T, (int32_t)(bc * p.tregion));
-  for (int I = threadIdx.x; I < T; I += blockDim.x) {
+  block_inclusive_scan(tcp + 1, T, (int32_t)(bc * p.tregion));
+  const uint32_t below = (1u << lane) - 1u;
+  for (int I = warp; I < T; I += nwarps) {
     int n = trp[I];
-    for (int J = 0; J <= I; ++J) {
-      const int k = gzip_tile_kind(p, lb, cls, f, I, J);
-      if (k >= 0) { p.tcol[n] = J; p.tkind[n] = (int8_t)k; ++n; }
+    for (int J0 = 0; J0 <= I; J0 += 32) {
+      const int J = J0 + lane;
+      const int k = J <= I ? gzip_tile_kind(p, lb, cls, f, I, J) : -1;
+      const uint32_t m = __ballot_sync(0xffffffffu, k >= 0);
+      if (k >= 0) {
+        p.tcol[n + __popc(m & below)] = J;
+        p.tkind[n + __popc(m & below)] = (int8_t)k;
+      }
+      n += __popc(m);
     }
   }
-  for (int J = threadIdx.x; J < T; J += blockDim.x) {
-    int cnt = 0;
-    for (int I = J; I < T; ++I) cnt += gzip_tile_kind(p, lb, cls, f, I, J) >= 0;
-    tcp[J + 1] = cnt;
-  }
-  if (threadIdx.x == 0) tcp[0] = (int32_t)(bc * p.tregion);
-  __syncthreads();
-  block_inclusive_scan(tcp + 1, T, (int32_t)(bc * p.tregion));
-  for (int J = threadIdx.x; J < T; J += blockDim.x) {
+  for (int J = warp; J < T; J += nwarps) {
     int n = tcp[J];
-    for (int I = J; I < T; ++I) {
-      const int k = gzip_tile_kind(p, lb, cls, f, I, J);
-      if (k >= 0) { p.trow[n] = I; p.tkind_t[n] = (int8_t)k; ++n; }
+    for (int I0 = J; I0 < T; I0 += 32) {
+      const int I = I0 + lane;
+      const int k = I < T ? gzip_tile_kind(p, lb, cls, f, I, J) : -1;
+      const uint32_t m = __ballot_sync(0xffffffffu, k >= 0);
+      if (k >= 0) {
+        p.trow[n + __popc(m & below)] = I;
+        p.tkind_t[n + __popc(m & below)] = (int8_t)k;
+      }
+      n += __popc(m);
     }
   }
 }
@@ -294,104 +311,122 @@ __device__ int gist_tile_kind(const GistBuild& p, int I, int J) {
   return (min_col >= kTile - p.tail) ? SA_TILE_TAIL : SA_TILE_MASKED;
 }
 
-__global__ void __launch_bounds__(1024) gist_build_kernel(GistBuild p) {
-  const int N = p.N, T = p.T;
-  const int nwords = (N + 31) / 32;
-  for (int k = threadIdx.x; k < nwords; k += blockDim.x) {
-    uint32_t word = 0;
-    for (int t = 0; t < 32; ++t) {
-      const int pos = k * 32 + t;
-      if (pos >= N) break;
-      bool g;
-      if (p.flags) g = p.flags[pos] != 0;
-      else g = pos >= p.sinks && ((pos - p.sinks) % (p.ratio + 1)) == p.ratio;
-      if (g) word |= 1u << t;
-    }
-    p.gist_bits[k] = word;
+// Gist bit of logical position pos (< N).
+__device__ __forceinline__ bool gist_at(const GistBuild& p, int pos) {
+  if (p.flags) return p.flags[pos] != 0;
+  return pos >= p.sinks && ((pos - p.sinks) % (p.ratio + 1)) == p.ratio;
+}
+
+// 1. One warp per 128-position tile J: its 4 gist-bit words, its part of the
+// shift permutation (raw tokens first, then gists, both in order), and its
+// count of keys visible to every later query (sinks and gists) in far_ptr[J + 1].
+__global__ void __launch_bounds__(256) gist_tile_kernel(GistBuild p) {
+  const int lane = threadIdx.x & 31, J = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (J >= p.T) return;
+  const int N = p.N, j0 = J * kTile, n = min(kTile, N - j0);
+  uint32_t gw[4];
+  int ng = 0, nf = 0;
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const int pos = j0 + c * 32 + lane;
+    const bool ok = pos < N;
+    const bool g = ok && gist_at(p, pos);
+    gw[c] = __ballot_sync(0xffffffffu, g);
+    nf += __popc(__ballot_sync(0xffffffffu, ok && (pos < p.sinks || g)));
+    ng += __popc(gw[c]);
+    if (lane == 0 && j0 + c * 32 < N) p.gist_bits[(j0 >> 5) + c] = gw[c];
   }
-  __syncthreads();
-  // shift permutation: one warp per tile
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-  for (int J = warp; J < T; J += nwarps) {
-    const int j0 = J * kTile, n = min(kTile, N - j0);
-    const int ng = count_gists(p.gist_bits, j0, j0 + n);
-    int before = 0;  // gists of this tile before the current 32-chunk
-    for (int c = 0; c < kTile / 32; ++c) {
-      const int off = c * 32 + lane, pos = j0 + off;
-      const uint32_t word = (j0 + c * 32 < N) ? p.gist_bits[(j0 >> 5) + c] : 0u;
-      const uint32_t valid = (n - c * 32 >= 32) ? 0xffffffffu
-                             : (n - c * 32 <= 0) ? 0u : ((1u << (n - c * 32)) - 1u);
-      const uint32_t gw = word & valid;
-      if (off < n) {
-        const int gb = before + __popc(gw & ((1u << lane) - 1u));
-        const bool g = (gw >> lane) & 1u;
-        const int phys = j0 + (g ? (n - ng) + gb : off - gb);
-        p.perm[phys] = pos;
-      }
-      before += __popc(gw);
+  int before = 0;  // gists of this tile before the current 32-chunk
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const int off = c * 32 + lane;
+    if (off < n) {
+      const int gb = before + __popc(gw[c] & ((1u << lane) - 1u));
+      const bool g = (gw[c] >> lane) & 1u;
+      p.perm[j0 + (g ? (n - ng) + gb : off - gb)] = j0 + off;
     }
-    // keys visible to every later query: sinks and gists of this tile
-    int nf = 0;
-    for (int c = 0; c < kTile / 32; ++c) {
-      const int pos = j0 + c * 32 + lane;
-      nf += __popc(__ballot_sync(0xffffffffu, pos < N && (pos < p.sinks || is_gist(p.gist_bits, pos))));
+    before += __popc(gw[c]);
+  }
+  if (lane == 0) p.far_ptr[J + 1] = nf;
+}
+
+// 2. One warp per query tile I (row counts) and per key tile J = I (column
+// counts) of the tile lists.
+__global__ void __launch_bounds__(256) gist_count_kernel(GistBuild p) {
+  const int lane = threadIdx.x & 31, X = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (X >= p.T) return;
+  int rows = 0, cols = 0;
+  for (int J0 = 0; J0 <= X; J0 += 32) {
+    const int J = J0 + lane;
+    rows += __popc(__ballot_sync(0xffffffffu, J <= X && gist_tile_kind(p, X, J) >= 0));
+  }
+  for (int I0 = X; I0 < p.T; I0 += 32) {
+    const int I = I0 + lane;
+    cols += __popc(__ballot_sync(0xffffffffu, I < p.T && gist_tile_kind(p, I, X) >= 0));
+  }
+  if (lane == 0) {
+    p.trp[X + 1] = rows;
+    p.tcp[X + 1] = cols;
+  }
+}
+
+// 3. Counts -> offsets (one CTA: T is at most 2^17).
+__global__ void __launch_bounds__(1024) gist_scan_kernel(GistBuild p) {
+  if (threadIdx.x == 0) {
+    p.trp[0] = 0;
+    p.tcp[0] = 0;
+    p.far_ptr[0] = 0;
+  }
+  block_inclusive_scan(p.trp + 1, p.T, 0);
+  block_inclusive_scan(p.tcp + 1, p.T, 0);
+  block_inclusive_scan(p.far_ptr + 1, p.T, 0);
+}
+
+// 4. One warp per tile: the row list of query tile X, the column list of key
+// tile X, and the physical index of every sink / gist of tile X at its
+// logical-order slot of far_idx.
+__global__ void __launch_bounds__(256) gist_fill_kernel(GistBuild p) {
+  const int lane = threadIdx.x & 31, X = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (X >= p.T) return;
+  const uint32_t below = (1u << lane) - 1u;
+  int n = p.trp[X];
+  for (int J0 = 0; J0 <= X; J0 += 32) {
+    const int J = J0 + lane;
+    const int k = J <= X ? gist_tile_kind(p, X, J) : -1;
+    const uint32_t m = __ballot_sync(0xffffffffu, k >= 0);
+    if (k >= 0) {
+      p.tcol[n + __popc(m & below)] = J;
+      p.tkind[n + __popc(m & below)] = (int8_t)k;
     }
-    if (lane == 0) p.far_ptr[J + 1] = nf;
+    n += __popc(m);
   }
-  if (threadIdx.x == 0) p.far_ptr[0] = 0;
-  __syncthreads();
-  block_inclusive_scan(p.far_ptr + 1, T, 0);
-  // far_idx: the physical index of every sink / gist, in logical order
-  for (int J = warp; J < T; J += nwarps) {
-    const int j0 = J * kTile, n = min(kTile, N - j0);
-    const int ng = count_gists(p.gist_bits, j0, j0 + n);
-    int f = p.far_ptr[J], gbefore = 0;
-    for (int c = 0; c < kTile / 32; ++c) {
-      const int off = c * 32 + lane, pos = j0 + off;
-      const bool ok = pos < N;
-      const bool g = ok && is_gist(p.gist_bits, pos);
-      const bool far = ok && (pos < p.sinks || g);
-      const uint32_t gmask = __ballot_sync(0xffffffffu, g);
-      const uint32_t fmask = __ballot_sync(0xffffffffu, far);
-      const uint32_t below = (1u << lane) - 1u;
-      if (far) {
-        const int gb = gbefore + __popc(gmask & below);
-        p.far_idx[f + __popc(fmask & below)] = j0 + (g ? (n - ng) + gb : off - gb);
-      }
-      f += __popc(fmask);
-      gbefore += __popc(gmask);
+  n = p.tcp[X];
+  for (int I0 = X; I0 < p.T; I0 += 32) {
+    const int I = I0 + lane;
+    const int k = I < p.T ? gist_tile_kind(p, I, X) : -1;
+    const uint32_t m = __ballot_sync(0xffffffffu, k >= 0);
+    if (k >= 0) {
+      p.trow[n + __popc(m & below)] = I;
+      p.tkind_t[n + __popc(m & below)] = (int8_t)k;
     }
+    n += __popc(m);
   }
-  __syncthreads();
-  for (int I = threadIdx.x; I < T; I += blockDim.x) {
-    int cnt = 0;
-    for (int J = 0; J <= I; ++J) cnt += gist_tile_kind(p, I, J) >= 0;
-    p.trp[I + 1] = cnt;
-  }
-  if (threadIdx.x == 0) p.trp[0] = 0;
-  __syncthreads();
-  block_inclusive_scan(p.trp + 1, T, 0);
-  for (int I = threadIdx.x; I < T; I += blockDim.x) {
-    int n = p.trp[I];
-    for (int J = 0; J <= I; ++J) {
-      const int k = gist_tile_kind(p, I, J);
-      if (k >= 0) { p.tcol[n] = J; p.tkind[n] = (int8_t)k; ++n; }
+  const int j0 = X * kTile, nt = min(kTile, p.N - j0);
+  const int ng = count_gists(p.gist_bits, j0, j0 + nt);
+  int f = p.far_ptr[X], gbefore = 0;
+  for (int c = 0; c < kTile / 32; ++c) {
+    const int off = c * 32 + lane, pos = j0 + off;
+    const bool ok = pos < p.N;
+    const bool g = ok && is_gist(p.gist_bits, pos);
+    const bool far = ok && (pos < p.sinks || g);
+    const uint32_t gmask = __ballot_sync(0xffffffffu, g);
+    const uint32_t fmask = __ballot_sync(0xffffffffu, far);
+    if (far) {
+      const int gb = gbefore + __popc(gmask & below);
+      p.far_idx[f + __popc(fmask & below)] = j0 + (g ? (nt - ng) + gb : off - gb);
     }
-  }
-  for (int J = threadIdx.x; J < T; J += blockDim.x) {
-    int cnt = 0;
-    for (int I = J; I < T; ++I) cnt += gist_tile_kind(p, I, J) >= 0;
-    p.tcp[J + 1] = cnt;
-  }
-  if (threadIdx.x == 0) p.tcp[0] = 0;
-  __syncthreads();
-  block_inclusive_scan(p.tcp + 1, T, 0);
-  for (int J = threadIdx.x; J < T; J += blockDim.x) {
-    int n = p.tcp[J];
-    for (int I = J; I < T; ++I) {
-      const int k = gist_tile_kind(p, I, J);
-      if (k >= 0) { p.trow[n] = I; p.tkind_t[n] = (int8_t)k; ++n; }
-    }
+    f += __popc(fmask);
+    gbefore += __popc(gmask);
   }
 }
 
@@ -439,7 +474,11 @@ cudaError_t launch_gist_build(const sa_mask_desc& d, const uint8_t* flags,
   p.far_ptr = L.far_ptr;
   p.trp = L.tile_row_ptr; p.tcol = L.tile_col; p.tkind = L.tile_kind;
   p.tcp = L.tile_col_ptr; p.trow = L.tile_row; p.tkind_t = L.tile_kind_t;
-  gist_build_kernel<<<1, 1024, 0, s>>>(p);
+  const unsigned grid = (unsigned)((p.T + 7) / 8);
+  gist_tile_kernel<<<grid, 256, 0, s>>>(p);
+  gist_count_kernel<<<grid, 256, 0, s>>>(p);
+  gist_scan_kernel<<<1, 1024, 0, s>>>(p);
+  gist_fill_kernel<<<grid, 256, 0, s>>>(p);
   return cudaGetLastError();
 }
 
