@@ -6,17 +6,27 @@
 // (the training use of the method: "UniGist ...", Approach, one-pass training;
 // forward/backward latency is a metric that page names).
 //
-// One CTA per (128-key tile J, KV head, sequence) walks the transposed tile
-// lists (every query tile I that visits J, for every query head of the KV
-// group). TMEM lanes are key rows:
-//   S^T = K_J Q_I^T and dP^T = V_J dO_I^T           (TMEM, 128 + 128 columns)
-//   four compute warps form P^T and dS^T rows (bf16, swizzled shared tiles)
-//   dV += P^T dO_I, dK += dS^T Q_I                   (TMEM accumulators)
-//   dQ_I = dS K_J (the dS^T tile read MN-major) into the S^T columns, then
-//   added to the fp32 dQ in global memory with vectorised reductions.
-// A preprocess kernel writes D and LSE * log2(e) into padded workspace rows so
-// that their 512-byte bulk copies never leave the buffer. All waits are
-// bounded (see sm100.cuh).
+// A work item is one (128-key tile J, KV head, sequence); its visits are every
+// query tile I that lists J, for every query head of the KV group (the
+// transposed tile lists). The kernel is persistent: one CTA per SM walks the
+// items blockIdx.x, blockIdx.x + gridDim.x, ... (early key tiles, which have
+// the longest lists, first). TMEM lanes are key rows:
+//   S^T = K_J Q_I^T (columns 0-127); each half h of the compute warps writes
+//     its bf16 P^T over the first 32 of its 64 S columns
+//   dP^T = V_J dO_I^T (columns 128-255), later reused for dQ_I = dS K_J
+//   dV += P^T dO_I (A = P^T from TMEM), dK += dS^T Q_I (TMEM accumulators)
+// dS^T goes to shared memory: it is the A operand of dK (key-major) and, read
+// query-major, of dQ. The dQ tile is read out of TMEM, its columns released,
+// and only then added to the fp32 dQ in global memory with vector reductions.
+//
+// Roles (352 threads): warp 0 TMA (K, V per item; Q, LSE, D double-buffered;
+// dO single-buffered), warp 1 one thread issuing tcgen05.mma, warps 2-9 two
+// groups of four compute warps (group h owns query columns [64h, 64h + 64) of
+// every tile; the backward needs no cross-column reduction since P comes from
+// the stored LSE), warp 10 the visit list and the visibility of each tile's
+// (key, query) pairs as 4 x 128 bit words in a shared-memory ring. Every wait
+// is bounded; on timeout the device status word is set and all roles leave
+// after draining their copies and MMAs.
 #include <cuda.h>
 
 #include "attn_mask.cuh"
@@ -35,23 +45,37 @@ struct BwdTcParams {
   int Tpad;            // T * 128
 };
 
+namespace bwd {
+
+constexpr int kSlots = 2;             // mask ring depth
+constexpr uint32_t kSlotBytes = 2048;  // [4 words][128 key rows]
+constexpr int kCompute = 256;          // compute threads
+constexpr int kThreads = 64 + kCompute + 32;
+constexpr int kMaskWarp = 10;
+
 template <int D>
-struct BwdLayout {
+struct Layout {
   static constexpr uint32_t kT = 128 * D * 2;     // a 128 x D bf16 tile
   static constexpr uint32_t kP = 128 * 128 * 2;   // a 128 x 128 bf16 tile
   static constexpr uint32_t kAtom = 128 * 128;    // [128 rows][64 bf16] swizzle atom
   static constexpr uint32_t k = 0;
   static constexpr uint32_t v = kT;
-  static constexpr uint32_t q = 2 * kT;
-  static constexpr uint32_t dO = 3 * kT;
-  static constexpr uint32_t pt = 4 * kT;          // P^T  [keys][queries]
-  static constexpr uint32_t dst = 4 * kT + kP;    // dS^T [keys][queries]
-  static constexpr uint32_t rowv = 4 * kT + 2 * kP;  // lse2[128], delta[128]
-  static constexpr uint32_t bars = rowv + 1024;
-  static constexpr uint32_t bytes = bars + 256 + 1024;
+  static constexpr uint32_t q = 2 * kT;           // 2 stages
+  static constexpr uint32_t dO = 4 * kT;
+  static constexpr uint32_t dst = 5 * kT;         // dS^T [keys][queries]
+  static constexpr uint32_t rowv = 5 * kT + kP;   // [2 stages][lse2 128 | delta 128] fp32
+  static constexpr uint32_t mask = rowv + 2 * 1024;
+  static constexpr uint32_t hdr = mask + kSlots * kSlotBytes;  // [slot] {h, I}
+  static constexpr uint32_t bars = hdr + 64;
+  static constexpr uint32_t bytes = bars + 512 + 1024;
 };
 
-enum { W_KV = 0, W_QF = 1, W_QE = 2, W_SF = 3, W_PF = 4, W_DQF = 5, W_DQE = 6, W_DRAIN = 7 };
+enum {
+  B_KVF = 0, B_KVE = 1, B_QF = 2, B_QE = 4, B_DOF = 6, B_DOE = 7, B_SF = 8, B_DPF = 9, B_PF = 10,
+  B_DQF = 11, B_DQE = 12, B_MF = 13, B_ME = 15, B_OF = 17, B_DRAIN = 18, kNumBars = 19
+};
+
+constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256;  // dK at 256 + D
 
 __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
   asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b),
@@ -68,39 +92,37 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
       : "memory");
 }
 
-template <int D>
-__global__ void __launch_bounds__(192, 1) bwd_tc_kernel(const __grid_constant__ BwdTcParams P) {
-  using L = BwdLayout<D>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-  const uint32_t sb = smem_u32(smem);
-  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + L::bars);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 16);
-  volatile int* abort = reinterpret_cast<volatile int*>(bar + 16) + 1;
-  float* s_lse2 = reinterpret_cast<float*>(smem + L::rowv);
-  float* s_delta = s_lse2 + 128;
+// Bits [0, n) set, n clamped to [0, 32].
+__device__ __forceinline__ uint32_t prefix_bits(int n) {
+  const int c = min(max(n, 0), 32);
+  return (uint32_t)((1ull << c) - 1ull);
+}
 
-  const AttnArgs& a = P.a;
-  const MaskArgs& m = P.m;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int T = m.T;
-  const int hb = a.Hkv * a.Bt;
-  const int J = (int)(blockIdx.x / hb);  // early key tiles (long lists) first
-  const int hk = (int)(blockIdx.x % hb) % a.Hkv, bt = (int)(blockIdx.x % hb) / a.Hkv;
-  const int rep = a.Hq / a.Hkv;
-  const int k0 = J * kTile;
-  DeviceStatus* st = a.status;
-
-  // total visits: every query tile that lists J, for every query head of the group
-  int n = 0;
-  for (int r = 0; r < rep; ++r) {
-    const int list = list_of(m, bt, hk * rep + r);
-    n += m.tcp[list * (T + 1) + J + 1] - m.tcp[list * (T + 1) + J];
+// Item -> (key tile J, KV head, sequence): early key tiles first.
+struct Item {
+  int J, hk, bt;
+  __device__ Item(int idx, int Hkv, int Bt) {
+    J = idx / (Hkv * Bt);
+    hk = (idx % (Hkv * Bt)) % Hkv;
+    bt = (idx % (Hkv * Bt)) / Hkv;
   }
-  auto entry = [&](int it, int& h, int& I, int& kind) {
+};
+
+// The visits of one item: query tile lists of every query head of the group.
+struct Visits {
+  int n;
+  __device__ void init(const MaskArgs& m, int bt, int hk, int rep, int J) {
+    n = 0;
     for (int r = 0; r < rep; ++r) {
       const int list = list_of(m, bt, hk * rep + r);
-      const int e0 = m.tcp[list * (T + 1) + J], cnt = m.tcp[list * (T + 1) + J + 1] - e0;
+      n += m.tcp[list * (m.T + 1) + J + 1] - m.tcp[list * (m.T + 1) + J];
+    }
+  }
+  __device__ static void entry(const MaskArgs& m, int bt, int hk, int rep, int J, int it, int& h,
+                               int& I, int& kind) {
+    for (int r = 0; r < rep; ++r) {
+      const int list = list_of(m, bt, hk * rep + r);
+      const int e0 = m.tcp[list * (m.T + 1) + J], cnt = m.tcp[list * (m.T + 1) + J + 1] - e0;
       if (it < cnt) {
         h = hk * rep + r;
         I = m.trow[e0 + it];
@@ -112,17 +134,81 @@ __global__ void __launch_bounds__(192, 1) bwd_tc_kernel(const __grid_constant__ 
     h = hk * rep;
     I = 0;
     kind = SA_TILE_MASKED;
-  };
+  }
+};
+
+// Visibility of query columns [32w, 32w + 32) of tile (I, J) from key row kq
+// ("Gzip-guided sparse attention ...", Core equations: the block mask, then the
+// causal cut q >= kq), with the key and query ranges cut at N.
+__device__ __forceinline__ uint32_t key_word(const MaskArgs& m, int list, int lb, int N, int kq,
+                                             int q0, int kind, int w) {
+  if (kq >= N) return 0u;
+  const int c0 = q0 + 32 * w;
+  const uint32_t in_range = prefix_bits(N - c0);
+  const uint32_t causal = ~prefix_bits(kq - c0);  // columns with q >= kq
+  if (kind == SA_TILE_FULL) return in_range & causal;
+  const int kb = kq / m.b;
+  const uint32_t* rows = m.bits + (int64_t)list * m.B * m.words;
+  uint32_t blk;
+  if (m.b >= kTile || lb >= 5) {
+    const int qb = min(m.B - 1, m.b >= kTile ? q0 / m.b : c0 >> lb);
+    blk = ((rows[(int64_t)qb * m.words + (kb >> 5)] >> (kb & 31)) & 1u) ? 0xffffffffu : 0u;
+  } else {
+    // 32 >> lb query blocks per word: one bit of each block row
+    const int nb = 32 >> lb, run = 1 << lb;
+    blk = 0u;
+    for (int t = 0; t < nb; ++t) {
+      const int qb = min(m.B - 1, (c0 >> lb) + t);
+      if ((rows[(int64_t)qb * m.words + (kb >> 5)] >> (kb & 31)) & 1u)
+        blk |= (uint32_t)((1ull << run) - 1ull) << (t * run);
+    }
+  }
+  return blk & in_range & causal;
+}
+
+}  // namespace bwd
+
+using namespace bwd;
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_constant__ BwdTcParams P) {
+  using L = Layout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  const uint32_t sb = smem_u32(smem);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + L::bars);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + kNumBars);
+  volatile int* abort = reinterpret_cast<volatile int*>(bar + kNumBars) + 1;
+  float* rowv = reinterpret_cast<float*>(smem + L::rowv);
+  uint32_t* mwords = reinterpret_cast<uint32_t*>(smem + L::mask);
+  int* hdr = reinterpret_cast<int*>(smem + L::hdr);
+
+  const AttnArgs& a = P.a;
+  const MaskArgs& m = P.m;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int T = m.T;
+  const int rep = a.Hq / a.Hkv;
+  const int n_items = T * a.Hkv * a.Bt;
+  DeviceStatus* st = a.status;
 
   if (threadIdx.x == 0) {
-    mbar_init(&bar[W_KV], 1);
-    mbar_init(&bar[W_QF], 1);
-    mbar_init(&bar[W_QE], 1);
-    mbar_init(&bar[W_SF], 1);
-    mbar_init(&bar[W_PF], 128);
-    mbar_init(&bar[W_DQF], 1);
-    mbar_init(&bar[W_DQE], 128);
-    mbar_init(&bar[W_DRAIN], 1);
+    mbar_init(&bar[B_KVF], 1);
+    mbar_init(&bar[B_KVE], 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bar[B_QF + s], 1);
+      mbar_init(&bar[B_QE + s], 1);
+      mbar_init(&bar[B_MF + s], 32);
+      mbar_init(&bar[B_ME + s], kCompute);
+    }
+    mbar_init(&bar[B_DOF], 1);
+    mbar_init(&bar[B_DOE], 1);
+    mbar_init(&bar[B_SF], 1);
+    mbar_init(&bar[B_DPF], 1);
+    mbar_init(&bar[B_PF], kCompute);
+    mbar_init(&bar[B_DQF], 1);
+    mbar_init(&bar[B_DQE], kCompute);
+    mbar_init(&bar[B_OF], kCompute);
+    mbar_init(&bar[B_DRAIN], 1);
     *abort = 0;
     fence_barrier_init();
   }
@@ -134,7 +220,6 @@ __global__ void __launch_bounds__(192, 1) bwd_tc_kernel(const __grid_constant__ 
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  constexpr uint32_t cS = 0, cDP = 128, cDV = 256, cDK = 256 + D;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -143,198 +228,324 @@ __global__ void __launch_bounds__(192, 1) bwd_tc_kernel(const __grid_constant__ 
       prefetch_tmap(&P.tmk);
       prefetch_tmap(&P.tmv);
       prefetch_tmap(&P.tmdo);
-      mbar_arrive_expect_tx(&bar[W_KV], 2 * L::kT);
-      for (int at = 0; at < D / 64; ++at) {
-        tma_load_4d(smem + L::k + at * L::kAtom, &P.tmk, &bar[W_KV], at * 64, hk, k0, bt);
-        tma_load_4d(smem + L::v + at * L::kAtom, &P.tmv, &bar[W_KV], at * 64, hk, k0, bt);
-      }
-      int issued = 0;
-      for (int it = 0; it < n; ++it) {
-        if (!mbar_wait(&bar[W_QE], (it & 1) ^ 1, abort, st, 101)) break;
-        int h, I, kind;
-        entry(it, h, I, kind);
-        mbar_arrive_expect_tx(&bar[W_QF], 2 * L::kT + 2 * 512);
+      int g = 0, k = 0, last_q = -1, last_do = -1, last_kv = -1;
+      bool ok = true;
+      for (int idx = blockIdx.x; ok && idx < n_items; idx += gridDim.x, ++k) {
+        const Item itm(idx, a.Hkv, a.Bt);
+        Visits vis;
+        vis.init(m, itm.bt, itm.hk, rep, itm.J);
+        // K and V of the previous item are no longer read
+        if (k > 0 && !mbar_wait(&bar[B_KVE], (k - 1) & 1, abort, st, 100)) break;
+        mbar_arrive_expect_tx(&bar[B_KVF], 2 * L::kT);
         for (int at = 0; at < D / 64; ++at) {
-          tma_load_4d(smem + L::q + at * L::kAtom, &P.tmq, &bar[W_QF], at * 64, h, I * kTile, bt);
-          tma_load_4d(smem + L::dO + at * L::kAtom, &P.tmdo, &bar[W_QF], at * 64, h, I * kTile, bt);
+          tma_load_4d(smem + L::k + at * L::kAtom, &P.tmk, &bar[B_KVF], at * 64, itm.hk,
+                      itm.J * kTile, itm.bt);
+          tma_load_4d(smem + L::v + at * L::kAtom, &P.tmv, &bar[B_KVF], at * 64, itm.hk,
+                      itm.J * kTile, itm.bt);
         }
-        const int64_t ro = ((int64_t)bt * a.Hq + h) * P.Tpad + (int64_t)I * kTile;
-        bulk_load(s_lse2, P.lse2 + ro, 512, &bar[W_QF]);
-        bulk_load(s_delta, P.delta + ro, 512, &bar[W_QF]);
-        issued = it + 1;
+        last_kv = k;
+        for (int it = 0; it < vis.n; ++it) {
+          const int gt = g + it, s = gt & 1;
+          int h, I, kind;
+          Visits::entry(m, itm.bt, itm.hk, rep, itm.J, it, h, I, kind);
+          if (!mbar_wait(&bar[B_QE + s], ((gt >> 1) & 1) ^ 1, abort, st, 101)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&bar[B_QF + s], L::kT + 2 * 512);
+          for (int at = 0; at < D / 64; ++at)
+            tma_load_4d(smem + L::q + s * L::kT + at * L::kAtom, &P.tmq, &bar[B_QF + s], at * 64,
+                        h, I * kTile, itm.bt);
+          const int64_t ro = ((int64_t)itm.bt * a.Hq + h) * P.Tpad + (int64_t)I * kTile;
+          bulk_load(rowv + s * 256, P.lse2 + ro, 512, &bar[B_QF + s]);
+          bulk_load(rowv + s * 256 + 128, P.delta + ro, 512, &bar[B_QF + s]);
+          last_q = gt;
+          if (!mbar_wait(&bar[B_DOE], (gt & 1) ^ 1, abort, st, 102)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&bar[B_DOF], L::kT);
+          for (int at = 0; at < D / 64; ++at)
+            tma_load_4d(smem + L::dO + at * L::kAtom, &P.tmdo, &bar[B_DOF], at * 64, h, I * kTile,
+                        itm.bt);
+          last_do = gt;
+        }
+        g += vis.n;
       }
+      // every copy this CTA started must land before the CTA may exit
       volatile int no_abort = 0;
-      mbar_wait(&bar[W_KV], 0, &no_abort, nullptr, 102);
-      if (issued > 0) mbar_wait(&bar[W_QF], (issued - 1) & 1, &no_abort, nullptr, 103);
+      if (last_kv >= 0) mbar_wait(&bar[B_KVF], last_kv & 1, &no_abort, nullptr, 103);
+      for (int s = 0; s < 2; ++s)
+        if (last_q >= s) {
+          const int gs = last_q - ((last_q - s) & 1);
+          mbar_wait(&bar[B_QF + s], (gs >> 1) & 1, &no_abort, nullptr, 104);
+        }
+      if (last_do >= 0) mbar_wait(&bar[B_DOF], last_do & 1, &no_abort, nullptr, 105);
     }
   } else if (warp == 1) {
     if (lane == 0) {
       // ---------------------------------------------------------- MMA issuer
       constexpr uint32_t kIdS = idesc_bf16_f32(128, 128, false, false);
-      constexpr uint32_t kIdAcc = idesc_bf16_f32(128, D, false, true);   // P^T dO, dS^T Q
-      constexpr uint32_t kIdDq = idesc_bf16_f32(128, D, true, true);     // (dS^T)^T K
-      bool ok = mbar_wait(&bar[W_KV], 0, abort, st, 110);
-      for (int it = 0; ok && it < n; ++it) {
-        if (!mbar_wait(&bar[W_QF], it & 1, abort, st, 111)) break;
-        // the S^T columns hold the previous dQ until it has been read out
-        if (!mbar_wait(&bar[W_DQE], (it & 1) ^ 1, abort, st, 112)) break;
-        tc_fence_after();
+      constexpr uint32_t kIdAcc = idesc_bf16_f32(128, D, false, true);  // P^T dO, dS^T Q
+      constexpr uint32_t kIdDq = idesc_bf16_f32(128, D, true, true);    // (dS^T)^T K
+      int g = 0, k = 0;
+      bool ok = true;
+      for (int idx = blockIdx.x; ok && idx < n_items; idx += gridDim.x, ++k) {
+        const Item itm(idx, a.Hkv, a.Bt);
+        Visits vis;
+        vis.init(m, itm.bt, itm.hk, rep, itm.J);
+        if (vis.n > 0 && !mbar_wait(&bar[B_KVF], k & 1, abort, st, 110)) break;
+        for (int it = 0; it < vis.n; ++it) {
+          const int gt = g + it, s = gt & 1;
+          // S^T = K Q^T (the S columns last held P^T(gt - 1), read by a P V
+          // issued before this MMA: tcgen05.mma ops of one thread run in order)
+          if (!mbar_wait(&bar[B_QF + s], (gt >> 1) & 1, abort, st, 111)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t qb = sb + L::q + s * L::kT;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * L::kAtom + (kk & 3) * 32;
-          mma_bf16(tmem + cS, smem_desc_sw128(sb + L::k + off, 16, 1024),
-                   smem_desc_sw128(sb + L::q + off, 16, 1024), kIdS, kk > 0);
-          mma_bf16(tmem + cDP, smem_desc_sw128(sb + L::v + off, 16, 1024),
-                   smem_desc_sw128(sb + L::dO + off, 16, 1024), kIdS, kk > 0);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * L::kAtom + (kk & 3) * 32;
+            mma_bf16(tmem + kColS, smem_desc_sw128(sb + L::k + off, 16, 1024),
+                     smem_desc_sw128(qb + off, 16, 1024), kIdS, kk > 0);
+          }
+          mma_commit(&bar[B_SF]);
+          // dP^T = V dO^T into the columns the previous dQ has left
+          if (!mbar_wait(&bar[B_DOF], gt & 1, abort, st, 112) ||
+              (gt > 0 && !mbar_wait(&bar[B_DQE], (gt - 1) & 1, abort, st, 113))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * L::kAtom + (kk & 3) * 32;
+            mma_bf16(tmem + kColDP, smem_desc_sw128(sb + L::v + off, 16, 1024),
+                     smem_desc_sw128(sb + L::dO + off, 16, 1024), kIdS, kk > 0);
+          }
+          mma_commit(&bar[B_DPF]);
+          // P^T (TMEM) and dS^T (shared memory) of both halves are written
+          if (!mbar_wait(&bar[B_PF], gt & 1, abort, st, 114) ||
+              (it == 0 && k > 0 && !mbar_wait(&bar[B_OF], (k - 1) & 1, abort, st, 115))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {  // K = 128 queries
+            const uint32_t pa = tmem + kColS + (kk >> 2) * 64 + (kk & 3) * 8;
+            mma_bf16_ts(tmem + kColDV, pa, smem_desc_sw128(sb + L::dO + kk * 2048, L::kAtom, 1024),
+                        kIdAcc, (it > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(&bar[B_DOE]);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t aoff = (kk >> 2) * L::kAtom + (kk & 3) * 32;
+            mma_bf16(tmem + kColDV + D, smem_desc_sw128(sb + L::dst + aoff, 16, 1024),
+                     smem_desc_sw128(qb + kk * 2048, L::kAtom, 1024), kIdAcc,
+                     (it > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(&bar[B_QE + s]);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)  // K = 128 keys; A = dS^T read query-major
+            mma_bf16(tmem + kColDP, smem_desc_sw128(sb + L::dst + kk * 2048, L::kAtom, 1024),
+                     smem_desc_sw128(sb + L::k + kk * 2048, L::kAtom, 1024), kIdDq, kk > 0);
+          mma_commit(&bar[B_DQF]);
         }
-        mma_commit(&bar[W_SF]);
-        if (!mbar_wait(&bar[W_PF], it & 1, abort, st, 113)) break;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {  // K = 128 queries
-          const uint32_t aoff = (kk >> 2) * L::kAtom + (kk & 3) * 32;
-          mma_bf16(tmem + cDV, smem_desc_sw128(sb + L::pt + aoff, 16, 1024),
-                   smem_desc_sw128(sb + L::dO + kk * 2048, L::kAtom, 1024), kIdAcc,
-                   (it > 0 || kk > 0) ? 1u : 0u);
-          mma_bf16(tmem + cDK, smem_desc_sw128(sb + L::dst + aoff, 16, 1024),
-                   smem_desc_sw128(sb + L::q + kk * 2048, L::kAtom, 1024), kIdAcc,
-                   (it > 0 || kk > 0) ? 1u : 0u);
-        }
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)  // K = 128 keys; A = dS^T read query-major
-          mma_bf16(tmem + cS, smem_desc_sw128(sb + L::dst + kk * 2048, L::kAtom, 1024),
-                   smem_desc_sw128(sb + L::k + kk * 2048, L::kAtom, 1024), kIdDq, kk > 0);
-        mma_commit(&bar[W_DQF]);
-        mma_commit(&bar[W_QE]);
+        if (!ok) break;
+        mma_commit(&bar[B_KVE]);  // every MMA of this item reading K and V is issued
+        g += vis.n;
       }
-      mma_commit(&bar[W_DRAIN]);
+      mma_commit(&bar[B_DRAIN]);
       volatile int no_abort = 0;
-      mbar_wait(&bar[W_DRAIN], 0, &no_abort, nullptr, 114);
+      mbar_wait(&bar[B_DRAIN], 0, &no_abort, nullptr, 116);
     }
-  } else {
-    // ------------------------------------------------------- compute warps
-    const int quarter = warp & 3;
-    const int j = quarter * 32 + lane;  // key row of the tile = TMEM lane
-    const int kq = k0 + j;
+  } else if (warp == kMaskWarp) {
+    // ------------------------------------------------- visits and their masks
+    const int lb = m.b < kTile ? __ffs(m.b) - 1 : 0;  // b < 128 is a power of two
+    int g = 0;
+    for (int idx = blockIdx.x; idx < n_items; idx += gridDim.x) {
+      const Item itm(idx, a.Hkv, a.Bt);
+      Visits vis;
+      vis.init(m, itm.bt, itm.hk, rep, itm.J);
+      bool ok = true;
+      for (int it = 0; it < vis.n; ++it) {
+        const int gt = g + it, s = gt & 1;
+        if (!__all_sync(0xffffffffu, mbar_wait(&bar[B_ME + s], ((gt >> 1) & 1) ^ 1, abort, st, 130))) {
+          ok = false;
+          break;
+        }
+        int h, I, kind;
+        Visits::entry(m, itm.bt, itm.hk, rep, itm.J, it, h, I, kind);
+        const int list = list_of(m, itm.bt, h);
+        if (lane == 0) {
+          hdr[2 * s] = h;
+          hdr[2 * s + 1] = I;
+        }
+        uint32_t* words = mwords + s * (kSlotBytes / 4);
+        const int q0 = I * kTile;
+        if (kind != SA_TILE_FULL && (m.b >= kTile || lb >= 5)) {
+          // one block bit per (key row, word): every load first, then the words
+          uint32_t u[4][4];
+          int qb[4];
+#pragma unroll
+          for (int w = 0; w < 4; ++w)
+            qb[w] = min(m.B - 1, m.b >= kTile ? q0 / m.b : (q0 + 32 * w) >> lb);
+          const uint32_t* rows = m.bits + (int64_t)list * m.B * m.words;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int kb = min(a.N - 1, itm.J * kTile + lane + 32 * i) / m.b;
+#pragma unroll
+            for (int w = 0; w < 4; ++w) u[i][w] = rows[(int64_t)qb[w] * m.words + (kb >> 5)];
+          }
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int kq = itm.J * kTile + lane + 32 * i;
+            const int kb = min(a.N - 1, kq) / m.b;
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+              const int c0 = q0 + 32 * w;
+              const uint32_t v = kq < a.N ? prefix_bits(a.N - c0) & ~prefix_bits(kq - c0) : 0u;
+              words[w * 128 + lane + 32 * i] = ((u[i][w] >> (kb & 31)) & 1u) ? v : 0u;
+            }
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int w = 0; w < 4; ++w)
+              words[w * 128 + lane + 32 * i] =
+                  key_word(m, list, lb, a.N, itm.J * kTile + lane + 32 * i, q0, kind, w);
+        }
+        mbar_arrive(&bar[B_MF + s]);  // release: header and words are visible to the waiter
+      }
+      if (!ok) break;
+      g += vis.n;
+    }
+  } else if (warp >= 2 && warp < 2 + kCompute / 32) {
+    // -------------------------------------------------------- compute warps
+    const int half = (warp - 2) >> 2;
+    const int quarter = warp & 3;  // TMEM lane quarter of this warp
+    const int r = quarter * 32 + lane;
     const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
     const float sl2 = a.scale * 1.4426950408889634f;
-    const bool key_ok = kq < a.N;
-    const int lb = m.b < kTile ? __ffs(m.b) - 1 : 0;
+    int g = 0, k = 0;
     bool ok = true;
-    for (int it = 0; it < n; ++it) {
-      int h, I, kind;
-      entry(it, h, I, kind);
-      const int list = list_of(m, bt, h);
-      if (!__all_sync(0xffffffffu, mbar_wait(&bar[W_SF], it & 1, abort, st, 120))) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      // row-block bits of this key over the query tile (gzip, masked tiles)
-      const int q0 = I * kTile;
-      uint32_t qbits = 0xffffffffu;  // bit g: query block g of the tile sees this key's block
-      if (kind != SA_TILE_FULL && m.b < kTile && key_ok) {
-        const int kb = kq >> lb, nqb = kTile >> lb;
-        qbits = 0;
-        for (int g = 0; g < nqb && g < 32; ++g) {
-          const int qb = (q0 >> lb) + g;
-          if (qb < m.B) {
-            const uint32_t* row = m.bits + ((int64_t)list * m.B + qb) * m.words;
-            qbits |= ((row[kb >> 5] >> (kb & 31)) & 1u) << g;
-          }
+    for (int idx = blockIdx.x; ok && idx < n_items; idx += gridDim.x, ++k) {
+      const Item itm(idx, a.Hkv, a.Bt);
+      Visits vis;
+      vis.init(m, itm.bt, itm.hk, rep, itm.J);
+      const int kq = itm.J * kTile + r;  // this thread's key row
+      for (int it = 0; it < vis.n; ++it) {
+        const int gt = g + it, s = gt & 1;
+        if (!__all_sync(0xffffffffu, mbar_wait(&bar[B_SF], gt & 1, abort, st, 120) &&
+                                         mbar_wait(&bar[B_MF + s], (gt >> 1) & 1, abort, st, 121) &&
+                                         mbar_wait(&bar[B_DPF], gt & 1, abort, st, 122))) {
+          ok = false;
+          break;
         }
-      }
-      uint32_t pk[64], dk[64];
-      __syncwarp();  // the TMEM loads below are warp-collective (.sync.aligned)
+        const uint32_t* words = mwords + s * (kSlotBytes / 4);
+        const uint32_t mw[2] = {words[(2 * half) * 128 + r], words[(2 * half + 1) * 128 + r]};
+        const int h = hdr[2 * s], I = hdr[2 * s + 1];
+        mbar_arrive(&bar[B_ME + s]);
+        const float* lse2 = rowv + s * 256 + half * 64;
+        const float* dlt = lse2 + 128;
+        tc_fence_after();
+        __syncwarp();  // the TMEM loads below are warp-collective (.sync.aligned)
+        uint32_t pk[32];
 #pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) {
-        float sv[32], dv[32];
-        tmem_ld32(lane_addr + cS + c4 * 32, sv);
-        tmem_ld32(lane_addr + cDP + c4 * 32, dv);
-        tmem_wait_ld();
+        for (int c2 = 0; c2 < 2; ++c2) {  // 32 query columns at a time
+          float sv[32], dv[32];
+          tmem_ld32(lane_addr + kColS + half * 64 + c2 * 32, sv);
+          tmem_ld32(lane_addr + kColDP + half * 64 + c2 * 32, dv);
+          tmem_wait_ld();
+          uint32_t dk[16];
 #pragma unroll
-        for (int c = 0; c < 32; c += 2) {
-          float pv[2], ds[2];
+          for (int c = 0; c < 32; c += 2) {
+            float pv[2], ds[2];
 #pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int i = c4 * 32 + c + u;
-            bool vis = key_ok;
-            if (kind != SA_TILE_FULL) {
-              vis = vis && kq <= q0 + i;
-              if (m.b < kTile) vis = vis && ((qbits >> (i >> lb)) & 1u);
+            for (int u = 0; u < 2; ++u) {
+              const int i = c2 * 32 + c + u;
+              const bool v = (mw[c2] >> (c + u)) & 1u;
+              const float p = v ? ex2(fmaf(sv[c + u], sl2, -lse2[i])) : 0.f;
+              pv[u] = p;
+              ds[u] = p * (dv[c + u] - dlt[i]);
             }
-            const float p = vis ? ex2(fmaf(sv[c + u], sl2, -s_lse2[i])) : 0.f;
-            pv[u] = p;
-            ds[u] = p * (dv[c + u] - s_delta[i]);
+            pk[(c2 * 32 + c) >> 1] = pack_bf16(pv[0], pv[1]);
+            dk[c >> 1] = pack_bf16(ds[0], ds[1]);
           }
-          pk[(c4 * 32 + c) >> 1] = pack_bf16(pv[0], pv[1]);
-          dk[(c4 * 32 + c) >> 1] = pack_bf16(ds[0], ds[1]);
+          // dS^T: key row r, query columns 64 half + 32 c2 + [0, 32)
+          const uint32_t base = sb + L::dst + half * L::kAtom;
+#pragma unroll
+          for (int ch = 0; ch < 4; ++ch)
+            st_shared_v4(base + sw128_offset(r, c2 * 32 + ch * 8), dk[ch * 4], dk[ch * 4 + 1],
+                         dk[ch * 4 + 2], dk[ch * 4 + 3]);
+        }
+        // P^T (bf16 pairs) over the first 32 of this half's S columns, all read
+        __syncwarp();
+        tmem_st32(lane_addr + kColS + half * 64, reinterpret_cast<const float*>(pk));
+        tmem_wait_st();
+        fence_async_shared();
+        tc_fence_before();
+        mbar_arrive(&bar[B_PF]);
+        // dQ_I: TMEM lane = query row, this half's D / 2 columns; released
+        // before the reductions are issued
+        if (!__all_sync(0xffffffffu, mbar_wait(&bar[B_DQF], gt & 1, abort, st, 123))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        __syncwarp();
+        float dq[D / 2];
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c) tmem_ld32(lane_addr + kColDP + half * (D / 2) + c * 32, dq + c * 32);
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(&bar[B_DQE]);
+        const int q = I * kTile + r;
+        if (q < a.N) {
+          float* dst = a.dq + (((int64_t)itm.bt * a.N + q) * a.Hq + h) * D + half * (D / 2);
+#pragma unroll
+          for (int c = 0; c < D / 2; c += 4)
+            red_add_v4(dst + c, dq[c] * a.scale, dq[c + 1] * a.scale, dq[c + 2] * a.scale,
+                       dq[c + 3] * a.scale);
         }
       }
+      if (!ok) break;
+      // ------------------------------------------------------------ epilogue
+      // dK and dV of this key tile and KV head (the last dQ commit of the item
+      // followed every dV / dK MMA); fp32, this half's D / 2 columns
+      float* dkr = a.dk + (((int64_t)itm.bt * a.N + kq) * a.Hkv + itm.hk) * D + half * (D / 2);
+      float* dvr = a.dv + (((int64_t)itm.bt * a.N + kq) * a.Hkv + itm.hk) * D + half * (D / 2);
+      if (vis.n > 0) {
+        tc_fence_after();
+        __syncwarp();
 #pragma unroll
-      for (int ch = 0; ch < 16; ++ch) {  // rows = keys, 128 query columns
-        const int col = ch * 8;
-        const uint32_t off = (col >> 6) * L::kAtom + sw128_offset(j, col & 63);
-        st_shared_v4(sb + L::pt + off, pk[ch * 4], pk[ch * 4 + 1], pk[ch * 4 + 2], pk[ch * 4 + 3]);
-        st_shared_v4(sb + L::dst + off, dk[ch * 4], dk[ch * 4 + 1], dk[ch * 4 + 2], dk[ch * 4 + 3]);
-      }
-      fence_async_shared();
-      tc_fence_before();
-      mbar_arrive(&bar[W_PF]);
-      // dQ tile: TMEM lane = query row of tile I
-      if (!__all_sync(0xffffffffu, mbar_wait(&bar[W_DQF], it & 1, abort, st, 121))) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      __syncwarp();
-      const int qrow = q0 + j;
-      float* dq = a.dq + (((int64_t)bt * a.N + qrow) * a.Hq + h) * D;
+        for (int c4 = 0; c4 < D / 64; ++c4) {
+          float x[32], y[32];
+          tmem_ld32(lane_addr + kColDV + D + half * (D / 2) + c4 * 32, x);
+          tmem_ld32(lane_addr + kColDV + half * (D / 2) + c4 * 32, y);
+          tmem_wait_ld();
+          if (kq < a.N) {
 #pragma unroll
-      for (int c4 = 0; c4 < D / 32; ++c4) {
-        float o[32];
-        tmem_ld32(lane_addr + cS + c4 * 32, o);
-        tmem_wait_ld();
-        if (qrow < a.N) {
-#pragma unroll
-          for (int v = 0; v < 32; v += 4)
-            red_add_v4(dq + c4 * 32 + v, o[v] * a.scale, o[v + 1] * a.scale, o[v + 2] * a.scale,
-                       o[v + 3] * a.scale);
-        }
-      }
-      tc_fence_before();
-      mbar_arrive(&bar[W_DQE]);
-    }
-    // ------------------------------------------------------------- epilogue
-    if (ok && n > 0) {
-      // the last dQ commit follows every dV / dK MMA
-      tc_fence_after();
-      __syncwarp();
-      float* dkr = a.dk + (((int64_t)bt * a.N + kq) * a.Hkv + hk) * D;
-      float* dvr = a.dv + (((int64_t)bt * a.N + kq) * a.Hkv + hk) * D;
-#pragma unroll
-      for (int c4 = 0; c4 < D / 32; ++c4) {
-        float x[32], y[32];
-        tmem_ld32(lane_addr + cDK + c4 * 32, x);
-        tmem_ld32(lane_addr + cDV + c4 * 32, y);
-        tmem_wait_ld();
-        if (key_ok) {
-#pragma unroll
-          for (int v = 0; v < 32; v += 4) {
-            *reinterpret_cast<float4*>(dkr + c4 * 32 + v) =
-                make_float4(x[v] * a.scale, x[v + 1] * a.scale, x[v + 2] * a.scale, x[v + 3] * a.scale);
-            *reinterpret_cast<float4*>(dvr + c4 * 32 + v) = make_float4(y[v], y[v + 1], y[v + 2], y[v + 3]);
+            for (int v = 0; v < 32; v += 4) {
+              *reinterpret_cast<float4*>(dkr + c4 * 32 + v) =
+                  make_float4(x[v] * a.scale, x[v + 1] * a.scale, x[v + 2] * a.scale, x[v + 3] * a.scale);
+              *reinterpret_cast<float4*>(dvr + c4 * 32 + v) = make_float4(y[v], y[v + 1], y[v + 2], y[v + 3]);
+            }
           }
         }
+      } else if (kq < a.N) {  // no query tile visits this key tile: zero gradients
+        for (int c = 0; c < D / 2; c += 4) {
+          *reinterpret_cast<float4*>(dkr + c) = make_float4(0.f, 0.f, 0.f, 0.f);
+          *reinterpret_cast<float4*>(dvr + c) = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
       }
-    } else if (ok && key_ok) {
-      // no query tile visits this key tile: its gradients are zero
-      float* dkr = a.dk + (((int64_t)bt * a.N + kq) * a.Hkv + hk) * D;
-      float* dvr = a.dv + (((int64_t)bt * a.N + kq) * a.Hkv + hk) * D;
-      for (int c = 0; c < D; c += 4) {
-        *reinterpret_cast<float4*>(dkr + c) = make_float4(0.f, 0.f, 0.f, 0.f);
-        *reinterpret_cast<float4*>(dvr + c) = make_float4(0.f, 0.f, 0.f, 0.f);
-      }
+      tc_fence_before();
+      mbar_arrive(&bar[B_OF]);  // dV and dK may be overwritten by the next item
+      g += vis.n;
     }
   }
   tc_fence_before();
@@ -344,26 +555,37 @@ __global__ void __launch_bounds__(192, 1) bwd_tc_kernel(const __grid_constant__ 
 }
 
 // D = rowsum(dO * O) and LSE * log2(e), into padded [Bt, Hq, T*128] rows
-// (+inf LSE and zero D past the end of the sequence); one warp per row.
+// (+inf LSE and zero D past the end of the sequence). D / 8 lanes per row,
+// one 16-byte load of O and of dO each.
 template <int D>
-__global__ void bwd_tc_prep_kernel(AttnArgs a, float* lse2, float* delta, int Tpad) {
-  const int64_t wid = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (wid >= (int64_t)a.Bt * a.Hq * Tpad) return;
-  const int p = wid % Tpad, h = (wid / Tpad) % a.Hq, bt = wid / ((int64_t)Tpad * a.Hq);
+__global__ void __launch_bounds__(256) bwd_tc_prep_kernel(AttnArgs a, float* lse2, float* delta,
+                                                          int Tpad) {
+  constexpr int kLanes = D / 8, kRowsPerWarp = 32 / kLanes;
+  const int lane = threadIdx.x & 31, sub = lane / kLanes, l = lane % kLanes;
+  const int64_t row = ((int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * kRowsPerWarp + sub;
+  const int64_t rows = (int64_t)a.Bt * a.Hq * Tpad;
+  const bool live = row < rows;
+  const int p = live ? (int)(row % Tpad) : 0;
+  const int h = live ? (int)((row / Tpad) % a.Hq) : 0;
+  const int bt = live ? (int)(row / ((int64_t)Tpad * a.Hq)) : 0;
   float s = 0.f;
-  if (p < a.N) {
-    const __nv_bfloat16* o = reinterpret_cast<const __nv_bfloat16*>(a.o) + bt * a.os[0] +
-                             (int64_t)p * a.os[1] + (int64_t)h * a.os[2];
-    const __nv_bfloat16* d = reinterpret_cast<const __nv_bfloat16*>(a.dout) + bt * a.os[0] +
-                             (int64_t)p * a.os[1] + (int64_t)h * a.os[2];
-    for (int c = lane; c < D; c += 32) s += __bfloat162float(o[c]) * __bfloat162float(d[c]);
+  if (live && p < a.N) {
+    const int64_t off = bt * a.os[0] + (int64_t)p * a.os[1] + (int64_t)h * a.os[2] + l * 8;
+    const uint4 ov = *reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(a.o) + off);
+    const uint4 dv = *reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(a.dout) + off);
+    const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&ov);
+    const __nv_bfloat162* d2 = reinterpret_cast<const __nv_bfloat162*>(&dv);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 x = __bfloat1622float2(o2[i]), y = __bfloat1622float2(d2[i]);
+      s = fmaf(x.x, y.x, fmaf(x.y, y.y, s));
+    }
   }
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-  if (lane == 0) {
-    delta[wid] = s;
-    lse2[wid] = p < a.N ? a.lse[((int64_t)bt * a.Hq + h) * a.N + p] * 1.4426950408889634f
+  for (int off = kLanes / 2; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+  if (live && l == 0) {
+    delta[row] = s;
+    lse2[row] = p < a.N ? a.lse[((int64_t)bt * a.Hq + h) * a.N + p] * 1.4426950408889634f
                         : INFINITY;
   }
 }
@@ -371,6 +593,7 @@ __global__ void bwd_tc_prep_kernel(AttnArgs a, float* lse2, float* delta, int Tp
 // [Bt, N, H, d] bf16 with element strides {batch, seq, head}; box 64 x 1 x 128 x 1.
 bool make_tile_map(CUtensorMap* map, const void* base, int d, int H, int N, int Bt,
                    const int64_t* s);
+int sm_count();
 
 template <int D>
 static cudaError_t bwd_tc_launch(const AttnArgs& a, const MaskArgs& m, void* ws, cudaStream_t s) {
@@ -389,15 +612,20 @@ static cudaError_t bwd_tc_launch(const AttnArgs& a, const MaskArgs& m, void* ws,
   P.lse2 = lse2;
   P.delta = delta;
   const int64_t rows = (int64_t)a.Bt * a.Hq * P.Tpad;
-  bwd_tc_prep_kernel<D><<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(a, lse2, delta, P.Tpad);
+  const int64_t rows_per_block = 8 * (32 / (D / 8));
+  bwd_tc_prep_kernel<D><<<(unsigned)((rows + rows_per_block - 1) / rows_per_block), 256, 0, s>>>(
+      a, lse2, delta, P.Tpad);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   e = cudaMemsetAsync(a.dq, 0, (size_t)a.Bt * a.N * a.Hq * D * sizeof(float), s);
   if (e != cudaSuccess) return e;
-  const int bytes = (int)BwdLayout<D>::bytes;
+  const int bytes = (int)Layout<D>::bytes;
   e = cudaFuncSetAttribute(bwd_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   if (e != cudaSuccess) return e;
-  bwd_tc_kernel<D><<<dim3(m.T * a.Hkv * a.Bt), 192, bytes, s>>>(P);
+  // persistent: one CTA per SM (TMEM and shared memory admit one)
+  const int items = m.T * a.Hkv * a.Bt;
+  const int grid = items < sm_count() ? items : sm_count();
+  bwd_tc_kernel<D><<<dim3(grid), kThreads, bytes, s>>>(P);
   return cudaGetLastError();
 }
 

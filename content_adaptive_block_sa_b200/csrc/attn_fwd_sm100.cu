@@ -788,7 +788,7 @@ __global__ void __launch_bounds__(256) gist_gather_kernel(AttnArgs a, MaskArgs m
 }
 
 // Streaming multiprocessors of the current device (cached per device).
-static int sm_count() {
+int sm_count() {
   static int cached[64] = {0};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
