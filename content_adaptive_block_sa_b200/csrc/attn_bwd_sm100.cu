@@ -38,6 +38,7 @@ using namespace sm100;
 
 struct BwdTcParams {
   CUtensorMap tmq, tmk, tmv, tmdo;
+  CUtensorMap tmdq;    // fp32 dQ [Bt, N, Hq, D], box 32 x 1 x 128 x 1, 128-byte swizzle
   AttnArgs a;
   MaskArgs m;
   const float* lse2;   // [Bt, Hq, Tpad] LSE * log2(e), +inf past N
@@ -70,18 +71,21 @@ struct Layout {
   static constexpr uint32_t bytes = bars + 512 + 1024;
 };
 
+// mbarriers. KVF/KVE: K, V of the item loaded / no longer read. QF/QE: Q
+// stage (with its LSE and D rows) full / free. DOF/DOE: dO full / free. SF,
+// DPF: S^T, dP^T in TMEM. PF1: P^T written to TMEM; PF2: dS^T written to
+// shared memory. DQF/DQE: dQ in TMEM / read out. MF/ME: mask slot full /
+// read. OF: dV and dK of the item read out. HS: one compute half has staged
+// its dQ columns for the bulk reduction. DRAIN: all MMAs done.
+// QE takes two arrivals (dK done; the dQ staged in that Q stage read by the
+// bulk reduction), DQE two (each half's staging read).
 enum {
-  B_KVF = 0, B_KVE = 1, B_QF = 2, B_QE = 4, B_DOF = 6, B_DOE = 7, B_SF = 8, B_DPF = 9, B_PF = 10,
-  B_DQF = 11, B_DQE = 12, B_MF = 13, B_ME = 15, B_OF = 17, B_DRAIN = 18, kNumBars = 19
+  B_KVF = 0, B_KVE = 1, B_QF = 2, B_QE = 4, B_DOF = 6, B_DOE = 7, B_SF = 8, B_DPF = 9, B_PF1 = 10,
+  B_PF2 = 11, B_DQF = 12, B_DQE = 13, B_MF = 14, B_ME = 16, B_OF = 18, B_HS = 19, B_DRAIN = 21,
+  kNumBars = 22
 };
 
 constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256;  // dK at 256 + D
-
-__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b),
-               "f"(c), "f"(d)
-               : "memory");
-}
 
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
                                           uint64_t* bar) {
@@ -196,7 +200,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
     mbar_init(&bar[B_KVE], 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bar[B_QF + s], 1);
-      mbar_init(&bar[B_QE + s], 1);
+      mbar_init(&bar[B_QE + s], 2);
+      mbar_init(&bar[B_HS + s], kCompute / 2);
       mbar_init(&bar[B_MF + s], 32);
       mbar_init(&bar[B_ME + s], kCompute);
     }
@@ -204,9 +209,10 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
     mbar_init(&bar[B_DOE], 1);
     mbar_init(&bar[B_SF], 1);
     mbar_init(&bar[B_DPF], 1);
-    mbar_init(&bar[B_PF], kCompute);
+    mbar_init(&bar[B_PF1], kCompute);
+    mbar_init(&bar[B_PF2], kCompute);
     mbar_init(&bar[B_DQF], 1);
-    mbar_init(&bar[B_DQE], kCompute);
+    mbar_init(&bar[B_DQE], 2);
     mbar_init(&bar[B_OF], kCompute);
     mbar_init(&bar[B_DRAIN], 1);
     *abort = 0;
@@ -290,44 +296,50 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
       constexpr uint32_t kIdDq = idesc_bf16_f32(128, D, true, true);    // (dS^T)^T K
       int g = 0, k = 0;
       bool ok = true;
+      // Per visit gt the order is: dV(gt) once P^T is written, then S^T(gt + 1)
+      // (its S columns held P^T(gt), read by the dV just issued: tcgen05.mma ops
+      // of one thread run in order), dK(gt) and dQ(gt) once dS^T is written,
+      // then dP^T(gt + 1) once dQ(gt) has been read out of its columns.
+      auto issue_s = [&](int gt) -> bool {  // S^T = K Q^T
+        const int s = gt & 1;
+        if (!mbar_wait(&bar[B_QF + s], (gt >> 1) & 1, abort, st, 111)) return false;
+        tc_fence_after();
+        const uint32_t qb = sb + L::q + s * L::kT;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * L::kAtom + (kk & 3) * 32;
+          mma_bf16(tmem + kColS, smem_desc_sw128(sb + L::k + off, 16, 1024),
+                   smem_desc_sw128(qb + off, 16, 1024), kIdS, kk > 0);
+        }
+        mma_commit(&bar[B_SF]);
+        return true;
+      };
+      auto issue_dp = [&](int gt) -> bool {  // dP^T = V dO^T into the columns dQ left
+        if (!mbar_wait(&bar[B_DOF], gt & 1, abort, st, 112) ||
+            (gt > 0 && !mbar_wait(&bar[B_DQE], (gt - 1) & 1, abort, st, 113)))
+          return false;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * L::kAtom + (kk & 3) * 32;
+          mma_bf16(tmem + kColDP, smem_desc_sw128(sb + L::v + off, 16, 1024),
+                   smem_desc_sw128(sb + L::dO + off, 16, 1024), kIdS, kk > 0);
+        }
+        mma_commit(&bar[B_DPF]);
+        return true;
+      };
       for (int idx = blockIdx.x; ok && idx < n_items; idx += gridDim.x, ++k) {
         const Item itm(idx, a.Hkv, a.Bt);
         Visits vis;
         vis.init(m, itm.bt, itm.hk, rep, itm.J);
-        if (vis.n > 0 && !mbar_wait(&bar[B_KVF], k & 1, abort, st, 110)) break;
+        if (vis.n > 0 && (!mbar_wait(&bar[B_KVF], k & 1, abort, st, 110) || !issue_s(g) ||
+                          !issue_dp(g)))
+          break;
         for (int it = 0; it < vis.n; ++it) {
           const int gt = g + it, s = gt & 1;
-          // S^T = K Q^T (the S columns last held P^T(gt - 1), read by a P V
-          // issued before this MMA: tcgen05.mma ops of one thread run in order)
-          if (!mbar_wait(&bar[B_QF + s], (gt >> 1) & 1, abort, st, 111)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t qb = sb + L::q + s * L::kT;
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * L::kAtom + (kk & 3) * 32;
-            mma_bf16(tmem + kColS, smem_desc_sw128(sb + L::k + off, 16, 1024),
-                     smem_desc_sw128(qb + off, 16, 1024), kIdS, kk > 0);
-          }
-          mma_commit(&bar[B_SF]);
-          // dP^T = V dO^T into the columns the previous dQ has left
-          if (!mbar_wait(&bar[B_DOF], gt & 1, abort, st, 112) ||
-              (gt > 0 && !mbar_wait(&bar[B_DQE], (gt - 1) & 1, abort, st, 113))) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * L::kAtom + (kk & 3) * 32;
-            mma_bf16(tmem + kColDP, smem_desc_sw128(sb + L::v + off, 16, 1024),
-                     smem_desc_sw128(sb + L::dO + off, 16, 1024), kIdS, kk > 0);
-          }
-          mma_commit(&bar[B_DPF]);
-          // P^T (TMEM) and dS^T (shared memory) of both halves are written
-          if (!mbar_wait(&bar[B_PF], gt & 1, abort, st, 114) ||
+          const bool more = it + 1 < vis.n;
+          // P^T in TMEM: dV += P^T dO (the previous item's dV, dK read out first)
+          if (!mbar_wait(&bar[B_PF1], gt & 1, abort, st, 114) ||
               (it == 0 && k > 0 && !mbar_wait(&bar[B_OF], (k - 1) & 1, abort, st, 115))) {
             ok = false;
             break;
@@ -340,6 +352,17 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
                         kIdAcc, (it > 0 || kk > 0) ? 1u : 0u);
           }
           mma_commit(&bar[B_DOE]);
+          if (more && !issue_s(gt + 1)) {
+            ok = false;
+            break;
+          }
+          // dS^T in shared memory: dK += dS^T Q, dQ = dS K
+          if (!mbar_wait(&bar[B_PF2], gt & 1, abort, st, 117)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t qb = sb + L::q + s * L::kT;
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
             const uint32_t aoff = (kk >> 2) * L::kAtom + (kk & 3) * 32;
@@ -353,6 +376,10 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
             mma_bf16(tmem + kColDP, smem_desc_sw128(sb + L::dst + kk * 2048, L::kAtom, 1024),
                      smem_desc_sw128(sb + L::k + kk * 2048, L::kAtom, 1024), kIdDq, kk > 0);
           mma_commit(&bar[B_DQF]);
+          if (more && !issue_dp(gt + 1)) {
+            ok = false;
+            break;
+          }
         }
         if (!ok) break;
         mma_commit(&bar[B_KVE]);  // every MMA of this item reading K and V is issued
@@ -440,9 +467,9 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
       const int kq = itm.J * kTile + r;  // this thread's key row
       for (int it = 0; it < vis.n; ++it) {
         const int gt = g + it, s = gt & 1;
+        // phase 1: P from S^T (needs only S^T and the stored LSE)
         if (!__all_sync(0xffffffffu, mbar_wait(&bar[B_SF], gt & 1, abort, st, 120) &&
-                                         mbar_wait(&bar[B_MF + s], (gt >> 1) & 1, abort, st, 121) &&
-                                         mbar_wait(&bar[B_DPF], gt & 1, abort, st, 122))) {
+                                         mbar_wait(&bar[B_MF + s], (gt >> 1) & 1, abort, st, 121))) {
           ok = false;
           break;
         }
@@ -454,44 +481,60 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
         const float* dlt = lse2 + 128;
         tc_fence_after();
         __syncwarp();  // the TMEM loads below are warp-collective (.sync.aligned)
+        float pv[64];
+        tmem_ld32(lane_addr + kColS + half * 64, pv);
+        tmem_ld32(lane_addr + kColS + half * 64 + 32, pv + 32);
+        tmem_wait_ld();
         uint32_t pk[32];
 #pragma unroll
+        for (int i = 0; i < 64; i += 2) {
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const bool v = (mw[(i + u) >> 5] >> ((i + u) & 31)) & 1u;
+            pv[i + u] = v ? ex2(fmaf(pv[i + u], sl2, -lse2[i + u])) : 0.f;
+          }
+          pk[i >> 1] = pack_bf16(pv[i], pv[i + 1]);
+        }
+        // P^T (bf16 pairs) over the first 32 of this half's S columns, all read
+        __syncwarp();
+        tmem_st32(lane_addr + kColS + half * 64, reinterpret_cast<const float*>(pk));
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&bar[B_PF1]);
+        // phase 2: dS = P (dP - D) into dS^T (key row r, this half's 64 query
+        // columns); the previous dS^T was read by MMAs that finished before
+        // dP^T of this visit
+        if (!__all_sync(0xffffffffu, mbar_wait(&bar[B_DPF], gt & 1, abort, st, 122))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        __syncwarp();
+#pragma unroll
         for (int c2 = 0; c2 < 2; ++c2) {  // 32 query columns at a time
-          float sv[32], dv[32];
-          tmem_ld32(lane_addr + kColS + half * 64 + c2 * 32, sv);
+          float dv[32];
           tmem_ld32(lane_addr + kColDP + half * 64 + c2 * 32, dv);
           tmem_wait_ld();
           uint32_t dk[16];
 #pragma unroll
           for (int c = 0; c < 32; c += 2) {
-            float pv[2], ds[2];
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-              const int i = c2 * 32 + c + u;
-              const bool v = (mw[c2] >> (c + u)) & 1u;
-              const float p = v ? ex2(fmaf(sv[c + u], sl2, -lse2[i])) : 0.f;
-              pv[u] = p;
-              ds[u] = p * (dv[c + u] - dlt[i]);
-            }
-            pk[(c2 * 32 + c) >> 1] = pack_bf16(pv[0], pv[1]);
-            dk[c >> 1] = pack_bf16(ds[0], ds[1]);
+            const int i = c2 * 32 + c;
+            dk[c >> 1] = pack_bf16(pv[i] * (dv[c] - dlt[i]), pv[i + 1] * (dv[c + 1] - dlt[i + 1]));
           }
-          // dS^T: key row r, query columns 64 half + 32 c2 + [0, 32)
           const uint32_t base = sb + L::dst + half * L::kAtom;
 #pragma unroll
           for (int ch = 0; ch < 4; ++ch)
             st_shared_v4(base + sw128_offset(r, c2 * 32 + ch * 8), dk[ch * 4], dk[ch * 4 + 1],
                          dk[ch * 4 + 2], dk[ch * 4 + 3]);
         }
-        // P^T (bf16 pairs) over the first 32 of this half's S columns, all read
-        __syncwarp();
-        tmem_st32(lane_addr + kColS + half * 64, reinterpret_cast<const float*>(pk));
-        tmem_wait_st();
         fence_async_shared();
         tc_fence_before();
-        mbar_arrive(&bar[B_PF]);
-        // dQ_I: TMEM lane = query row, this half's D / 2 columns; released
-        // before the reductions are issued
+        mbar_arrive(&bar[B_PF2]);
+        // dQ_I: TMEM lane = query row, this half's D / 2 columns, staged in
+        // fp32 (32-column chunks, 128-byte swizzle) and added to the global dQ
+        // by bulk tensor reductions. Half 0 stages in the Q stage of this
+        // visit (dK is its last reader), half 1 in the dS^T tile (dK and dQ
+        // are its last readers); both are released only once read.
         if (!__all_sync(0xffffffffu, mbar_wait(&bar[B_DQF], gt & 1, abort, st, 123))) {
           ok = false;
           break;
@@ -503,15 +546,33 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
         for (int c = 0; c < D / 64; ++c) tmem_ld32(lane_addr + kColDP + half * (D / 2) + c * 32, dq + c * 32);
         tmem_wait_ld();
         tc_fence_before();
-        mbar_arrive(&bar[B_DQE]);
-        const int q = I * kTile + r;
-        if (q < a.N) {
-          float* dst = a.dq + (((int64_t)itm.bt * a.N + q) * a.Hq + h) * D + half * (D / 2);
+        const uint32_t stage = half == 0 ? sb + L::q + s * L::kT : sb + L::dst;
 #pragma unroll
-          for (int c = 0; c < D / 2; c += 4)
-            red_add_v4(dst + c, dq[c] * a.scale, dq[c + 1] * a.scale, dq[c + 2] * a.scale,
-                       dq[c + 3] * a.scale);
+        for (int c = 0; c < D / 64; ++c)
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {  // 16-byte granule j of the 128-byte row
+            const float* v = dq + c * 32 + j * 4;
+            st_shared_v4(stage + c * 16384 + r * 128 + ((j ^ (r & 7)) << 4),
+                         __float_as_uint(v[0] * a.scale), __float_as_uint(v[1] * a.scale),
+                         __float_as_uint(v[2] * a.scale), __float_as_uint(v[3] * a.scale));
+          }
+        fence_async_shared();
+        mbar_arrive(&bar[B_HS + half]);
+        if (quarter == 0 && lane == 0) {  // one thread per half issues the reductions
+          if (!mbar_wait(&bar[B_HS + half], gt & 1, abort, st, 124)) {
+            ok = false;
+          } else {
+#pragma unroll
+            for (int c = 0; c < D / 64; ++c)
+              tma_reduce_add_4d(&P.tmdq, stage + c * 16384, half * (D / 2) + c * 32, h, I * kTile,
+                                itm.bt);
+            bulk_commit_group();
+            bulk_wait_read_all();
+            if (half == 0) mbar_arrive(&bar[B_QE + s]);
+            mbar_arrive(&bar[B_DQE]);
+          }
         }
+        if (!__all_sync(0xffffffffu, ok)) break;
       }
       if (!ok) break;
       // ------------------------------------------------------------ epilogue
@@ -547,6 +608,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
       mbar_arrive(&bar[B_OF]);  // dV and dK may be overwritten by the next item
       g += vis.n;
     }
+    if (quarter == 0 && lane == 0) bulk_wait_all();  // the dQ reductions have landed
   }
   tc_fence_before();
   __syncthreads();
@@ -593,6 +655,8 @@ __global__ void __launch_bounds__(256) bwd_tc_prep_kernel(AttnArgs a, float* lse
 // [Bt, N, H, d] bf16 with element strides {batch, seq, head}; box 64 x 1 x 128 x 1.
 bool make_tile_map(CUtensorMap* map, const void* base, int d, int H, int N, int Bt,
                    const int64_t* s);
+bool make_map_4d(CUtensorMap* map, CUtensorMapDataType dtype, int ebytes, const void* base, int d,
+                 int H, int N, int Bt, const int64_t* s, int box_d, int rows);
 int sm_count();
 
 template <int D>
@@ -603,6 +667,10 @@ static cudaError_t bwd_tc_launch(const AttnArgs& a, const MaskArgs& m, void* ws,
       !make_tile_map(&P.tmk, a.k, D, a.Hkv, a.N, a.Bt, a.ks) ||
       !make_tile_map(&P.tmv, a.v, D, a.Hkv, a.N, a.Bt, a.vs) ||
       !make_tile_map(&P.tmdo, a.dout, D, a.Hq, a.N, a.Bt, a.os))
+    return cudaErrorInvalidValue;
+  const int64_t dqs[3] = {(int64_t)a.N * a.Hq * D, (int64_t)a.Hq * D, D};  // dense fp32 dQ
+  if (!make_map_4d(&P.tmdq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.dq, D, a.Hq, a.N, a.Bt, dqs, 32,
+                   kTile))
     return cudaErrorInvalidValue;
   P.a = a;
   P.m = m;

@@ -737,21 +737,28 @@ static EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// [Bt, N, H, d] bf16 with element strides {batch, seq, head}; box 64 x 1 x rows x 1,
-// 128-byte swizzle.
-bool make_tile_map_box(CUtensorMap* map, const void* base, int d, int H, int N, int Bt,
-                       const int64_t* s, int rows) {
+// [Bt, N, H, d] of `ebytes`-byte elements with element strides {batch, seq,
+// head}; box box_d x 1 x rows x 1, 128-byte swizzle (box_d * ebytes <= 128).
+bool make_map_4d(CUtensorMap* map, CUtensorMapDataType dtype, int ebytes, const void* base, int d,
+                 int H, int N, int Bt, const int64_t* s, int box_d, int rows) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   const int64_t sh = s[2] > 0 ? s[2] : d, sn = s[1];
   const int64_t sbat = (Bt > 1) ? s[0] : sn * N;
   cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)N, (cuuint64_t)Bt};
-  cuuint64_t strides[3] = {(cuuint64_t)(sh * 2), (cuuint64_t)(sn * 2), (cuuint64_t)(sbat * 2)};
-  cuuint32_t box[4] = {64, 1, (cuuint32_t)rows, 1};
+  cuuint64_t strides[3] = {(cuuint64_t)(sh * ebytes), (cuuint64_t)(sn * ebytes),
+                           (cuuint64_t)(sbat * ebytes)};
+  cuuint32_t box[4] = {(cuuint32_t)box_d, 1, (cuuint32_t)rows, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
-  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
-             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+  return enc(map, dtype, 4, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// bf16 with a box of 64 x 1 x rows x 1.
+bool make_tile_map_box(CUtensorMap* map, const void* base, int d, int H, int N, int Bt,
+                       const int64_t* s, int rows) {
+  return make_map_4d(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, d, H, N, Bt, s, 64, rows);
 }
 
 bool make_tile_map(CUtensorMap* map, const void* base, int d, int H, int N, int Bt,
