@@ -122,7 +122,7 @@ struct Item {
 };
 
 
-constexpr int kMaskSlots = 4;              // mask ring depth (tiles)
+constexpr int kMaskSlots = 8;              // mask ring depth (tiles)
 constexpr uint32_t kMaskSlotBytes = 2048;  // [4 words][128 rows] uint32
 constexpr int kRowCacheWords = 1024;       // gzip: the item's block-row bits
 
@@ -130,11 +130,17 @@ template <int D>
 struct FwdLayout {
   static constexpr int kKStages = D == 64 ? 4 : 3;  // K ring depth
   static constexpr int kVStages = D == 64 ? 4 : 2;  // V ring depth
+  static constexpr int kQStages = D == 64 ? 2 : 1;  // Q tiles (next item's loads early)
+  // d = 64: K and V of a tile share a stage and one full / free barrier pair,
+  // so the MMA thread waits once per tile for both (every mbarrier wait on
+  // that thread leaves the tensor core idle for its latency, as tcgen05.mma
+  // issue blocks until the previous MMA has started)
+  static constexpr bool kMergedKV = D == 64;
   static constexpr uint32_t kQ = 128 * D * 2;        // Q tile
   static constexpr uint32_t kKV = 128 * D * 2;       // one K or V tile
   static constexpr uint32_t kAtom = 128 * 128;       // [128 rows][64 bf16] swizzle atom
   static constexpr uint32_t q = 0;
-  static constexpr uint32_t k0 = kQ;
+  static constexpr uint32_t k0 = kQStages * kQ;
   static constexpr uint32_t v0 = k0 + kKStages * kKV;
   static constexpr uint32_t mask = v0 + kVStages * kKV;
   static constexpr uint32_t rows = mask + kMaskSlots * kMaskSlotBytes;
@@ -143,15 +149,19 @@ struct FwdLayout {
   static constexpr uint32_t bytes = bars + 512 + 1024;  // + alignment slack
 };
 
-// mbarriers. QF/QE: Q tile full / consumed (per item). KF/KE, VF/VE: K or V
-// stage full / free. SF: S buffer written. PF: P half written (TMEM). OD: P V
-// of the half done (per tile). MF/ME: mask slot written / read. OI: every MMA
-// of the item done. OF: both halves have read O (per item). ML: (max, sum)
-// exchanged. DRAIN: all MMAs done before exit.
+// mbarriers. QF/QE: Q stage full / consumed (per item). KF/KE, VF/VE: K or V
+// stage full / free (d = 64: KF/KE cover K and V). SF: S buffer written. PF:
+// P written to TMEM by both halves, one barrier per S buffer: the softmax can
+// finish tile j + 1 before the MMA thread has seen tile j's P, but not tile
+// j + 2 (its S needs P V(j) issued), so a barrier per S buffer is never two
+// phases ahead of its waiter. OD: P V done, one barrier per S buffer (waited
+// for only before an O rescale). MF/ME: mask slot
+// written / read. OI: every MMA of the item done. OF: both halves have read O
+// (per item). ML: (max, sum) exchanged. DRAIN: all MMAs done before exit.
 enum {
-  B_QF = 0, B_QE = 1, B_KF = 2, B_KE = 6, B_VF = 10, B_VE = 14, B_SF = 18, B_PF = 20,
-  B_OD = 22, B_MF = 24, B_ME = 28, B_OI = 32, B_OF = 33, B_ML = 34, B_DRAIN = 35,
-  kNumBars = 36
+  B_QF = 0, B_QE = 2, B_KF = 4, B_KE = 8, B_VF = 12, B_VE = 16, B_SF = 20, B_PF = 22,
+  B_OD = 24, B_MF = 26, B_ME = B_MF + kMaskSlots, B_OI = B_ME + kMaskSlots, B_OF, B_ML, B_DRAIN,
+  kNumBars
 };
 
 constexpr uint32_t kTmemCols = 512;
@@ -270,7 +280,7 @@ __device__ __forceinline__ int item_tiles(const MaskArgs& m, int idx, int T, int
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1) fwd_tc_kernel(const __grid_constant__ FwdTcParams P) {
   using L = FwdLayout<D>;
-  constexpr int KS = L::kKStages, VS = L::kVStages;
+  constexpr int KS = L::kKStages, VS = L::kVStages, QS = L::kQStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const uint32_t sb = smem_u32(smem);
@@ -288,8 +298,10 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_kernel(const __grid_consta
   DeviceStatus* st = a.status;
 
   if (threadIdx.x == 0) {
-    mbar_init(&bar[B_QF], 1);
-    mbar_init(&bar[B_QE], 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bar[B_QF + s], 1);
+      mbar_init(&bar[B_QE + s], 1);
+    }
     for (int s = 0; s < KS; ++s) {
       mbar_init(&bar[B_KF + s], 1);
       mbar_init(&bar[B_KE + s], 1);
@@ -300,9 +312,10 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_kernel(const __grid_consta
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bar[B_SF + s], 1);
-      mbar_init(&bar[B_PF + s], kSoftmaxThreads / 2);
-      mbar_init(&bar[B_OD + s], 1);
+      mbar_init(&bar[B_PF + s], kSoftmaxThreads);
     }
+    mbar_init(&bar[B_OD], 1);
+    mbar_init(&bar[B_OD + 1], 1);
     for (int s = 0; s < kMaskSlots; ++s) {
       mbar_init(&bar[B_MF + s], 32);
       mbar_init(&bar[B_ME + s], kSoftmaxThreads);
@@ -335,17 +348,27 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_kernel(const __grid_consta
       }
       int g = 0, k = 0, last_k = -1, last_v = -1, last_q = -1;
       bool ok = true;
+      WorkList wl_next;  // the next item's list, read one item ahead
+      if (blockIdx.x < n_items) {
+        const Item f(blockIdx.x, T, a.Hq, a.Bt);
+        wl_next.init(m, list_of(m, f.bt, f.h), f.I);
+      }
       for (int idx = blockIdx.x; ok && idx < n_items; idx += gridDim.x, ++k) {
         const Item itm(idx, T, a.Hq, a.Bt);
-        WorkList wl;
-        wl.init(m, list_of(m, itm.bt, itm.h), itm.I);
+        const WorkList wl = wl_next;
+        const bool more = idx + (int)gridDim.x < n_items;
+        if (more) {
+          const Item nx(idx + gridDim.x, T, a.Hq, a.Bt);
+          wl_next.init(m, list_of(m, nx.bt, nx.h), nx.I);
+        }
         const int hk = itm.h / (a.Hq / a.Hkv);
-        // the previous item's last Q K^T has read Q
-        if (k > 0 && !mbar_wait(&bar[B_QE], (k - 1) & 1, abort, st, 1)) break;
-        mbar_arrive_expect_tx(&bar[B_QF], L::kQ);
+        // Q stage k % QS last held item k - QS, whose last Q K^T has read it
+        const int qs = k % QS;
+        if (k >= QS && !mbar_wait(&bar[B_QE + qs], ((k / QS) - 1) & 1, abort, st, 1)) break;
+        mbar_arrive_expect_tx(&bar[B_QF + qs], L::kQ);
         for (int at = 0; at < D / 64; ++at)
-          tma_load_4d(smem + L::q + at * L::kAtom, &P.tmq, &bar[B_QF], at * 64, itm.h,
-                      itm.I * kTile, itm.bt);
+          tma_load_4d(smem + L::q + qs * L::kQ + at * L::kAtom, &P.tmq, &bar[B_QF + qs], at * 64,
+                      itm.h, itm.I * kTile, itm.bt);
         last_q = k;
         // K of tile it + 1 is requested before V of tile it
         auto load = [&](bool is_k, int it) -> bool {
@@ -364,16 +387,43 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_kernel(const __grid_consta
           if (is_k) last_k = gt; else last_v = gt;
           return true;
         };
-        if (wl.n > 0) ok = load(true, 0);
-        for (int it = 0; ok && it < wl.n; ++it) {
-          if (it + 1 < wl.n) ok = load(true, it + 1);
-          if (ok) ok = load(false, it);
+        // d = 64: K and V of tile it on one barrier of stage (g + it) % KS
+        auto load_kv = [&](int it) -> bool {
+          const int gt = g + it, s = gt % KS;
+          if (!mbar_wait(&bar[B_KE + s], ((gt / KS) & 1) ^ 1, abort, st, 2)) return false;
+          int src, k0, kind, cnt;
+          wl.entry(m, it, src, k0, kind, cnt);
+          mbar_arrive_expect_tx(&bar[B_KF + s], 2 * L::kKV);
+          for (int at = 0; at < D / 64; ++at) {
+            tma_load_4d(smem + L::k0 + s * L::kKV + at * L::kAtom, src ? &P.tmkc : &P.tmk,
+                        &bar[B_KF + s], at * 64, hk, k0, itm.bt);
+            tma_load_4d(smem + L::v0 + s * L::kKV + at * L::kAtom, src ? &P.tmvc : &P.tmv,
+                        &bar[B_KF + s], at * 64, hk, k0, itm.bt);
+          }
+          last_k = gt;
+          return true;
+        };
+        if (L::kMergedKV) {
+          for (int it = 0; ok && it < wl.n; ++it) ok = load_kv(it);
+        } else {
+          if (wl.n > 0) ok = load(true, 0);
+          for (int it = 0; ok && it < wl.n; ++it) {
+            if (it + 1 < wl.n) ok = load(true, it + 1);
+            if (ok) ok = load(false, it);
+          }
+        }
+        if (more && m.kind == SA_MASK_GZIP) {
+          // the next item's first entries, so that its first K load is not
+          // held up by a list lookup
+          prefetch_l1(m.tcol + wl_next.e0);
+          prefetch_l1(m.tkind + wl_next.e0);
         }
         g += wl.n;
       }
       // every copy this CTA started must land before the CTA may exit
       volatile int no_abort = 0;
-      if (last_q >= 0) mbar_wait(&bar[B_QF], last_q & 1, &no_abort, nullptr, 3);
+      for (int q = last_q; q >= 0 && q > last_q - QS; --q)
+        mbar_wait(&bar[B_QF + q % QS], (q / QS) & 1, &no_abort, nullptr, 3);
       for (int s = 0; s < KS; ++s) {
         if (last_k >= s) {
           const int gs = last_k - ((last_k - s) % KS);
@@ -390,6 +440,12 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_kernel(const __grid_consta
   } else if (warp == 1) {
     if (lane == 0) {
       // --------------------------------------------------------- MMA issuer
+      // One thread issues S_j = Q K_j^T and then O += P_{j-1} V_{j-1}: tcgen05
+      // ops of one thread run in issue order, so Q K^T(j + 1) may reuse the S
+      // buffer of P(j - 1) right after P V(j - 1) is issued. tcgen05.mma issue
+      // blocks until the tensor core has taken the previous MMA and a barrier
+      // wait after it waits for the queued MMAs, so the waits are kept to two
+      // per tile (K/V landed, P written).
       constexpr uint32_t kIdQK = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t kIdPV = idesc_bf16_f32(128, D, false, true);
       int g = 0, k = 0;
@@ -398,14 +454,13 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_kernel(const __grid_consta
       for (int idx = blockIdx.x; ok && idx < n_items; idx += gridDim.x, ++k) {
         const int n = n_next;
         n_next = idx + (int)gridDim.x < n_items ? item_tiles(m, idx + gridDim.x, T, a.Hq, a.Bt) : 0;
-        if (!mbar_wait(&bar[B_QF], k & 1, abort, st, 10)) break;
+        const int qs = k % QS;
+        const uint32_t qa = sb + L::q + qs * L::kQ;
+        if (!mbar_wait(&bar[B_QF + qs], (k / QS) & 1, abort, st, 10)) break;
         // both halves have read the previous item's O before it is overwritten
         bool o_free = k == 0;
         for (int it = 0; it <= n; ++it) {
           if (it < n) {
-            // S buffer gq & 1 last held P(gq - 2), read by P V(gq - 2), which
-            // was issued before this Q K^T; tcgen05.mma ops of one thread run in
-            // issue order, so no wait is needed for it
             const int gq = g + it, s = gq % KS, sb2 = gq & 1;
             if (!mbar_wait(&bar[B_KF + s], (gq / KS) & 1, abort, st, 11)) {
               ok = false;
@@ -416,15 +471,15 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_kernel(const __grid_consta
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
               const uint32_t off = (kk >> 2) * L::kAtom + (kk & 3) * 32;
-              mma_bf16(tmem + sb2 * 128, smem_desc_sw128(sb + L::q + off, 16, 1024),
+              mma_bf16(tmem + sb2 * 128, smem_desc_sw128(qa + off, 16, 1024),
                        smem_desc_sw128(kb + off, 16, 1024), kIdQK, kk > 0);
             }
             mma_commit(&bar[B_SF + sb2]);
-            mma_commit(&bar[B_KE + s]);
-            if (it == n - 1) mma_commit(&bar[B_QE]);
+            if (!L::kMergedKV) mma_commit(&bar[B_KE + s]);
+            if (it == n - 1) mma_commit(&bar[B_QE + qs]);
           }
           if (it >= 1) {
-            const int gp = g + it - 1, s = gp % VS;
+            const int gp = g + it - 1, s = gp % (L::kMergedKV ? KS : VS);
             if (!o_free) {
               if (!mbar_wait(&bar[B_OF], (k - 1) & 1, abort, st, 13)) {
                 ok = false;
@@ -432,17 +487,18 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_kernel(const __grid_consta
               }
               o_free = true;
             }
-            if (!mbar_wait(&bar[B_VF + s], (gp / VS) & 1, abort, st, 14)) {
+            if (!L::kMergedKV && !mbar_wait(&bar[B_VF + s], (gp / VS) & 1, abort, st, 14)) {
               ok = false;
               break;
             }
+            if (!mbar_wait(&bar[B_PF + (gp & 1)], (gp >> 1) & 1, abort, st, 15)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
             const uint32_t vb = sb + L::v0 + s * L::kKV;
+#pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
-              if (!mbar_wait(&bar[B_PF + hf], gp & 1, abort, st, 15 + hf)) {
-                ok = false;
-                break;
-              }
-              tc_fence_after();
               // P of this half: bf16 pairs in the first 32 columns of its S columns
               const uint32_t pa = tmem + (gp & 1) * 128 + hf * 64;
 #pragma unroll
@@ -451,15 +507,14 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_kernel(const __grid_consta
                 mma_bf16_ts(tmem + kTmemO + hf * D, pa + kk * 8, bd, kIdPV,
                             (it > 1 || kk > 0) ? 1u : 0u);
               }
-              mma_commit(&bar[B_OD + hf]);
             }
-            if (!ok) break;
-            mma_commit(&bar[B_VE + s]);
+            mma_commit(&bar[B_OD + (gp & 1)]);
+            mma_commit(&bar[L::kMergedKV ? B_KE + s : B_VE + s]);
           }
         }
         if (!ok) break;
         if (n == 0) {
-          mma_commit(&bar[B_QE]);
+          mma_commit(&bar[B_QE + qs]);
           if (!o_free && !mbar_wait(&bar[B_OF], (k - 1) & 1, abort, st, 13)) break;
         }
         mma_commit(&bar[B_OI]);
@@ -477,20 +532,57 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_kernel(const __grid_consta
     const int gzip = m.kind == SA_MASK_GZIP;
     const int lb = (gzip && m.b < kTile) ? __ffs(m.b) - 1 : 0;  // b < 128 is a power of two
     uint32_t* rcache = reinterpret_cast<uint32_t*>(smem + L::rows);
+    // gzip: the block rows of a query tile (first and last block row)
+    auto row_span = [&](int I, int& rb0, int& rb1) {
+      rb0 = I * kTile / (gzip ? m.b : 1);
+      rb1 = gzip ? min(m.B - 1, (I * kTile + kTile - 1) / m.b) : rb0;
+    };
+    // The next item's list, its first 32 block-row words and its first 32
+    // tile entries are read one item ahead, into registers, so that no
+    // global round trip sits between two items.
+    WorkList wl_next;
+    uint32_t row_next = 0u;
+    int col_next = 0, kind_next = 0;
+    auto fetch_head = [&](int idx) {
+      const Item nx(idx, T, a.Hq, a.Bt);
+      const int list = list_of(m, nx.bt, nx.h);
+      wl_next.init(m, list, nx.I);
+      if (gzip) {
+        int rb0, rb1;
+        row_span(nx.I, rb0, rb1);
+        const int nw = (rb1 - rb0 + 1) * m.words;
+        row_next = lane < nw ? m.bits[((int64_t)list * m.B + rb0) * m.words + lane] : 0u;
+      }
+    };
+    auto fetch_entries = [&]() {
+      if (gzip) {
+        col_next = lane < wl_next.n ? m.tcol[wl_next.e0 + lane] : 0;
+        kind_next = lane < wl_next.n ? m.tkind[wl_next.e0 + lane] : 0;
+      }
+    };
+    if (blockIdx.x < n_items) {
+      fetch_head(blockIdx.x);
+      fetch_entries();
+    }
     int g = 0;
     for (int idx = blockIdx.x; idx < n_items; idx += gridDim.x) {
       const Item itm(idx, T, a.Hq, a.Bt);
       const int list = list_of(m, itm.bt, itm.h);
-      WorkList wl;
-      wl.init(m, list, itm.I);
+      const WorkList wl = wl_next;
+      const uint32_t row_pre = row_next;
+      int col_reg = col_next, kind_reg = kind_next;  // gzip: tile list entries it0 + lane
+      const bool more = idx + (int)gridDim.x < n_items;
+      if (more) fetch_head(idx + gridDim.x);  // in flight during this item
       // gzip: the block rows of this query tile, copied once per item when they fit
-      const int rb0 = itm.I * kTile / (gzip ? m.b : 1);
-      const int rb1 = gzip ? min(m.B - 1, (itm.I * kTile + kTile - 1) / m.b) : rb0;
-      const bool cached = gzip && (rb1 - rb0 + 1) * m.words <= kRowCacheWords;
+      int rb0, rb1;
+      row_span(itm.I, rb0, rb1);
+      const int nw = (rb1 - rb0 + 1) * m.words;
+      const bool cached = gzip && nw <= kRowCacheWords;
       __syncwarp();  // the previous item's lookups are done
       if (cached) {
         const uint32_t* src = m.bits + ((int64_t)list * m.B + rb0) * m.words;
-        for (int x = lane; x < (rb1 - rb0 + 1) * m.words; x += 32) rcache[x] = src[x];
+        if (lane < nw) rcache[lane] = row_pre;
+        for (int x = lane + 32; x < nw; x += 32) rcache[x] = src[x];
       }
       __syncwarp();
       RowCtx rc[4];
@@ -507,9 +599,8 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_kernel(const __grid_consta
         rc[i].li = 0;
       }
       bool ok = true;
-      int col_reg = 0, kind_reg = 0;  // gzip: tile list entries it0 + lane
       for (int it = 0; it < wl.n; ++it) {
-        if (gzip && (it & 31) == 0) {
+        if (gzip && it > 0 && (it & 31) == 0) {
           const int e = it + lane;
           col_reg = e < wl.n ? m.tcol[wl.e0 + e] : 0;
           kind_reg = e < wl.n ? m.tkind[wl.e0 + e] : 0;
@@ -552,6 +643,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_kernel(const __grid_consta
         mbar_arrive(&bar[B_MF + slot]);  // release: the words above are visible to the waiter
       }
       if (!ok) break;
+      if (more) fetch_entries();  // the next list's head has arrived by now
       g += wl.n;
     }
   } else if (warp >= 2 && warp < 2 + kSoftmaxThreads / 32) {
@@ -597,40 +689,56 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_kernel(const __grid_consta
             x[32 + i] = ((mw1 >> i) & 1u) ? x[32 + i] : -INFINITY;
           }
         }
-        float t[16];
+        // row max of the 64 scores with three-input max: 21 + 7 + 3 + 1
+        float t[21], u[7];
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-          t[i] = fmaxf(fmaxf(x[4 * i], x[4 * i + 1]), fmaxf(x[4 * i + 2], x[4 * i + 3]));
+        for (int i = 0; i < 21; ++i) t[i] = fmax3(x[3 * i], x[3 * i + 1], x[3 * i + 2]);
 #pragma unroll
-        for (int w = 8; w >= 1; w >>= 1)
-#pragma unroll
-          for (int i = 0; i < w; ++i) t[i] = fmaxf(t[i], t[i + w]);
-        const float m_new = fmaxf(m_run, t[0] * sl2);  // scale > 0 keeps the order
+        for (int i = 0; i < 7; ++i) u[i] = fmax3(t[3 * i], t[3 * i + 1], t[3 * i + 2]);
+        const float tmax = fmax3(fmax3(u[0], u[1], u[2]), fmax3(u[3], u[4], u[5]),
+                                 fmaxf(u[6], x[63]));
+        const float m_new = fmaxf(m_run, tmax * sl2);  // scale > 0 keeps the order
         const bool resc = m_new > m_run + 8.f;          // true on the first finite max
         const float m_use = resc ? m_new : m_run;
         uint32_t pk[32];
-        float sum[4] = {0.f, 0.f, 0.f, 0.f};
+        float2 sum2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
         if (m_use == -INFINITY) {
 #pragma unroll
           for (int i = 0; i < 32; ++i) pk[i] = 0u;
         } else {
+          // pairs in packed fp32 arithmetic; three of every eight pairs take
+          // 2^x on the FMA pipe (polynomial), the rest on the special-function
+          // unit, whose 16 results per clock and SM bound this loop otherwise
+          const float2 sc = make_float2(sl2, sl2), nm = make_float2(-m_use, -m_use);
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
-            const float p0 = ex2(fmaf(x[2 * i], sl2, -m_use));
-            const float p1 = ex2(fmaf(x[2 * i + 1], sl2, -m_use));
-            sum[i & 3] += p0 + p1;
-            pk[i] = pack_bf16(p0, p1);
+            const float2 e = ffma2(make_float2(x[2 * i], x[2 * i + 1]), sc, nm);
+            float2 p;
+            if ((i & 7) >= 5) {
+              p = exp2_poly2(e);
+            } else {
+              p.x = ex2(e.x);
+              p.y = ex2(e.y);
+            }
+            sum2[i & 1] = fadd2(sum2[i & 1], p);
+            pk[i] = pack_bf16(p.x, p.y);
           }
         }
-        const float rowsum = (sum[0] + sum[1]) + (sum[2] + sum[3]);
+        const float rowsum = (sum2[0].x + sum2[0].y) + (sum2[1].x + sum2[1].y);
         const float alpha = !resc ? 1.f : (m_run == -INFINITY ? 0.f : ex2(m_run - m_use));
-        // O_h was last accumulated by P V of tile gq - 1
-        if (gq >= 1 && !__all_sync(0xffffffffu,
-                                   mbar_wait(&bar[B_OD + half], (gq - 1) & 1, abort, st, 21))) {
-          ok = false;
-          break;
-        }
         if (it >= 1 && __any_sync(0xffffffffu, resc)) {
+          // O_h was last accumulated by P V of tile gq - 1, which must be done
+          // before O_h is rescaled. Only then is it waited for: the OD barrier
+          // of that S buffer has completed P V(gq - 3) (issued before Q K^T(gq
+          // - 1), whose S this softmax has read) and cannot have completed
+          // P V(gq + 1) (no P yet), so the parity of P V(gq - 1)'s phase is
+          // unambiguous. Without a rescale, P(gq) goes to the other S buffer
+          // while P V(gq - 1) may still run.
+          if (!__all_sync(0xffffffffu, mbar_wait(&bar[B_OD + ((gq - 1) & 1)], ((gq - 1) >> 1) & 1,
+                                                  abort, st, 21))) {
+            ok = false;
+            break;
+          }
           // the whole warp takes part; rows that keep their max use alpha = 1
           tc_fence_after();
           __syncwarp();
@@ -651,7 +759,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_kernel(const __grid_consta
         tmem_st32(lane_addr + s * 128 + half * 64, reinterpret_cast<const float*>(pk));
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(&bar[B_PF + half]);
+        mbar_arrive(&bar[B_PF + s]);
       }
       if (!ok) break;
       // ------------------------------------------------------------ epilogue
