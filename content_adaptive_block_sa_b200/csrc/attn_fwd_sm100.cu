@@ -4,33 +4,39 @@
 // tiles are visited in order and everything else is skipped ("UniGist ...",
 // Approach: skipping non-visible blocks is what makes the sparse layout fast;
 // "Gzip-guided sparse attention ...", Scope: dense-then-mask gives no
-// speed-up). The kernel is persistent: one CTA per SM walks the items
-// blockIdx.x, blockIdx.x + gridDim.x, ... (late query tiles, which have the
-// longest lists, first). Ring slots and mbarrier phases run on across items,
-// so the loads and the first Q K^T of the next item overlap the softmax and
-// epilogue of the current one.
+// speed-up). With gzip blocks of 64 tokens ("pair mode") an item is a pair of
+// 64-row query blocks and a visit a pair of 64-key blocks, so that a 128 x 128
+// tensor-core tile holds only block pairs of the mask (see gzip_pair_kernel).
+// The kernel is persistent: one CTA per SM walks the items blockIdx.x,
+// blockIdx.x + gridDim.x, ... (the longest lists first). Ring slots and
+// mbarrier phases run on across items, so the loads and the first Q K^T of the
+// next item overlap the softmax and epilogue of the current one.
 //
-// Roles (352 threads):
-//   warp 0      TMA producer: Q per item; K and V in separate rings, K one
-//               tile ahead of V (K_j is free once Q K_j^T is done, V_j only
-//               after P_j V_j); TMEM allocation.
+// Roles (480 threads):
+//   warp 0      TMA producer: Q per item (d = 64: two Q stages, so the next
+//               item's Q loads early); K and V per visit (d = 64: one stage
+//               and one barrier for both; d = 128: separate rings, K one tile
+//               ahead of V); TMEM allocation.
 //   warp 1      one thread issues tcgen05.mma: S_j = Q K_j^T into one of two
 //               TMEM S buffers, then O_h += P_j[:, h-half] V_j[h-half, :] for
 //               the two column halves h = 0, 1, each into its own TMEM
 //               accumulator, with P_j read from TMEM (A operand) and V_j from
 //               shared memory. Completion is signalled with tcgen05.commit.
+//               (d = 64: two O buffers, items alternate.)
 //   warps 2-9   softmax, two groups of four warps: group h owns key columns
 //               [64h, 64h + 64) of every S tile; thread (h, r) owns query row
 //               r (TMEM lane r) within that half. Each half keeps its own
 //               running max (log2 domain) and row sum, so the two halves never
 //               synchronise per tile; O_h is rescaled lazily, only when the
-//               half's max grew by more than 2^8 (P <= 256 otherwise). The
-//               epilogue exchanges (max, sum) between the halves and merges:
-//               O = (2^(m_0-m) O_0 + 2^(m_1-m) O_1) / (2^(m_0-m) l_0 + 2^(m_1-m) l_1).
+//               half's max grew by more than 2^8 (P <= 256 otherwise). At the
+//               end of an item each half leaves its (max, sum) in shared memory.
 //   warp 10     mask: for each visited tile, ahead of the softmax, the
 //               visibility of its 128 x 128 (row, key) pairs as 4 x 128 bit
 //               words in a shared-memory ring, so that no global load or
 //               mask arithmetic sits on the softmax's path.
+//   warps 11-14 epilogue: thread r merges row r of the two halves,
+//               O = (2^(m_0-m) O_0 + 2^(m_1-m) O_1) / (2^(m_0-m) l_0 + 2^(m_1-m) l_1),
+//               and stores O and LSE while the softmax works on the next item.
 // S is double-buffered (Q K^T of tile j+1 runs while tile j's softmax runs).
 // Each half writes its bf16 P over the first 32 of its own 64 S columns, so P
 // never passes through shared memory; Q K^T(j+2) may overwrite that buffer
@@ -49,6 +55,7 @@ using namespace sm100;
 
 struct FwdTcParams {
   CUtensorMap tmq, tmk, tmv;
+  CUtensorMap tmq64, tmk64, tmv64;  // pair mode: 64-row boxes
   CUtensorMap tmkc, tmvc;  // gist mode: sinks + gists compacted in logical order
   AttnArgs a;
   MaskArgs m;
@@ -74,7 +81,11 @@ struct WorkList {
   int gist, e0, n, nft, nf, jlo;
   __device__ void init(const MaskArgs& m, int list, int I) {
     gist = m.kind == SA_MASK_GIST;
-    if (gist) {
+    if (m.pair) {  // I is the pair index
+      e0 = m.pair_ptr[list * (m.P + 1) + I];
+      n = m.pair_ptr[list * (m.P + 1) + I + 1] - e0;
+      nft = nf = jlo = 0;
+    } else if (gist) {
       jlo = max(0, I - (m.window - 1 + kTile - 1) / kTile);
       nf = m.far_ptr[jlo];
       nft = (nf + kTile - 1) / kTile;
@@ -85,6 +96,14 @@ struct WorkList {
       n = m.trp[list * (m.T + 1) + I + 1] - e0;
       nft = nf = jlo = 0;
     }
+  }
+  // pair mode: first rows of the two 64-key blocks of visit it (the second
+  // repeats the first when the visit has one block; its columns are masked)
+  __device__ void pair_entry(const MaskArgs& m, int it, int& k0a, int& k0b) const {
+    const uint32_t v = (uint32_t)m.visits[e0 + it];
+    const int j1 = v & 0xfff, j2 = (v >> 12) & 0xfff;
+    k0a = j1 * 64;
+    k0b = (j2 == 0xfff ? j1 : j2) * 64;
   }
   // source (0 = sequence, 1 = compacted keys), first key row, kind, valid columns
   __device__ void entry(const MaskArgs& m, int it, int& src, int& k0, int& kind, int& cnt) const {
@@ -136,6 +155,9 @@ struct FwdLayout {
   // that thread leaves the tensor core idle for its latency, as tcgen05.mma
   // issue blocks until the previous MMA has started)
   static constexpr bool kMergedKV = D == 64;
+  // d = 64: two O accumulators in TMEM (items alternate), so the next item's
+  // P V never waits for the epilogue warps to read the previous O
+  static constexpr int kOBufs = D == 64 ? 2 : 1;
   static constexpr uint32_t kQ = 128 * D * 2;        // Q tile
   static constexpr uint32_t kKV = 128 * D * 2;       // one K or V tile
   static constexpr uint32_t kAtom = 128 * 128;       // [128 rows][64 bf16] swizzle atom
@@ -144,8 +166,8 @@ struct FwdLayout {
   static constexpr uint32_t v0 = k0 + kKStages * kKV;
   static constexpr uint32_t mask = v0 + kVStages * kKV;
   static constexpr uint32_t rows = mask + kMaskSlots * kMaskSlotBytes;
-  static constexpr uint32_t ml = rows + kRowCacheWords * 4;  // [2 halves][128] (max, sum)
-  static constexpr uint32_t bars = ml + 2 * 128 * 8;
+  static constexpr uint32_t ml = rows + kRowCacheWords * 4;  // [2 items][2 halves][128] (max, sum)
+  static constexpr uint32_t bars = ml + 2 * 2 * 128 * 8;
   static constexpr uint32_t bytes = bars + 512 + 1024;  // + alignment slack
 };
 
@@ -157,18 +179,22 @@ struct FwdLayout {
 // phases ahead of its waiter. OD: P V done, one barrier per S buffer (waited
 // for only before an O rescale). MF/ME: mask slot
 // written / read. OI: every MMA of the item done. OF: both halves have read O
-// (per item). ML: (max, sum) exchanged. DRAIN: all MMAs done before exit.
+// (per item). OI/OF/ML, one barrier per item parity: OI every MMA of the item
+// done; OF the epilogue warps have read O and (max, sum); ML the softmax
+// halves have written (max, sum). DRAIN: all MMAs done before exit.
 enum {
   B_QF = 0, B_QE = 2, B_KF = 4, B_KE = 8, B_VF = 12, B_VE = 16, B_SF = 20, B_PF = 22,
-  B_OD = 24, B_MF = 26, B_ME = B_MF + kMaskSlots, B_OI = B_ME + kMaskSlots, B_OF, B_ML, B_DRAIN,
-  kNumBars
+  B_OD = 24, B_MF = 26, B_ME = B_MF + kMaskSlots, B_OI = B_ME + kMaskSlots, B_OF = B_OI + 2,
+  B_ML = B_OF + 2, B_DRAIN = B_ML + 2, kNumBars
 };
 
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemO = 256;  // O_0 at 256, O_1 at 256 + D
 constexpr int kSoftmaxThreads = 256;
-constexpr int kThreads = 64 + kSoftmaxThreads + 32;
+constexpr int kEpiThreads = 128;
+constexpr int kThreads = 64 + kSoftmaxThreads + 32 + kEpiThreads;
 constexpr int kMaskWarp = 10;
+constexpr int kEpiWarp0 = 11;  // warps 11-14: epilogue (one per TMEM lane quarter)
 
 // Bits [0, n) set, n clamped to [0, 32] (no branch).
 __device__ __forceinline__ uint32_t prefix_bits(int n) {
@@ -269,6 +295,28 @@ __device__ __forceinline__ void gzip_tile_words(const MaskArgs& m, int lb, int N
     }
 }
 
+// Pair mode: visibility words of one visit (v = j1 | j2 << 12 | vis << 24)
+// for rows lane + 32 i: rows 0-63 belong to query block qa, 64-127 to qb
+// (qb < 0: none). Key columns 0-63 are block j1, 64-127 block j2. A visited
+// block is either below the row's block (fully visible) or the row's own
+// block (causal: columns up to the row).
+__device__ __forceinline__ void pair_tile_words(uint32_t v, int qa, int qb, int lane,
+                                                uint32_t* out) {
+  const int j1 = v & 0xfff, j2 = (v >> 12) & 0xfff;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int blk = i < 2 ? qa : qb, rr = lane + 32 * (i & 1);
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const int j = w < 2 ? j1 : j2;
+      const uint32_t seen = (v >> (24 + 2 * (w >> 1) + (i >> 1))) & 1u;
+      uint32_t word = 0u;
+      if (blk >= 0 && seen) word = j < blk ? 0xffffffffu : prefix_bits(rr - 32 * (w & 1) + 1);
+      out[w * 128 + lane + 32 * i] = word;
+    }
+  }
+}
+
 // Number of visited tiles of item idx.
 __device__ __forceinline__ int item_tiles(const MaskArgs& m, int idx, int T, int Hq, int Bt) {
   const Item itm(idx, T, Hq, Bt);
@@ -293,7 +341,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_kernel(const __grid_consta
   const AttnArgs& a = P.a;
   const MaskArgs& m = P.m;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int T = m.T;
+  const int T = m.pair ? m.P : m.T;  // items per (head, sequence)
   const int n_items = T * a.Hq * a.Bt;
   DeviceStatus* st = a.status;
 
@@ -320,9 +368,11 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_kernel(const __grid_consta
       mbar_init(&bar[B_MF + s], 32);
       mbar_init(&bar[B_ME + s], kSoftmaxThreads);
     }
-    mbar_init(&bar[B_OI], 1);
-    mbar_init(&bar[B_OF], kSoftmaxThreads);
-    mbar_init(&bar[B_ML], kSoftmaxThreads);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bar[B_OI + s], 1);
+      mbar_init(&bar[B_OF + s], kEpiThreads);
+      mbar_init(&bar[B_ML + s], kSoftmaxThreads);
+    }
     mbar_init(&bar[B_DRAIN], 1);
     *abort = 0;
     fence_barrier_init();
@@ -366,9 +416,20 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_kernel(const __grid_consta
         const int qs = k % QS;
         if (k >= QS && !mbar_wait(&bar[B_QE + qs], ((k / QS) - 1) & 1, abort, st, 1)) break;
         mbar_arrive_expect_tx(&bar[B_QF + qs], L::kQ);
-        for (int at = 0; at < D / 64; ++at)
-          tma_load_4d(smem + L::q + qs * L::kQ + at * L::kAtom, &P.tmq, &bar[B_QF + qs], at * 64,
-                      itm.h, itm.I * kTile, itm.bt);
+        if (m.pair) {
+          // rows 0-63: query block qa, rows 64-127: qb (qa again when there is none)
+          const uint32_t pq = (uint32_t)m.pair_q[list_of(m, itm.bt, itm.h) * m.P + itm.I];
+          const int qa = pq & 0xffff, qb = (pq >> 16) == 0xffff ? qa : (int)(pq >> 16);
+          for (int at = 0; at < D / 64; ++at) {
+            uint8_t* dst = smem + L::q + qs * L::kQ + at * L::kAtom;
+            tma_load_4d(dst, &P.tmq64, &bar[B_QF + qs], at * 64, itm.h, qa * 64, itm.bt);
+            tma_load_4d(dst + 64 * 128, &P.tmq64, &bar[B_QF + qs], at * 64, itm.h, qb * 64, itm.bt);
+          }
+        } else {
+          for (int at = 0; at < D / 64; ++at)
+            tma_load_4d(smem + L::q + qs * L::kQ + at * L::kAtom, &P.tmq, &bar[B_QF + qs], at * 64,
+                        itm.h, itm.I * kTile, itm.bt);
+        }
         last_q = k;
         // K of tile it + 1 is requested before V of tile it
         auto load = [&](bool is_k, int it) -> bool {
@@ -377,13 +438,23 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_kernel(const __grid_consta
           uint64_t* full = &bar[(is_k ? B_KF : B_VF) + s];
           if (!mbar_wait(&bar[(is_k ? B_KE : B_VE) + s], ((gt / ns) & 1) ^ 1, abort, st, 2))
             return false;
-          int src, k0, kind, cnt;
-          wl.entry(m, it, src, k0, kind, cnt);
-          const CUtensorMap* map = is_k ? (src ? &P.tmkc : &P.tmk) : (src ? &P.tmvc : &P.tmv);
           const uint32_t dst = (is_k ? L::k0 : L::v0) + s * L::kKV;
           mbar_arrive_expect_tx(full, L::kKV);
-          for (int at = 0; at < D / 64; ++at)
-            tma_load_4d(smem + dst + at * L::kAtom, map, full, at * 64, hk, k0, itm.bt);
+          if (m.pair) {
+            int ka, kb;
+            wl.pair_entry(m, it, ka, kb);
+            const CUtensorMap* map = is_k ? &P.tmk64 : &P.tmv64;
+            for (int at = 0; at < D / 64; ++at) {
+              tma_load_4d(smem + dst + at * L::kAtom, map, full, at * 64, hk, ka, itm.bt);
+              tma_load_4d(smem + dst + at * L::kAtom + 64 * 128, map, full, at * 64, hk, kb, itm.bt);
+            }
+          } else {
+            int src, k0, kind, cnt;
+            wl.entry(m, it, src, k0, kind, cnt);
+            const CUtensorMap* map = is_k ? (src ? &P.tmkc : &P.tmk) : (src ? &P.tmvc : &P.tmv);
+            for (int at = 0; at < D / 64; ++at)
+              tma_load_4d(smem + dst + at * L::kAtom, map, full, at * 64, hk, k0, itm.bt);
+          }
           if (is_k) last_k = gt; else last_v = gt;
           return true;
         };
@@ -391,14 +462,27 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_kernel(const __grid_consta
         auto load_kv = [&](int it) -> bool {
           const int gt = g + it, s = gt % KS;
           if (!mbar_wait(&bar[B_KE + s], ((gt / KS) & 1) ^ 1, abort, st, 2)) return false;
-          int src, k0, kind, cnt;
-          wl.entry(m, it, src, k0, kind, cnt);
           mbar_arrive_expect_tx(&bar[B_KF + s], 2 * L::kKV);
-          for (int at = 0; at < D / 64; ++at) {
-            tma_load_4d(smem + L::k0 + s * L::kKV + at * L::kAtom, src ? &P.tmkc : &P.tmk,
-                        &bar[B_KF + s], at * 64, hk, k0, itm.bt);
-            tma_load_4d(smem + L::v0 + s * L::kKV + at * L::kAtom, src ? &P.tmvc : &P.tmv,
-                        &bar[B_KF + s], at * 64, hk, k0, itm.bt);
+          if (m.pair) {
+            int ka, kb;
+            wl.pair_entry(m, it, ka, kb);
+            for (int at = 0; at < D / 64; ++at) {
+              const uint32_t ko = L::k0 + s * L::kKV + at * L::kAtom;
+              const uint32_t vo = L::v0 + s * L::kKV + at * L::kAtom;
+              tma_load_4d(smem + ko, &P.tmk64, &bar[B_KF + s], at * 64, hk, ka, itm.bt);
+              tma_load_4d(smem + ko + 64 * 128, &P.tmk64, &bar[B_KF + s], at * 64, hk, kb, itm.bt);
+              tma_load_4d(smem + vo, &P.tmv64, &bar[B_KF + s], at * 64, hk, ka, itm.bt);
+              tma_load_4d(smem + vo + 64 * 128, &P.tmv64, &bar[B_KF + s], at * 64, hk, kb, itm.bt);
+            }
+          } else {
+            int src, k0, kind, cnt;
+            wl.entry(m, it, src, k0, kind, cnt);
+            for (int at = 0; at < D / 64; ++at) {
+              tma_load_4d(smem + L::k0 + s * L::kKV + at * L::kAtom, src ? &P.tmkc : &P.tmk,
+                          &bar[B_KF + s], at * 64, hk, k0, itm.bt);
+              tma_load_4d(smem + L::v0 + s * L::kKV + at * L::kAtom, src ? &P.tmvc : &P.tmv,
+                          &bar[B_KF + s], at * 64, hk, k0, itm.bt);
+            }
           }
           last_k = gt;
           return true;
@@ -415,8 +499,12 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_kernel(const __grid_consta
         if (more && m.kind == SA_MASK_GZIP) {
           // the next item's first entries, so that its first K load is not
           // held up by a list lookup
-          prefetch_l1(m.tcol + wl_next.e0);
-          prefetch_l1(m.tkind + wl_next.e0);
+          if (m.pair) {
+            prefetch_l1(m.visits + wl_next.e0);
+          } else {
+            prefetch_l1(m.tcol + wl_next.e0);
+            prefetch_l1(m.tkind + wl_next.e0);
+          }
         }
         g += wl.n;
       }
@@ -457,8 +545,12 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_kernel(const __grid_consta
         const int qs = k % QS;
         const uint32_t qa = sb + L::q + qs * L::kQ;
         if (!mbar_wait(&bar[B_QF + qs], (k / QS) & 1, abort, st, 10)) break;
-        // both halves have read the previous item's O before it is overwritten
-        bool o_free = k == 0;
+        // O buffer k % kOBufs last held item k - kOBufs: its epilogue must have
+        // read it (waited for once per item, in order, so the per-parity
+        // barrier is never two phases ahead)
+        const int kp = k - L::kOBufs;
+        const uint32_t ob = kTmemO + (uint32_t)((k % L::kOBufs) * 2 * D);
+        bool o_free = kp < 0;
         for (int it = 0; it <= n; ++it) {
           if (it < n) {
             const int gq = g + it, s = gq % KS, sb2 = gq & 1;
@@ -481,7 +573,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_kernel(const __grid_consta
           if (it >= 1) {
             const int gp = g + it - 1, s = gp % (L::kMergedKV ? KS : VS);
             if (!o_free) {
-              if (!mbar_wait(&bar[B_OF], (k - 1) & 1, abort, st, 13)) {
+              if (!mbar_wait(&bar[B_OF + (kp & 1)], (kp >> 1) & 1, abort, st, 13)) {
                 ok = false;
                 break;
               }
@@ -504,7 +596,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_kernel(const __grid_consta
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk) {
                 const uint64_t bd = smem_desc_sw128(vb + (hf * 4 + kk) * 2048, L::kAtom, 1024);
-                mma_bf16_ts(tmem + kTmemO + hf * D, pa + kk * 8, bd, kIdPV,
+                mma_bf16_ts(tmem + ob + hf * D, pa + kk * 8, bd, kIdPV,
                             (it > 1 || kk > 0) ? 1u : 0u);
               }
             }
@@ -515,9 +607,9 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_kernel(const __grid_consta
         if (!ok) break;
         if (n == 0) {
           mma_commit(&bar[B_QE + qs]);
-          if (!o_free && !mbar_wait(&bar[B_OF], (k - 1) & 1, abort, st, 13)) break;
+          if (!o_free && !mbar_wait(&bar[B_OF + (kp & 1)], (kp >> 1) & 1, abort, st, 13)) break;
         }
-        mma_commit(&bar[B_OI]);
+        mma_commit(&bar[B_OI + (k & 1)]);
         g += n;
       }
       // drain: every MMA issued above has completed
@@ -541,13 +633,15 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_kernel(const __grid_consta
     // tile entries are read one item ahead, into registers, so that no
     // global round trip sits between two items.
     WorkList wl_next;
-    uint32_t row_next = 0u;
+    uint32_t row_next = 0u, pq_next = 0u;
     int col_next = 0, kind_next = 0;
     auto fetch_head = [&](int idx) {
       const Item nx(idx, T, a.Hq, a.Bt);
       const int list = list_of(m, nx.bt, nx.h);
       wl_next.init(m, list, nx.I);
-      if (gzip) {
+      if (m.pair) {
+        pq_next = (uint32_t)m.pair_q[list * m.P + nx.I];
+      } else if (gzip) {
         int rb0, rb1;
         row_span(nx.I, rb0, rb1);
         const int nw = (rb1 - rb0 + 1) * m.words;
@@ -555,7 +649,9 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_kernel(const __grid_consta
       }
     };
     auto fetch_entries = [&]() {
-      if (gzip) {
+      if (m.pair) {
+        col_next = lane < wl_next.n ? m.visits[wl_next.e0 + lane] : 0;
+      } else if (gzip) {
         col_next = lane < wl_next.n ? m.tcol[wl_next.e0 + lane] : 0;
         kind_next = lane < wl_next.n ? m.tkind[wl_next.e0 + lane] : 0;
       }
@@ -569,7 +665,8 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_kernel(const __grid_consta
       const Item itm(idx, T, a.Hq, a.Bt);
       const int list = list_of(m, itm.bt, itm.h);
       const WorkList wl = wl_next;
-      const uint32_t row_pre = row_next;
+      const uint32_t row_pre = row_next, pq = pq_next;
+      const int pqa = pq & 0xffff, pqb = (pq >> 16) == 0xffff ? -1 : (int)(pq >> 16);
       int col_reg = col_next, kind_reg = kind_next;  // gzip: tile list entries it0 + lane
       const bool more = idx + (int)gridDim.x < n_items;
       if (more) fetch_head(idx + gridDim.x);  // in flight during this item
@@ -577,7 +674,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_kernel(const __grid_consta
       int rb0, rb1;
       row_span(itm.I, rb0, rb1);
       const int nw = (rb1 - rb0 + 1) * m.words;
-      const bool cached = gzip && nw <= kRowCacheWords;
+      const bool cached = gzip && !m.pair && nw <= kRowCacheWords;
       __syncwarp();  // the previous item's lookups are done
       if (cached) {
         const uint32_t* src = m.bits + ((int64_t)list * m.B + rb0) * m.words;
@@ -602,8 +699,12 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_kernel(const __grid_consta
       for (int it = 0; it < wl.n; ++it) {
         if (gzip && it > 0 && (it & 31) == 0) {
           const int e = it + lane;
-          col_reg = e < wl.n ? m.tcol[wl.e0 + e] : 0;
-          kind_reg = e < wl.n ? m.tkind[wl.e0 + e] : 0;
+          if (m.pair) {
+            col_reg = e < wl.n ? m.visits[wl.e0 + e] : 0;
+          } else {
+            col_reg = e < wl.n ? m.tcol[wl.e0 + e] : 0;
+            kind_reg = e < wl.n ? m.tkind[wl.e0 + e] : 0;
+          }
         }
         const int gq = g + it, slot = gq % kMaskSlots;
         if (!__all_sync(0xffffffffu, mbar_wait(&bar[B_ME + slot], ((gq / kMaskSlots) & 1) ^ 1,
@@ -622,7 +723,10 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_kernel(const __grid_consta
           wl.entry(m, it, src, kbase, kind, cnt);
         }
         uint32_t* words = mwords + slot * (kMaskSlotBytes / 4);
-        if (!gzip && src == 0) {
+        if (m.pair) {
+          pair_tile_words((uint32_t)__shfl_sync(0xffffffffu, col_reg, it & 31), pqa, pqb, lane,
+                          words);
+        } else if (!gzip && src == 0) {
           // gist near tile: the element rule was evaluated once for every head
           const uint4* from = reinterpret_cast<const uint4*>(
               P.near + ((int64_t)itm.I * P.near_nt + (kbase / kTile - itm.I + P.near_nt - 1)) * 512);
@@ -653,7 +757,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_kernel(const __grid_consta
     const int r = quarter * 32 + lane;
     const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
     const float sl2 = a.scale * 1.4426950408889634f;
-    int g = 0, k = 0, xk = 0;
+    int g = 0, k = 0;
     bool ok = true;
     int n_next = blockIdx.x < n_items ? item_tiles(m, blockIdx.x, T, a.Hq, a.Bt) : 0;
     // Every tcgen05.ld/st below is warp-collective: the branches around them
@@ -662,7 +766,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_kernel(const __grid_consta
       const Item itm(idx, T, a.Hq, a.Bt);
       const int n = n_next;
       n_next = idx + (int)gridDim.x < n_items ? item_tiles(m, idx + gridDim.x, T, a.Hq, a.Bt) : 0;
-      const int p = itm.I * kTile + r;
+      const uint32_t ob = kTmemO + (uint32_t)((k % L::kOBufs) * 2 * D);  // this item's O
       float m_run = -INFINITY, l_run = 0.f;
       for (int it = 0; it < n; ++it) {
         const int gq = g + it, s = gq & 1, slot = gq % kMaskSlots;
@@ -745,11 +849,11 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_kernel(const __grid_consta
 #pragma unroll
           for (int cc = 0; cc < D / 32; ++cc) {
             float o[32];
-            tmem_ld32(lane_addr + kTmemO + half * D + cc * 32, o);
+            tmem_ld32(lane_addr + ob + half * D + cc * 32, o);
             tmem_wait_ld();
 #pragma unroll
             for (int i = 0; i < 32; ++i) o[i] *= alpha;
-            tmem_st32(lane_addr + kTmemO + half * D + cc * 32, o);
+            tmem_st32(lane_addr + ob + half * D + cc * 32, o);
           }
         }
         l_run = l_run * alpha + rowsum;
@@ -762,35 +866,63 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_kernel(const __grid_consta
         mbar_arrive(&bar[B_PF + s]);
       }
       if (!ok) break;
-      // ------------------------------------------------------------ epilogue
-      if (!__all_sync(0xffffffffu, mbar_wait(&bar[B_OI], k & 1, abort, st, 22))) break;
-      const bool row_ok = p < a.N;
+      // hand (max, sum) to the epilogue warps; the slot of this item's parity
+      // was last read by the epilogue of item k - 2
+      if (k >= 2 && !__all_sync(0xffffffffu, mbar_wait(&bar[B_OF + (k & 1)], ((k - 2) >> 1) & 1,
+                                                        abort, st, 23)))
+        break;
+      ml[((k & 1) * 2 + half) * 128 + r] = make_float2(m_run, l_run);
+      mbar_arrive(&bar[B_ML + (k & 1)]);
+      g += n;
+    }
+  } else if (warp >= kEpiWarp0 && warp < kEpiWarp0 + kEpiThreads / 32) {
+    // ------------------------------------------------------------ epilogue
+    // Thread r owns output row r (TMEM lane r): once every MMA of the item is
+    // done and both softmax halves have left (max, sum), it merges
+    // O = (2^(m_0-m) O_0 + 2^(m_1-m) O_1) / (2^(m_0-m) l_0 + 2^(m_1-m) l_1)
+    // and stores O and LSE, while the softmax warps already work on the next
+    // item.
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
+    int k = 0;
+    int n_next = blockIdx.x < n_items ? item_tiles(m, blockIdx.x, T, a.Hq, a.Bt) : 0;
+    for (int idx = blockIdx.x; idx < n_items; idx += gridDim.x, ++k) {
+      const Item itm(idx, T, a.Hq, a.Bt);
+      const int n = n_next;
+      n_next = idx + (int)gridDim.x < n_items ? item_tiles(m, idx + gridDim.x, T, a.Hq, a.Bt) : 0;
+      // query position of this row (pair mode: rows 0-63 are query block qa,
+      // rows 64-127 block qb, which may not exist)
+      int p = itm.I * kTile + r;
+      bool row_in = true;
+      if (m.pair) {
+        const uint32_t pq = (uint32_t)m.pair_q[list_of(m, itm.bt, itm.h) * m.P + itm.I];
+        const int qb = (int)(pq >> 16);
+        p = r < 64 ? (int)(pq & 0xffff) * 64 + r : qb * 64 + (r - 64);
+        row_in = r < 64 || qb != 0xffff;
+      }
+      const bool row_ok = row_in && p < a.N;
+      if (!__all_sync(0xffffffffu, mbar_wait(&bar[B_ML + (k & 1)], (k >> 1) & 1, abort, st, 25) &&
+                                       mbar_wait(&bar[B_OI + (k & 1)], (k >> 1) & 1, abort, st, 22)))
+        break;
+      const float2 h0 = ml[((k & 1) * 2 + 0) * 128 + r], h1 = ml[((k & 1) * 2 + 1) * 128 + r];
+      const float mm = fmaxf(h0.x, h1.x);
+      const float a0 = h0.x == -INFINITY ? 0.f : ex2(h0.x - mm);
+      const float a1 = h1.x == -INFINITY ? 0.f : ex2(h1.x - mm);
+      const float l = h0.y * a0 + h1.y * a1;
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      const float c0 = a0 * inv, c1 = a1 * inv;
       __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.o) + itm.bt * a.os[0] +
-                            (int64_t)p * a.os[1] + (int64_t)itm.h * a.os[2] + half * (D / 2);
-      float mm = -INFINITY, l = 0.f;
+                            (int64_t)p * a.os[1] + (int64_t)itm.h * a.os[2];
       if (n > 0) {
-        // exchange (max, sum) with the other half of the same rows
-        ml[half * 128 + r] = make_float2(m_run, l_run);
-        mbar_arrive(&bar[B_ML]);
-        if (!__all_sync(0xffffffffu, mbar_wait(&bar[B_ML], xk & 1, abort, st, 23))) break;
-        ++xk;
-        const float2 other = ml[(half ^ 1) * 128 + r];
-        const float m0 = half ? other.x : m_run, l0 = half ? other.y : l_run;
-        const float m1 = half ? m_run : other.x, l1 = half ? l_run : other.y;
-        mm = fmaxf(m0, m1);
-        const float a0 = m0 == -INFINITY ? 0.f : ex2(m0 - mm);
-        const float a1 = m1 == -INFINITY ? 0.f : ex2(m1 - mm);
-        l = l0 * a0 + l1 * a1;
-        const float inv = l > 0.f ? 1.f / l : 0.f;
-        const float c0 = a0 * inv, c1 = a1 * inv;
+        const uint32_t ob = kTmemO + (uint32_t)((k % L::kOBufs) * 2 * D);
         tc_fence_after();
         __syncwarp();
-#pragma unroll
-        for (int cc = 0; cc < D / 64; ++cc) {  // this half's D/2 output columns
-          const uint32_t col = half * (D / 2) + cc * 32;
+#pragma unroll 1
+        for (int cc = 0; cc < D / 32; ++cc) {
           float o0[32], o1[32];
-          tmem_ld32(lane_addr + kTmemO + col, o0);  // all lanes: collective
-          tmem_ld32(lane_addr + kTmemO + D + col, o1);
+          tmem_ld32(lane_addr + ob + cc * 32, o0);  // all lanes: collective
+          tmem_ld32(lane_addr + ob + D + cc * 32, o1);
           tmem_wait_ld();
           if (row_ok) {
 #pragma unroll
@@ -809,15 +941,14 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_kernel(const __grid_consta
           }
         }
       } else if (row_ok) {
-        for (int cc = 0; cc < D / 2; cc += 8)
+        for (int cc = 0; cc < D; cc += 8)
           *reinterpret_cast<uint4*>(orow + cc) = make_uint4(0u, 0u, 0u, 0u);
       }
       tc_fence_before();
-      mbar_arrive(&bar[B_OF]);  // O may be overwritten by the next item
-      if (half == 0 && row_ok)
+      mbar_arrive(&bar[B_OF + (k & 1)]);  // O and (max, sum) of this parity may be reused
+      if (row_ok)
         a.lse[((int64_t)itm.bt * a.Hq + itm.h) * a.N + p] =
             l > 0.f ? (mm + __log2f(l)) * 0.6931471805599453f : -INFINITY;
-      g += n;
     }
   }
   tc_fence_before();
@@ -954,11 +1085,115 @@ __global__ void __launch_bounds__(128) gist_near_mask_kernel(MaskArgs m, int N, 
   }
 }
 
+// Pair mode (gzip, b = 64): the query blocks of each (sequence, class) list
+// are paired and every pair gets the ascending union of its two key-block
+// lists, two key blocks per visit ("Gzip-guided sparse attention ...", Core
+// equations: a query block sees exactly the key blocks of its mask row).
+// Blocks whose row holds more than the diagonal (literal class) or more than
+// the local window (hybrid class) are "long"; short blocks are paired first
+// and long ones after, both ascending, so that two long rows, which share
+// most of their literal key blocks, are merged with each other. Local lists
+// pair neighbours. The pairing only schedules work: every (query block, key
+// block) pair of the mask is visited exactly once whatever it is. One CTA per
+// list; pair k is handled by thread k.
+__global__ void __launch_bounds__(512) gzip_pair_kernel(MaskArgs m, int32_t* pair_q,
+                                                        int32_t* pair_ptr, int32_t* visits) {
+  extern __shared__ int32_t psh[];
+  const int l = blockIdx.x, cls = l % 3;
+  const int B = m.B, W = m.words, P = (B + 1) / 2;
+  const uint32_t* bits = m.bits + (int64_t)l * B * W;
+  int32_t* order = psh;           // [B]   pair order of the query blocks
+  int32_t* longs = psh + B;       // [B]   inclusive count of long rows
+  int32_t* vis = psh + 2 * B;     // [P]   inclusive count of visits
+  for (int i = threadIdx.x; i < B; i += blockDim.x) {
+    int len = 0;
+    for (int w = 0; w < W; ++w) len += __popc(bits[(int64_t)i * W + w]);
+    const int base = cls == SA_CLASS_LOCAL ? len : cls == SA_CLASS_LITERAL ? 1 : min(i, m.wb) + 1;
+    longs[i] = len > base ? 1 : 0;
+  }
+  __syncthreads();
+  block_inclusive_scan(longs, B, 0);
+  const int n_long = longs[B - 1], n_short = B - n_long;
+  for (int i = threadIdx.x; i < B; i += blockDim.x) {
+    const int before = i > 0 ? longs[i - 1] : 0, is_long = longs[i] - before;
+    order[is_long ? n_short + before : i - before] = i;
+  }
+  __syncthreads();
+  for (int k = threadIdx.x; k < P; k += blockDim.x) {
+    const uint32_t* ra = bits + (int64_t)order[2 * k] * W;
+    const uint32_t* rb = 2 * k + 1 < B ? bits + (int64_t)order[2 * k + 1] * W : ra;
+    int c = 0;
+    for (int w = 0; w < W; ++w) c += __popc(ra[w] | rb[w]);
+    vis[k] = (c + 1) / 2;
+  }
+  __syncthreads();
+  const int64_t region = (int64_t)B * (B + 1) / 2;
+  block_inclusive_scan(vis, P, (int32_t)(l * region));
+  if (threadIdx.x == 0) pair_ptr[(int64_t)l * (P + 1)] = (int32_t)(l * region);
+  for (int k = threadIdx.x; k < P; k += blockDim.x) {
+    pair_ptr[(int64_t)l * (P + 1) + k + 1] = vis[k];
+    const int qa = order[2 * k], qb = 2 * k + 1 < B ? order[2 * k + 1] : -1;
+    pair_q[(int64_t)l * P + k] = qa | ((qb < 0 ? 0xffff : qb) << 16);
+    const uint32_t* ra = bits + (int64_t)qa * W;
+    const uint32_t* rb = qb >= 0 ? bits + (int64_t)qb * W : nullptr;
+    int32_t* out = visits + (k > 0 ? vis[k - 1] : l * region);
+    uint32_t cur = 0u;
+    bool second = false;
+    for (int w = 0; w < W; ++w) {
+      const uint32_t a = ra[w], b = rb ? rb[w] : 0u;
+      uint32_t u = a | b;
+      while (u) {
+        const int bit = __ffs(u) - 1;
+        u &= u - 1u;
+        const uint32_t j = (uint32_t)(32 * w + bit);
+        const uint32_t sa = (a >> bit) & 1u, sb2 = (b >> bit) & 1u;
+        if (!second) {
+          cur = j | (sa << 24) | (sb2 << 25);
+        } else {
+          *out++ = (int32_t)(cur | (j << 12) | (sa << 26) | (sb2 << 27));
+        }
+        second = !second;
+      }
+    }
+    if (second) *out = (int32_t)(cur | (0xfffu << 12));
+  }
+}
+
+// Workspace of pair mode: pair_q, pair_ptr and visits of every list.
+size_t fwd_pair_workspace(int Bt, int B) {
+  const size_t lists = (size_t)Bt * 3, P = (size_t)(B + 1) / 2;
+  auto r256 = [](size_t x) { return (x + 255) / 256 * 256; };
+  return r256(lists * P * 4) + r256(lists * (P + 1) * 4) + r256(lists * ((size_t)B * (B + 1) / 2) * 4);
+}
+
 template <int D>
-static cudaError_t fwd_tc_launch(const AttnArgs& a, const MaskArgs& m, void* compact,
-                                 void* near, cudaStream_t s) {
+static cudaError_t fwd_tc_launch(const AttnArgs& a, const MaskArgs& m_in, void* compact,
+                                 void* near, void* pair_ws, cudaStream_t s) {
   FwdTcParams P;
   memset(&P, 0, sizeof(P));
+  MaskArgs m = m_in;
+  if (pair_ws != nullptr) {
+    // pair mode (gzip, b = 64): pairs and merged visit lists, then 64-row boxes
+    const int lists = a.Bt * 3, np = (m.B + 1) / 2;
+    auto r256 = [](size_t x) { return (x + 255) / 256 * 256; };
+    char* w = static_cast<char*>(pair_ws);
+    int32_t* pair_q = reinterpret_cast<int32_t*>(w);
+    int32_t* pair_ptr = reinterpret_cast<int32_t*>(w + r256((size_t)lists * np * 4));
+    int32_t* visits = reinterpret_cast<int32_t*>(reinterpret_cast<char*>(pair_ptr) +
+                                                 r256((size_t)lists * (np + 1) * 4));
+    gzip_pair_kernel<<<lists, 512, (size_t)(2 * m.B + np) * 4, s>>>(m, pair_q, pair_ptr, visits);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    m.pair = 1;
+    m.P = np;
+    m.pair_q = pair_q;
+    m.pair_ptr = pair_ptr;
+    m.visits = visits;
+    if (!make_tile_map_box(&P.tmq64, a.q, D, a.Hq, a.N, a.Bt, a.qs, 64) ||
+        !make_tile_map_box(&P.tmk64, a.k, D, a.Hkv, a.N, a.Bt, a.ks, 64) ||
+        !make_tile_map_box(&P.tmv64, a.v, D, a.Hkv, a.N, a.Bt, a.vs, 64))
+      return cudaErrorInvalidValue;
+  }
   if (!make_tile_map(&P.tmq, a.q, D, a.Hq, a.N, a.Bt, a.qs) ||
       !make_tile_map(&P.tmk, a.k, D, a.Hkv, a.N, a.Bt, a.ks) ||
       !make_tile_map(&P.tmv, a.v, D, a.Hkv, a.N, a.Bt, a.vs))
@@ -990,18 +1225,19 @@ static cudaError_t fwd_tc_launch(const AttnArgs& a, const MaskArgs& m, void* com
                                        bytes);
   if (e != cudaSuccess) return e;
   // persistent: one CTA per SM (TMEM and shared memory admit one per SM)
-  const int items = m.T * a.Hq * a.Bt;
+  const int items = (m.pair ? m.P : m.T) * a.Hq * a.Bt;
   const int grid = items < sm_count() ? items : sm_count();
   fwd_tc_kernel<D><<<dim3(grid), kThreads, bytes, s>>>(P);
   return cudaGetLastError();
 }
 
 // Gist mode only: `compact`, 2 * Bt * N * Hkv * d bf16 of workspace; `near`,
-// T * fwd_tc_near_tiles(window) * 2048 bytes.
+// T * fwd_tc_near_tiles(window) * 2048 bytes. Gzip with b = 64: `pair_ws`,
+// fwd_pair_workspace(Bt, B) bytes, selects pair mode (null: 128-row tiles).
 cudaError_t launch_fwd_tc(int d, const AttnArgs& a, const MaskArgs& m, void* compact, void* near,
-                          cudaStream_t s) {
-  if (d == 64) return fwd_tc_launch<64>(a, m, compact, near, s);
-  if (d == 128) return fwd_tc_launch<128>(a, m, compact, near, s);
+                          void* pair_ws, cudaStream_t s) {
+  if (d == 64) return fwd_tc_launch<64>(a, m, compact, near, pair_ws, s);
+  if (d == 128) return fwd_tc_launch<128>(a, m, compact, near, pair_ws, s);
   return cudaErrorInvalidValue;
 }
 

@@ -21,6 +21,18 @@ struct MaskArgs {
   // gzip
   const uint32_t* bits;     // [batch*3*B*words]
   int B, b, words;
+  int wb;                   // window w in blocks
+  // gzip, b = 64, tensor-core forward ("pair mode"): a 128-row query tile
+  // holds two 64-row query blocks and a 128-key tile two 64-key blocks.
+  // Per list l: P pairs of query blocks pair_q[l * P + k] = qa | qb << 16
+  // (qb = 0xffff: none); the visits of pair k are visits[pair_ptr[l * (P + 1)
+  // + k] .. pair_ptr[l * (P + 1) + k + 1]) (absolute), each j1 | j2 << 12 |
+  // vis << 24 with j2 = 0xfff for none and vis bits (qa sees j1, qb sees j1,
+  // qa sees j2, qb sees j2).
+  int pair, P;
+  const int32_t* pair_q;
+  const int32_t* pair_ptr;
+  const int32_t* visits;
   // gist
   const int32_t* perm;      // physical -> logical
   const uint32_t* gist_bits;

@@ -14,8 +14,9 @@ cudaError_t launch_gist_build(const sa_mask_desc&, const uint8_t*, const sa_bloc
 cudaError_t launch_fwd_simt(int dtype, int d, const AttnArgs&, const MaskArgs&, cudaStream_t);
 cudaError_t launch_bwd_simt(int dtype, int d, const AttnArgs&, const MaskArgs&, cudaStream_t);
 cudaError_t launch_fwd_tc(int d, const AttnArgs&, const MaskArgs&, void* compact, void* near,
-                          cudaStream_t);
+                          void* pair_ws, cudaStream_t);
 int fwd_tc_near_tiles(int window);
+size_t fwd_pair_workspace(int Bt, int B);
 cudaError_t launch_bwd_tc(int d, const AttnArgs&, const MaskArgs&, void* ws, cudaStream_t);
 size_t bwd_tc_workspace(int Bt, int Hq, int T);
 cudaError_t launch_decode(const sa_decode_desc&, const void*, const void*, const void*,
@@ -155,6 +156,7 @@ MaskArgs make_mask_args(const sa_mask_desc& d, const sa_block_lists& L) {
     m.b = d.block_size;
     m.B = (int)(d.seq_len / d.block_size);
     m.words = (m.B + 31) / 32;
+    m.wb = d.window;
     const int H = d.num_heads, n_loc = H / 2, n_lit = H / 4;
     for (int h = 0; h < H; ++h)
       m.head_class[h] = d.head_class ? (uint8_t)d.head_class[h]
@@ -280,12 +282,19 @@ sa_status sa_build_block_mask(const sa_mask_desc* desc, const uint8_t* d_flags,
   return cuda_status(e);
 }
 
+// The tensor-core forward pairs 64-token query blocks into 128-row tiles
+// (b = 64; block indices must fit the 12-bit fields of its visit entries).
+static bool pair_mode(const sa_mask_desc& m) {
+  return m.kind == SA_MASK_GZIP && m.block_size == 64 && m.seq_len / 64 <= 4094;
+}
+
 sa_status sa_forward_workspace_size(const sa_attn_desc* attn, const sa_mask_desc* mask,
                                     size_t* bytes) {
   sa_status st = check_attn(attn, mask);
   if (st != SA_OK) return st;
   SA_CHECK(bytes != nullptr, SA_ERR_INVALID_ARG);
   *bytes = kStatusBytes;
+  if (pair_mode(*mask)) *bytes += fwd_pair_workspace(mask->batch, (int)(mask->seq_len / 64));
   if (mask->kind == SA_MASK_GIST) {
     // tensor-core path: compacted sink/gist K and V, then the element masks of
     // every (query tile, near key tile) pair, 128 x 128 bits each
@@ -325,7 +334,8 @@ sa_status sa_forward(const sa_attn_desc* attn, const sa_mask_desc* mask, const v
     char* compact = (char*)ws + kStatusBytes;
     char* near = compact + 2 * round256((size_t)attn->batch * attn->seq_len *
                                         attn->num_kv_heads * attn->head_dim * 2);
-    return cuda_status(launch_fwd_tc(attn->head_dim, a, m, compact, near, stream));
+    void* pair_ws = pair_mode(*mask) ? (char*)ws + kStatusBytes : nullptr;
+    return cuda_status(launch_fwd_tc(attn->head_dim, a, m, compact, near, pair_ws, stream));
   }
   return cuda_status(launch_fwd_simt(attn->dtype, attn->head_dim, a, m, stream));
 }

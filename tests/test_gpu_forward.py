@@ -41,8 +41,12 @@ def gzip_case(index, batch, N, b, w, H, d, dtype, p=0.3):
     gzip_case(105, 1, 64 * 12, 64, 20, 4, 64, "fp32"),
     gzip_case(106, 2, 32 * 40, 32, 1, 8, 128, "bf16", p=0.5),
     gzip_case(107, 1, 16 * 72, 16, 4, 4, 64, "bf16", p=0.4),
+    gzip_case(108, 2, 64 * 33, 64, 1, 8, 128, "bf16", p=0.5),
+    gzip_case(109, 1, 64 * 40, 64, 3, 4, 64, "bf16", p=1.0),
+    gzip_case(110, 3, 64 * 8, 64, 0, 4, 64, "bf16", p=0.0),
 ], ids=["tiny_fp32", "b64_ragged_bf16", "b128_h6_bf16", "b16_fp32", "b256_bf16", "wide_w_fp32",
-        "b32_d128_bf16", "b16_d64_bf16"])
+        "b32_d128_bf16", "b16_d64_bf16", "b64_d128_odd_bf16", "b64_all_literal_bf16",
+        "b64_no_literal_w0_bf16"])
 @pytest.mark.parametrize("impl", list(IMPLS))
 def test_gzip_forward_small(sa, w, impl):
     if w["dtype"] == "fp32" and impl == "tensor_cores":
