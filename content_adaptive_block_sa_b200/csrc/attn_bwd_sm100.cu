@@ -6,18 +6,18 @@
 // (the training use of the method: "UniGist ...", Approach, one-pass training;
 // forward/backward latency is a metric that page names).
 //
-// A work item is one (128-key tile J, KV head, sequence); its visits are every
-// query tile I that lists J, for every query head of the KV group (the
-// transposed tile lists). The kernel is persistent: one CTA per SM walks the
+// This key-major pass computes dK and dV; dQ comes from the query-major pass
+// (attn_dq_sm100.cu), which recomputes S and dP instead of adding partial dQ
+// tiles into global memory. A work item is one (128-key tile J, KV head,
+// sequence); its visits are every query tile I that lists J, for every query
+// head of the KV group (the transposed tile lists). The kernel is persistent: one CTA per SM walks the
 // items blockIdx.x, blockIdx.x + gridDim.x, ... (early key tiles, which have
 // the longest lists, first). TMEM lanes are key rows:
 //   S^T = K_J Q_I^T (columns 0-127); each half h of the compute warps writes
 //     its bf16 P^T over the first 32 of its 64 S columns
-//   dP^T = V_J dO_I^T (columns 128-255), later reused for dQ_I = dS K_J
+//   dP^T = V_J dO_I^T (columns 128-255)
 //   dV += P^T dO_I (A = P^T from TMEM), dK += dS^T Q_I (TMEM accumulators)
-// dS^T goes to shared memory: it is the A operand of dK (key-major) and, read
-// query-major, of dQ. The dQ tile is read out of TMEM, its columns released,
-// and only then added to the fp32 dQ in global memory with vector reductions.
+// dS^T goes to shared memory: it is the A operand of dK.
 //
 // Roles (352 threads): warp 0 TMA (K, V per item; Q, LSE, D double-buffered;
 // dO single-buffered), warp 1 one thread issuing tcgen05.mma, warps 2-9 two
@@ -38,7 +38,6 @@ using namespace sm100;
 
 struct BwdTcParams {
   CUtensorMap tmq, tmk, tmv, tmdo;
-  CUtensorMap tmdq;    // fp32 dQ [Bt, N, Hq, D], box 32 x 1 x 128 x 1, 128-byte swizzle
   AttnArgs a;
   MaskArgs m;
   const float* lse2;   // [Bt, Hq, Tpad] LSE * log2(e), +inf past N
@@ -74,15 +73,11 @@ struct Layout {
 // mbarriers. KVF/KVE: K, V of the item loaded / no longer read. QF/QE: Q
 // stage (with its LSE and D rows) full / free. DOF/DOE: dO full / free. SF,
 // DPF: S^T, dP^T in TMEM. PF1: P^T written to TMEM; PF2: dS^T written to
-// shared memory. DQF/DQE: dQ in TMEM / read out. MF/ME: mask slot full /
-// read. OF: dV and dK of the item read out. HS: one compute half has staged
-// its dQ columns for the bulk reduction. DRAIN: all MMAs done.
-// QE takes two arrivals (dK done; the dQ staged in that Q stage read by the
-// bulk reduction), DQE two (each half's staging read).
+// shared memory. MF/ME: mask slot full / read. OI: every MMA of the item done.
+// OF: dV and dK of the item read out. DRAIN: all MMAs done.
 enum {
   B_KVF = 0, B_KVE = 1, B_QF = 2, B_QE = 4, B_DOF = 6, B_DOE = 7, B_SF = 8, B_DPF = 9, B_PF1 = 10,
-  B_PF2 = 11, B_DQF = 12, B_DQE = 13, B_MF = 14, B_ME = 16, B_OF = 18, B_HS = 19, B_DRAIN = 21,
-  kNumBars = 22
+  B_PF2 = 11, B_OI = 12, B_MF = 14, B_ME = 16, B_OF = 18, B_DRAIN = 21, kNumBars = 22
 };
 
 constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256;  // dK at 256 + D
@@ -94,12 +89,6 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
           "r"(smem_u32(dst)),
       "l"(src), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
-}
-
-// Bits [0, n) set, n clamped to [0, 32].
-__device__ __forceinline__ uint32_t prefix_bits(int n) {
-  const int c = min(max(n, 0), 32);
-  return (uint32_t)((1ull << c) - 1ull);
 }
 
 // Item -> (key tile J, KV head, sequence): early key tiles first.
@@ -200,8 +189,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
     mbar_init(&bar[B_KVE], 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bar[B_QF + s], 1);
-      mbar_init(&bar[B_QE + s], 2);
-      mbar_init(&bar[B_HS + s], kCompute / 2);
+      mbar_init(&bar[B_QE + s], 1);
       mbar_init(&bar[B_MF + s], 32);
       mbar_init(&bar[B_ME + s], kCompute);
     }
@@ -211,9 +199,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
     mbar_init(&bar[B_DPF], 1);
     mbar_init(&bar[B_PF1], kCompute);
     mbar_init(&bar[B_PF2], kCompute);
-    mbar_init(&bar[B_DQF], 1);
-    mbar_init(&bar[B_DQE], 2);
     mbar_init(&bar[B_OF], kCompute);
+    mbar_init(&bar[B_OI], 1);
     mbar_init(&bar[B_DRAIN], 1);
     *abort = 0;
     fence_barrier_init();
@@ -293,13 +280,12 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
       // ---------------------------------------------------------- MMA issuer
       constexpr uint32_t kIdS = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t kIdAcc = idesc_bf16_f32(128, D, false, true);  // P^T dO, dS^T Q
-      constexpr uint32_t kIdDq = idesc_bf16_f32(128, D, true, true);    // (dS^T)^T K
       int g = 0, k = 0;
       bool ok = true;
       // Per visit gt the order is: dV(gt) once P^T is written, then S^T(gt + 1)
       // (its S columns held P^T(gt), read by the dV just issued: tcgen05.mma ops
-      // of one thread run in order), dK(gt) and dQ(gt) once dS^T is written,
-      // then dP^T(gt + 1) once dQ(gt) has been read out of its columns.
+      // of one thread run in order), dK(gt) once dS^T is written, then
+      // dP^T(gt + 1) (dS^T(gt) being written means dP^T(gt) has been read).
       auto issue_s = [&](int gt) -> bool {  // S^T = K Q^T
         const int s = gt & 1;
         if (!mbar_wait(&bar[B_QF + s], (gt >> 1) & 1, abort, st, 111)) return false;
@@ -314,10 +300,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
         mma_commit(&bar[B_SF]);
         return true;
       };
-      auto issue_dp = [&](int gt) -> bool {  // dP^T = V dO^T into the columns dQ left
-        if (!mbar_wait(&bar[B_DOF], gt & 1, abort, st, 112) ||
-            (gt > 0 && !mbar_wait(&bar[B_DQE], (gt - 1) & 1, abort, st, 113)))
-          return false;
+      auto issue_dp = [&](int gt) -> bool {  // dP^T = V dO^T
+        if (!mbar_wait(&bar[B_DOF], gt & 1, abort, st, 112)) return false;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
@@ -356,7 +340,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
             ok = false;
             break;
           }
-          // dS^T in shared memory: dK += dS^T Q, dQ = dS K
+          // dS^T in shared memory: dK += dS^T Q
           if (!mbar_wait(&bar[B_PF2], gt & 1, abort, st, 117)) {
             ok = false;
             break;
@@ -371,18 +355,17 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
                      (it > 0 || kk > 0) ? 1u : 0u);
           }
           mma_commit(&bar[B_QE + s]);
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)  // K = 128 keys; A = dS^T read query-major
-            mma_bf16(tmem + kColDP, smem_desc_sw128(sb + L::dst + kk * 2048, L::kAtom, 1024),
-                     smem_desc_sw128(sb + L::k + kk * 2048, L::kAtom, 1024), kIdDq, kk > 0);
-          mma_commit(&bar[B_DQF]);
           if (more && !issue_dp(gt + 1)) {
             ok = false;
             break;
           }
         }
         if (!ok) break;
+        // an item without visits still takes its turn of OF and OI, so that
+        // OI never runs two phases ahead of the compute warps
+        if (vis.n == 0 && k > 0 && !mbar_wait(&bar[B_OF], (k - 1) & 1, abort, st, 115)) break;
         mma_commit(&bar[B_KVE]);  // every MMA of this item reading K and V is issued
+        mma_commit(&bar[B_OI]);   // dK and dV of the item complete
         g += vis.n;
       }
       mma_commit(&bar[B_DRAIN]);
@@ -485,15 +468,31 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
         tmem_ld32(lane_addr + kColS + half * 64, pv);
         tmem_ld32(lane_addr + kColS + half * 64 + 32, pv + 32);
         tmem_wait_ld();
+        // P = 2^(s * scale * log2 e - LSE * log2 e) on visible pairs: the
+        // per-column LSE four at a time (the whole warp reads the same words),
+        // packed fp32 pairs, three of every eight exponentials on the FMA pipe
         uint32_t pk[32];
+        const float2 sc = make_float2(sl2, sl2);
 #pragma unroll
-        for (int i = 0; i < 64; i += 2) {
+        for (int i4 = 0; i4 < 16; ++i4) {
+          const float4 l4 = reinterpret_cast<const float4*>(lse2)[i4];
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
-            const bool v = (mw[(i + u) >> 5] >> ((i + u) & 31)) & 1u;
-            pv[i + u] = v ? ex2(fmaf(pv[i + u], sl2, -lse2[i + u])) : 0.f;
+            const int i = 4 * i4 + 2 * u;
+            const float2 nl = u == 0 ? make_float2(-l4.x, -l4.y) : make_float2(-l4.z, -l4.w);
+            const float2 e = ffma2(make_float2(pv[i], pv[i + 1]), sc, nl);
+            float2 p;
+            if (((i >> 1) & 7) >= 5) {
+              p = exp2_poly2(e);
+            } else {
+              p.x = ex2(e.x);
+              p.y = ex2(e.y);
+            }
+            const uint32_t w = mw[i >> 5];
+            pv[i] = ((w >> (i & 31)) & 1u) ? p.x : 0.f;
+            pv[i + 1] = ((w >> ((i + 1) & 31)) & 1u) ? p.y : 0.f;
+            pk[i >> 1] = pack_bf16(pv[i], pv[i + 1]);
           }
-          pk[i >> 1] = pack_bf16(pv[i], pv[i + 1]);
         }
         // P^T (bf16 pairs) over the first 32 of this half's S columns, all read
         __syncwarp();
@@ -517,9 +516,15 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
           tmem_wait_ld();
           uint32_t dk[16];
 #pragma unroll
-          for (int c = 0; c < 32; c += 2) {
+          for (int c = 0; c < 32; c += 4) {
             const int i = c2 * 32 + c;
-            dk[c >> 1] = pack_bf16(pv[i] * (dv[c] - dlt[i]), pv[i + 1] * (dv[c + 1] - dlt[i + 1]));
+            const float4 d4 = reinterpret_cast<const float4*>(dlt)[i >> 2];
+            const float2 s0 = fmul2(make_float2(pv[i], pv[i + 1]),
+                                    fadd2(make_float2(dv[c], dv[c + 1]), make_float2(-d4.x, -d4.y)));
+            const float2 s1 = fmul2(make_float2(pv[i + 2], pv[i + 3]),
+                                    fadd2(make_float2(dv[c + 2], dv[c + 3]), make_float2(-d4.z, -d4.w)));
+            dk[c >> 1] = pack_bf16(s0.x, s0.y);
+            dk[(c >> 1) + 1] = pack_bf16(s1.x, s1.y);
           }
           const uint32_t base = sb + L::dst + half * L::kAtom;
 #pragma unroll
@@ -530,54 +535,13 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
         fence_async_shared();
         tc_fence_before();
         mbar_arrive(&bar[B_PF2]);
-        // dQ_I: TMEM lane = query row, this half's D / 2 columns, staged in
-        // fp32 (32-column chunks, 128-byte swizzle) and added to the global dQ
-        // by bulk tensor reductions. Half 0 stages in the Q stage of this
-        // visit (dK is its last reader), half 1 in the dS^T tile (dK and dQ
-        // are its last readers); both are released only once read.
-        if (!__all_sync(0xffffffffu, mbar_wait(&bar[B_DQF], gt & 1, abort, st, 123))) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        __syncwarp();
-        float dq[D / 2];
-#pragma unroll
-        for (int c = 0; c < D / 64; ++c) tmem_ld32(lane_addr + kColDP + half * (D / 2) + c * 32, dq + c * 32);
-        tmem_wait_ld();
-        tc_fence_before();
-        const uint32_t stage = half == 0 ? sb + L::q + s * L::kT : sb + L::dst;
-#pragma unroll
-        for (int c = 0; c < D / 64; ++c)
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {  // 16-byte granule j of the 128-byte row
-            const float* v = dq + c * 32 + j * 4;
-            st_shared_v4(stage + c * 16384 + r * 128 + ((j ^ (r & 7)) << 4),
-                         __float_as_uint(v[0] * a.scale), __float_as_uint(v[1] * a.scale),
-                         __float_as_uint(v[2] * a.scale), __float_as_uint(v[3] * a.scale));
-          }
-        fence_async_shared();
-        mbar_arrive(&bar[B_HS + half]);
-        if (quarter == 0 && lane == 0) {  // one thread per half issues the reductions
-          if (!mbar_wait(&bar[B_HS + half], gt & 1, abort, st, 124)) {
-            ok = false;
-          } else {
-#pragma unroll
-            for (int c = 0; c < D / 64; ++c)
-              tma_reduce_add_4d(&P.tmdq, stage + c * 16384, half * (D / 2) + c * 32, h, I * kTile,
-                                itm.bt);
-            bulk_commit_group();
-            bulk_wait_read_all();
-            if (half == 0) mbar_arrive(&bar[B_QE + s]);
-            mbar_arrive(&bar[B_DQE]);
-          }
-        }
-        if (!__all_sync(0xffffffffu, ok)) break;
       }
       if (!ok) break;
       // ------------------------------------------------------------ epilogue
-      // dK and dV of this key tile and KV head (the last dQ commit of the item
-      // followed every dV / dK MMA); fp32, this half's D / 2 columns
+      // dK and dV of this key tile and KV head once every MMA of the item is
+      // done (the next item's first dV / dK wait for OF); fp32, this half's
+      // D / 2 columns
+      if (!__all_sync(0xffffffffu, mbar_wait(&bar[B_OI], k & 1, abort, st, 125))) break;
       float* dkr = a.dk + (((int64_t)itm.bt * a.N + kq) * a.Hkv + itm.hk) * D + half * (D / 2);
       float* dvr = a.dv + (((int64_t)itm.bt * a.N + kq) * a.Hkv + itm.hk) * D + half * (D / 2);
       if (vis.n > 0) {
@@ -608,7 +572,6 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
       mbar_arrive(&bar[B_OF]);  // dV and dK may be overwritten by the next item
       g += vis.n;
     }
-    if (quarter == 0 && lane == 0) bulk_wait_all();  // the dQ reductions have landed
   }
   tc_fence_before();
   __syncthreads();
@@ -658,6 +621,8 @@ bool make_tile_map(CUtensorMap* map, const void* base, int d, int H, int N, int 
 bool make_map_4d(CUtensorMap* map, CUtensorMapDataType dtype, int ebytes, const void* base, int d,
                  int H, int N, int Bt, const int64_t* s, int box_d, int rows);
 int sm_count();
+cudaError_t launch_dq_tc(int d, const AttnArgs& a, const MaskArgs& m, const float* lse2,
+                         const float* delta, int Tpad, cudaStream_t s);
 
 template <int D>
 static cudaError_t bwd_tc_launch(const AttnArgs& a, const MaskArgs& m, void* ws, cudaStream_t s) {
@@ -667,10 +632,6 @@ static cudaError_t bwd_tc_launch(const AttnArgs& a, const MaskArgs& m, void* ws,
       !make_tile_map(&P.tmk, a.k, D, a.Hkv, a.N, a.Bt, a.ks) ||
       !make_tile_map(&P.tmv, a.v, D, a.Hkv, a.N, a.Bt, a.vs) ||
       !make_tile_map(&P.tmdo, a.dout, D, a.Hq, a.N, a.Bt, a.os))
-    return cudaErrorInvalidValue;
-  const int64_t dqs[3] = {(int64_t)a.N * a.Hq * D, (int64_t)a.Hq * D, D};  // dense fp32 dQ
-  if (!make_map_4d(&P.tmdq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.dq, D, a.Hq, a.N, a.Bt, dqs, 32,
-                   kTile))
     return cudaErrorInvalidValue;
   P.a = a;
   P.m = m;
@@ -685,7 +646,8 @@ static cudaError_t bwd_tc_launch(const AttnArgs& a, const MaskArgs& m, void* ws,
       a, lse2, delta, P.Tpad);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  e = cudaMemsetAsync(a.dq, 0, (size_t)a.Bt * a.N * a.Hq * D * sizeof(float), s);
+  // dQ: the query-major pass
+  e = launch_dq_tc(D, a, m, lse2, delta, P.Tpad, s);
   if (e != cudaSuccess) return e;
   const int bytes = (int)Layout<D>::bytes;
   e = cudaFuncSetAttribute(bwd_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);

@@ -79,4 +79,77 @@ __device__ __forceinline__ bool element_visible(const MaskArgs& m, int list, int
   return j < m.sinks || g || (i - j) < m.window;
 }
 
+// ---- visibility words of gzip tiles (forward and query-major backward)
+// Bits [0, n) set, n clamped to [0, 32] (no branch).
+__device__ __forceinline__ uint32_t prefix_bits(int n) {
+  const int c = min(max(n, 0), 32);
+  return (uint32_t)((1ull << c) - 1ull);
+}
+
+// Each set bit of e (nb bits) widened to a run of 2^lb bits (lb <= 4).
+__device__ __forceinline__ uint32_t widen_bits(uint32_t e, int lb, int nb) {
+  if (lb == 0) return e;
+  uint32_t w = 0u;
+  const uint32_t run = (1u << (1 << lb)) - 1u;
+  for (int i = 0; i < nb; ++i)
+    if ((e >> i) & 1u) w |= run << (i << lb);
+  return w;
+}
+
+// One query row as the mask warp sees it: position, logical position (gist
+// layout), in range, and its packed block bits (gzip).
+struct RowCtx {
+  int p, li;
+  bool ok;
+  const uint32_t* bits;
+};
+
+// Gzip tiles: words w = 0..3 of rows i = 0..3 of one lane (rows lane + 32 i),
+// out[w * 128 + lane + 32 i]. Same rule as tile_word, arranged so that every
+// bit-word load is issued before any of them is used: rc[i].bits always
+// points at valid words (rows past N read some row and are cleared by lim).
+__device__ __forceinline__ void gzip_tile_words(const MaskArgs& m, int lb, int N, const RowCtx* rc,
+                                                int kbase, int kind, int lane, uint32_t* out) {
+  if (kind == SA_TILE_FULL && kbase + kTile <= N) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int w = 0; w < 4; ++w) out[w * 128 + lane + 32 * i] = rc[i].ok ? 0xffffffffu : 0u;
+    return;
+  }
+  int lim[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) lim[i] = rc[i].ok ? min(rc[i].p, N - 1) : -1;
+  if (m.b >= kTile || lb >= 5) {
+    // one block bit per (row, word): the whole tile (b >= 128) or 32 columns
+    uint32_t u[4][4];
+    int jb[4];
+#pragma unroll
+    for (int w = 0; w < 4; ++w)  // clamped: columns past N are cleared by lim anyway
+      jb[w] = min(m.B - 1, m.b >= kTile ? kbase / m.b : (kbase + 32 * w) >> lb);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int w = 0; w < 4; ++w) u[i][w] = rc[i].bits[jb[w] >> 5];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        const uint32_t causal = prefix_bits(lim[i] - (kbase + 32 * w) + 1);
+        out[w * 128 + lane + 32 * i] = ((u[i][w] >> (jb[w] & 31)) & 1u) ? causal : 0u;
+      }
+    return;
+  }
+  // b < 32: 32 >> lb blocks per word, inside one bit word
+  const int nb = 32 >> lb;
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const int cw0 = kbase + 32 * w, kb = min(cw0 >> lb, m.B - 1);  // clamped as above
+      const uint32_t e = (rc[i].bits[kb >> 5] >> (kb & 31)) & prefix_bits(nb);
+      out[w * 128 + lane + 32 * i] = widen_bits(e, lb, nb) & prefix_bits(lim[i] - cw0 + 1);
+    }
+}
+
 }  // namespace sa
