@@ -97,8 +97,12 @@ class ClockSampler:
 _host_out = {}
 
 
-KERNEL_SOURCES = {"fwd_tc_kernel": "attn_fwd_sm100.cu", "bwd_tc_kernel": "attn_bwd_sm100.cu",
-                  "decode_tc_kernel": "decode_sm100.cu"}
+# the kernels whose DRAM traffic profiles/traffic.md records, and their sources; the
+# backward is reported as one unit: row prep, the query-major dQ pass and the
+# key-major dK/dV pass
+KERNEL_SOURCES = {"fwd_tc_kernel": ["attn_fwd_sm100.cu"],
+                  "backward": ["attn_bwd_sm100.cu", "attn_dq_sm100.cu"],
+                  "decode_tc_kernel": ["decode_sm100.cu"]}
 
 
 def kernel_digest(kernel):
@@ -106,7 +110,7 @@ def kernel_digest(kernel):
     import hashlib
     csrc = os.path.join(ROOT, "content_adaptive_block_sa_b200", "csrc")
     m = hashlib.sha256()
-    for f in [KERNEL_SOURCES[kernel], "sm100.cuh", "attn_mask.cuh", "sa_common.cuh"]:
+    for f in KERNEL_SOURCES[kernel] + ["sm100.cuh", "attn_mask.cuh", "sa_common.cuh"]:
         with open(os.path.join(csrc, f), "rb") as fh:
             m.update(fh.read())
     return m.hexdigest()[:16]
@@ -175,8 +179,9 @@ class GzipWorkload:
         self.pairs = pairs
         self.flops_fwd = 4.0 * d * b * b * pairs
         self.flops = self.flops_fwd * (1 + (2.5 if backward else 0))
-        # builder + forward (+ backward: row prep + key-major kernel)
-        self.kernels_per_step = 2 + (2 if backward else 0)
+        # builder + forward (+ the pairing pre-pass for 64-token blocks) (+ backward:
+        # row prep, query-major dQ pass, key-major dK/dV pass)
+        self.kernels_per_step = 2 + (1 if b == 64 else 0) + (3 if backward else 0)
         self.kernel = "fwd_tc_kernel"
         self.unit = "TFLOP/s"
 
@@ -551,7 +556,7 @@ def main():
         fwd_ach = wl.flops_fwd / (kern_ms * 1e-3) / 1e12
         if bwd_ms is not None and bwd_ms > kern_ms:  # the backward dominates the step
             ach = (wl.flops - wl.flops_fwd) / (bwd_ms * 1e-3) / 1e12
-            kname = "bwd_tc_kernel"
+            kname = "backward"
         else:
             ach, kname = fwd_ach, wl.kernel
         roof = {"bound": "tensor", "achieved": ach, "peak": bf16, "unit": "TFLOP/s",
