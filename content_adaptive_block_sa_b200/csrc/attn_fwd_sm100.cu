@@ -734,7 +734,10 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_kernel(const __grid_consta
         const float m_use = resc ? m_new : m_run;
         uint32_t pk[32];
         float2 sum2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-        if (m_use == -INFINITY) {
+        // a warp whose 32 rows see none of this half's keys (pair mode: a query
+        // block that does not list a visited key block) skips the exponentials
+        const bool warp_masked = __all_sync(0xffffffffu, (mw0 | mw1) == 0u);
+        if (m_use == -INFINITY || warp_masked) {
 #pragma unroll
           for (int i = 0; i < 32; ++i) pk[i] = 0u;
         } else {
@@ -1024,15 +1027,24 @@ __global__ void __launch_bounds__(128) gist_near_mask_kernel(MaskArgs m, int N, 
 // pair neighbours. The pairing only schedules work: every (query block, key
 // block) pair of the mask is visited exactly once whatever it is. One CTA per
 // list; pair k is handled by thread k.
+constexpr int kPairStageWords = 8192;  // bit rows staged in shared memory up to 32 KB
+
 __global__ void __launch_bounds__(512) gzip_pair_kernel(MaskArgs m, int32_t* pair_q,
                                                         int32_t* pair_ptr, int32_t* visits) {
   extern __shared__ int32_t psh[];
   const int l = blockIdx.x, cls = l % 3;
   const int B = m.B, W = m.words, P = (B + 1) / 2;
-  const uint32_t* bits = m.bits + (int64_t)l * B * W;
   int32_t* order = psh;           // [B]   pair order of the query blocks
   int32_t* longs = psh + B;       // [B]   inclusive count of long rows
   int32_t* vis = psh + 2 * B;     // [P]   inclusive count of visits
+  // the list's bit rows, staged in shared memory when the launch gave room
+  const uint32_t* bits = m.bits + (int64_t)l * B * W;
+  if (kPairStageWords > 0 && B * W <= kPairStageWords) {
+    uint32_t* staged = reinterpret_cast<uint32_t*>(psh + 2 * B + P);
+    for (int x = threadIdx.x; x < B * W; x += blockDim.x) staged[x] = bits[x];
+    bits = staged;
+    __syncthreads();
+  }
   for (int i = threadIdx.x; i < B; i += blockDim.x) {
     int len = 0;
     for (int w = 0; w < W; ++w) len += __popc(bits[(int64_t)i * W + w]);
@@ -1109,7 +1121,9 @@ static cudaError_t fwd_tc_launch(const AttnArgs& a, const MaskArgs& m_in, void* 
     int32_t* pair_ptr = reinterpret_cast<int32_t*>(w + r256((size_t)lists * np * 4));
     int32_t* visits = reinterpret_cast<int32_t*>(reinterpret_cast<char*>(pair_ptr) +
                                                  r256((size_t)lists * (np + 1) * 4));
-    gzip_pair_kernel<<<lists, 512, (size_t)(2 * m.B + np) * 4, s>>>(m, pair_q, pair_ptr, visits);
+    const int stage = m.B * m.words <= kPairStageWords ? m.B * m.words : 0;
+    gzip_pair_kernel<<<lists, 512, (size_t)(2 * m.B + np + stage) * 4, s>>>(m, pair_q, pair_ptr,
+                                                                         visits);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     m.pair = 1;

@@ -16,7 +16,8 @@
 //   vis(i, j) = j <= i and (j < sinks or gist(j) or i - j < window)
 // with FULL / MASKED / TAIL kinds.
 //
-// Gzip: one CTA builds one (sequence, class) pair; counts become absolute
+// Gzip: five CTAs per (sequence, class) pair, one per output (block CSR, block
+// CSC, bit rows, tile lists, transposed tile lists); counts become absolute
 // offsets with a block-wide scan into fixed per-pair regions, and every list
 // is filled by one warp per row (column) with its lanes over the entries.
 // Gist: four launches, one warp per 128-position tile in each (bits and
@@ -61,13 +62,20 @@ __device__ int gzip_tile_kind(const GzipBuild& p, int lb, int cls, const uint8_t
   return any ? (all ? SA_TILE_FULL : SA_TILE_MASKED) : -1;
 }
 
+// Five roles per (sequence, class) pair, one CTA each (blockIdx.y): 0 the
+// CSR block lists, 1 their transpose (CSC), 2 the packed bit rows, 3 the tile
+// lists, 4 their transpose. Every role first derives the literal prefix counts
+// and the ascending literal blocks from the flags; the block-list entries have
+// closed forms in those, so no role reads another role's output.
 __global__ void __launch_bounds__(1024) gzip_build_kernel(GzipBuild p) {
   extern __shared__ int32_t smem[];
-  const int bc = blockIdx.x, bt = bc / 3, cls = bc % 3;
+  const int bc = blockIdx.x, bt = bc / 3, cls = bc % 3, role = blockIdx.y;
   const int B = p.B;
-  int32_t* lp = smem;            // [B+1]: literals in [0, i)
-  int32_t* lit_idx = lp + B + 1;  // [B]: ascending literal blocks
-  uint8_t* f = reinterpret_cast<uint8_t*>(lit_idx + B);  // [B]
+  int32_t* lp = smem;                 // [B+1]: literals in [0, i)
+  int32_t* lit_idx = lp + B + 1;      // [B]: ascending literal blocks
+  int32_t* rp = lit_idx + B;          // [B+1]: CSR row pointers (absolute)
+  int32_t* cp = rp + B + 1;           // [B+1]: CSC column pointers (absolute)
+  uint8_t* f = reinterpret_cast<uint8_t*>(cp + B + 1);  // [B]
   for (int i = threadIdx.x; i < B; i += blockDim.x) {
     f[i] = p.flags[(int64_t)bt * B + i] ? 1 : 0;
     lp[i + 1] = f[i];
@@ -79,167 +87,198 @@ __global__ void __launch_bounds__(1024) gzip_build_kernel(GzipBuild p) {
     if (f[i]) lit_idx[lp[i]] = i;
   __syncthreads();
   const int L = lp[B], w = p.w;
-
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  const int32_t base = (int32_t)(bc * p.region);
 
-  // ---- CSR: query block i -> ascending key blocks (literal blocks below the
-  // window first, then the window lo..i; the literal class: literal blocks
-  // up to i, or i alone)
-  int32_t* rp = p.row_ptr + (int64_t)bc * (B + 1);
-  for (int i = threadIdx.x; i < B; i += blockDim.x) {
+  // Entry t of CSR row i (query block i -> ascending key blocks: literal blocks
+  // below the window first, then the window lo..i; the literal class: literal
+  // blocks up to i, or i alone).
+  auto csr_entry = [&](int i, int t) -> int {
     const int lo = max(0, i - w);
-    int cnt;
-    if (cls == SA_CLASS_LOCAL) cnt = i - lo + 1;
-    else if (cls == SA_CLASS_LITERAL) cnt = f[i] ? lp[i + 1] : 1;
-    else cnt = (i - lo + 1) + (f[i] ? lp[lo] : 0);
-    rp[i + 1] = cnt;
-  }
-  if (threadIdx.x == 0) rp[0] = (int32_t)(bc * p.region);
-  __syncthreads();
-  block_inclusive_scan(rp + 1, B, (int32_t)(bc * p.region));
-  for (int i = warp; i < B; i += nwarps) {  // one warp per row, lanes over entries
-    int32_t* out = p.col_idx + rp[i];
-    const int lo = max(0, i - w), n = rp[i + 1] - rp[i];
-    const int nlit = cls == SA_CLASS_LITERAL ? (f[i] ? n : 0)
+    const int nlit = cls == SA_CLASS_LITERAL ? (f[i] ? lp[i + 1] : 0)
                      : (cls == SA_CLASS_HYBRID && f[i] ? lp[lo] : 0);
-    for (int t = lane; t < n; t += 32)
-      out[t] = t < nlit ? lit_idx[t] : (cls == SA_CLASS_LITERAL ? i : lo + (t - nlit));
-  }
-
-  // ---- CSC: key block j -> ascending query blocks (the window j..hi, then
-  // literal blocks above it; the literal class: literal blocks from j, or j)
-  int32_t* cp = p.col_ptr + (int64_t)bc * (B + 1);
-  for (int j = threadIdx.x; j < B; j += blockDim.x) {
+    return t < nlit ? lit_idx[t] : (cls == SA_CLASS_LITERAL ? i : lo + (t - nlit));
+  };
+  // Entry t of CSC column j (key block j -> ascending query blocks: the window
+  // j..hi, then literal blocks above it; the literal class: literal blocks from
+  // j, or j).
+  auto csc_entry = [&](int j, int t) -> int {
     const int hi = min(B - 1, j + w);
-    int cnt;
-    if (cls == SA_CLASS_LOCAL) cnt = hi - j + 1;
-    else if (cls == SA_CLASS_LITERAL) cnt = f[j] ? (L - lp[j]) : 1;
-    else cnt = (hi - j + 1) + (f[j] ? (L - lp[hi + 1]) : 0);
-    cp[j + 1] = cnt;
-  }
-  if (threadIdx.x == 0) cp[0] = (int32_t)(bc * p.region);
-  __syncthreads();
-  block_inclusive_scan(cp + 1, B, (int32_t)(bc * p.region));
-  for (int j = warp; j < B; j += nwarps) {
-    int32_t* out = p.row_idx + cp[j];
-    const int hi = min(B - 1, j + w), n = cp[j + 1] - cp[j];
-    for (int t = lane; t < n; t += 32) {
-      int v;
-      if (cls == SA_CLASS_LITERAL) v = f[j] ? lit_idx[lp[j] + t] : j;
-      else v = t <= hi - j ? j + t : lit_idx[lp[hi + 1] + (t - (hi - j + 1))];
-      out[t] = v;
+    if (cls == SA_CLASS_LITERAL) return f[j] ? lit_idx[lp[j] + t] : j;
+    return t <= hi - j ? j + t : lit_idx[lp[hi + 1] + (t - (hi - j + 1))];
+  };
+  // CSR row pointers (roles 0 and 3) and CSC column pointers (roles 1 and 4)
+  if (role == 0 || role == 3) {
+    for (int i = threadIdx.x; i < B; i += blockDim.x) {
+      const int lo = max(0, i - w);
+      int cnt;
+      if (cls == SA_CLASS_LOCAL) cnt = i - lo + 1;
+      else if (cls == SA_CLASS_LITERAL) cnt = f[i] ? lp[i + 1] : 1;
+      else cnt = (i - lo + 1) + (f[i] ? lp[lo] : 0);
+      rp[i + 1] = cnt;
     }
+    if (threadIdx.x == 0) rp[0] = base;
+    __syncthreads();
+    block_inclusive_scan(rp + 1, B, base);
+  }
+  if (role == 1 || role == 4) {
+    for (int j = threadIdx.x; j < B; j += blockDim.x) {
+      const int hi = min(B - 1, j + w);
+      int cnt;
+      if (cls == SA_CLASS_LOCAL) cnt = hi - j + 1;
+      else if (cls == SA_CLASS_LITERAL) cnt = f[j] ? (L - lp[j]) : 1;
+      else cnt = (hi - j + 1) + (f[j] ? (L - lp[hi + 1]) : 0);
+      cp[j + 1] = cnt;
+    }
+    if (threadIdx.x == 0) cp[0] = base;
+    __syncthreads();
+    block_inclusive_scan(cp + 1, B, base);
   }
 
-  // ---- packed bit rows
-  uint32_t* bits = p.bits + (int64_t)bc * B * p.words;
-  for (int e = threadIdx.x; e < B * p.words; e += blockDim.x) {
-    const int i = e / p.words, k = e % p.words;
-    uint32_t word = 0;
-    for (int t = 0; t < 32; ++t) {
-      const int j = k * 32 + t;
-      if (j <= i && j < B && block_visible(cls, f, w, i, j)) word |= 1u << t;
+  if (role == 0) {  // ---- CSR
+    int32_t* rpg = p.row_ptr + (int64_t)bc * (B + 1);
+    for (int i = threadIdx.x; i <= B; i += blockDim.x) rpg[i] = rp[i];
+    for (int i = warp; i < B; i += nwarps) {  // one warp per row, lanes over entries
+      int32_t* out = p.col_idx + rp[i];
+      const int n = rp[i + 1] - rp[i];
+      for (int t = lane; t < n; t += 32) out[t] = csr_entry(i, t);
     }
-    bits[e] = word;
+    return;
+  }
+  if (role == 1) {  // ---- CSC
+    int32_t* cpg = p.col_ptr + (int64_t)bc * (B + 1);
+    for (int j = threadIdx.x; j <= B; j += blockDim.x) cpg[j] = cp[j];
+    for (int j = warp; j < B; j += nwarps) {
+      int32_t* out = p.row_idx + cp[j];
+      const int n = cp[j + 1] - cp[j];
+      for (int t = lane; t < n; t += 32) out[t] = csc_entry(j, t);
+    }
+    return;
+  }
+  if (role == 2) {  // ---- packed bit rows
+    uint32_t* bits = p.bits + (int64_t)bc * B * p.words;
+    for (int e = threadIdx.x; e < B * p.words; e += blockDim.x) {
+      const int i = e / p.words, k = e % p.words;
+      uint32_t word = 0;
+      for (int t = 0; t < 32; ++t) {
+        const int j = k * 32 + t;
+        if (j <= i && j < B && block_visible(cls, f, w, i, j)) word |= 1u << t;
+      }
+      bits[e] = word;
+    }
+    return;
   }
 
-  // ---- tile lists (CSR) and their transpose (CSC)
-  __syncthreads();  // the block lists above are read below
+  // ---- tile lists (role 3: CSR) and their transpose (role 4: CSC); the row
+  // pointers are scanned in shared memory, after the block pointers
   const int T = p.T;
-  int32_t* trp = p.trp + (int64_t)bc * (T + 1);
-  int32_t* tcp = p.tcp + (int64_t)bc * (T + 1);
+  const int32_t tbase = (int32_t)(bc * p.tregion);
+  int32_t* tp = cp + B + 1 + (B + 3) / 4;  // [T+1] (after f)
   if (p.b >= kTile) {
     // r whole tiles per block: key tile J of a visited block kb is FULL,
     // except the diagonal tile; tiles of the diagonal block past I are skipped
     const int r = p.b / kTile;
-    for (int I = threadIdx.x; I < T; I += blockDim.x) {
-      const int i = I / r;
-      trp[I + 1] = (rp[i + 1] - rp[i] - 1) * r + (I - i * r + 1);
-    }
-    if (threadIdx.x == 0) trp[0] = (int32_t)(bc * p.tregion);
-    __syncthreads();
-    block_inclusive_scan(trp + 1, T, (int32_t)(bc * p.tregion));
-    for (int I = warp; I < T; I += nwarps) {
-      // entry x of the row: block entry x / r (the diagonal block, last in
-      // the list, contributes the tiles i r .. I)
-      const int i = I / r, e0 = rp[i], ne = rp[i + 1] - e0, n = trp[I + 1] - trp[I];
-      for (int x = lane; x < n; x += 32) {
-        const int k = min(x / r, ne - 1);
-        const int J = k < ne - 1 ? p.col_idx[e0 + k] * r + (x % r) : i * r + (x - (ne - 1) * r);
-        p.tcol[trp[I] + x] = J;
-        p.tkind[trp[I] + x] = (int8_t)(J == I ? SA_TILE_MASKED : SA_TILE_FULL);
+    if (role == 3) {
+      for (int I = threadIdx.x; I < T; I += blockDim.x) {
+        const int i = I / r;
+        tp[I + 1] = (rp[i + 1] - rp[i] - 1) * r + (I - i * r + 1);
       }
-    }
-    for (int J = threadIdx.x; J < T; J += blockDim.x) {
-      const int j = J / r;
-      tcp[J + 1] = (cp[j + 1] - cp[j] - 1) * r + (j * r + r - J);
-    }
-    if (threadIdx.x == 0) tcp[0] = (int32_t)(bc * p.tregion);
-    __syncthreads();
-    block_inclusive_scan(tcp + 1, T, (int32_t)(bc * p.tregion));
-    for (int J = warp; J < T; J += nwarps) {
-      // the diagonal block, first in the column list, contributes J .. j r + r - 1
-      const int j = J / r, e0 = cp[j], n = tcp[J + 1] - tcp[J], nd = j * r + r - J;
-      for (int x = lane; x < n; x += 32) {
-        const int I = x < nd ? J + x : p.row_idx[e0 + 1 + (x - nd) / r] * r + (x - nd) % r;
-        p.trow[tcp[J] + x] = I;
-        p.tkind_t[tcp[J] + x] = (int8_t)(I == J ? SA_TILE_MASKED : SA_TILE_FULL);
+      if (threadIdx.x == 0) tp[0] = tbase;
+      __syncthreads();
+      block_inclusive_scan(tp + 1, T, tbase);
+      int32_t* trp = p.trp + (int64_t)bc * (T + 1);
+      for (int I = threadIdx.x; I <= T; I += blockDim.x) trp[I] = tp[I];
+      for (int I = warp; I < T; I += nwarps) {
+        // entry x of the row: block entry x / r (the diagonal block, last in
+        // the list, contributes the tiles i r .. I)
+        const int i = I / r, ne = rp[i + 1] - rp[i], n = tp[I + 1] - tp[I];
+        for (int x = lane; x < n; x += 32) {
+          const int k = min(x / r, ne - 1);
+          const int J = k < ne - 1 ? csr_entry(i, k) * r + (x % r) : i * r + (x - (ne - 1) * r);
+          p.tcol[tp[I] + x] = J;
+          p.tkind[tp[I] + x] = (int8_t)(J == I ? SA_TILE_MASKED : SA_TILE_FULL);
+        }
+      }
+    } else {
+      for (int J = threadIdx.x; J < T; J += blockDim.x) {
+        const int j = J / r;
+        tp[J + 1] = (cp[j + 1] - cp[j] - 1) * r + (j * r + r - J);
+      }
+      if (threadIdx.x == 0) tp[0] = tbase;
+      __syncthreads();
+      block_inclusive_scan(tp + 1, T, tbase);
+      int32_t* tcp = p.tcp + (int64_t)bc * (T + 1);
+      for (int J = threadIdx.x; J <= T; J += blockDim.x) tcp[J] = tp[J];
+      for (int J = warp; J < T; J += nwarps) {
+        // the diagonal block, first in the column list, contributes J .. j r + r - 1
+        const int j = J / r, n = tp[J + 1] - tp[J], nd = j * r + r - J;
+        for (int x = lane; x < n; x += 32) {
+          const int I = x < nd ? J + x : csc_entry(j, 1 + (x - nd) / r) * r + (x - nd) % r;
+          p.trow[tp[J] + x] = I;
+          p.tkind_t[tp[J] + x] = (int8_t)(I == J ? SA_TILE_MASKED : SA_TILE_FULL);
+        }
       }
     }
     return;
   }
-  // b < 128 (a power of two): the kind of every tile pair from the block
-  // bits; one warp per row (column), lanes over 32 candidate tiles at a time,
-  // compacted with ballots
+  // b < 128 (a power of two): the kind of every tile pair from the flags; one
+  // warp per row (column), lanes over 32 candidate tiles at a time, compacted
+  // with ballots
   const int lb = __ffs(p.b) - 1;
-  for (int I = warp; I < T; I += nwarps) {
-    int cnt = 0;
-    for (int J0 = 0; J0 <= I; J0 += 32) {
-      const int J = J0 + lane;
-      cnt += __popc(__ballot_sync(0xffffffffu, J <= I && gzip_tile_kind(p, lb, cls, f, I, J) >= 0));
-    }
-    if (lane == 0) trp[I + 1] = cnt;
-  }
-  for (int J = warp; J < T; J += nwarps) {
-    int cnt = 0;
-    for (int I0 = J; I0 < T; I0 += 32) {
-      const int I = I0 + lane;
-      cnt += __popc(__ballot_sync(0xffffffffu, I < T && gzip_tile_kind(p, lb, cls, f, I, J) >= 0));
-    }
-    if (lane == 0) tcp[J + 1] = cnt;
-  }
-  if (threadIdx.x == 0) {
-    trp[0] = (int32_t)(bc * p.tregion);
-    tcp[0] = (int32_t)(bc * p.tregion);
-  }
-  __syncthreads();
-  block_inclusive_scan(trp + 1, T, (int32_t)(bc * p.tregion));
-  block_inclusive_scan(tcp + 1, T, (int32_t)(bc * p.tregion));
   const uint32_t below = (1u << lane) - 1u;
-  for (int I = warp; I < T; I += nwarps) {
-    int n = trp[I];
-    for (int J0 = 0; J0 <= I; J0 += 32) {
-      const int J = J0 + lane;
-      const int k = J <= I ? gzip_tile_kind(p, lb, cls, f, I, J) : -1;
-      const uint32_t m = __ballot_sync(0xffffffffu, k >= 0);
-      if (k >= 0) {
-        p.tcol[n + __popc(m & below)] = J;
-        p.tkind[n + __popc(m & below)] = (int8_t)k;
+  if (role == 3) {
+    for (int I = warp; I < T; I += nwarps) {
+      int cnt = 0;
+      for (int J0 = 0; J0 <= I; J0 += 32) {
+        const int J = J0 + lane;
+        cnt += __popc(__ballot_sync(0xffffffffu, J <= I && gzip_tile_kind(p, lb, cls, f, I, J) >= 0));
       }
-      n += __popc(m);
+      if (lane == 0) tp[I + 1] = cnt;
     }
-  }
-  for (int J = warp; J < T; J += nwarps) {
-    int n = tcp[J];
-    for (int I0 = J; I0 < T; I0 += 32) {
-      const int I = I0 + lane;
-      const int k = I < T ? gzip_tile_kind(p, lb, cls, f, I, J) : -1;
-      const uint32_t m = __ballot_sync(0xffffffffu, k >= 0);
-      if (k >= 0) {
-        p.trow[n + __popc(m & below)] = I;
-        p.tkind_t[n + __popc(m & below)] = (int8_t)k;
+    if (threadIdx.x == 0) tp[0] = tbase;
+    __syncthreads();
+    block_inclusive_scan(tp + 1, T, tbase);
+    int32_t* trp = p.trp + (int64_t)bc * (T + 1);
+    for (int I = threadIdx.x; I <= T; I += blockDim.x) trp[I] = tp[I];
+    for (int I = warp; I < T; I += nwarps) {
+      int n = tp[I];
+      for (int J0 = 0; J0 <= I; J0 += 32) {
+        const int J = J0 + lane;
+        const int k = J <= I ? gzip_tile_kind(p, lb, cls, f, I, J) : -1;
+        const uint32_t m = __ballot_sync(0xffffffffu, k >= 0);
+        if (k >= 0) {
+          p.tcol[n + __popc(m & below)] = J;
+          p.tkind[n + __popc(m & below)] = (int8_t)k;
+        }
+        n += __popc(m);
       }
-      n += __popc(m);
+    }
+  } else {
+    for (int J = warp; J < T; J += nwarps) {
+      int cnt = 0;
+      for (int I0 = J; I0 < T; I0 += 32) {
+        const int I = I0 + lane;
+        cnt += __popc(__ballot_sync(0xffffffffu, I < T && gzip_tile_kind(p, lb, cls, f, I, J) >= 0));
+      }
+      if (lane == 0) tp[J + 1] = cnt;
+    }
+    if (threadIdx.x == 0) tp[0] = tbase;
+    __syncthreads();
+    block_inclusive_scan(tp + 1, T, tbase);
+    int32_t* tcp = p.tcp + (int64_t)bc * (T + 1);
+    for (int J = threadIdx.x; J <= T; J += blockDim.x) tcp[J] = tp[J];
+    for (int J = warp; J < T; J += nwarps) {
+      int n = tp[J];
+      for (int I0 = J; I0 < T; I0 += 32) {
+        const int I = I0 + lane;
+        const int k = I < T ? gzip_tile_kind(p, lb, cls, f, I, J) : -1;
+        const uint32_t m = __ballot_sync(0xffffffffu, k >= 0);
+        if (k >= 0) {
+          p.trow[n + __popc(m & below)] = I;
+          p.tkind_t[n + __popc(m & below)] = (int8_t)k;
+        }
+        n += __popc(m);
+      }
     }
   }
 }
@@ -447,13 +486,14 @@ cudaError_t launch_gzip_build(const sa_mask_desc& d, const uint8_t* flags,
   p.bits = L.bits;
   p.trp = L.tile_row_ptr; p.tcol = L.tile_col; p.tkind = L.tile_kind;
   p.tcp = L.tile_col_ptr; p.trow = L.tile_row; p.tkind_t = L.tile_kind_t;
-  const size_t smem = (size_t)(2 * p.B + 1) * 4 + p.B;
+  // lp, lit_idx, rp, cp (ints), the flags (bytes, rounded to ints), tile pointers
+  const size_t smem = ((size_t)4 * p.B + 3 + (p.B + 3) / 4 + p.T + 1) * 4;
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(gzip_build_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
   }
-  gzip_build_kernel<<<d.batch * 3, 1024, smem, s>>>(p);
+  gzip_build_kernel<<<dim3(d.batch * 3, 5), 1024, smem, s>>>(p);
   return cudaGetLastError();
 }
 
