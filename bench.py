@@ -9,6 +9,7 @@ seeded input already resident in HBM:
   gzip_64k_fwdbwd    mask build + forward + backward (batch 2, N=65536, b=128)
   gist_prefill_32k   layout build + forward    (N=32768, 32q/8kv heads)
   gist_decode_128k   one decode step           (16 seqs, 131072-token caches)
+  gist_prefill_32k_fwdbwd  layout build + forward + backward on the 32K gist inputs
 Prefill/backward workloads report visited-tile TFLOP/s (every visited block
 pair counted as a full b x b tile: 4*d*b^2 forward, 10*d*b^2 backward); the
 decode workload reports algorithmic HBM GB/s. Inputs are larger than the
@@ -252,13 +253,14 @@ class GzipWorkload:
 
 
 class GistWorkload(GzipWorkload):
-    def __init__(self, sa, torch, w):
-        self.sa, self.torch, self.backward = sa, torch, False
+    def __init__(self, sa, torch, w, backward=False):
+        self.sa, self.torch, self.backward = sa, torch, backward
         self.w = w
         N, H, Hkv, d = w["seq_len"], w["heads"], w["kv_heads"], w["head_dim"]
         self.h_in = {t: torch.from_numpy(W.qkv(w, t, 0)[None]).to(torch.bfloat16).pin_memory()
-                     for t in ("q", "k", "v")}
+                     for t in ("q", "k", "v") + (("do",) if backward else ())}
         self.q, self.k, self.v = (self.h_in[t].cuda() for t in ("q", "k", "v"))
+        self.do = self.h_in["do"].cuda() if backward else None
         self.md = sa.gist_mask(N, H, w["sinks"], w["ratio"], w["window"], gist_tail=w["gist_tail"])
         self.lists = sa.BlockLists(self.md)
         self.flags = None
@@ -268,6 +270,11 @@ class GistWorkload(GzipWorkload):
         self.lse = torch.empty(1, H, N, dtype=torch.float32, device="cuda")
         self.ad = sa.attn_desc(self.q, self.k, self.v, self.o)
         self.fws = sa.forward_workspace(self.ad, self.md)
+        if backward:
+            self.dq = torch.empty(self.q.shape, dtype=torch.float32, device="cuda")
+            self.dk = torch.empty(self.k.shape, dtype=torch.float32, device="cuda")
+            self.dv = torch.empty_like(self.dk)
+            self.bws = sa.backward_workspace(self.ad, self.md)
         self.step()
         torch.cuda.synchronize()
         T = (N + 127) // 128
@@ -275,9 +282,10 @@ class GistWorkload(GzipWorkload):
         kinds = self.lists.tile_kind.cpu().numpy()[: rp[-1]]
         width = np.where(kinds == 2, w["gist_tail"], 128)
         self.flops_fwd = 4.0 * d * H * 128 * float(width.sum())
-        self.flops = self.flops_fwd
-        # builder + sink/gist gather + near-tile masks + forward
-        self.kernels_per_step = 4
+        self.flops = self.flops_fwd * (1 + (2.5 if backward else 0))
+        # builder (4 launches) + sink/gist gather + near-tile masks + forward (+ backward:
+        # row prep, the three gist pre-passes, dQ pass, dK/dV pass, far scatter)
+        self.kernels_per_step = 7 + (7 if backward else 0)
         self.kernel = "fwd_tc_kernel"
         self.unit = "TFLOP/s"
 
@@ -285,7 +293,12 @@ class GistWorkload(GzipWorkload):
         for t, h in self.h_in.items():
             getattr(self, t).copy_(h, non_blocking=True)
         self.step()
-        return copy_out([self.o, self.lse])
+        return copy_out([self.o, self.lse] + ([self.dq, self.dk, self.dv] if self.backward else []))
+
+    def io_bytes(self):
+        h2d = sum(x.numel() * x.element_size() for x in self.h_in.values())
+        outs = [self.o, self.lse] + ([self.dq, self.dk, self.dv] if self.backward else [])
+        return h2d, sum(x.numel() * x.element_size() for x in outs)
 
     def cpu_baseline(self):
         from oracle import attention as A
@@ -300,12 +313,18 @@ class GistWorkload(GzipWorkload):
         q = W.qkv(w, "q", 0, head=0)[inv]
         k = W.qkv(w, "k", 0, head=0)[inv]
         v = W.qkv(w, "v", 0, head=0)[inv]
+        mask = lambda r: Gi.visibility(g, w["sinks"], w["window"], rows=rows[r])
         t0 = time.perf_counter()
-        A.forward(q[rows], k, v, lambda r: Gi.visibility(g, w["sinks"], w["window"], rows=rows[r]))
+        if self.backward:
+            do = W.qkv(w, "do", 0, head=0)[inv]
+            A.backward(q[rows], k, v, do[rows], mask)
+        else:
+            A.forward(q[rows], k, v, mask)
         dt = time.perf_counter() - t0
-        # algorithmic FLOPs of those rows: exact visible pairs x 4d
+        # algorithmic FLOPs of those rows: exact visible pairs x 4d (+ 10d backward)
         n_vis = int(Gi.visibility(g, w["sinks"], w["window"], rows=rows).sum())
-        return 4.0 * w["head_dim"] * n_vis / dt / 1e12, \
+        per = 4.0 + (10.0 if self.backward else 0.0)
+        return per * w["head_dim"] * n_vis / dt / 1e12, \
             "head 0, last 2048 query rows, exact visible pairs, fp64", dt
 
 
@@ -384,9 +403,12 @@ class DecodeWorkload:
 
 SMALL = {"gzip_8k": dict(batch=8), "gzip_64k_fwdbwd": dict(batch=1, heads=4, kv_heads=4),
          "gist_prefill_32k": dict(heads=8, kv_heads=2), "gist_decode_128k": dict(n_seq=4)}
+# workloads that run another one's inputs with the backward added
+FWDBWD_OF = {"gist_prefill_32k_fwdbwd": "gist_prefill_32k"}
 
 
 def workload_params(name, rank, size):
+    name = FWDBWD_OF.get(name, name)
     w = dict(W.WORKLOADS[name])
     if size == "small":
         w.update(SMALL[name])
@@ -400,7 +422,7 @@ def make(sa, torch, name, rank, size="full"):
     if name.startswith("gzip"):
         return GzipWorkload(sa, torch, w, name.endswith("fwdbwd"))
     if name.startswith("gist_prefill"):
-        return GistWorkload(sa, torch, w)
+        return GistWorkload(sa, torch, w, name.endswith("fwdbwd"))
     return DecodeWorkload(sa, torch, w)
 
 
@@ -440,7 +462,7 @@ def run_reference(args):
         return
     torch.set_num_threads(len(os.sched_getaffinity(0)))
     wl = Stub()
-    wl.w = dict(W.WORKLOADS[args.workload])
+    wl.w = dict(W.WORKLOADS[FWDBWD_OF.get(args.workload, args.workload)])
     wl.backward = args.workload.endswith("fwdbwd")
     cls = {"gzip": GzipWorkload, "gist": GistWorkload, "deco": DecodeWorkload}
     fn = cls[args.workload[:4]].cpu_baseline
@@ -475,7 +497,8 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="gzip_8k",
-                    choices=["gzip_8k", "gzip_64k_fwdbwd", "gist_prefill_32k", "gist_decode_128k"])
+                    choices=["gzip_8k", "gzip_64k_fwdbwd", "gist_prefill_32k", "gist_decode_128k",
+                             "gist_prefill_32k_fwdbwd"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--size", default="full", choices=["full", "small"],
                     help="small: fewer heads/sequences (inputs still larger than L2), for profiling")

@@ -38,6 +38,11 @@ using namespace sm100;
 
 struct BwdTcParams {
   CUtensorMap tmq, tmk, tmv, tmdo;
+  CUtensorMap tmkc, tmvc;  // gist mode: sinks + gists compacted in logical order
+  const uint32_t* near_t;  // gist mode: transposed near-tile masks
+  int near_nt;
+  float* dkf;              // gist mode: dK, dV of the compacted keys from far queries
+  float* dvf;
   AttnArgs a;
   MaskArgs m;
   const float* lse2;   // [Bt, Hq, Tpad] LSE * log2(e), +inf past N
@@ -91,40 +96,74 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
       : "memory");
 }
 
-// Item -> (key tile J, KV head, sequence): early key tiles first.
+// Item -> (key tile J, KV head, sequence): early key tiles first. The gist
+// layout has two kinds of items: "far" items (tile J of the sinks and gists
+// compacted in logical order, visited by every query tile whose window lies
+// past them) first, then "near" items (physical key tile J, visited by the
+// query tiles that hold it among their near tiles).
 struct Item {
-  int J, hk, bt;
-  __device__ Item(int idx, int Hkv, int Bt) {
+  int J, hk, bt, far;
+  __device__ Item(int idx, int Hkv, int Bt, int T, bool gist) {
+    const int per = T * Hkv * Bt;
+    far = gist && idx < per;
+    if (gist && !far) idx -= per;
     J = idx / (Hkv * Bt);
     hk = (idx % (Hkv * Bt)) % Hkv;
     bt = (idx % (Hkv * Bt)) / Hkv;
   }
 };
 
-// The visits of one item: query tile lists of every query head of the group.
+// The visits of one item, for every query head of the KV group: gzip, the
+// transposed tile list; gist near items, query tiles J .. J + nt - 1; gist far
+// items, the query tiles whose far-key prefix reaches past 128 J (a suffix of
+// the query tiles, found by bisection: far_ptr is non-decreasing).
 struct Visits {
-  int n;
-  __device__ void init(const MaskArgs& m, int bt, int hk, int rep, int J) {
+  int n, cnt, i0;
+  __device__ void init(const MaskArgs& m, const Item& itm, int rep, int nt) {
+    if (m.kind == SA_MASK_GIST) {
+      if (itm.far) {
+        int lo = 0, hi = m.T;
+        while (lo < hi) {
+          const int mid = (lo + hi) >> 1;
+          if (m.far_ptr[max(0, mid - (nt - 1))] > itm.J * kTile) hi = mid;
+          else lo = mid + 1;
+        }
+        i0 = lo;
+        cnt = m.T - lo;
+      } else {
+        i0 = itm.J;
+        cnt = min(m.T - 1, itm.J + nt - 1) - itm.J + 1;
+      }
+      n = rep * cnt;
+      return;
+    }
     n = 0;
     for (int r = 0; r < rep; ++r) {
-      const int list = list_of(m, bt, hk * rep + r);
-      n += m.tcp[list * (m.T + 1) + J + 1] - m.tcp[list * (m.T + 1) + J];
+      const int list = list_of(m, itm.bt, itm.hk * rep + r);
+      n += m.tcp[list * (m.T + 1) + itm.J + 1] - m.tcp[list * (m.T + 1) + itm.J];
     }
   }
-  __device__ static void entry(const MaskArgs& m, int bt, int hk, int rep, int J, int it, int& h,
-                               int& I, int& kind) {
+  __device__ void entry(const MaskArgs& m, const Item& itm, int rep, int it, int& h, int& I,
+                        int& kind) const {
+    if (m.kind == SA_MASK_GIST) {
+      h = itm.hk * rep + it / cnt;
+      I = i0 + it % cnt;
+      kind = SA_TILE_MASKED;
+      return;
+    }
     for (int r = 0; r < rep; ++r) {
-      const int list = list_of(m, bt, hk * rep + r);
-      const int e0 = m.tcp[list * (m.T + 1) + J], cnt = m.tcp[list * (m.T + 1) + J + 1] - e0;
-      if (it < cnt) {
-        h = hk * rep + r;
+      const int list = list_of(m, itm.bt, itm.hk * rep + r);
+      const int e0 = m.tcp[list * (m.T + 1) + itm.J];
+      const int c = m.tcp[list * (m.T + 1) + itm.J + 1] - e0;
+      if (it < c) {
+        h = itm.hk * rep + r;
         I = m.trow[e0 + it];
         kind = m.tkind_t[e0 + it];
         return;
       }
-      it -= cnt;
+      it -= c;
     }
-    h = hk * rep;
+    h = itm.hk * rep;
     I = 0;
     kind = SA_TILE_MASKED;
   }
@@ -181,7 +220,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int T = m.T;
   const int rep = a.Hq / a.Hkv;
-  const int n_items = T * a.Hkv * a.Bt;
+  const bool gist = m.kind == SA_MASK_GIST;
+  const int n_items = (gist ? 2 : 1) * T * a.Hkv * a.Bt;
   DeviceStatus* st = a.status;
 
   if (threadIdx.x == 0) {
@@ -221,26 +261,30 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
       prefetch_tmap(&P.tmk);
       prefetch_tmap(&P.tmv);
       prefetch_tmap(&P.tmdo);
+      if (gist) {
+        prefetch_tmap(&P.tmkc);
+        prefetch_tmap(&P.tmvc);
+      }
       int g = 0, k = 0, last_q = -1, last_do = -1, last_kv = -1;
       bool ok = true;
       for (int idx = blockIdx.x; ok && idx < n_items; idx += gridDim.x, ++k) {
-        const Item itm(idx, a.Hkv, a.Bt);
+        const Item itm(idx, a.Hkv, a.Bt, T, gist);
         Visits vis;
-        vis.init(m, itm.bt, itm.hk, rep, itm.J);
+        vis.init(m, itm, rep, P.near_nt);
         // K and V of the previous item are no longer read
         if (k > 0 && !mbar_wait(&bar[B_KVE], (k - 1) & 1, abort, st, 100)) break;
         mbar_arrive_expect_tx(&bar[B_KVF], 2 * L::kT);
         for (int at = 0; at < D / 64; ++at) {
-          tma_load_4d(smem + L::k + at * L::kAtom, &P.tmk, &bar[B_KVF], at * 64, itm.hk,
-                      itm.J * kTile, itm.bt);
-          tma_load_4d(smem + L::v + at * L::kAtom, &P.tmv, &bar[B_KVF], at * 64, itm.hk,
-                      itm.J * kTile, itm.bt);
+          tma_load_4d(smem + L::k + at * L::kAtom, itm.far ? &P.tmkc : &P.tmk, &bar[B_KVF], at * 64,
+                      itm.hk, itm.J * kTile, itm.bt);
+          tma_load_4d(smem + L::v + at * L::kAtom, itm.far ? &P.tmvc : &P.tmv, &bar[B_KVF], at * 64,
+                      itm.hk, itm.J * kTile, itm.bt);
         }
         last_kv = k;
         for (int it = 0; it < vis.n; ++it) {
           const int gt = g + it, s = gt & 1;
           int h, I, kind;
-          Visits::entry(m, itm.bt, itm.hk, rep, itm.J, it, h, I, kind);
+          vis.entry(m, itm, rep, it, h, I, kind);
           if (!mbar_wait(&bar[B_QE + s], ((gt >> 1) & 1) ^ 1, abort, st, 101)) {
             ok = false;
             break;
@@ -313,9 +357,9 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
         return true;
       };
       for (int idx = blockIdx.x; ok && idx < n_items; idx += gridDim.x, ++k) {
-        const Item itm(idx, a.Hkv, a.Bt);
+        const Item itm(idx, a.Hkv, a.Bt, T, gist);
         Visits vis;
-        vis.init(m, itm.bt, itm.hk, rep, itm.J);
+        vis.init(m, itm, rep, P.near_nt);
         if (vis.n > 0 && (!mbar_wait(&bar[B_KVF], k & 1, abort, st, 110) || !issue_s(g) ||
                           !issue_dp(g)))
           break;
@@ -374,12 +418,12 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
     }
   } else if (warp == kMaskWarp) {
     // ------------------------------------------------- visits and their masks
-    const int lb = m.b < kTile ? __ffs(m.b) - 1 : 0;  // b < 128 is a power of two
+    const int lb = !gist && m.b < kTile ? __ffs(m.b) - 1 : 0;  // b < 128 is a power of two
     int g = 0;
     for (int idx = blockIdx.x; idx < n_items; idx += gridDim.x) {
-      const Item itm(idx, a.Hkv, a.Bt);
+      const Item itm(idx, a.Hkv, a.Bt, T, gist);
       Visits vis;
-      vis.init(m, itm.bt, itm.hk, rep, itm.J);
+      vis.init(m, itm, rep, P.near_nt);
       bool ok = true;
       for (int it = 0; it < vis.n; ++it) {
         const int gt = g + it, s = gt & 1;
@@ -388,7 +432,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
           break;
         }
         int h, I, kind;
-        Visits::entry(m, itm.bt, itm.hk, rep, itm.J, it, h, I, kind);
+        vis.entry(m, itm, rep, it, h, I, kind);
         const int list = list_of(m, itm.bt, h);
         if (lane == 0) {
           hdr[2 * s] = h;
@@ -396,7 +440,27 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
         }
         uint32_t* words = mwords + s * (kSlotBytes / 4);
         const int q0 = I * kTile;
-        if (kind != SA_TILE_FULL && (m.b >= kTile || lb >= 5)) {
+        if (gist && !itm.far) {
+          // near tile: the transposed element masks of the pre-pass
+          const uint4* from = reinterpret_cast<const uint4*>(
+              P.near_t + ((int64_t)I * P.near_nt + (itm.J - I + P.near_nt - 1)) * 512);
+          uint4 v[4];
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) v[q4] = from[lane + 32 * q4];
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) reinterpret_cast<uint4*>(words)[lane + 32 * q4] = v[q4];
+        } else if (gist) {
+          // far tile: compacted keys below this query tile's far prefix are seen
+          // by every query row of the tile
+          const int nf = m.far_ptr[max(0, I - (P.near_nt - 1))];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const bool seen = itm.J * kTile + lane + 32 * i < nf;
+#pragma unroll
+            for (int w = 0; w < 4; ++w)
+              words[w * 128 + lane + 32 * i] = seen ? prefix_bits(a.N - (q0 + 32 * w)) : 0u;
+          }
+        } else if (kind != SA_TILE_FULL && (m.b >= kTile || lb >= 5)) {
           // one block bit per (key row, word): every load first, then the words
           uint32_t u[4][4];
           int qb[4];
@@ -444,9 +508,9 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
     int g = 0, k = 0;
     bool ok = true;
     for (int idx = blockIdx.x; ok && idx < n_items; idx += gridDim.x, ++k) {
-      const Item itm(idx, a.Hkv, a.Bt);
+      const Item itm(idx, a.Hkv, a.Bt, T, gist);
       Visits vis;
-      vis.init(m, itm.bt, itm.hk, rep, itm.J);
+      vis.init(m, itm, rep, P.near_nt);
       const int kq = itm.J * kTile + r;  // this thread's key row
       for (int it = 0; it < vis.n; ++it) {
         const int gt = g + it, s = gt & 1;
@@ -542,8 +606,12 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
       // done (the next item's first dV / dK wait for OF); fp32, this half's
       // D / 2 columns
       if (!__all_sync(0xffffffffu, mbar_wait(&bar[B_OI], k & 1, abort, st, 125))) break;
-      float* dkr = a.dk + (((int64_t)itm.bt * a.N + kq) * a.Hkv + itm.hk) * D + half * (D / 2);
-      float* dvr = a.dv + (((int64_t)itm.bt * a.N + kq) * a.Hkv + itm.hk) * D + half * (D / 2);
+      // far items write the compacted keys' far contributions (added to their
+      // rows by gist_far_scatter_kernel)
+      float* dkr = (itm.far ? P.dkf : a.dk) + (((int64_t)itm.bt * a.N + kq) * a.Hkv + itm.hk) * D +
+                   half * (D / 2);
+      float* dvr = (itm.far ? P.dvf : a.dv) + (((int64_t)itm.bt * a.N + kq) * a.Hkv + itm.hk) * D +
+                   half * (D / 2);
       if (vis.n > 0) {
         tc_fence_after();
         __syncwarp();
@@ -577,6 +645,29 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
   __syncthreads();
   tc_fence_after();
   if (warp == 0) tmem_dealloc(tmem, 512);
+}
+
+// Gist mode: adds the far contributions of every sink and gist (compacted
+// index f, key far_idx[f]) to its dK and dV row; each key appears once in the
+// compacted list, so no two threads add to the same element.
+template <int D>
+__global__ void __launch_bounds__(256) gist_far_scatter_kernel(AttnArgs a, MaskArgs m,
+                                                               const float* dkf, const float* dvf) {
+  const int f = blockIdx.x * 8 + (threadIdx.x >> 5), bt = blockIdx.y, lane = threadIdx.x & 31;
+  if (f >= m.far_ptr[m.T]) return;
+  const int64_t row = (int64_t)a.Hkv * D;
+  const int64_t src = ((int64_t)bt * a.N + f) * row, dst = ((int64_t)bt * a.N + m.far_idx[f]) * row;
+  for (int x = lane * 4; x < row; x += 32 * 4) {
+    const float4 k4 = *reinterpret_cast<const float4*>(dkf + src + x);
+    const float4 v4 = *reinterpret_cast<const float4*>(dvf + src + x);
+    float4* pk = reinterpret_cast<float4*>(a.dk + dst + x);
+    float4* pv = reinterpret_cast<float4*>(a.dv + dst + x);
+    float4 ok = *pk, ov = *pv;
+    ok.x += k4.x; ok.y += k4.y; ok.z += k4.z; ok.w += k4.w;
+    ov.x += v4.x; ov.y += v4.y; ov.z += v4.z; ov.w += v4.w;
+    *pk = ok;
+    *pv = ov;
+  }
 }
 
 // D = rowsum(dO * O) and LSE * log2(e), into padded [Bt, Hq, T*128] rows
@@ -622,7 +713,33 @@ bool make_map_4d(CUtensorMap* map, CUtensorMapDataType dtype, int ebytes, const 
                  int H, int N, int Bt, const int64_t* s, int box_d, int rows);
 int sm_count();
 cudaError_t launch_dq_tc(int d, const AttnArgs& a, const MaskArgs& m, const float* lse2,
-                         const float* delta, int Tpad, cudaStream_t s);
+                         const float* delta, int Tpad, const void* compact, const void* near,
+                         cudaStream_t s);
+cudaError_t launch_gist_prepass(int d, const AttnArgs& a, const MaskArgs& m, void* compact,
+                                void* near, void* near_t, cudaStream_t s);
+
+// Workspace bytes after the status header: lse2 and delta, [Bt, Hq, T*128]
+// fp32 each; gist mode also the compacted sink / gist K and V (bf16), the
+// near-tile masks and their transpose, and the far dK and dV of the compacted
+// keys (fp32, [Bt, N, Hkv, d] each).
+struct BwdWs {
+  size_t rows, compact, near, far;
+};
+static size_t r256b(size_t x) { return (x + 255) / 256 * 256; }
+static BwdWs bwd_ws_parts(int Bt, int Hq, int Hkv, int64_t N, int d, int T, int window, bool gist) {
+  BwdWs w{};
+  w.rows = r256b((size_t)2 * Bt * Hq * T * kTile * 4);
+  if (gist) {
+    w.compact = 2 * r256b((size_t)Bt * N * Hkv * d * 2);
+    w.near = r256b((size_t)T * fwd_tc_near_tiles(window) * 2048);
+    w.far = 2 * r256b((size_t)Bt * N * Hkv * d * 4);
+  }
+  return w;
+}
+size_t bwd_tc_workspace(int Bt, int Hq, int Hkv, int64_t N, int d, int T, int window, bool gist) {
+  const BwdWs w = bwd_ws_parts(Bt, Hq, Hkv, N, d, T, window, gist);
+  return w.rows + w.compact + 2 * w.near + w.far;
+}
 
 template <int D>
 static cudaError_t bwd_tc_launch(const AttnArgs& a, const MaskArgs& m, void* ws, cudaStream_t s) {
@@ -633,10 +750,15 @@ static cudaError_t bwd_tc_launch(const AttnArgs& a, const MaskArgs& m, void* ws,
       !make_tile_map(&P.tmv, a.v, D, a.Hkv, a.N, a.Bt, a.vs) ||
       !make_tile_map(&P.tmdo, a.dout, D, a.Hq, a.N, a.Bt, a.os))
     return cudaErrorInvalidValue;
+  P.tmkc = P.tmk;
+  P.tmvc = P.tmv;
   P.a = a;
   P.m = m;
   P.Tpad = m.T * kTile;
-  float* lse2 = static_cast<float*>(ws);
+  const bool gist = m.kind == SA_MASK_GIST;
+  const BwdWs parts = bwd_ws_parts(a.Bt, a.Hq, a.Hkv, a.N, D, m.T, m.window, gist);
+  char* base = static_cast<char*>(ws);
+  float* lse2 = reinterpret_cast<float*>(base);
   float* delta = lse2 + (size_t)a.Bt * a.Hq * P.Tpad;
   P.lse2 = lse2;
   P.delta = delta;
@@ -646,21 +768,43 @@ static cudaError_t bwd_tc_launch(const AttnArgs& a, const MaskArgs& m, void* ws,
       a, lse2, delta, P.Tpad);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  void *compact = nullptr, *near = nullptr;
+  if (gist) {
+    // the forward's pre-passes (compacted sinks / gists, near-tile masks) and
+    // the transposed masks the key-major pass reads
+    compact = base + parts.rows;
+    near = base + parts.rows + parts.compact;
+    void* near_t = static_cast<char*>(near) + parts.near;
+    float* far = reinterpret_cast<float*>(static_cast<char*>(near_t) + parts.near);
+    e = launch_gist_prepass(D, a, m, compact, near, near_t, s);
+    if (e != cudaSuccess) return e;
+    const int64_t row = (int64_t)a.Hkv * D;
+    const __nv_bfloat16* kc = static_cast<const __nv_bfloat16*>(compact);
+    const __nv_bfloat16* vc = kc + (int64_t)a.Bt * a.N * row;
+    const int64_t cs[3] = {(int64_t)a.N * row, row, D};
+    if (!make_tile_map(&P.tmkc, kc, D, a.Hkv, a.N, a.Bt, cs) ||
+        !make_tile_map(&P.tmvc, vc, D, a.Hkv, a.N, a.Bt, cs))
+      return cudaErrorInvalidValue;
+    P.near_t = static_cast<const uint32_t*>(near_t);
+    P.near_nt = fwd_tc_near_tiles(m.window);
+    P.dkf = far;
+    P.dvf = reinterpret_cast<float*>(reinterpret_cast<char*>(far) + parts.far / 2);
+  }
   // dQ: the query-major pass
-  e = launch_dq_tc(D, a, m, lse2, delta, P.Tpad, s);
+  e = launch_dq_tc(D, a, m, lse2, delta, P.Tpad, compact, near, s);
   if (e != cudaSuccess) return e;
   const int bytes = (int)Layout<D>::bytes;
   e = cudaFuncSetAttribute(bwd_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   if (e != cudaSuccess) return e;
   // persistent: one CTA per SM (TMEM and shared memory admit one)
-  const int items = m.T * a.Hkv * a.Bt;
+  const int items = (gist ? 2 : 1) * m.T * a.Hkv * a.Bt;
   const int grid = items < sm_count() ? items : sm_count();
   bwd_tc_kernel<D><<<dim3(grid), kThreads, bytes, s>>>(P);
+  e = cudaGetLastError();
+  if (e != cudaSuccess || !gist) return e;
+  gist_far_scatter_kernel<D><<<dim3((a.N + 7) / 8, a.Bt), 256, 0, s>>>(a, m, P.dkf, P.dvf);
   return cudaGetLastError();
 }
-
-// Workspace bytes after the status header: lse2 and delta, [Bt, Hq, T*128] fp32 each.
-size_t bwd_tc_workspace(int Bt, int Hq, int T) { return (size_t)2 * Bt * Hq * T * kTile * 4; }
 
 cudaError_t launch_bwd_tc(int d, const AttnArgs& a, const MaskArgs& m, void* ws, cudaStream_t s) {
   if (d == 64) return bwd_tc_launch<64>(a, m, ws, s);

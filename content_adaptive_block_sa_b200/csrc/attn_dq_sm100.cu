@@ -35,6 +35,9 @@ using namespace sm100;
 
 struct DqTcParams {
   CUtensorMap tmq, tmk, tmv, tmdo;
+  CUtensorMap tmkc, tmvc;  // gist mode: sinks + gists compacted in logical order
+  const uint32_t* near;    // gist mode: element masks of (query tile, near key tile)
+  int near_nt;
   AttnArgs a;
   MaskArgs m;
   const float* lse2;   // [Bt, Hq, Tpad] LSE * log2(e), +inf past N
@@ -86,10 +89,6 @@ struct Item {
   }
 };
 
-__device__ __forceinline__ void visits_of(const MaskArgs& m, int list, int I, int& e0, int& n) {
-  e0 = m.trp[list * (m.T + 1) + I];
-  n = m.trp[list * (m.T + 1) + I + 1] - e0;
-}
 
 }  // namespace dqk
 
@@ -152,13 +151,18 @@ __global__ void __launch_bounds__(kThreads, 1) dq_tc_kernel(const __grid_constan
       prefetch_tmap(&P.tmk);
       prefetch_tmap(&P.tmv);
       prefetch_tmap(&P.tmdo);
+      if (m.kind == SA_MASK_GIST) {
+        prefetch_tmap(&P.tmkc);
+        prefetch_tmap(&P.tmvc);
+      }
       int g = 0, k = 0, last_q = -1, last_kv = -1;
       bool ok = true;
       for (int idx = blockIdx.x; ok && idx < n_items; idx += gridDim.x, ++k) {
         const Item itm(idx, T, a.Hq, a.Bt);
         const int list = list_of(m, itm.bt, itm.h), hk = itm.h / (a.Hq / a.Hkv);
-        int e0, n;
-        visits_of(m, list, itm.I, e0, n);
+        WorkList wl;
+        wl.init(m, list, itm.I);
+        const int n = wl.n;
         const int qs = k % QS;
         if (k >= QS && !mbar_wait(&bar[B_QE + qs], ((k / QS) - 1) & 1, abort, st, 200)) break;
         mbar_arrive_expect_tx(&bar[B_QF + qs], 2 * L::kT);
@@ -174,13 +178,16 @@ __global__ void __launch_bounds__(kThreads, 1) dq_tc_kernel(const __grid_constan
             ok = false;
             break;
           }
-          const int k0 = m.tcol[e0 + it] * kTile;
+          int src, k0, kind, cnt;
+          wl.entry(m, it, src, k0, kind, cnt);
+          const CUtensorMap* mk = src ? &P.tmkc : &P.tmk;
+          const CUtensorMap* mv = src ? &P.tmvc : &P.tmv;
           mbar_arrive_expect_tx(&bar[B_KVF + s], 2 * L::kT);
           for (int at = 0; at < D / 64; ++at) {
-            tma_load_4d(smem + L::k + s * L::kT + at * L::kAtom, &P.tmk, &bar[B_KVF + s], at * 64, hk,
-                        k0, itm.bt);
-            tma_load_4d(smem + L::v + s * L::kT + at * L::kAtom, &P.tmv, &bar[B_KVF + s], at * 64, hk,
-                        k0, itm.bt);
+            tma_load_4d(smem + L::k + s * L::kT + at * L::kAtom, mk, &bar[B_KVF + s], at * 64, hk, k0,
+                        itm.bt);
+            tma_load_4d(smem + L::v + s * L::kT + at * L::kAtom, mv, &bar[B_KVF + s], at * 64, hk, k0,
+                        itm.bt);
           }
           last_kv = gt;
         }
@@ -233,8 +240,9 @@ __global__ void __launch_bounds__(kThreads, 1) dq_tc_kernel(const __grid_constan
       };
       for (int idx = blockIdx.x; ok && idx < n_items; idx += gridDim.x, ++k) {
         const Item itm(idx, T, a.Hq, a.Bt);
-        int e0, n;
-        visits_of(m, list_of(m, itm.bt, itm.h), itm.I, e0, n);
+        WorkList wl;
+        wl.init(m, list_of(m, itm.bt, itm.h), itm.I);
+        const int n = wl.n;
         const int qs = k % QS;
         const uint32_t qa = sb + L::q + 2 * qs * L::kT, da = qa + L::kT;
         if (!mbar_wait(&bar[B_QF + qs], (k / QS) & 1, abort, st, 211)) break;
@@ -281,18 +289,21 @@ __global__ void __launch_bounds__(kThreads, 1) dq_tc_kernel(const __grid_constan
     }
   } else if (warp == kMaskWarp) {
     // -------------------------------------------------------------- mask
-    const int lb = m.b < kTile ? __ffs(m.b) - 1 : 0;  // b < 128 is a power of two
+    const int gzip = m.kind == SA_MASK_GZIP;
+    const int lb = gzip && m.b < kTile ? __ffs(m.b) - 1 : 0;  // b < 128 is a power of two
     uint32_t* rcache = reinterpret_cast<uint32_t*>(smem + L::rows);
     int g = 0;
     for (int idx = blockIdx.x; idx < n_items; idx += gridDim.x) {
       const Item itm(idx, T, a.Hq, a.Bt);
       const int list = list_of(m, itm.bt, itm.h);
-      int e0, n;
-      visits_of(m, list, itm.I, e0, n);
-      // the block rows of this query tile, copied once per item when they fit
-      const int rb0 = itm.I * kTile / m.b, rb1 = min(m.B - 1, (itm.I * kTile + kTile - 1) / m.b);
+      WorkList wl;
+      wl.init(m, list, itm.I);
+      const int n = wl.n;
+      // gzip: the block rows of this query tile, copied once per item when they fit
+      const int rb0 = gzip ? itm.I * kTile / m.b : 0;
+      const int rb1 = gzip ? min(m.B - 1, (itm.I * kTile + kTile - 1) / m.b) : 0;
       const int nw = (rb1 - rb0 + 1) * m.words;
-      const bool cached = nw <= kRowWords;
+      const bool cached = gzip && nw <= kRowWords;
       __syncwarp();
       if (cached) {
         const uint32_t* src = m.bits + ((int64_t)list * m.B + rb0) * m.words;
@@ -304,18 +315,21 @@ __global__ void __launch_bounds__(kThreads, 1) dq_tc_kernel(const __grid_constan
       for (int i = 0; i < 4; ++i) {
         rc[i].p = itm.I * kTile + lane + 32 * i;
         rc[i].ok = rc[i].p < a.N;
-        const int rb = rc[i].ok ? rc[i].p / m.b : rb0;
-        rc[i].bits = cached ? rcache + (rb - rb0) * m.words
-                            : m.bits + ((int64_t)list * m.B + rb) * m.words;
+        rc[i].bits = nullptr;
+        if (gzip) {
+          const int rb = rc[i].ok ? rc[i].p / m.b : rb0;
+          rc[i].bits = cached ? rcache + (rb - rb0) * m.words
+                              : m.bits + ((int64_t)list * m.B + rb) * m.words;
+        }
         rc[i].li = 0;
       }
       bool ok = true;
       int col_reg = 0, kind_reg = 0;
       for (int it = 0; it < n; ++it) {
-        if ((it & 31) == 0) {
+        if (gzip && (it & 31) == 0) {
           const int e = it + lane;
-          col_reg = e < n ? m.tcol[e0 + e] : 0;
-          kind_reg = e < n ? m.tkind[e0 + e] : 0;
+          col_reg = e < n ? m.tcol[wl.e0 + e] : 0;
+          kind_reg = e < n ? m.tkind[wl.e0 + e] : 0;
         }
         const int gq = g + it, slot = gq % kSlots;
         if (!__all_sync(0xffffffffu, mbar_wait(&bar[B_ME + slot], ((gq / kSlots) & 1) ^ 1, abort,
@@ -323,10 +337,32 @@ __global__ void __launch_bounds__(kThreads, 1) dq_tc_kernel(const __grid_constan
           ok = false;
           break;
         }
-        const int kbase = __shfl_sync(0xffffffffu, col_reg, it & 31) * kTile;
-        const int kind = __shfl_sync(0xffffffffu, kind_reg, it & 31) == SA_TILE_FULL ? SA_TILE_FULL
-                                                                                      : SA_TILE_MASKED;
-        gzip_tile_words(m, lb, a.N, rc, kbase, kind, lane, mwords + slot * (kSlotBytes / 4));
+        uint32_t* words = mwords + slot * (kSlotBytes / 4);
+        if (gzip) {
+          const int kbase = __shfl_sync(0xffffffffu, col_reg, it & 31) * kTile;
+          const int kind = __shfl_sync(0xffffffffu, kind_reg, it & 31) == SA_TILE_FULL
+                               ? SA_TILE_FULL : SA_TILE_MASKED;
+          gzip_tile_words(m, lb, a.N, rc, kbase, kind, lane, words);
+        } else {
+          int src, kbase, kind, cnt;
+          wl.entry(m, it, src, kbase, kind, cnt);
+          if (src == 0) {
+            // gist near tile: the element rule, evaluated once for every head
+            const uint4* from = reinterpret_cast<const uint4*>(
+                P.near + ((int64_t)itm.I * P.near_nt + (kbase / kTile - itm.I + P.near_nt - 1)) * 512);
+            uint4 v[4];
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) v[q4] = from[lane + 32 * q4];
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) reinterpret_cast<uint4*>(words)[lane + 32 * q4] = v[q4];
+          } else {
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+              for (int w = 0; w < 4; ++w)
+                words[w * 128 + lane + 32 * i] = tile_word(m, 0, lb, a.N, rc[i], kbase, kind, cnt, w);
+          }
+        }
         mbar_arrive(&bar[B_MF + slot]);  // release: the words above are visible to the waiter
       }
       if (!ok) break;
@@ -343,8 +379,9 @@ __global__ void __launch_bounds__(kThreads, 1) dq_tc_kernel(const __grid_constan
     bool ok = true;
     for (int idx = blockIdx.x; ok && idx < n_items; idx += gridDim.x, ++k) {
       const Item itm(idx, T, a.Hq, a.Bt);
-      int e0, n;
-      visits_of(m, list_of(m, itm.bt, itm.h), itm.I, e0, n);
+      WorkList wl;
+      wl.init(m, list_of(m, itm.bt, itm.h), itm.I);
+      const int n = wl.n;
       const int p = itm.I * kTile + r;
       const int64_t ro = ((int64_t)itm.bt * a.Hq + itm.h) * P.Tpad + p;
       const float lse2 = P.lse2[ro], dlt = P.delta[ro];
@@ -438,7 +475,8 @@ int sm_count();
 
 template <int D>
 static cudaError_t dq_tc_launch(const AttnArgs& a, const MaskArgs& m, const float* lse2,
-                                const float* delta, int Tpad, cudaStream_t s) {
+                                const float* delta, int Tpad, const void* compact, const void* near,
+                                cudaStream_t s) {
   DqTcParams P;
   memset(&P, 0, sizeof(P));
   if (!make_tile_map(&P.tmq, a.q, D, a.Hq, a.N, a.Bt, a.qs) ||
@@ -446,6 +484,20 @@ static cudaError_t dq_tc_launch(const AttnArgs& a, const MaskArgs& m, const floa
       !make_tile_map(&P.tmv, a.v, D, a.Hkv, a.N, a.Bt, a.vs) ||
       !make_tile_map(&P.tmdo, a.dout, D, a.Hq, a.N, a.Bt, a.os))
     return cudaErrorInvalidValue;
+  P.tmkc = P.tmk;
+  P.tmvc = P.tmv;
+  if (m.kind == SA_MASK_GIST) {
+    // the compacted sink / gist K and V and the near-tile masks of the forward's pre-passes
+    const int64_t row = (int64_t)a.Hkv * D;
+    const __nv_bfloat16* kc = static_cast<const __nv_bfloat16*>(compact);
+    const __nv_bfloat16* vc = kc + (int64_t)a.Bt * a.N * row;
+    const int64_t cs[3] = {(int64_t)a.N * row, row, D};
+    if (!make_tile_map(&P.tmkc, kc, D, a.Hkv, a.N, a.Bt, cs) ||
+        !make_tile_map(&P.tmvc, vc, D, a.Hkv, a.N, a.Bt, cs))
+      return cudaErrorInvalidValue;
+    P.near = static_cast<const uint32_t*>(near);
+    P.near_nt = fwd_tc_near_tiles(m.window);
+  }
   P.a = a;
   P.m = m;
   P.lse2 = lse2;
@@ -462,11 +514,13 @@ static cudaError_t dq_tc_launch(const AttnArgs& a, const MaskArgs& m, const floa
 }
 
 // dQ of every query row (fp32, dense [Bt, N, Hq, d]), from the padded
-// LSE * log2(e) and D rows the backward's preparation kernel wrote.
+// LSE * log2(e) and D rows the backward's preparation kernel wrote. Gist mode:
+// `compact` and `near` as the forward's pre-passes leave them.
 cudaError_t launch_dq_tc(int d, const AttnArgs& a, const MaskArgs& m, const float* lse2,
-                         const float* delta, int Tpad, cudaStream_t s) {
-  if (d == 64) return dq_tc_launch<64>(a, m, lse2, delta, Tpad, s);
-  if (d == 128) return dq_tc_launch<128>(a, m, lse2, delta, Tpad, s);
+                         const float* delta, int Tpad, const void* compact, const void* near,
+                         cudaStream_t s) {
+  if (d == 64) return dq_tc_launch<64>(a, m, lse2, delta, Tpad, compact, near, s);
+  if (d == 128) return dq_tc_launch<128>(a, m, lse2, delta, Tpad, compact, near, s);
   return cudaErrorInvalidValue;
 }
 

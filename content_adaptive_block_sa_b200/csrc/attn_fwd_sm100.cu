@@ -65,69 +65,6 @@ struct FwdTcParams {
   int near_nt;
 };
 
-// Near key tiles of a query tile in gist mode: Jlo..I with
-// Jlo = I - ceil((window - 1) / 128).
-int fwd_tc_near_tiles(int window) { return (window - 1 + kTile - 1) / kTile + 1; }
-
-// Internal tile kind: only the first `cnt` columns hold keys (the last tile of
-// the compacted sink/gist keys).
-constexpr int kTileCount = 3;
-
-// The visit list of one item, the same in every role. Gzip mode: the tile list
-// of (sequence, head class, query tile). Gist mode: the dense prefix of the
-// compacted sink/gist keys that lie below the near tiles, then the near tiles
-// Jlo..I of the physical sequence, which take the element rule.
-struct WorkList {
-  int gist, e0, n, nft, nf, jlo;
-  __device__ void init(const MaskArgs& m, int list, int I) {
-    gist = m.kind == SA_MASK_GIST;
-    if (m.pair) {  // I is the pair index
-      e0 = m.pair_ptr[list * (m.P + 1) + I];
-      n = m.pair_ptr[list * (m.P + 1) + I + 1] - e0;
-      nft = nf = jlo = 0;
-    } else if (gist) {
-      jlo = max(0, I - (m.window - 1 + kTile - 1) / kTile);
-      nf = m.far_ptr[jlo];
-      nft = (nf + kTile - 1) / kTile;
-      n = nft + (I - jlo + 1);
-      e0 = 0;
-    } else {
-      e0 = m.trp[list * (m.T + 1) + I];
-      n = m.trp[list * (m.T + 1) + I + 1] - e0;
-      nft = nf = jlo = 0;
-    }
-  }
-  // pair mode: first rows of the two 64-key blocks of visit it (the second
-  // repeats the first when the visit has one block; its columns are masked)
-  __device__ void pair_entry(const MaskArgs& m, int it, int& k0a, int& k0b) const {
-    const uint32_t v = (uint32_t)m.visits[e0 + it];
-    const int j1 = v & 0xfff, j2 = (v >> 12) & 0xfff;
-    k0a = j1 * 64;
-    k0b = (j2 == 0xfff ? j1 : j2) * 64;
-  }
-  // source (0 = sequence, 1 = compacted keys), first key row, kind, valid columns
-  __device__ void entry(const MaskArgs& m, int it, int& src, int& k0, int& kind, int& cnt) const {
-    if (gist) {
-      if (it < nft) {
-        src = 1;
-        k0 = it * kTile;
-        cnt = min(kTile, nf - k0);
-        kind = cnt == kTile ? SA_TILE_FULL : kTileCount;
-      } else {
-        src = 0;
-        k0 = (jlo + it - nft) * kTile;
-        kind = SA_TILE_MASKED;
-        cnt = kTile;
-      }
-    } else {
-      src = 0;
-      k0 = m.tcol[e0 + it] * kTile;
-      kind = m.tkind[e0 + it] == SA_TILE_FULL ? SA_TILE_FULL : SA_TILE_MASKED;
-      cnt = kTile;
-    }
-  }
-};
-
 // Item -> (query tile, head, sequence): late query tiles of every head and
 // sequence first.
 struct Item {
@@ -195,33 +132,6 @@ constexpr int kEpiThreads = 128;
 constexpr int kThreads = 64 + kSoftmaxThreads + 32 + kEpiThreads;
 constexpr int kMaskWarp = 10;
 constexpr int kEpiWarp0 = 11;  // warps 11-14: epilogue (one per TMEM lane quarter)
-
-// Visibility of key columns [32w, 32w + 32) of a tile from one row, for gzip
-// tiles and compacted sink/gist tiles (gist near tiles take the element rule,
-// evaluated with the whole warp in the mask role). Gzip: the row's block bits
-// over the tile, then the causal cut ("Gzip-guided sparse attention ...", Core
-// equations: M restricted to j <= i). Compacted tiles: the first cnt columns.
-__device__ __forceinline__ uint32_t tile_word(const MaskArgs& m, int gzip, int lb, int N,
-                                              const RowCtx& rc, int kbase, int kind, int cnt,
-                                              int w) {
-  if (!rc.ok) return 0u;
-  if (!gzip) return kind == SA_TILE_FULL ? 0xffffffffu : prefix_bits(cnt - 32 * w);
-  if (kind == SA_TILE_FULL && kbase + kTile <= N) return 0xffffffffu;
-  const int cw0 = kbase + 32 * w;
-  const uint32_t causal = prefix_bits(min(rc.p, N - 1) - cw0 + 1);
-  if (causal == 0u) return 0u;
-  if (m.b >= kTile) {
-    const int jb = kbase / m.b;  // the whole key tile lies in one block
-    return ((rc.bits[jb >> 5] >> (jb & 31)) & 1u) ? causal : 0u;
-  }
-  if (lb >= 5) {
-    const int jb = cw0 >> lb;  // 32 columns lie in one block
-    return ((rc.bits[jb >> 5] >> (jb & 31)) & 1u) ? causal : 0u;
-  }
-  const int kb = cw0 >> lb, nb = 32 >> lb;  // nb blocks inside one bit word
-  const uint32_t e = (rc.bits[kb >> 5] >> (kb & 31)) & prefix_bits(nb);
-  return widen_bits(e, lb, nb) & causal;
-}
 
 // Pair mode: visibility words of one visit (v = j1 | j2 << 12 | vis << 24)
 // for rows lane + 32 i: rows 0-63 belong to query block qa, 64-127 to qb
@@ -1106,6 +1016,67 @@ size_t fwd_pair_workspace(int Bt, int B) {
   return r256(lists * P * 4) + r256(lists * (P + 1) * 4) + r256(lists * ((size_t)B * (B + 1) / 2) * 4);
 }
 
+// The same masks transposed for the key-major backward: block (I, J - I + nt
+// - 1), thread r = key row; bit c of word w tells whether key 128 J + r is
+// visible from query 128 I + 32 w + c.
+__global__ void __launch_bounds__(128) gist_near_mask_t_kernel(MaskArgs m, int N, int nt_count,
+                                                               uint32_t* near_t) {
+  const int I = blockIdx.x, nt = blockIdx.y, r = threadIdx.x;
+  const int J = I - (nt_count - 1) + nt;
+  if (J < 0) return;  // not a key tile of this query tile
+  __shared__ int li_s[kTile];
+  __shared__ int ok_s[kTile];
+  const int p = I * kTile + r;
+  li_s[r] = p < N ? m.perm[p] : 0;
+  ok_s[r] = p < N;
+  __syncthreads();
+  const int kq = J * kTile + r;
+  int lj = 0;
+  uint32_t lim = 0u;  // no key: never visible
+  if (kq < N) {
+    lj = m.perm[kq];
+    const bool always = lj < m.sinks || ((m.gist_bits[lj >> 5] >> (lj & 31)) & 1u);
+    lim = always ? 0x80000000u : (uint32_t)m.window;
+  }
+  uint32_t* out = near_t + ((int64_t)I * nt_count + nt) * 512;
+#pragma unroll 1
+  for (int w = 0; w < 4; ++w) {
+    uint32_t word = 0u;
+#pragma unroll 8
+    for (int c = 0; c < 32; ++c)
+      word |= (ok_s[32 * w + c] && (uint32_t)(li_s[32 * w + c] - lj) < lim ? 1u : 0u) << c;
+    out[w * 128 + r] = word;
+  }
+}
+
+// Gist pre-passes shared by the forward and the backward: the compacted sink /
+// gist K and V (`compact`, 2 * Bt * N * Hkv * d bf16), the near-tile masks
+// (`near`, T * fwd_tc_near_tiles(window) * 2048 bytes) and, for the key-major
+// backward, their transpose (`near_t`, same size, or null).
+template <int D>
+static cudaError_t gist_prepass(const AttnArgs& a, const MaskArgs& m, void* compact, void* near,
+                                void* near_t, cudaStream_t s) {
+  const int64_t row = (int64_t)a.Hkv * D;
+  __nv_bfloat16* kc = static_cast<__nv_bfloat16*>(compact);
+  __nv_bfloat16* vc = kc + (int64_t)a.Bt * a.N * row;
+  gist_gather_kernel<D><<<dim3((a.N + 7) / 8, a.Bt), 256, 0, s>>>(a, m, kc, vc);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int nt = fwd_tc_near_tiles(m.window);
+  gist_near_mask_kernel<<<dim3(m.T, nt), kTile, 0, s>>>(m, a.N, nt, static_cast<uint32_t*>(near));
+  e = cudaGetLastError();
+  if (e != cudaSuccess || near_t == nullptr) return e;
+  gist_near_mask_t_kernel<<<dim3(m.T, nt), kTile, 0, s>>>(m, a.N, nt, static_cast<uint32_t*>(near_t));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gist_prepass(int d, const AttnArgs& a, const MaskArgs& m, void* compact,
+                                void* near, void* near_t, cudaStream_t s) {
+  if (d == 64) return gist_prepass<64>(a, m, compact, near, near_t, s);
+  if (d == 128) return gist_prepass<128>(a, m, compact, near, near_t, s);
+  return cudaErrorInvalidValue;
+}
+
 template <int D>
 static cudaError_t fwd_tc_launch(const AttnArgs& a, const MaskArgs& m_in, void* compact,
                                  void* near, void* pair_ws, cudaStream_t s) {
@@ -1150,15 +1121,10 @@ static cudaError_t fwd_tc_launch(const AttnArgs& a, const MaskArgs& m_in, void* 
     if (!make_tile_map(&P.tmkc, kc, D, a.Hkv, a.N, a.Bt, cs) ||
         !make_tile_map(&P.tmvc, vc, D, a.Hkv, a.N, a.Bt, cs))
       return cudaErrorInvalidValue;
-    gist_gather_kernel<D><<<dim3((a.N + 7) / 8, a.Bt), 256, 0, s>>>(a, m, kc, vc);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = gist_prepass<D>(a, m, compact, near, nullptr, s);
     if (e != cudaSuccess) return e;
     P.near = static_cast<const uint32_t*>(near);
     P.near_nt = fwd_tc_near_tiles(m.window);
-    gist_near_mask_kernel<<<dim3(m.T, P.near_nt), kTile, 0, s>>>(m, a.N, P.near_nt,
-                                                               static_cast<uint32_t*>(near));
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
   }
   P.a = a;
   P.m = m;

@@ -152,4 +152,97 @@ __device__ __forceinline__ void gzip_tile_words(const MaskArgs& m, int lb, int N
     }
 }
 
+// ---- visit lists of a query tile (forward and query-major backward)
+// Near key tiles of a query tile in gist mode: Jlo..I with
+// Jlo = I - ceil((window - 1) / 128).
+__host__ __device__ inline int fwd_tc_near_tiles(int window) {
+  return (window - 1 + kTile - 1) / kTile + 1;
+}
+
+// Internal tile kind: only the first `cnt` columns hold keys (the last tile of
+// the compacted sink/gist keys).
+constexpr int kTileCount = 3;
+
+// The visit list of one item, the same in every role. Gzip mode: the tile list
+// of (sequence, head class, query tile). Gist mode: the dense prefix of the
+// compacted sink/gist keys that lie below the near tiles, then the near tiles
+// Jlo..I of the physical sequence, which take the element rule.
+struct WorkList {
+  int gist, e0, n, nft, nf, jlo;
+  __device__ void init(const MaskArgs& m, int list, int I) {
+    gist = m.kind == SA_MASK_GIST;
+    if (m.pair) {  // I is the pair index
+      e0 = m.pair_ptr[list * (m.P + 1) + I];
+      n = m.pair_ptr[list * (m.P + 1) + I + 1] - e0;
+      nft = nf = jlo = 0;
+    } else if (gist) {
+      jlo = max(0, I - (m.window - 1 + kTile - 1) / kTile);
+      nf = m.far_ptr[jlo];
+      nft = (nf + kTile - 1) / kTile;
+      n = nft + (I - jlo + 1);
+      e0 = 0;
+    } else {
+      e0 = m.trp[list * (m.T + 1) + I];
+      n = m.trp[list * (m.T + 1) + I + 1] - e0;
+      nft = nf = jlo = 0;
+    }
+  }
+  // pair mode: first rows of the two 64-key blocks of visit it (the second
+  // repeats the first when the visit has one block; its columns are masked)
+  __device__ void pair_entry(const MaskArgs& m, int it, int& k0a, int& k0b) const {
+    const uint32_t v = (uint32_t)m.visits[e0 + it];
+    const int j1 = v & 0xfff, j2 = (v >> 12) & 0xfff;
+    k0a = j1 * 64;
+    k0b = (j2 == 0xfff ? j1 : j2) * 64;
+  }
+  // source (0 = sequence, 1 = compacted keys), first key row, kind, valid columns
+  __device__ void entry(const MaskArgs& m, int it, int& src, int& k0, int& kind, int& cnt) const {
+    if (gist) {
+      if (it < nft) {
+        src = 1;
+        k0 = it * kTile;
+        cnt = min(kTile, nf - k0);
+        kind = cnt == kTile ? SA_TILE_FULL : kTileCount;
+      } else {
+        src = 0;
+        k0 = (jlo + it - nft) * kTile;
+        kind = SA_TILE_MASKED;
+        cnt = kTile;
+      }
+    } else {
+      src = 0;
+      k0 = m.tcol[e0 + it] * kTile;
+      kind = m.tkind[e0 + it] == SA_TILE_FULL ? SA_TILE_FULL : SA_TILE_MASKED;
+      cnt = kTile;
+    }
+  }
+};
+
+// Visibility of key columns [32w, 32w + 32) of a tile from one row, for gzip
+// tiles and compacted sink/gist tiles (gist near tiles take the element rule,
+// evaluated with the whole warp in the mask role). Gzip: the row's block bits
+// over the tile, then the causal cut ("Gzip-guided sparse attention ...", Core
+// equations: M restricted to j <= i). Compacted tiles: the first cnt columns.
+__device__ __forceinline__ uint32_t tile_word(const MaskArgs& m, int gzip, int lb, int N,
+                                              const RowCtx& rc, int kbase, int kind, int cnt,
+                                              int w) {
+  if (!rc.ok) return 0u;
+  if (!gzip) return kind == SA_TILE_FULL ? 0xffffffffu : prefix_bits(cnt - 32 * w);
+  if (kind == SA_TILE_FULL && kbase + kTile <= N) return 0xffffffffu;
+  const int cw0 = kbase + 32 * w;
+  const uint32_t causal = prefix_bits(min(rc.p, N - 1) - cw0 + 1);
+  if (causal == 0u) return 0u;
+  if (m.b >= kTile) {
+    const int jb = kbase / m.b;  // the whole key tile lies in one block
+    return ((rc.bits[jb >> 5] >> (jb & 31)) & 1u) ? causal : 0u;
+  }
+  if (lb >= 5) {
+    const int jb = cw0 >> lb;  // 32 columns lie in one block
+    return ((rc.bits[jb >> 5] >> (jb & 31)) & 1u) ? causal : 0u;
+  }
+  const int kb = cw0 >> lb, nb = 32 >> lb;  // nb blocks inside one bit word
+  const uint32_t e = (rc.bits[kb >> 5] >> (kb & 31)) & prefix_bits(nb);
+  return widen_bits(e, lb, nb) & causal;
+}
+
 }  // namespace sa

@@ -15,10 +15,10 @@ cudaError_t launch_fwd_simt(int dtype, int d, const AttnArgs&, const MaskArgs&, 
 cudaError_t launch_bwd_simt(int dtype, int d, const AttnArgs&, const MaskArgs&, cudaStream_t);
 cudaError_t launch_fwd_tc(int d, const AttnArgs&, const MaskArgs&, void* compact, void* near,
                           void* pair_ws, cudaStream_t);
-int fwd_tc_near_tiles(int window);
+
 size_t fwd_pair_workspace(int Bt, int B);
 cudaError_t launch_bwd_tc(int d, const AttnArgs&, const MaskArgs&, void* ws, cudaStream_t);
-size_t bwd_tc_workspace(int Bt, int Hq, int T);
+size_t bwd_tc_workspace(int Bt, int Hq, int Hkv, int64_t N, int d, int T, int window, bool gist);
 cudaError_t launch_decode(const sa_decode_desc&, const void*, const void*, const void*,
                           const void*, const void*, int32_t*, void*, float*, void*,
                           cudaStream_t);
@@ -346,7 +346,9 @@ sa_status sa_backward_workspace_size(const sa_attn_desc* attn, const sa_mask_des
   if (st != SA_OK) return st;
   SA_CHECK(bytes != nullptr, SA_ERR_INVALID_ARG);
   const size_t simt = (size_t)attn->batch * attn->num_q_heads * attn->seq_len * sizeof(float);
-  const size_t tc = bwd_tc_workspace(attn->batch, attn->num_q_heads, tiles_of(attn->seq_len));
+  const size_t tc = bwd_tc_workspace(attn->batch, attn->num_q_heads, attn->num_kv_heads,
+                                     attn->seq_len, attn->head_dim, tiles_of(attn->seq_len),
+                                     mask->window, mask->kind == SA_MASK_GIST);
   *bytes = kStatusBytes + round256(simt > tc ? simt : tc);
   return SA_OK;
 }
@@ -364,12 +366,12 @@ sa_status sa_backward(const sa_attn_desc* attn, const sa_mask_desc* mask, const 
   if (st != SA_OK) return st;
   st = check_ws(ws, ws_bytes, need);
   if (st != SA_OK) return st;
-  // tensor cores: bf16, gzip masks with b >= 4 (gist-mode gradients and fp32
+  // tensor cores: bf16, gzip masks with b >= 4 or the gist layout (fp32
   // inputs use the CUDA-core kernels)
   const void* ptrs[5] = {q, k, v, o, dout};
-  const bool tc_ok = tensor_core_ok(*attn, ptrs, 5) && mask->kind == SA_MASK_GZIP &&
-                     mask->block_size >= 4 && aligned(dq, 16) && aligned(dk, 16) &&
-                     aligned(dv, 16);
+  const bool tc_ok = tensor_core_ok(*attn, ptrs, 5) &&
+                     (mask->kind == SA_MASK_GIST || mask->block_size >= 4) && aligned(dq, 16) &&
+                     aligned(dk, 16) && aligned(dv, 16);
   const int impl = pick_impl(*attn, tc_ok);
   if (impl < 0) return SA_ERR_UNSUPPORTED;
   st = clear_status(ws, stream);

@@ -7,9 +7,11 @@ import torch
 
 import sa_workloads as W
 from oracle import attention as A
+from oracle import gist as Gi
 from oracle import gzip_mask as G
 
-from _cases import check_close, gzip_flags_oracle, gzip_flags_product, gzip_inputs, to_dev, to_np
+from _cases import (check_close, gist_layout, gzip_flags_oracle, gzip_flags_product, gzip_inputs,
+                    to_dev, to_np)
 
 pytestmark = pytest.mark.gpu
 
@@ -93,3 +95,76 @@ def test_backward_full_size(sa):
             rk, rv = A.backward_cols(q[bt, :, h], k[bt, :, h], v[bt, :, h], do[bt, :, h], keys_of, rows_of, cols)
             check_close(dk[bt, cols, h], rk, "bf16", f"dK cols b{bt} h{h}")
             check_close(dv[bt, cols, h], rv, "bf16", f"dV cols b{bt} h{h}")
+
+
+# ------------------------------------------------------------------ gist layout
+def run_gist_backward(sa, w, q, k, v, do, impl):
+    md = sa.gist_mask(w["seq_len"], w["heads"], w["sinks"], w["ratio"], w["window"],
+                      gist_tail=w.get("gist_tail", 32))
+    lists = sa.build_block_mask(md, None)
+    tq, tk, tv, tdo = (to_dev(x, "bf16") for x in (q, k, v, do))
+    o, lse = sa.forward(tq, tk, tv, md, lists)
+    dq, dk, dv = sa.backward(tq, tk, tv, o, lse, tdo, md, lists, impl=impl)
+    torch.cuda.synchronize()
+    return to_np(dq), to_np(dk), to_np(dv)
+
+
+@pytest.mark.parametrize("N,sinks,window,heads,kv_heads,d", [
+    (1000, 16, 32, 4, 2, 64), (128 * 6, 128, 128, 4, 2, 128), (2000, 130, 200, 4, 1, 128),
+    (700, 0, 300, 2, 2, 64)])
+@pytest.mark.parametrize("impl", list(IMPLS))
+def test_gist_backward_small(sa, N, sinks, window, heads, kv_heads, d, impl):
+    """Gist layout (UniGist, Approach): dQ, dK, dV in physical order against the
+    oracle in logical order; dK and dV of a KV head sum the group's query heads."""
+    w = W.scaled("gist_prefill_32k", index=400 + N + d, seq_len=N, sinks=sinks, window=window,
+                 heads=heads, kv_heads=kv_heads, head_dim=d)
+    q, k, v, do = (W.qkv(w, t, 0)[None] for t in ("q", "k", "v", "do"))  # physical order
+    dq, dk, dv = run_gist_backward(sa, w, q, k, v, do, IMPLS[impl])
+    g, perm, inv = gist_layout(N, sinks, w["ratio"])
+    vis = Gi.visibility(g, sinks, window)
+    rep = heads // kv_heads
+    rk = np.zeros((N, kv_heads, d))
+    rv = np.zeros((N, kv_heads, d))
+    for h in range(heads):
+        hk = h // rep
+        rq, rk_h, rv_h, _, _ = A.backward(q[0, inv, h], k[0, inv, hk], v[0, inv, hk], do[0, inv, h], vis)
+        check_close(dq[0, inv, h], rq, "bf16", f"dQ h{h}")
+        rk[:, hk] += rk_h
+        rv[:, hk] += rv_h
+    for hk in range(kv_heads):
+        check_close(dk[0, inv, hk], rk[:, hk], "bf16", f"dK kv{hk}")
+        check_close(dv[0, inv, hk], rv[:, hk], "bf16", f"dV kv{hk}")
+
+
+def test_gist_backward_full_size_sampled(sa):
+    """The 32K gist workload (32 query / 8 KV heads): sampled dQ rows, dK/dV of
+    sampled raw keys (seen only by the queries of their window), and the
+    identity sum_j dV_j = sum over the group's rows of dO, which holds at any size."""
+    from _cases import sample_rows
+    w = W.WORKLOADS["gist_prefill_32k"]
+    q, k, v, do = (W.qkv(w, t, 0)[None] for t in ("q", "k", "v", "do"))
+    dq, dk, dv = run_gist_backward(sa, w, q, k, v, do, 0)
+    assert all(np.isfinite(x).all() for x in (dq, dk, dv))
+    N, S, Wn = w["seq_len"], w["sinks"], w["window"]
+    rep = w["heads"] // w["kv_heads"]
+    g, perm, inv = gist_layout(N, S, w["ratio"])
+    for hk in range(w["kv_heads"]):
+        want = do[0, :, hk * rep:(hk + 1) * rep].astype(np.float64).sum((0, 1))
+        np.testing.assert_allclose(dv[0, :, hk].sum(0), want, rtol=1e-3, atol=0.5)
+    keys_of = lambda P: np.sort(inv[Gi.visible_keys(g, S, Wn, int(perm[P]))])  # ascending physical
+    for h in (0, 13, w["heads"] - 1):
+        rows = sample_rows(N, 8, seed=h)
+        rq = A.backward_rows(q[0, :, h], k[0, :, h // rep], v[0, :, h // rep], do[0, :, h], keys_of, rows)
+        check_close(dq[0, rows, h], rq, "bf16", f"dQ rows h{h}")
+    raw = [j for j in (S + 1, 5000, 16001, N - 130) if not g[j]]
+    cols = inv[np.array(raw)]
+    rows_of = lambda P: inv[np.arange(int(perm[P]), min(N, int(perm[P]) + Wn))]
+    for hk in (0, w["kv_heads"] - 1):
+        rk = np.zeros((len(cols), w["head_dim"]))
+        rv = np.zeros_like(rk)
+        for h in range(hk * rep, (hk + 1) * rep):
+            a, b = A.backward_cols(q[0, :, h], k[0, :, hk], v[0, :, hk], do[0, :, h], keys_of, rows_of, cols)
+            rk += a
+            rv += b
+        check_close(dk[0, cols, hk], rk, "bf16", f"dK raw cols kv{hk}")
+        check_close(dv[0, cols, hk], rv, "bf16", f"dV raw cols kv{hk}")
