@@ -328,7 +328,11 @@ sa_status sa_backward_workspace_size(const sa_attn_desc* attn, const sa_mask_des
  * dS = P * (dP - D), dQ = dS K * scale, dK = dS^T Q * scale.
  * o and lse must come from sa_forward with the same inputs.
  * dq fp32 dense [Bt, N, Hq, d]; dk, dv fp32 dense [Bt, N, Hkv, d] (summed over
- * the query heads of a group). */
+ * the query heads of a group). The tensor-core path (bf16, d 64 or 128, gzip
+ * masks or the gist layout) runs two passes: a query-major one for dQ (S and dP
+ * recomputed, dQ written once per row, no float atomics) and a key-major one
+ * for dK and dV; gist mode adds the far-key contributions of every sink and
+ * gist in a last scatter. Deterministic: the same inputs give the same bits. */
 sa_status sa_backward(const sa_attn_desc* attn, const sa_mask_desc* mask,
                       const void* q, const void* k, const void* v,
                       const void* o, const float* lse, const void* dout,
