@@ -17,6 +17,20 @@ Readings taken where the pages are silent:
   included); gist queries use the same rule as raw queries;
 * the gist shift acts inside each tile of ``tile`` positions: the tile's raw
   tokens keep their order and come first, its gists follow in order.
+
+Segment-wise (coarse) layout, from the same study (section 2: coarse gists
+follow all raw tokens of a segment; section 6: gist compression as
+segment-wise sparse attention with full attention inside each segment;
+appendix E: 16K input, ratio 4, 1K segments give at most 4.75K positions for
+a block to model). Readings:
+* after the sinks the sequence is a run of segments, each ``seg_len`` raw
+  tokens followed by ``seg_len / ratio`` gists (one period of
+  ``seg_len + seg_len / ratio`` positions); a ragged last segment keeps the
+  same positions;
+* a segment's own gists belong to it, so a gist sees its whole segment;
+* query i sees the sinks, every gist that is not in its future and every
+  position of its own segment up to itself: the window rule with "i - j <
+  window" replaced by "same segment".
 """
 from __future__ import annotations
 
@@ -119,3 +133,48 @@ def near_tile_start(I: int, window: int, tile: int) -> int:
     """First key tile that query tile I must visit with the element rule: for
     every key below tile * Jlo and query at or above tile * I, i - j >= window."""
     return max(0, I - (window - 1 + tile - 1) // tile)
+
+
+# ---------------------------------------------------------------- coarse layout
+def coarse_gist_flags(N: int, sinks: int, seg_len: int, ratio: int) -> np.ndarray:
+    """Gist bit of each position: the last seg_len / ratio positions of every
+    period of seg_len + seg_len / ratio positions after the sinks."""
+    assert seg_len % ratio == 0
+    period = seg_len + seg_len // ratio
+    p = np.arange(N)
+    return (p >= sinks) & ((p - sinks) % period >= seg_len)
+
+
+def segment_ids(N: int, sinks: int, seg_len: int, ratio: int) -> np.ndarray:
+    """Segment of each position (-1 for the sinks)."""
+    period = seg_len + seg_len // ratio
+    p = np.arange(N)
+    return np.where(p < sinks, -1, (p - sinks) // period)
+
+
+def coarse_visibility(is_gist, seg, sinks: int, rows=None) -> np.ndarray:
+    """vis[i, j] = j <= i and (j < sinks or gist(j) or seg(i) == seg(j))."""
+    g = np.asarray(is_gist, bool)
+    sg = np.asarray(seg)
+    N = len(g)
+    i = (np.arange(N) if rows is None else np.asarray(rows))[:, None]
+    j = np.arange(N)[None, :]
+    return (j <= i) & ((j < sinks) | g[None, :] | (sg[i] == sg[None, :]))
+
+
+def coarse_visible_keys(is_gist, seg, sinks: int, i: int) -> np.ndarray:
+    """Logical key positions visible from query i under the coarse rule."""
+    return np.nonzero(coarse_visibility(is_gist, seg, sinks, rows=[i])[0])[0]
+
+
+def coarse_near_tile_start(I: int, sinks: int, seg_len: int, ratio: int, tile: int) -> int:
+    """First key tile query tile I visits with the element rule: the tile that
+    holds the start of the segment of the tile's first row (I itself while that
+    row is a sink: everything below it is a sink). Keys below it are sinks or
+    earlier segments' positions, seen by the whole query tile exactly when they
+    are sinks or gists."""
+    p = I * tile
+    if p < sinks:
+        return I
+    period = seg_len + seg_len // ratio
+    return (sinks + (p - sinks) // period * period) // tile

@@ -122,3 +122,94 @@ def test_far_prefix_covers_exactly_the_visible_keys_outside_the_near_tiles(N, si
         assert vis[:, cols].all()
         assert np.array_equal(np.sort(perm[far_idx[: far_ptr[Jlo]]]), cols)
     assert far_ptr[-1] == len(far_idx) == sinks + g[sinks:].sum()
+
+
+# ---------------------------------------------------------------- coarse layout
+def _coarse_vis_by_scanning(g, sinks):
+    """Visibility from the gist flags alone: a segment starts at the first raw
+    token after the sinks or after a run of gists; query i sees the sinks, the
+    gists before it, and every position from its segment's start to itself."""
+    N = len(g)
+    vis = np.zeros((N, N), bool)
+    for i in range(N):
+        if i < sinks:
+            vis[i, : i + 1] = True
+            continue
+        s = i  # back to the segment's start: a raw token after a gist, or the sinks' end
+        while s > sinks and not (g[s - 1] and not g[s]):
+            s -= 1
+        for j in range(i + 1):
+            vis[i, j] = j < sinks or g[j] or j >= s
+    return vis
+
+
+def test_coarse_flags_closed_form():
+    g = Gi.coarse_gist_flags(20480, 0, 1024, 4)
+    assert g.sum() == 16 * 256
+    for s in range(16):
+        assert not g[s * 1280: s * 1280 + 1024].any() and g[s * 1280 + 1024:(s + 1) * 1280].all()
+    seg = Gi.segment_ids(20480, 0, 1024, 4)
+    assert np.array_equal(np.bincount(seg), np.full(16, 1280))
+    # sinks are not part of any segment
+    assert (Gi.segment_ids(300, 7, 40, 4)[:7] == -1).all()
+
+
+def test_coarse_max_block_length_matches_page():
+    gold = GOLD["segment_wise_max_length"]
+    L, r, n_in = gold["segment"], gold["ratio"], gold["input_tokens"]
+    nseg = n_in // L
+    N = nseg * (L + L // r)
+    g = Gi.coarse_gist_flags(N, 0, L, r)
+    seg = Gi.segment_ids(N, 0, L, r)
+    raw = np.nonzero(~g)[0]
+    counts = Gi.coarse_visibility(g, seg, 0, rows=raw[-L:]).sum(1)  # last segment's raw tokens
+    assert counts.max() == gold["max_positions"] == (n_in - L) // r + L
+    # every raw query: earlier segments' gists plus its segment's raw tokens up to itself
+    rows = raw[:: 97]
+    want = seg[rows] * (L // r) + (rows - seg[rows] * (L + L // r)) + 1
+    assert np.array_equal(Gi.coarse_visibility(g, seg, 0, rows=rows).sum(1), want)
+
+
+@pytest.mark.parametrize("N,sinks,L,r", [(300, 7, 40, 4), (257, 0, 16, 8), (190, 33, 20, 2)])
+def test_coarse_visibility_matches_scan_from_flags(N, sinks, L, r):
+    g = Gi.coarse_gist_flags(N, sinks, L, r)
+    seg = Gi.segment_ids(N, sinks, L, r)
+    assert np.array_equal(Gi.coarse_visibility(g, seg, sinks), _coarse_vis_by_scanning(g, sinks))
+
+
+def test_coarse_single_segment_is_dense_causal():
+    N = 180
+    g = Gi.coarse_gist_flags(N, 5, 160, 4)  # 5 sinks, one segment of 200 positions
+    seg = Gi.segment_ids(N, 5, 160, 4)
+    assert np.array_equal(Gi.coarse_visibility(g, seg, 5), np.tril(np.ones((N, N), bool)))
+
+
+@pytest.mark.parametrize("N,sinks,L,r", [(3000, 128, 1024, 4), (2500, 5, 96, 4), (1300, 300, 200, 8),
+                                         (900, 0, 64, 2)])
+def test_coarse_far_prefix_covers_exactly_the_visible_keys_outside_the_near_tiles(N, sinks, L, r):
+    g = Gi.coarse_gist_flags(N, sinks, L, r)
+    seg = Gi.segment_ids(N, sinks, L, r)
+    perm = Gi.shift_permutation(g, 128)
+    far_idx, far_ptr = Gi.always_visible_keys(g, sinks, perm, 128)
+    period = L + L // r
+    for I in range((N + 127) // 128):
+        Jlo = Gi.coarse_near_tile_start(I, sinks, L, r, 128)
+        assert 0 <= I - Jlo <= (period + 126) // 128
+        rows = np.arange(I * 128, min(N, I * 128 + 128))
+        vis = Gi.coarse_visibility(g, seg, sinks, rows=rows)[:, : 128 * Jlo]
+        cols = np.nonzero(vis.any(axis=0))[0]
+        assert vis[:, cols].all()
+        assert np.array_equal(np.sort(perm[far_idx[: far_ptr[Jlo]]]), cols)
+
+
+def test_coarse_attention_matches_torch_sdpa():
+    N, d = 260, 16
+    g = Gi.coarse_gist_flags(N, 6, 48, 4)
+    vis = Gi.coarse_visibility(g, Gi.segment_ids(N, 6, 48, 4), 6)
+    rng = np.random.default_rng(2)
+    q, k, v = rng.standard_normal((3, N, d))
+    o, _ = A.forward(q, k, v, vis)
+    t = lambda x: torch.from_numpy(x)[None, None]
+    ref = torch.nn.functional.scaled_dot_product_attention(t(q), t(k), t(v),
+                                                           attn_mask=torch.from_numpy(vis)[None, None])
+    np.testing.assert_allclose(o, ref[0, 0].numpy(), atol=1e-12)
