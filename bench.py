@@ -10,6 +10,9 @@ seeded input already resident in HBM:
   gist_prefill_32k   layout build + forward    (N=32768, 32q/8kv heads)
   gist_decode_128k   one decode step           (16 seqs, 131072-token caches)
   gist_prefill_32k_fwdbwd  layout build + forward + backward on the 32K gist inputs
+  gist_coarse_20k    coarse (segment-wise) layout build + forward: 16 segments
+                     of 1024 raw tokens + 256 gists (20480 positions, 32q/8kv)
+  gist_coarse_20k_fwdbwd   the same with the backward
 Prefill/backward workloads report visited-tile TFLOP/s (every visited block
 pair counted as a full b x b tile: 4*d*b^2 forward, 10*d*b^2 backward); the
 decode workload reports algorithmic HBM GB/s. Inputs are larger than the
@@ -261,7 +264,8 @@ class GistWorkload(GzipWorkload):
                      for t in ("q", "k", "v") + (("do",) if backward else ())}
         self.q, self.k, self.v = (self.h_in[t].cuda() for t in ("q", "k", "v"))
         self.do = self.h_in["do"].cuda() if backward else None
-        self.md = sa.gist_mask(N, H, w["sinks"], w["ratio"], w["window"], gist_tail=w["gist_tail"])
+        self.md = sa.gist_mask(N, H, w["sinks"], w["ratio"], w["window"], gist_tail=w["gist_tail"],
+                               segment=w.get("gist_segment", 0))
         self.lists = sa.BlockLists(self.md)
         self.flags = None
         self.h_flags = torch.zeros(1, dtype=torch.uint8)
@@ -304,8 +308,14 @@ class GistWorkload(GzipWorkload):
         from oracle import attention as A
         from oracle import gist as Gi
         w = self.w
-        N = w["seq_len"]
-        g = Gi.gist_flags(N, w["sinks"], w["ratio"])
+        N, L = w["seq_len"], w.get("gist_segment", 0)
+        if L:  # coarse layout: segments of L raw tokens, then L / ratio gists
+            g = Gi.coarse_gist_flags(N, w["sinks"], L, w["ratio"])
+            seg = Gi.segment_ids(N, w["sinks"], L, w["ratio"])
+            vis_rows = lambda r: Gi.coarse_visibility(g, seg, w["sinks"], rows=r)
+        else:
+            g = Gi.gist_flags(N, w["sinks"], w["ratio"])
+            vis_rows = lambda r: Gi.visibility(g, w["sinks"], w["window"], rows=r)
         perm = Gi.shift_permutation(g, 128)
         inv = np.empty_like(perm)
         inv[perm] = np.arange(N)
@@ -313,7 +323,7 @@ class GistWorkload(GzipWorkload):
         q = W.qkv(w, "q", 0, head=0)[inv]
         k = W.qkv(w, "k", 0, head=0)[inv]
         v = W.qkv(w, "v", 0, head=0)[inv]
-        mask = lambda r: Gi.visibility(g, w["sinks"], w["window"], rows=rows[r])
+        mask = lambda r: vis_rows(rows[r])
         t0 = time.perf_counter()
         if self.backward:
             do = W.qkv(w, "do", 0, head=0)[inv]
@@ -322,7 +332,7 @@ class GistWorkload(GzipWorkload):
             A.forward(q[rows], k, v, mask)
         dt = time.perf_counter() - t0
         # algorithmic FLOPs of those rows: exact visible pairs x 4d (+ 10d backward)
-        n_vis = int(Gi.visibility(g, w["sinks"], w["window"], rows=rows).sum())
+        n_vis = int(vis_rows(rows).sum())
         per = 4.0 + (10.0 if self.backward else 0.0)
         return per * w["head_dim"] * n_vis / dt / 1e12, \
             "head 0, last 2048 query rows, exact visible pairs, fp64", dt
@@ -402,9 +412,11 @@ class DecodeWorkload:
 
 
 SMALL = {"gzip_8k": dict(batch=8), "gzip_64k_fwdbwd": dict(batch=1, heads=4, kv_heads=4),
-         "gist_prefill_32k": dict(heads=8, kv_heads=2), "gist_decode_128k": dict(n_seq=4)}
+         "gist_prefill_32k": dict(heads=8, kv_heads=2), "gist_decode_128k": dict(n_seq=4),
+         "gist_coarse_20k": dict(heads=8, kv_heads=2)}
 # workloads that run another one's inputs with the backward added
-FWDBWD_OF = {"gist_prefill_32k_fwdbwd": "gist_prefill_32k"}
+FWDBWD_OF = {"gist_prefill_32k_fwdbwd": "gist_prefill_32k",
+             "gist_coarse_20k_fwdbwd": "gist_coarse_20k"}
 
 
 def workload_params(name, rank, size):
@@ -421,7 +433,7 @@ def make(sa, torch, name, rank, size="full"):
     w = workload_params(name, rank, size)
     if name.startswith("gzip"):
         return GzipWorkload(sa, torch, w, name.endswith("fwdbwd"))
-    if name.startswith("gist_prefill"):
+    if w["kind"] == "gist":
         return GistWorkload(sa, torch, w, name.endswith("fwdbwd"))
     return DecodeWorkload(sa, torch, w)
 
@@ -464,8 +476,8 @@ def run_reference(args):
     wl = Stub()
     wl.w = dict(W.WORKLOADS[FWDBWD_OF.get(args.workload, args.workload)])
     wl.backward = args.workload.endswith("fwdbwd")
-    cls = {"gzip": GzipWorkload, "gist": GistWorkload, "deco": DecodeWorkload}
-    fn = cls[args.workload[:4]].cpu_baseline
+    cls = {"gzip": GzipWorkload, "gist": GistWorkload, "decode": DecodeWorkload}
+    fn = cls[wl.w["kind"]].cpu_baseline
     vals = []
     H = wl.w["heads"]
     for i in range(args.warmup + args.steps):
@@ -498,7 +510,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="gzip_8k",
                     choices=["gzip_8k", "gzip_64k_fwdbwd", "gist_prefill_32k", "gist_decode_128k",
-                             "gist_prefill_32k_fwdbwd"])
+                             "gist_prefill_32k_fwdbwd", "gist_coarse_20k", "gist_coarse_20k_fwdbwd"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--size", default="full", choices=["full", "small"],
                     help="small: fewer heads/sequences (inputs still larger than L2), for profiling")

@@ -94,9 +94,13 @@ def gzip_mask(batch, seq_len, block_size, window, num_heads, head_class=None):
                      window=window, head_class=head_class)
 
 
-def gist_mask(seq_len, num_heads, sinks, gist_ratio, window, gist_tail=32):
+def gist_mask(seq_len, num_heads, sinks, gist_ratio, window, gist_tail=32, segment=0):
+    """Gist layout. segment = 0: interleaved gists and a local window of
+    `window` positions; segment = L > 0: the coarse layout, L raw tokens then
+    L / gist_ratio gists per segment, full attention inside a segment (window
+    ignored)."""
     return mask_desc(_abi.SA_MASK_GIST, seq_len, num_heads, sinks=sinks, gist_ratio=gist_ratio,
-                     window=window, gist_tail=gist_tail)
+                     window=window, gist_tail=gist_tail, block_size=segment)
 
 
 class BlockLists:

@@ -98,9 +98,9 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
 
 // Item -> (key tile J, KV head, sequence): early key tiles first. The gist
 // layout has two kinds of items: "far" items (tile J of the sinks and gists
-// compacted in logical order, visited by every query tile whose window lies
-// past them) first, then "near" items (physical key tile J, visited by the
-// query tiles that hold it among their near tiles).
+// compacted in logical order, visited by every query tile whose near tiles
+// start past them) first, then "near" items (physical key tile J, visited by
+// the query tiles that hold it among their near tiles).
 struct Item {
   int J, hk, bt, far;
   __device__ Item(int idx, int Hkv, int Bt, int T, bool gist) {
@@ -114,9 +114,11 @@ struct Item {
 };
 
 // The visits of one item, for every query head of the KV group: gzip, the
-// transposed tile list; gist near items, query tiles J .. J + nt - 1; gist far
-// items, the query tiles whose far-key prefix reaches past 128 J (a suffix of
-// the query tiles, found by bisection: far_ptr is non-decreasing).
+// transposed tile list; gist near items, the query tiles I >= J whose near
+// tiles start at or below J (I = J .. J + c - 1: the start is non-decreasing
+// in I and at most nt - 1 tiles below it); gist far items, the query tiles
+// whose far-key prefix reaches past 128 J (a suffix of the query tiles, found
+// by bisection: far_ptr and the near start are non-decreasing).
 struct Visits {
   int n, cnt, i0;
   __device__ void init(const MaskArgs& m, const Item& itm, int rep, int nt) {
@@ -125,14 +127,17 @@ struct Visits {
         int lo = 0, hi = m.T;
         while (lo < hi) {
           const int mid = (lo + hi) >> 1;
-          if (m.far_ptr[max(0, mid - (nt - 1))] > itm.J * kTile) hi = mid;
+          if (m.far_ptr[gist_near_lo(mid, m.sinks, m.window, m.period)] > itm.J * kTile) hi = mid;
           else lo = mid + 1;
         }
         i0 = lo;
         cnt = m.T - lo;
       } else {
         i0 = itm.J;
-        cnt = min(m.T - 1, itm.J + nt - 1) - itm.J + 1;
+        const int last = min(m.T - 1, itm.J + nt - 1);
+        cnt = 1;
+        while (itm.J + cnt <= last && gist_near_lo(itm.J + cnt, m.sinks, m.window, m.period) <= itm.J)
+          ++cnt;
       }
       n = rep * cnt;
       return;
@@ -452,7 +457,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
         } else if (gist) {
           // far tile: compacted keys below this query tile's far prefix are seen
           // by every query row of the tile
-          const int nf = m.far_ptr[max(0, I - (P.near_nt - 1))];
+          const int nf = m.far_ptr[gist_near_lo(I, m.sinks, m.window, m.period)];
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             const bool seen = itm.J * kTile + lane + 32 * i < nf;
@@ -726,18 +731,18 @@ struct BwdWs {
   size_t rows, compact, near, far;
 };
 static size_t r256b(size_t x) { return (x + 255) / 256 * 256; }
-static BwdWs bwd_ws_parts(int Bt, int Hq, int Hkv, int64_t N, int d, int T, int window, bool gist) {
+static BwdWs bwd_ws_parts(int Bt, int Hq, int Hkv, int64_t N, int d, int T, int near_nt, bool gist) {
   BwdWs w{};
   w.rows = r256b((size_t)2 * Bt * Hq * T * kTile * 4);
   if (gist) {
     w.compact = 2 * r256b((size_t)Bt * N * Hkv * d * 2);
-    w.near = r256b((size_t)T * fwd_tc_near_tiles(window) * 2048);
+    w.near = r256b((size_t)T * near_nt * 2048);
     w.far = 2 * r256b((size_t)Bt * N * Hkv * d * 4);
   }
   return w;
 }
-size_t bwd_tc_workspace(int Bt, int Hq, int Hkv, int64_t N, int d, int T, int window, bool gist) {
-  const BwdWs w = bwd_ws_parts(Bt, Hq, Hkv, N, d, T, window, gist);
+size_t bwd_tc_workspace(int Bt, int Hq, int Hkv, int64_t N, int d, int T, int near_nt, bool gist) {
+  const BwdWs w = bwd_ws_parts(Bt, Hq, Hkv, N, d, T, near_nt, gist);
   return w.rows + w.compact + 2 * w.near + w.far;
 }
 
@@ -756,7 +761,7 @@ static cudaError_t bwd_tc_launch(const AttnArgs& a, const MaskArgs& m, void* ws,
   P.m = m;
   P.Tpad = m.T * kTile;
   const bool gist = m.kind == SA_MASK_GIST;
-  const BwdWs parts = bwd_ws_parts(a.Bt, a.Hq, a.Hkv, a.N, D, m.T, m.window, gist);
+  const BwdWs parts = bwd_ws_parts(a.Bt, a.Hq, a.Hkv, a.N, D, m.T, gist_near_tiles(m.window, m.period), gist);
   char* base = static_cast<char*>(ws);
   float* lse2 = reinterpret_cast<float*>(base);
   float* delta = lse2 + (size_t)a.Bt * a.Hq * P.Tpad;
@@ -786,7 +791,7 @@ static cudaError_t bwd_tc_launch(const AttnArgs& a, const MaskArgs& m, void* ws,
         !make_tile_map(&P.tmvc, vc, D, a.Hkv, a.N, a.Bt, cs))
       return cudaErrorInvalidValue;
     P.near_t = static_cast<const uint32_t*>(near_t);
-    P.near_nt = fwd_tc_near_tiles(m.window);
+    P.near_nt = gist_near_tiles(m.window, m.period);
     P.dkf = far;
     P.dvf = reinterpret_cast<float*>(reinterpret_cast<char*>(far) + parts.far / 2);
   }

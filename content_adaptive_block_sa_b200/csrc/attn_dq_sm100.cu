@@ -496,7 +496,7 @@ static cudaError_t dq_tc_launch(const AttnArgs& a, const MaskArgs& m, const floa
         !make_tile_map(&P.tmvc, vc, D, a.Hkv, a.N, a.Bt, cs))
       return cudaErrorInvalidValue;
     P.near = static_cast<const uint32_t*>(near);
-    P.near_nt = fwd_tc_near_tiles(m.window);
+    P.near_nt = gist_near_tiles(m.window, m.period);
   }
   P.a = a;
   P.m = m;

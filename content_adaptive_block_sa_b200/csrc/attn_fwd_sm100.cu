@@ -890,11 +890,12 @@ int sm_count() {
 
 // Gist mode: the element masks of every (query tile I, near key tile J) pair,
 // the same for every head ("UniGist ...", Approach: a query sees the sinks and
-// the gists that are not in its future, and the raw tokens of its window).
-// Block (I, J - I + nt - 1), thread r = query row; bit c of word w tells
-// whether key 128 J + 32 w + c is visible from row 128 I + r. With d = li - lj
-// (logical positions) the rule is (unsigned)d < lim, lim = 2^31 for sinks and
-// gists (d >= 0) and the window for raw tokens (0 <= d < window).
+// the gists that are not in its future, and the raw tokens of its window; in
+// the coarse layout of "A Silver Bullet or a Compromise ...", sections 2 and
+// 6, the raw tokens of its segment instead). Block (I, J - I + nt - 1),
+// thread r = query row; bit c of word w tells whether key 128 J + 32 w + c is
+// visible from row 128 I + r. With d = li - lj (logical positions) the rule is
+// (unsigned)d < lim, lim = gist_reach(lj).
 __global__ void __launch_bounds__(128) gist_near_mask_kernel(MaskArgs m, int N, int nt_count,
                                                              uint32_t* near) {
   const int I = blockIdx.x, nt = blockIdx.y, r = threadIdx.x;
@@ -908,7 +909,7 @@ __global__ void __launch_bounds__(128) gist_near_mask_kernel(MaskArgs m, int N, 
   if (kq < N) {
     lj = m.perm[kq];
     const bool always = lj < m.sinks || ((m.gist_bits[lj >> 5] >> (lj & 31)) & 1u);
-    lim = always ? 0x80000000u : (uint32_t)m.window;
+    lim = gist_reach(always, lj, m.sinks, m.window, m.period);
   }
   lj_s[r] = lj;
   lim_s[r] = lim;
@@ -1036,7 +1037,7 @@ __global__ void __launch_bounds__(128) gist_near_mask_t_kernel(MaskArgs m, int N
   if (kq < N) {
     lj = m.perm[kq];
     const bool always = lj < m.sinks || ((m.gist_bits[lj >> 5] >> (lj & 31)) & 1u);
-    lim = always ? 0x80000000u : (uint32_t)m.window;
+    lim = gist_reach(always, lj, m.sinks, m.window, m.period);
   }
   uint32_t* out = near_t + ((int64_t)I * nt_count + nt) * 512;
 #pragma unroll 1
@@ -1051,7 +1052,7 @@ __global__ void __launch_bounds__(128) gist_near_mask_t_kernel(MaskArgs m, int N
 
 // Gist pre-passes shared by the forward and the backward: the compacted sink /
 // gist K and V (`compact`, 2 * Bt * N * Hkv * d bf16), the near-tile masks
-// (`near`, T * fwd_tc_near_tiles(window) * 2048 bytes) and, for the key-major
+// (`near`, T * gist_near_tiles(window, period) * 2048 bytes) and, for the key-major
 // backward, their transpose (`near_t`, same size, or null).
 template <int D>
 static cudaError_t gist_prepass(const AttnArgs& a, const MaskArgs& m, void* compact, void* near,
@@ -1062,7 +1063,7 @@ static cudaError_t gist_prepass(const AttnArgs& a, const MaskArgs& m, void* comp
   gist_gather_kernel<D><<<dim3((a.N + 7) / 8, a.Bt), 256, 0, s>>>(a, m, kc, vc);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const int nt = fwd_tc_near_tiles(m.window);
+  const int nt = gist_near_tiles(m.window, m.period);
   gist_near_mask_kernel<<<dim3(m.T, nt), kTile, 0, s>>>(m, a.N, nt, static_cast<uint32_t*>(near));
   e = cudaGetLastError();
   if (e != cudaSuccess || near_t == nullptr) return e;
@@ -1124,7 +1125,7 @@ static cudaError_t fwd_tc_launch(const AttnArgs& a, const MaskArgs& m_in, void* 
     cudaError_t e = gist_prepass<D>(a, m, compact, near, nullptr, s);
     if (e != cudaSuccess) return e;
     P.near = static_cast<const uint32_t*>(near);
-    P.near_nt = fwd_tc_near_tiles(m.window);
+    P.near_nt = gist_near_tiles(m.window, m.period);
   }
   P.a = a;
   P.m = m;
@@ -1140,7 +1141,7 @@ static cudaError_t fwd_tc_launch(const AttnArgs& a, const MaskArgs& m_in, void* 
 }
 
 // Gist mode only: `compact`, 2 * Bt * N * Hkv * d bf16 of workspace; `near`,
-// T * fwd_tc_near_tiles(window) * 2048 bytes. Gzip with b = 64: `pair_ws`,
+// T * gist_near_tiles(window, period) * 2048 bytes. Gzip with b = 64: `pair_ws`,
 // fwd_pair_workspace(Bt, B) bytes, selects pair mode (null: 128-row tiles).
 cudaError_t launch_fwd_tc(int d, const AttnArgs& a, const MaskArgs& m, void* compact, void* near,
                           void* pair_ws, cudaStream_t s) {

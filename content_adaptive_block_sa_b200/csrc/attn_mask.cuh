@@ -39,6 +39,7 @@ struct MaskArgs {
   const int32_t* far_idx;   // sinks + gists in logical order (physical indices)
   const int32_t* far_ptr;   // [T+1] far keys below each key tile
   int sinks, window;
+  int period;               // coarse layout: positions per segment (raw + gists); 0: fine
   uint8_t head_class[kMaxHeads];  // gzip: class of each query head
 };
 
@@ -60,6 +61,37 @@ struct AttnArgs {
   DeviceStatus* status;
 };
 
+// ---- gist visibility ("UniGist ...", Approach; "A Silver Bullet or a
+// Compromise ...", sections 2 and 6). A sink or gist key j is seen by every
+// query i >= j; a raw key by the queries of its window (fine layout: i - j <
+// window) or of its own segment (coarse layout: segments of `period`
+// positions after the sinks). Both are "(unsigned)(i - j) < reach(j)".
+__host__ __device__ inline uint32_t gist_reach(bool always, int lj, int sinks, int window,
+                                               int period) {
+  if (always) return 0x80000000u;
+  if (period > 0) return (uint32_t)(sinks + ((lj - sinks) / period + 1) * period - lj);
+  return (uint32_t)window;
+}
+
+// First key tile that query tile I visits with the element rule: every key
+// below it is seen by the whole tile if it is a sink or a gist, else by none
+// of it. Fine layout: I - ceil((window - 1) / 128). Coarse layout: the tile
+// holding the start of the segment of the tile's first row (I while that row
+// is a sink).
+__host__ __device__ inline int gist_near_lo(int I, int sinks, int window, int period) {
+  if (period > 0) {
+    const int p = I * kTile;
+    return p < sinks ? I : (sinks + (p - sinks) / period * period) / kTile;
+  }
+  return max(0, I - (window - 1 + kTile - 1) / kTile);
+}
+
+// Bound on the near tiles of one query tile (I - gist_near_lo(I) + 1).
+__host__ __device__ inline int gist_near_tiles(int window, int period) {
+  if (period > 0) return (period + kTile - 2) / kTile + 1;
+  return (window - 1 + kTile - 1) / kTile + 1;
+}
+
 // Index of the list used by (batch row, query head).
 __device__ __forceinline__ int list_of(const MaskArgs& m, int bt, int h) {
   return m.kind == SA_MASK_GZIP ? bt * 3 + m.head_class[h] : 0;
@@ -74,9 +106,8 @@ __device__ __forceinline__ bool element_visible(const MaskArgs& m, int list, int
     return (row[j >> 5] >> (j & 31)) & 1u;
   }
   const int i = m.perm[p], j = m.perm[q];
-  if (j > i) return false;
   const bool g = (m.gist_bits[j >> 5] >> (j & 31)) & 1u;
-  return j < m.sinks || g || (i - j) < m.window;
+  return (uint32_t)(i - j) < gist_reach(j < m.sinks || g, j, m.sinks, m.window, m.period);
 }
 
 // ---- visibility words of gzip tiles (forward and query-major backward)
@@ -153,12 +184,6 @@ __device__ __forceinline__ void gzip_tile_words(const MaskArgs& m, int lb, int N
 }
 
 // ---- visit lists of a query tile (forward and query-major backward)
-// Near key tiles of a query tile in gist mode: Jlo..I with
-// Jlo = I - ceil((window - 1) / 128).
-__host__ __device__ inline int fwd_tc_near_tiles(int window) {
-  return (window - 1 + kTile - 1) / kTile + 1;
-}
-
 // Internal tile kind: only the first `cnt` columns hold keys (the last tile of
 // the compacted sink/gist keys).
 constexpr int kTileCount = 3;
@@ -176,7 +201,7 @@ struct WorkList {
       n = m.pair_ptr[list * (m.P + 1) + I + 1] - e0;
       nft = nf = jlo = 0;
     } else if (gist) {
-      jlo = max(0, I - (m.window - 1 + kTile - 1) / kTile);
+      jlo = gist_near_lo(I, m.sinks, m.window, m.period);
       nf = m.far_ptr[jlo];
       nft = (nf + kTile - 1) / kTile;
       n = nft + (I - jlo + 1);

@@ -14,7 +14,13 @@
 // per-tile shift permutation (raw tokens first, gists last, both stable) and
 // the tile lists of the visibility rule
 //   vis(i, j) = j <= i and (j < sinks or gist(j) or i - j < window)
-// with FULL / MASKED / TAIL kinds.
+// with FULL / MASKED / TAIL kinds. The segment-wise coarse layout ("A Silver
+// Bullet or a Compromise for Full Attention? ...", sections 2 and 6: each
+// segment's gists follow all of its raw tokens; full attention inside a
+// segment) puts `seg` raw tokens and seg / ratio gists in every period after
+// the sinks and replaces the window by the segment:
+//   vis(i, j) = j <= i and (j < sinks or gist(j) or segment(i) == segment(j)).
+// Both rules read "raw key j is seen by query i iff lo(i) <= j <= i".
 //
 // Gzip: five CTAs per (sequence, class) pair, one per output (block CSR, block
 // CSC, bit rows, tile lists, transposed tile lists); counts become absolute
@@ -287,6 +293,7 @@ __global__ void __launch_bounds__(1024) gzip_build_kernel(GzipBuild p) {
 struct GistBuild {
   const uint8_t* flags;  // [N] or null
   int N, T, sinks, ratio, window, tail;
+  int seg, period;  // coarse layout: raw tokens and positions per segment; 0: fine
   int64_t tregion;
   uint32_t* gist_bits;
   int32_t* perm;
@@ -326,6 +333,14 @@ __device__ int first_raw(const uint32_t* gb, int a, int b) {
   return -1;
 }
 
+// Smallest raw key position query i sees (any j <= i at or above it): the
+// window's start, or the start of i's segment (0 for sink rows, whose keys
+// are all sinks).
+__device__ __forceinline__ int raw_lo(const GistBuild& p, int i) {
+  if (p.period > 0) return i < p.sinks ? 0 : p.sinks + (i - p.sinks) / p.period * p.period;
+  return i - p.window + 1;
+}
+
 // Kind of tile pair (I, J) under the gist visibility rule, or -1.
 __device__ int gist_tile_kind(const GistBuild& p, int I, int J) {
   if (J > I) return -1;
@@ -335,17 +350,18 @@ __device__ int gist_tile_kind(const GistBuild& p, int I, int J) {
   const uint32_t* gb = p.gist_bits;
   const int ng = count_gists(gb, j0, j1);
   const bool has_sink = j0 < p.sinks;
-  const bool any = has_sink || ng > 0 || (i_min - (j1 - 1) < p.window);
+  const bool any = has_sink || ng > 0 || j1 - 1 >= raw_lo(p, i_min);
   if (!any) return -1;
-  // all pairs visible iff every non-gist, non-sink key is in every query's window
+  // all pairs visible iff every non-gist, non-sink key is seen by every query
+  // (lo is non-decreasing in i: the last row binds)
   const int jr = first_raw(gb, max(j0, p.sinks), j1);
-  if (jr < 0 || i_max - jr < p.window) return SA_TILE_FULL;
+  if (jr < 0 || jr >= raw_lo(p, i_max)) return SA_TILE_FULL;
   // smallest physical column visible to some query of tile I
   const int n_raw = (j1 - j0) - ng;
   int min_col = kTile;
   if (ng > 0) min_col = n_raw;  // gists sit after the raw tokens
   int r = first_raw(gb, j0, min(j1, p.sinks));  // raw sink tokens
-  if (r < 0) r = first_raw(gb, max(j0, i_min - p.window + 1), j1);  // raw window tokens
+  if (r < 0) r = first_raw(gb, max(j0, raw_lo(p, i_min)), j1);  // raw window / segment tokens
   if (r >= 0) min_col = min(min_col, (r - j0) - count_gists(gb, j0, r));
   return (min_col >= kTile - p.tail) ? SA_TILE_TAIL : SA_TILE_MASKED;
 }
@@ -353,6 +369,7 @@ __device__ int gist_tile_kind(const GistBuild& p, int I, int J) {
 // Gist bit of logical position pos (< N).
 __device__ __forceinline__ bool gist_at(const GistBuild& p, int pos) {
   if (p.flags) return p.flags[pos] != 0;
+  if (p.period > 0) return pos >= p.sinks && (pos - p.sinks) % p.period >= p.seg;
   return pos >= p.sinks && ((pos - p.sinks) % (p.ratio + 1)) == p.ratio;
 }
 
@@ -506,6 +523,8 @@ cudaError_t launch_gist_build(const sa_mask_desc& d, const uint8_t* flags,
   p.sinks = d.sinks;
   p.ratio = d.gist_ratio;
   p.window = d.window;
+  p.seg = d.block_size;
+  p.period = d.block_size > 0 ? d.block_size + d.block_size / d.gist_ratio : 0;
   p.tail = d.gist_tail > 0 ? d.gist_tail : 32;
   p.tregion = (int64_t)p.T * (p.T + 1) / 2;
   p.gist_bits = L.gist_bits;

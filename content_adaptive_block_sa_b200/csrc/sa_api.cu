@@ -18,7 +18,7 @@ cudaError_t launch_fwd_tc(int d, const AttnArgs&, const MaskArgs&, void* compact
 
 size_t fwd_pair_workspace(int Bt, int B);
 cudaError_t launch_bwd_tc(int d, const AttnArgs&, const MaskArgs&, void* ws, cudaStream_t);
-size_t bwd_tc_workspace(int Bt, int Hq, int Hkv, int64_t N, int d, int T, int window, bool gist);
+size_t bwd_tc_workspace(int Bt, int Hq, int Hkv, int64_t N, int d, int T, int near_nt, bool gist);
 cudaError_t launch_decode(const sa_decode_desc&, const void*, const void*, const void*,
                           const void*, const void*, int32_t*, void*, float*, void*,
                           cudaStream_t);
@@ -44,6 +44,12 @@ int tiles_of(int64_t n) { return (int)((n + kTile - 1) / kTile); }
 // Number of lists of a mask (gzip: batch x 3 classes; gist: 1).
 int64_t n_lists(const sa_mask_desc& d) { return d.kind == SA_MASK_GZIP ? (int64_t)d.batch * 3 : 1; }
 
+// Coarse gist layout: positions per segment (raw tokens + gists); 0: fine.
+int gist_period(const sa_mask_desc& d) {
+  return d.kind == SA_MASK_GIST && d.block_size > 0 ? d.block_size + d.block_size / d.gist_ratio
+                                                    : 0;
+}
+
 sa_status check_mask(const sa_mask_desc* d) {
   SA_CHECK(d != nullptr, SA_ERR_INVALID_ARG);
   SA_CHECK(d->seq_len >= 1 && d->seq_len <= kMaxSeq, SA_ERR_INVALID_ARG);
@@ -65,8 +71,12 @@ sa_status check_mask(const sa_mask_desc* d) {
   }
   if (d->kind == SA_MASK_GIST) {
     SA_CHECK(d->batch == 1, SA_ERR_INVALID_ARG);
-    SA_CHECK(d->sinks >= 0 && d->window >= 1, SA_ERR_INVALID_ARG);
-    SA_CHECK(d->gist_ratio >= 1, SA_ERR_INVALID_ARG);
+    SA_CHECK(d->gist_ratio >= 1 && d->sinks >= 0, SA_ERR_INVALID_ARG);
+    // block_size 0: fine layout (window >= 1); > 0: coarse layout, segments
+    // of block_size raw tokens and block_size / gist_ratio gists
+    SA_CHECK(d->block_size >= 0 && d->block_size <= kMaxSeq, SA_ERR_INVALID_ARG);
+    SA_CHECK(d->block_size > 0 ? d->block_size % d->gist_ratio == 0 : d->window >= 1,
+             SA_ERR_INVALID_ARG);
     SA_CHECK(d->gist_tail == 0 || (d->gist_tail % 16 == 0 && d->gist_tail <= kTile),
              SA_ERR_INVALID_ARG);
     SA_CHECK(T * (T + 1) / 2 < INT32_MAX, SA_ERR_UNSUPPORTED);
@@ -170,6 +180,7 @@ MaskArgs make_mask_args(const sa_mask_desc& d, const sa_block_lists& L) {
     m.far_ptr = L.far_ptr;
     m.sinks = d.sinks;
     m.window = d.window;
+    m.period = gist_period(d);
   }
   return m;
 }
@@ -271,6 +282,9 @@ sa_status sa_build_block_mask(const sa_mask_desc* desc, const uint8_t* d_flags,
   sa_status st = check_mask(desc);
   if (st != SA_OK) return st;
   if (desc->kind == SA_MASK_GZIP) SA_CHECK(d_flags != nullptr, SA_ERR_INVALID_ARG);
+  // the coarse gist layout takes its regular pattern only
+  if (desc->kind == SA_MASK_GIST && desc->block_size > 0)
+    SA_CHECK(d_flags == nullptr, SA_ERR_INVALID_ARG);
   st = check_lists(*desc, out);
   if (st != SA_OK) return st;
   st = check_ws(ws, ws_bytes, kStatusBytes);
@@ -300,7 +314,8 @@ sa_status sa_forward_workspace_size(const sa_attn_desc* attn, const sa_mask_desc
     // every (query tile, near key tile) pair, 128 x 128 bits each
     *bytes += 2 * round256((size_t)attn->batch * attn->seq_len * attn->num_kv_heads *
                            attn->head_dim * 2);
-    *bytes += round256((size_t)tiles_of(attn->seq_len) * fwd_tc_near_tiles(mask->window) * 2048);
+    *bytes += round256((size_t)tiles_of(attn->seq_len) *
+                       gist_near_tiles(mask->window, gist_period(*mask)) * 2048);
   }
   return SA_OK;
 }
@@ -348,7 +363,8 @@ sa_status sa_backward_workspace_size(const sa_attn_desc* attn, const sa_mask_des
   const size_t simt = (size_t)attn->batch * attn->num_q_heads * attn->seq_len * sizeof(float);
   const size_t tc = bwd_tc_workspace(attn->batch, attn->num_q_heads, attn->num_kv_heads,
                                      attn->seq_len, attn->head_dim, tiles_of(attn->seq_len),
-                                     mask->window, mask->kind == SA_MASK_GIST);
+                                     gist_near_tiles(mask->window, gist_period(*mask)),
+                                     mask->kind == SA_MASK_GIST);
   *bytes = kStatusBytes + round256(simt > tc ? simt : tc);
   return SA_OK;
 }

@@ -95,16 +95,24 @@ typedef enum {
  *              gist: must be 1 - the layout is shared by every batch row.
  *  seq_len     N, tokens (gzip) or positions including gists (gist).
  *  block_size  gzip: b, tokens per block, N % b == 0, and either b % 128 == 0
- *              or 128 % b == 0. gist: ignored.
+ *              or 128 % b == 0. gist: 0 for the fine (interleaved) layout; L > 0
+ *              for the segment-wise coarse layout of "A Silver Bullet or a
+ *              Compromise for Full Attention? ..." (sections 2 and 6): after the
+ *              sinks, segments of L raw tokens followed by L / gist_ratio gists
+ *              (L % gist_ratio == 0), and query i sees the sinks, the gists not
+ *              in its future and every position of its own segment up to i.
+ *              The coarse layout takes no explicit flags.
  *  window      gzip: w in BLOCKS (key block j is local to i iff i - j <= w).
- *              gist: W in POSITIONS (key j is in the window of i iff i - j < W).
+ *              gist, fine layout: W >= 1 in POSITIONS (key j is in the window
+ *              of i iff i - j < W). gist, coarse layout: ignored.
  *  num_heads   number of query heads H.
  *  head_class  gzip: HOST array [H] of sa_head_class, or NULL for the default
  *              split floor(H/2) local, floor(H/4) literal, rest hybrid, in
  *              that head order. gist: ignored.
  *  sinks       gist: positions [0, sinks) are sink tokens visible to all.
- *  gist_ratio  gist: raw tokens per gist; after the sinks a gist follows every
- *              gist_ratio raw tokens (used when no explicit flags are given).
+ *  gist_ratio  gist: raw tokens per gist; fine layout: after the sinks a gist
+ *              follows every gist_ratio raw tokens (used when no explicit
+ *              flags are given).
  *  gist_tail   gist: width of the tail sub-block that holds a tile's gists
  *              after the shift (multiple of 16, <= 128; 0 means 32).
  */
@@ -155,9 +163,11 @@ typedef struct sa_mask_desc {
  *  far_idx    int32 [N]: the keys every later query sees whatever its window
  *             (sinks and gists), in logical order, as PHYSICAL indices.
  *  far_ptr    int32 [T+1]: far_ptr[J] = number of those keys at logical
- *             positions below 128*J. Query tile I's window cannot reach below
- *             key tile Jlo = max(0, I - ceil((W-1)/128)), so the keys it sees
- *             there are exactly far_idx[0 .. far_ptr[Jlo]).
+ *             positions below 128*J. Query tile I's window (segment) cannot
+ *             reach below key tile Jlo = max(0, I - ceil((W-1)/128)) (coarse:
+ *             the tile holding the start of the segment of position 128*I, or
+ *             I while that position is a sink), so the keys it sees there are
+ *             exactly far_idx[0 .. far_ptr[Jlo]).
  */
 typedef struct sa_block_lists {
   int32_t* row_ptr;
@@ -296,7 +306,8 @@ sa_status sa_build_block_mask_workspace_size(const sa_mask_desc* desc, size_t* b
  *  d_flags  gzip: DEVICE uint8 [batch, B] literal flags (0/1), e.g. from
  *           sa_literal_flags_from_sizes. gist: DEVICE uint8 [N] with 1 for
  *           the LOGICAL positions that are gists, or NULL for the regular
- *           pattern (sinks, then one gist after every gist_ratio raw tokens).
+ *           pattern (sinks, then one gist after every gist_ratio raw tokens;
+ *           coarse layout: NULL only, its segments as block_size states).
  *  out      lists to fill; capacities checked against sa_block_lists_capacity.
  * Bit-exact: the lists depend only on integers. */
 sa_status sa_build_block_mask(const sa_mask_desc* desc, const uint8_t* d_flags,

@@ -21,6 +21,9 @@ settings; no real corpus is used anywhere):
                         4096 gists, top-64, window 512, 32 q / 8 kv heads.
 5. ``gzip_64k_fwdbwd`` - batch 2, N=65536, block 128, window 2, 16 heads,
                         d=128, bf16, flags from synthetic mixed text/random bytes.
+6. ``gist_coarse_20k`` - segment-wise coarse gist layout: 16 segments of 1024
+                        raw tokens, each followed by 256 gists (ratio 4), no
+                        sinks (20480 positions), 32 q / 8 kv heads, d=128, bf16.
 """
 from __future__ import annotations
 
@@ -46,6 +49,9 @@ WORKLOADS = {
     "gist_decode_128k": dict(index=4, kind="decode", n_seq=16, cache_len=131072,
                              chunk=32, n_gists=4096, top_k=64, window=512,
                              heads=32, kv_heads=8, head_dim=128, dtype="bf16"),
+    "gist_coarse_20k": dict(index=6, kind="gist", batch=1, seq_len=20480,
+                            sinks=0, ratio=4, window=0, gist_segment=1024, heads=32,
+                            kv_heads=8, head_dim=128, dtype="bf16", tile=128, gist_tail=32),
     "gzip_64k_fwdbwd": dict(index=5, kind="gzip", batch=2, seq_len=65536,
                             block=128, window=2, heads=16, kv_heads=16,
                             head_dim=128, dtype="bf16", flags_from="bytes_mixed",

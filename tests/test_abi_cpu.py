@@ -97,11 +97,24 @@ def test_capacity_and_validation(sa):
            sa.gzip_mask(0, 1024, 64, 1, 4),      # no batch
            sa.gist_mask(4096, 8, 128, 0, 128),   # ratio 0
            sa.gist_mask(4096, 8, 128, 4, 0),     # empty window
-           sa.gist_mask(4096, 8, 128, 4, 128, gist_tail=40)]
+           sa.gist_mask(4096, 8, 128, 4, 128, gist_tail=40),
+           sa.gist_mask(4096, 8, 0, 4, 0, segment=1022),   # segment not a multiple of the ratio
+           sa.gist_mask(4096, 8, 0, 4, 0, segment=-4)]     # negative segment
     codes = [_caps(sa, d)[0] for d in bad]
     assert all(c in (1, 2) for c in codes), codes
     d = sa.gzip_mask(1, 1024, 64, 1, 4, head_class=[0, 1, 2, 3])
     assert _caps(sa, d)[0] == 1
+    # the coarse layout ignores the window
+    assert _caps(sa, sa.gist_mask(20480, 32, 0, 4, 0, segment=1024))[0] == 0
+
+
+def test_coarse_layout_rejects_explicit_flags_without_a_device(sa):
+    md = sa.gist_mask(4096, 8, 0, 4, 0, segment=1024)
+    caps = sa._abi.sa_block_lists_sizes()
+    assert sa.lib().sa_block_lists_capacity(C.byref(md), C.byref(caps)) == 0
+    lists = sa._abi.sa_block_lists()
+    flags = C.c_void_p(16)  # never dereferenced: the descriptor check comes first
+    assert sa.lib().sa_build_block_mask(C.byref(md), flags, C.byref(lists), None, 0, None) == 1
 
 
 def test_calls_reject_null_and_small_workspace_without_a_device(sa):
