@@ -19,6 +19,16 @@ Readings taken where the pages are silent:
   fewer than k chunks are eligible);
 * every head attends over all gists of its group, the raw tokens of the
   selected chunks and the last ``window`` raw tokens, with one softmax.
+
+Selection variants (the first page's record names a top-p routine next to the
+top-k one; the pages give nothing more):
+* sum of probabilities: each query head's softmax over all gists of its
+  group (the attention it would pay to the gists alone), summed over the
+  group's heads, ranks the chunks; top-k as above;
+* top-p: the group scores (sum of logits) are turned into probabilities by a
+  softmax over the eligible chunks; taking chunks in score order (ties to the
+  lower index), the smallest prefix whose probability reaches p is kept, at
+  most k chunks.
 """
 from __future__ import annotations
 
@@ -42,6 +52,23 @@ def group_scores(q, gist_k, scale=None) -> np.ndarray:
     return out
 
 
+def group_prob_scores(q, gist_k, scale=None) -> np.ndarray:
+    """s[g, c] = sum over q heads h of group g of softmax_c(q_h . gist_k[g, c] * scale),
+    each head's softmax taken over all the group's gists."""
+    q = np.asarray(q, np.float64)
+    gk = np.asarray(gist_k, np.float64)
+    Hq, d = q.shape
+    Hkv = gk.shape[0]
+    rep = Hq // Hkv
+    scale = 1.0 / np.sqrt(d) if scale is None else float(scale)
+    out = np.zeros((Hkv, gk.shape[1]))
+    for h in range(Hq):
+        logits = (gk[h // rep] @ q[h]) * scale
+        e = np.exp(logits - logits.max())
+        out[h // rep] += e / e.sum()
+    return out
+
+
 def eligible_chunks(n_gists: int, chunk: int, cache_len: int, window: int) -> np.ndarray:
     """Chunks whose raw tokens all lie before the last ``window`` positions."""
     c = np.arange(n_gists)
@@ -54,6 +81,27 @@ def select_top_k(scores, eligible, k: int) -> np.ndarray:
     idx = [c for c in range(len(scores)) if eligible[c]]
     idx.sort(key=lambda c: (-float(scores[c]), c))
     chosen = sorted(idx[:k])
+    return np.asarray(chosen + [-1] * (k - len(chosen)), dtype=np.int32)
+
+
+def select_top_p(scores, eligible, k: int, p: float) -> np.ndarray:
+    """Ascending indices of the smallest score-ordered prefix of the eligible
+    chunks whose softmax probability (over the eligible chunks) reaches p, at
+    most k of them; padded with -1 to length k."""
+    idx = [c for c in range(len(scores)) if eligible[c]]
+    idx.sort(key=lambda c: (-float(scores[c]), c))
+    chosen = []
+    if idx:
+        s = np.asarray([scores[c] for c in idx], np.float64)
+        prob = np.exp(s - s.max())
+        prob /= prob.sum()
+        cum = 0.0
+        for c, pc in zip(idx[:k], prob[:k]):
+            if chosen and cum >= p:
+                break
+            chosen.append(c)
+            cum += pc
+    chosen = sorted(chosen)
     return np.asarray(chosen + [-1] * (k - len(chosen)), dtype=np.int32)
 
 
@@ -71,8 +119,14 @@ def attend(qh, keys, values, scale):
     return np.exp(s - lse) @ np.asarray(values, np.float64), lse
 
 
-def decode_one(q, gist_k, gist_v, raw_k, raw_v, chunk, window, top_k, scale=None):
-    """One sequence.
+SUM_LOGITS, SUM_PROBS, TOP_P = 0, 1, 2
+
+
+def decode_one(q, gist_k, gist_v, raw_k, raw_v, chunk, window, top_k, scale=None,
+               rule=SUM_LOGITS, top_p=1.0):
+    """One sequence. ``rule``: SUM_LOGITS (top-k of the summed logits),
+    SUM_PROBS (top-k of the summed per-head probabilities) or TOP_P (top-p of
+    the summed logits, at most top_k chunks).
 
     q [Hq, d]; gist_k/gist_v [Hkv, G, d]; raw_k/raw_v: callables
     (kv_head) -> [cache_len, d] (or arrays [Hkv, cache_len, d]).
@@ -85,7 +139,7 @@ def decode_one(q, gist_k, gist_v, raw_k, raw_v, chunk, window, top_k, scale=None
     scale = 1.0 / np.sqrt(d) if scale is None else float(scale)
     get_k = raw_k if callable(raw_k) else (lambda g: raw_k[g])
     get_v = raw_v if callable(raw_v) else (lambda g: raw_v[g])
-    scores = group_scores(q, gist_k, scale)
+    scores = group_prob_scores(q, gist_k, scale) if rule == SUM_PROBS else group_scores(q, gist_k, scale)
     sel = np.empty((Hkv, top_k), np.int32)
     o = np.empty((Hq, d))
     lse = np.empty(Hq)
@@ -93,7 +147,8 @@ def decode_one(q, gist_k, gist_v, raw_k, raw_v, chunk, window, top_k, scale=None
         rk, rv = get_k(g), get_v(g)
         cache_len = rk.shape[0]
         elig = eligible_chunks(G, chunk, cache_len, window)
-        sel[g] = select_top_k(scores[g], elig, top_k)
+        sel[g] = (select_top_p(scores[g], elig, top_k, top_p) if rule == TOP_P
+                  else select_top_k(scores[g], elig, top_k))
         pos = raw_key_positions(sel[g], chunk, cache_len, window)
         keys = np.concatenate([np.asarray(gist_k[g], np.float64), np.asarray(rk[pos], np.float64)])
         vals = np.concatenate([np.asarray(gist_v[g], np.float64), np.asarray(rv[pos], np.float64)])

@@ -80,3 +80,81 @@ def test_selection_is_the_best_eligible_set():
 def test_gist_kv_is_one_chunk_th_of_raw():
     # one gist key/value per chunk: the scored set is cache_len / chunk rows
     assert D.eligible_chunks(4096, 32, 131072, 0).sum() * 32 == 131072
+
+
+# ---------------------------------------------------------------- selection variants
+def test_prob_scores_sum_to_group_size_and_match_torch_softmax():
+    q, gk, *_ = _case(3)
+    s = D.group_prob_scores(q, gk)
+    np.testing.assert_allclose(s.sum(1), [4.0, 4.0], atol=1e-12)  # 4 heads, each sums to one
+    logits = torch.einsum("gcd,ghd->ghc", torch.from_numpy(gk),
+                          torch.from_numpy(q).reshape(2, 4, 16)) / 4.0
+    np.testing.assert_allclose(s, torch.softmax(logits, -1).sum(1).numpy(), atol=1e-12)
+
+
+def test_prob_scores_rank_like_logits_for_one_head_per_group():
+    # one head per group: a softmax is monotone, so the two rules select the same chunks
+    q, gk, *_ = _case(4, Hq=2, Hkv=2)
+    elig = np.ones(gk.shape[1], bool)
+    for g in range(2):
+        assert np.array_equal(D.select_top_k(D.group_prob_scores(q, gk)[g], elig, 7),
+                              D.select_top_k(D.group_scores(q, gk)[g], elig, 7))
+
+
+def test_prob_scores_differ_from_logit_sums_across_heads():
+    # head 0 is sharp on chunk 0, head 1 flat but slightly higher on chunk 1:
+    # logit sums prefer chunk 1, probability sums chunk 0
+    logits = np.array([[10.0, 0.0, 0.0], [0.0, 10.5, 10.4]])
+    d = 2
+    q = np.eye(d)
+    gk = logits.T[None] * np.sqrt(d)  # gist c's key = column c, so q_h . k_c * scale = logits[h, c]
+    sl = D.group_scores(q, gk)[0]
+    sp = D.group_prob_scores(q, gk)[0]
+    assert np.argmax(sl) == 1 and np.argmax(sp) == 0
+
+
+def test_top_p_closed_form():
+    probs = np.array([0.2, 0.5, 0.3])
+    s = np.log(probs)
+    elig = np.ones(3, bool)
+    assert D.select_top_p(s, elig, 3, 0.45).tolist() == [1, -1, -1]
+    assert D.select_top_p(s, elig, 3, 0.75).tolist() == [1, 2, -1]
+    assert D.select_top_p(s, elig, 3, 0.85).tolist() == [0, 1, 2]
+    assert D.select_top_p(s, elig, 2, 0.85).tolist() == [1, 2]  # capped at k
+    assert D.select_top_p(s, elig, 3, 1e-9).tolist() == [1, -1, -1]  # never empty
+    elig[1] = False  # renormalised over the eligible chunks: 0.2 / 0.5 and 0.3 / 0.5
+    assert D.select_top_p(s, elig, 3, 0.55).tolist() == [2, -1, -1]
+    assert D.select_top_p(s, elig, 3, 0.65).tolist() == [0, 2, -1]
+    assert D.select_top_p(s, np.zeros(3, bool), 2, 0.5).tolist() == [-1, -1]
+
+
+def test_top_p_is_the_smallest_set_reaching_p_by_brute_force():
+    from itertools import combinations
+    rng = np.random.default_rng(7)
+    for trial in range(40):
+        n = 7
+        s = rng.standard_normal(n) * 2
+        elig = rng.random(n) < 0.8
+        p = rng.uniform(0.05, 0.99)
+        ids = np.nonzero(elig)[0]
+        if len(ids) == 0:
+            continue
+        prob = np.zeros(n)
+        prob[ids] = np.exp(s[ids] - s[ids].max())
+        prob /= prob.sum()
+        best = None
+        for m in range(1, len(ids) + 1):
+            sets = [c for c in combinations(ids, m) if prob[list(c)].sum() >= p]
+            if sets:
+                best = max(sets, key=lambda c: prob[list(c)].sum())
+                break
+        got = D.select_top_p(s, elig, n, p)
+        assert sorted(got[got >= 0].tolist()) == sorted(best), (trial, p)
+
+
+def test_top_p_one_equals_top_k():
+    q, gk, *_ = _case(5)
+    s = D.group_scores(q, gk)[1]
+    elig = D.eligible_chunks(len(s), 16, 512, 64)
+    for k in (1, 5, 20):
+        assert np.array_equal(D.select_top_p(s, elig, k, 1.0), D.select_top_k(s, elig, k))
