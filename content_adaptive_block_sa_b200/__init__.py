@@ -242,14 +242,15 @@ def backward(q, k, v, o, lse, dout, mdesc, lists, softmax_scale: float = 0.0, st
 
 # ------------------------------------------------------------------- decode
 def decode_desc(q, gist_k, k_cache, o, chunk: int, top_k: int, window: int,
-                softmax_scale: float = 0.0) -> _abi.sa_decode_desc:
+                softmax_scale: float = 0.0, select_rule: int = 0,
+                top_p: float = 1.0) -> _abi.sa_decode_desc:
     n_seq, Hq, d = q.shape
     _, Hkv, G, _ = gist_k.shape
     L = k_cache.shape[2]
     return _abi.sa_decode_desc(
         n_seq=n_seq, cache_len=L, chunk=chunk, n_gists=G, top_k=top_k, window=window,
         num_q_heads=Hq, num_kv_heads=Hkv, head_dim=d,
-        select_rule=_abi.SA_SELECT_SUM_LOGITS_PER_GROUP, softmax_scale=softmax_scale,
+        select_rule=select_rule, softmax_scale=softmax_scale, top_p=top_p,
         q_strides=(i64 * 2)(q.stride(0), q.stride(1)),
         gist_strides=(i64 * 3)(gist_k.stride(0), gist_k.stride(1), gist_k.stride(2)),
         cache_strides=(i64 * 3)(k_cache.stride(0), k_cache.stride(1), k_cache.stride(2)),
@@ -270,8 +271,10 @@ def sa_gist_decode(ddesc, q, gist_k, gist_v, k_cache, v_cache, sel, o, lse, ws, 
 
 
 def gist_decode(q, gist_k, gist_v, k_cache, v_cache, chunk: int, top_k: int, window: int,
-                softmax_scale: float = 0.0, stream=None):
-    """(sel int32 [n_seq, Hkv, top_k], o bf16 [n_seq, Hq, d], lse fp32 [n_seq, Hq])."""
+                softmax_scale: float = 0.0, stream=None, select_rule: int = 0, top_p: float = 1.0):
+    """(sel int32 [n_seq, Hkv, top_k], o bf16 [n_seq, Hq, d], lse fp32 [n_seq, Hq]).
+    select_rule: 0 top-k of summed logits, 1 top-k of summed per-head
+    probabilities, 2 top-p (at most top_k chunks) of the summed logits."""
     if gist_v.stride() != gist_k.stride() or v_cache.stride() != k_cache.stride():
         raise ValueError("K and V must share strides")
     n_seq, Hq, d = q.shape
@@ -279,7 +282,7 @@ def gist_decode(q, gist_k, gist_v, k_cache, v_cache, chunk: int, top_k: int, win
     o = torch.empty_like(q)
     lse = torch.empty(n_seq, Hq, dtype=torch.float32, device=q.device)
     sel = torch.empty(n_seq, Hkv, max(top_k, 1), dtype=torch.int32, device=q.device)
-    dd = decode_desc(q, gist_k, k_cache, o, chunk, top_k, window, softmax_scale)
+    dd = decode_desc(q, gist_k, k_cache, o, chunk, top_k, window, softmax_scale, select_rule, top_p)
     ws = decode_workspace(dd, q.device)
     sa_gist_decode(dd, q, gist_k, gist_v, k_cache, v_cache, sel, o, lse, ws, stream)
     gist_decode.last_workspace = ws

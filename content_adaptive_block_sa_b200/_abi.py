@@ -16,6 +16,8 @@ SA_CLASS_LOCAL, SA_CLASS_LITERAL, SA_CLASS_HYBRID = 0, 1, 2
 SA_DTYPE_BF16, SA_DTYPE_FP32 = 0, 1
 SA_TILE_FULL, SA_TILE_MASKED, SA_TILE_TAIL = 0, 1, 2
 SA_SELECT_SUM_LOGITS_PER_GROUP = 0
+SA_SELECT_SUM_PROBS_PER_GROUP = 1
+SA_SELECT_TOP_P_PER_GROUP = 2
 SA_IMPL_AUTO, SA_IMPL_CUDA_CORES, SA_IMPL_TENSOR_CORES = 0, 1, 2
 SA_TILE = 128
 
@@ -53,7 +55,7 @@ class sa_decode_desc(C.Structure):
                 ("top_k", i32), ("window", i32), ("num_q_heads", i32), ("num_kv_heads", i32),
                 ("head_dim", i32), ("select_rule", i32), ("softmax_scale", f32),
                 ("q_strides", i64 * 2), ("gist_strides", i64 * 3), ("cache_strides", i64 * 3),
-                ("o_strides", i64 * 2)]
+                ("o_strides", i64 * 2), ("top_p", f32)]
 
 
 P = C.POINTER

@@ -13,7 +13,12 @@
 //      (max m, sum l, unnormalised o) per head and slice. Gist K and V are
 //      streamed once.
 //   2. select: top_k eligible chunks (wholly before the window) by score,
-//      ties to the lower index, written ascending (-1 padded).
+//      ties to the lower index, written ascending (-1 padded). The score is
+//      the sum of the group's logits, or (sum-of-probabilities rule) the sum
+//      of each head's softmax over all gists, from per-head logits the gist
+//      pass stores and the heads' gist-slice partials; the top-p rule keeps
+//      the shortest score-ordered prefix whose softmax over the eligible
+//      chunks reaches p.
 //   3. raw pass (split over the unfolded keys): the same partials over the
 //      raw tokens of the selected chunks followed by the last `window`
 //      tokens.
@@ -38,6 +43,9 @@ struct DecodeArgs {
   float* lse;
   float* scores;   // [n_seq, Hkv, G]
   float* part;     // [n_seq, Hq, n_part, 2 + D]
+  float* logits;   // [n_seq, Hq, G] scaled logits (sum-of-probabilities rule)
+  int rule;
+  float top_p;
   int n_seq, cache_len, chunk, G, top_k, window, Hq, Hkv, rep;
   int n_gslices, n_rslices, n_part;
   float scale;
@@ -74,7 +82,8 @@ struct HalfState {
 // pointers) and writes one partial per head to `out` (slot `slot`).
 template <int REP, typename RowFn>
 __device__ void attend_slice(const DecodeArgs& a, const float (*qf)[kDecD], int e0, int e1,
-                             RowFn row, float* score_out, int seq, int g, int slot) {
+                             RowFn row, float* score_out, float* logit_out, int seq, int g,
+                             int slot) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int half = lane >> 4, hl = lane & 15;  // 16 lanes per key row
   HalfState<REP> st;
@@ -111,6 +120,9 @@ __device__ void attend_slice(const DecodeArgs& a, const float (*qf)[kDecD], int 
       ssum += s[h];
     }
     if (valid && score_out != nullptr && hl == 0) score_out[e] = ssum;
+    if (valid && logit_out != nullptr && hl == 0)
+#pragma unroll
+      for (int h = 0; h < REP; ++h) logit_out[(int64_t)h * a.G + e] = s[h];
     if (!valid) continue;
 #pragma unroll
     for (int h = 0; h < REP; ++h) {
@@ -180,25 +192,53 @@ __global__ void __launch_bounds__(kDecThreads) decode_gist_kernel(DecodeArgs a) 
   };
   const int e0 = slice * kGistSlice, e1 = min(a.G, e0 + kGistSlice);
   float* sc = a.scores + ((int64_t)seq * a.Hkv + g) * a.G;
-  attend_slice<REP>(a, qf, e0, e1, row, sc, seq, g, slice);
+  float* lg = a.rule == SA_SELECT_SUM_PROBS_PER_GROUP
+                  ? a.logits + ((int64_t)seq * a.Hq + g * a.rep) * a.G
+                  : nullptr;
+  attend_slice<REP>(a, qf, e0, e1, row, sc, lg, seq, g, slice);
 }
 
-// Order-preserving map of a float to an unsigned key.
+// Order-preserving map of a float to an unsigned key, and back.
 __device__ __forceinline__ uint32_t float_key(float f) {
   const uint32_t u = __float_as_uint(f);
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float key_float(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
 }
 
 __global__ void __launch_bounds__(1024) decode_select_kernel(DecodeArgs a, int pow2) {
   extern __shared__ unsigned long long keys[];
   __shared__ int chosen[256];
   const int g = blockIdx.x, seq = blockIdx.y;
+  __shared__ float lse_h[kDecMaxRep];
+  __shared__ float red[32];
+  __shared__ int n_keep_s;
   const float* sc = a.scores + ((int64_t)seq * a.Hkv + g) * a.G;
+  const bool probs = a.rule == SA_SELECT_SUM_PROBS_PER_GROUP;
+  const float* lg = a.logits + ((int64_t)seq * a.Hq + g * a.rep) * a.G;
+  if (probs && threadIdx.x < a.rep) {
+    // head h's log-sum-exp over all gists, from its gist-slice partials
+    const float* p = a.part + ((int64_t)seq * a.Hq + g * a.rep + threadIdx.x) * a.n_part * (2 + kDecD);
+    float M = -INFINITY;
+    for (int t = 0; t < a.n_gslices; ++t) M = fmaxf(M, p[t * (2 + kDecD)]);
+    float L = 0.f;
+    for (int t = 0; t < a.n_gslices; ++t)
+      if (p[t * (2 + kDecD)] != -INFINITY) L += p[t * (2 + kDecD) + 1] * expf(p[t * (2 + kDecD)] - M);
+    lse_h[threadIdx.x] = M + logf(L);
+  }
+  __syncthreads();
   const int last_ok = a.cache_len - a.window;  // chunk c eligible iff (c+1)*chunk <= last_ok
   for (int i = threadIdx.x; i < pow2; i += blockDim.x) {
     unsigned long long kk = 0ull;
-    if (i < a.G && (int64_t)(i + 1) * a.chunk <= last_ok)
-      kk = ((unsigned long long)float_key(sc[i]) << 32) | (0xFFFFFFFFu - (uint32_t)i);
+    if (i < a.G && (int64_t)(i + 1) * a.chunk <= last_ok) {
+      float v = sc[i];
+      if (probs) {
+        v = 0.f;
+        for (int h = 0; h < a.rep; ++h) v += expf(lg[(int64_t)h * a.G + i] - lse_h[h]);
+      }
+      kk = ((unsigned long long)float_key(v) << 32) | (0xFFFFFFFFu - (uint32_t)i);
+    }
     keys[i] = kk;
   }
   __syncthreads();
@@ -217,9 +257,38 @@ __global__ void __launch_bounds__(1024) decode_select_kernel(DecodeArgs a, int p
     }
   }
   const int k = a.top_k;
+  if (threadIdx.x == 0) n_keep_s = k;
+  if (a.rule == SA_SELECT_TOP_P_PER_GROUP && k > 0 && keys[0] != 0ull) {
+    // softmax over the eligible chunks (keys[0] holds the best score), then the
+    // shortest prefix of the sorted keys whose probability reaches p
+    const float smax = key_float((uint32_t)(keys[0] >> 32));
+    float z = 0.f;
+    for (int i = threadIdx.x; i < pow2; i += blockDim.x)
+      if (keys[i] != 0ull) z += expf(key_float((uint32_t)(keys[i] >> 32)) - smax);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = z;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      float Z = 0.f;
+      for (int w = 0; w < (int)(blockDim.x >> 5); ++w) Z += red[w];
+      const float thr = a.top_p * Z;
+      float cum = 0.f;
+      int n = 0;
+      for (int t = 0; t < k && t < pow2 && keys[t] != 0ull; ++t) {
+        if (n > 0 && cum >= thr) break;
+        cum += expf(key_float((uint32_t)(keys[t] >> 32)) - smax);
+        ++n;
+      }
+      n_keep_s = n;
+    }
+  }
+  __syncthreads();
+  const int n_keep = n_keep_s;
   for (int t = threadIdx.x; t < k; t += blockDim.x)
-    chosen[t] = (t < pow2 && keys[t] != 0ull) ? (int)(0xFFFFFFFFu - (uint32_t)(keys[t] & 0xFFFFFFFFull))
-                                              : 0x7FFFFFFF;
+    chosen[t] = (t < n_keep && t < pow2 && keys[t] != 0ull)
+                    ? (int)(0xFFFFFFFFu - (uint32_t)(keys[t] & 0xFFFFFFFFull))
+                    : 0x7FFFFFFF;
   __syncthreads();
   int32_t* out = a.sel + ((int64_t)seq * a.Hkv + g) * k;
   for (int t = threadIdx.x; t < k; t += blockDim.x) {
@@ -258,7 +327,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_raw_kernel(DecodeArgs a) {
     vr = vc + pos * rs;
   };
   const int e0 = min(total, slice * kRawSlice), e1 = min(total, e0 + kRawSlice);
-  attend_slice<REP>(a, qf, e0, e1, row, nullptr, seq, g, a.n_gslices + slice);
+  attend_slice<REP>(a, qf, e0, e1, row, nullptr, nullptr, seq, g, a.n_gslices + slice);
 }
 
 __global__ void decode_combine_kernel(DecodeArgs a) {
@@ -281,7 +350,7 @@ __global__ void decode_combine_kernel(DecodeArgs a) {
 // ------------------------------------------------------------- host side
 struct DecodePlan {
   int n_gslices, n_rslices, n_part, pow2;
-  size_t scores_off, part_off, bytes;
+  size_t scores_off, part_off, logits_off, bytes;
 };
 
 DecodePlan decode_plan(const sa_decode_desc& d) {
@@ -296,7 +365,11 @@ DecodePlan decode_plan(const sa_decode_desc& d) {
   size_t sb = (size_t)d.n_seq * d.num_kv_heads * d.n_gists * sizeof(float);
   p.part_off = p.scores_off + ((sb + 255) / 256) * 256;
   size_t pb = (size_t)d.n_seq * d.num_q_heads * p.n_part * (2 + kDecD) * sizeof(float);
-  p.bytes = p.part_off + pb;
+  p.logits_off = p.part_off + ((pb + 255) / 256) * 256;
+  size_t lb = d.select_rule == SA_SELECT_SUM_PROBS_PER_GROUP
+                  ? (size_t)d.n_seq * d.num_q_heads * d.n_gists * sizeof(float)
+                  : 0;
+  p.bytes = p.logits_off + lb;
   return p;
 }
 
@@ -324,16 +397,17 @@ static cudaError_t decode_launch_rep(const DecodeArgs& a, const DecodePlan& pl, 
 bool decode_tc_supported(const sa_decode_desc& d);
 cudaError_t launch_decode_tc(const sa_decode_desc& d, const void* q, const void* gk,
                              const void* gv, const void* kc, const void* vc, int32_t* sel, void* o,
-                             float* lse, void* ws, cudaStream_t s);
+                             float* lse, void* ws, float* logits, cudaStream_t s);
 
 // The tensor-core kernel (one CTA per sequence and KV head) takes the shapes it
 // supports; the four-pass CUDA-core kernels below take the rest.
 cudaError_t launch_decode(const sa_decode_desc& d, const void* q, const void* gk, const void* gv,
                           const void* kc, const void* vc, int32_t* sel, void* o, float* lse,
                           void* ws, cudaStream_t s) {
-  if (decode_tc_supported(d))
-    return launch_decode_tc(d, q, gk, gv, kc, vc, sel, o, lse, ws, s);
   const DecodePlan pl = decode_plan(d);
+  float* logits = (float*)((char*)ws + pl.logits_off);
+  if (decode_tc_supported(d))
+    return launch_decode_tc(d, q, gk, gv, kc, vc, sel, o, lse, ws, logits, s);
   DecodeArgs a{};
   a.q = (const __nv_bfloat16*)q;
   a.gk = (const __nv_bfloat16*)gk;
@@ -345,6 +419,9 @@ cudaError_t launch_decode(const sa_decode_desc& d, const void* q, const void* gk
   a.lse = lse;
   a.scores = (float*)((char*)ws + pl.scores_off);
   a.part = (float*)((char*)ws + pl.part_off);
+  a.logits = logits;
+  a.rule = d.select_rule;
+  a.top_p = d.top_p;
   a.n_seq = d.n_seq; a.cache_len = d.cache_len; a.chunk = d.chunk; a.G = d.n_gists;
   a.top_k = d.top_k; a.window = d.window; a.Hq = d.num_q_heads; a.Hkv = d.num_kv_heads;
   a.rep = d.num_q_heads / d.num_kv_heads;

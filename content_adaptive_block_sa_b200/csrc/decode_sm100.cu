@@ -14,7 +14,11 @@
 //      loaded while step 3 runs).
 //   3. top-k selection over the eligible chunks (wholly before the window) by
 //      a 4-pass radix select on the order-preserving 32-bit key of the score,
-//      ties to the lower chunk index, written ascending (-1 padded).
+//      ties to the lower chunk index, written ascending (-1 padded). The
+//      sum-of-probabilities rule stores each head's logits during step 1 and
+//      scores gist j by sum_h 2^(s_hj - m_h) / l_h with the heads' gist-only
+//      softmax state; the top-p rule then keeps the shortest score-ordered
+//      prefix of the top_k whose softmax over the eligible chunks reaches p.
 //   4. chunk blocks: 128 / chunk selected chunks per block, each brought in
 //      by its own TMA box.
 // The output O = O^T / l and LSE follow from the single softmax state; no
@@ -60,7 +64,10 @@ struct Params {
   __nv_bfloat16* o;
   float* lse;
   int32_t* sel;
+  float* logits;         // [n_seq, Hq, G] raw dot products (sum-of-probabilities rule)
   DeviceStatus* status;
+  int rule;
+  float top_p;
   int n_seq, Hkv, rep, G, cache_len, chunk, top_k, window;
   int nG, nW, nC;        // gist, window and chunk blocks
   float scale;
@@ -366,7 +373,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
       if (b < P.nG) {
         const int key = b * kBlk + r;
         valid = key < P.G;
-        if (valid) {  // selection score: sum over the group's heads of q_h . k * scale
+        if (valid && P.rule == SA_SELECT_SUM_PROBS_PER_GROUP) {
+          float* lg = P.logits + (int64_t)(seq * P.Hkv + g) * REP * P.G + key;
+#pragma unroll
+          for (int h = 0; h < REP; ++h) lg[(int64_t)h * P.G] = sv[h];
+        } else if (valid) {  // selection score: sum over the group's heads of q_h . k * scale
           float sum = 0.f;
 #pragma unroll
           for (int h = 0; h < REP; ++h) sum += sv[h];
@@ -435,8 +446,41 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
         // ---------------------------------------------------- top-k select
         // thread r owns gists [r * per, r * per + per): ascending index order
         // across threads, so an exclusive scan keeps the output ascending
-        ok = ok && gs(30);  // every score is written
+        __threadfence_block();
+        ok = ok && gs(30);  // every score (or logit) is written
         const int per = (P.G + 127) / 128, j0 = r * per, j1 = min(P.G, j0 + per);
+        // sum or max over the 128 softmax threads (hist serves as scratch)
+        auto group_reduce = [&](float v, bool is_max) -> float {
+#pragma unroll
+          for (int off = 16; off > 0; off >>= 1) {
+            const float y = __shfl_xor_sync(0xffffffffu, v, off);
+            v = is_max ? fmaxf(v, y) : v + y;
+          }
+          float* buf = reinterpret_cast<float*>(hist);
+          if (lane == 0) buf[sw] = v;
+          ok = ok && gs(42);
+          const float t = is_max ? fmaxf(fmaxf(buf[0], buf[1]), fmaxf(buf[2], buf[3]))
+                                 : (buf[0] + buf[1]) + (buf[2] + buf[3]);
+          ok = ok && gs(43);  // buf may be reused after this
+          return t;
+        };
+        if (P.rule == SA_SELECT_SUM_PROBS_PER_GROUP) {
+          // each head's softmax over all gists: the state after the gist blocks
+          float inv_l[REP];
+#pragma unroll
+          for (int h = 0; h < REP; ++h) {
+            const float l = group_reduce(l_part[h], false);
+            inv_l[h] = l > 0.f ? 1.f / l : 0.f;
+          }
+          const float* lg = P.logits + (int64_t)(seq * P.Hkv + g) * REP * P.G;
+          for (int j = j0; j < j1; ++j) {
+            float sum = 0.f;
+#pragma unroll
+            for (int h = 0; h < REP; ++h)
+              sum += ex2(fmaf(lg[(int64_t)h * P.G + j], sl2, -m_run[h])) * inv_l[h];
+            scores[j] = sum;
+          }
+        }
         const int64_t last_ok = (int64_t)P.cache_len - P.window;
         auto key_of = [&](int j) -> uint32_t {
           return ((int64_t)(j + 1) * P.chunk <= last_ok) ? float_key(scores[j]) : 0u;
@@ -515,6 +559,43 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
         for (int x = r; x < P.top_k; x += 128)
           if (x >= (int)sel_total) sel_s[x] = -1;
         ok = ok && gs(35);
+        const int nsel = min((int)sel_total, P.top_k);
+        if (P.rule == SA_SELECT_TOP_P_PER_GROUP && nsel > 0) {
+          // softmax over the eligible chunks (the best score is among the
+          // selected); selected entry x is kept iff the probability of the
+          // entries ranked above it (score descending, lower index first) is
+          // below p: the shortest prefix reaching p. Thread r decides for
+          // entries 2r and 2r + 1, so a scan keeps the ascending order.
+          float smax = -INFINITY;
+          for (int x = r; x < nsel; x += 128) smax = fmaxf(smax, scores[sel_s[x]]);
+          smax = group_reduce(smax, true);
+          float z = 0.f;
+          for (int j = j0; j < j1; ++j)
+            if (key_of(j) != 0u) z += __expf(scores[j] - smax);
+          const float thr = P.top_p * group_reduce(z, false);
+          int val[2];
+          uint32_t nk = 0u;
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int x = 2 * r + u;
+            val[u] = -1;
+            if (x < nsel) {
+              const float sx = scores[sel_s[x]];
+              float above = 0.f;
+              for (int y = 0; y < nsel; ++y) {
+                const float sy = scores[sel_s[y]];
+                if (sy > sx || (sy == sx && y < x)) above += __expf(sy - smax);
+              }
+              if (above < thr) val[nk++] = sel_s[x];
+            }
+          }
+          uint32_t kept = 0u;
+          const uint32_t base = group_exclusive_scan(nk, r, scan, gs, ok, &kept);
+          for (uint32_t u = 0; u < nk; ++u) sel_s[base + u] = val[u];
+          for (int x = r; x < P.top_k; x += 128)
+            if (x >= (int)kept) sel_s[x] = -1;
+          ok = ok && gs(39);
+        }
         int32_t* sel_out = P.sel + ((int64_t)seq * P.Hkv + g) * P.top_k;
         for (int x = r; x < P.top_k; x += 128) sel_out[x] = sel_s[x];
         mbar_arrive(&bar[B_SELD]);  // release: sel_s is complete
@@ -578,7 +659,7 @@ static cudaError_t decode_tc_launch(const Params& P, cudaStream_t s) {
 
 cudaError_t launch_decode_tc(const sa_decode_desc& d, const void* q, const void* gk,
                              const void* gv, const void* kc, const void* vc, int32_t* sel, void* o,
-                             float* lse, void* ws, cudaStream_t s) {
+                             float* lse, void* ws, float* logits, cudaStream_t s) {
   Params P;
   memset(&P, 0, sizeof(P));
   const int64_t gstr[3] = {d.gist_strides[0], d.gist_strides[2], d.gist_strides[1]};
@@ -594,6 +675,9 @@ cudaError_t launch_decode_tc(const sa_decode_desc& d, const void* q, const void*
   P.o = static_cast<__nv_bfloat16*>(o);
   P.lse = lse;
   P.sel = sel;
+  P.logits = logits;
+  P.rule = d.select_rule;
+  P.top_p = d.top_p;
   P.status = static_cast<DeviceStatus*>(ws);
   P.n_seq = d.n_seq;
   P.Hkv = d.num_kv_heads;

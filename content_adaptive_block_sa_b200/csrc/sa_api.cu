@@ -414,7 +414,11 @@ static sa_status check_decode(const sa_decode_desc* d) {
   const int rep = d->num_q_heads / d->num_kv_heads;
   SA_CHECK(rep == 1 || rep == 2 || rep == 4 || rep == 8, SA_ERR_UNSUPPORTED);
   SA_CHECK(d->head_dim == 128, SA_ERR_UNSUPPORTED);
-  SA_CHECK(d->select_rule == SA_SELECT_SUM_LOGITS_PER_GROUP, SA_ERR_UNSUPPORTED);
+  SA_CHECK(d->select_rule >= SA_SELECT_SUM_LOGITS_PER_GROUP &&
+               d->select_rule <= SA_SELECT_TOP_P_PER_GROUP,
+           SA_ERR_INVALID_ARG);
+  if (d->select_rule == SA_SELECT_TOP_P_PER_GROUP)
+    SA_CHECK(d->top_p > 0.f && d->top_p <= 1.f, SA_ERR_INVALID_ARG);
   SA_CHECK(d->softmax_scale >= 0.f && isfinite(d->softmax_scale), SA_ERR_INVALID_ARG);
   // 16-byte row loads
   SA_CHECK(d->gist_strides[2] % 8 == 0 && d->cache_strides[2] % 8 == 0, SA_ERR_INVALID_ARG);

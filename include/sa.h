@@ -234,7 +234,23 @@ typedef struct sa_attn_desc {
   int32_t impl;
 } sa_attn_desc;
 
-typedef enum { SA_SELECT_SUM_LOGITS_PER_GROUP = 0 } sa_select_rule;
+/* Chunk selection at decode (one selection per KV group).
+ *  SUM_LOGITS_PER_GROUP  top_k chunks by the sum over the group's query heads
+ *                        of q_h . gist_k * scale.
+ *  SUM_PROBS_PER_GROUP   top_k chunks by the sum over the group's query heads
+ *                        of each head's softmax over all the group's gists.
+ *  TOP_P_PER_GROUP       the group's summed logits, softmax over the eligible
+ *                        chunks: the smallest score-ordered prefix whose
+ *                        probability reaches top_p, at most top_k chunks.
+ * Ties go to the lower chunk index in every rule. The pages of "Simplified
+ * Sparse Attention via Gist Tokens" name a top-k and a top-p selection from
+ * logits and a per-group selection; the three readings above are this
+ * library's. */
+typedef enum {
+  SA_SELECT_SUM_LOGITS_PER_GROUP = 0,
+  SA_SELECT_SUM_PROBS_PER_GROUP = 1,
+  SA_SELECT_TOP_P_PER_GROUP = 2
+} sa_select_rule;
 
 /* Decode shapes (one new query token per sequence).
  *  q          [n_seq, Hq, d]            strides q_strides {seq, head}
@@ -248,9 +264,8 @@ typedef enum { SA_SELECT_SUM_LOGITS_PER_GROUP = 0 } sa_select_rule;
  *  window     the last `window` cache positions are always attended; a chunk
  *             is eligible for selection iff it lies entirely before them.
  *  top_k      chunks unfolded per (sequence, KV head), 0 <= top_k <= 256.
- *  select_rule  SA_SELECT_SUM_LOGITS_PER_GROUP: a chunk's score is the sum
- *             over the KV group's query heads of q_h . gist_k * scale; ties go
- *             to the lower chunk index.
+ *  select_rule  an sa_select_rule (see above).
+ *  top_p      TOP_P_PER_GROUP only: 0 < top_p <= 1.
  * All bf16; head_dim 128; Hq / Hkv <= 8.
  */
 typedef struct sa_decode_desc {
@@ -269,6 +284,7 @@ typedef struct sa_decode_desc {
   int64_t gist_strides[3];
   int64_t cache_strides[3];
   int64_t o_strides[2];
+  float top_p;
 } sa_decode_desc;
 
 /* ------------------------------------------------------------------ misc */

@@ -42,9 +42,55 @@ def upload_workload(w):
     return q, gk, gv, dev(q), dev(gk), dev(gv), kc, vc
 
 
-def check(sa, w, seqs=None):
+def logit_bound(q, gk, s, g, rep, d):
+    """Float32 accumulation bound of each chunk's summed logit (see above)."""
+    qg = np.abs(q[s, g * rep:(g + 1) * rep].astype(np.float64))
+    return lambda c: 2 * d * 2.0 ** -24 / np.sqrt(d) * (qg @ np.abs(gk[s, g, c])).sum()
+
+
+def valid_alternative(w, rule, top_p, q, gk, s, g, got, want_scores):
+    """Is the kernel's selection `got` (ascending, -1 padded) one the rule
+    admits given float32 near ties? Sum of logits / of probabilities: a top-k
+    set whose boundary scores are within their rounding bounds. Top-p: a
+    score-ordered prefix (up to the same near ties) that reaches p and is
+    shortest, each up to 1e-4 of probability."""
+    d, rep = w["head_dim"], w["heads"] // w["kv_heads"]
+    elig = D.eligible_chunks(w["n_gists"], w["chunk"], w["cache_len"], w["window"])
+    K = got[got >= 0]
+    assert elig[K].all() and len(set(K.tolist())) == len(K)
+    sc = np.where(elig, want_scores, -np.inf)
+    if rule == D.SUM_PROBS:
+        # a probability moves by about p * (its logit error + the normaliser's)
+        b = logit_bound(q, gk, s, g, rep, d)
+        bound = lambda c: want_scores[c] * (b(c) + 1e-5)
+    else:
+        bound = logit_bound(q, gk, s, g, rep, d)
+    rest = np.setdiff1d(np.nonzero(elig)[0], K)
+    if len(K) and len(rest):
+        c_in = K[np.argmin(sc[K])]
+        c_out = rest[np.argmax(sc[rest])]
+        assert sc[c_out] - sc[c_in] <= bound(c_in) + bound(c_out), (s, g, sc[c_in], sc[c_out])
+    n_el = int(elig.sum())
+    if rule != D.TOP_P:
+        assert len(K) == min(w["top_k"], n_el)
+        return
+    if n_el == 0 or w["top_k"] == 0:
+        assert len(K) == 0
+        return
+    e = np.exp(sc[elig] - sc[elig].max())
+    prob = np.zeros(len(sc))
+    prob[elig] = e / e.sum()
+    assert 1 <= len(K) <= w["top_k"]
+    if len(K) < min(w["top_k"], n_el):
+        assert prob[K].sum() >= top_p - 1e-4
+    shorter = np.delete(K, np.argmin(sc[K]))
+    assert prob[shorter].sum() < top_p + 1e-4
+
+
+def check(sa, w, seqs=None, rule=0, top_p=1.0):
     q, gk, gv, tq, tgk, tgv, kc, vc = upload_workload(w)
-    sel, o, lse = sa.gist_decode(tq, tgk, tgv, kc, vc, w["chunk"], w["top_k"], w["window"])
+    sel, o, lse = sa.gist_decode(tq, tgk, tgv, kc, vc, w["chunk"], w["top_k"], w["window"],
+                                 select_rule=rule, top_p=top_p)
     torch.cuda.synchronize()
     ws = sa.gist_decode.last_workspace
     st = ws[:8].view(torch.int32).cpu().tolist()
@@ -55,19 +101,11 @@ def check(sa, w, seqs=None):
         raw_k = lambda g: to_np(kc[s, g])
         raw_v = lambda g: to_np(vc[s, g])
         osel, oo, ol, scores = D.decode_one(q[s], gk[s], gv[s], raw_k, raw_v, w["chunk"],
-                                            w["window"], w["top_k"])
+                                            w["window"], w["top_k"], rule=rule, top_p=top_p)
         for g in range(w["kv_heads"]):
             if not np.array_equal(sel[s, g], osel[g]):
-                # accept a different set only across a float32-level near tie
-                elig = D.eligible_chunks(w["n_gists"], w["chunk"], w["cache_len"], w["window"])
-                sc = np.where(elig, scores[g], -np.inf)
-                order = np.argsort(-sc, kind="stable")
-                c_in, c_out = order[w["top_k"] - 1], order[w["top_k"]]
-                d = w["head_dim"]
-                qg = np.abs(q[s, g * rep:(g + 1) * rep].astype(np.float64))
-                bound = lambda c: 2 * d * 2.0 ** -24 / np.sqrt(d) * (qg @ np.abs(gk[s, g, c])).sum()
-                gap = sc[c_in] - sc[c_out]
-                assert gap <= bound(c_in) + bound(c_out), (s, g, gap, sel[s, g], osel[g])
+                # accept a different set only where float32 rounding can decide it
+                valid_alternative(w, rule, top_p, q, gk, s, g, sel[s, g], scores[g])
                 # O must then match the oracle evaluated on the GPU's own set
                 pos = D.raw_key_positions(sel[s, g], w["chunk"], w["cache_len"], w["window"])
                 keys = np.concatenate([gk[s, g], raw_k(g)[pos]])
@@ -110,3 +148,25 @@ def test_decode_tensor_core_shapes(sa, top_k, window, chunk, G):
     w = W.scaled("gist_decode_128k", index=500 + top_k + G, n_seq=2, cache_len=chunk * G,
                  chunk=chunk, n_gists=G, top_k=top_k, window=window, heads=8, kv_heads=2)
     check(sa, w)
+
+
+RULES = {"sum_probs": (1, 1.0), "top_p_0.3": (2, 0.3), "top_p_0.9": (2, 0.9), "top_p_1": (2, 1.0)}
+
+
+@pytest.mark.parametrize("rule", list(RULES))
+@pytest.mark.parametrize("top_k,window,chunk,G", [(8, 64, 16, 64), (60, 64, 16, 64), (5, 0, 32, 40),
+                                                  (40, 0, 32, 256), (256, 128, 8, 200),
+                                                  (33, 300, 64, 777)])
+def test_decode_select_rules(sa, rule, top_k, window, chunk, G):
+    """Sum-of-probabilities and top-p selection on both kernels (G < 128 or a
+    chunk of 16 with 64 gists takes the CUDA-core path, the rest the tensor cores)."""
+    w = W.scaled("gist_decode_128k", index=600 + top_k + G, n_seq=2, cache_len=chunk * G,
+                 chunk=chunk, n_gists=G, top_k=top_k, window=window, heads=8, kv_heads=2)
+    r, p = RULES[rule]
+    check(sa, w, rule=r, top_p=p)
+
+
+@pytest.mark.parametrize("rule", ["sum_probs", "top_p_0.9"])
+def test_decode_select_rules_full_size(sa, rule):
+    r, p = RULES[rule]
+    check(sa, W.WORKLOADS["gist_decode_128k"], seqs=[0, 15], rule=r, top_p=p)
