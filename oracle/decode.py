@@ -25,6 +25,9 @@ top-k one; the pages give nothing more):
 * sum of probabilities: each query head's softmax over all gists of its
   group (the attention it would pay to the gists alone), summed over the
   group's heads, ranks the chunks; top-k as above;
+* per query head: every query head ranks the chunks by its own q_h . k_gist
+  * scale and unfolds its own top-k; it attends over the gists, its own
+  chunks and the window (the selection is reported per query head);
 * top-p: the group scores (sum of logits) are turned into probabilities by a
   softmax over the eligible chunks; taking chunks in score order (ties to the
   lower index), the smallest prefix whose probability reaches p is kept, at
@@ -119,14 +122,15 @@ def attend(qh, keys, values, scale):
     return np.exp(s - lse) @ np.asarray(values, np.float64), lse
 
 
-SUM_LOGITS, SUM_PROBS, TOP_P = 0, 1, 2
+SUM_LOGITS, SUM_PROBS, TOP_P, PER_HEAD = 0, 1, 2, 3
 
 
 def decode_one(q, gist_k, gist_v, raw_k, raw_v, chunk, window, top_k, scale=None,
                rule=SUM_LOGITS, top_p=1.0):
     """One sequence. ``rule``: SUM_LOGITS (top-k of the summed logits),
-    SUM_PROBS (top-k of the summed per-head probabilities) or TOP_P (top-p of
-    the summed logits, at most top_k chunks).
+    SUM_PROBS (top-k of the summed per-head probabilities), TOP_P (top-p of
+    the summed logits, at most top_k chunks) or PER_HEAD (each query head's
+    own top-k; then sel is [Hq, top_k] and scores [Hq, G]).
 
     q [Hq, d]; gist_k/gist_v [Hkv, G, d]; raw_k/raw_v: callables
     (kv_head) -> [cache_len, d] (or arrays [Hkv, cache_len, d]).
@@ -143,6 +147,22 @@ def decode_one(q, gist_k, gist_v, raw_k, raw_v, chunk, window, top_k, scale=None
     sel = np.empty((Hkv, top_k), np.int32)
     o = np.empty((Hq, d))
     lse = np.empty(Hq)
+    if rule == PER_HEAD:
+        # one selection per query head, from that head's own logits
+        scores = np.stack([(np.asarray(gist_k[h // rep], np.float64) @ q[h]) * scale
+                           for h in range(Hq)])
+        sel = np.empty((Hq, top_k), np.int32)
+        for h in range(Hq):
+            rk, rv = get_k(h // rep), get_v(h // rep)
+            cache_len = rk.shape[0]
+            sel[h] = select_top_k(scores[h], eligible_chunks(G, chunk, cache_len, window), top_k)
+            pos = raw_key_positions(sel[h], chunk, cache_len, window)
+            keys = np.concatenate([np.asarray(gist_k[h // rep], np.float64),
+                                   np.asarray(rk[pos], np.float64)])
+            vals = np.concatenate([np.asarray(gist_v[h // rep], np.float64),
+                                   np.asarray(rv[pos], np.float64)])
+            o[h], lse[h] = attend(q[h], keys, vals, scale)
+        return sel, o, lse, scores
     for g in range(Hkv):
         rk, rv = get_k(g), get_v(g)
         cache_len = rk.shape[0]

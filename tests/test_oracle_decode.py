@@ -158,3 +158,29 @@ def test_top_p_one_equals_top_k():
     elig = D.eligible_chunks(len(s), 16, 512, 64)
     for k in (1, 5, 20):
         assert np.array_equal(D.select_top_p(s, elig, k, 1.0), D.select_top_k(s, elig, k))
+
+
+def test_per_head_selection_reduces_to_group_rule_with_one_head_per_group():
+    q, gk, gv, rk, rv = _case(6, Hq=2, Hkv=2)
+    a = D.decode_one(q, gk, gv, rk, rv, 16, 64, 5, rule=D.PER_HEAD)
+    b = D.decode_one(q, gk, gv, rk, rv, 16, 64, 5)
+    assert np.array_equal(a[0], b[0])
+    np.testing.assert_allclose(a[1], b[1], atol=1e-12)
+
+
+def test_per_head_selection_is_each_heads_best_set_and_its_own_attention():
+    q, gk, gv, rk, rv = _case(8)
+    sel, o, lse, scores = D.decode_one(q, gk, gv, rk, rv, 16, 64, 6, rule=D.PER_HEAD)
+    elig = D.eligible_chunks(32, 16, 512, 64)
+    for h in range(8):
+        g = h // 4
+        s_h = gk[g] @ q[h] / 4.0
+        best = np.argsort(-np.where(elig, s_h, -np.inf), kind="stable")[:6]
+        assert sorted(best.tolist()) == sel[h].tolist()
+        pos = np.concatenate([np.arange(c * 16, c * 16 + 16) for c in sel[h]] + [np.arange(448, 512)])
+        ref_o, ref_l = _softmax_attend(q[h], np.concatenate([gk[g], rk[g][pos]]),
+                                       np.concatenate([gv[g], rv[g][pos]]))
+        np.testing.assert_allclose(o[h], ref_o, atol=1e-12)
+        assert abs(lse[h] - ref_l) < 1e-12
+    # heads of one group generally pick different chunks
+    assert any(not np.array_equal(sel[0], sel[h]) for h in range(1, 4))
