@@ -274,14 +274,16 @@ def gist_decode(q, gist_k, gist_v, k_cache, v_cache, chunk: int, top_k: int, win
                 softmax_scale: float = 0.0, stream=None, select_rule: int = 0, top_p: float = 1.0):
     """(sel int32 [n_seq, Hkv, top_k], o bf16 [n_seq, Hq, d], lse fp32 [n_seq, Hq]).
     select_rule: 0 top-k of summed logits, 1 top-k of summed per-head
-    probabilities, 2 top-p (at most top_k chunks) of the summed logits."""
+    probabilities, 2 top-p (at most top_k chunks) of the summed logits, 3 each
+    query head's own top-k (sel is then [n_seq, Hq, top_k])."""
     if gist_v.stride() != gist_k.stride() or v_cache.stride() != k_cache.stride():
         raise ValueError("K and V must share strides")
     n_seq, Hq, d = q.shape
     Hkv = gist_k.shape[1]
     o = torch.empty_like(q)
     lse = torch.empty(n_seq, Hq, dtype=torch.float32, device=q.device)
-    sel = torch.empty(n_seq, Hkv, max(top_k, 1), dtype=torch.int32, device=q.device)
+    rows = Hq if select_rule == _abi.SA_SELECT_TOP_K_PER_HEAD else Hkv
+    sel = torch.empty(n_seq, rows, max(top_k, 1), dtype=torch.int32, device=q.device)
     dd = decode_desc(q, gist_k, k_cache, o, chunk, top_k, window, softmax_scale, select_rule, top_p)
     ws = decode_workspace(dd, q.device)
     sa_gist_decode(dd, q, gist_k, gist_v, k_cache, v_cache, sel, o, lse, ws, stream)

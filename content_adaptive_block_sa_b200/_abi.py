@@ -18,6 +18,7 @@ SA_TILE_FULL, SA_TILE_MASKED, SA_TILE_TAIL = 0, 1, 2
 SA_SELECT_SUM_LOGITS_PER_GROUP = 0
 SA_SELECT_SUM_PROBS_PER_GROUP = 1
 SA_SELECT_TOP_P_PER_GROUP = 2
+SA_SELECT_TOP_K_PER_HEAD = 3
 SA_IMPL_AUTO, SA_IMPL_CUDA_CORES, SA_IMPL_TENSOR_CORES = 0, 1, 2
 SA_TILE = 128
 

@@ -80,10 +80,11 @@ struct HalfState {
 
 // Processes keys [e0, e1) of a key list given by `row` (returns k/v row
 // pointers) and writes one partial per head to `out` (slot `slot`).
-template <int REP, typename RowFn>
+// heads_of(e) gives the query heads (bits) that see key e.
+template <int REP, typename RowFn, typename HeadsFn>
 __device__ void attend_slice(const DecodeArgs& a, const float (*qf)[kDecD], int e0, int e1,
-                             RowFn row, float* score_out, float* logit_out, int seq, int g,
-                             int slot) {
+                             RowFn row, HeadsFn heads_of, float* score_out, float* logit_out,
+                             int seq, int g, int slot) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int half = lane >> 4, hl = lane & 15;  // 16 lanes per key row
   HalfState<REP> st;
@@ -124,8 +125,10 @@ __device__ void attend_slice(const DecodeArgs& a, const float (*qf)[kDecD], int 
 #pragma unroll
       for (int h = 0; h < REP; ++h) logit_out[(int64_t)h * a.G + e] = s[h];
     if (!valid) continue;
+    const uint32_t hv = heads_of(e);
 #pragma unroll
     for (int h = 0; h < REP; ++h) {
+      if (!((hv >> h) & 1u)) continue;
       const float mnew = fmaxf(st.m[h], s[h]);
       const float alpha = expf(st.m[h] - mnew);
       const float p = expf(s[h] - mnew);
@@ -192,10 +195,10 @@ __global__ void __launch_bounds__(kDecThreads) decode_gist_kernel(DecodeArgs a) 
   };
   const int e0 = slice * kGistSlice, e1 = min(a.G, e0 + kGistSlice);
   float* sc = a.scores + ((int64_t)seq * a.Hkv + g) * a.G;
-  float* lg = a.rule == SA_SELECT_SUM_PROBS_PER_GROUP
+  float* lg = (a.rule == SA_SELECT_SUM_PROBS_PER_GROUP || a.rule == SA_SELECT_TOP_K_PER_HEAD)
                   ? a.logits + ((int64_t)seq * a.Hq + g * a.rep) * a.G
                   : nullptr;
-  attend_slice<REP>(a, qf, e0, e1, row, sc, lg, seq, g, slice);
+  attend_slice<REP>(a, qf, e0, e1, row, [](int) { return 0xFFFFFFFFu; }, sc, lg, seq, g, slice);
 }
 
 // Order-preserving map of a float to an unsigned key, and back.
@@ -214,7 +217,10 @@ __global__ void __launch_bounds__(1024) decode_select_kernel(DecodeArgs a, int p
   __shared__ float lse_h[kDecMaxRep];
   __shared__ float red[32];
   __shared__ int n_keep_s;
-  const float* sc = a.scores + ((int64_t)seq * a.Hkv + g) * a.G;
+  // per-head rule: blockIdx.x is the query head and its logits are the scores
+  const bool per_head = a.rule == SA_SELECT_TOP_K_PER_HEAD;
+  const float* sc = per_head ? a.logits + ((int64_t)seq * a.Hq + g) * a.G
+                             : a.scores + ((int64_t)seq * a.Hkv + g) * a.G;
   const bool probs = a.rule == SA_SELECT_SUM_PROBS_PER_GROUP;
   const float* lg = a.logits + ((int64_t)seq * a.Hq + g * a.rep) * a.G;
   if (probs && threadIdx.x < a.rep) {
@@ -290,7 +296,7 @@ __global__ void __launch_bounds__(1024) decode_select_kernel(DecodeArgs a, int p
                     ? (int)(0xFFFFFFFFu - (uint32_t)(keys[t] & 0xFFFFFFFFull))
                     : 0x7FFFFFFF;
   __syncthreads();
-  int32_t* out = a.sel + ((int64_t)seq * a.Hkv + g) * k;
+  int32_t* out = a.sel + ((int64_t)seq * (per_head ? a.Hq : a.Hkv) + g) * k;
   for (int t = threadIdx.x; t < k; t += blockDim.x) {
     const int v = chosen[t];
     int rank = 0;
@@ -302,11 +308,16 @@ __global__ void __launch_bounds__(1024) decode_select_kernel(DecodeArgs a, int p
 template <int REP>
 __global__ void __launch_bounds__(kDecThreads) decode_raw_kernel(DecodeArgs a) {
   __shared__ float qf[kDecMaxRep][kDecD];
-  __shared__ int sel_s[256];
+  __shared__ int sel_s[kDecMaxRep * 256];
   __shared__ int n_sel_s;
   const int slice = blockIdx.x, g = blockIdx.y, seq = blockIdx.z;
-  const int32_t* sel = a.sel + ((int64_t)seq * a.Hkv + g) * a.top_k;
-  for (int t = threadIdx.x; t < a.top_k; t += blockDim.x) sel_s[t] = sel[t];
+  // per-head rule: the group's heads' selections one after another (every
+  // head takes the same number of chunks); a key of head hh's chunks is seen
+  // by that head only
+  const bool per_head = a.rule == SA_SELECT_TOP_K_PER_HEAD;
+  const int nh = per_head ? a.rep : 1;
+  const int32_t* sel = a.sel + ((int64_t)seq * a.Hkv + g) * nh * a.top_k;
+  for (int t = threadIdx.x; t < nh * a.top_k; t += blockDim.x) sel_s[t] = sel[t];
   __syncthreads();
   if (threadIdx.x == 0) {
     int n = 0;
@@ -314,20 +325,30 @@ __global__ void __launch_bounds__(kDecThreads) decode_raw_kernel(DecodeArgs a) {
     n_sel_s = n;
   }
   load_group_q(a, seq, g, qf);
-  const int n_chunk_keys = n_sel_s * a.chunk;
+  const int head_keys = n_sel_s * a.chunk;
+  const int n_chunk_keys = nh * head_keys;
   const int total = n_chunk_keys + a.window;
   const __nv_bfloat16* kc = a.kc + seq * a.cs[0] + (int64_t)g * a.cs[1];
   const __nv_bfloat16* vc = a.vc + seq * a.cs[0] + (int64_t)g * a.cs[1];
   const int64_t rs = a.cs[2];
   const int chunk = a.chunk, wstart = a.cache_len - a.window;
+  const int ktop = a.top_k;
   auto row = [&](int e, const __nv_bfloat16*& kr, const __nv_bfloat16*& vr) {
-    const int pos = e < n_chunk_keys ? sel_s[e / chunk] * chunk + e % chunk
-                                     : wstart + (e - n_chunk_keys);
+    int pos;
+    if (e < n_chunk_keys) {
+      const int hh = e / head_keys, x = e - hh * head_keys;
+      pos = sel_s[hh * ktop + x / chunk] * chunk + x % chunk;
+    } else {
+      pos = wstart + (e - n_chunk_keys);
+    }
     kr = kc + pos * rs;
     vr = vc + pos * rs;
   };
+  auto heads_of = [&](int e) -> uint32_t {
+    return (per_head && e < n_chunk_keys) ? 1u << (e / head_keys) : 0xFFFFFFFFu;
+  };
   const int e0 = min(total, slice * kRawSlice), e1 = min(total, e0 + kRawSlice);
-  attend_slice<REP>(a, qf, e0, e1, row, nullptr, nullptr, seq, g, a.n_gslices + slice);
+  attend_slice<REP>(a, qf, e0, e1, row, heads_of, nullptr, nullptr, seq, g, a.n_gslices + slice);
 }
 
 __global__ void decode_combine_kernel(DecodeArgs a) {
@@ -356,7 +377,8 @@ struct DecodePlan {
 DecodePlan decode_plan(const sa_decode_desc& d) {
   DecodePlan p{};
   p.n_gslices = (d.n_gists + kGistSlice - 1) / kGistSlice;
-  const int max_raw = d.top_k * d.chunk + d.window;
+  const int heads = d.select_rule == SA_SELECT_TOP_K_PER_HEAD ? d.num_q_heads / d.num_kv_heads : 1;
+  const int max_raw = heads * d.top_k * d.chunk + d.window;
   p.n_rslices = max(1, (max_raw + kRawSlice - 1) / kRawSlice);
   p.n_part = p.n_gslices + p.n_rslices;
   p.pow2 = 1;
@@ -366,7 +388,8 @@ DecodePlan decode_plan(const sa_decode_desc& d) {
   p.part_off = p.scores_off + ((sb + 255) / 256) * 256;
   size_t pb = (size_t)d.n_seq * d.num_q_heads * p.n_part * (2 + kDecD) * sizeof(float);
   p.logits_off = p.part_off + ((pb + 255) / 256) * 256;
-  size_t lb = d.select_rule == SA_SELECT_SUM_PROBS_PER_GROUP
+  size_t lb = (d.select_rule == SA_SELECT_SUM_PROBS_PER_GROUP ||
+               d.select_rule == SA_SELECT_TOP_K_PER_HEAD)
                   ? (size_t)d.n_seq * d.num_q_heads * d.n_gists * sizeof(float)
                   : 0;
   p.bytes = p.logits_off + lb;
@@ -384,7 +407,8 @@ static cudaError_t decode_launch_rep(const DecodeArgs& a, const DecodePlan& pl, 
                              (int)smem);
     if (e != cudaSuccess) return e;
   }
-  decode_select_kernel<<<dim3(a.Hkv, a.n_seq), 1024, smem, s>>>(a, pl.pow2);
+  const int sel_rows = a.rule == SA_SELECT_TOP_K_PER_HEAD ? a.Hq : a.Hkv;
+  decode_select_kernel<<<dim3(sel_rows, a.n_seq), 1024, smem, s>>>(a, pl.pow2);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   decode_raw_kernel<REP><<<dim3(pl.n_rslices, a.Hkv, a.n_seq), kDecThreads, 0, s>>>(a);

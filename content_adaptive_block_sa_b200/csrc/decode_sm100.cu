@@ -69,6 +69,7 @@ struct Params {
   int rule;
   float top_p;
   int n_seq, Hkv, rep, G, cache_len, chunk, top_k, window;
+  int n_slots;           // unfolded chunk slots: top_k, or rep * top_k (per-head rule)
   int nG, nW, nC;        // gist, window and chunk blocks
   float scale;
   int64_t qs[2], os[2];
@@ -89,7 +90,8 @@ constexpr uint32_t OFF_HIST = OFF_SCORE + kMaxG * 4;     // uint32 [256]
 constexpr uint32_t OFF_SEL = OFF_HIST + 256 * 4;         // int32 [kMaxTopK]
 constexpr uint32_t OFF_RED = OFF_SEL + kMaxTopK * 4;     // float [2][4 warps][kN]
 constexpr uint32_t OFF_SCAN = OFF_RED + 2 * 4 * kN * 4;  // uint32 [8] + misc
-constexpr uint32_t OFF_BARS = OFF_SCAN + 64;
+constexpr uint32_t OFF_HMASK = OFF_SCAN + 64;            // uint8 [kMaxTopK]: heads per slot
+constexpr uint32_t OFF_BARS = OFF_HMASK + kMaxTopK;
 constexpr uint32_t kSmemBytes = OFF_BARS + 256 + 1024;
 
 enum {
@@ -159,6 +161,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + kNumBars);
   volatile int* abort = reinterpret_cast<volatile int*>(bar + kNumBars) + 1;
   int32_t* sel_s = reinterpret_cast<int32_t*>(smem + OFF_SEL);
+  uint8_t* hmask_s = smem + OFF_HMASK;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = blockIdx.x % P.Hkv, seq = blockIdx.x / P.Hkv;
@@ -228,7 +231,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
           for (int i = 0; i < cpb; ++i) {
             const int slot = cb * cpb + i;
             // an empty slot loads chunk 0 (finite values; its keys are masked)
-            const int c = (slot < P.top_k && sel_s[slot] >= 0) ? sel_s[slot] : 0;
+            const int c = (slot < P.n_slots && sel_s[slot] >= 0) ? sel_s[slot] : 0;
             const uint32_t roff = (uint32_t)(i * P.chunk) * 128u;
             for (int at = 0; at < 2; ++at)
               tma_load_4d(dst + at * kAtom + roff, map, full, at * 64, g, c * P.chunk, seq);
@@ -370,10 +373,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
       tc_fence_before();
       mbar_arrive(&bar[B_SE + s]);
       bool valid;
+      uint32_t hv = 0xFFFFFFFFu;  // heads that see this key (unfolded chunks of one head)
       if (b < P.nG) {
         const int key = b * kBlk + r;
         valid = key < P.G;
-        if (valid && P.rule == SA_SELECT_SUM_PROBS_PER_GROUP) {
+        if (valid && (P.rule == SA_SELECT_SUM_PROBS_PER_GROUP || P.rule == SA_SELECT_TOP_K_PER_HEAD)) {
           float* lg = P.logits + (int64_t)(seq * P.Hkv + g) * REP * P.G + key;
 #pragma unroll
           for (int h = 0; h < REP; ++h) lg[(int64_t)h * P.G] = sv[h];
@@ -387,13 +391,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
         valid = wstart + (b - P.nG) * kBlk + r < P.cache_len;
       } else {
         const int slot = (b - P.nG - P.nW) * cpb + r / P.chunk;
-        valid = slot < P.top_k && sel_s[slot] >= 0;
+        valid = slot < P.n_slots && sel_s[slot] >= 0;
+        if (valid && P.rule == SA_SELECT_TOP_K_PER_HEAD) hv = hmask_s[slot];
       }
       // block maximum per head over the four softmax warps
       float* rb = red + s * 4 * kN;
 #pragma unroll
       for (int h = 0; h < REP; ++h) {
-        float v = valid ? sv[h] : -INFINITY;
+        float v = (valid && ((hv >> h) & 1u)) ? sv[h] : -INFINITY;
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
         if (lane == 0) rb[sw * kN + h] = v;
@@ -412,7 +417,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
         const bool resc = m_new > m_run[h] + 8.f;       // the same in every thread
         const float m_use = resc ? m_new : m_run[h];
         alpha[h] = !resc ? 1.f : (m_run[h] == -INFINITY ? 0.f : ex2(m_run[h] - m_use));
-        pv[h] = (valid && m_use != -INFINITY) ? ex2(fmaf(sv[h], sl2, -m_use)) : 0.f;
+        pv[h] = (valid && ((hv >> h) & 1u) && m_use != -INFINITY) ? ex2(fmaf(sv[h], sl2, -m_use))
+                                                                  : 0.f;
         l_part[h] = l_part[h] * alpha[h] + pv[h];
         m_run[h] = m_use;
         any_resc = any_resc || resc;
@@ -485,6 +491,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
         auto key_of = [&](int j) -> uint32_t {
           return ((int64_t)(j + 1) * P.chunk <= last_ok) ? float_key(scores[j]) : 0u;
         };
+        // top_k of scores[] into sel_s (ascending, -1 padded); returns the
+        // number of eligible chunks taken
+        auto radix_select = [&]() -> uint32_t {
         uint32_t n_elig = 0;
         for (int j = j0; j < j1; ++j) n_elig += key_of(j) != 0u;
         uint32_t E = 0;
@@ -559,6 +568,60 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
         for (int x = r; x < P.top_k; x += 128)
           if (x >= (int)sel_total) sel_s[x] = -1;
         ok = ok && gs(35);
+        return sel_total;
+        };
+        if (P.rule == SA_SELECT_TOP_K_PER_HEAD) {
+          // each query head's own top_k from its logits, written to its row of
+          // sel; then the union of the group's chunks (ascending) into sel_s
+          // with, per slot, the heads that chose it
+          const float* lg = P.logits + (int64_t)(seq * P.Hkv + g) * REP * P.G;
+          int32_t* hsel = P.sel + (int64_t)(seq * P.Hkv + g) * REP * P.top_k;
+          for (int h = 0; h < REP; ++h) {
+            for (int j = j0; j < j1; ++j) scores[j] = lg[(int64_t)h * P.G + j] * P.scale;
+            radix_select();
+            for (int x = r; x < P.top_k; x += 128) hsel[h * P.top_k + x] = sel_s[x];
+            __threadfence_block();
+            ok = ok && gs(44);  // scores and sel_s are rewritten by the next head
+          }
+          uint32_t* bm = reinterpret_cast<uint32_t*>(scores);  // [REP][W] chunk bitmaps
+          const int W = (P.G + 31) / 32;
+          for (int x = r; x < REP * W; x += 128) bm[x] = 0u;
+          ok = ok && gs(45);
+          for (int x = r; x < REP * P.top_k; x += 128) {
+            const int c = hsel[x];
+            if (c >= 0) atomicOr(&bm[(x / P.top_k) * W + (c >> 5)], 1u << (c & 31));
+          }
+          ok = ok && gs(46);
+          const int wper = (W + 127) / 128, w0 = r * wper, w1 = min(W, w0 + wper);
+          uint32_t cnt = 0u;
+          for (int w = w0; w < w1; ++w) {
+            uint32_t u = 0u;
+#pragma unroll
+            for (int h = 0; h < REP; ++h) u |= bm[h * W + w];
+            cnt += __popc(u);
+          }
+          uint32_t n_union = 0u;
+          uint32_t pos = group_exclusive_scan(cnt, r, scan, gs, ok, &n_union);
+          for (int w = w0; w < w1; ++w) {
+            uint32_t u = 0u;
+#pragma unroll
+            for (int h = 0; h < REP; ++h) u |= bm[h * W + w];
+            while (u != 0u && pos < (uint32_t)P.n_slots) {
+              const int bit = __ffs(u) - 1;
+              u &= u - 1u;
+              uint32_t hm = 0u;
+#pragma unroll
+              for (int h = 0; h < REP; ++h) hm |= ((bm[h * W + w] >> bit) & 1u) << h;
+              sel_s[pos] = w * 32 + bit;
+              hmask_s[pos] = (uint8_t)hm;
+              ++pos;
+            }
+          }
+          for (int x = r; x < P.n_slots; x += 128)
+            if (x >= (int)n_union) sel_s[x] = -1;
+          ok = ok && gs(47);
+        } else {
+        const uint32_t sel_total = radix_select();
         const int nsel = min((int)sel_total, P.top_k);
         if (P.rule == SA_SELECT_TOP_P_PER_GROUP && nsel > 0) {
           // softmax over the eligible chunks (the best score is among the
@@ -598,6 +661,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
         }
         int32_t* sel_out = P.sel + ((int64_t)seq * P.Hkv + g) * P.top_k;
         for (int x = r; x < P.top_k; x += 128) sel_out[x] = sel_s[x];
+        }
         mbar_arrive(&bar[B_SELD]);  // release: sel_s is complete
         if (!__all_sync(0xffffffffu, ok)) break;
       }
@@ -645,7 +709,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
 bool decode_tc_supported(const sa_decode_desc& d) {
   return d.head_dim == kD && d.chunk >= 8 && d.chunk <= kBlk && kBlk % d.chunk == 0 &&
          d.n_gists >= kBlk && d.n_gists <= kMaxG && d.cache_len >= kBlk &&
-         d.top_k <= kMaxTopK && d.num_q_heads / d.num_kv_heads <= 8;
+         d.top_k <= kMaxTopK && d.num_q_heads / d.num_kv_heads <= 8 &&
+         (d.select_rule != SA_SELECT_TOP_K_PER_HEAD ||
+          d.num_q_heads / d.num_kv_heads * d.top_k <= kMaxTopK);
 }
 
 template <int REP>
@@ -690,7 +756,8 @@ cudaError_t launch_decode_tc(const sa_decode_desc& d, const void* q, const void*
   P.nG = (d.n_gists + kBlk - 1) / kBlk;
   P.nW = (d.window + kBlk - 1) / kBlk;
   const int cpb = kBlk / d.chunk;
-  P.nC = (d.top_k + cpb - 1) / cpb;
+  P.n_slots = d.select_rule == SA_SELECT_TOP_K_PER_HEAD ? P.rep * d.top_k : d.top_k;
+  P.nC = (P.n_slots + cpb - 1) / cpb;
   P.scale = d.softmax_scale > 0.f ? d.softmax_scale : 1.f / sqrtf((float)d.head_dim);
   for (int i = 0; i < 2; ++i) {
     P.qs[i] = d.q_strides[i];

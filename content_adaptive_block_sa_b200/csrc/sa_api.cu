@@ -415,7 +415,7 @@ static sa_status check_decode(const sa_decode_desc* d) {
   SA_CHECK(rep == 1 || rep == 2 || rep == 4 || rep == 8, SA_ERR_UNSUPPORTED);
   SA_CHECK(d->head_dim == 128, SA_ERR_UNSUPPORTED);
   SA_CHECK(d->select_rule >= SA_SELECT_SUM_LOGITS_PER_GROUP &&
-               d->select_rule <= SA_SELECT_TOP_P_PER_GROUP,
+               d->select_rule <= SA_SELECT_TOP_K_PER_HEAD,
            SA_ERR_INVALID_ARG);
   if (d->select_rule == SA_SELECT_TOP_P_PER_GROUP)
     SA_CHECK(d->top_p > 0.f && d->top_p <= 1.f, SA_ERR_INVALID_ARG);

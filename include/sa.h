@@ -242,6 +242,9 @@ typedef struct sa_attn_desc {
  *  TOP_P_PER_GROUP       the group's summed logits, softmax over the eligible
  *                        chunks: the smallest score-ordered prefix whose
  *                        probability reaches top_p, at most top_k chunks.
+ *  TOP_K_PER_HEAD        every query head takes the top_k chunks of its own
+ *                        q_h . gist_k * scale and attends over its own chunks
+ *                        (sel is then [n_seq, Hq, top_k]).
  * Ties go to the lower chunk index in every rule. The pages of "Simplified
  * Sparse Attention via Gist Tokens" name a top-k and a top-p selection from
  * logits and a per-group selection; the three readings above are this
@@ -249,7 +252,8 @@ typedef struct sa_attn_desc {
 typedef enum {
   SA_SELECT_SUM_LOGITS_PER_GROUP = 0,
   SA_SELECT_SUM_PROBS_PER_GROUP = 1,
-  SA_SELECT_TOP_P_PER_GROUP = 2
+  SA_SELECT_TOP_P_PER_GROUP = 2,
+  SA_SELECT_TOP_K_PER_HEAD = 3
 } sa_select_rule;
 
 /* Decode shapes (one new query token per sequence).
@@ -258,7 +262,8 @@ typedef enum {
  *  k/v_cache  [n_seq, Hkv, cache_len, d] strides cache_strides {seq, head, pos}
  *  o          [n_seq, Hq, d]            strides o_strides {seq, head}
  *  lse        fp32 [n_seq, Hq] dense
- *  sel        int32 [n_seq, Hkv, top_k] dense: the selected chunk indices,
+ *  sel        int32 [n_seq, Hkv, top_k] dense ([n_seq, Hq, top_k] under
+ *             SA_SELECT_TOP_K_PER_HEAD): the selected chunk indices,
  *             ascending, -1 padded when fewer chunks are eligible.
  *  chunk      raw tokens per gist; n_gists * chunk == cache_len.
  *  window     the last `window` cache positions are always attended; a chunk

@@ -42,19 +42,23 @@ def upload_workload(w):
     return q, gk, gv, dev(q), dev(gk), dev(gv), kc, vc
 
 
-def logit_bound(q, gk, s, g, rep, d):
-    """Float32 accumulation bound of each chunk's summed logit (see above)."""
-    qg = np.abs(q[s, g * rep:(g + 1) * rep].astype(np.float64))
+def logit_bound(q, gk, s, g, rep, d, heads=None):
+    """Float32 accumulation bound of each chunk's summed logit (see above),
+    over the group's heads or the given ones."""
+    hs = range(g * rep, (g + 1) * rep) if heads is None else heads
+    qg = np.abs(q[s, list(hs)].astype(np.float64))
     return lambda c: 2 * d * 2.0 ** -24 / np.sqrt(d) * (qg @ np.abs(gk[s, g, c])).sum()
 
 
-def valid_alternative(w, rule, top_p, q, gk, s, g, got, want_scores):
+def valid_alternative(w, rule, top_p, q, gk, s, x, got, want_scores):
     """Is the kernel's selection `got` (ascending, -1 padded) one the rule
     admits given float32 near ties? Sum of logits / of probabilities: a top-k
     set whose boundary scores are within their rounding bounds. Top-p: a
     score-ordered prefix (up to the same near ties) that reaches p and is
     shortest, each up to 1e-4 of probability."""
     d, rep = w["head_dim"], w["heads"] // w["kv_heads"]
+    # x is the KV group, or the query head under the per-head rule
+    g, heads = (x // rep, [x]) if rule == D.PER_HEAD else (x, None)
     elig = D.eligible_chunks(w["n_gists"], w["chunk"], w["cache_len"], w["window"])
     K = got[got >= 0]
     assert elig[K].all() and len(set(K.tolist())) == len(K)
@@ -64,7 +68,7 @@ def valid_alternative(w, rule, top_p, q, gk, s, g, got, want_scores):
         b = logit_bound(q, gk, s, g, rep, d)
         bound = lambda c: want_scores[c] * (b(c) + 1e-5)
     else:
-        bound = logit_bound(q, gk, s, g, rep, d)
+        bound = logit_bound(q, gk, s, g, rep, d, heads)
     rest = np.setdiff1d(np.nonzero(elig)[0], K)
     if len(K) and len(rest):
         c_in = K[np.argmin(sc[K])]
@@ -102,15 +106,17 @@ def check(sa, w, seqs=None, rule=0, top_p=1.0):
         raw_v = lambda g: to_np(vc[s, g])
         osel, oo, ol, scores = D.decode_one(q[s], gk[s], gv[s], raw_k, raw_v, w["chunk"],
                                             w["window"], w["top_k"], rule=rule, top_p=top_p)
-        for g in range(w["kv_heads"]):
-            if not np.array_equal(sel[s, g], osel[g]):
+        per_head = rule == D.PER_HEAD
+        for x in range(w["heads"] if per_head else w["kv_heads"]):
+            if not np.array_equal(sel[s, x], osel[x]):
                 # accept a different set only where float32 rounding can decide it
-                valid_alternative(w, rule, top_p, q, gk, s, g, sel[s, g], scores[g])
+                valid_alternative(w, rule, top_p, q, gk, s, x, sel[s, x], scores[x])
+                g = x // rep if per_head else x
                 # O must then match the oracle evaluated on the GPU's own set
-                pos = D.raw_key_positions(sel[s, g], w["chunk"], w["cache_len"], w["window"])
+                pos = D.raw_key_positions(sel[s, x], w["chunk"], w["cache_len"], w["window"])
                 keys = np.concatenate([gk[s, g], raw_k(g)[pos]])
                 vals = np.concatenate([gv[s, g], raw_v(g)[pos]])
-                for h in range(g * rep, (g + 1) * rep):
+                for h in ([x] if per_head else range(g * rep, (g + 1) * rep)):
                     oo[h], ol[h] = D.attend(q[s, h], keys, vals, 1 / np.sqrt(w["head_dim"]))
         check_close(o[s], oo, "bf16", f"O seq {s}")
         check_close(lse[s], ol, "bf16", f"LSE seq {s}")
@@ -150,7 +156,8 @@ def test_decode_tensor_core_shapes(sa, top_k, window, chunk, G):
     check(sa, w)
 
 
-RULES = {"sum_probs": (1, 1.0), "top_p_0.3": (2, 0.3), "top_p_0.9": (2, 0.9), "top_p_1": (2, 1.0)}
+RULES = {"sum_probs": (1, 1.0), "top_p_0.3": (2, 0.3), "top_p_0.9": (2, 0.9), "top_p_1": (2, 1.0),
+         "per_head": (3, 1.0)}
 
 
 @pytest.mark.parametrize("rule", list(RULES))
@@ -166,7 +173,23 @@ def test_decode_select_rules(sa, rule, top_k, window, chunk, G):
     check(sa, w, rule=r, top_p=p)
 
 
-@pytest.mark.parametrize("rule", ["sum_probs", "top_p_0.9"])
+@pytest.mark.parametrize("rep", [1, 8])
+def test_decode_per_head_group_sizes(sa, rep):
+    """Per-head selection with one and eight query heads per KV head; with
+    eight, 8 * top_k = 256 unfolded slots is the tensor-core kernel's limit."""
+    w = W.scaled("gist_decode_128k", index=650 + rep, n_seq=2, cache_len=32 * 256, chunk=32,
+                 n_gists=256, top_k=32, window=128, heads=2 * rep, kv_heads=2)
+    check(sa, w, rule=3)
+
+
+def test_decode_per_head_past_the_union_limit(sa):
+    """8 heads per group x top_k 40 > 256 slots: the CUDA-core kernels take it."""
+    w = W.scaled("gist_decode_128k", index=660, n_seq=1, cache_len=16 * 512, chunk=16,
+                 n_gists=512, top_k=40, window=64, heads=16, kv_heads=2)
+    check(sa, w, rule=3)
+
+
+@pytest.mark.parametrize("rule", ["sum_probs", "top_p_0.9", "per_head"])
 def test_decode_select_rules_full_size(sa, rule):
     r, p = RULES[rule]
     check(sa, W.WORKLOADS["gist_decode_128k"], seqs=[0, 15], rule=r, top_p=p)
