@@ -338,6 +338,10 @@ class GistWorkload(GzipWorkload):
             "head 0, last 2048 query rows, exact visible pairs, fp64", dt
 
 
+# decode chunk selection rules (sa_select_rule)
+SELECT_RULES = {"sum_logits": 0, "sum_probs": 1, "top_p": 2, "per_head": 3}
+
+
 class DecodeWorkload:
     def __init__(self, sa, torch, w):
         self.sa, self.torch = sa, torch
@@ -363,13 +367,21 @@ class DecodeWorkload:
         self.q, self.gk, self.gv = self.h_q.cuda(), self.h_gk.cuda(), self.h_gv.cuda()
         self.o = torch.empty_like(self.q)
         self.lse = torch.empty(n, w["heads"], dtype=torch.float32, device="cuda")
-        self.sel = torch.empty(n, Hkv, w["top_k"], dtype=torch.int32, device="cuda")
-        self.dd = sa.decode_desc(self.q, self.gk, self.kc, self.o, w["chunk"], w["top_k"], w["window"])
+        rule = SELECT_RULES[w.get("select", "sum_logits")]
+        rows = w["heads"] if rule == 3 else Hkv  # per-head rule: one selection per query head
+        self.sel = torch.empty(n, rows, w["top_k"], dtype=torch.int32, device="cuda")
+        self.dd = sa.decode_desc(self.q, self.gk, self.kc, self.o, w["chunk"], w["top_k"], w["window"],
+                                 select_rule=rule, top_p=w.get("top_p", 1.0))
         self.ws = sa.decode_workspace(self.dd)
         self.step()
         torch.cuda.synchronize()
-        per = (G + w["top_k"] * w["chunk"] + w["window"]) * d * 2 * 2
-        self.bytes = float(n * Hkv * per + 2 * self.q.numel() * 2 + self.lse.numel() * 4
+        # algorithmic bytes: every gist, each distinct unfolded chunk of a KV
+        # group once (the union over its heads under the per-head rule) and the
+        # window, K and V in bf16
+        sel = self.sel.cpu().numpy().reshape(n, Hkv, -1)
+        n_chunks = sum(len(np.unique(sel[s_, g_][sel[s_, g_] >= 0])) for s_ in range(n) for g_ in range(Hkv))
+        kv_rows = n * Hkv * (G + w["window"]) + n_chunks * w["chunk"]
+        self.bytes = float(kv_rows * d * 2 * 2 + 2 * self.q.numel() * 2 + self.lse.numel() * 4
                            + self.sel.numel() * 4)
         # one tensor-core kernel for these shapes, else the four CUDA-core passes
         c = w["chunk"]
@@ -403,11 +415,15 @@ class DecodeWorkload:
         rk = [W.decode_raw(w, 0, g, "k") for g in range(w["kv_heads"])]
         rv = [W.decode_raw(w, 0, g, "v") for g in range(w["kv_heads"])]
         raw_k, raw_v = (lambda g: rk[g]), (lambda g: rv[g])
+        rule = SELECT_RULES[w.get("select", "sum_logits")]
         t0 = time.perf_counter()
-        D.decode_one(q, gk, gv, raw_k, raw_v, w["chunk"], w["window"], w["top_k"])
+        sel = D.decode_one(q, gk, gv, raw_k, raw_v, w["chunk"], w["window"], w["top_k"],
+                           rule=rule, top_p=w.get("top_p", 1.0))[0]
         dt = time.perf_counter() - t0
-        per = (w["n_gists"] + w["top_k"] * w["chunk"] + w["window"]) * w["head_dim"] * 2 * 2
-        return w["kv_heads"] * per / dt / 1e9, \
+        sel = sel.reshape(w["kv_heads"], -1)  # the group's rows (one per head under the per-head rule)
+        n_chunks = sum(len(np.unique(r_[r_ >= 0])) for r_ in sel)
+        rows = w["kv_heads"] * (w["n_gists"] + w["window"]) + n_chunks * w["chunk"]
+        return rows * w["head_dim"] * 2 * 2 / dt / 1e9, \
             "sequence 0, all kv heads (raw cache generation excluded), fp64", dt
 
 
@@ -429,8 +445,10 @@ def workload_params(name, rank, size):
     return w
 
 
-def make(sa, torch, name, rank, size="full"):
+def make(sa, torch, name, rank, size="full", select=None):
     w = workload_params(name, rank, size)
+    if select is not None:
+        w["select"], w["top_p"] = select, 0.9  # top-p keeps 90% of the probability
     if name.startswith("gzip"):
         return GzipWorkload(sa, torch, w, name.endswith("fwdbwd"))
     if w["kind"] == "gist":
@@ -476,6 +494,8 @@ def run_reference(args):
     wl = Stub()
     wl.w = dict(W.WORKLOADS[FWDBWD_OF.get(args.workload, args.workload)])
     wl.backward = args.workload.endswith("fwdbwd")
+    if args.select is not None:
+        wl.w["select"], wl.w["top_p"] = args.select, 0.9
     cls = {"gzip": GzipWorkload, "gist": GistWorkload, "decode": DecodeWorkload}
     fn = cls[wl.w["kind"]].cpu_baseline
     vals = []
@@ -497,7 +517,8 @@ def run_reference(args):
         "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": float(np.mean([dt for _, dt in vals]) * 1e3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": {"workload": args.workload},
+        "data": "synthetic",
+        "config": {"workload": args.workload, **({"select": args.select} if args.select else {})},
         "cpu_baseline": {"value": value, "unit": unit, "cores": cores, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}))
@@ -515,6 +536,8 @@ def main():
     ap.add_argument("--size", default="full", choices=["full", "small"],
                     help="small: fewer heads/sequences (inputs still larger than L2), for profiling")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--select", default=None, choices=list(SELECT_RULES),
+                    help="gist_decode_128k: chunk selection rule (default sum_logits; top_p at p = 0.9)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -536,7 +559,7 @@ def main():
     barrier = lambda: rank_barrier(world)
     max_over_ranks = lambda x: rank_max(x, world, "cuda")
 
-    wl = make(sa, torch, args.workload, rank, args.size)
+    wl = make(sa, torch, args.workload, rank, args.size, args.select)
     for _ in range(args.warmup):
         wl.step()
     torch.cuda.synchronize()
@@ -609,7 +632,8 @@ def main():
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "fp32" if wl.w.get("dtype") == "fp32" else "bf16",
         "data": "synthetic (seeded generators in sa_workloads)",
-        "config": {"workload": args.workload, "l2": "inputs larger than L2, no flush",
+        "config": {"workload": args.workload, **({"select": args.select} if args.select else {}),
+                   "l2": "inputs larger than L2, no flush",
                    "parallelism": f"independent replica per rank x{world}"},
         "roofline": roof, "clocks": clk,
         "e2e": {"value": e2e_value, "unit": wl.unit, "h2d_bytes_per_step": int(h2d),
