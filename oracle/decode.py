@@ -175,3 +175,63 @@ def decode_one(q, gist_k, gist_v, raw_k, raw_v, chunk, window, top_k, scale=None
         for h in range(g * rep, (g + 1) * rep):
             o[h], lse[h] = attend(q[h], keys, vals, scale)
     return sel, o, lse, scores
+
+
+# ---------------------------------------------------------------- gist-of-gist
+# "Forget, Then Recall: ... Gist Sparse Attention" (abstract) and "Simplified
+# Sparse Attention via Gist Tokens" (abstract) extend the selection
+# hierarchically: gists of gists give multi-resolution access with a
+# logarithmic per-step cost. The pages give no more; the readings taken:
+# * level 1 is the chunk gists above (one per `chunk` raw tokens); level 2 has
+#   one gist per `fanout` consecutive level-1 gists (a "group");
+# * a group is eligible iff all of its raw tokens lie before the window;
+# * step 1 scores every level-2 gist with the group's summed logits and keeps
+#   the top k2 eligible groups; step 2 scores the level-1 gists of those groups
+#   the same way and keeps the top k1 of them; ties go to the lower index;
+# * every head attends, in one softmax, over all level-2 gists, the level-1
+#   gists of the kept groups, the raw tokens of the kept chunks and the last
+#   `window` raw tokens. Deeper hierarchies repeat step 1 per level.
+def hier_key_counts(n2: int, fanout: int, chunk: int, k2: int, k1: int, window: int) -> int:
+    """Keys one head attends when every selection is full."""
+    return n2 + k2 * fanout + k1 * chunk + window
+
+
+def hier_decode_one(q, g2k, g2v, g1k, g1v, raw_k, raw_v, chunk, fanout, k2, k1, window,
+                    scale=None):
+    """One sequence. q [Hq, d]; g2k/g2v [Hkv, n2, d]; g1k/g1v [Hkv, n1, d]
+    (n1 = n2 * fanout); raw_k/raw_v callables (kv head) -> [cache_len, d] or
+    arrays. Returns (sel2 [Hkv, k2], sel1 [Hkv, k1] chunk indices, o, lse)."""
+    q = np.asarray(q, np.float64)
+    Hq, d = q.shape
+    Hkv, n2, _ = np.shape(g2k)
+    n1 = np.shape(g1k)[1]
+    assert n1 == n2 * fanout
+    rep = Hq // Hkv
+    scale = 1.0 / np.sqrt(d) if scale is None else float(scale)
+    get_k = raw_k if callable(raw_k) else (lambda g: raw_k[g])
+    get_v = raw_v if callable(raw_v) else (lambda g: raw_v[g])
+    s2 = group_scores(q, g2k, scale)
+    s1 = group_scores(q, g1k, scale)
+    sel2 = np.empty((Hkv, k2), np.int32)
+    sel1 = np.empty((Hkv, k1), np.int32)
+    o = np.empty((Hq, d))
+    lse = np.empty(Hq)
+    for g in range(Hkv):
+        rk, rv = get_k(g), get_v(g)
+        cache_len = rk.shape[0]
+        elig2 = (np.arange(n2) + 1) * fanout * chunk <= cache_len - window
+        sel2[g] = select_top_k(s2[g], elig2, k2)
+        groups = [c for c in sel2[g] if c >= 0]
+        cand = np.zeros(n1, bool)
+        for c in groups:
+            cand[c * fanout:(c + 1) * fanout] = True
+        sel1[g] = select_top_k(s1[g], cand, k1)
+        pos = raw_key_positions(sel1[g], chunk, cache_len, window)
+        lvl1 = np.nonzero(cand)[0]
+        keys = np.concatenate([np.asarray(g2k[g], np.float64), np.asarray(g1k[g], np.float64)[lvl1],
+                               np.asarray(rk[pos], np.float64)])
+        vals = np.concatenate([np.asarray(g2v[g], np.float64), np.asarray(g1v[g], np.float64)[lvl1],
+                               np.asarray(rv[pos], np.float64)])
+        for h in range(g * rep, (g + 1) * rep):
+            o[h], lse[h] = attend(q[h], keys, vals, scale)
+    return sel2, sel1, o, lse

@@ -184,3 +184,50 @@ def test_per_head_selection_is_each_heads_best_set_and_its_own_attention():
         assert abs(lse[h] - ref_l) < 1e-12
     # heads of one group generally pick different chunks
     assert any(not np.array_equal(sel[0], sel[h]) for h in range(1, 4))
+
+
+# ---------------------------------------------------------------- gist-of-gist
+def _hier_case(seed, Hq=8, Hkv=2, d=16, chunk=8, fanout=4, n2=16):
+    rng = np.random.default_rng(seed)
+    n1 = n2 * fanout
+    L = n1 * chunk
+    r = lambda *s: rng.standard_normal(s)
+    return r(Hq, d), r(Hkv, n2, d), r(Hkv, n2, d), r(Hkv, n1, d), r(Hkv, n1, d), r(Hkv, L, d), r(Hkv, L, d)
+
+
+def test_hier_selection_with_every_group_unfolded_is_the_flat_selection():
+    q, g2k, g2v, g1k, g1v, rk, rv = _hier_case(10)
+    window = 64
+    sel2, sel1, _, _ = D.hier_decode_one(q, g2k, g2v, g1k, g1v, rk, rv, 8, 4, 16, 9, window)
+    flat_sel = D.decode_one(q, g1k, g1v, rk, rv, 8, window, 9)[0]
+    assert np.array_equal(sel1, flat_sel)
+    elig2 = (np.arange(16) + 1) * 32 <= 512 - window
+    assert (sel2 >= 0).sum(1).tolist() == [int(elig2.sum())] * 2
+
+
+def test_hier_attention_is_one_softmax_over_the_stated_keys():
+    q, g2k, g2v, g1k, g1v, rk, rv = _hier_case(11)
+    chunk, fanout, k2, k1, window = 8, 4, 3, 5, 40
+    sel2, sel1, o, lse = D.hier_decode_one(q, g2k, g2v, g1k, g1v, rk, rv, chunk, fanout, k2, k1, window)
+    for g in range(2):
+        # the unfolded chunks lie inside the kept groups and are the best of them
+        groups = sel2[g][sel2[g] >= 0]
+        assert len(groups) == k2 and set(sel1[g] // fanout) <= set(groups)
+        cand = np.concatenate([np.arange(c * fanout, (c + 1) * fanout) for c in groups])
+        s1 = (g1k[g] @ q[g * 4:(g + 1) * 4].T).sum(1) / 4.0
+        assert sorted(cand[np.argsort(-s1[cand], kind="stable")][:k1].tolist()) == sel1[g].tolist()
+        raw = np.concatenate([np.arange(c * chunk, (c + 1) * chunk) for c in sel1[g]] +
+                             [np.arange(512 - window, 512)])
+        keys = np.concatenate([g2k[g], g1k[g][cand], rk[g][raw]])
+        vals = np.concatenate([g2v[g], g1v[g][cand], rv[g][raw]])
+        assert len(keys) == D.hier_key_counts(16, fanout, chunk, k2, k1, window)
+        for h in range(g * 4, (g + 1) * 4):
+            ref_o, ref_l = _softmax_attend(q[h], keys, vals)
+            np.testing.assert_allclose(o[h], ref_o, atol=1e-12)
+            assert abs(lse[h] - ref_l) < 1e-12
+
+
+def test_hier_key_count_is_logarithmic_against_flat():
+    # 128K cache, 32-token chunks, 32 chunk gists per group: 128 level-2 gists
+    assert D.hier_key_counts(128, 32, 32, 8, 64, 512) == 128 + 256 + 2048 + 512
+    assert 4096 + 64 * 32 + 512 == 6656  # the flat selection over the same cache
