@@ -13,6 +13,8 @@ seeded input already resident in HBM:
   gist_coarse_20k    coarse (segment-wise) layout build + forward: 16 segments
                      of 1024 raw tokens + 256 gists (20480 positions, 32q/8kv)
   gist_coarse_20k_fwdbwd   the same with the backward
+  gist_hier_decode_128k    gist-of-gist decode step over the decode cache shape
+                     (128 level-2 gists, top-8 groups, top-64 chunks)
 Prefill/backward workloads report visited-tile TFLOP/s (every visited block
 pair counted as a full b x b tile: 4*d*b^2 forward, 10*d*b^2 backward); the
 decode workload reports algorithmic HBM GB/s. Inputs are larger than the
@@ -427,9 +429,94 @@ class DecodeWorkload:
             "sequence 0, all kv heads (raw cache generation excluded), fp64", dt
 
 
+class HierDecodeWorkload(DecodeWorkload):
+    """Gist-of-gist decode: level-2 gists, the kept groups' level-1 gists, the
+    unfolded chunks and the window (six CUDA-core passes)."""
+
+    def __init__(self, sa, torch, w):
+        self.sa, self.torch = sa, torch
+        self.w = w
+        n, Hkv, L, d = w["n_seq"], w["kv_heads"], w["cache_len"], w["head_dim"]
+        self.kc = torch.empty(n, Hkv, L, d, dtype=torch.bfloat16, device="cuda")
+        self.vc = torch.empty_like(self.kc)
+        from concurrent.futures import ThreadPoolExecutor
+
+        def one(i):
+            s, g = divmod(i, Hkv)
+            return i, W.decode_raw(w, s, g, "k"), W.decode_raw(w, s, g, "v")
+
+        with ThreadPoolExecutor(8) as ex:
+            for i, rk, rv in ex.map(one, range(n * Hkv)):
+                s, g = divmod(i, Hkv)
+                self.kc[s, g] = torch.from_numpy(rk).to("cuda", torch.bfloat16)
+                self.vc[s, g] = torch.from_numpy(rv).to("cuda", torch.bfloat16)
+        bf = lambda a: torch.from_numpy(a).to(torch.bfloat16)
+        self.h_q = bf(W.decode_query(w)).pin_memory()
+        self.q = self.h_q.cuda()
+        self.g2k, self.g2v, self.gk, self.gv = (
+            bf(np.stack([fn(w, s, kv) for s in range(n)])).cuda()
+            for fn, kv in ((W.decode_gists2, "k"), (W.decode_gists2, "v"),
+                           (W.decode_gists, "k"), (W.decode_gists, "v")))
+        self.o = torch.empty_like(self.q)
+        self.lse = torch.empty(n, w["heads"], dtype=torch.float32, device="cuda")
+        self.sel2 = torch.empty(n, Hkv, w["top_k2"], dtype=torch.int32, device="cuda")
+        self.sel = torch.empty(n, Hkv, w["top_k"], dtype=torch.int32, device="cuda")
+        self.hd = sa.hier_decode_desc(self.q, self.g2k, self.gk, self.kc, self.o, w["chunk"],
+                                      w["fanout"], w["top_k2"], w["top_k"], w["window"])
+        self.ws = sa.hier_decode_workspace(self.hd)
+        self.step()
+        torch.cuda.synchronize()
+        # algorithmic bytes: every level-2 gist, the kept groups' level-1 gists,
+        # the unfolded chunks and the window, K and V in bf16
+        n2 = w["n_gists"] // w["fanout"]
+        kept = int((self.sel2.cpu() >= 0).sum()) * w["fanout"]
+        chunks = int((self.sel.cpu() >= 0).sum()) * w["chunk"]
+        rows = n * Hkv * (n2 + w["window"]) + kept + chunks
+        self.bytes = float(rows * d * 2 * 2 + 2 * self.q.numel() * 2 + self.lse.numel() * 4
+                           + (self.sel.numel() + self.sel2.numel()) * 4)
+        self.kernels_per_step = 6
+        self.kernel = "hier decode (6 CUDA-core passes)"
+        self.unit = "GB/s"
+
+    def step(self, ev=None):
+        if ev is not None:
+            ev[0].record()
+        self.sa.sa_gist_hier_decode(self.hd, self.q, self.g2k, self.g2v, self.gk, self.gv, self.kc,
+                                    self.vc, self.sel2, self.sel, self.o, self.lse, self.ws)
+        if ev is not None:
+            ev[1].record()
+
+    def e2e_step(self):
+        self.q.copy_(self.h_q, non_blocking=True)
+        self.step()
+        return copy_out([self.o, self.lse, self.sel2, self.sel])
+
+    def io_bytes(self):
+        return (self.h_q.numel() * 2,
+                self.o.numel() * 2 + self.lse.numel() * 4 + (self.sel.numel() + self.sel2.numel()) * 4)
+
+    def cpu_baseline(self):
+        from oracle import decode as D
+        w = self.w
+        q = W.decode_query(w)[0]
+        g2k, g2v = W.decode_gists2(w, 0, "k"), W.decode_gists2(w, 0, "v")
+        gk, gv = W.decode_gists(w, 0, "k"), W.decode_gists(w, 0, "v")
+        rk = [W.decode_raw(w, 0, g, "k") for g in range(w["kv_heads"])]
+        rv = [W.decode_raw(w, 0, g, "v") for g in range(w["kv_heads"])]
+        t0 = time.perf_counter()
+        sel2, sel1, _, _ = D.hier_decode_one(q, g2k, g2v, gk, gv, rk, rv, w["chunk"], w["fanout"],
+                                             w["top_k2"], w["top_k"], w["window"])
+        dt = time.perf_counter() - t0
+        n2 = w["n_gists"] // w["fanout"]
+        rows = (w["kv_heads"] * (n2 + w["window"]) + int((sel2 >= 0).sum()) * w["fanout"]
+                + int((sel1 >= 0).sum()) * w["chunk"])
+        return rows * w["head_dim"] * 2 * 2 / dt / 1e9, \
+            "sequence 0, all kv heads (raw cache generation excluded), fp64", dt
+
+
 SMALL = {"gzip_8k": dict(batch=8), "gzip_64k_fwdbwd": dict(batch=1, heads=4, kv_heads=4),
          "gist_prefill_32k": dict(heads=8, kv_heads=2), "gist_decode_128k": dict(n_seq=4),
-         "gist_coarse_20k": dict(heads=8, kv_heads=2)}
+         "gist_coarse_20k": dict(heads=8, kv_heads=2), "gist_hier_decode_128k": dict(n_seq=4)}
 # workloads that run another one's inputs with the backward added
 FWDBWD_OF = {"gist_prefill_32k_fwdbwd": "gist_prefill_32k",
              "gist_coarse_20k_fwdbwd": "gist_coarse_20k"}
@@ -453,6 +540,8 @@ def make(sa, torch, name, rank, size="full", select=None):
         return GzipWorkload(sa, torch, w, name.endswith("fwdbwd"))
     if w["kind"] == "gist":
         return GistWorkload(sa, torch, w, name.endswith("fwdbwd"))
+    if w["kind"] == "hier":
+        return HierDecodeWorkload(sa, torch, w)
     return DecodeWorkload(sa, torch, w)
 
 
@@ -496,7 +585,8 @@ def run_reference(args):
     wl.backward = args.workload.endswith("fwdbwd")
     if args.select is not None:
         wl.w["select"], wl.w["top_p"] = args.select, 0.9
-    cls = {"gzip": GzipWorkload, "gist": GistWorkload, "decode": DecodeWorkload}
+    cls = {"gzip": GzipWorkload, "gist": GistWorkload, "decode": DecodeWorkload,
+           "hier": HierDecodeWorkload}
     fn = cls[wl.w["kind"]].cpu_baseline
     vals = []
     H = wl.w["heads"]
@@ -510,7 +600,7 @@ def run_reference(args):
         if i >= args.warmup:
             vals.append((v, dt))
     value = float(np.mean([v for v, _ in vals]))
-    unit = "GB/s" if args.workload.startswith("gist_decode") else "TFLOP/s"
+    unit = "GB/s" if wl.w["kind"] in ("decode", "hier") else "TFLOP/s"
     cores = len(os.sched_getaffinity(0))
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": value, "unit": unit, "n_gpus": args.gpus,
@@ -531,7 +621,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="gzip_8k",
                     choices=["gzip_8k", "gzip_64k_fwdbwd", "gist_prefill_32k", "gist_decode_128k",
-                             "gist_prefill_32k_fwdbwd", "gist_coarse_20k", "gist_coarse_20k_fwdbwd"])
+                             "gist_prefill_32k_fwdbwd", "gist_coarse_20k", "gist_coarse_20k_fwdbwd",
+                             "gist_hier_decode_128k"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--size", default="full", choices=["full", "small"],
                     help="small: fewer heads/sequences (inputs still larger than L2), for profiling")

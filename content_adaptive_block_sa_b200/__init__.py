@@ -291,6 +291,55 @@ def gist_decode(q, gist_k, gist_v, k_cache, v_cache, chunk: int, top_k: int, win
     return sel[:, :, :top_k], o, lse
 
 
+def hier_decode_desc(q, gist2_k, gist_k, k_cache, o, chunk: int, fanout: int, top_k2: int,
+                     top_k: int, window: int, softmax_scale: float = 0.0) -> _abi.sa_hier_decode_desc:
+    n_seq, Hq, d = q.shape
+    _, Hkv, G, _ = gist_k.shape
+    return _abi.sa_hier_decode_desc(
+        n_seq=n_seq, cache_len=k_cache.shape[2], chunk=chunk, n_gists=G, fanout=fanout,
+        top_k2=top_k2, top_k=top_k, window=window, num_q_heads=Hq, num_kv_heads=Hkv, head_dim=d,
+        softmax_scale=softmax_scale, q_strides=(i64 * 2)(q.stride(0), q.stride(1)),
+        gist_strides=(i64 * 3)(*gist_k.stride()[:3]), gist2_strides=(i64 * 3)(*gist2_k.stride()[:3]),
+        cache_strides=(i64 * 3)(*k_cache.stride()[:3]), o_strides=(i64 * 2)(o.stride(0), o.stride(1)))
+
+
+def hier_decode_workspace(hdesc, device="cuda") -> torch.Tensor:
+    n = C.c_size_t()
+    _check(lib().sa_gist_hier_decode_workspace_size(C.byref(hdesc), C.byref(n)),
+           "sa_gist_hier_decode_workspace_size")
+    return _workspace(n.value, device)
+
+
+def sa_gist_hier_decode(hdesc, q, gist2_k, gist2_v, gist_k, gist_v, k_cache, v_cache, sel2, sel1,
+                        o, lse, ws, stream=None):
+    _check(lib().sa_gist_hier_decode(C.byref(hdesc), _ptr(q), _ptr(gist2_k), _ptr(gist2_v),
+                                     _ptr(gist_k), _ptr(gist_v), _ptr(k_cache), _ptr(v_cache),
+                                     _ptr(sel2), _ptr(sel1), _ptr(o), _ptr(lse), _ptr(ws),
+                                     ws.numel(), _stream(stream)), "sa_gist_hier_decode")
+
+
+def gist_hier_decode(q, gist2_k, gist2_v, gist_k, gist_v, k_cache, v_cache, chunk: int, fanout: int,
+                     top_k2: int, top_k: int, window: int, softmax_scale: float = 0.0, stream=None):
+    """Gist-of-gist decode: (sel2 int32 [n_seq, Hkv, top_k2], sel1 int32
+    [n_seq, Hkv, top_k], o bf16 [n_seq, Hq, d], lse fp32 [n_seq, Hq])."""
+    for a, b in ((gist2_k, gist2_v), (gist_k, gist_v), (k_cache, v_cache)):
+        if a.stride() != b.stride():
+            raise ValueError("K and V must share strides")
+    n_seq, Hq, d = q.shape
+    Hkv = gist_k.shape[1]
+    o = torch.empty_like(q)
+    lse = torch.empty(n_seq, Hq, dtype=torch.float32, device=q.device)
+    sel2 = torch.empty(n_seq, Hkv, max(top_k2, 1), dtype=torch.int32, device=q.device)
+    sel1 = torch.empty(n_seq, Hkv, max(top_k, 1), dtype=torch.int32, device=q.device)
+    hd = hier_decode_desc(q, gist2_k, gist_k, k_cache, o, chunk, fanout, top_k2, top_k, window,
+                          softmax_scale)
+    ws = hier_decode_workspace(hd, q.device)
+    sa_gist_hier_decode(hd, q, gist2_k, gist2_v, gist_k, gist_v, k_cache, v_cache, sel2, sel1, o, lse,
+                        ws, stream)
+    gist_hier_decode.last_workspace = ws
+    return sel2[:, :, :top_k2], sel1[:, :, :top_k], o, lse
+
+
 def device_status(ws: torch.Tensor, stream=None) -> int:
     st = C.c_int()
     _check(lib().sa_get_device_status(_ptr(ws), _stream(stream), C.byref(st)),

@@ -59,6 +59,14 @@ class sa_decode_desc(C.Structure):
                 ("o_strides", i64 * 2), ("top_p", f32)]
 
 
+class sa_hier_decode_desc(C.Structure):
+    _fields_ = [("n_seq", i32), ("cache_len", i32), ("chunk", i32), ("n_gists", i32),
+                ("fanout", i32), ("top_k2", i32), ("top_k", i32), ("window", i32),
+                ("num_q_heads", i32), ("num_kv_heads", i32), ("head_dim", i32),
+                ("softmax_scale", f32), ("q_strides", i64 * 2), ("gist_strides", i64 * 3),
+                ("gist2_strides", i64 * 3), ("cache_strides", i64 * 3), ("o_strides", i64 * 2)]
+
+
 P = C.POINTER
 PROTOTYPES = {
     "sa_version": (C.c_char_p, []),
@@ -78,6 +86,9 @@ PROTOTYPES = {
     "sa_gist_decode": (C.c_int, [P(sa_decode_desc), vp, vp, vp, vp, vp, vp, vp, vp, vp,
                                  C.c_size_t, vp]),
     "sa_gist_decode_noalloc": (C.c_int, [P(sa_decode_desc), vp, vp, vp, vp, vp, vp, vp, vp, vp]),
+    "sa_gist_hier_decode_workspace_size": (C.c_int, [P(sa_hier_decode_desc), P(C.c_size_t)]),
+    "sa_gist_hier_decode": (C.c_int, [P(sa_hier_decode_desc), vp, vp, vp, vp, vp, vp, vp, vp, vp,
+                                      vp, vp, vp, C.c_size_t, vp]),
 }
 
 

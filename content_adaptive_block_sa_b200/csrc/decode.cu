@@ -46,6 +46,13 @@ struct DecodeArgs {
   float* logits;   // [n_seq, Hq, G] scaled logits (sum-of-probabilities rule)
   int rule;
   float top_p;
+  // gist of gists: level-2 gists, their selection, and (selecting level 1)
+  // the kept groups whose level-1 gists are the candidates
+  const __nv_bfloat16 *g2k, *g2v;
+  int64_t g2s[3];
+  int32_t* sel2;
+  const int32_t* cand_groups;
+  int n2, fanout, top_k2;
   int n_seq, cache_len, chunk, G, top_k, window, Hq, Hkv, rep;
   int n_gslices, n_rslices, n_part;
   float scale;
@@ -235,9 +242,14 @@ __global__ void __launch_bounds__(1024) decode_select_kernel(DecodeArgs a, int p
   }
   __syncthreads();
   const int last_ok = a.cache_len - a.window;  // chunk c eligible iff (c+1)*chunk <= last_ok
+  // level-1 selection of the gist of gists: candidate i is level-1 gist
+  // i % fanout of kept group cg[i / fanout] (every kept group is eligible)
+  const int32_t* cg = a.cand_groups ? a.cand_groups + ((int64_t)seq * a.Hkv + g) * a.top_k2 : nullptr;
   for (int i = threadIdx.x; i < pow2; i += blockDim.x) {
     unsigned long long kk = 0ull;
-    if (i < a.G && (int64_t)(i + 1) * a.chunk <= last_ok) {
+    const bool elig = cg ? (i < a.G && cg[i / a.fanout] >= 0)
+                         : (i < a.G && (int64_t)(i + 1) * a.chunk <= last_ok);
+    if (elig) {
       float v = sc[i];
       if (probs) {
         v = 0.f;
@@ -301,7 +313,7 @@ __global__ void __launch_bounds__(1024) decode_select_kernel(DecodeArgs a, int p
     const int v = chosen[t];
     int rank = 0;
     for (int u = 0; u < k; ++u) rank += chosen[u] < v || (chosen[u] == v && u < t);
-    out[rank] = (v == 0x7FFFFFFF) ? -1 : v;
+    out[rank] = (v == 0x7FFFFFFF) ? -1 : cg ? cg[v / a.fanout] * a.fanout + v % a.fanout : v;
   }
 }
 
@@ -349,6 +361,60 @@ __global__ void __launch_bounds__(kDecThreads) decode_raw_kernel(DecodeArgs a) {
   };
   const int e0 = min(total, slice * kRawSlice), e1 = min(total, e0 + kRawSlice);
   attend_slice<REP>(a, qf, e0, e1, row, heads_of, nullptr, nullptr, seq, g, a.n_gslices + slice);
+}
+
+// Gist of gists, step 1: every level-2 gist, its summed logit into scores
+// (the level-2 score row) and its partial into slot `slice`.
+template <int REP>
+__global__ void __launch_bounds__(kDecThreads) hier_gist2_kernel(DecodeArgs a, float* scores2) {
+  __shared__ float qf[kDecMaxRep][kDecD];
+  const int slice = blockIdx.x, g = blockIdx.y, seq = blockIdx.z;
+  load_group_q(a, seq, g, qf);
+  const __nv_bfloat16* gk = a.g2k + seq * a.g2s[0] + (int64_t)g * a.g2s[1];
+  const __nv_bfloat16* gv = a.g2v + seq * a.g2s[0] + (int64_t)g * a.g2s[1];
+  const int64_t rs = a.g2s[2];
+  auto row = [&](int e, const __nv_bfloat16*& kr, const __nv_bfloat16*& vr) {
+    kr = gk + e * rs;
+    vr = gv + e * rs;
+  };
+  const int e0 = slice * kGistSlice, e1 = min(a.n2, e0 + kGistSlice);
+  attend_slice<REP>(a, qf, e0, e1, row, [](int) { return 0xFFFFFFFFu; },
+                    scores2 + ((int64_t)seq * a.Hkv + g) * a.n2, nullptr, seq, g, slice);
+}
+
+// Step 2: the level-1 gists of the kept groups (a prefix of sel2: it is
+// ascending, -1 padded), candidate e = level-1 gist e % fanout of group
+// sel2[e / fanout]; summed logits into scores1 [.., top_k2 * fanout] and
+// partials into the slots after step 1's.
+template <int REP>
+__global__ void __launch_bounds__(kDecThreads) hier_gist1_kernel(DecodeArgs a, float* scores1,
+                                                                 int slot0) {
+  __shared__ float qf[kDecMaxRep][kDecD];
+  __shared__ int grp[256];
+  __shared__ int n_grp_s;
+  const int slice = blockIdx.x, g = blockIdx.y, seq = blockIdx.z;
+  const int32_t* sel2 = a.sel2 + ((int64_t)seq * a.Hkv + g) * a.top_k2;
+  for (int t = threadIdx.x; t < a.top_k2; t += blockDim.x) grp[t] = sel2[t];
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int n = 0;
+    for (int t = 0; t < a.top_k2; ++t) n += grp[t] >= 0;
+    n_grp_s = n;
+  }
+  load_group_q(a, seq, g, qf);
+  const int n_cand = n_grp_s * a.fanout, fo = a.fanout;
+  const __nv_bfloat16* gk = a.gk + seq * a.gs[0] + (int64_t)g * a.gs[1];
+  const __nv_bfloat16* gv = a.gv + seq * a.gs[0] + (int64_t)g * a.gs[1];
+  const int64_t rs = a.gs[2];
+  auto row = [&](int e, const __nv_bfloat16*& kr, const __nv_bfloat16*& vr) {
+    const int j = grp[e / fo] * fo + e % fo;
+    kr = gk + j * rs;
+    vr = gv + j * rs;
+  };
+  const int e0 = min(n_cand, slice * kGistSlice), e1 = min(n_cand, e0 + kGistSlice);
+  attend_slice<REP>(a, qf, e0, e1, row, [](int) { return 0xFFFFFFFFu; },
+                    scores1 + ((int64_t)seq * a.Hkv + g) * a.top_k2 * fo, nullptr, seq, g,
+                    slot0 + slice);
 }
 
 __global__ void decode_combine_kernel(DecodeArgs a) {
@@ -463,6 +529,125 @@ cudaError_t launch_decode(const sa_decode_desc& d, const void* q, const void* gk
 }
 
 size_t decode_workspace_bytes(const sa_decode_desc& d) { return decode_plan(d).bytes; }
+
+// ---------------------------------------------------- gist of gists, host side
+// Six launches: level-2 pass, group selection, level-1 pass over the kept
+// groups, chunk selection among their level-1 gists, raw pass, combine.
+struct HierPlan {
+  int n2, n_cand, n_g2slices, n_cslices, n_rslices, n_part, pow2_2, pow2_1;
+  size_t scores2_off, scores1_off, part_off, bytes;
+};
+
+HierPlan hier_plan(const sa_hier_decode_desc& d) {
+  HierPlan p{};
+  auto r256 = [](size_t x) { return (x + 255) / 256 * 256; };
+  p.n2 = d.n_gists / d.fanout;
+  p.n_cand = d.top_k2 * d.fanout;
+  p.n_g2slices = (p.n2 + kGistSlice - 1) / kGistSlice;
+  p.n_cslices = max(1, (p.n_cand + kGistSlice - 1) / kGistSlice);
+  p.n_rslices = max(1, (d.top_k * d.chunk + d.window + kRawSlice - 1) / kRawSlice);
+  p.n_part = p.n_g2slices + p.n_cslices + p.n_rslices;
+  p.pow2_2 = 1;
+  while (p.pow2_2 < p.n2) p.pow2_2 <<= 1;
+  p.pow2_1 = 1;
+  while (p.pow2_1 < p.n_cand) p.pow2_1 <<= 1;
+  p.scores2_off = kStatusBytes;
+  p.scores1_off = p.scores2_off + r256((size_t)d.n_seq * d.num_kv_heads * p.n2 * sizeof(float));
+  p.part_off = p.scores1_off +
+               r256((size_t)d.n_seq * d.num_kv_heads * max(p.n_cand, 1) * sizeof(float));
+  p.bytes = p.part_off +
+            (size_t)d.n_seq * d.num_q_heads * p.n_part * (2 + kDecD) * sizeof(float);
+  return p;
+}
+
+size_t hier_decode_workspace_bytes(const sa_hier_decode_desc& d) { return hier_plan(d).bytes; }
+
+static cudaError_t launch_select(const DecodeArgs& a, int pow2, cudaStream_t s) {
+  const size_t smem = (size_t)pow2 * sizeof(unsigned long long);
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(decode_select_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  decode_select_kernel<<<dim3(a.Hkv, a.n_seq), 1024, smem, s>>>(a, pow2);
+  return cudaGetLastError();
+}
+
+template <int REP>
+static cudaError_t hier_launch_rep(const DecodeArgs& a, const HierPlan& pl, float* scores2,
+                                   float* scores1, int32_t* sel1, int top_k1, cudaStream_t s) {
+  hier_gist2_kernel<REP><<<dim3(pl.n_g2slices, a.Hkv, a.n_seq), kDecThreads, 0, s>>>(a, scores2);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  // groups: eligible iff all fanout * chunk raw tokens lie before the window
+  DecodeArgs a2 = a;
+  a2.G = a.n2;
+  a2.chunk = a.fanout * a.chunk;
+  a2.scores = scores2;
+  a2.sel = a.sel2;
+  a2.top_k = a.top_k2;
+  a2.cand_groups = nullptr;
+  if ((e = launch_select(a2, pl.pow2_2, s)) != cudaSuccess) return e;
+  hier_gist1_kernel<REP><<<dim3(pl.n_cslices, a.Hkv, a.n_seq), kDecThreads, 0, s>>>(
+      a, scores1, pl.n_g2slices);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  DecodeArgs a1 = a;
+  a1.G = pl.n_cand;
+  a1.scores = scores1;
+  a1.sel = sel1;
+  a1.top_k = top_k1;
+  a1.cand_groups = a.sel2;
+  if ((e = launch_select(a1, pl.pow2_1, s)) != cudaSuccess) return e;
+  DecodeArgs ar = a;
+  ar.sel = sel1;
+  ar.top_k = top_k1;
+  ar.n_gslices = pl.n_g2slices + pl.n_cslices;  // the raw partials' first slot
+  decode_raw_kernel<REP><<<dim3(pl.n_rslices, a.Hkv, a.n_seq), kDecThreads, 0, s>>>(ar);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  decode_combine_kernel<<<dim3(a.Hq, a.n_seq), kDecD, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_hier_decode(const sa_hier_decode_desc& d, const void* q, const void* g2k,
+                               const void* g2v, const void* gk, const void* gv, const void* kc,
+                               const void* vc, int32_t* sel2, int32_t* sel1, void* o, float* lse,
+                               void* ws, cudaStream_t s) {
+  const HierPlan pl = hier_plan(d);
+  DecodeArgs a{};
+  a.q = (const __nv_bfloat16*)q;
+  a.g2k = (const __nv_bfloat16*)g2k;
+  a.g2v = (const __nv_bfloat16*)g2v;
+  a.gk = (const __nv_bfloat16*)gk;
+  a.gv = (const __nv_bfloat16*)gv;
+  a.kc = (const __nv_bfloat16*)kc;
+  a.vc = (const __nv_bfloat16*)vc;
+  a.sel2 = sel2;
+  a.o = (__nv_bfloat16*)o;
+  a.lse = lse;
+  a.part = (float*)((char*)ws + pl.part_off);
+  a.rule = SA_SELECT_SUM_LOGITS_PER_GROUP;
+  a.n_seq = d.n_seq; a.cache_len = d.cache_len; a.chunk = d.chunk; a.G = d.n_gists;
+  a.window = d.window; a.Hq = d.num_q_heads; a.Hkv = d.num_kv_heads;
+  a.rep = d.num_q_heads / d.num_kv_heads;
+  a.n2 = pl.n2; a.fanout = d.fanout; a.top_k2 = d.top_k2;
+  a.n_part = pl.n_part;
+  a.scale = d.softmax_scale > 0.f ? d.softmax_scale : 1.f / sqrtf((float)d.head_dim);
+  for (int i = 0; i < 2; ++i) { a.qs[i] = d.q_strides[i]; a.os[i] = d.o_strides[i]; }
+  for (int i = 0; i < 3; ++i) {
+    a.gs[i] = d.gist_strides[i];
+    a.g2s[i] = d.gist2_strides[i];
+    a.cs[i] = d.cache_strides[i];
+  }
+  float* scores2 = (float*)((char*)ws + pl.scores2_off);
+  float* scores1 = (float*)((char*)ws + pl.scores1_off);
+  switch (a.rep) {
+    case 1: return hier_launch_rep<1>(a, pl, scores2, scores1, sel1, d.top_k, s);
+    case 2: return hier_launch_rep<2>(a, pl, scores2, scores1, sel1, d.top_k, s);
+    case 4: return hier_launch_rep<4>(a, pl, scores2, scores1, sel1, d.top_k, s);
+    case 8: return hier_launch_rep<8>(a, pl, scores2, scores1, sel1, d.top_k, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
 
 }  // namespace sa
 

@@ -23,6 +23,10 @@ cudaError_t launch_decode(const sa_decode_desc&, const void*, const void*, const
                           const void*, const void*, int32_t*, void*, float*, void*,
                           cudaStream_t);
 size_t decode_workspace_bytes(const sa_decode_desc&);
+cudaError_t launch_hier_decode(const sa_hier_decode_desc&, const void*, const void*, const void*,
+                               const void*, const void*, const void*, const void*, int32_t*,
+                               int32_t*, void*, float*, void*, cudaStream_t);
+size_t hier_decode_workspace_bytes(const sa_hier_decode_desc&);
 }  // namespace sa
 
 using namespace sa;
@@ -453,6 +457,61 @@ sa_status sa_gist_decode(const sa_decode_desc* desc, const void* q, const void* 
   if (st != SA_OK) return st;
   return cuda_status(launch_decode(*desc, q, gist_k, gist_v, k_cache, v_cache, sel_chunks, o,
                                    lse, ws, stream));
+}
+
+static sa_status check_hier_decode(const sa_hier_decode_desc* d) {
+  SA_CHECK(d != nullptr, SA_ERR_INVALID_ARG);
+  SA_CHECK(d->n_seq >= 1 && d->chunk >= 1 && d->fanout >= 1 && d->n_gists >= 1,
+           SA_ERR_INVALID_ARG);
+  SA_CHECK(d->n_gists % d->fanout == 0, SA_ERR_INVALID_ARG);
+  SA_CHECK((int64_t)d->n_gists * d->chunk == d->cache_len, SA_ERR_INVALID_ARG);
+  SA_CHECK(d->n_gists / d->fanout <= 8192, SA_ERR_UNSUPPORTED);
+  SA_CHECK(d->top_k2 >= 0 && d->top_k2 <= 256 && d->top_k >= 0 && d->top_k <= 256,
+           SA_ERR_UNSUPPORTED);
+  SA_CHECK((int64_t)d->top_k2 * d->fanout <= 8192, SA_ERR_UNSUPPORTED);
+  SA_CHECK(d->window >= 0 && d->window <= d->cache_len, SA_ERR_INVALID_ARG);
+  SA_CHECK(d->num_kv_heads >= 1 && d->num_q_heads % d->num_kv_heads == 0, SA_ERR_INVALID_ARG);
+  const int rep = d->num_q_heads / d->num_kv_heads;
+  SA_CHECK(rep == 1 || rep == 2 || rep == 4 || rep == 8, SA_ERR_UNSUPPORTED);
+  SA_CHECK(d->head_dim == 128, SA_ERR_UNSUPPORTED);
+  SA_CHECK(d->softmax_scale >= 0.f && isfinite(d->softmax_scale), SA_ERR_INVALID_ARG);
+  for (int i = 0; i < 3; ++i)  // 16-byte row loads
+    SA_CHECK(d->gist_strides[i] % 8 == 0 && d->gist2_strides[i] % 8 == 0 &&
+                 d->cache_strides[i] % 8 == 0,
+             SA_ERR_INVALID_ARG);
+  return SA_OK;
+}
+
+sa_status sa_gist_hier_decode_workspace_size(const sa_hier_decode_desc* desc, size_t* bytes) {
+  sa_status st = check_hier_decode(desc);
+  if (st != SA_OK) return st;
+  SA_CHECK(bytes != nullptr, SA_ERR_INVALID_ARG);
+  *bytes = hier_decode_workspace_bytes(*desc);
+  return SA_OK;
+}
+
+sa_status sa_gist_hier_decode(const sa_hier_decode_desc* desc, const void* q, const void* gist2_k,
+                              const void* gist2_v, const void* gist_k, const void* gist_v,
+                              const void* k_cache, const void* v_cache, int32_t* sel_groups,
+                              int32_t* sel_chunks, void* o, float* lse, void* ws,
+                              size_t ws_bytes, sa_stream_t stream) {
+  size_t need = 0;
+  sa_status st = sa_gist_hier_decode_workspace_size(desc, &need);
+  if (st != SA_OK) return st;
+  SA_CHECK(q && gist2_k && gist2_v && gist_k && gist_v && k_cache && v_cache && o && lse,
+           SA_ERR_INVALID_ARG);
+  SA_CHECK(sel_groups != nullptr || desc->top_k2 == 0, SA_ERR_INVALID_ARG);
+  SA_CHECK(sel_chunks != nullptr || desc->top_k == 0, SA_ERR_INVALID_ARG);
+  SA_CHECK(aligned(gist2_k, 16) && aligned(gist2_v, 16) && aligned(gist_k, 16) &&
+               aligned(gist_v, 16) && aligned(k_cache, 16) && aligned(v_cache, 16) &&
+               aligned(q, 2) && aligned(o, 2),
+           SA_ERR_INVALID_ARG);
+  st = check_ws(ws, ws_bytes, need);
+  if (st != SA_OK) return st;
+  st = clear_status(ws, stream);
+  if (st != SA_OK) return st;
+  return cuda_status(launch_hier_decode(*desc, q, gist2_k, gist2_v, gist_k, gist_v, k_cache,
+                                        v_cache, sel_groups, sel_chunks, o, lse, ws, stream));
 }
 
 }  // extern "C"

@@ -292,6 +292,57 @@ typedef struct sa_decode_desc {
   float top_p;
 } sa_decode_desc;
 
+/* Gist-of-gist decode shapes ("Forget, Then Recall: ... Gist Sparse
+ * Attention", abstract: recursive gist-of-gist construction for
+ * multi-resolution access with logarithmic per-step cost; the level structure
+ * below is this library's reading). Level 1 has one gist per `chunk` raw
+ * tokens (n_gists of them), level 2 one gist per `fanout` consecutive level-1
+ * gists (n_gists / fanout of them, a "group").
+ *  q           [n_seq, Hq, d]                   strides q_strides {seq, head}
+ *  gist2_k/v   [n_seq, Hkv, n_gists/fanout, d]  strides gist2_strides
+ *  gist_k/v    [n_seq, Hkv, n_gists, d]         strides gist_strides
+ *  k/v_cache   [n_seq, Hkv, cache_len, d]       strides cache_strides
+ *  o, lse      as for sa_gist_decode.
+ *  sel_groups  int32 [n_seq, Hkv, top_k2]: kept groups, ascending, -1 padded.
+ *  sel_chunks  int32 [n_seq, Hkv, top_k]: unfolded chunks, ascending, -1 padded.
+ * Per (sequence, KV group): the top_k2 groups wholly before the window by the
+ * summed logit of their level-2 gist, then the top_k chunks among those
+ * groups' level-1 gists by the same score (ties to the lower index); every
+ * head attends in one softmax over all level-2 gists, the kept groups'
+ * level-1 gists, the unfolded chunks' raw tokens and the last `window` raw
+ * tokens. All bf16, head_dim 128, Hq / Hkv in {1, 2, 4, 8}; n_gists % fanout
+ * == 0, n_gists * chunk == cache_len, top_k2, top_k <= 256, n_gists / fanout
+ * and top_k2 * fanout <= 8192. K and V of a level share strides. */
+typedef struct sa_hier_decode_desc {
+  int32_t n_seq;
+  int32_t cache_len;
+  int32_t chunk;
+  int32_t n_gists;
+  int32_t fanout;
+  int32_t top_k2;
+  int32_t top_k;
+  int32_t window;
+  int32_t num_q_heads;
+  int32_t num_kv_heads;
+  int32_t head_dim;
+  float softmax_scale;
+  int64_t q_strides[2];
+  int64_t gist_strides[3];
+  int64_t gist2_strides[3];
+  int64_t cache_strides[3];
+  int64_t o_strides[2];
+} sa_hier_decode_desc;
+
+sa_status sa_gist_hier_decode_workspace_size(const sa_hier_decode_desc* desc, size_t* bytes);
+
+/* One gist-of-gist decode step (CUDA cores: level-2 pass, group selection,
+ * level-1 pass over the kept groups, chunk selection, raw pass, combine). */
+sa_status sa_gist_hier_decode(const sa_hier_decode_desc* desc, const void* q,
+                              const void* gist2_k, const void* gist2_v, const void* gist_k,
+                              const void* gist_v, const void* k_cache, const void* v_cache,
+                              int32_t* sel_groups, int32_t* sel_chunks, void* o, float* lse,
+                              void* ws, size_t ws_bytes, sa_stream_t stream);
+
 /* ------------------------------------------------------------------ misc */
 
 /* Library version string, e.g. "0.1.0 (sm_100a)". Never NULL. */

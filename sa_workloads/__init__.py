@@ -21,6 +21,9 @@ settings; no real corpus is used anywhere):
                         4096 gists, top-64, window 512, 32 q / 8 kv heads.
 5. ``gzip_64k_fwdbwd`` - batch 2, N=65536, block 128, window 2, 16 heads,
                         d=128, bf16, flags from synthetic mixed text/random bytes.
+7. ``gist_hier_decode_128k`` - gist-of-gist decode over the decode workload's
+                        cache shape: 32 chunk gists per level-2 gist (128 of
+                        them), top-8 groups, then top-64 chunks, window 512.
 6. ``gist_coarse_20k`` - segment-wise coarse gist layout: 16 segments of 1024
                         raw tokens, each followed by 256 gists (ratio 4), no
                         sinks (20480 positions), 32 q / 8 kv heads, d=128, bf16.
@@ -33,7 +36,7 @@ import numpy as np
 import torch
 
 # stream ids: one per independently drawn tensor
-S_BYTES, S_FLAGS, S_Q, S_K, S_V, S_DO, S_GK, S_GV, S_RK, S_RV, S_VOCAB = range(11)
+S_BYTES, S_FLAGS, S_Q, S_K, S_V, S_DO, S_GK, S_GV, S_RK, S_RV, S_VOCAB, S_G2K, S_G2V = range(13)
 
 WORKLOADS = {
     "gzip_tiny_fp32": dict(index=1, kind="gzip", batch=1, seq_len=256, block=16,
@@ -52,6 +55,9 @@ WORKLOADS = {
     "gist_coarse_20k": dict(index=6, kind="gist", batch=1, seq_len=20480,
                             sinks=0, ratio=4, window=0, gist_segment=1024, heads=32,
                             kv_heads=8, head_dim=128, dtype="bf16", tile=128, gist_tail=32),
+    "gist_hier_decode_128k": dict(index=7, kind="hier", n_seq=16, cache_len=131072,
+                                  chunk=32, n_gists=4096, fanout=32, top_k2=8, top_k=64,
+                                  window=512, heads=32, kv_heads=8, head_dim=128, dtype="bf16"),
     "gzip_64k_fwdbwd": dict(index=5, kind="gzip", batch=2, seq_len=65536,
                             block=128, window=2, heads=16, kv_heads=16,
                             head_dim=128, dtype="bf16", flags_from="bytes_mixed",
@@ -182,6 +188,14 @@ def decode_gists(w, seq: int, which: str) -> np.ndarray:
     w = _w(w)
     stream = S_GK if which == "k" else S_GV
     return normal(w["index"], stream, (w["kv_heads"], w["n_gists"], w["head_dim"]), True, seq)
+
+
+def decode_gists2(w, seq: int, which: str) -> np.ndarray:
+    """Level-2 gist K or V of one sequence (gist of gists): [kv_heads, n_gists / fanout, d]."""
+    w = _w(w)
+    stream = S_G2K if which == "k" else S_G2V
+    return normal(w["index"], stream, (w["kv_heads"], w["n_gists"] // w["fanout"], w["head_dim"]),
+                  True, seq)
 
 
 def decode_raw(w, seq: int, kv_head: int, which: str) -> np.ndarray:
