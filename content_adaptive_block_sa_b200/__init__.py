@@ -75,6 +75,21 @@ def literal_flags(x: bytes, b: int) -> np.ndarray:
     return sa_literal_flags_from_sizes(block_compressed_sizes(x, b))
 
 
+def literal_flags_device(x: torch.Tensor, b: int, stream=None):
+    """Flags from device bytes x (uint8 [batch, n_bytes]) by the library's
+    fixed-Huffman DEFLATE size estimate: (sizes uint32 as int32 [batch, B],
+    flags uint8 [batch, B])."""
+    if x.dtype != torch.uint8 or x.dim() != 2 or not x.is_contiguous():
+        raise ValueError("x must be a contiguous uint8 [batch, n_bytes] tensor")
+    batch, n = x.shape
+    B = n // b
+    sizes = torch.empty(batch, B, dtype=torch.int32, device=x.device)
+    flags = torch.empty(batch, B, dtype=torch.uint8, device=x.device)
+    _check(lib().sa_literal_flags_device(_ptr(x), batch, n, b, _ptr(sizes), _ptr(flags),
+                                         _stream(stream)), "sa_literal_flags_device")
+    return sizes, flags
+
+
 # ---------------------------------------------------------------- mask desc
 def mask_desc(kind: int, seq_len: int, num_heads: int, batch: int = 1, block_size: int = 0,
               window: int = 0, sinks: int = 0, gist_ratio: int = 0, gist_tail: int = 0,

@@ -27,6 +27,8 @@ cudaError_t launch_hier_decode(const sa_hier_decode_desc&, const void*, const vo
                                const void*, const void*, const void*, const void*, int32_t*,
                                int32_t*, void*, float*, void*, cudaStream_t);
 size_t hier_decode_workspace_bytes(const sa_hier_decode_desc&);
+cudaError_t launch_literal_flags_device(const uint8_t*, int, int64_t, int, uint32_t*, uint8_t*,
+                                        cudaStream_t);
 }  // namespace sa
 
 using namespace sa;
@@ -278,6 +280,19 @@ sa_status sa_build_block_mask_workspace_size(const sa_mask_desc* desc, size_t* b
   SA_CHECK(bytes != nullptr, SA_ERR_INVALID_ARG);
   *bytes = kStatusBytes;
   return SA_OK;
+}
+
+sa_status sa_literal_flags_device(const uint8_t* bytes, int32_t batch, int64_t n_bytes,
+                                  int32_t block_bytes, uint32_t* sizes, uint8_t* flags,
+                                  sa_stream_t stream) {
+  SA_CHECK(bytes && sizes && flags, SA_ERR_INVALID_ARG);
+  SA_CHECK(batch >= 1 && n_bytes >= 1, SA_ERR_INVALID_ARG);
+  SA_CHECK(block_bytes >= 1 && n_bytes % block_bytes == 0, SA_ERR_INVALID_ARG);
+  SA_CHECK(block_bytes <= 1024, SA_ERR_UNSUPPORTED);
+  SA_CHECK(n_bytes / block_bytes <= kMaxBlocks, SA_ERR_UNSUPPORTED);
+  SA_CHECK(aligned(sizes, 4), SA_ERR_INVALID_ARG);
+  return cuda_status(launch_literal_flags_device(bytes, batch, n_bytes, block_bytes, sizes, flags,
+                                                 (cudaStream_t)stream));
 }
 
 sa_status sa_build_block_mask(const sa_mask_desc* desc, const uint8_t* d_flags,

@@ -129,6 +129,24 @@ typedef struct sa_mask_desc {
   const int8_t* head_class;
 } sa_mask_desc;
 
+/* Literal flags computed on the device from raw bytes: an ESTIMATE of the
+ * gzip-based flags ("Gzip-guided sparse attention ...", Core equations: block
+ * i is literal iff its compression ratio exceeds the mean). Each block's size
+ * c_i comes from a plain DEFLATE encoder of RFC 1951 (one final block with the
+ * fixed Huffman codes of section 3.2.6; greedy LZ77 whose candidate at p is
+ * the nearest earlier position with the same three bytes; c_i = ceil(bits /
+ * 8)), not from zlib, so c_i and the flags can differ from gzip's near the
+ * mean. Then flags[i] = c_i * B > sum_j c_j.
+ *  bytes        DEVICE uint8 [batch, n_bytes]
+ *  block_bytes  b, 1 <= b <= 1024, n_bytes % b == 0, B = n_bytes / b
+ *  sizes        DEVICE uint32 [batch, B] out: c_i
+ *  flags        DEVICE uint8 [batch, B] out: the literal flags, ready for
+ *               sa_build_block_mask.
+ * Two launches on `stream`; no workspace. */
+sa_status sa_literal_flags_device(const uint8_t* bytes, int32_t batch, int64_t n_bytes,
+                                  int32_t block_bytes, uint32_t* sizes, uint8_t* flags,
+                                  sa_stream_t stream);
+
 /* Output of sa_build_block_mask. All pointers are caller-owned DEVICE memory
  * sized from sa_block_lists_capacity. Unused members may be NULL.
  *

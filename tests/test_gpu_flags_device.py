@@ -1,0 +1,47 @@
+"""sa_literal_flags_device vs the oracle's fixed-Huffman DEFLATE sizes:
+every block size and every flag bit-exact, on the workloads' byte
+generators, random and degenerate blocks, and ragged block sizes."""
+import numpy as np
+import pytest
+import torch
+
+import sa_workloads as W
+from oracle import deflate_size as F
+
+pytestmark = pytest.mark.gpu
+
+
+def run(sa, rows, b):
+    x = torch.from_numpy(np.stack([np.frombuffer(r, np.uint8) for r in rows])).cuda()
+    sizes, flags = sa.literal_flags_device(x, b)
+    torch.cuda.synchronize()
+    return sizes.cpu().numpy().view(np.uint32), flags.cpu().numpy()
+
+
+def check(sa, rows, b):
+    sizes, flags = run(sa, rows, b)
+    for i, r in enumerate(rows):
+        want = F.block_sizes(r, b)
+        np.testing.assert_array_equal(sizes[i], want)
+        np.testing.assert_array_equal(flags[i], F.literal_flags(r, b))
+
+
+def test_workload_bytes_64k(sa):
+    w = W.WORKLOADS["gzip_64k_fwdbwd"]
+    check(sa, [W.workload_bytes(w, bt) for bt in range(w["batch"])], w["block"])
+
+
+def test_tiny_pattern_bytes(sa):
+    w = W.WORKLOADS["gzip_tiny_fp32"]
+    check(sa, [W.workload_bytes(w, 0)], w["block"])
+
+
+@pytest.mark.parametrize("b", [1, 3, 16, 100, 128, 1000, 1024])
+def test_random_text_and_degenerate_blocks(sa, b):
+    rng = np.random.default_rng(b)
+    n = b * 12
+    rows = [rng.integers(0, 256, n, dtype=np.uint8).tobytes(),       # incompressible
+            bytes(n),                                                  # all zeros
+            (b"the cat sat on the mat. " * (n // 24 + 1))[:n],         # periodic text
+            rng.integers(0, 3, n, dtype=np.uint8).tobytes()]           # three symbols
+    check(sa, rows, b)
