@@ -15,6 +15,7 @@ seeded input already resident in HBM:
   gist_coarse_20k_fwdbwd   the same with the backward
   gist_hier_decode_128k    gist-of-gist decode step over the decode cache shape
                      (128 level-2 gists, top-8 groups, top-64 chunks)
+  gzip_flags_128m    on-device literal flags over 2048 rows of 64 KiB (b=128)
 Prefill/backward workloads report visited-tile TFLOP/s (every visited block
 pair counted as a full b x b tile: 4*d*b^2 forward, 10*d*b^2 backward); the
 decode workload reports algorithmic HBM GB/s. Inputs are larger than the
@@ -514,6 +515,50 @@ class HierDecodeWorkload(DecodeWorkload):
             "sequence 0, all kv heads (raw cache generation excluded), fp64", dt
 
 
+class FlagsWorkload:
+    """On-device literal flags (fixed-Huffman DEFLATE size estimate per block,
+    then the mean rule) over rows of bytes already in HBM."""
+
+    def __init__(self, sa, torch, w):
+        self.sa, self.torch, self.w = sa, torch, w
+        src = W.WORKLOADS[w["rows_from"]]
+        rows = [np.frombuffer(W.workload_bytes(src, i % src["batch"]), np.uint8)
+                for i in range(src["batch"])]
+        x = np.stack([rows[i % len(rows)] for i in range(w["batch"])])
+        self.h_x = torch.from_numpy(x).pin_memory()
+        self.x = self.h_x.cuda()
+        self.step()
+        torch.cuda.synchronize()
+        self.bytes = float(self.x.numel() + 2 * self.flags.numel() + 4 * self.sizes.numel())
+        self.kernels_per_step = 2
+        self.kernel = "deflate_size_kernel + literal_flags_kernel"
+        self.unit = "GB/s"
+
+    def step(self, ev=None):
+        if ev is not None:
+            ev[0].record()
+        self.sizes, self.flags = self.sa.literal_flags_device(self.x, self.w["block"])
+        if ev is not None:
+            ev[1].record()
+
+    def e2e_step(self):
+        self.x.copy_(self.h_x, non_blocking=True)
+        self.step()
+        return copy_out([self.flags])
+
+    def io_bytes(self):
+        return self.h_x.numel(), self.flags.numel()
+
+    def cpu_baseline(self):
+        from oracle import deflate_size as F
+        src = W.WORKLOADS[self.w["rows_from"]]
+        x = W.workload_bytes(src, 0)[:8192]  # 64 blocks of the first row
+        t0 = time.perf_counter()
+        F.block_sizes(x, self.w["block"])
+        dt = time.perf_counter() - t0
+        return len(x) / dt / 1e9, "first 8 KiB of row 0 (64 blocks), pure Python", dt
+
+
 SMALL = {"gzip_8k": dict(batch=8), "gzip_64k_fwdbwd": dict(batch=1, heads=4, kv_heads=4),
          "gist_prefill_32k": dict(heads=8, kv_heads=2), "gist_decode_128k": dict(n_seq=4),
          "gist_coarse_20k": dict(heads=8, kv_heads=2), "gist_hier_decode_128k": dict(n_seq=4)}
@@ -542,6 +587,8 @@ def make(sa, torch, name, rank, size="full", select=None):
         return GistWorkload(sa, torch, w, name.endswith("fwdbwd"))
     if w["kind"] == "hier":
         return HierDecodeWorkload(sa, torch, w)
+    if w["kind"] == "flags":
+        return FlagsWorkload(sa, torch, w)
     return DecodeWorkload(sa, torch, w)
 
 
@@ -586,12 +633,12 @@ def run_reference(args):
     if args.select is not None:
         wl.w["select"], wl.w["top_p"] = args.select, 0.9
     cls = {"gzip": GzipWorkload, "gist": GistWorkload, "decode": DecodeWorkload,
-           "hier": HierDecodeWorkload}
+           "hier": HierDecodeWorkload, "flags": FlagsWorkload}
     fn = cls[wl.w["kind"]].cpu_baseline
     vals = []
-    H = wl.w["heads"]
+    H = wl.w.get("heads", 1)
     for i in range(args.warmup + args.steps):
-        if args.workload.startswith("gzip"):
+        if wl.w["kind"] == "gzip":
             # one whole head per step, cycling through the three classes
             v, sample, dt = fn(wl, heads=[(0, H // 2, H - 1)[i % 3]])
             sample = "batch row 0, one whole head per step cycling local/literal/hybrid, fp64"
@@ -600,13 +647,14 @@ def run_reference(args):
         if i >= args.warmup:
             vals.append((v, dt))
     value = float(np.mean([v for v, _ in vals]))
-    unit = "GB/s" if wl.w["kind"] in ("decode", "hier") else "TFLOP/s"
+    unit = "GB/s" if wl.w["kind"] in ("decode", "hier", "flags") else "TFLOP/s"
     cores = len(os.sched_getaffinity(0))
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": value, "unit": unit, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": float(np.mean([dt for _, dt in vals]) * 1e3),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "u8" if wl.w["kind"] == "flags" else "f64",
         "data": "synthetic",
         "config": {"workload": args.workload, **({"select": args.select} if args.select else {})},
         "cpu_baseline": {"value": value, "unit": unit, "cores": cores, "kind": "oracle",
@@ -622,7 +670,7 @@ def main():
     ap.add_argument("--workload", default="gzip_8k",
                     choices=["gzip_8k", "gzip_64k_fwdbwd", "gist_prefill_32k", "gist_decode_128k",
                              "gist_prefill_32k_fwdbwd", "gist_coarse_20k", "gist_coarse_20k_fwdbwd",
-                             "gist_hier_decode_128k"])
+                             "gist_hier_decode_128k", "gzip_flags_128m"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--size", default="full", choices=["full", "small"],
                     help="small: fewer heads/sequences (inputs still larger than L2), for profiling")
@@ -721,7 +769,8 @@ def main():
     line = {
         "metric": METRIC, "value": value, "unit": wl.unit, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "fp32" if wl.w.get("dtype") == "fp32" else "bf16",
+        "vs_baseline": None,
+        "dtype": {"fp32": "fp32", "bf16": "bf16"}.get(wl.w.get("dtype"), "u8"),
         "data": "synthetic (seeded generators in sa_workloads)",
         "config": {"workload": args.workload, **({"select": args.select} if args.select else {}),
                    "l2": "inputs larger than L2, no flush",

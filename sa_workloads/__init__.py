@@ -21,6 +21,8 @@ settings; no real corpus is used anywhere):
                         4096 gists, top-64, window 512, 32 q / 8 kv heads.
 5. ``gzip_64k_fwdbwd`` - batch 2, N=65536, block 128, window 2, 16 heads,
                         d=128, bf16, flags from synthetic mixed text/random bytes.
+8. ``gzip_flags_128m``  - on-device literal flags: the 64K workload's two byte
+                        rows repeated to 2048 rows of 64 KiB (128 MiB), b=128.
 7. ``gist_hier_decode_128k`` - gist-of-gist decode over the decode workload's
                         cache shape: 32 chunk gists per level-2 gist (128 of
                         them), top-8 groups, then top-64 chunks, window 512.
@@ -58,6 +60,8 @@ WORKLOADS = {
     "gist_hier_decode_128k": dict(index=7, kind="hier", n_seq=16, cache_len=131072,
                                   chunk=32, n_gists=4096, fanout=32, top_k2=8, top_k=64,
                                   window=512, heads=32, kv_heads=8, head_dim=128, dtype="bf16"),
+    "gzip_flags_128m": dict(index=8, kind="flags", rows_from="gzip_64k_fwdbwd", batch=2048,
+                            n_bytes=65536, block=128),
     "gzip_64k_fwdbwd": dict(index=5, kind="gzip", batch=2, seq_len=65536,
                             block=128, window=2, heads=16, kv_heads=16,
                             head_dim=128, dtype="bf16", flags_from="bytes_mixed",
