@@ -581,7 +581,7 @@ def make(sa, torch, name, rank, size="full", select=None):
     w = workload_params(name, rank, size)
     if select is not None:
         w["select"], w["top_p"] = select, 0.9  # top-p keeps 90% of the probability
-    if name.startswith("gzip"):
+    if w["kind"] == "gzip":
         return GzipWorkload(sa, torch, w, name.endswith("fwdbwd"))
     if w["kind"] == "gist":
         return GistWorkload(sa, torch, w, name.endswith("fwdbwd"))
