@@ -109,7 +109,9 @@ _host_out = {}
 # key-major dK/dV pass
 KERNEL_SOURCES = {"fwd_tc_kernel": ["attn_fwd_sm100.cu"],
                   "backward": ["attn_bwd_sm100.cu", "attn_dq_sm100.cu"],
-                  "decode_tc_kernel": ["decode_sm100.cu"]}
+                  "decode_tc_kernel": ["decode_sm100.cu"],
+                  "hier decode (6 CUDA-core passes)": ["decode.cu"],
+                  "deflate_size_kernel + literal_flags_kernel": ["compress.cu"]}
 
 
 def kernel_digest(kernel):
