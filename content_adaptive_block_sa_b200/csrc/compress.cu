@@ -17,53 +17,63 @@
 //     bits and 280..287 8; distance codes 5 bits; plus the extra bits of
 //     section 3.2.5's length and distance tables;
 //   * c_i = ceil(bits / 8).
-// Two launches: one CTA per block (threads find every position's match in
-// shared memory, then one thread walks the greedy parse), then one CTA per
+// Two launches: one warp per block (lanes find every position's nearest
+// match over 32-bit three-byte keys in shared memory, then one lane walks the
+// greedy parse with the code lengths in closed form), then one CTA per
 // sequence for l_i = 1[c_i * B > sum_j c_j] in 64-bit integers.
 #include "sa_common.cuh"
 
 namespace sa {
 
 constexpr int kMaxBlockBytes = 1024;
-constexpr int kCompThreads = 128;
+constexpr int kBlocksPerCta = 4;  // one warp per block
+constexpr int kCompThreads = 32 * kBlocksPerCta;
 
-// RFC 1951 section 3.2.5: first length of symbols 257..285 with their extra
-// bits, and first distance of codes 0..29 with theirs.
-__constant__ int16_t c_len_base[29] = {3,  4,  5,  6,  7,  8,  9,  10, 11,  13,  15,  17,  19,  23, 27,
-                                       31, 35, 43, 51, 59, 67, 83, 99, 115, 131, 163, 195, 227, 258};
-__constant__ int8_t c_len_extra[29] = {0, 0, 0, 0, 0, 0, 0, 0, 1, 1, 1, 1, 2, 2, 2,
-                                       2, 3, 3, 3, 3, 4, 4, 4, 4, 5, 5, 5, 5, 0};
-__constant__ int32_t c_dist_base[30] = {1,    2,    3,    4,    5,    7,     9,     13,    17,  25,
-                                        33,   49,   65,   97,   129,  193,   257,   385,   513, 769,
-                                        1025, 1537, 2049, 3073, 4097, 6145, 8193, 12289, 16385, 24577};
-__constant__ int8_t c_dist_extra[30] = {0, 0, 0, 0, 1, 1, 2, 2,  3,  3,  4,  4,  5,  5,  6,
-                                        6, 7, 7, 8, 8, 9, 9, 10, 10, 11, 11, 12, 12, 13, 13};
+// Code lengths in closed form (RFC 1951 section 3.2.5 and 3.2.6).
+// Length n: symbols 257..279 take 7 bits, 280..287 8; with the symbol's
+// extra bits a match length costs 7 (3..10), 8 (11..18), 9 (19..34),
+// 10 (35..66), 11 (67..114, symbols 277..279), 12 (115..130, symbol 280),
+// 13 (131..257) or 8 (258, symbol 285) bits.
+__device__ __forceinline__ int length_bits(int n) {
+  return n <= 10 ? 7 : n <= 18 ? 8 : n <= 34 ? 9 : n <= 66 ? 10 : n <= 114 ? 11
+       : n <= 130 ? 12 : n <= 257 ? 13 : 8;
+}
+// Distance d: a 5-bit code; distances 1..4 have no extra bits, and the two
+// codes covering (2^k, 2^(k+1)] carry k - 1 extra bits.
+__device__ __forceinline__ int distance_bits(int d) {
+  return 5 + (d <= 4 ? 0 : (31 - __clz(d - 1)) - 1);
+}
 
-// Bits of a match: length symbol (7 or 8 bits) + its extra bits + distance
-// code (5 bits) + its extra bits.
-__device__ int match_bits(int len, int dist) {
-  int s = 28;
-  while (c_len_base[s] > len) --s;
-  int d = 29;
-  while (c_dist_base[d] > dist) --d;
-  return (257 + s <= 279 ? 7 : 8) + c_len_extra[s] + 5 + c_dist_extra[d];
+__host__ __device__ constexpr size_t deflate_warp_smem(int b) {
+  return ((size_t)9 * b + 15) / 16 * 16;
 }
 
 __global__ void __launch_bounds__(kCompThreads) deflate_size_kernel(const uint8_t* x, int64_t n_bytes,
                                                                     int b, int B, uint32_t* sizes) {
-  __shared__ uint8_t xs[kMaxBlockBytes];
-  __shared__ uint16_t mlen[kMaxBlockBytes];
-  __shared__ uint16_t mdist[kMaxBlockBytes];
-  const int blk = blockIdx.x, bt = blockIdx.y;
+  // per warp, deflate_warp_smem(b) bytes: keys (x[p] | x[p+1] << 8 | x[p+2] << 16),
+  // match lengths, match distances, the block's bytes
+  extern __shared__ __align__(16) uint8_t dyn_s[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int blk = blockIdx.x * kBlocksPerCta + warp, bt = blockIdx.y;
+  if (blk >= B) return;  // warp-uniform; no CTA-wide barrier below
+  uint8_t* base = dyn_s + (size_t)warp * deflate_warp_smem(b);
+  uint32_t* key = reinterpret_cast<uint32_t*>(base);
+  uint16_t* mlen = reinterpret_cast<uint16_t*>(base + 4 * b);
+  uint16_t* mdist = mlen + b;
+  uint8_t* xs = base + 8 * b;
   const uint8_t* src = x + (int64_t)bt * n_bytes + (int64_t)blk * b;
-  for (int i = threadIdx.x; i < b; i += blockDim.x) xs[i] = src[i];
-  __syncthreads();
-  for (int p = threadIdx.x; p < b; p += blockDim.x) {
+  for (int i = lane; i < b; i += 32) xs[i] = src[i];
+  __syncwarp();
+  for (int p = lane; p + 3 <= b; p += 32)
+    key[p] = (uint32_t)xs[p] | ((uint32_t)xs[p + 1] << 8) | ((uint32_t)xs[p + 2] << 16);
+  __syncwarp();
+  for (int p = lane; p < b; p += 32) {
     int m = 0, dist = 0;
     if (p + 3 <= b) {
-      const uint8_t a0 = xs[p], a1 = xs[p + 1], a2 = xs[p + 2];
+      const uint32_t k = key[p];
       for (int q = p - 1; q >= 0 && p - q <= 32768; --q) {
-        if (xs[q] == a0 && xs[q + 1] == a1 && xs[q + 2] == a2) {  // nearest earlier match
+        if (key[q] == k) {  // the nearest earlier position with the same three bytes
+          m = 3;
           while (p + m < b && m < 258 && xs[q + m] == xs[p + m]) ++m;
           dist = p - q;
           break;
@@ -73,13 +83,13 @@ __global__ void __launch_bounds__(kCompThreads) deflate_size_kernel(const uint8_
     mlen[p] = (uint16_t)m;
     mdist[p] = (uint16_t)dist;
   }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    int64_t bits = 3 + 7;  // block header, end of block (symbol 256: 7 bits)
+  __syncwarp();
+  if (lane == 0) {
+    int bits = 3 + 7;  // block header, end of block (symbol 256: 7 bits)
     for (int p = 0; p < b;) {
       const int m = mlen[p];
       if (m >= 3) {
-        bits += match_bits(m, mdist[p]);
+        bits += length_bits(m) + distance_bits(mdist[p]);
         p += m;
       } else {
         bits += xs[p] <= 143 ? 8 : 9;
@@ -110,7 +120,9 @@ __global__ void __launch_bounds__(256) literal_flags_kernel(const uint32_t* size
 cudaError_t launch_literal_flags_device(const uint8_t* bytes, int batch, int64_t n_bytes, int b,
                                         uint32_t* sizes, uint8_t* flags, cudaStream_t s) {
   const int B = (int)(n_bytes / b);
-  deflate_size_kernel<<<dim3(B, batch), kCompThreads, 0, s>>>(bytes, n_bytes, b, B, sizes);
+  const size_t smem = kBlocksPerCta * deflate_warp_smem(b);  // <= 36 KB (b <= 1024)
+  deflate_size_kernel<<<dim3((B + kBlocksPerCta - 1) / kBlocksPerCta, batch), kCompThreads, smem, s>>>(
+      bytes, n_bytes, b, B, sizes);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   literal_flags_kernel<<<batch, 256, 0, s>>>(sizes, B, flags);
