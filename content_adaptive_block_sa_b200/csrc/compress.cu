@@ -17,10 +17,11 @@
 //     bits and 280..287 8; distance codes 5 bits; plus the extra bits of
 //     section 3.2.5's length and distance tables;
 //   * c_i = ceil(bits / 8).
-// Two launches: one warp per block (lanes find every position's nearest
-// match over 32-bit three-byte keys in shared memory, then one lane walks the
-// greedy parse with the code lengths in closed form), then one CTA per
-// sequence for l_i = 1[c_i * B > sum_j c_j] in 64-bit integers.
+// Two launches: one warp per block (a bitonic sort of (three-byte key,
+// position) pairs in shared memory gives every position its nearest earlier
+// match; binary lifting over the next-position pointers marks the positions
+// the greedy parse visits; the code lengths are in closed form), then one CTA
+// per sequence for l_i = 1[c_i * B > sum_j c_j] in 64-bit integers.
 #include "sa_common.cuh"
 
 namespace sa {
@@ -44,60 +45,106 @@ __device__ __forceinline__ int distance_bits(int d) {
   return 5 + (d <= 4 ? 0 : (31 - __clz(d - 1)) - 1);
 }
 
+__host__ __device__ constexpr int pow2_at_least(int n) {
+  int p = 1;
+  while (p < n) p <<= 1;
+  return p;
+}
+
+// Per warp: the sort buffer (uint64 [pow2 >= b]), match lengths and
+// distances, next-position pointers (uint16 [b + 1] each), parse marks and
+// the block's bytes (uint8 [b + 1] each), 16-byte aligned.
 __host__ __device__ constexpr size_t deflate_warp_smem(int b) {
-  return ((size_t)9 * b + 15) / 16 * 16;
+  return ((size_t)8 * pow2_at_least(b) + 6 * ((size_t)b + 1) + 2 * ((size_t)b + 1) + 15) / 16 * 16;
+}
+
+__device__ __forceinline__ int position_bits(const uint16_t* mlen, const uint16_t* mdist,
+                                             const uint8_t* xs, int p) {
+  const int m = mlen[p];
+  return m >= 3 ? length_bits(m) + distance_bits(mdist[p]) : (xs[p] <= 143 ? 8 : 9);
 }
 
 __global__ void __launch_bounds__(kCompThreads) deflate_size_kernel(const uint8_t* x, int64_t n_bytes,
                                                                     int b, int B, uint32_t* sizes) {
-  // per warp, deflate_warp_smem(b) bytes: keys (x[p] | x[p+1] << 8 | x[p+2] << 16),
-  // match lengths, match distances, the block's bytes
   extern __shared__ __align__(16) uint8_t dyn_s[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int blk = blockIdx.x * kBlocksPerCta + warp, bt = blockIdx.y;
   if (blk >= B) return;  // warp-uniform; no CTA-wide barrier below
+  const int np2 = pow2_at_least(b);
   uint8_t* base = dyn_s + (size_t)warp * deflate_warp_smem(b);
-  uint32_t* key = reinterpret_cast<uint32_t*>(base);
-  uint16_t* mlen = reinterpret_cast<uint16_t*>(base + 4 * b);
-  uint16_t* mdist = mlen + b;
-  uint8_t* xs = base + 8 * b;
+  uint64_t* srt = reinterpret_cast<uint64_t*>(base);
+  uint16_t* mlen = reinterpret_cast<uint16_t*>(base + 8 * (size_t)np2);
+  uint16_t* mdist = mlen + (b + 1);
+  uint16_t* nxt = mdist + (b + 1);
+  uint8_t* mark = reinterpret_cast<uint8_t*>(nxt + (b + 1));
+  uint8_t* xs = mark + (b + 1);
   const uint8_t* src = x + (int64_t)bt * n_bytes + (int64_t)blk * b;
   for (int i = lane; i < b; i += 32) xs[i] = src[i];
   __syncwarp();
-  for (int p = lane; p + 3 <= b; p += 32)
-    key[p] = (uint32_t)xs[p] | ((uint32_t)xs[p + 1] << 8) | ((uint32_t)xs[p + 2] << 16);
+  // (three-byte key, position) of every position with three bytes left,
+  // padded with the largest value; sorted ascending, an entry whose
+  // predecessor has the same key finds there its nearest earlier match
+  for (int i = lane; i < np2; i += 32) {
+    uint64_t v = ~0ull;
+    if (i + 3 <= b)
+      v = ((uint64_t)((uint32_t)xs[i] | ((uint32_t)xs[i + 1] << 8) | ((uint32_t)xs[i + 2] << 16)) << 32) |
+          (uint32_t)i;
+    srt[i] = v;
+    if (i <= b) mlen[i] = 0;
+  }
   __syncwarp();
-  for (int p = lane; p < b; p += 32) {
-    int m = 0, dist = 0;
-    if (p + 3 <= b) {
-      const uint32_t k = key[p];
-      for (int q = p - 1; q >= 0 && p - q <= 32768; --q) {
-        if (key[q] == k) {  // the nearest earlier position with the same three bytes
-          m = 3;
-          while (p + m < b && m < 258 && xs[q + m] == xs[p + m]) ++m;
-          dist = p - q;
-          break;
+  for (int size = 2; size <= np2; size <<= 1) {  // bitonic sort, ascending
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int i = lane; i < np2 / 2; i += 32) {
+        const int lo = 2 * i - (i & (stride - 1)), hi = lo + stride;
+        const bool up = (lo & size) == 0;
+        const uint64_t a = srt[lo], c = srt[hi];
+        if ((a > c) == up) {
+          srt[lo] = c;
+          srt[hi] = a;
         }
       }
+      __syncwarp();
     }
-    mlen[p] = (uint16_t)m;
-    mdist[p] = (uint16_t)dist;
+  }
+  for (int t = 1 + lane; t < np2; t += 32) {
+    const uint64_t cur = srt[t], prev = srt[t - 1];
+    if (cur != ~0ull && (cur >> 32) == (prev >> 32)) {
+      const int p = (int)(uint32_t)cur, q = (int)(uint32_t)prev;
+      int m = 3;
+      while (p + m < b && m < 258 && xs[q + m] == xs[p + m]) ++m;
+      mlen[p] = (uint16_t)m;
+      mdist[p] = (uint16_t)(p - q);
+    }
   }
   __syncwarp();
-  if (lane == 0) {
-    int bits = 3 + 7;  // block header, end of block (symbol 256: 7 bits)
-    for (int p = 0; p < b;) {
-      const int m = mlen[p];
-      if (m >= 3) {
-        bits += length_bits(m) + distance_bits(mdist[p]);
-        p += m;
-      } else {
-        bits += xs[p] <= 143 ? 8 : 9;
-        ++p;
-      }
-    }
-    sizes[(int64_t)bt * B + blk] = (uint32_t)((bits + 7) / 8);
+  // the greedy parse visits 0, next(0), next(next(0)), ... with next(p) =
+  // p + (match length or 1): mark that orbit by binary lifting (round k
+  // follows next^(2^k) from every marked position), then sum the costs
+  for (int p = lane; p <= b; p += 32) {
+    nxt[p] = (uint16_t)(p == b ? b : p + (mlen[p] >= 3 ? mlen[p] : 1));
+    mark[p] = p == 0 ? 1 : 0;
   }
+  __syncwarp();
+  for (int span = 1; span < 2 * b; span <<= 1) {
+    for (int p = lane; p < b; p += 32)
+      if (mark[p]) mark[nxt[p]] = 1;
+    __syncwarp();
+    uint16_t j2[kMaxBlockBytes / 32 + 1];
+    int c = 0;
+    for (int p = lane; p <= b; p += 32) j2[c++] = nxt[nxt[p]];
+    __syncwarp();
+    c = 0;
+    for (int p = lane; p <= b; p += 32) nxt[p] = j2[c++];
+    __syncwarp();
+  }
+  int bits = 0;
+  for (int p = lane; p < b; p += 32)
+    if (mark[p]) bits += position_bits(mlen, mdist, xs, p);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) bits += __shfl_xor_sync(0xffffffffu, bits, off);
+  if (lane == 0)  // + block header (3) + end of block (symbol 256: 7 bits)
+    sizes[(int64_t)bt * B + blk] = (uint32_t)((bits + 10 + 7) / 8);
 }
 
 __global__ void __launch_bounds__(256) literal_flags_kernel(const uint32_t* sizes, int B,
@@ -120,7 +167,12 @@ __global__ void __launch_bounds__(256) literal_flags_kernel(const uint32_t* size
 cudaError_t launch_literal_flags_device(const uint8_t* bytes, int batch, int64_t n_bytes, int b,
                                         uint32_t* sizes, uint8_t* flags, cudaStream_t s) {
   const int B = (int)(n_bytes / b);
-  const size_t smem = kBlocksPerCta * deflate_warp_smem(b);  // <= 36 KB (b <= 1024)
+  const size_t smem = kBlocksPerCta * deflate_warp_smem(b);  // <= 73 KB (b <= 1024)
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(deflate_size_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+  }
   deflate_size_kernel<<<dim3((B + kBlocksPerCta - 1) / kBlocksPerCta, batch), kCompThreads, smem, s>>>(
       bytes, n_bytes, b, B, sizes);
   cudaError_t e = cudaGetLastError();
