@@ -40,7 +40,11 @@ def _rank_main(rank, world, port, out):
         q = W.qkv(w, "q", 0, head=0)[:64]
         args = type("A", (), dict(workload="gzip_8k", steps=1, warmup=0, gpus=world))()
         ref = bench.run_reference(args) if rank == 1 else None  # must return at once
-        out[rank] = dict(slowest=slowest, index=w["index"], q=q, ref=ref,
+        # every workload's copy on this rank, and a level-2 gist of the gist-of-gist decode
+        idx = {n: bench.workload_params(n, rank, "full")["index"]
+               for n in ("gist_coarse_20k", "gist_hier_decode_128k", "gzip_flags_128m", "gist_decode_128k")}
+        g2 = W.decode_gists2(bench.workload_params("gist_hier_decode_128k", rank, "small"), 0, "k")[0, :4]
+        out[rank] = dict(slowest=slowest, index=w["index"], q=q, ref=ref, idx=idx, g2=g2,
                          value=bench.weak_scaling_value(1e12, world, slowest, 1e12))
     finally:
         dist.destroy_process_group()
@@ -56,4 +60,6 @@ def test_two_gloo_ranks():
     assert r0["index"] != r1["index"]                 # independent problems
     assert not np.array_equal(r0["q"], r1["q"])       # different seeded inputs
     assert r1["ref"] is None                          # reference arm: rank 0 only
+    assert all(r1["idx"][n] == r0["idx"][n] + 1000 for n in r0["idx"])
+    assert not np.array_equal(r0["g2"], r1["g2"])
     assert r0["value"] == pytest.approx(2 / 15e-3)    # all ranks' work / slowest time
