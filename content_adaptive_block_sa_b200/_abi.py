@@ -74,7 +74,7 @@ PROTOTYPES = {
     "sa_get_device_status": (C.c_int, [vp, vp, P(C.c_int)]),
     "sa_literal_flags_from_sizes": (C.c_int, [P(C.c_uint32), i32, P(C.c_uint8)]),
     "sa_literal_flags_device": (C.c_int, [vp, i32, i64, i32, vp, vp, vp]),
-    "sa_selftest_wait_timeout": (C.c_int, [vp, C.c_size_t, i32, i64, vp]),
+    "sa_selftest_wait_timeout": (C.c_int, [vp, C.c_size_t, i32, vp]),
     "sa_block_lists_capacity": (C.c_int, [P(sa_mask_desc), P(sa_block_lists_sizes)]),
     "sa_build_block_mask_workspace_size": (C.c_int, [P(sa_mask_desc), P(C.c_size_t)]),
     "sa_build_block_mask": (C.c_int, [P(sa_mask_desc), vp, P(sa_block_lists), vp, C.c_size_t, vp]),

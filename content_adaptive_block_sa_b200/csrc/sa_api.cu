@@ -29,7 +29,7 @@ cudaError_t launch_hier_decode(const sa_hier_decode_desc&, const void*, const vo
 size_t hier_decode_workspace_bytes(const sa_hier_decode_desc&);
 cudaError_t launch_literal_flags_device(const uint8_t*, int, int64_t, int, uint32_t*, uint8_t*,
                                         cudaStream_t);
-cudaError_t launch_wait_timeout_selftest(void*, int, uint64_t, cudaStream_t);
+cudaError_t launch_wait_timeout_selftest(void*, int, cudaStream_t);
 }  // namespace sa
 
 using namespace sa;
@@ -258,15 +258,14 @@ sa_status sa_get_device_status(const void* ws, sa_stream_t stream, sa_status* ou
   return SA_OK;
 }
 
-sa_status sa_selftest_wait_timeout(void* ws, size_t ws_bytes, int32_t n_ctas, int64_t limit_ns,
+sa_status sa_selftest_wait_timeout(void* ws, size_t ws_bytes, int32_t n_ctas,
                                    sa_stream_t stream) {
   SA_CHECK(n_ctas >= 1 && n_ctas <= 1024, SA_ERR_INVALID_ARG);
-  SA_CHECK(limit_ns >= 1000 && limit_ns <= 100000000, SA_ERR_INVALID_ARG);  // 1 us .. 100 ms
   sa_status st = check_ws(ws, ws_bytes, kStatusBytes);
   if (st != SA_OK) return st;
   st = clear_status(ws, (cudaStream_t)stream);
   if (st != SA_OK) return st;
-  return cuda_status(launch_wait_timeout_selftest(ws, n_ctas, (uint64_t)limit_ns, (cudaStream_t)stream));
+  return cuda_status(launch_wait_timeout_selftest(ws, n_ctas, (cudaStream_t)stream));
 }
 
 sa_status sa_literal_flags_from_sizes(const uint32_t* sizes, int32_t num_blocks, uint8_t* flags) {

@@ -60,8 +60,7 @@ __device__ __forceinline__ uint64_t global_ns() {
 constexpr uint64_t kWaitNs = 4000000000ull;
 
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                          DeviceStatus* st, int where,
-                                          uint64_t limit_ns = kWaitNs) {
+                                          DeviceStatus* st, int where) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_ns();
   for (uint32_t i = 1;; ++i) {
@@ -72,7 +71,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
         *abort = 1;
         return false;
       }
-      if (global_ns() - t0 > limit_ns) {
+      if (global_ns() - t0 > kWaitNs) {
         report(st, SA_ERR_TIMEOUT, where);
         *abort = 1;
         return false;

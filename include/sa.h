@@ -361,15 +361,15 @@ sa_status sa_gist_hier_decode(const sa_hier_decode_desc* desc, const void* q,
                               int32_t* sel_groups, int32_t* sel_chunks, void* o, float* lse,
                               void* ws, size_t ws_bytes, sa_stream_t stream);
 
-/* Self-test of the device failure path (no fault is raised): n_ctas CTAs each
- * wait on an mbarrier that nothing completes, through the same bounded wait
- * every kernel of this library uses, with a wall-time limit of limit_ns
- * (1 us .. 100 ms). The first to give up records SA_ERR_TIMEOUT and the
- * location code 900 in the workspace's status word (read it with
- * sa_get_device_status after the stream synchronises); the rest leave on
- * seeing the word. Returns SA_OK once launched; SA_ERR_INVALID_ARG or
- * SA_ERR_WORKSPACE (ws shorter than 256 bytes) before any launch. */
-sa_status sa_selftest_wait_timeout(void* ws, size_t ws_bytes, int32_t n_ctas, int64_t limit_ns,
+/* Self-test of the device failure path (no fault is raised): n_ctas (1..1024)
+ * CTAs each wait on an mbarrier that nothing completes, through the same
+ * bounded wait every kernel of this library uses, 4 s wall-time limit
+ * included. The first to give up records SA_ERR_TIMEOUT and the location code
+ * 900 in the workspace's status word (read it with sa_get_device_status after
+ * the stream synchronises, about 4 s later); the rest leave on seeing the
+ * word. Returns SA_OK once launched; SA_ERR_INVALID_ARG or SA_ERR_WORKSPACE
+ * (ws shorter than 256 bytes) before any launch. */
+sa_status sa_selftest_wait_timeout(void* ws, size_t ws_bytes, int32_t n_ctas,
                                    sa_stream_t stream);
 
 /* ------------------------------------------------------------------ misc */

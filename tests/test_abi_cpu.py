@@ -168,8 +168,6 @@ def test_tensor_core_request_on_fp32_is_unsupported_before_any_launch(sa):
 def test_selftest_rejects_bad_arguments_without_a_device(sa):
     f = sa.lib().sa_selftest_wait_timeout
     fake = C.c_void_p(256)  # never dereferenced: every check comes before a launch
-    assert f(fake, 256, 0, 1_000_000, None) == 1          # no CTA
-    assert f(fake, 256, 2000, 1_000_000, None) == 1       # too many CTAs
-    assert f(fake, 256, 4, 10, None) == 1                 # limit below 1 us
-    assert f(fake, 256, 4, 10**9, None) == 1              # limit above 100 ms
-    assert f(fake, 16, 4, 1_000_000, None) == 3           # workspace shorter than the status word
+    assert f(fake, 256, 0, None) == 1      # no CTA
+    assert f(fake, 256, 2000, None) == 1   # too many CTAs
+    assert f(fake, 16, 4, None) == 3       # workspace shorter than the status word

@@ -1,6 +1,6 @@
-"""Device failure path without a fault: the library's bounded wait, given a
-flag nothing sets and a short limit, records SA_ERR_TIMEOUT with its location
-in the status word, every CTA leaves, and the context keeps working."""
+"""Device failure path without a fault: the library's bounded wait (4 s), given
+a flag nothing sets, records SA_ERR_TIMEOUT with its location in the status
+word, every CTA leaves, and the context keeps working."""
 import numpy as np
 import pytest
 import torch
@@ -17,12 +17,12 @@ SA_ERR_TIMEOUT = 5
 
 @pytest.mark.parametrize("n_ctas", [1, 148])
 def test_bounded_wait_reports_timeout(sa, n_ctas):
-    code, where = sa.selftest_wait_timeout(n_ctas=n_ctas, limit_ns=2_000_000)
+    code, where = sa.selftest_wait_timeout(n_ctas=n_ctas)
     assert (code, where) == (SA_ERR_TIMEOUT, 900)
 
 
 def test_context_still_works_after_a_timeout(sa):
-    assert sa.selftest_wait_timeout(n_ctas=4, limit_ns=1_000_000)[0] == SA_ERR_TIMEOUT
+    assert sa.selftest_wait_timeout(n_ctas=4)[0] == SA_ERR_TIMEOUT
     w = W.scaled("gist_decode_128k", index=990, n_seq=1, cache_len=16 * 64, chunk=16, n_gists=64,
                  top_k=4, window=32, heads=4, kv_heads=2)
     q = W.decode_query(w)
