@@ -171,3 +171,63 @@ def test_selftest_rejects_bad_arguments_without_a_device(sa):
     assert f(fake, 256, 0, None) == 1      # no CTA
     assert f(fake, 256, 2000, None) == 1   # too many CTAs
     assert f(fake, 16, 4, None) == 3       # workspace shorter than the status word
+
+
+def _decode_desc(sa, **kw):
+    L = sa._abi
+    d = dict(n_seq=16, cache_len=131072, chunk=32, n_gists=4096, top_k=64, window=512,
+             num_q_heads=32, num_kv_heads=8, head_dim=128, select_rule=0, softmax_scale=0.0,
+             q_strides=(C.c_int64 * 2)(4096, 128), gist_strides=(C.c_int64 * 3)(4096 * 1024, 4096 * 128, 128),
+             cache_strides=(C.c_int64 * 3)(131072 * 1024, 131072 * 128, 128),
+             o_strides=(C.c_int64 * 2)(4096, 128), top_p=1.0)
+    d.update(kw)
+    return L.sa_decode_desc(**d)
+
+
+def test_decode_select_rules_validated_without_a_device(sa):
+    n = C.c_size_t()
+    f = lambda d: sa.lib().sa_gist_decode_workspace_size(C.byref(d), C.byref(n))
+    for rule in range(4):
+        assert f(_decode_desc(sa, select_rule=rule, top_p=0.5)) == 0
+    assert f(_decode_desc(sa)) == 0
+    base = n.value
+    assert f(_decode_desc(sa, select_rule=1)) == 0 and n.value > base  # per-head logits kept
+    assert f(_decode_desc(sa, select_rule=4)) == 1                     # no such rule
+    assert f(_decode_desc(sa, select_rule=2, top_p=0.0)) == 1          # empty nucleus
+    assert f(_decode_desc(sa, select_rule=2, top_p=1.5)) == 1
+
+
+def _hier_desc(sa, **kw):
+    d = dict(n_seq=16, cache_len=131072, chunk=32, n_gists=4096, fanout=32, top_k2=8, top_k=64,
+             window=512, num_q_heads=32, num_kv_heads=8, head_dim=128, softmax_scale=0.0,
+             q_strides=(C.c_int64 * 2)(4096, 128), gist_strides=(C.c_int64 * 3)(4096 * 1024, 4096 * 128, 128),
+             gist2_strides=(C.c_int64 * 3)(128 * 1024, 128 * 128, 128),
+             cache_strides=(C.c_int64 * 3)(131072 * 1024, 131072 * 128, 128),
+             o_strides=(C.c_int64 * 2)(4096, 128))
+    d.update(kw)
+    return sa._abi.sa_hier_decode_desc(**d)
+
+
+def test_hier_decode_validated_without_a_device(sa):
+    n = C.c_size_t()
+    f = lambda d: sa.lib().sa_gist_hier_decode_workspace_size(C.byref(d), C.byref(n))
+    assert f(_hier_desc(sa)) == 0 and n.value >= 256
+    assert f(_hier_desc(sa, fanout=3)) == 1          # n_gists % fanout != 0
+    assert f(_hier_desc(sa, cache_len=1000)) == 1    # n_gists * chunk != cache_len
+    assert f(_hier_desc(sa, top_k2=300)) == 2        # above 256
+    assert f(_hier_desc(sa, head_dim=64)) == 2
+    assert f(_hier_desc(sa, num_kv_heads=3)) == 1
+    # null outputs are refused before any launch
+    d = _hier_desc(sa)
+    fake = C.c_void_p(4096)
+    assert sa.lib().sa_gist_hier_decode(C.byref(d), fake, fake, fake, fake, fake, fake, fake, None, fake,
+                                        fake, fake, fake, 1 << 30, None) == 1
+
+
+def test_device_flags_validated_without_a_device(sa):
+    f = sa.lib().sa_literal_flags_device
+    fake = C.c_void_p(4096)
+    assert f(None, 1, 1024, 128, fake, fake, None) == 1      # no bytes
+    assert f(fake, 1, 1000, 128, fake, fake, None) == 1      # n_bytes % b != 0
+    assert f(fake, 1, 4096, 2048, fake, fake, None) == 2     # b above 1024
+    assert f(fake, 0, 1024, 128, fake, fake, None) == 1      # no sequence
