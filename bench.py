@@ -343,6 +343,17 @@ class GistWorkload(GzipWorkload):
             "head 0, last 2048 query rows, exact visible pairs, fp64", dt
 
 
+def repeat_for(budget_s, fn):
+    """Calls fn until budget_s seconds have passed (at least once): (calls, seconds)."""
+    n, t0 = 0, time.perf_counter()
+    while True:
+        fn()
+        n += 1
+        dt = time.perf_counter() - t0
+        if dt >= budget_s:
+            return n, dt
+
+
 # decode chunk selection rules (sa_select_rule)
 SELECT_RULES = {"sum_logits": 0, "sum_probs": 1, "top_p": 2, "per_head": 3}
 
@@ -412,7 +423,7 @@ class DecodeWorkload:
     def io_bytes(self):
         return self.h_q.numel() * 2, self.o.numel() * 2 + self.lse.numel() * 4 + self.sel.numel() * 4
 
-    def cpu_baseline(self):
+    def cpu_baseline(self, budget_s=10.0):
         from oracle import decode as D
         w = self.w
         q = W.decode_query(w)[0]
@@ -421,15 +432,17 @@ class DecodeWorkload:
         rv = [W.decode_raw(w, 0, g, "v") for g in range(w["kv_heads"])]
         raw_k, raw_v = (lambda g: rk[g]), (lambda g: rv[g])
         rule = SELECT_RULES[w.get("select", "sum_logits")]
-        t0 = time.perf_counter()
-        sel = D.decode_one(q, gk, gv, raw_k, raw_v, w["chunk"], w["window"], w["top_k"],
-                           rule=rule, top_p=w.get("top_p", 1.0))[0]
-        dt = time.perf_counter() - t0
-        sel = sel.reshape(w["kv_heads"], -1)  # the group's rows (one per head under the per-head rule)
+        out = {}
+
+        def one():
+            out["sel"] = D.decode_one(q, gk, gv, raw_k, raw_v, w["chunk"], w["window"], w["top_k"],
+                                      rule=rule, top_p=w.get("top_p", 1.0))[0]
+        n, dt = repeat_for(budget_s, one)
+        sel = out["sel"].reshape(w["kv_heads"], -1)  # the group's rows (one per head: per-head rule)
         n_chunks = sum(len(np.unique(r_[r_ >= 0])) for r_ in sel)
         rows = w["kv_heads"] * (w["n_gists"] + w["window"]) + n_chunks * w["chunk"]
-        return rows * w["head_dim"] * 2 * 2 / dt / 1e9, \
-            "sequence 0, all kv heads (raw cache generation excluded), fp64", dt
+        return n * rows * w["head_dim"] * 2 * 2 / dt / 1e9, \
+            f"sequence 0 decoded {n} times, all kv heads (raw cache generation excluded), fp64", dt
 
 
 class HierDecodeWorkload(DecodeWorkload):
@@ -498,7 +511,7 @@ class HierDecodeWorkload(DecodeWorkload):
         return (self.h_q.numel() * 2,
                 self.o.numel() * 2 + self.lse.numel() * 4 + (self.sel.numel() + self.sel2.numel()) * 4)
 
-    def cpu_baseline(self):
+    def cpu_baseline(self, budget_s=10.0):
         from oracle import decode as D
         w = self.w
         q = W.decode_query(w)[0]
@@ -506,15 +519,18 @@ class HierDecodeWorkload(DecodeWorkload):
         gk, gv = W.decode_gists(w, 0, "k"), W.decode_gists(w, 0, "v")
         rk = [W.decode_raw(w, 0, g, "k") for g in range(w["kv_heads"])]
         rv = [W.decode_raw(w, 0, g, "v") for g in range(w["kv_heads"])]
-        t0 = time.perf_counter()
-        sel2, sel1, _, _ = D.hier_decode_one(q, g2k, g2v, gk, gv, rk, rv, w["chunk"], w["fanout"],
-                                             w["top_k2"], w["top_k"], w["window"])
-        dt = time.perf_counter() - t0
+        out = {}
+
+        def one():
+            out["sel"] = D.hier_decode_one(q, g2k, g2v, gk, gv, rk, rv, w["chunk"], w["fanout"],
+                                           w["top_k2"], w["top_k"], w["window"])[:2]
+        n, dt = repeat_for(budget_s, one)
+        sel2, sel1 = out["sel"]
         n2 = w["n_gists"] // w["fanout"]
         rows = (w["kv_heads"] * (n2 + w["window"]) + int((sel2 >= 0).sum()) * w["fanout"]
                 + int((sel1 >= 0).sum()) * w["chunk"])
-        return rows * w["head_dim"] * 2 * 2 / dt / 1e9, \
-            "sequence 0, all kv heads (raw cache generation excluded), fp64", dt
+        return n * rows * w["head_dim"] * 2 * 2 / dt / 1e9, \
+            f"sequence 0 decoded {n} times, all kv heads (raw cache generation excluded), fp64", dt
 
 
 class FlagsWorkload:
@@ -551,14 +567,18 @@ class FlagsWorkload:
     def io_bytes(self):
         return self.h_x.numel(), self.flags.numel()
 
-    def cpu_baseline(self):
+    def cpu_baseline(self, budget_s=10.0):
         from oracle import deflate_size as F
         src = W.WORKLOADS[self.w["rows_from"]]
-        x = W.workload_bytes(src, 0)[:8192]  # 64 blocks of the first row
-        t0 = time.perf_counter()
-        F.block_sizes(x, self.w["block"])
-        dt = time.perf_counter() - t0
-        return len(x) / dt / 1e9, "first 8 KiB of row 0 (64 blocks), pure Python", dt
+        rows = [W.workload_bytes(src, i) for i in range(src["batch"])]
+        chunks = [r[i:i + 8192] for r in rows for i in range(0, len(r), 8192)]  # 64 blocks each
+        k = [0]
+
+        def one():
+            F.block_sizes(chunks[k[0] % len(chunks)], self.w["block"])
+            k[0] += 1
+        n, dt = repeat_for(budget_s, one)
+        return n * 8192 / dt / 1e9, f"{n} successive 8 KiB pieces of the rows (64 blocks each), pure Python", dt
 
 
 SMALL = {"gzip_8k": dict(batch=8), "gzip_64k_fwdbwd": dict(batch=1, heads=4, kv_heads=4),
@@ -644,6 +664,9 @@ def run_reference(args):
             # one whole head per step, cycling through the three classes
             v, sample, dt = fn(wl, heads=[(0, H // 2, H - 1)[i % 3]])
             sample = "batch row 0, one whole head per step cycling local/literal/hybrid, fp64"
+        elif wl.w["kind"] in ("decode", "hier", "flags"):
+            # each step a bounded sample: the whole run stays within a few minutes
+            v, sample, dt = fn(wl, budget_s=max(0.2, min(10.0, 120.0 / (args.steps + args.warmup))))
         else:
             v, sample, dt = fn(wl)
         if i >= args.warmup:
