@@ -166,3 +166,40 @@ def backward_cols(q, k, v, do, keys_of_row, rows_of_key, cols, scale=None):
             dk[n] += ds * np.asarray(q[p], np.float64) * scale
             dv[n] += pj * dop
     return dk, dv
+
+
+def backward_cols_chunked(q, k, v, do, mask, rows, cols, scale=None, row_chunk=256):
+    """dK and dV for selected keys only, by whole chunks of query rows.
+
+    The same sums as ``backward_cols`` (over the query rows p that attend key
+    j: dS_pj q_p * scale and P_pj dO_p), evaluated a chunk of rows at a time:
+    each row's softmax is taken over its own allowed keys, restricted to the
+    union of the chunk's keys (a key no row of the chunk may attend adds
+    nothing). ``rows`` must hold every query row that attends any of ``cols``
+    (extra rows add zero); ``mask`` is a callable rows -> bool [len(rows), Nk].
+    """
+    q = np.asarray(q, np.float64)
+    scale = 1.0 / np.sqrt(q.shape[1]) if scale is None else float(scale)
+    cols = np.asarray(cols)
+    rows = np.asarray(rows)
+    vc = np.asarray(v[cols], np.float64)
+    dk = np.zeros((len(cols), k.shape[1]))
+    dv = np.zeros((len(cols), v.shape[1]))
+    for r0 in range(0, len(rows), row_chunk):
+        rr = rows[r0:r0 + row_chunk]
+        allowed = np.asarray(mask(rr), dtype=bool)
+        keys = np.nonzero(allowed.any(axis=0))[0]
+        qc = q[rr]
+        doc = np.asarray(do[rr], np.float64)
+        s = _scores(qc, np.asarray(k[keys], np.float64), allowed[:, keys], scale)
+        m = s.max(axis=1, keepdims=True)
+        lse = m[:, 0] + np.log(np.exp(s - m).sum(axis=1))
+        p = np.exp(s - lse[:, None])
+        D = (doc * (p @ np.asarray(v[keys], np.float64))).sum(axis=1)
+        at = np.searchsorted(keys, cols)
+        seen = (at < len(keys)) & (keys[np.minimum(at, len(keys) - 1)] == cols)
+        pc = np.where(seen[None, :], p[:, np.minimum(at, len(keys) - 1)], 0.0)
+        ds = pc * (doc @ vc.T - D[:, None])
+        dk += (ds.T @ qc) * scale
+        dv += pc.T @ doc
+    return dk, dv

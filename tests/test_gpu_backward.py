@@ -1,6 +1,8 @@
-"""sa_backward vs the oracle: dQ, dK, dV element by element on small cases;
-at the 64K workload sampled dQ rows, sampled dK/dV keys, and the identities
-sum_j dK_j = 0 and sum_j dV_j = sum_p dO_p that hold at any size."""
+"""sa_backward vs the oracle: dQ, dK, dV element by element on small cases
+and on whole heads whose lists are long (a 16K sequence with 60% literal
+blocks); at the 64K workload sampled dQ rows, whole key blocks that every
+later literal query block sees (the longest column lists) and keys seen only
+nearby, and the identity sum_j dV_j = sum_p dO_p that holds at any size."""
 import numpy as np
 import pytest
 import torch
@@ -95,6 +97,45 @@ def test_backward_full_size(sa):
             rk, rv = A.backward_cols(q[bt, :, h], k[bt, :, h], v[bt, :, h], do[bt, :, h], keys_of, rows_of, cols)
             check_close(dk[bt, cols, h], rk, "bf16", f"dK cols b{bt} h{h}")
             check_close(dv[bt, cols, h], rv, "bf16", f"dV cols b{bt} h{h}")
+        # long column lists: the first and a middle literal key block of the
+        # literal and hybrid heads, seen by every later literal query block
+        # (the key-major pass walks about 200 query blocks for each)
+        lit_blocks = np.nonzero(fo[bt])[0]
+        for h in (w["heads"] // 2, w["heads"] - 1):
+            bm = masks[cls[h]]
+            jb = [int(lit_blocks[0]), int(lit_blocks[len(lit_blocks) // 2])]
+            cols = np.concatenate([np.arange(j * b, (j + 1) * b) for j in jb])
+            qblocks = np.nonzero(bm[:, jb].any(axis=1))[0]
+            assert len(qblocks) >= 100, len(qblocks)
+            rows = (qblocks[:, None] * b + np.arange(b)[None, :]).ravel()
+            mask = lambda r: G.token_mask(bm, b, rows=r)
+            rk, rv = A.backward_cols_chunked(q[bt, :, h], k[bt, :, h], v[bt, :, h], do[bt, :, h],
+                                             mask, rows, cols)
+            check_close(dk[bt, cols, h], rk, "bf16", f"dK literal blocks {jb} b{bt} h{h}")
+            check_close(dv[bt, cols, h], rv, "bf16", f"dV literal blocks {jb} b{bt} h{h}")
+
+
+def test_backward_long_lists_whole_heads(sa):
+    """Whole literal and hybrid heads of a 16K sequence with 60% literal
+    128-token blocks: row lists and column lists of 60 to 80 blocks, compared
+    element by element (dQ, dK, dV) with the oracle, on both implementations."""
+    w = W.scaled("gzip_8k", index=310, batch=1, seq_len=16384, block=128, window=2, heads=4,
+                 kv_heads=4, head_dim=128, dtype="bf16", p_literal=0.6)
+    q, k, v, do = gzip_inputs(w, with_do=True)
+    flags = gzip_flags_oracle(w)
+    assert np.array_equal(flags, gzip_flags_product(sa, w))
+    masks = G.block_masks(flags[0], w["window"])
+    cls = G.head_classes(w["heads"])
+    got = {impl: run(sa, w, q, k, v, do, flags, IMPLS[impl]) for impl in IMPLS}
+    for h in (2, 3):  # the literal head and the hybrid head
+        bm = masks[cls[h]]
+        assert bm.sum(axis=0).max() >= 60 and bm.sum(axis=1).max() >= 60
+        allowed = G.token_mask(bm, w["block"])
+        rq, rk, rv, _, _ = A.backward(q[0, :, h], k[0, :, h], v[0, :, h], do[0, :, h], allowed)
+        for impl, (o, dq, dk, dv) in got.items():
+            check_close(dq[0, :, h], rq, "bf16", f"{impl} dQ h{h}")
+            check_close(dk[0, :, h], rk, "bf16", f"{impl} dK h{h}")
+            check_close(dv[0, :, h], rv, "bf16", f"{impl} dV h{h}")
 
 
 # ------------------------------------------------------------------ gist layout
@@ -168,3 +209,20 @@ def test_gist_backward_full_size_sampled(sa):
             rv += b
         check_close(dk[0, cols, hk], rk, "bf16", f"dK raw cols kv{hk}")
         check_close(dv[0, cols, hk], rv, "bf16", f"dV raw cols kv{hk}")
+    # keys every later query sees (sinks and gists): their gradients come from the
+    # far items of the dK/dV pass (about 256 query tiles each) and the far scatter
+    gists = np.nonzero(g)[0]
+    far = {0: [3, S - 1, int(gists[len(gists) // 2])], w["kv_heads"] - 1: [int(gists[-40])]}
+    vis = lambda r: Gi.visibility(g, S, Wn, rows=r)
+    for hk, logical in far.items():
+        logical = np.array(logical)
+        rows = np.arange(logical.min(), N)
+        rk = np.zeros((len(logical), w["head_dim"]))
+        rv = np.zeros_like(rk)
+        for h in range(hk * rep, (hk + 1) * rep):
+            a, b = A.backward_cols_chunked(q[0, inv, h], k[0, inv, hk], v[0, inv, hk], do[0, inv, h],
+                                           vis, rows, logical)
+            rk += a
+            rv += b
+        check_close(dk[0, inv[logical], hk], rk, "bf16", f"dK far keys {logical.tolist()} kv{hk}")
+        check_close(dv[0, inv[logical], hk], rv, "bf16", f"dV far keys {logical.tolist()} kv{hk}")

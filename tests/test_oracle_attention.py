@@ -129,3 +129,14 @@ def test_row_and_column_forms_of_backward_agree_with_dense():
     dk2, dv2 = A.backward_cols(q, k, v, do, keys_of, rows_of, sel)
     np.testing.assert_allclose(dk2, dk[sel], atol=1e-12)
     np.testing.assert_allclose(dv2, dv[sel], atol=1e-12)
+    # chunked column form: every row, or only the rows that attend the keys,
+    # in chunks that split query blocks
+    mask = lambda r: allowed[r]
+    for rows in (np.arange(N), np.unique(np.concatenate([rows_of(j) for j in sel]))):
+        dk3, dv3 = A.backward_cols_chunked(q, k, v, do, mask, rows, sel, row_chunk=7)
+        np.testing.assert_allclose(dk3, dk[sel], atol=1e-12)
+        np.testing.assert_allclose(dv3, dv[sel], atol=1e-12)
+    # rows that do not attend a key add nothing to its gradients
+    others = np.setdiff1d(np.arange(N), rows_of(sel[1]))
+    z = A.backward_cols_chunked(q, k, v, do, mask, others, sel[1:2])
+    assert others.size and not z[0].any() and not z[1].any()
