@@ -5,9 +5,9 @@
 
 One step = one pass of the workload's hot path over one batch of synthetic,
 seeded input already resident in HBM:
-  gzip_8k            mask build + forward      (default; batch 8, N=8192, b=64)
+  gist_prefill_32k   layout build + forward    (default; N=32768, 32q/8kv heads)
+  gzip_8k            mask build + forward      (batch 8, N=8192, b=64)
   gzip_64k_fwdbwd    mask build + forward + backward (batch 2, N=65536, b=128)
-  gist_prefill_32k   layout build + forward    (N=32768, 32q/8kv heads)
   gist_decode_128k   one decode step           (16 seqs, 131072-token caches)
   gist_prefill_32k_fwdbwd  layout build + forward + backward on the 32K gist inputs
   gist_coarse_20k    coarse (segment-wise) layout build + forward: 16 segments
@@ -17,8 +17,10 @@ seeded input already resident in HBM:
                      (128 level-2 gists, top-8 groups, top-64 chunks)
   gzip_flags_128m    on-device literal flags over 2048 rows of 64 KiB (b=128)
 Prefill/backward workloads report visited-tile TFLOP/s (every visited block
-pair counted as a full b x b tile: 4*d*b^2 forward, 10*d*b^2 backward); the
-decode workload reports algorithmic HBM GB/s. Inputs are larger than the
+pair counted as a full b x b tile: 4*d*b^2 forward, 10*d*b^2 backward; gist
+layouts count their tile-list sub-blocks, 128 or 32 columns wide), and beside
+it the same step counted by exact (query, key) edges (4*d per edge forward,
+10*d backward); the decode workloads report algorithmic HBM GB/s. Inputs are larger than the
 126 MB L2, so no flush is needed between steps. Under torchrun each rank runs
 its own independent copy of the workload (weak scaling, no collective on the
 data path); the time is the max over ranks.
@@ -104,13 +106,14 @@ class ClockSampler:
 _host_out = {}
 
 
-# the kernels whose DRAM traffic profiles/traffic.md records, and their sources; the
+# the kernels whose DRAM traffic profiles/traffic.json records, and their sources; the
 # backward is reported as one unit: row prep, the query-major dQ pass and the
 # key-major dK/dV pass
 KERNEL_SOURCES = {"fwd_tc_kernel": ["attn_fwd_sm100.cu"],
                   "backward": ["attn_bwd_sm100.cu", "attn_dq_sm100.cu"],
                   "decode_tc_kernel": ["decode_sm100.cu"],
                   "hier decode (6 CUDA-core passes)": ["decode.cu"],
+                  "hier_tc_kernel": ["decode_sm100.cu"],
                   "deflate_size_kernel + literal_flags_kernel": ["compress.cu"]}
 
 
@@ -126,15 +129,15 @@ def kernel_digest(kernel):
 
 
 def recorded_traffic(workload, kernel):
-    """DRAM bytes per launch from profiles/traffic.md, or None when no row
-    exists or the kernel's sources changed since the counters were taken."""
-    path = os.path.join(ROOT, "profiles", "traffic.md")
+    """DRAM bytes per full-size launch from profiles/traffic.json, or None when
+    no row exists or the kernel's sources changed since the counters were taken
+    (a stale row is reported as null until a new capture replaces it)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
     if kernel not in KERNEL_SOURCES or not os.path.exists(path):
         return None
-    for line in open(path):
-        cells = [c.strip() for c in line.strip().strip("|").split("|")]
-        if len(cells) == 8 and cells[0] == workload and cells[1] == kernel:
-            return int(cells[5]) if cells[2] == kernel_digest(kernel) else None
+    for row in json.load(open(path))["rows"]:
+        if row["workload"] == workload and row["kernel"] == kernel:
+            return int(row["traffic"]) if row["source"] == kernel_digest(kernel) else None
     return None
 
 
@@ -188,6 +191,11 @@ class GzipWorkload:
         self.pairs = pairs
         self.flops_fwd = 4.0 * d * b * b * pairs
         self.flops = self.flops_fwd * (1 + (2.5 if backward else 0))
+        # exact token edges: every list row holds its diagonal block, whose
+        # b(b+1)/2 causal pairs replace the b*b of a full tile
+        diag = Bt * H * B
+        self.exact_fwd = 4.0 * d * (b * b * (pairs - diag) + diag * b * (b + 1) // 2)
+        self.exact = self.exact_fwd * (1 + (2.5 if backward else 0))
         # builder + forward (+ the pairing pre-pass for 64-token blocks) (+ backward:
         # row prep, query-major dQ pass, key-major dK/dV pass)
         self.kernels_per_step = 2 + (1 if b == 64 else 0) + (3 if backward else 0)
@@ -244,7 +252,7 @@ class GzipWorkload:
         rows = np.arange(N - R, N)
         data = {h: [W.qkv(w, t, 0, head=h) for t in ("q", "k", "v", "do")] for h in heads}
         t0 = time.perf_counter()
-        flops = 0.0
+        flops = exact = 0.0
         for h in heads:
             bm = masks[cls[h]]
             q, k, v, do = data[h]
@@ -254,10 +262,12 @@ class GzipWorkload:
             else:
                 A.forward(q[rows], k, v, mask)
             pairs = int(bm[(N - R) // b:].sum())
-            flops += (4.0 + (10.0 if self.backward else 0.0)) * w["head_dim"] * b * b * pairs
+            per = (4.0 + (10.0 if self.backward else 0.0)) * w["head_dim"]
+            flops += per * b * b * pairs
+            exact += per * (b * b * (pairs - R // b) + (R // b) * b * (b + 1) // 2)
         dt = time.perf_counter() - t0
         return flops / dt / 1e12, (f"batch row 0, heads {heads} (one per class), last {R} query "
-                                   "rows each, fp64"), dt
+                                   "rows each, fp64"), dt, exact / dt / 1e12
 
 
 class GistWorkload(GzipWorkload):
@@ -292,6 +302,8 @@ class GistWorkload(GzipWorkload):
         width = np.where(kinds == 2, w["gist_tail"], 128)
         self.flops_fwd = 4.0 * d * H * 128 * float(width.sum())
         self.flops = self.flops_fwd * (1 + (2.5 if backward else 0))
+        self.exact_fwd = 4.0 * d * H * float(gist_visible_pairs(w))
+        self.exact = self.exact_fwd * (1 + (2.5 if backward else 0))
         # builder (4 launches) + sink/gist gather + near-tile masks + forward (+ backward:
         # row prep, the three gist pre-passes, dQ pass, dK/dV pass, far scatter)
         self.kernels_per_step = 7 + (7 if backward else 0)
@@ -336,11 +348,38 @@ class GistWorkload(GzipWorkload):
         else:
             A.forward(q[rows], k, v, mask)
         dt = time.perf_counter() - t0
-        # algorithmic FLOPs of those rows: exact visible pairs x 4d (+ 10d backward)
+        # the GPU leg's two counts for those rows (the last 16 tiles hold exactly
+        # the last 2048 logical positions: the shift stays inside a tile):
+        # tile-list sub-blocks, and exact visible pairs
+        T = N // 128
+        _, _, kinds = Gi.tile_lists(lambda r: vis_rows(perm[r])[:, perm], 128, w["gist_tail"], N=N,
+                                    query_tiles=range(T - 16, T))
+        width = float(np.where(kinds == Gi.TAIL, w["gist_tail"], 128).sum())
         n_vis = int(vis_rows(rows).sum())
-        per = 4.0 + (10.0 if self.backward else 0.0)
-        return per * w["head_dim"] * n_vis / dt / 1e12, \
-            "head 0, last 2048 query rows, exact visible pairs, fp64", dt
+        per = (4.0 + (10.0 if self.backward else 0.0)) * w["head_dim"]
+        return per * 128 * width / dt / 1e12, \
+            "head 0, last 2048 query rows, fp64", dt, per * n_vis / dt / 1e12
+
+
+def gist_visible_pairs(w):
+    """Visible (query, key) pairs of one head of a gist layout, counted from
+    its rule: key j <= query i is seen when j is a sink or a gist, or lies in
+    i's window (fine layout: i - j < window) or segment (coarse layout)."""
+    N, S, r = w["seq_len"], w["sinks"], w["ratio"]
+    p = np.arange(N, dtype=np.int64)
+    L = w.get("gist_segment", 0)
+    if L:
+        period = L + L // r
+        gist = (p >= S) & ((p - S) % period >= L)
+    else:
+        gist = (p >= S) & ((p - S) % (r + 1) == r)
+    pref = np.concatenate([[0], np.cumsum((p < S) | gist)])  # sinks + gists below x
+    if L:
+        start = np.where(p < S, 0, S + (p - S) // period * period)  # own segment's first position
+        near = p - start + 1
+        return int((near + np.where(p < S, 0, pref[start])).sum())
+    Wn = w["window"]
+    return int((np.minimum(Wn, p + 1) + pref[np.maximum(0, p - Wn + 1)]).sum())
 
 
 def repeat_for(budget_s, fn):
@@ -661,29 +700,32 @@ def run_reference(args):
     H = wl.w.get("heads", 1)
     for i in range(args.warmup + args.steps):
         if wl.w["kind"] == "gzip":
-            # one whole head per step, cycling through the three classes
-            v, sample, dt = fn(wl, heads=[(0, H // 2, H - 1)[i % 3]])
-            sample = "batch row 0, one whole head per step cycling local/literal/hybrid, fp64"
+            # one head per step, cycling through the three classes
+            res = fn(wl, heads=[(0, H // 2, H - 1)[i % 3]])
+            sample = res[1].replace("heads", "one head per step cycling local/literal/hybrid:", 1)
         elif wl.w["kind"] in ("decode", "hier", "flags"):
             # each step a bounded sample: the whole run stays within a few minutes
-            v, sample, dt = fn(wl, budget_s=max(0.2, min(10.0, 120.0 / (args.steps + args.warmup))))
+            res = fn(wl, budget_s=max(0.2, min(10.0, 120.0 / (args.steps + args.warmup))))
+            sample = res[1]
         else:
-            v, sample, dt = fn(wl)
+            res = fn(wl)
+            sample = res[1]
         if i >= args.warmup:
-            vals.append((v, dt))
-    value = float(np.mean([v for v, _ in vals]))
+            vals.append((res[0], res[2], res[3] if len(res) > 3 else None))
+    value = float(np.mean([v[0] for v in vals]))
+    exact = None if vals[0][2] is None else float(np.mean([v[2] for v in vals]))
     unit = "GB/s" if wl.w["kind"] in ("decode", "hier", "flags") else "TFLOP/s"
     cores = len(os.sched_getaffinity(0))
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": value, "unit": unit, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": float(np.mean([dt for _, dt in vals]) * 1e3),
+        "ms_per_step": float(np.mean([v[1] for v in vals]) * 1e3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "u8" if wl.w["kind"] == "flags" else "f64",
         "data": "synthetic",
         "config": {"workload": args.workload, **({"select": args.select} if args.select else {})},
         "cpu_baseline": {"value": value, "unit": unit, "cores": cores, "kind": "oracle",
-                         "sample": sample},
+                         "sample": sample, **({"exact_edges_value": exact} if exact else {})},
         "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}))
 
 
@@ -692,7 +734,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="gzip_8k",
+    ap.add_argument("--workload", default="gist_prefill_32k",
                     choices=["gzip_8k", "gzip_64k_fwdbwd", "gist_prefill_32k", "gist_decode_128k",
                              "gist_prefill_32k_fwdbwd", "gist_coarse_20k", "gist_coarse_20k_fwdbwd",
                              "gist_hier_decode_128k", "gzip_flags_128m"])
@@ -775,14 +817,18 @@ def main():
     else:
         value = weak_scaling_value(wl.flops, world, ms, 1e12)
         e2e_value = weak_scaling_value(wl.flops, world, e2e_ms, 1e12)
+        value_exact = weak_scaling_value(wl.exact, world, ms, 1e12)
         fwd_ach = wl.flops_fwd / (kern_ms * 1e-3) / 1e12
         if bwd_ms is not None and bwd_ms > kern_ms:  # the backward dominates the step
             ach = (wl.flops - wl.flops_fwd) / (bwd_ms * 1e-3) / 1e12
+            ach_exact = (wl.exact - wl.exact_fwd) / (bwd_ms * 1e-3) / 1e12
             kname = "backward"
         else:
             ach, kname = fwd_ach, wl.kernel
+            ach_exact = wl.exact_fwd / (kern_ms * 1e-3) / 1e12
         roof = {"bound": "tensor", "achieved": ach, "peak": bf16, "unit": "TFLOP/s",
-                "frac": ach / bf16, "traffic": None, "peak_source": src, "kernel": kname}
+                "frac": ach / bf16, "traffic": None, "peak_source": src, "kernel": kname,
+                "exact_tflops": ach_exact, "exact_frac": ach_exact / bf16}
         if bwd_ms is not None:
             roof["forward_tflops"] = fwd_ach
             roof["backward_ms"] = bwd_ms
@@ -806,11 +852,16 @@ def main():
         "gpu_launches": int(wl.kernels_per_step * args.steps),
         "kernel_ms": kern_ms,
     }
+    if wl.unit == "TFLOP/s":
+        # the same step counted by exact (query, key) edges instead of visited tiles
+        line["value_exact_edges"] = value_exact
     if world == 1 and not args.no_cpu_baseline:
         torch.set_num_threads(len(os.sched_getaffinity(0)))
-        v, sample, dt = wl.cpu_baseline()
-        line["cpu_baseline"] = {"value": v, "unit": wl.unit, "cores": len(os.sched_getaffinity(0)),
-                                "kind": "oracle", "sample": sample, "seconds": dt}
+        res = wl.cpu_baseline()
+        line["cpu_baseline"] = {"value": res[0], "unit": wl.unit, "cores": len(os.sched_getaffinity(0)),
+                                "kind": "oracle", "sample": res[1], "seconds": res[2]}
+        if len(res) > 3:
+            line["cpu_baseline"]["exact_edges_value"] = res[3]
     print(json.dumps(line))
     if world > 1:
         dist.destroy_process_group()

@@ -73,7 +73,7 @@ def shift_permutation(is_gist, tile: int) -> np.ndarray:
     return np.asarray(perm, dtype=np.int32)
 
 
-def tile_lists(vis_phys, tile: int, tail: int, N: int | None = None):
+def tile_lists(vis_phys, tile: int, tail: int, N: int | None = None, query_tiles=None):
     """Per query tile, the key tiles that hold at least one visible pair.
 
     ``vis_phys`` is the visibility matrix in physical (shifted) order. Each
@@ -83,12 +83,14 @@ def tile_lists(vis_phys, tile: int, tail: int, N: int | None = None):
     gists), MASKED otherwise. Returned as
     (row_ptr [T+1], key_tile [nnz], kind [nnz]) int32 with key tiles ascending.
     ``vis_phys`` may also be a callable rows -> bool [len(rows), N] (then N
-    must be given), evaluated one query tile at a time.
+    must be given), evaluated one query tile at a time. ``query_tiles``
+    restricts the lists to some query tiles (row_ptr then has one entry per
+    listed tile, plus one).
     """
     N = vis_phys.shape[0] if N is None else N
     T = (N + tile - 1) // tile
     row_ptr, keys, kinds = [0], [], []
-    for I in range(T):
+    for I in (range(T) if query_tiles is None else query_tiles):
         rows = np.arange(I * tile, min(N, (I + 1) * tile))
         vrows = vis_phys(rows) if callable(vis_phys) else vis_phys[rows]
         for J in range(T):

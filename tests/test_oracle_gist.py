@@ -105,6 +105,12 @@ def test_tile_lists_row_callable_matches_dense():
     fn = lambda rows: Gi.visibility(g, 16, 40, rows=perm[rows])[:, perm]
     for a, b in zip(Gi.tile_lists(dense, 128, 32), Gi.tile_lists(fn, 128, 32, N=N)):
         assert np.array_equal(a, b)
+    # the lists of some query tiles are those tiles' rows of the full lists
+    rp, kt, kd = Gi.tile_lists(dense, 128, 32)
+    rp2, kt2, kd2 = Gi.tile_lists(fn, 128, 32, N=N, query_tiles=[1, 4])
+    want = np.r_[rp[1]:rp[2], rp[4]:rp[5]]
+    assert np.array_equal(kt2, kt[want]) and np.array_equal(kd2, kd[want])
+    assert np.array_equal(np.diff(rp2), [rp[2] - rp[1], rp[5] - rp[4]])
 
 
 @pytest.mark.parametrize("N,sinks,window", [(2000, 128, 128), (1500, 5, 300), (777, 0, 1)])
