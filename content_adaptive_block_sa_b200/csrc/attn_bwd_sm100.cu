@@ -312,6 +312,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
                         itm.bt);
           last_do = gt;
         }
+        if (ok) count_tiles(st, CNT_DKDV_VISITS, vis.n);
         g += vis.n;
       }
       // every copy this CTA started must land before the CTA may exit

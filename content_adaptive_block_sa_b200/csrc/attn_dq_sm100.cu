@@ -191,6 +191,7 @@ __global__ void __launch_bounds__(kThreads, 1) dq_tc_kernel(const __grid_constan
           }
           last_kv = gt;
         }
+        if (ok) count_tiles(st, CNT_DQ_VISITS, n);
         g += n;
       }
       // every copy this CTA started must land before the CTA may exit

@@ -334,6 +334,21 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_kernel(const __grid_consta
             if (ok) ok = load(false, it);
           }
         }
+#ifdef SA_COUNT_TILES
+        if (ok) {
+          count_tiles(st, CNT_FWD_VISITS, wl.n);
+          if (m.pair) {
+            const uint32_t pq = (uint32_t)m.pair_q[list_of(m, itm.bt, itm.h) * m.P + itm.I];
+            const int qa = pq & 0xffff, qb = (pq >> 16) == 0xffff ? -1 : (int)(pq >> 16);
+            int blocks = 0;
+            for (int it = 0; it < wl.n; ++it) blocks += __popc(((uint32_t)m.visits[wl.e0 + it] >> 24) & 0xfu);
+            count_tiles(st, CNT_PAIR_BLOCKS, blocks);
+            count_tiles(st, CNT_PAIR_DENSE, (qa + 1) + (qb + 1));
+          } else {
+            count_tiles(st, CNT_FWD_DENSE, itm.I + 1);
+          }
+        }
+#endif
         if (more && m.kind == SA_MASK_GZIP) {
           // the next item's first entries, so that its first K load is not
           // held up by a list lookup

@@ -20,6 +20,32 @@ struct DeviceStatus {
 constexpr size_t kStatusBytes = 256;
 static_assert(sizeof(DeviceStatus) == kStatusBytes, "status header is 256 bytes");
 
+// Tile counters of the instrumented build (compiled with -DSA_COUNT_TILES into
+// a separate library; the product build has none): 64-bit counters in the
+// status header from aux[8] on, cleared with it by every call. Units:
+//  FWD_VISITS   128 x 128 tiles the forward loads and multiplies
+//  FWD_DENSE    tiles of the dense causal lower triangle of the same items
+//               (one per key tile at or below the query tile; not in pair mode)
+//  PAIR_BLOCKS  pair mode: b x b block pairs of the mask among the visits
+//  PAIR_DENSE   pair mode: block pairs of the dense causal triangle of the
+//               items' query blocks
+//  DQ_VISITS    tiles of the query-major dQ pass (every query head)
+//  DKDV_VISITS  tiles of the key-major dK/dV pass (every query head)
+enum {
+  CNT_FWD_VISITS = 0, CNT_FWD_DENSE, CNT_PAIR_BLOCKS, CNT_PAIR_DENSE, CNT_DQ_VISITS,
+  CNT_DKDV_VISITS, kNumTileCounters
+};
+constexpr int kTileCounterWord = 8;  // first aux word (8-byte aligned in the header)
+
+__device__ __forceinline__ void count_tiles(DeviceStatus* st, int which, long long v) {
+#ifdef SA_COUNT_TILES
+  atomicAdd(reinterpret_cast<unsigned long long*>(st->aux + kTileCounterWord) + which,
+            (unsigned long long)v);
+#else
+  (void)st, (void)which, (void)v;
+#endif
+}
+
 // Records the first device-side problem; later ones are dropped.
 __device__ __forceinline__ void report(DeviceStatus* st, int code, int where) {
   if (st != nullptr && atomicCAS(&st->code, 0, code) == 0) st->where = where;
