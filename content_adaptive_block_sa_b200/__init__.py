@@ -356,8 +356,9 @@ def gist_hier_decode(q, gist2_k, gist2_v, gist_k, gist_v, k_cache, v_cache, chun
 
 
 def selftest_wait_timeout(n_ctas: int = 8, device="cuda", stream=None):
-    """Runs the device failure-path self-test (about 4 s); returns (status
-    code, location) read from the status word after the stream synchronises."""
+    """Runs the device failure-path self-test (about 4 s; a test-only export of
+    the library, declared outside the public header); returns (status code,
+    location) read from the status word after the stream synchronises."""
     ws = _workspace(256, device)
     _check(lib().sa_selftest_wait_timeout(_ptr(ws), ws.numel(), n_ctas, _stream(stream)),
            "sa_selftest_wait_timeout")
@@ -366,7 +367,10 @@ def selftest_wait_timeout(n_ctas: int = 8, device="cuda", stream=None):
     return code, where
 
 
-def device_status(ws: torch.Tensor, stream=None) -> int:
+def device_status(ws: torch.Tensor | None, stream=None) -> int:
+    """The device status word of a workspace an earlier call used (None: the
+    fixed scratch array of the allocation-free decode on the current device).
+    Synchronises the stream."""
     st = C.c_int()
     _check(lib().sa_get_device_status(_ptr(ws), _stream(stream), C.byref(st)),
            "sa_get_device_status")

@@ -665,7 +665,7 @@ static void* g_scratch_addr[kMaxDevices];
 // Device address of the array on the current device. In host code the
 // array's name is only a stand-in, so the address is looked up once per
 // device (with that device current) and cached.
-static cudaError_t decode_scratch_address(void** out) {
+cudaError_t decode_scratch_address(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;

@@ -23,13 +23,13 @@ cudaError_t launch_decode(const sa_decode_desc&, const void*, const void*, const
                           const void*, const void*, int32_t*, void*, float*, void*,
                           cudaStream_t);
 size_t decode_workspace_bytes(const sa_decode_desc&);
+cudaError_t decode_scratch_address(void** out);
 cudaError_t launch_hier_decode(const sa_hier_decode_desc&, const void*, const void*, const void*,
                                const void*, const void*, const void*, const void*, int32_t*,
                                int32_t*, void*, float*, void*, cudaStream_t);
 size_t hier_decode_workspace_bytes(const sa_hier_decode_desc&);
 cudaError_t launch_literal_flags_device(const uint8_t*, int, int64_t, int, uint32_t*, uint8_t*,
                                         cudaStream_t);
-cudaError_t launch_wait_timeout_selftest(void*, int, cudaStream_t);
 }  // namespace sa
 
 using namespace sa;
@@ -249,23 +249,18 @@ const char* sa_status_string(sa_status st) {
 }
 
 sa_status sa_get_device_status(const void* ws, sa_stream_t stream, sa_status* out) {
-  SA_CHECK(ws != nullptr && out != nullptr, SA_ERR_INVALID_ARG);
+  SA_CHECK(out != nullptr, SA_ERR_INVALID_ARG);
+  if (ws == nullptr) {  // the allocation-free decode's fixed scratch array
+    void* p = nullptr;
+    if (decode_scratch_address(&p) != cudaSuccess) return SA_ERR_CUDA;
+    ws = p;
+  }
   int32_t code = 0;
   cudaError_t e = cudaMemcpyAsync(&code, ws, sizeof(code), cudaMemcpyDeviceToHost, stream);
   if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
   if (e != cudaSuccess) return SA_ERR_CUDA;
   *out = (sa_status)code;
   return SA_OK;
-}
-
-sa_status sa_selftest_wait_timeout(void* ws, size_t ws_bytes, int32_t n_ctas,
-                                   sa_stream_t stream) {
-  SA_CHECK(n_ctas >= 1 && n_ctas <= 1024, SA_ERR_INVALID_ARG);
-  sa_status st = check_ws(ws, ws_bytes, kStatusBytes);
-  if (st != SA_OK) return st;
-  st = clear_status(ws, (cudaStream_t)stream);
-  if (st != SA_OK) return st;
-  return cuda_status(launch_wait_timeout_selftest(ws, n_ctas, (cudaStream_t)stream));
 }
 
 sa_status sa_literal_flags_from_sizes(const uint32_t* sizes, int32_t num_blocks, uint8_t* flags) {

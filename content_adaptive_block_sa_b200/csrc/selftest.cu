@@ -4,6 +4,7 @@
 // up records SA_ERR_TIMEOUT at location kSelftestWhere in the status word; the
 // others leave on seeing the word. Nothing traps, and the context stays usable.
 #include "sa_common.cuh"
+#include "sa_selftest.h"
 #include "sm100.cuh"
 
 namespace sa {
@@ -23,9 +24,15 @@ __global__ void __launch_bounds__(32) wait_timeout_kernel(DeviceStatus* st) {
     sm100::mbar_wait(&bar, 0, &abort_flag, st, kSelftestWhere);  // nobody arrives
 }
 
-cudaError_t launch_wait_timeout_selftest(void* ws, int n_ctas, cudaStream_t s) {
-  wait_timeout_kernel<<<n_ctas, 32, 0, s>>>(static_cast<DeviceStatus*>(ws));
-  return cudaGetLastError();
-}
-
 }  // namespace sa
+
+extern "C" sa_status sa_selftest_wait_timeout(void* ws, size_t ws_bytes, int32_t n_ctas,
+                                              sa_stream_t stream) {
+  if (n_ctas < 1 || n_ctas > 1024 || ws == nullptr) return SA_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(ws) % 256 != 0) return SA_ERR_INVALID_ARG;
+  if (ws_bytes < sa::kStatusBytes) return SA_ERR_WORKSPACE;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (cudaMemsetAsync(ws, 0, sa::kStatusBytes, s) != cudaSuccess) return SA_ERR_CUDA;
+  sa::wait_timeout_kernel<<<n_ctas, 32, 0, s>>>(static_cast<sa::DeviceStatus*>(ws));
+  return cudaGetLastError() == cudaSuccess ? SA_OK : SA_ERR_CUDA;
+}

@@ -361,17 +361,6 @@ sa_status sa_gist_hier_decode(const sa_hier_decode_desc* desc, const void* q,
                               int32_t* sel_groups, int32_t* sel_chunks, void* o, float* lse,
                               void* ws, size_t ws_bytes, sa_stream_t stream);
 
-/* Self-test of the device failure path (no fault is raised): n_ctas (1..1024)
- * CTAs each wait on an mbarrier that nothing completes, through the same
- * bounded wait every kernel of this library uses, 4 s wall-time limit
- * included. The first to give up records SA_ERR_TIMEOUT and the location code
- * 900 in the workspace's status word (read it with sa_get_device_status after
- * the stream synchronises, about 4 s later); the rest leave on seeing the
- * word. Returns SA_OK once launched; SA_ERR_INVALID_ARG or SA_ERR_WORKSPACE
- * (ws shorter than 256 bytes) before any launch. */
-sa_status sa_selftest_wait_timeout(void* ws, size_t ws_bytes, int32_t n_ctas,
-                                   sa_stream_t stream);
-
 /* ------------------------------------------------------------------ misc */
 
 /* Library version string, e.g. "0.1.0 (sm_100a)". Never NULL. */
@@ -383,7 +372,8 @@ const char* sa_status_string(sa_status st);
 /* Reads the device status word at the start of a workspace used by an
  * earlier call: copies it to *out on `stream` and synchronises that stream
  * (the only call of this library that blocks). SA_OK, SA_ERR_TIMEOUT or
- * SA_ERR_DEVICE. */
+ * SA_ERR_DEVICE. ws == NULL reads the status word of the fixed scratch array
+ * of sa_gist_decode_noalloc on the current device instead. */
 sa_status sa_get_device_status(const void* ws, sa_stream_t stream, sa_status* out);
 
 /* Literal flags from per-block compressed sizes (HOST helper, no CUDA).
@@ -404,6 +394,11 @@ sa_status sa_block_lists_capacity(const sa_mask_desc* desc,
 sa_status sa_build_block_mask_workspace_size(const sa_mask_desc* desc, size_t* bytes);
 
 /* Builds the block and tile lists on the GPU.
+ * Defined by "Gzip-guided sparse attention: Selecting long-range content by
+ * compressibility" (Core equations: M = (M^lit U M^local U I) intersected with
+ * the causal mask, per head class) and "UniGist: Towards General and
+ * Hardware-aligned Sequence-level Long Context Compression" (Approach: sinks,
+ * gists and a local window under one rule; gists shifted to each tile's end).
  *  d_flags  gzip: DEVICE uint8 [batch, B] literal flags (0/1), e.g. from
  *           sa_literal_flags_from_sizes. gist: DEVICE uint8 [N] with 1 for
  *           the LOGICAL positions that are gists, or NULL for the regular
@@ -420,7 +415,11 @@ sa_status sa_build_block_mask(const sa_mask_desc* desc, const uint8_t* d_flags,
 sa_status sa_forward_workspace_size(const sa_attn_desc* attn, const sa_mask_desc* mask,
                                     size_t* bytes);
 
-/* O and LSE of causal attention restricted to the mask. For every query row
+/* O and LSE of causal attention restricted to the mask ("Gzip-guided sparse
+ * attention ...", Core equations: attention sees only the mask's blocks;
+ * Scope: skipping the masked blocks is what turns sparsity into speed;
+ * "UniGist ...", Approach: kernels skip the blocks no query of a tile sees).
+ * For every query row
  * p: s_pq = q_p . k_q * scale over the keys q the mask allows,
  * LSE_p = log sum_q exp(s_pq), O_p = sum_q exp(s_pq - LSE_p) v_q.
  * Only key tiles listed in `lists` are read. Gist mode takes q, k, v, o and
@@ -435,7 +434,9 @@ sa_status sa_forward(const sa_attn_desc* attn, const sa_mask_desc* mask,
 sa_status sa_backward_workspace_size(const sa_attn_desc* attn, const sa_mask_desc* mask,
                                      size_t* bytes);
 
-/* Gradients of the forward for an upstream dO (same layout/strides as o):
+/* Gradients of the forward for an upstream dO ("UniGist ...", Approach:
+ * one-pass training under the same sparse pattern, measured by forward and
+ * backward latency), same layout/strides as o:
  * D_p = sum dO_p * O_p, P = exp(s - LSE), dV = P^T dO, dP = dO V^T,
  * dS = P * (dP - D), dQ = dS K * scale, dK = dS^T Q * scale.
  * o and lse must come from sa_forward with the same inputs.
@@ -456,7 +457,10 @@ sa_status sa_backward(const sa_attn_desc* attn, const sa_mask_desc* mask,
 sa_status sa_gist_decode_workspace_size(const sa_decode_desc* desc, size_t* bytes);
 
 /* One decode step: gist scores -> per-group top-k -> attention over
- * {all gists} U {raw tokens of the selected chunks} U {last `window` tokens}.
+ * {all gists} U {raw tokens of the selected chunks} U {last `window` tokens}
+ * ("Simplified Sparse Attention via Gist Tokens", record: score the query
+ * against the gists only and unfold the selected chunks; "Forget, Then
+ * Recall: ... Gist Sparse Attention", abstract: selective unfolding).
  * Outputs o (bf16), lse (fp32) and the selected chunks. */
 sa_status sa_gist_decode(const sa_decode_desc* desc, const void* q,
                          const void* gist_k, const void* gist_v,
@@ -479,12 +483,16 @@ sa_status sa_gist_decode(const sa_decode_desc* desc, const void* q,
  *    return SA_ERR_WORKSPACE; use sa_gist_decode for them.
  *  - The first call on a device looks up the array's device address (with
  *    that device current) and caches it; make that first call before any
- *    stream capture.
+ *    stream capture. The cached address belongs to the device's context of
+ *    that time: after cudaDeviceReset it is stale, so do not call this entry
+ *    point again in a process that has reset the device.
  *  - Every call on a device shares the one array, which keeps the last call's
  *    contents (its status word is cleared by each call). Calls that overlap on
  *    the GPU - on different streams, or from different host threads without
  *    ordering - race on it; serialise them.
- *  - sa_get_device_status cannot read this array's status word. */
+ *  - A device-side problem (a bounded wait that ran out) sets the status
+ *    word at the start of the array: read it with sa_get_device_status(NULL,
+ *    stream, &st) after the call, with the same device current. */
 sa_status sa_gist_decode_noalloc(const sa_decode_desc* desc, const void* q,
                                  const void* gist_k, const void* gist_v,
                                  const void* k_cache, const void* v_cache,
