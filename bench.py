@@ -113,7 +113,7 @@ KERNEL_SOURCES = {"fwd_tc_kernel": ["attn_fwd_sm100.cu"],
                   "backward": ["attn_bwd_sm100.cu", "attn_dq_sm100.cu"],
                   "decode_tc_kernel": ["decode_sm100.cu"],
                   "hier decode (6 CUDA-core passes)": ["decode.cu"],
-                  "hier_tc_kernel": ["decode_sm100.cu"],
+                  "decode_tc_kernel (gist of gists)": ["decode_sm100.cu"],
                   "deflate_size_kernel + literal_flags_kernel": ["compress.cu"]}
 
 
@@ -486,7 +486,7 @@ class DecodeWorkload:
 
 class HierDecodeWorkload(DecodeWorkload):
     """Gist-of-gist decode: level-2 gists, the kept groups' level-1 gists, the
-    unfolded chunks and the window (six CUDA-core passes)."""
+    unfolded chunks and the window (one tensor-core kernel)."""
 
     def __init__(self, sa, torch, w):
         self.sa, self.torch = sa, torch
@@ -529,8 +529,13 @@ class HierDecodeWorkload(DecodeWorkload):
         rows = n * Hkv * (n2 + w["window"]) + kept + chunks
         self.bytes = float(rows * d * 2 * 2 + 2 * self.q.numel() * 2 + self.lse.numel() * 4
                            + (self.sel.numel() + self.sel2.numel()) * 4)
-        self.kernels_per_step = 6
-        self.kernel = "hier decode (6 CUDA-core passes)"
+        # one tensor-core kernel for these shapes (both selections inside it),
+        # else the six CUDA-core passes
+        c, fo, n2 = w["chunk"], w["fanout"], w["n_gists"] // w["fanout"]
+        tc = (8 <= c <= 128 and 128 % c == 0 and 8 <= fo <= 128 and 128 % fo == 0
+              and 128 <= n2 <= 8192 and L >= 128)
+        self.kernels_per_step = 1 if tc else 6
+        self.kernel = "decode_tc_kernel (gist of gists)" if tc else "hier decode (6 CUDA-core passes)"
         self.unit = "GB/s"
 
     def step(self, ev=None):

@@ -82,11 +82,24 @@ constexpr int kMaskSlots = 8;              // mask ring depth (tiles)
 constexpr uint32_t kMaskSlotBytes = 2048;  // [4 words][128 rows] uint32
 constexpr int kRowCacheWords = 1024;       // gzip: the item's block-row bits
 
+// exponential pairs i with i % 8 >= SA_FWD_POLY_FROM take the FMA-pipe polynomial
+#ifndef SA_FWD_POLY_FROM
+#define SA_FWD_POLY_FROM 5
+#endif
+#ifndef SA_FWD64_QSTAGES
+#define SA_FWD64_QSTAGES 2
+#endif
+static_assert(SA_FWD64_QSTAGES >= 1 && SA_FWD64_QSTAGES <= 4, "Q stages at d = 64: 1..4");
+
 template <int D>
 struct FwdLayout {
   static constexpr int kKStages = D == 64 ? 4 : 3;  // K ring depth
   static constexpr int kVStages = D == 64 ? 4 : 2;  // V ring depth
-  static constexpr int kQStages = D == 64 ? 2 : 1;  // Q tiles (next item's loads early)
+  // Q tiles: d = 64 keeps several, so that an item's Q is requested kQAhead
+  // items before it starts (its stage was last read by the item kQStages
+  // earlier, whose Q K^T is long done by then)
+  static constexpr int kQStages = D == 64 ? SA_FWD64_QSTAGES : 1;
+  static constexpr int kQAhead = kQStages >= 3 ? kQStages - 2 : 0;
   // d = 64: K and V of a tile share a stage and one full / free barrier pair,
   // so the MMA thread waits once per tile for both (every mbarrier wait on
   // that thread leaves the tensor core idle for its latency, as tcgen05.mma
@@ -120,8 +133,8 @@ struct FwdLayout {
 // done; OF the epilogue warps have read O and (max, sum); ML the softmax
 // halves have written (max, sum). DRAIN: all MMAs done before exit.
 enum {
-  B_QF = 0, B_QE = 2, B_KF = 4, B_KE = 8, B_VF = 12, B_VE = 16, B_SF = 20, B_PF = 22,
-  B_OD = 24, B_MF = 26, B_ME = B_MF + kMaskSlots, B_OI = B_ME + kMaskSlots, B_OF = B_OI + 2,
+  B_QF = 0, B_QE = 4, B_KF = 8, B_KE = 12, B_VF = 16, B_VE = 20, B_SF = 24, B_PF = 26,
+  B_OD = 28, B_MF = 30, B_ME = B_MF + kMaskSlots, B_OI = B_ME + kMaskSlots, B_OF = B_OI + 2,
   B_ML = B_OF + 2, B_DRAIN = B_ML + 2, kNumBars
 };
 
@@ -184,7 +197,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_kernel(const __grid_consta
   DeviceStatus* st = a.status;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < QS; ++s) {
       mbar_init(&bar[B_QF + s], 1);
       mbar_init(&bar[B_QE + s], 1);
     }
@@ -241,6 +254,34 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_kernel(const __grid_consta
         const Item f(blockIdx.x, T, a.Hq, a.Bt);
         wl_next.init(m, list_of(m, f.bt, f.h), f.I);
       }
+      // Q of this CTA's item kq (global index iq) into stage kq % QS, whose
+      // last occupant, item kq - QS, must have finished its Q K^T
+      auto load_q = [&](int kq, int iq) -> bool {
+        const Item itq(iq, T, a.Hq, a.Bt);
+        const int qs = kq % QS;
+        if (kq >= QS && !mbar_wait(&bar[B_QE + qs], ((kq / QS) - 1) & 1, abort, st, 1))
+          return false;
+        mbar_arrive_expect_tx(&bar[B_QF + qs], L::kQ);
+        if (m.pair) {
+          // rows 0-63: query block qa, rows 64-127: qb (qa again when there is none)
+          const uint32_t pq = (uint32_t)m.pair_q[list_of(m, itq.bt, itq.h) * m.P + itq.I];
+          const int qa = pq & 0xffff, qb = (pq >> 16) == 0xffff ? qa : (int)(pq >> 16);
+          for (int at = 0; at < D / 64; ++at) {
+            uint8_t* dst = smem + L::q + qs * L::kQ + at * L::kAtom;
+            tma_load_4d(dst, &P.tmq64, &bar[B_QF + qs], at * 64, itq.h, qa * 64, itq.bt);
+            tma_load_4d(dst + 64 * 128, &P.tmq64, &bar[B_QF + qs], at * 64, itq.h, qb * 64, itq.bt);
+          }
+        } else {
+          for (int at = 0; at < D / 64; ++at)
+            tma_load_4d(smem + L::q + qs * L::kQ + at * L::kAtom, &P.tmq, &bar[B_QF + qs], at * 64,
+                        itq.h, itq.I * kTile, itq.bt);
+        }
+        last_q = kq;
+        return true;
+      };
+      constexpr int QA = L::kQAhead;
+      for (int j = 0; ok && j < QA && blockIdx.x + j * (int)gridDim.x < n_items; ++j)
+        ok = load_q(j, blockIdx.x + j * gridDim.x);
       for (int idx = blockIdx.x; ok && idx < n_items; idx += gridDim.x, ++k) {
         const Item itm(idx, T, a.Hq, a.Bt);
         const WorkList wl = wl_next;
@@ -250,25 +291,11 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_kernel(const __grid_consta
           wl_next.init(m, list_of(m, nx.bt, nx.h), nx.I);
         }
         const int hk = itm.h / (a.Hq / a.Hkv);
-        // Q stage k % QS last held item k - QS, whose last Q K^T has read it
-        const int qs = k % QS;
-        if (k >= QS && !mbar_wait(&bar[B_QE + qs], ((k / QS) - 1) & 1, abort, st, 1)) break;
-        mbar_arrive_expect_tx(&bar[B_QF + qs], L::kQ);
-        if (m.pair) {
-          // rows 0-63: query block qa, rows 64-127: qb (qa again when there is none)
-          const uint32_t pq = (uint32_t)m.pair_q[list_of(m, itm.bt, itm.h) * m.P + itm.I];
-          const int qa = pq & 0xffff, qb = (pq >> 16) == 0xffff ? qa : (int)(pq >> 16);
-          for (int at = 0; at < D / 64; ++at) {
-            uint8_t* dst = smem + L::q + qs * L::kQ + at * L::kAtom;
-            tma_load_4d(dst, &P.tmq64, &bar[B_QF + qs], at * 64, itm.h, qa * 64, itm.bt);
-            tma_load_4d(dst + 64 * 128, &P.tmq64, &bar[B_QF + qs], at * 64, itm.h, qb * 64, itm.bt);
-          }
-        } else {
-          for (int at = 0; at < D / 64; ++at)
-            tma_load_4d(smem + L::q + qs * L::kQ + at * L::kAtom, &P.tmq, &bar[B_QF + qs], at * 64,
-                        itm.h, itm.I * kTile, itm.bt);
+        if (QA == 0) {
+          if (!load_q(k, idx)) break;
+        } else if (idx + QA * (int)gridDim.x < n_items) {
+          if (!load_q(k + QA, idx + QA * gridDim.x)) break;
         }
-        last_q = k;
         // K of tile it + 1 is requested before V of tile it
         auto load = [&](bool is_k, int it) -> bool {
           const int ns = is_k ? KS : VS;
@@ -674,7 +701,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_kernel(const __grid_consta
           for (int i = 0; i < 32; ++i) {
             const float2 e = ffma2(make_float2(x[2 * i], x[2 * i + 1]), sc, nm);
             float2 p;
-            if ((i & 7) >= 5) {
+            if ((i & 7) >= SA_FWD_POLY_FROM) {
               p = exp2_poly2(e);
             } else {
               p.x = ex2(e.x);

@@ -608,10 +608,20 @@ static cudaError_t hier_launch_rep(const DecodeArgs& a, const HierPlan& pl, floa
   return cudaGetLastError();
 }
 
+bool hier_tc_supported(const sa_hier_decode_desc& d);
+cudaError_t launch_hier_decode_tc(const sa_hier_decode_desc& d, const void* q, const void* g2k,
+                                  const void* g2v, const void* gk, const void* gv, const void* kc,
+                                  const void* vc, int32_t* sel2, int32_t* sel1, void* o, float* lse,
+                                  void* ws, cudaStream_t s);
+
+// The tensor-core kernel (one CTA per sequence and KV head, both selections
+// inside it) takes the shapes it supports; the six CUDA-core passes the rest.
 cudaError_t launch_hier_decode(const sa_hier_decode_desc& d, const void* q, const void* g2k,
                                const void* g2v, const void* gk, const void* gv, const void* kc,
                                const void* vc, int32_t* sel2, int32_t* sel1, void* o, float* lse,
                                void* ws, cudaStream_t s) {
+  if (hier_tc_supported(d))
+    return launch_hier_decode_tc(d, q, g2k, g2v, gk, gv, kc, vc, sel2, sel1, o, lse, ws, s);
   const HierPlan pl = hier_plan(d);
   DecodeArgs a{};
   a.q = (const __nv_bfloat16*)q;

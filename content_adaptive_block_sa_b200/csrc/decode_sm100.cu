@@ -52,14 +52,31 @@ namespace dec {
 constexpr int kD = 128;        // head dim
 constexpr int kBlk = 128;      // keys per block
 constexpr int kN = 16;         // MMA N: query-head columns (rep <= 8 used)
-constexpr int kMaxG = 8192;    // gists held in shared memory for the selection
+#ifndef SA_DECODE_VSTAGES
+#define SA_DECODE_VSTAGES 2
+#endif
+// gists held in shared memory for the selection (a third V stage takes half)
+constexpr int kMaxG = SA_DECODE_VSTAGES >= 3 ? 4096 : 8192;
 constexpr int kMaxTopK = 256;
 constexpr int kThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2-5 softmax
+// chunk blocks beyond the selected slots are skipped (the count is fixed by the selection)
+#ifndef SA_DECODE_TRIM
+#define SA_DECODE_TRIM 1
+#endif
+#ifndef SA_DECODE_WAIT_PREV_PV
+#define SA_DECODE_WAIT_PREV_PV 0
+#endif
+#ifndef SA_DECODE_SPLIT_PRODUCER
+#define SA_DECODE_SPLIT_PRODUCER 0
+#endif
+// TMA producer threads: one for both rings, or lane 0 for K and lane 1 for V
+constexpr int kProducerLanes = SA_DECODE_SPLIT_PRODUCER ? 2 : 1;
 
 struct Params {
-  CUtensorMap gk, gv;    // gists, box 128 rows
+  CUtensorMap gk, gv;    // gists (gist of gists: the level-2 gists), box 128 rows
   CUtensorMap ck, cv;    // raw cache, box 128 rows (window)
   CUtensorMap ckc, cvc;  // raw cache, box `chunk` rows (unfolded chunks)
+  CUtensorMap g1k, g1v;  // gist of gists: level-1 gists, box `fanout` rows (kept groups)
   const __nv_bfloat16* q;
   __nv_bfloat16* o;
   float* lse;
@@ -71,14 +88,37 @@ struct Params {
   int n_seq, Hkv, rep, G, cache_len, chunk, top_k, window;
   int n_slots;           // unfolded chunk slots: top_k, or rep * top_k (per-head rule)
   int nG, nW, nC;        // gist, window and chunk blocks
+  // gist of gists: G and nG describe the level-2 gists; the blocks run
+  // [level-2][first nW1 window][nB1 level-1 of the kept groups][other window][chunks]
+  // (flat decode: nW1 = nW, nB1 = 0)
+  int hier, fanout, top_k2, nW1, nB1;
+  int32_t* sel2;         // [n_seq, Hkv, top_k2] kept groups
   float scale;
   int64_t qs[2], os[2];
+};
+
+// Kind and index (within its kind; window blocks 0..nW-1) of block b in
+// stream order.
+enum { BK_GIST = 0, BK_WIN, BK_L1, BK_CHUNK };
+struct BlockOf {
+  int kind, idx;
+  __device__ BlockOf(const Params& P, int b) {
+    if (b < P.nG) { kind = BK_GIST; idx = b; return; }
+    b -= P.nG;
+    if (b < P.nW1) { kind = BK_WIN; idx = b; return; }
+    b -= P.nW1;
+    if (b < P.nB1) { kind = BK_L1; idx = b; return; }
+    b -= P.nB1;
+    if (b < P.nW - P.nW1) { kind = BK_WIN; idx = P.nW1 + b; return; }
+    kind = BK_CHUNK;
+    idx = b - (P.nW - P.nW1);
+  }
 };
 
 // Shared memory (offsets from a 1024-aligned base).
 constexpr uint32_t kAtom = kBlk * 128;          // [128 rows][64 bf16]
 constexpr uint32_t kTileBytes = 2 * kAtom;      // one K or V block, 2 atoms
-constexpr int kKStages = 3, kVStages = 2;
+constexpr int kKStages = 3, kVStages = SA_DECODE_VSTAGES;
 constexpr int kKAhead = 2;                      // K blocks requested ahead of V
 constexpr uint32_t kQtAtom = kN * 128;          // [16 rows][64 bf16]
 constexpr uint32_t OFF_K = 0;
@@ -89,14 +129,17 @@ constexpr uint32_t OFF_SCORE = OFF_PT + 2 * 2 * kQtAtom;  // float [kMaxG]
 constexpr uint32_t OFF_HIST = OFF_SCORE + kMaxG * 4;     // uint32 [256]
 constexpr uint32_t OFF_SEL = OFF_HIST + 256 * 4;         // int32 [kMaxTopK]
 constexpr uint32_t OFF_RED = OFF_SEL + kMaxTopK * 4;     // float [2][4 warps][kN]
-constexpr uint32_t OFF_SCAN = OFF_RED + 2 * 4 * kN * 4;  // uint32 [8] + misc
+constexpr uint32_t OFF_SCAN = OFF_RED + 2 * 4 * kN * 4;  // uint32 [16]: scans, radix, kScanNC
+constexpr int kScanNC = 15;  // scan word: chunk blocks in use after the selection
 constexpr uint32_t OFF_HMASK = OFF_SCAN + 64;            // uint8 [kMaxTopK]: heads per slot
-constexpr uint32_t OFF_BARS = OFF_HMASK + kMaxTopK;
+constexpr uint32_t OFF_SEL2 = OFF_HMASK + kMaxTopK;      // int32 [kMaxTopK]: kept groups
+constexpr uint32_t OFF_BARS = OFF_SEL2 + kMaxTopK * 4;
 constexpr uint32_t kSmemBytes = OFF_BARS + 256 + 1024;
 
 enum {
-  B_KF = 0, B_KE = 3, B_VF = 6, B_VE = 8, B_SF = 10, B_SE = 12, B_PF = 14, B_PD = 16, B_MX = 17,
-  B_GS = 18, B_QR = 19, B_SELD = 20, B_DRAIN = 21, kNumBars = 22
+  B_KF = 0, B_KE = B_KF + kKStages, B_VF = B_KE + kKStages, B_VE = B_VF + kVStages,
+  B_SF = B_VE + kVStages, B_SE = B_SF + 2, B_PF = B_SE + 2, B_PD = B_PF + 2, B_MX = B_PD + 2,
+  B_GS, B_QR, B_SELD, B_DRAIN, B_SEL2, kNumBars
 };
 
 constexpr uint32_t kTmemCols = 64;  // S^T buffers at 0 and 16, O^T at 32
@@ -161,11 +204,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + kNumBars);
   volatile int* abort = reinterpret_cast<volatile int*>(bar + kNumBars) + 1;
   int32_t* sel_s = reinterpret_cast<int32_t*>(smem + OFF_SEL);
+  int32_t* sel2_s = reinterpret_cast<int32_t*>(smem + OFF_SEL2);
   uint8_t* hmask_s = smem + OFF_HMASK;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = blockIdx.x % P.Hkv, seq = blockIdx.x / P.Hkv;
-  const int nb = P.nG + P.nW + P.nC;
+  // blocks: gists, window (and the kept groups' level-1 gists), then at most nC
+  // chunk blocks; the chunk blocks in use (selected slots, rounded up to whole
+  // blocks) are fixed by the selection
+  const int nb = P.nG + P.nW + P.nB1 + P.nC;
   DeviceStatus* st = P.status;
 
   if (threadIdx.x == 0) {
@@ -183,10 +230,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
       mbar_init(&bar[B_PF + s], 128);
     }
     mbar_init(&bar[B_PD], 1);
+    mbar_init(&bar[B_PD + 1], 1);
     mbar_init(&bar[B_MX], 128);
     mbar_init(&bar[B_GS], 128);
     mbar_init(&bar[B_QR], 128);
     mbar_init(&bar[B_SELD], 128);
+    mbar_init(&bar[B_SEL2], 128);
     mbar_init(&bar[B_DRAIN], 1);
     *abort = 0;
     fence_barrier_init();
@@ -201,14 +250,20 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
-    if (lane == 0) {
+    if (lane < kProducerLanes) {
       // ------------------------------------------------------ TMA producer
-      prefetch_tmap(&P.gk);
-      prefetch_tmap(&P.gv);
-      prefetch_tmap(&P.ck);
-      prefetch_tmap(&P.cv);
-      prefetch_tmap(&P.ckc);
-      prefetch_tmap(&P.cvc);
+      if (lane == 0) {
+        prefetch_tmap(&P.gk);
+        prefetch_tmap(&P.gv);
+        prefetch_tmap(&P.ck);
+        prefetch_tmap(&P.cv);
+        prefetch_tmap(&P.ckc);
+        prefetch_tmap(&P.cvc);
+        if (P.hier) {
+          prefetch_tmap(&P.g1k);
+          prefetch_tmap(&P.g1v);
+        }
+      }
       const int ws = P.cache_len - P.window;
       const int cpb = kBlk / P.chunk;  // chunks per block
       int last_k = -1, last_v = -1;
@@ -220,13 +275,26 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
         uint8_t* dst = smem + (is_k ? OFF_K : OFF_V) + s * kTileBytes;
         uint64_t* full = &bar[(is_k ? B_KF : B_VF) + s];
         mbar_arrive_expect_tx(full, kTileBytes);
-        if (b < P.nG + P.nW) {  // a gist block or a window block
-          const bool gist = b < P.nG;
-          const int row0 = gist ? b * kBlk : ws + (b - P.nG) * kBlk;
+        const BlockOf bk(P, b);
+        if (bk.kind == BK_GIST || bk.kind == BK_WIN) {
+          const bool gist = bk.kind == BK_GIST;
+          const int row0 = gist ? bk.idx * kBlk : ws + bk.idx * kBlk;
           const CUtensorMap* map = gist ? (is_k ? &P.gk : &P.gv) : (is_k ? &P.ck : &P.cv);
           for (int at = 0; at < 2; ++at) tma_load_4d(dst + at * kAtom, map, full, at * 64, g, row0, seq);
+        } else if (bk.kind == BK_L1) {
+          // the level-1 gists of 128 / fanout kept groups, one box per group
+          const int gpb = kBlk / P.fanout;
+          const CUtensorMap* map = is_k ? &P.g1k : &P.g1v;
+          for (int i = 0; i < gpb; ++i) {
+            const int slot = bk.idx * gpb + i;
+            // an empty slot loads group 0 (finite values; its keys are masked)
+            const int c = (slot < P.top_k2 && sel2_s[slot] >= 0) ? sel2_s[slot] : 0;
+            const uint32_t roff = (uint32_t)(i * P.fanout) * 128u;
+            for (int at = 0; at < 2; ++at)
+              tma_load_4d(dst + at * kAtom + roff, map, full, at * 64, g, c * P.fanout, seq);
+          }
         } else {
-          const int cb = b - P.nG - P.nW;
+          const int cb = bk.idx;
           const CUtensorMap* map = is_k ? &P.ckc : &P.cvc;
           for (int i = 0; i < cpb; ++i) {
             const int slot = cb * cpb + i;
@@ -244,22 +312,56 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
       // selection: it is prefetched only once the selection is known, and
       // waited for only when it is the K of the current block (by then every
       // earlier V has been requested, so the softmax can reach the selection).
-      bool ok = true, seld = P.nC == 0;
-      int nk = 0;
-      for (int b = 0; ok && b < nb; ++b) {
-        while (ok && nk < nb && nk <= b + kKAhead) {
-          if (nk >= P.nG + P.nW && !seld) {
+#if SA_DECODE_SPLIT_PRODUCER
+      {
+        // lane 0 streams the K blocks, lane 1 the V blocks, each as far ahead as
+        // its ring allows; a level-1 or chunk block waits for its selection
+        const bool is_k = lane == 0;
+        bool ok = true, seld = P.nC == 0, sel2d = P.nB1 == 0;
+        int nbd = nb;
+        for (int b = 0; ok && b < nbd; ++b) {
+          if (!sel2d && BlockOf(P, b).kind == BK_L1) {
+            if (!mbar_wait(&bar[B_SEL2], 0, abort, st, 5)) break;
+            sel2d = true;
+          }
+          if (b >= P.nG + P.nW + P.nB1 && !seld) {
+            if (!mbar_wait(&bar[B_SELD], 0, abort, st, 2)) break;
+            seld = true;
+            if (SA_DECODE_TRIM) nbd = P.nG + P.nW + P.nB1 +
+                  (int)reinterpret_cast<volatile uint32_t*>(smem + OFF_SCAN)[kScanNC];
+            if (b >= nbd) break;
+          }
+          ok = load(is_k, b);
+        }
+      }
+#else
+      bool ok = true, seld = P.nC == 0, sel2d = P.nB1 == 0;
+      int nk = 0, nbd = nb;  // nbd: blocks in use, known once the selection is
+      for (int b = 0; ok && b < nbd; ++b) {
+        while (ok && nk < nbd && nk <= b + kKAhead) {
+          if (!sel2d && BlockOf(P, nk).kind == BK_L1) {  // needs the kept groups
+            if (nk > b) break;
+            if (!mbar_wait(&bar[B_SEL2], 0, abort, st, 5)) {
+              ok = false;
+              break;
+            }
+            sel2d = true;
+          }
+          if (nk >= P.nG + P.nW + P.nB1 && !seld) {
             if (nk > b) break;
             if (!mbar_wait(&bar[B_SELD], 0, abort, st, 2)) {
               ok = false;
               break;
             }
             seld = true;
+            if (SA_DECODE_TRIM) nbd = P.nG + P.nW + P.nB1 + (int)reinterpret_cast<volatile uint32_t*>(smem + OFF_SCAN)[kScanNC];
+            if (nk >= nbd) break;
           }
           ok = load(true, nk++);
         }
-        if (ok) ok = load(false, b);
+        if (ok && b < nbd) ok = load(false, b);
       }
+#endif
       // every copy this CTA started must land before the CTA may exit
       volatile int no_abort = 0;
       for (int s = 0; s < kKStages; ++s)
@@ -279,8 +381,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
       constexpr uint32_t kIdQK = idesc_bf16_f32(kBlk, kN, false, false);
       constexpr uint32_t kIdPV = idesc_bf16_f32(kD, kN, true, false);
       bool ok = mbar_wait(&bar[B_QR], 0, abort, st, 10);
-      for (int b = 0; ok && b <= nb; ++b) {
-        if (b < nb) {
+      int nbd = nb;
+      for (int b = 0; ok && b <= nbd; ++b) {
+        if (SA_DECODE_TRIM && b == P.nG + P.nW + P.nB1 && P.nC > 0) {
+          // the chunk blocks in use are fixed by the selection
+          if (!mbar_wait(&bar[B_SELD], 0, abort, st, 16)) break;
+          if (SA_DECODE_TRIM) nbd = P.nG + P.nW + P.nB1 + (int)reinterpret_cast<volatile uint32_t*>(smem + OFF_SCAN)[kScanNC];
+        }
+        if (b < nbd) {
           const int s = b & 1, sk = b % kKStages;
           if (!mbar_wait(&bar[B_KF + sk], (b / kKStages) & 1, abort, st, 11) ||
               !mbar_wait(&bar[B_SE + s], ((b >> 1) & 1) ^ 1, abort, st, 12))
@@ -312,7 +420,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
             const uint64_t bd = smem_desc_sw128(pb + (kk >> 2) * kQtAtom + (kk & 3) * 32, 16, 1024);
             mma_bf16(tmem + kTmemO, ad, bd, kIdPV, (bp > 0 || kk > 0) ? 1u : 0u);
           }
-          mma_commit(&bar[B_PD]);
+          mma_commit(&bar[B_PD + s]);  // one barrier per P^T buffer
           mma_commit(&bar[B_VE + sv]);
         }
       }
@@ -359,7 +467,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
     }
     const int wstart = P.cache_len - P.window, cpb = kBlk / P.chunk;
     bool ok = true;
-    for (int b = 0; b < nb; ++b) {
+    int nbd = nb;  // fixed by the selection below
+    for (int b = 0; b < nbd; ++b) {
       const int s = b & 1;
       if (!__all_sync(0xffffffffu, mbar_wait(&bar[B_SF + s], (b >> 1) & 1, abort, st, 20))) {
         ok = false;
@@ -374,8 +483,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
       mbar_arrive(&bar[B_SE + s]);
       bool valid;
       uint32_t hv = 0xFFFFFFFFu;  // heads that see this key (unfolded chunks of one head)
-      if (b < P.nG) {
-        const int key = b * kBlk + r;
+      const BlockOf bk(P, b);
+      if (bk.kind == BK_GIST) {
+        const int key = bk.idx * kBlk + r;
         valid = key < P.G;
         if (valid && (P.rule == SA_SELECT_SUM_PROBS_PER_GROUP || P.rule == SA_SELECT_TOP_K_PER_HEAD)) {
           float* lg = P.logits + (int64_t)(seq * P.Hkv + g) * REP * P.G + key;
@@ -387,10 +497,20 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
           for (int h = 0; h < REP; ++h) sum += sv[h];
           scores[key] = sum * P.scale;
         }
-      } else if (b < P.nG + P.nW) {
-        valid = wstart + (b - P.nG) * kBlk + r < P.cache_len;
+      } else if (bk.kind == BK_WIN) {
+        valid = wstart + bk.idx * kBlk + r < P.cache_len;
+      } else if (bk.kind == BK_L1) {
+        // candidate c = 128 idx + r: level-1 gist c % fanout of kept group slot c / fanout
+        const int slot = (bk.idx * kBlk + r) / P.fanout;
+        valid = slot < P.top_k2 && sel2_s[slot] >= 0;
+        if (valid) {
+          float sum = 0.f;
+#pragma unroll
+          for (int h = 0; h < REP; ++h) sum += sv[h];
+          scores[bk.idx * kBlk + r] = sum * P.scale;
+        }
       } else {
-        const int slot = (b - P.nG - P.nW) * cpb + r / P.chunk;
+        const int slot = bk.idx * cpb + r / P.chunk;
         valid = slot < P.n_slots && sel_s[slot] >= 0;
         if (valid && P.rule == SA_SELECT_TOP_K_PER_HEAD) hv = hmask_s[slot];
       }
@@ -423,9 +543,19 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
         m_run[h] = m_use;
         any_resc = any_resc || resc;
       }
-      // P V(b - 1) is done: P^T buffer s (read by P V(b - 2)) is free, O^T is quiet
-      if (b >= 1 &&
-          !__all_sync(0xffffffffu, mbar_wait(&bar[B_PD], (b - 1) & 1, abort, st, 22))) {
+      // P^T buffer s was read by P V(b - 2), whose completion is the next phase
+      // of its barrier (the wait of block b - 2 saw P V(b - 4)); P V(b - 1) may
+      // still run, unless O^T must be rescaled: then O^T must be quiet, and
+      // the other barrier's next phase is P V(b - 1) (completion of a commit
+      // covers every earlier MMA)
+      if (b >= 2 &&
+          !__all_sync(0xffffffffu, mbar_wait(&bar[B_PD + s], ((b - 2) >> 1) & 1, abort, st, 22))) {
+        ok = false;
+        break;
+      }
+      if ((SA_DECODE_WAIT_PREV_PV || any_resc) && b >= 1 &&
+          !__all_sync(0xffffffffu,
+                      mbar_wait(&bar[B_PD + (s ^ 1)], ((b - 1) >> 1) & 1, abort, st, 24))) {
         ok = false;
         break;
       }
@@ -448,13 +578,25 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
       tc_fence_before();
       mbar_arrive(&bar[B_PF + s]);
 
-      if (b == P.nG - 1 && P.top_k > 0) {
+      // selection points: flat decode, the chunks after the gist blocks; gist of
+      // gists, the groups after the level-2 blocks, the chunks after the kept
+      // groups' level-1 blocks
+      const bool sel_groups = P.hier && b == P.nG - 1 && P.top_k2 > 0;
+      const bool sel_chunks = P.top_k > 0 && b == (P.hier ? P.nG + P.nW1 + P.nB1 - 1 : P.nG - 1);
+      if (sel_groups || sel_chunks) {
         // ---------------------------------------------------- top-k select
-        // thread r owns gists [r * per, r * per + per): ascending index order
-        // across threads, so an exclusive scan keeps the output ascending
+        // mode 0: chunks by their gists (flat); 1: groups by their level-2
+        // gists; 2: chunks among the kept groups' level-1 gists (candidate c is
+        // level-1 gist c % fanout of kept group slot c / fanout)
+        const int mode = !P.hier ? 0 : (sel_groups ? 1 : 2);
+        const int sel_n = mode == 2 ? P.nB1 * kBlk : P.G;
+        const int sel_k = mode == 1 ? P.top_k2 : P.top_k;
+        int32_t* sel_dst = mode == 1 ? sel2_s : sel_s;
+        // thread r owns candidates [r * per, r * per + per): ascending index
+        // order across threads, so an exclusive scan keeps the output ascending
         __threadfence_block();
         ok = ok && gs(30);  // every score (or logit) is written
-        const int per = (P.G + 127) / 128, j0 = r * per, j1 = min(P.G, j0 + per);
+        const int per = (sel_n + 127) / 128, j0 = r * per, j1 = min(sel_n, j0 + per);
         // sum or max over the 128 softmax threads (hist serves as scratch)
         auto group_reduce = [&](float v, bool is_max) -> float {
 #pragma unroll
@@ -488,11 +630,25 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
           }
         }
         const int64_t last_ok = (int64_t)P.cache_len - P.window;
+        // a chunk (group) is eligible iff all its raw tokens lie before the
+        // window; a candidate iff its group slot holds a kept group
         auto key_of = [&](int j) -> uint32_t {
-          return ((int64_t)(j + 1) * P.chunk <= last_ok) ? float_key(scores[j]) : 0u;
+          bool e;
+          if (mode == 0) {
+            e = (int64_t)(j + 1) * P.chunk <= last_ok;
+          } else if (mode == 1) {
+            e = (int64_t)(j + 1) * P.fanout * P.chunk <= last_ok;
+          } else {
+            const int sl = j / P.fanout;
+            e = sl < P.top_k2 && sel2_s[sl] >= 0;
+          }
+          return e ? float_key(scores[j]) : 0u;
         };
-        // top_k of scores[] into sel_s (ascending, -1 padded); returns the
-        // number of eligible chunks taken
+        auto value_of = [&](int j) -> int32_t {
+          return mode == 2 ? sel2_s[j / P.fanout] * P.fanout + j % P.fanout : j;
+        };
+        // sel_k of scores[] into sel_dst (ascending, -1 padded); returns the
+        // number of eligible candidates taken
         auto radix_select = [&]() -> uint32_t {
         uint32_t n_elig = 0;
         for (int j = j0; j < j1; ++j) n_elig += key_of(j) != 0u;
@@ -500,9 +656,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
         group_exclusive_scan(n_elig, r, scan, gs, ok, &E);
         // threshold T and the number of keys equal to T to take (lowest indices)
         uint32_t T = 0u, want = 0u;
-        if (E > (uint32_t)P.top_k) {
+        if (E > (uint32_t)sel_k) {
           uint32_t prefix = 0u, pmask = 0u;
-          want = (uint32_t)P.top_k;
+          want = (uint32_t)sel_k;
           for (int pass = 0; pass < 4 && ok; ++pass) {
             const int shift = 24 - 8 * pass;
             hist[r] = 0u;
@@ -563,10 +719,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
         for (int j = j0; j < j1; ++j) {
           const uint32_t k = key_of(j);
           const bool take = k > T || (k == T && k != 0u && eq_seen++ < take_eq);
-          if (take && off < (uint32_t)P.top_k) sel_s[off++] = j;
+          if (take && off < (uint32_t)sel_k) sel_dst[off++] = value_of(j);
         }
-        for (int x = r; x < P.top_k; x += 128)
-          if (x >= (int)sel_total) sel_s[x] = -1;
+        for (int x = r; x < sel_k; x += 128)
+          if (x >= (int)sel_total) sel_dst[x] = -1;
         ok = ok && gs(35);
         return sel_total;
         };
@@ -620,9 +776,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
           for (int x = r; x < P.n_slots; x += 128)
             if (x >= (int)n_union) sel_s[x] = -1;
           ok = ok && gs(47);
+          if (SA_DECODE_TRIM) nbd = P.nG + P.nW + P.nB1 + (min((int)n_union, P.n_slots) + cpb - 1) / cpb;
         } else {
         const uint32_t sel_total = radix_select();
-        const int nsel = min((int)sel_total, P.top_k);
+        const int nsel = min((int)sel_total, sel_k);
+        if (mode != 1 && SA_DECODE_TRIM) nbd = P.nG + P.nW + P.nB1 + (nsel + cpb - 1) / cpb;
         if (P.rule == SA_SELECT_TOP_P_PER_GROUP && nsel > 0) {
           // softmax over the eligible chunks (the best score is among the
           // selected); selected entry x is kept iff the probability of the
@@ -658,18 +816,28 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
           for (int x = r; x < P.top_k; x += 128)
             if (x >= (int)kept) sel_s[x] = -1;
           ok = ok && gs(39);
+          if (SA_DECODE_TRIM) nbd = P.nG + P.nW + P.nB1 + ((int)kept + cpb - 1) / cpb;
         }
-        int32_t* sel_out = P.sel + ((int64_t)seq * P.Hkv + g) * P.top_k;
-        for (int x = r; x < P.top_k; x += 128) sel_out[x] = sel_s[x];
+        int32_t* sel_out = mode == 1 ? P.sel2 + ((int64_t)seq * P.Hkv + g) * P.top_k2
+                                     : P.sel + ((int64_t)seq * P.Hkv + g) * P.top_k;
+        for (int x = r; x < sel_k; x += 128) sel_out[x] = sel_dst[x];
         }
-        mbar_arrive(&bar[B_SELD]);  // release: sel_s is complete
+        if (mode == 1) {
+          mbar_arrive(&bar[B_SEL2]);  // release: sel2_s is complete
+        } else {
+          if (r == 0)
+            reinterpret_cast<volatile uint32_t*>(scan)[kScanNC] = (uint32_t)(nbd - P.nG - P.nW - P.nB1);
+          mbar_arrive(&bar[B_SELD]);  // release: sel_s and the block count are complete
+        }
         if (!__all_sync(0xffffffffu, ok)) break;
       }
     }
     // -------------------------------------------------------------- epilogue
-    if (ok && nb > 0 &&
-        __all_sync(0xffffffffu, mbar_wait(&bar[B_PD], (nb - 1) & 1, abort, st, 23))) {
-      float* lr = red + (nb & 1) * 4 * kN;  // the slot no thread reads any more
+    // the last P V covers every earlier one; its barrier's next phase is it
+    if (ok && nbd > 0 &&
+        __all_sync(0xffffffffu, mbar_wait(&bar[B_PD + ((nbd - 1) & 1)], ((nbd - 1) >> 1) & 1, abort,
+                                          st, 23))) {
+      float* lr = red + (nbd & 1) * 4 * kN;  // the slot no thread reads any more
 #pragma unroll
       for (int h = 0; h < REP; ++h) {
         float v = l_part[h];
@@ -755,9 +923,81 @@ cudaError_t launch_decode_tc(const sa_decode_desc& d, const void* q, const void*
   P.window = d.window;
   P.nG = (d.n_gists + kBlk - 1) / kBlk;
   P.nW = (d.window + kBlk - 1) / kBlk;
+  P.nW1 = P.nW;  // no level-1 blocks: gists, window, chunks
   const int cpb = kBlk / d.chunk;
   P.n_slots = d.select_rule == SA_SELECT_TOP_K_PER_HEAD ? P.rep * d.top_k : d.top_k;
   P.nC = (P.n_slots + cpb - 1) / cpb;
+  P.scale = d.softmax_scale > 0.f ? d.softmax_scale : 1.f / sqrtf((float)d.head_dim);
+  for (int i = 0; i < 2; ++i) {
+    P.qs[i] = d.q_strides[i];
+    P.os[i] = d.o_strides[i];
+  }
+  switch (P.rep) {
+    case 1: return decode_tc_launch<1>(P, s);
+    case 2: return decode_tc_launch<2>(P, s);
+    case 4: return decode_tc_launch<4>(P, s);
+    case 8: return decode_tc_launch<8>(P, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+// ------------------------------------------------- gist of gists, host side
+// Shapes the tensor-core kernel takes for the two-level decode: whole 8-row
+// swizzle groups per chunk and per group of level-1 gists, a full 128-row box
+// of level-2 gists and of cache positions, and the selection buffers' bounds.
+bool hier_tc_supported(const sa_hier_decode_desc& d) {
+  const int rep = d.num_q_heads / d.num_kv_heads;
+  const int n2 = d.fanout > 0 ? d.n_gists / d.fanout : 0;
+  return d.head_dim == kD && d.chunk >= 8 && d.chunk <= kBlk && kBlk % d.chunk == 0 &&
+         d.fanout >= 8 && d.fanout <= kBlk && kBlk % d.fanout == 0 && n2 >= kBlk && n2 <= kMaxG &&
+         d.cache_len >= kBlk && d.top_k <= kMaxTopK && d.top_k2 <= kMaxTopK &&
+         d.top_k2 * d.fanout <= kMaxG && (rep == 1 || rep == 2 || rep == 4 || rep == 8);
+}
+
+cudaError_t launch_hier_decode_tc(const sa_hier_decode_desc& d, const void* q, const void* g2k,
+                                  const void* g2v, const void* gk, const void* gv, const void* kc,
+                                  const void* vc, int32_t* sel2, int32_t* sel1, void* o, float* lse,
+                                  void* ws, cudaStream_t s) {
+  Params P;
+  memset(&P, 0, sizeof(P));
+  const int n2 = d.n_gists / d.fanout;
+  const int64_t g2str[3] = {d.gist2_strides[0], d.gist2_strides[2], d.gist2_strides[1]};
+  const int64_t gstr[3] = {d.gist_strides[0], d.gist_strides[2], d.gist_strides[1]};
+  const int64_t cstr[3] = {d.cache_strides[0], d.cache_strides[2], d.cache_strides[1]};
+  if (!make_tile_map_box(&P.gk, g2k, kD, d.num_kv_heads, n2, d.n_seq, g2str, kBlk) ||
+      !make_tile_map_box(&P.gv, g2v, kD, d.num_kv_heads, n2, d.n_seq, g2str, kBlk) ||
+      !make_tile_map_box(&P.g1k, gk, kD, d.num_kv_heads, d.n_gists, d.n_seq, gstr, d.fanout) ||
+      !make_tile_map_box(&P.g1v, gv, kD, d.num_kv_heads, d.n_gists, d.n_seq, gstr, d.fanout) ||
+      !make_tile_map_box(&P.ck, kc, kD, d.num_kv_heads, d.cache_len, d.n_seq, cstr, kBlk) ||
+      !make_tile_map_box(&P.cv, vc, kD, d.num_kv_heads, d.cache_len, d.n_seq, cstr, kBlk) ||
+      !make_tile_map_box(&P.ckc, kc, kD, d.num_kv_heads, d.cache_len, d.n_seq, cstr, d.chunk) ||
+      !make_tile_map_box(&P.cvc, vc, kD, d.num_kv_heads, d.cache_len, d.n_seq, cstr, d.chunk))
+    return cudaErrorInvalidValue;
+  P.q = static_cast<const __nv_bfloat16*>(q);
+  P.o = static_cast<__nv_bfloat16*>(o);
+  P.lse = lse;
+  P.sel = sel1;
+  P.sel2 = sel2;
+  P.rule = SA_SELECT_SUM_LOGITS_PER_GROUP;
+  P.top_p = 1.f;
+  P.status = static_cast<DeviceStatus*>(ws);
+  P.n_seq = d.n_seq;
+  P.Hkv = d.num_kv_heads;
+  P.rep = d.num_q_heads / d.num_kv_heads;
+  P.G = n2;
+  P.cache_len = d.cache_len;
+  P.chunk = d.chunk;
+  P.top_k = d.top_k;
+  P.window = d.window;
+  P.hier = 1;
+  P.fanout = d.fanout;
+  P.top_k2 = d.top_k2;
+  P.nG = (n2 + kBlk - 1) / kBlk;
+  P.nW = (d.window + kBlk - 1) / kBlk;
+  P.nW1 = (P.nW + 1) / 2;  // half the window loads while the groups are selected
+  P.nB1 = (d.top_k2 * d.fanout + kBlk - 1) / kBlk;
+  P.n_slots = d.top_k;
+  P.nC = (d.top_k + kBlk / d.chunk - 1) / (kBlk / d.chunk);
   P.scale = d.softmax_scale > 0.f ? d.softmax_scale : 1.f / sqrtf((float)d.head_dim);
   for (int i = 0; i < 2; ++i) {
     P.qs[i] = d.q_strides[i];

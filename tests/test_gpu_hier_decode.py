@@ -1,6 +1,9 @@
 """sa_gist_hier_decode (gist of gists) vs the oracle: the kept groups and
 chunks (exact, except across float32-level near ties of the summed logits,
-see the flat decode's tests) and O / LSE over the selected key set."""
+see the flat decode's tests) and O / LSE over the selected key set, on shapes
+of both implementations (the tensor-core kernel takes at least 128 level-2
+gists and groups of 8 to 128 level-1 gists that divide 128; the CUDA-core
+passes the rest)."""
 from concurrent.futures import ThreadPoolExecutor
 
 import numpy as np
@@ -95,6 +98,13 @@ def check(sa, w, seqs=None):
     (16, 96, 4, 4, 0, 32, 16),      # nothing unfolded to raw tokens (GQA 8)
     (16, 96, 4, 0, 6, 32, 2),       # no group kept: nothing to unfold
     (32, 4096, 32, 8, 64, 512, 8),  # the workload's level sizes, two sequences
+    # shapes the tensor-core kernel takes (at least 128 level-2 gists, 8 <= fanout | 128)
+    (16, 2048, 16, 3, 10, 64, 8),     # GQA 4, groups of 16 level-1 gists
+    (8, 1024, 8, 200, 5, 1792, 4),    # 200 groups asked, 100 eligible
+    (16, 2048, 16, 4, 0, 32, 16),     # nothing unfolded to raw tokens (GQA 8)
+    (16, 2048, 16, 0, 6, 32, 2),      # no group kept (one query head per KV head)
+    (32, 4096, 32, 8, 64, 0, 8),      # no window
+    (8, 8192, 64, 5, 20, 300, 8),     # groups of 64 level-1 gists, a ragged window
 ])
 def test_hier_decode_small(sa, chunk, n_gists, fanout, k2, k1, window, heads):
     w = W.scaled("gist_hier_decode_128k", index=700 + n_gists + k2, n_seq=2, cache_len=chunk * n_gists,
