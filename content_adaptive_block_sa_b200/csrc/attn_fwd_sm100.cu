@@ -82,9 +82,17 @@ constexpr int kMaskSlots = 8;              // mask ring depth (tiles)
 constexpr uint32_t kMaskSlotBytes = 2048;  // [4 words][128 rows] uint32
 constexpr int kRowCacheWords = 1024;       // gzip: the item's block-row bits
 
-// exponential pairs i with i % 8 >= SA_FWD_POLY_FROM take the FMA-pipe polynomial
-#ifndef SA_FWD_POLY_FROM
-#define SA_FWD_POLY_FROM 5
+#ifndef SA_FWD_SPLIT_PRODUCER
+#define SA_FWD_SPLIT_PRODUCER 0
+#endif
+// exponential pairs i with i % 8 >= the threshold take the FMA-pipe polynomial,
+// the rest the exp unit: d = 64 is bound by the exp unit's 16 results per clock
+// and SM, d = 128 is not (measured fastest with no polynomial at all)
+#ifndef SA_FWD64_POLY_FROM
+#define SA_FWD64_POLY_FROM 5
+#endif
+#ifndef SA_FWD128_POLY_FROM
+#define SA_FWD128_POLY_FROM 8
 #endif
 #ifndef SA_FWD64_QSTAGES
 #define SA_FWD64_QSTAGES 2
@@ -237,15 +245,21 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_kernel(const __grid_consta
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  // separate K and V rings (d = 128): lane 0 issues Q and K, lane 1 V, so that a
+  // K load never waits behind a V slot (and the reverse)
+  constexpr bool kSplit = SA_FWD_SPLIT_PRODUCER && !L::kMergedKV;
   if (warp == 0) {
-    if (lane == 0) {
+    if (lane < (kSplit ? 2 : 1)) {
       // ------------------------------------------------------ TMA producer
-      prefetch_tmap(&P.tmq);
-      prefetch_tmap(&P.tmk);
-      prefetch_tmap(&P.tmv);
-      if (m.kind == SA_MASK_GIST) {
-        prefetch_tmap(&P.tmkc);
-        prefetch_tmap(&P.tmvc);
+      const bool do_k = lane == 0;  // Q and K (and V unless split)
+      if (do_k) {
+        prefetch_tmap(&P.tmq);
+        prefetch_tmap(&P.tmk);
+        prefetch_tmap(&P.tmv);
+        if (m.kind == SA_MASK_GIST) {
+          prefetch_tmap(&P.tmkc);
+          prefetch_tmap(&P.tmvc);
+        }
       }
       int g = 0, k = 0, last_k = -1, last_v = -1, last_q = -1;
       bool ok = true;
@@ -280,7 +294,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_kernel(const __grid_consta
         return true;
       };
       constexpr int QA = L::kQAhead;
-      for (int j = 0; ok && j < QA && blockIdx.x + j * (int)gridDim.x < n_items; ++j)
+      for (int j = 0; do_k && ok && j < QA && blockIdx.x + j * (int)gridDim.x < n_items; ++j)
         ok = load_q(j, blockIdx.x + j * gridDim.x);
       for (int idx = blockIdx.x; ok && idx < n_items; idx += gridDim.x, ++k) {
         const Item itm(idx, T, a.Hq, a.Bt);
@@ -291,7 +305,8 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_kernel(const __grid_consta
           wl_next.init(m, list_of(m, nx.bt, nx.h), nx.I);
         }
         const int hk = itm.h / (a.Hq / a.Hkv);
-        if (QA == 0) {
+        if (!do_k) {
+        } else if (QA == 0) {
           if (!load_q(k, idx)) break;
         } else if (idx + QA * (int)gridDim.x < n_items) {
           if (!load_q(k + QA, idx + QA * gridDim.x)) break;
@@ -354,6 +369,8 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_kernel(const __grid_consta
         };
         if (L::kMergedKV) {
           for (int it = 0; ok && it < wl.n; ++it) ok = load_kv(it);
+        } else if (kSplit) {
+          for (int it = 0; ok && it < wl.n; ++it) ok = load(do_k, it);
         } else {
           if (wl.n > 0) ok = load(true, 0);
           for (int it = 0; ok && it < wl.n; ++it) {
@@ -362,7 +379,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_kernel(const __grid_consta
           }
         }
 #ifdef SA_COUNT_TILES
-        if (ok) {
+        if (ok && do_k) {
           count_tiles(st, CNT_FWD_VISITS, wl.n);
           if (m.pair) {
             const uint32_t pq = (uint32_t)m.pair_q[list_of(m, itm.bt, itm.h) * m.P + itm.I];
@@ -376,7 +393,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_kernel(const __grid_consta
           }
         }
 #endif
-        if (more && m.kind == SA_MASK_GZIP) {
+        if (do_k && more && m.kind == SA_MASK_GZIP) {
           // the next item's first entries, so that its first K load is not
           // held up by a list lookup
           if (m.pair) {
@@ -701,7 +718,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_kernel(const __grid_consta
           for (int i = 0; i < 32; ++i) {
             const float2 e = ffma2(make_float2(x[2 * i], x[2 * i + 1]), sc, nm);
             float2 p;
-            if ((i & 7) >= SA_FWD_POLY_FROM) {
+            if ((i & 7) >= (D == 64 ? SA_FWD64_POLY_FROM : SA_FWD128_POLY_FROM)) {
               p = exp2_poly2(e);
             } else {
               p.x = ex2(e.x);

@@ -24,6 +24,13 @@
 // The output O = O^T / l and LSE follow from the single softmax state; no
 // partial results leave the CTA.
 //
+// Gist of gists ("Forget, Then Recall: ...", abstract: recursive gist-of-gist
+// construction with logarithmic per-step cost), the HIER instantiation: the
+// same CTA streams the level-2 gists, selects the top groups after them, then
+// half the window, the kept groups' level-1 gists (one TMA box of `fanout`
+// rows per group), selects the top chunks among those candidates, then the
+// rest of the window and the chunks, all in the one online softmax.
+//
 // Roles (192 threads): warp 0 issues the TMA loads (K blocks into a 3-stage
 // ring, up to two blocks ahead, freed once Q K^T has read them; V blocks into
 // a 2-stage ring, freed after P V) and owns the TMEM allocation; one thread of warp 1 issues
@@ -52,25 +59,9 @@ namespace dec {
 constexpr int kD = 128;        // head dim
 constexpr int kBlk = 128;      // keys per block
 constexpr int kN = 16;         // MMA N: query-head columns (rep <= 8 used)
-#ifndef SA_DECODE_VSTAGES
-#define SA_DECODE_VSTAGES 2
-#endif
-// gists held in shared memory for the selection (a third V stage takes half)
-constexpr int kMaxG = SA_DECODE_VSTAGES >= 3 ? 4096 : 8192;
+constexpr int kMaxG = 8192;    // gists held in shared memory for the selection
 constexpr int kMaxTopK = 256;
 constexpr int kThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2-5 softmax
-// chunk blocks beyond the selected slots are skipped (the count is fixed by the selection)
-#ifndef SA_DECODE_TRIM
-#define SA_DECODE_TRIM 1
-#endif
-#ifndef SA_DECODE_WAIT_PREV_PV
-#define SA_DECODE_WAIT_PREV_PV 0
-#endif
-#ifndef SA_DECODE_SPLIT_PRODUCER
-#define SA_DECODE_SPLIT_PRODUCER 0
-#endif
-// TMA producer threads: one for both rings, or lane 0 for K and lane 1 for V
-constexpr int kProducerLanes = SA_DECODE_SPLIT_PRODUCER ? 2 : 1;
 
 struct Params {
   CUtensorMap gk, gv;    // gists (gist of gists: the level-2 gists), box 128 rows
@@ -90,15 +81,14 @@ struct Params {
   int nG, nW, nC;        // gist, window and chunk blocks
   // gist of gists: G and nG describe the level-2 gists; the blocks run
   // [level-2][first nW1 window][nB1 level-1 of the kept groups][other window][chunks]
-  // (flat decode: nW1 = nW, nB1 = 0)
-  int hier, fanout, top_k2, nW1, nB1;
+  int fanout, top_k2, nW1, nB1;
   int32_t* sel2;         // [n_seq, Hkv, top_k2] kept groups
   float scale;
   int64_t qs[2], os[2];
 };
 
-// Kind and index (within its kind; window blocks 0..nW-1) of block b in
-// stream order.
+// Gist of gists: kind and index (within its kind; window blocks 0..nW-1) of
+// block b in stream order.
 enum { BK_GIST = 0, BK_WIN, BK_L1, BK_CHUNK };
 struct BlockOf {
   int kind, idx;
@@ -118,7 +108,7 @@ struct BlockOf {
 // Shared memory (offsets from a 1024-aligned base).
 constexpr uint32_t kAtom = kBlk * 128;          // [128 rows][64 bf16]
 constexpr uint32_t kTileBytes = 2 * kAtom;      // one K or V block, 2 atoms
-constexpr int kKStages = 3, kVStages = SA_DECODE_VSTAGES;
+constexpr int kKStages = 3, kVStages = 2;
 constexpr int kKAhead = 2;                      // K blocks requested ahead of V
 constexpr uint32_t kQtAtom = kN * 128;          // [16 rows][64 bf16]
 constexpr uint32_t OFF_K = 0;
@@ -129,17 +119,15 @@ constexpr uint32_t OFF_SCORE = OFF_PT + 2 * 2 * kQtAtom;  // float [kMaxG]
 constexpr uint32_t OFF_HIST = OFF_SCORE + kMaxG * 4;     // uint32 [256]
 constexpr uint32_t OFF_SEL = OFF_HIST + 256 * 4;         // int32 [kMaxTopK]
 constexpr uint32_t OFF_RED = OFF_SEL + kMaxTopK * 4;     // float [2][4 warps][kN]
-constexpr uint32_t OFF_SCAN = OFF_RED + 2 * 4 * kN * 4;  // uint32 [16]: scans, radix, kScanNC
-constexpr int kScanNC = 15;  // scan word: chunk blocks in use after the selection
+constexpr uint32_t OFF_SCAN = OFF_RED + 2 * 4 * kN * 4;  // uint32 [8] + misc
 constexpr uint32_t OFF_HMASK = OFF_SCAN + 64;            // uint8 [kMaxTopK]: heads per slot
 constexpr uint32_t OFF_SEL2 = OFF_HMASK + kMaxTopK;      // int32 [kMaxTopK]: kept groups
 constexpr uint32_t OFF_BARS = OFF_SEL2 + kMaxTopK * 4;
 constexpr uint32_t kSmemBytes = OFF_BARS + 256 + 1024;
 
 enum {
-  B_KF = 0, B_KE = B_KF + kKStages, B_VF = B_KE + kKStages, B_VE = B_VF + kVStages,
-  B_SF = B_VE + kVStages, B_SE = B_SF + 2, B_PF = B_SE + 2, B_PD = B_PF + 2, B_MX = B_PD + 2,
-  B_GS, B_QR, B_SELD, B_DRAIN, B_SEL2, kNumBars
+  B_KF = 0, B_KE = 3, B_VF = 6, B_VE = 8, B_SF = 10, B_SE = 12, B_PF = 14, B_PD = 16, B_MX = 17,
+  B_GS = 18, B_QR = 19, B_SELD = 20, B_DRAIN = 21, B_SEL2 = 22, kNumBars = 23
 };
 
 constexpr uint32_t kTmemCols = 64;  // S^T buffers at 0 and 16, O^T at 32
@@ -195,7 +183,7 @@ __device__ __forceinline__ uint32_t group_exclusive_scan(uint32_t v, int t, uint
 
 using namespace dec;
 
-template <int REP>
+template <int REP, bool HIER>
 __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_constant__ Params P) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -209,10 +197,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = blockIdx.x % P.Hkv, seq = blockIdx.x / P.Hkv;
-  // blocks: gists, window (and the kept groups' level-1 gists), then at most nC
-  // chunk blocks; the chunk blocks in use (selected slots, rounded up to whole
-  // blocks) are fixed by the selection
-  const int nb = P.nG + P.nW + P.nB1 + P.nC;
+  const int nb = P.nG + P.nW + (HIER ? P.nB1 : 0) + P.nC;
   DeviceStatus* st = P.status;
 
   if (threadIdx.x == 0) {
@@ -230,7 +215,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
       mbar_init(&bar[B_PF + s], 128);
     }
     mbar_init(&bar[B_PD], 1);
-    mbar_init(&bar[B_PD + 1], 1);
     mbar_init(&bar[B_MX], 128);
     mbar_init(&bar[B_GS], 128);
     mbar_init(&bar[B_QR], 128);
@@ -250,19 +234,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
-    if (lane < kProducerLanes) {
+    if (lane == 0) {
       // ------------------------------------------------------ TMA producer
-      if (lane == 0) {
-        prefetch_tmap(&P.gk);
-        prefetch_tmap(&P.gv);
-        prefetch_tmap(&P.ck);
-        prefetch_tmap(&P.cv);
-        prefetch_tmap(&P.ckc);
-        prefetch_tmap(&P.cvc);
-        if (P.hier) {
-          prefetch_tmap(&P.g1k);
-          prefetch_tmap(&P.g1v);
-        }
+      prefetch_tmap(&P.gk);
+      prefetch_tmap(&P.gv);
+      prefetch_tmap(&P.ck);
+      prefetch_tmap(&P.cv);
+      prefetch_tmap(&P.ckc);
+      prefetch_tmap(&P.cvc);
+      if (HIER) {
+        prefetch_tmap(&P.g1k);
+        prefetch_tmap(&P.g1v);
       }
       const int ws = P.cache_len - P.window;
       const int cpb = kBlk / P.chunk;  // chunks per block
@@ -275,18 +257,26 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
         uint8_t* dst = smem + (is_k ? OFF_K : OFF_V) + s * kTileBytes;
         uint64_t* full = &bar[(is_k ? B_KF : B_VF) + s];
         mbar_arrive_expect_tx(full, kTileBytes);
-        const BlockOf bk(P, b);
-        if (bk.kind == BK_GIST || bk.kind == BK_WIN) {
-          const bool gist = bk.kind == BK_GIST;
-          const int row0 = gist ? bk.idx * kBlk : ws + bk.idx * kBlk;
+        int kind, idx;  // block kind and its index within the kind
+        if constexpr (HIER) {
+          const BlockOf bo(P, b);
+          kind = bo.kind;
+          idx = bo.idx;
+        } else {
+          kind = b < P.nG ? BK_GIST : (b < P.nG + P.nW ? BK_WIN : BK_CHUNK);
+          idx = b < P.nG ? b : (b < P.nG + P.nW ? b - P.nG : b - P.nG - P.nW);
+        }
+        if (kind == BK_GIST || kind == BK_WIN) {  // a gist block or a window block
+          const bool gist = kind == BK_GIST;
+          const int row0 = gist ? idx * kBlk : ws + idx * kBlk;
           const CUtensorMap* map = gist ? (is_k ? &P.gk : &P.gv) : (is_k ? &P.ck : &P.cv);
           for (int at = 0; at < 2; ++at) tma_load_4d(dst + at * kAtom, map, full, at * 64, g, row0, seq);
-        } else if (bk.kind == BK_L1) {
+        } else if (HIER && kind == BK_L1) {
           // the level-1 gists of 128 / fanout kept groups, one box per group
           const int gpb = kBlk / P.fanout;
           const CUtensorMap* map = is_k ? &P.g1k : &P.g1v;
           for (int i = 0; i < gpb; ++i) {
-            const int slot = bk.idx * gpb + i;
+            const int slot = idx * gpb + i;
             // an empty slot loads group 0 (finite values; its keys are masked)
             const int c = (slot < P.top_k2 && sel2_s[slot] >= 0) ? sel2_s[slot] : 0;
             const uint32_t roff = (uint32_t)(i * P.fanout) * 128u;
@@ -294,7 +284,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
               tma_load_4d(dst + at * kAtom + roff, map, full, at * 64, g, c * P.fanout, seq);
           }
         } else {
-          const int cb = bk.idx;
+          const int cb = idx;
           const CUtensorMap* map = is_k ? &P.ckc : &P.cvc;
           for (int i = 0; i < cpb; ++i) {
             const int slot = cb * cpb + i;
@@ -312,34 +302,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
       // selection: it is prefetched only once the selection is known, and
       // waited for only when it is the K of the current block (by then every
       // earlier V has been requested, so the softmax can reach the selection).
-#if SA_DECODE_SPLIT_PRODUCER
-      {
-        // lane 0 streams the K blocks, lane 1 the V blocks, each as far ahead as
-        // its ring allows; a level-1 or chunk block waits for its selection
-        const bool is_k = lane == 0;
-        bool ok = true, seld = P.nC == 0, sel2d = P.nB1 == 0;
-        int nbd = nb;
-        for (int b = 0; ok && b < nbd; ++b) {
-          if (!sel2d && BlockOf(P, b).kind == BK_L1) {
-            if (!mbar_wait(&bar[B_SEL2], 0, abort, st, 5)) break;
-            sel2d = true;
-          }
-          if (b >= P.nG + P.nW + P.nB1 && !seld) {
-            if (!mbar_wait(&bar[B_SELD], 0, abort, st, 2)) break;
-            seld = true;
-            if (SA_DECODE_TRIM) nbd = P.nG + P.nW + P.nB1 +
-                  (int)reinterpret_cast<volatile uint32_t*>(smem + OFF_SCAN)[kScanNC];
-            if (b >= nbd) break;
-          }
-          ok = load(is_k, b);
-        }
-      }
-#else
-      bool ok = true, seld = P.nC == 0, sel2d = P.nB1 == 0;
-      int nk = 0, nbd = nb;  // nbd: blocks in use, known once the selection is
-      for (int b = 0; ok && b < nbd; ++b) {
-        while (ok && nk < nbd && nk <= b + kKAhead) {
-          if (!sel2d && BlockOf(P, nk).kind == BK_L1) {  // needs the kept groups
+      bool ok = true, seld = P.nC == 0, sel2d = !HIER || P.nB1 == 0;
+      int nk = 0;
+      const int chunk0 = P.nG + P.nW + (HIER ? P.nB1 : 0);  // first chunk block
+      for (int b = 0; ok && b < nb; ++b) {
+        while (ok && nk < nb && nk <= b + kKAhead) {
+          if (HIER && !sel2d && BlockOf(P, nk).kind == BK_L1) {  // needs the kept groups
             if (nk > b) break;
             if (!mbar_wait(&bar[B_SEL2], 0, abort, st, 5)) {
               ok = false;
@@ -347,21 +315,18 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
             }
             sel2d = true;
           }
-          if (nk >= P.nG + P.nW + P.nB1 && !seld) {
+          if (nk >= chunk0 && !seld) {
             if (nk > b) break;
             if (!mbar_wait(&bar[B_SELD], 0, abort, st, 2)) {
               ok = false;
               break;
             }
             seld = true;
-            if (SA_DECODE_TRIM) nbd = P.nG + P.nW + P.nB1 + (int)reinterpret_cast<volatile uint32_t*>(smem + OFF_SCAN)[kScanNC];
-            if (nk >= nbd) break;
           }
           ok = load(true, nk++);
         }
-        if (ok && b < nbd) ok = load(false, b);
+        if (ok) ok = load(false, b);
       }
-#endif
       // every copy this CTA started must land before the CTA may exit
       volatile int no_abort = 0;
       for (int s = 0; s < kKStages; ++s)
@@ -381,14 +346,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
       constexpr uint32_t kIdQK = idesc_bf16_f32(kBlk, kN, false, false);
       constexpr uint32_t kIdPV = idesc_bf16_f32(kD, kN, true, false);
       bool ok = mbar_wait(&bar[B_QR], 0, abort, st, 10);
-      int nbd = nb;
-      for (int b = 0; ok && b <= nbd; ++b) {
-        if (SA_DECODE_TRIM && b == P.nG + P.nW + P.nB1 && P.nC > 0) {
-          // the chunk blocks in use are fixed by the selection
-          if (!mbar_wait(&bar[B_SELD], 0, abort, st, 16)) break;
-          if (SA_DECODE_TRIM) nbd = P.nG + P.nW + P.nB1 + (int)reinterpret_cast<volatile uint32_t*>(smem + OFF_SCAN)[kScanNC];
-        }
-        if (b < nbd) {
+      for (int b = 0; ok && b <= nb; ++b) {
+        if (b < nb) {
           const int s = b & 1, sk = b % kKStages;
           if (!mbar_wait(&bar[B_KF + sk], (b / kKStages) & 1, abort, st, 11) ||
               !mbar_wait(&bar[B_SE + s], ((b >> 1) & 1) ^ 1, abort, st, 12))
@@ -420,7 +379,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
             const uint64_t bd = smem_desc_sw128(pb + (kk >> 2) * kQtAtom + (kk & 3) * 32, 16, 1024);
             mma_bf16(tmem + kTmemO, ad, bd, kIdPV, (bp > 0 || kk > 0) ? 1u : 0u);
           }
-          mma_commit(&bar[B_PD + s]);  // one barrier per P^T buffer
+          mma_commit(&bar[B_PD]);
           mma_commit(&bar[B_VE + sv]);
         }
       }
@@ -467,8 +426,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
     }
     const int wstart = P.cache_len - P.window, cpb = kBlk / P.chunk;
     bool ok = true;
-    int nbd = nb;  // fixed by the selection below
-    for (int b = 0; b < nbd; ++b) {
+    for (int b = 0; b < nb; ++b) {
       const int s = b & 1;
       if (!__all_sync(0xffffffffu, mbar_wait(&bar[B_SF + s], (b >> 1) & 1, abort, st, 20))) {
         ok = false;
@@ -483,9 +441,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
       mbar_arrive(&bar[B_SE + s]);
       bool valid;
       uint32_t hv = 0xFFFFFFFFu;  // heads that see this key (unfolded chunks of one head)
-      const BlockOf bk(P, b);
-      if (bk.kind == BK_GIST) {
-        const int key = bk.idx * kBlk + r;
+      int kind, idx;  // block kind and its index within the kind
+      if constexpr (HIER) {
+        const BlockOf bo(P, b);
+        kind = bo.kind;
+        idx = bo.idx;
+      } else {
+        kind = b < P.nG ? BK_GIST : (b < P.nG + P.nW ? BK_WIN : BK_CHUNK);
+        idx = b < P.nG ? b : (b < P.nG + P.nW ? b - P.nG : b - P.nG - P.nW);
+      }
+      if (kind == BK_GIST) {
+        const int key = idx * kBlk + r;
         valid = key < P.G;
         if (valid && (P.rule == SA_SELECT_SUM_PROBS_PER_GROUP || P.rule == SA_SELECT_TOP_K_PER_HEAD)) {
           float* lg = P.logits + (int64_t)(seq * P.Hkv + g) * REP * P.G + key;
@@ -497,20 +463,20 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
           for (int h = 0; h < REP; ++h) sum += sv[h];
           scores[key] = sum * P.scale;
         }
-      } else if (bk.kind == BK_WIN) {
-        valid = wstart + bk.idx * kBlk + r < P.cache_len;
-      } else if (bk.kind == BK_L1) {
+      } else if (kind == BK_WIN) {
+        valid = wstart + idx * kBlk + r < P.cache_len;
+      } else if (HIER && kind == BK_L1) {
         // candidate c = 128 idx + r: level-1 gist c % fanout of kept group slot c / fanout
-        const int slot = (bk.idx * kBlk + r) / P.fanout;
+        const int slot = (idx * kBlk + r) / P.fanout;
         valid = slot < P.top_k2 && sel2_s[slot] >= 0;
         if (valid) {
           float sum = 0.f;
 #pragma unroll
           for (int h = 0; h < REP; ++h) sum += sv[h];
-          scores[bk.idx * kBlk + r] = sum * P.scale;
+          scores[idx * kBlk + r] = sum * P.scale;
         }
       } else {
-        const int slot = bk.idx * cpb + r / P.chunk;
+        const int slot = idx * cpb + r / P.chunk;
         valid = slot < P.n_slots && sel_s[slot] >= 0;
         if (valid && P.rule == SA_SELECT_TOP_K_PER_HEAD) hv = hmask_s[slot];
       }
@@ -543,19 +509,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
         m_run[h] = m_use;
         any_resc = any_resc || resc;
       }
-      // P^T buffer s was read by P V(b - 2), whose completion is the next phase
-      // of its barrier (the wait of block b - 2 saw P V(b - 4)); P V(b - 1) may
-      // still run, unless O^T must be rescaled: then O^T must be quiet, and
-      // the other barrier's next phase is P V(b - 1) (completion of a commit
-      // covers every earlier MMA)
-      if (b >= 2 &&
-          !__all_sync(0xffffffffu, mbar_wait(&bar[B_PD + s], ((b - 2) >> 1) & 1, abort, st, 22))) {
-        ok = false;
-        break;
-      }
-      if ((SA_DECODE_WAIT_PREV_PV || any_resc) && b >= 1 &&
-          !__all_sync(0xffffffffu,
-                      mbar_wait(&bar[B_PD + (s ^ 1)], ((b - 1) >> 1) & 1, abort, st, 24))) {
+      // P V(b - 1) is done: P^T buffer s (read by P V(b - 2)) is free, O^T is quiet
+      if (b >= 1 &&
+          !__all_sync(0xffffffffu, mbar_wait(&bar[B_PD], (b - 1) & 1, abort, st, 22))) {
         ok = false;
         break;
       }
@@ -579,16 +535,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
       mbar_arrive(&bar[B_PF + s]);
 
       // selection points: flat decode, the chunks after the gist blocks; gist of
-      // gists, the groups after the level-2 blocks, the chunks after the kept
-      // groups' level-1 blocks
-      const bool sel_groups = P.hier && b == P.nG - 1 && P.top_k2 > 0;
-      const bool sel_chunks = P.top_k > 0 && b == (P.hier ? P.nG + P.nW1 + P.nB1 - 1 : P.nG - 1);
+      // gists, the groups after the level-2 blocks and the chunks after the
+      // kept groups' level-1 blocks
+      const bool sel_groups = HIER && b == P.nG - 1 && P.top_k2 > 0;
+      const bool sel_chunks = P.top_k > 0 && b == (HIER ? P.nG + P.nW1 + P.nB1 - 1 : P.nG - 1);
       if (sel_groups || sel_chunks) {
         // ---------------------------------------------------- top-k select
         // mode 0: chunks by their gists (flat); 1: groups by their level-2
         // gists; 2: chunks among the kept groups' level-1 gists (candidate c is
         // level-1 gist c % fanout of kept group slot c / fanout)
-        const int mode = !P.hier ? 0 : (sel_groups ? 1 : 2);
+        const int mode = !HIER ? 0 : (sel_groups ? 1 : 2);
         const int sel_n = mode == 2 ? P.nB1 * kBlk : P.G;
         const int sel_k = mode == 1 ? P.top_k2 : P.top_k;
         int32_t* sel_dst = mode == 1 ? sel2_s : sel_s;
@@ -647,8 +603,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
         auto value_of = [&](int j) -> int32_t {
           return mode == 2 ? sel2_s[j / P.fanout] * P.fanout + j % P.fanout : j;
         };
-        // sel_k of scores[] into sel_dst (ascending, -1 padded); returns the
-        // number of eligible candidates taken
+        // top_k of scores[] into sel_s (ascending, -1 padded); returns the
+        // number of eligible chunks taken
         auto radix_select = [&]() -> uint32_t {
         uint32_t n_elig = 0;
         for (int j = j0; j < j1; ++j) n_elig += key_of(j) != 0u;
@@ -776,11 +732,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
           for (int x = r; x < P.n_slots; x += 128)
             if (x >= (int)n_union) sel_s[x] = -1;
           ok = ok && gs(47);
-          if (SA_DECODE_TRIM) nbd = P.nG + P.nW + P.nB1 + (min((int)n_union, P.n_slots) + cpb - 1) / cpb;
         } else {
         const uint32_t sel_total = radix_select();
         const int nsel = min((int)sel_total, sel_k);
-        if (mode != 1 && SA_DECODE_TRIM) nbd = P.nG + P.nW + P.nB1 + (nsel + cpb - 1) / cpb;
         if (P.rule == SA_SELECT_TOP_P_PER_GROUP && nsel > 0) {
           // softmax over the eligible chunks (the best score is among the
           // selected); selected entry x is kept iff the probability of the
@@ -816,28 +770,19 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
           for (int x = r; x < P.top_k; x += 128)
             if (x >= (int)kept) sel_s[x] = -1;
           ok = ok && gs(39);
-          if (SA_DECODE_TRIM) nbd = P.nG + P.nW + P.nB1 + ((int)kept + cpb - 1) / cpb;
         }
         int32_t* sel_out = mode == 1 ? P.sel2 + ((int64_t)seq * P.Hkv + g) * P.top_k2
                                      : P.sel + ((int64_t)seq * P.Hkv + g) * P.top_k;
         for (int x = r; x < sel_k; x += 128) sel_out[x] = sel_dst[x];
         }
-        if (mode == 1) {
-          mbar_arrive(&bar[B_SEL2]);  // release: sel2_s is complete
-        } else {
-          if (r == 0)
-            reinterpret_cast<volatile uint32_t*>(scan)[kScanNC] = (uint32_t)(nbd - P.nG - P.nW - P.nB1);
-          mbar_arrive(&bar[B_SELD]);  // release: sel_s and the block count are complete
-        }
+        mbar_arrive(&bar[mode == 1 ? B_SEL2 : B_SELD]);  // release: the selection is complete
         if (!__all_sync(0xffffffffu, ok)) break;
       }
     }
     // -------------------------------------------------------------- epilogue
-    // the last P V covers every earlier one; its barrier's next phase is it
-    if (ok && nbd > 0 &&
-        __all_sync(0xffffffffu, mbar_wait(&bar[B_PD + ((nbd - 1) & 1)], ((nbd - 1) >> 1) & 1, abort,
-                                          st, 23))) {
-      float* lr = red + (nbd & 1) * 4 * kN;  // the slot no thread reads any more
+    if (ok && nb > 0 &&
+        __all_sync(0xffffffffu, mbar_wait(&bar[B_PD], (nb - 1) & 1, abort, st, 23))) {
+      float* lr = red + (nb & 1) * 4 * kN;  // the slot no thread reads any more
 #pragma unroll
       for (int h = 0; h < REP; ++h) {
         float v = l_part[h];
@@ -882,12 +827,12 @@ bool decode_tc_supported(const sa_decode_desc& d) {
           d.num_q_heads / d.num_kv_heads * d.top_k <= kMaxTopK);
 }
 
-template <int REP>
+template <int REP, bool HIER>
 static cudaError_t decode_tc_launch(const Params& P, cudaStream_t s) {
-  cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel<REP>,
+  cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel<REP, HIER>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
-  decode_tc_kernel<REP><<<dim3(P.n_seq * P.Hkv), kThreads, kSmemBytes, s>>>(P);
+  decode_tc_kernel<REP, HIER><<<dim3(P.n_seq * P.Hkv), kThreads, kSmemBytes, s>>>(P);
   return cudaGetLastError();
 }
 
@@ -923,7 +868,6 @@ cudaError_t launch_decode_tc(const sa_decode_desc& d, const void* q, const void*
   P.window = d.window;
   P.nG = (d.n_gists + kBlk - 1) / kBlk;
   P.nW = (d.window + kBlk - 1) / kBlk;
-  P.nW1 = P.nW;  // no level-1 blocks: gists, window, chunks
   const int cpb = kBlk / d.chunk;
   P.n_slots = d.select_rule == SA_SELECT_TOP_K_PER_HEAD ? P.rep * d.top_k : d.top_k;
   P.nC = (P.n_slots + cpb - 1) / cpb;
@@ -933,10 +877,10 @@ cudaError_t launch_decode_tc(const sa_decode_desc& d, const void* q, const void*
     P.os[i] = d.o_strides[i];
   }
   switch (P.rep) {
-    case 1: return decode_tc_launch<1>(P, s);
-    case 2: return decode_tc_launch<2>(P, s);
-    case 4: return decode_tc_launch<4>(P, s);
-    case 8: return decode_tc_launch<8>(P, s);
+    case 1: return decode_tc_launch<1, false>(P, s);
+    case 2: return decode_tc_launch<2, false>(P, s);
+    case 4: return decode_tc_launch<4, false>(P, s);
+    case 8: return decode_tc_launch<8, false>(P, s);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -989,7 +933,6 @@ cudaError_t launch_hier_decode_tc(const sa_hier_decode_desc& d, const void* q, c
   P.chunk = d.chunk;
   P.top_k = d.top_k;
   P.window = d.window;
-  P.hier = 1;
   P.fanout = d.fanout;
   P.top_k2 = d.top_k2;
   P.nG = (n2 + kBlk - 1) / kBlk;
@@ -1004,10 +947,10 @@ cudaError_t launch_hier_decode_tc(const sa_hier_decode_desc& d, const void* q, c
     P.os[i] = d.o_strides[i];
   }
   switch (P.rep) {
-    case 1: return decode_tc_launch<1>(P, s);
-    case 2: return decode_tc_launch<2>(P, s);
-    case 4: return decode_tc_launch<4>(P, s);
-    case 8: return decode_tc_launch<8>(P, s);
+    case 1: return decode_tc_launch<1, true>(P, s);
+    case 2: return decode_tc_launch<2, true>(P, s);
+    case 4: return decode_tc_launch<4, true>(P, s);
+    case 8: return decode_tc_launch<8, true>(P, s);
     default: return cudaErrorInvalidValue;
   }
 }
