@@ -82,9 +82,6 @@ constexpr int kMaskSlots = 8;              // mask ring depth (tiles)
 constexpr uint32_t kMaskSlotBytes = 2048;  // [4 words][128 rows] uint32
 constexpr int kRowCacheWords = 1024;       // gzip: the item's block-row bits
 
-#ifndef SA_FWD_SPLIT_PRODUCER
-#define SA_FWD_SPLIT_PRODUCER 0
-#endif
 // exponential pairs i with i % 8 >= the threshold take the FMA-pipe polynomial,
 // the rest the exp unit: d = 64 is bound by the exp unit's 16 results per clock
 // and SM, d = 128 is not (measured fastest with no polynomial at all)
@@ -245,21 +242,15 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_kernel(const __grid_consta
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  // separate K and V rings (d = 128): lane 0 issues Q and K, lane 1 V, so that a
-  // K load never waits behind a V slot (and the reverse)
-  constexpr bool kSplit = SA_FWD_SPLIT_PRODUCER && !L::kMergedKV;
   if (warp == 0) {
-    if (lane < (kSplit ? 2 : 1)) {
+    if (lane == 0) {
       // ------------------------------------------------------ TMA producer
-      const bool do_k = lane == 0;  // Q and K (and V unless split)
-      if (do_k) {
-        prefetch_tmap(&P.tmq);
-        prefetch_tmap(&P.tmk);
-        prefetch_tmap(&P.tmv);
-        if (m.kind == SA_MASK_GIST) {
-          prefetch_tmap(&P.tmkc);
-          prefetch_tmap(&P.tmvc);
-        }
+      prefetch_tmap(&P.tmq);
+      prefetch_tmap(&P.tmk);
+      prefetch_tmap(&P.tmv);
+      if (m.kind == SA_MASK_GIST) {
+        prefetch_tmap(&P.tmkc);
+        prefetch_tmap(&P.tmvc);
       }
       int g = 0, k = 0, last_k = -1, last_v = -1, last_q = -1;
       bool ok = true;
@@ -294,7 +285,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_kernel(const __grid_consta
         return true;
       };
       constexpr int QA = L::kQAhead;
-      for (int j = 0; do_k && ok && j < QA && blockIdx.x + j * (int)gridDim.x < n_items; ++j)
+      for (int j = 0; ok && j < QA && blockIdx.x + j * (int)gridDim.x < n_items; ++j)
         ok = load_q(j, blockIdx.x + j * gridDim.x);
       for (int idx = blockIdx.x; ok && idx < n_items; idx += gridDim.x, ++k) {
         const Item itm(idx, T, a.Hq, a.Bt);
@@ -305,8 +296,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_kernel(const __grid_consta
           wl_next.init(m, list_of(m, nx.bt, nx.h), nx.I);
         }
         const int hk = itm.h / (a.Hq / a.Hkv);
-        if (!do_k) {
-        } else if (QA == 0) {
+        if (QA == 0) {
           if (!load_q(k, idx)) break;
         } else if (idx + QA * (int)gridDim.x < n_items) {
           if (!load_q(k + QA, idx + QA * gridDim.x)) break;
@@ -369,8 +359,6 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_kernel(const __grid_consta
         };
         if (L::kMergedKV) {
           for (int it = 0; ok && it < wl.n; ++it) ok = load_kv(it);
-        } else if (kSplit) {
-          for (int it = 0; ok && it < wl.n; ++it) ok = load(do_k, it);
         } else {
           if (wl.n > 0) ok = load(true, 0);
           for (int it = 0; ok && it < wl.n; ++it) {
@@ -379,7 +367,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_kernel(const __grid_consta
           }
         }
 #ifdef SA_COUNT_TILES
-        if (ok && do_k) {
+        if (ok) {
           count_tiles(st, CNT_FWD_VISITS, wl.n);
           if (m.pair) {
             const uint32_t pq = (uint32_t)m.pair_q[list_of(m, itm.bt, itm.h) * m.P + itm.I];
@@ -393,7 +381,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_kernel(const __grid_consta
           }
         }
 #endif
-        if (do_k && more && m.kind == SA_MASK_GZIP) {
+        if (more && m.kind == SA_MASK_GZIP) {
           // the next item's first entries, so that its first K load is not
           // held up by a list lookup
           if (m.pair) {
