@@ -10,9 +10,10 @@
 // (attn_dq_sm100.cu), which recomputes S and dP instead of adding partial dQ
 // tiles into global memory. A work item is one (128-key tile J, KV head,
 // sequence); its visits are every query tile I that lists J, for every query
-// head of the KV group (the transposed tile lists). The kernel is persistent: one CTA per SM walks the
-// items blockIdx.x, blockIdx.x + gridDim.x, ... (early key tiles, which have
-// the longest lists, first). TMEM lanes are key rows:
+// head of the KV group (the transposed tile lists). The kernel is persistent:
+// one CTA per SM takes items from a run-time queue in (sequence, KV head)
+// order, early key tiles (the longest lists) first within a head, so that the
+// CTAs running together read the query tiles of one head through L2. TMEM lanes are key rows:
 //   S^T = K_J Q_I^T (columns 0-127); each half h of the compute warps writes
 //     its bf16 P^T over the first 32 of its 64 S columns
 //   dP^T = V_J dO_I^T (columns 128-255)
@@ -82,8 +83,12 @@ struct Layout {
 // OF: dV and dK of the item read out. DRAIN: all MMAs done.
 enum {
   B_KVF = 0, B_KVE = 1, B_QF = 2, B_QE = 4, B_DOF = 6, B_DOE = 7, B_SF = 8, B_DPF = 9, B_PF1 = 10,
-  B_PF2 = 11, B_OI = 12, B_MF = 14, B_ME = 16, B_OF = 18, B_DRAIN = 21, kNumBars = 22
+  B_PF2 = 11, B_OI = 12, B_MF = 14, B_ME = 16, B_OF = 18, B_DRAIN = 21, B_IQF = 22,
+  B_IQE = B_IQF + kItemRing, kNumBars = B_IQE + kItemRing
 };
+// consumers of each item of the run-time queue: the MMA thread, the mask warp
+// and the eight compute warps
+constexpr int kQueueConsumers = 1 + 1 + kCompute / 32;
 
 constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256;  // dK at 256 + D
 
@@ -104,12 +109,14 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
 struct Item {
   int J, hk, bt, far;
   __device__ Item(int idx, int Hkv, int Bt, int T, bool gist) {
-    const int per = T * Hkv * Bt;
-    far = gist && idx < per;
-    if (gist && !far) idx -= per;
-    J = idx / (Hkv * Bt);
-    hk = (idx % (Hkv * Bt)) % Hkv;
-    bt = (idx % (Hkv * Bt)) / Hkv;
+    // (sequence, KV head) outermost, so that the CTAs running together share the
+    // query tiles of one head through L2; then the far items, then the key tiles
+    const int per = (gist ? 2 : 1) * T;
+    const int hb = idx / per, local = idx % per;
+    hk = hb % Hkv;
+    bt = hb / Hkv;
+    far = gist && local < T;
+    J = far || !gist ? local : local - T;
   }
 };
 
@@ -247,9 +254,15 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
     mbar_init(&bar[B_OF], kCompute);
     mbar_init(&bar[B_OI], 1);
     mbar_init(&bar[B_DRAIN], 1);
+    for (int s = 0; s < kItemRing; ++s) {
+      mbar_init(&bar[B_IQF + s], 1);
+      mbar_init(&bar[B_IQE + s], kQueueConsumers);
+    }
     *abort = 0;
     fence_barrier_init();
   }
+  ItemQueue queue{hdr + 8, &bar[B_IQF], &bar[B_IQE],
+                  reinterpret_cast<unsigned int*>(st->aux + kQueueWordDkdv)};
   if (warp == 0) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
@@ -272,18 +285,27 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
       }
       int g = 0, k = 0, last_q = -1, last_do = -1, last_kv = -1;
       bool ok = true;
-      for (int idx = blockIdx.x; ok && idx < n_items; idx += gridDim.x, ++k) {
+      for (;; ++k) {
+        int idx;
+        if (!queue.publish(k, idx, abort, st, 106) || idx >= n_items) break;
         const Item itm(idx, a.Hkv, a.Bt, T, gist);
         Visits vis;
         vis.init(m, itm, rep, P.near_nt);
         // K and V of the previous item are no longer read
         if (k > 0 && !mbar_wait(&bar[B_KVE], (k - 1) & 1, abort, st, 100)) break;
-        mbar_arrive_expect_tx(&bar[B_KVF], 2 * L::kT);
-        for (int at = 0; at < D / 64; ++at) {
-          tma_load_4d(smem + L::k + at * L::kAtom, itm.far ? &P.tmkc : &P.tmk, &bar[B_KVF], at * 64,
-                      itm.hk, itm.J * kTile, itm.bt);
-          tma_load_4d(smem + L::v + at * L::kAtom, itm.far ? &P.tmvc : &P.tmv, &bar[B_KVF], at * 64,
-                      itm.hk, itm.J * kTile, itm.bt);
+        if (vis.n == 0) {
+          // nothing to load (a far tile no query tile reaches): the phase of
+          // this item completes at once, so that no load of the next item can
+          // fall into it
+          mbar_arrive(&bar[B_KVF]);
+        } else {
+          mbar_arrive_expect_tx(&bar[B_KVF], 2 * L::kT);
+          for (int at = 0; at < D / 64; ++at) {
+            tma_load_4d(smem + L::k + at * L::kAtom, itm.far ? &P.tmkc : &P.tmk, &bar[B_KVF],
+                        at * 64, itm.hk, itm.J * kTile, itm.bt);
+            tma_load_4d(smem + L::v + at * L::kAtom, itm.far ? &P.tmvc : &P.tmv, &bar[B_KVF],
+                        at * 64, itm.hk, itm.J * kTile, itm.bt);
+          }
         }
         last_kv = k;
         for (int it = 0; it < vis.n; ++it) {
@@ -314,6 +336,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
         }
         if (ok) count_tiles(st, CNT_DKDV_VISITS, vis.n);
         g += vis.n;
+        if (!ok) break;
       }
       // every copy this CTA started must land before the CTA may exit
       volatile int no_abort = 0;
@@ -362,13 +385,18 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
         mma_commit(&bar[B_DPF]);
         return true;
       };
-      for (int idx = blockIdx.x; ok && idx < n_items; idx += gridDim.x, ++k) {
+      for (;; ++k) {
+        int idx;
+        if (!queue.take(k, idx, abort, st, 118)) break;
+        queue.release(k);
+        if (idx >= n_items) break;
         const Item itm(idx, a.Hkv, a.Bt, T, gist);
         Visits vis;
         vis.init(m, itm, rep, P.near_nt);
-        if (vis.n > 0 && (!mbar_wait(&bar[B_KVF], k & 1, abort, st, 110) || !issue_s(g) ||
-                          !issue_dp(g)))
-          break;
+        // every item's K/V phase is waited for, empty items included, so that the
+        // phases of the producer and this thread never drift apart
+        if (!mbar_wait(&bar[B_KVF], k & 1, abort, st, 110)) break;
+        if (vis.n > 0 && (!issue_s(g) || !issue_dp(g))) break;
         for (int it = 0; it < vis.n; ++it) {
           const int gt = g + it, s = gt & 1;
           const bool more = it + 1 < vis.n;
@@ -426,7 +454,12 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
     // ------------------------------------------------- visits and their masks
     const int lb = !gist && m.b < kTile ? __ffs(m.b) - 1 : 0;  // b < 128 is a power of two
     int g = 0;
-    for (int idx = blockIdx.x; idx < n_items; idx += gridDim.x) {
+    for (int k = 0;; ++k) {
+      int idx;
+      if (!__all_sync(0xffffffffu, queue.take(k, idx, abort, st, 131))) break;
+      __syncwarp();
+      if (lane == 0) queue.release(k);
+      if (idx >= n_items) break;
       const Item itm(idx, a.Hkv, a.Bt, T, gist);
       Visits vis;
       vis.init(m, itm, rep, P.near_nt);
@@ -513,7 +546,12 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
     const float sl2 = a.scale * 1.4426950408889634f;
     int g = 0, k = 0;
     bool ok = true;
-    for (int idx = blockIdx.x; ok && idx < n_items; idx += gridDim.x, ++k) {
+    for (; ok; ++k) {
+      int idx;
+      if (!__all_sync(0xffffffffu, queue.take(k, idx, abort, st, 125))) break;
+      __syncwarp();
+      if (lane == 0) queue.release(k);
+      if (idx >= n_items) break;
       const Item itm(idx, a.Hkv, a.Bt, T, gist);
       Visits vis;
       vis.init(m, itm, rep, P.near_nt);

@@ -6,7 +6,9 @@
 // (the gradient of the masked softmax attention; "UniGist ...", Approach:
 // one-pass training needs the backward). A work item is one (128-query tile
 // I, head, sequence) and visits the key tiles J of I's tile list, as the
-// forward does. S and dP are recomputed per visit and dQ accumulates in TMEM,
+// forward does, the items taken from a run-time queue in (sequence, KV head)
+// order so that the CTAs running together read one KV head's K/V tiles
+// through L2. S and dP are recomputed per visit and dQ accumulates in TMEM,
 // so every dQ row is written once, with no reductions in global memory; the
 // key-major pass (attn_bwd_sm100.cu) computes dK and dV only.
 //
@@ -76,16 +78,24 @@ struct Layout {
 // both halves have read dQ. DRAIN: all MMAs done.
 enum {
   B_QF = 0, B_QE = 2, B_KVF = 4, B_KVE = 8, B_SF = 12, B_DPF = 14, B_DS = 15, B_MF = 16,
-  B_ME = B_MF + kSlots, B_OI = B_ME + kSlots, B_OF, B_DRAIN, kNumBars
+  B_ME = B_MF + kSlots, B_OI = B_ME + kSlots, B_OF, B_DRAIN, B_IQF,
+  B_IQE = B_IQF + kItemRing, kNumBars = B_IQE + kItemRing
 };
+// consumers of each item of the run-time queue: the MMA thread, the mask warp
+// and the eight compute warps
+constexpr int kQueueConsumers = 1 + 1 + kCompute / 32;
 
 struct Item {
   int I, h, bt;
-  __device__ Item(int idx, int T, int Hq, int Bt) {
-    const int hb = Hq * Bt;
-    I = T - 1 - idx / hb;  // late query tiles (long lists) first
-    h = (idx % hb) % Hq;
-    bt = (idx % hb) / Hq;
+  __device__ Item(int idx, int T, int Hq, int Hkv, int Bt) {
+    // (sequence, KV head) outermost, so that the CTAs running together share the
+    // K/V tiles of one KV head through L2; then late query tiles (long lists)
+    // first, the group's query heads of one tile next to each other
+    const int rep = Hq / Hkv, per = T * rep;
+    const int hb = idx / per, local = idx % per;
+    bt = hb / Hkv;
+    h = (hb % Hkv) * rep + local % rep;
+    I = T - 1 - local / rep;
   }
 };
 
@@ -132,9 +142,15 @@ __global__ void __launch_bounds__(kThreads, 1) dq_tc_kernel(const __grid_constan
     mbar_init(&bar[B_OI], 1);
     mbar_init(&bar[B_OF], kCompute);
     mbar_init(&bar[B_DRAIN], 1);
+    for (int s = 0; s < kItemRing; ++s) {
+      mbar_init(&bar[B_IQF + s], 1);
+      mbar_init(&bar[B_IQE + s], kQueueConsumers);
+    }
     *abort = 0;
     fence_barrier_init();
   }
+  ItemQueue queue{reinterpret_cast<int*>(bar + kNumBars) + 2, &bar[B_IQF], &bar[B_IQE],
+                  reinterpret_cast<unsigned int*>(st->aux + kQueueWordDq)};
   if (warp == 0) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
@@ -157,8 +173,10 @@ __global__ void __launch_bounds__(kThreads, 1) dq_tc_kernel(const __grid_constan
       }
       int g = 0, k = 0, last_q = -1, last_kv = -1;
       bool ok = true;
-      for (int idx = blockIdx.x; ok && idx < n_items; idx += gridDim.x, ++k) {
-        const Item itm(idx, T, a.Hq, a.Bt);
+      for (; ok; ++k) {
+        int idx;
+        if (!queue.publish(k, idx, abort, st, 204) || idx >= n_items) break;
+        const Item itm(idx, T, a.Hq, a.Hkv, a.Bt);
         const int list = list_of(m, itm.bt, itm.h), hk = itm.h / (a.Hq / a.Hkv);
         WorkList wl;
         wl.init(m, list, itm.I);
@@ -239,8 +257,12 @@ __global__ void __launch_bounds__(kThreads, 1) dq_tc_kernel(const __grid_constan
         }
         mma_commit(&bar[B_DPF]);
       };
-      for (int idx = blockIdx.x; ok && idx < n_items; idx += gridDim.x, ++k) {
-        const Item itm(idx, T, a.Hq, a.Bt);
+      for (; ok; ++k) {
+        int idx;
+        if (!queue.take(k, idx, abort, st, 215)) break;
+        queue.release(k);
+        if (idx >= n_items) break;
+        const Item itm(idx, T, a.Hq, a.Hkv, a.Bt);
         WorkList wl;
         wl.init(m, list_of(m, itm.bt, itm.h), itm.I);
         const int n = wl.n;
@@ -294,8 +316,13 @@ __global__ void __launch_bounds__(kThreads, 1) dq_tc_kernel(const __grid_constan
     const int lb = gzip && m.b < kTile ? __ffs(m.b) - 1 : 0;  // b < 128 is a power of two
     uint32_t* rcache = reinterpret_cast<uint32_t*>(smem + L::rows);
     int g = 0;
-    for (int idx = blockIdx.x; idx < n_items; idx += gridDim.x) {
-      const Item itm(idx, T, a.Hq, a.Bt);
+    for (int k = 0;; ++k) {
+      int idx;
+      if (!__all_sync(0xffffffffu, queue.take(k, idx, abort, st, 231))) break;
+      __syncwarp();
+      if (lane == 0) queue.release(k);
+      if (idx >= n_items) break;
+      const Item itm(idx, T, a.Hq, a.Hkv, a.Bt);
       const int list = list_of(m, itm.bt, itm.h);
       WorkList wl;
       wl.init(m, list, itm.I);
@@ -378,8 +405,13 @@ __global__ void __launch_bounds__(kThreads, 1) dq_tc_kernel(const __grid_constan
     const float sl2 = a.scale * 1.4426950408889634f;
     int g = 0, k = 0;
     bool ok = true;
-    for (int idx = blockIdx.x; ok && idx < n_items; idx += gridDim.x, ++k) {
-      const Item itm(idx, T, a.Hq, a.Bt);
+    for (; ok; ++k) {
+      int idx;
+      if (!__all_sync(0xffffffffu, queue.take(k, idx, abort, st, 225))) break;
+      __syncwarp();
+      if (lane == 0) queue.release(k);
+      if (idx >= n_items) break;
+      const Item itm(idx, T, a.Hq, a.Hkv, a.Bt);
       WorkList wl;
       wl.init(m, list_of(m, itm.bt, itm.h), itm.I);
       const int n = wl.n;

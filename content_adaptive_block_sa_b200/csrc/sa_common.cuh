@@ -36,6 +36,8 @@ enum {
   CNT_DKDV_VISITS, kNumTileCounters
 };
 constexpr int kTileCounterWord = 8;  // first aux word (8-byte aligned in the header)
+// item counters of the run-time queues of the backward passes (aux words)
+constexpr int kQueueWordDq = 24, kQueueWordDkdv = 25;
 
 __device__ __forceinline__ void count_tiles(DeviceStatus* st, int which, long long v) {
 #ifdef SA_COUNT_TILES

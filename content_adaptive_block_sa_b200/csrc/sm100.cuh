@@ -351,5 +351,37 @@ __device__ __forceinline__ uint32_t sw128_offset(int row, int col) {
   return (uint32_t)(row * 128 + chunk * 16 + (col & 7) * 2);
 }
 
+// ------------------------------------------------------ run-time item queue
+// Work items handed out at run time in one global order, so that the CTAs
+// running at the same moment work on neighbouring items (those sharing K/V or
+// Q/dO tiles through L2) whatever each item costs. One producer thread takes
+// the next index with an atomic add on a counter (zero at the start of the
+// launch) and publishes it in a ring of kItemRing shared slots; every
+// consumer role reads slot k for its k-th item and releases it. An index >=
+// the number of items ends the CTA (every role sees it).
+constexpr int kItemRing = 4;
+struct ItemQueue {
+  int* slots;            // [kItemRing], shared memory
+  uint64_t* full;        // [kItemRing] mbarriers, count 1
+  uint64_t* empty;       // [kItemRing] mbarriers, count = consumer arrivals per item
+  unsigned int* counter; // global
+  __device__ bool publish(int k, int& idx, volatile int* abort, DeviceStatus* st, int where) {
+    const int s = k % kItemRing;
+    if (k >= kItemRing && !mbar_wait(&empty[s], ((k / kItemRing) - 1) & 1, abort, st, where))
+      return false;
+    idx = (int)atomicAdd(counter, 1u);
+    slots[s] = idx;
+    mbar_arrive(&full[s]);  // release: the slot is visible to the waiters
+    return true;
+  }
+  __device__ bool take(int k, int& idx, volatile int* abort, DeviceStatus* st, int where) {
+    const int s = k % kItemRing;
+    if (!mbar_wait(&full[s], (k / kItemRing) & 1, abort, st, where)) return false;
+    idx = *reinterpret_cast<volatile int*>(&slots[s]);
+    return true;
+  }
+  __device__ void release(int k) { mbar_arrive(&empty[k % kItemRing]); }
+};
+
 }  // namespace sm100
 }  // namespace sa
