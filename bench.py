@@ -153,11 +153,22 @@ def copy_out(tensors):
     return outs
 
 class GzipWorkload:
-    def __init__(self, sa, torch, w, backward):
+    def __init__(self, sa, torch, w, backward, device_flags=False):
         self.sa, self.torch, self.backward = sa, torch, backward
         self.w = w
         Bt, N, H, d, b = w["batch"], w["seq_len"], w["heads"], w["head_dim"], w["block"]
-        if w.get("flags_from") == "bernoulli":
+        # a1 on the device: every step computes the flags from the raw bytes
+        # (sa_literal_flags_device) instead of taking host-made flags
+        self.device_flags = device_flags
+        if device_flags:
+            if w.get("flags_from") == "bernoulli":
+                raise ValueError("this workload draws its flags; it has no bytes to compress")
+            raw = np.stack([np.frombuffer(W.workload_bytes(w, i), np.uint8) for i in range(Bt)])
+            self.h_bytes = torch.from_numpy(raw).pin_memory()
+            self.x = self.h_bytes.cuda()
+            self.sizes = torch.empty(Bt, N // b, dtype=torch.int32, device="cuda")
+            flags = np.zeros((Bt, N // b), np.uint8)
+        elif w.get("flags_from") == "bernoulli":
             flags = W.bernoulli_flags(w)
         else:
             flags = np.stack([sa.literal_flags(W.workload_bytes(w, i), b) for i in range(Bt)])
@@ -198,7 +209,8 @@ class GzipWorkload:
         self.exact = self.exact_fwd * (1 + (2.5 if backward else 0))
         # builder + forward (+ the pairing pre-pass for 64-token blocks) (+ backward:
         # row prep, query-major dQ pass, key-major dK/dV pass)
-        self.kernels_per_step = 2 + (1 if b == 64 else 0) + (3 if backward else 0)
+        self.kernels_per_step = 2 + (1 if b == 64 else 0) + (3 if backward else 0) + \
+            (2 if device_flags else 0)
         self.kernel = "fwd_tc_kernel"
         self.unit = "TFLOP/s"
 
@@ -208,6 +220,8 @@ class GzipWorkload:
 
     def step(self, ev=None):
         sa = self.sa
+        if self.device_flags:
+            sa.literal_flags_device(self.x, self.w["block"], sizes=self.sizes, flags=self.flags)
         sa.sa_build_block_mask(self.md, self.flags, self.lists, self.build_ws)
         if ev is not None:
             ev[0].record()
@@ -224,13 +238,17 @@ class GzipWorkload:
         """Host buffers in, result out: the public API with H2D/D2H copies."""
         for t, h in self.h_in.items():
             getattr(self, t).copy_(h, non_blocking=True)
-        self.flags.copy_(self.h_flags, non_blocking=True)
+        if self.device_flags:
+            self.x.copy_(self.h_bytes, non_blocking=True)
+        else:
+            self.flags.copy_(self.h_flags, non_blocking=True)
         self.step()
         out = [self.o, self.lse] + ([self.dq, self.dk, self.dv] if self.backward else [])
         return copy_out(out)
 
     def io_bytes(self):
-        h2d = sum(x.numel() * x.element_size() for x in self.h_in.values()) + self.h_flags.numel()
+        h2d = sum(x.numel() * x.element_size() for x in self.h_in.values()) + \
+            (self.h_bytes.numel() if self.device_flags else self.h_flags.numel())
         d2h = self.o.numel() * 2 + self.lse.numel() * 4
         if self.backward:
             d2h += 3 * self.dq.numel() * 4
@@ -627,7 +645,8 @@ class FlagsWorkload:
 
 SMALL = {"gzip_8k": dict(batch=8), "gzip_64k_fwdbwd": dict(batch=1, heads=4, kv_heads=4),
          "gist_prefill_32k": dict(heads=8, kv_heads=2), "gist_decode_128k": dict(n_seq=4),
-         "gist_coarse_20k": dict(heads=8, kv_heads=2), "gist_hier_decode_128k": dict(n_seq=4)}
+         "gist_coarse_20k": dict(heads=8, kv_heads=2), "gist_hier_decode_128k": dict(n_seq=4),
+         "gzip_flags_128m": dict(batch=1024)}
 # workloads that run another one's inputs with the backward added
 FWDBWD_OF = {"gist_prefill_32k_fwdbwd": "gist_prefill_32k",
              "gist_coarse_20k_fwdbwd": "gist_coarse_20k"}
@@ -643,12 +662,14 @@ def workload_params(name, rank, size):
     return w
 
 
-def make(sa, torch, name, rank, size="full", select=None):
+def make(sa, torch, name, rank, size="full", select=None, device_flags=False):
     w = workload_params(name, rank, size)
     if select is not None:
         w["select"], w["top_p"] = select, 0.9  # top-p keeps 90% of the probability
     if w["kind"] == "gzip":
-        return GzipWorkload(sa, torch, w, name.endswith("fwdbwd"))
+        return GzipWorkload(sa, torch, w, name.endswith("fwdbwd"), device_flags)
+    if device_flags:
+        raise ValueError("--flags-on-device applies to the gzip workloads")
     if w["kind"] == "gist":
         return GistWorkload(sa, torch, w, name.endswith("fwdbwd"))
     if w["kind"] == "hier":
@@ -749,6 +770,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--select", default=None, choices=list(SELECT_RULES),
                     help="gist_decode_128k: chunk selection rule (default sum_logits; top_p at p = 0.9)")
+    ap.add_argument("--flags-on-device", action="store_true",
+                    help="gzip_64k_fwdbwd: each step computes the literal flags from the raw bytes "
+                         "on the GPU (DEFLATE size estimate) instead of taking host zlib flags")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -770,7 +794,7 @@ def main():
     barrier = lambda: rank_barrier(world)
     max_over_ranks = lambda x: rank_max(x, world, "cuda")
 
-    wl = make(sa, torch, args.workload, rank, args.size, args.select)
+    wl = make(sa, torch, args.workload, rank, args.size, args.select, args.flags_on_device)
     for _ in range(args.warmup):
         wl.step()
     torch.cuda.synchronize()
@@ -849,6 +873,8 @@ def main():
         "dtype": {"fp32": "fp32", "bf16": "bf16"}.get(wl.w.get("dtype"), "u8"),
         "data": "synthetic (seeded generators in sa_workloads)",
         "config": {"workload": args.workload, **({"select": args.select} if args.select else {}),
+                   **({"a1": "literal flags computed on the device each step"}
+                      if args.flags_on_device else {}),
                    "l2": "inputs larger than L2, no flush",
                    "parallelism": f"independent replica per rank x{world}"},
         "roofline": roof, "clocks": clk,

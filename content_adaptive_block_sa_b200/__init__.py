@@ -75,16 +75,23 @@ def literal_flags(x: bytes, b: int) -> np.ndarray:
     return sa_literal_flags_from_sizes(block_compressed_sizes(x, b))
 
 
-def literal_flags_device(x: torch.Tensor, b: int, stream=None):
+def literal_flags_device(x: torch.Tensor, b: int, stream=None, sizes=None, flags=None):
     """Flags from device bytes x (uint8 [batch, n_bytes]) by the library's
-    fixed-Huffman DEFLATE size estimate: (sizes uint32 as int32 [batch, B],
-    flags uint8 [batch, B])."""
+    DEFLATE size estimate (greedy fast-table parse, the smallest of the fixed,
+    dynamic and stored block): (sizes uint32 as int32 [batch, B], flags uint8
+    [batch, B]), written into `sizes`/`flags` when given."""
     if x.dtype != torch.uint8 or x.dim() != 2 or not x.is_contiguous():
         raise ValueError("x must be a contiguous uint8 [batch, n_bytes] tensor")
     batch, n = x.shape
     B = n // b
-    sizes = torch.empty(batch, B, dtype=torch.int32, device=x.device)
-    flags = torch.empty(batch, B, dtype=torch.uint8, device=x.device)
+    if sizes is None:
+        sizes = torch.empty(batch, B, dtype=torch.int32, device=x.device)
+    if flags is None:
+        flags = torch.empty(batch, B, dtype=torch.uint8, device=x.device)
+    for t, dt in ((sizes, torch.int32), (flags, torch.uint8)):
+        if t.dtype != dt or t.shape != (batch, B) or not t.is_contiguous() or t.device != x.device:
+            raise ValueError("sizes/flags must be contiguous [batch, n_bytes // b] int32/uint8 "
+                             "tensors on x's device")
     _check(lib().sa_literal_flags_device(_ptr(x), batch, n, b, _ptr(sizes), _ptr(flags),
                                          _stream(stream)), "sa_literal_flags_device")
     return sizes, flags

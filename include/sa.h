@@ -132,11 +132,15 @@ typedef struct sa_mask_desc {
 /* Literal flags computed on the device from raw bytes: an ESTIMATE of the
  * gzip-based flags ("Gzip-guided sparse attention ...", Core equations: block
  * i is literal iff its compression ratio exceeds the mean). Each block's size
- * c_i comes from a plain DEFLATE encoder of RFC 1951 (one final block with the
- * fixed Huffman codes of section 3.2.6; greedy LZ77 whose candidate at p is
- * the nearest earlier position with the same three bytes; c_i = ceil(bits /
- * 8)), not from zlib, so c_i and the flags can differ from gzip's near the
- * mean. Then flags[i] = c_i * B > sum_j c_j.
+ * c_i comes from a plain DEFLATE encoder of RFC 1951, not from zlib: greedy
+ * LZ77 whose candidate at p is the most recent earlier position with the same
+ * three bytes that the section-4 table holds in its fast form (every position
+ * the parse stops at, and the inside of matches of at most 4 bytes); one
+ * final block of the smallest of the fixed-code (section 3.2.6), dynamic-code
+ * (section 3.2.7) and stored (section 3.2.4) types; c_i = ceil(bits / 8). On
+ * the workloads' bytes the flags equal zlib level 1's, but c_i and the flags
+ * can differ from gzip's elsewhere near the mean. Then flags[i] = c_i * B >
+ * sum_j c_j.
  *  bytes        DEVICE uint8 [batch, n_bytes]
  *  block_bytes  b, 1 <= b <= 1024, n_bytes % b == 0, B = n_bytes / b
  *  sizes        DEVICE uint32 [batch, B] out: c_i

@@ -1,12 +1,14 @@
-"""sa_literal_flags_device vs the oracle's fixed-Huffman DEFLATE sizes:
-every block size and every flag bit-exact, on the workloads' byte
-generators, random and degenerate blocks, and ragged block sizes."""
+"""sa_literal_flags_device vs the oracle's DEFLATE sizes: every block size
+and every flag bit-exact, on the workloads' byte generators, random and
+degenerate blocks, and ragged block sizes; and the device flags against
+zlib level 1's on the workloads' bytes."""
 import numpy as np
 import pytest
 import torch
 
 import sa_workloads as W
 from oracle import deflate_size as F
+from oracle import gzip_mask as G
 
 pytestmark = pytest.mark.gpu
 
@@ -34,6 +36,17 @@ def test_workload_bytes_64k(sa):
 def test_tiny_pattern_bytes(sa):
     w = W.WORKLOADS["gzip_tiny_fp32"]
     check(sa, [W.workload_bytes(w, 0)], w["block"])
+
+
+@pytest.mark.parametrize("name", ["gzip_tiny_fp32", "gzip_64k_fwdbwd"])
+def test_device_flags_equal_zlib_flags(sa, name):
+    # the method's flags come from gzip level 1: on these workloads' bytes
+    # the device estimate gives the same flag on every block
+    w = W.WORKLOADS[name]
+    rows = [W.workload_bytes(w, bt) for bt in range(w["batch"])]
+    _, flags = run(sa, rows, w["block"])
+    for i, r in enumerate(rows):
+        np.testing.assert_array_equal(flags[i], G.literal_flags(r, w["block"]))
 
 
 @pytest.mark.parametrize("b", [1, 3, 16, 100, 128, 1000, 1024])
