@@ -553,6 +553,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
         __threadfence_block();
         ok = ok && gs(30);  // every score (or logit) is written
         const int per = (sel_n + 127) / 128, j0 = r * per, j1 = min(sel_n, j0 + per);
+        // Thread r visits its candidates starting at offset lane % per, so that
+        // at per = 32 the lanes of a warp read 32 different banks of scores[]
+        // (in index order every lane would read the same bank).
+        const int o_first = per > 0 ? lane % per : 0;
+        auto o_next = [&](int o) -> int { return o + 1 == per ? 0 : o + 1; };
         // sum or max over the 128 softmax threads (hist serves as scratch)
         auto group_reduce = [&](float v, bool is_max) -> float {
 #pragma unroll
@@ -577,7 +582,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
             inv_l[h] = l > 0.f ? 1.f / l : 0.f;
           }
           const float* lg = P.logits + (int64_t)(seq * P.Hkv + g) * REP * P.G;
-          for (int j = j0; j < j1; ++j) {
+          for (int t = 0, o = o_first; t < per; ++t, o = o_next(o)) {
+            const int j = j0 + o;
+            if (j >= j1) continue;
             float sum = 0.f;
 #pragma unroll
             for (int h = 0; h < REP; ++h)
@@ -603,9 +610,175 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
         auto value_of = [&](int j) -> int32_t {
           return mode == 2 ? sel2_s[j / P.fanout] * P.fanout + j % P.fanout : j;
         };
+        // top_k through a short list (per <= 32, sel_k <= 128): the thread's
+        // keys are read once into registers, and the threshold comes from
+        // ranking at most 128 listed candidates instead of radix passes, whose
+        // shared-memory histogram serializes on the few bins that similar
+        // scores share. Same result as the radix path; returns false (having
+        // written nothing) when the list would exceed 128 entries, and the
+        // radix path runs instead.
+        auto list_select = [&](uint32_t& total) __attribute__((always_inline)) -> bool {
+          uint32_t kr[32];  // slot t: candidate j0 + o_t, o_t = (o_first + t) mod per
+          uint32_t n_elig = 0u, mx = 0u;
+          {
+            int o = o_first;
+#pragma unroll
+            for (int t = 0; t < 32; ++t) {
+              const uint32_t k = (t < per && j0 + o < j1) ? key_of(j0 + o) : 0u;
+              kr[t] = k;
+              n_elig += k != 0u ? 1u : 0u;
+              mx = max(mx, k);
+              o = o_next(o);
+            }
+          }
+          // T0 <= the sel_k-th largest key: the sel_k-th largest thread
+          // maximum (sel_k threads hold a key >= it). Each warp sorts its 32
+          // maxima (bitonic, descending, in registers) into hist; a maximum's
+          // rank among all 128 is its lane plus a binary search in each other
+          // warp's list (ties: the lower warp first).
+          uint32_t v = mx;
+#pragma unroll
+          for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+            for (int stride = size >> 1; stride > 0; stride >>= 1) {
+              const uint32_t y = __shfl_xor_sync(0xffffffffu, v, stride);
+              const bool lower = (lane & stride) == 0;
+              const bool desc = (lane & size) == 0 || size == 32;
+              v = (lower == desc) ? max(v, y) : min(v, y);
+            }
+          }
+          hist[sw * 32 + lane] = v;
+          // the eligible total in the same exchange
+#pragma unroll
+          for (int off = 16; off > 0; off >>= 1) n_elig += __shfl_xor_sync(0xffffffffu, n_elig, off);
+          if (lane == 0) scan[8 + sw] = n_elig;
+          ok = ok && gs(48);
+          const uint32_t E = scan[8] + scan[9] + scan[10] + scan[11];
+          uint32_t T = 0u, want = 0u;
+          if (E > (uint32_t)sel_k) {
+            // with at most 128 eligible keys every one is on the list
+            uint32_t T0 = 1u;
+            if (E > 128u) {
+              uint32_t rank = (uint32_t)lane;
+#pragma unroll
+              for (int w2 = 0; w2 < 4; ++w2) {
+                if (w2 == sw) continue;
+                const uint32_t* L = hist + w2 * 32;
+                // entries ranked above v (e > v, or e == v in a lower warp): a
+                // prefix of the descending list, found a bit at a time
+                int pos = 0;
+#pragma unroll
+                for (int step = 16; step >= 1; step >>= 1) {
+                  const uint32_t e = L[pos + step - 1];
+                  if (e > v || (e == v && w2 < sw)) pos += step;
+                }
+                if (pos == 31 && (L[31] > v || (L[31] == v && w2 < sw))) pos = 32;
+                rank += (uint32_t)pos;
+              }
+              if (rank == (uint32_t)sel_k - 1u) scan[6] = v;
+              ok = ok && gs(49);
+              T0 = max(scan[6], 1u);
+            }
+            uint32_t nc = 0u;
+#pragma unroll
+            for (int t = 0; t < 32; ++t) nc += kr[t] >= T0 ? 1u : 0u;
+            uint32_t C = 0u;
+            // (its barriers also order the reads of hist above before the writes below)
+            uint32_t pos = group_exclusive_scan(nc, r, scan, gs, ok, &C);
+            if (C > 128u) return false;
+            uint32_t* ckey = hist;        // the list, padded with zero keys to a
+            uint32_t* cidx = hist + 128;  // multiple of 4 entries
+            {
+              int o = o_first;
+#pragma unroll
+              for (int t = 0; t < 32; ++t) {
+                if (kr[t] >= T0) {
+                  ckey[pos] = kr[t];
+                  cidx[pos] = (uint32_t)(j0 + o);
+                  ++pos;
+                }
+                o = o_next(o);
+              }
+            }
+            const int C4 = ((int)C + 3) >> 2;
+            if (r >= (int)C && r < 4 * C4) ckey[r] = 0u;
+            ok = ok && gs(50);
+            // rank by (key descending, index ascending): the entry of rank
+            // sel_k - 1 is the threshold T; want = how many keys equal to T to take
+            if (r < (int)C) {
+              const uint32_t key = ckey[r], idx = cidx[r];
+              const uint4* k4 = reinterpret_cast<const uint4*>(ckey);
+              const uint4* i4 = reinterpret_cast<const uint4*>(cidx);
+              uint32_t rank = 0u, gt = 0u;
+#pragma unroll 4
+              for (int c = 0; c < C4; ++c) {
+                const uint4 kk = k4[c], ii = i4[c];
+                gt += (kk.x > key ? 1u : 0u) + (kk.y > key ? 1u : 0u) + (kk.z > key ? 1u : 0u) +
+                      (kk.w > key ? 1u : 0u);
+                rank += (kk.x == key && ii.x < idx ? 1u : 0u) + (kk.y == key && ii.y < idx ? 1u : 0u) +
+                        (kk.z == key && ii.z < idx ? 1u : 0u) + (kk.w == key && ii.w < idx ? 1u : 0u);
+              }
+              rank += gt;
+              if (rank == (uint32_t)sel_k - 1u) {
+                scan[4] = key;
+                scan[5] = (uint32_t)sel_k - gt;
+              }
+            }
+            ok = ok && gs(51);
+            T = scan[4];
+            want = scan[5];
+          }
+          // take key > T, and the first `want` keys equal to T in index order;
+          // bit o of the masks is candidate j0 + o. One scan of the packed
+          // counts (equal << 16 | greater) gives both prefixes: the threads
+          // before r take min(want, equal keys before r) of the equal keys.
+          uint32_t gtm = 0u, eqm = 0u;
+          {
+            int o = o_first;
+#pragma unroll
+            for (int t = 0; t < 32; ++t) {
+              const uint32_t bit = t < per ? 1u << o : 0u;
+              gtm |= kr[t] > T ? bit : 0u;
+              eqm |= (kr[t] == T && kr[t] != 0u) ? bit : 0u;
+              o = o_next(o);
+            }
+          }
+          const uint32_t n_eq = (uint32_t)__popc(eqm);
+          uint32_t tot = 0u;
+          const uint32_t pre = group_exclusive_scan((n_eq << 16) | (uint32_t)__popc(gtm), r, scan, gs,
+                                                    ok, &tot);
+          const uint32_t eq_before = pre >> 16;
+          const uint32_t take_eq = want > eq_before ? min(n_eq, want - eq_before) : 0u;
+          for (uint32_t u = 0; u < take_eq; ++u) {
+            const uint32_t low = eqm & (0u - eqm);
+            gtm |= low;
+            eqm ^= low;
+          }
+          uint32_t off = (pre & 0xFFFFu) + min(want, eq_before);
+          const uint32_t sel_total = (tot & 0xFFFFu) + min(want, tot >> 16);
+          while (gtm != 0u) {
+            const int o = __ffs(gtm) - 1;
+            gtm &= gtm - 1u;
+            if (off < (uint32_t)sel_k) sel_dst[off++] = value_of(j0 + o);
+          }
+          for (int x = r; x < sel_k; x += 128)
+            if (x >= (int)sel_total) sel_dst[x] = -1;
+          ok = ok && gs(35);
+          total = sel_total;
+          return true;
+        };
         // top_k of scores[] into sel_s (ascending, -1 padded); returns the
         // number of eligible chunks taken
-        auto radix_select = [&]() -> uint32_t {
+        auto radix_select = [&]() __attribute__((always_inline)) -> uint32_t {
+        // (with a few candidates per thread the radix passes are cheaper; the
+        // gist-of-gists selections have 1 or 2, and leave the list path out of
+        // that kernel's register budget)
+        if constexpr (!HIER) {
+          if (per >= 8 && per <= 32 && sel_k <= 128) {
+            uint32_t total = 0u;
+            if (list_select(total)) return total;
+          }
+        }
         uint32_t n_elig = 0;
         for (int j = j0; j < j1; ++j) n_elig += key_of(j) != 0u;
         uint32_t E = 0;
@@ -689,7 +862,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
           const float* lg = P.logits + (int64_t)(seq * P.Hkv + g) * REP * P.G;
           int32_t* hsel = P.sel + (int64_t)(seq * P.Hkv + g) * REP * P.top_k;
           for (int h = 0; h < REP; ++h) {
-            for (int j = j0; j < j1; ++j) scores[j] = lg[(int64_t)h * P.G + j] * P.scale;
+            for (int t = 0, o = o_first; t < per; ++t, o = o_next(o))
+              if (j0 + o < j1) scores[j0 + o] = lg[(int64_t)h * P.G + j0 + o] * P.scale;
             radix_select();
             for (int x = r; x < P.top_k; x += 128) hsel[h * P.top_k + x] = sel_s[x];
             __threadfence_block();
@@ -745,8 +919,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
           for (int x = r; x < nsel; x += 128) smax = fmaxf(smax, scores[sel_s[x]]);
           smax = group_reduce(smax, true);
           float z = 0.f;
-          for (int j = j0; j < j1; ++j)
-            if (key_of(j) != 0u) z += __expf(scores[j] - smax);
+          for (int t = 0, o = o_first; t < per; ++t, o = o_next(o))
+            if (j0 + o < j1 && key_of(j0 + o) != 0u) z += __expf(scores[j0 + o] - smax);
           const float thr = P.top_p * group_reduce(z, false);
           int val[2];
           uint32_t nk = 0u;
