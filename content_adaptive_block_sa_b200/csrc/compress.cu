@@ -26,11 +26,12 @@
 //
 // The warp's steps: a bitonic sort of (three-byte key, position) pairs gives
 // every position its nearest earlier position with the same key and their
-// common prefix; lane 0 walks the parse (the table rule only matters where
-// that nearest position lies inside a long match, and then the walk follows
-// the same-key chain further back); the symbol counts are gathered in
-// parallel; lane 0 runs the two-queue merges; the run-length coding of the
-// code lengths is counted in closed form per run.
+// common prefix; lane 0 walks the parse, a run of positions without such a
+// position in one step (the table rule only matters where the nearest
+// position lies inside a long match, and then the walk follows the same-key
+// chain further back); the symbol counts are gathered in parallel; lane 0
+// runs the two-queue merges; the run-length coding of the code lengths is
+// counted in closed form per run.
 #include "sa_common.cuh"
 
 namespace sa {
@@ -98,17 +99,18 @@ struct DeflateSmem {
   uint32_t* skip;  // [32] bit p: p lies inside a match longer than kMaxInsert
   uint32_t* vis;   // [32] bit p: the parse stops at p
   uint32_t* mat;   // [32] bit p: ... with a match
+  uint32_t* cand;  // [32] bit p: p has an earlier position with its key
   uint32_t* runs;  // [16] run starts of the code-length sequence
   uint32_t* freq;  // [kNumSyms] literal/length, distance, code-length symbol counts
   uint8_t* len;    // [kNumSyms] their code lengths
   uint32_t* hkey;  // [kNumLitLen] used symbols as (count << 9 | symbol), ascending
-  uint32_t* hw;    // [kMaxNodes] node weights (then depths as bytes)
+  uint32_t* hw;    // [kMaxNodes] node weights
   uint16_t* hpar;  // [kMaxNodes] node parents
 };
 
 __host__ __device__ constexpr size_t deflate_warp_smem(int b) {
   return align16(8 * (size_t)pow2_at_least(b)) + 2 * align16(2 * ((size_t)b + 1)) +
-         align16((size_t)b + 1) + 4 * 32 * 3 + 4 * 16 + align16(4 * kNumSyms) +
+         align16((size_t)b + 1) + 4 * 32 * 4 + 4 * 16 + align16(4 * kNumSyms) +
          align16(kNumSyms) + align16(4 * kNumLitLen) + align16(4 * kMaxNodes) +
          align16(2 * kMaxNodes);
 }
@@ -128,9 +130,10 @@ __device__ DeflateSmem deflate_carve(uint8_t* base, int b) {
   m.mlen = reinterpret_cast<uint16_t*>(take(2 * ((size_t)b + 1)));
   m.mdist = reinterpret_cast<uint16_t*>(take(2 * ((size_t)b + 1)));
   m.xs = take((size_t)b + 1);
-  m.skip = reinterpret_cast<uint32_t*>(take(4 * 32 * 3));
+  m.skip = reinterpret_cast<uint32_t*>(take(4 * 32 * 4));
   m.vis = m.skip + 32;
   m.mat = m.skip + 64;
+  m.cand = m.skip + 96;
   m.runs = reinterpret_cast<uint32_t*>(take(4 * 16));
   m.freq = reinterpret_cast<uint32_t*>(take(4 * kNumSyms));
   m.len = take(kNumSyms);
@@ -237,19 +240,30 @@ __device__ void huffman_lengths(const DeflateSmem& S, const uint32_t* freq, int 
   }
   __syncwarp();
   if (lane == 0) {
+    // the fronts of both queues stay in registers; each take loads the next
     uint32_t* w = S.hw;
     for (int i = 0; i < m; ++i) w[i] = S.hkey[i] >> 9;
     int li = 0, ii = m, nn = m;  // next leaf, next merged node to take, next node id
-    auto take = [&]() -> int {
-      if (li < m && (ii >= nn || w[li] <= w[ii])) return li++;
-      return ii++;
-    };
+    uint32_t wl = w[0], wi = 0u;  // their weights (wi valid while ii < nn)
     for (int step = 0; step < m - 1; ++step) {
-      const int a = take();
-      const int c = take();
-      w[nn] = w[a] + w[c];
-      S.hpar[a] = (uint16_t)nn;
-      S.hpar[c] = (uint16_t)nn;
+      int who[2];
+      uint32_t sum = 0u;
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        if (li < m && (ii >= nn || wl <= wi)) {
+          who[u] = li++;
+          sum += wl;
+          wl = w[li];  // (w[m] is the first merged node: read, never used as a leaf)
+        } else {
+          who[u] = ii++;
+          sum += wi;
+          wi = w[ii];
+        }
+      }
+      w[nn] = sum;
+      if (ii == nn) wi = sum;  // the merged queue was empty: the new node is its front
+      S.hpar[who[0]] = (uint16_t)nn;
+      S.hpar[who[1]] = (uint16_t)nn;
       ++nn;
     }
   }
@@ -285,7 +299,7 @@ __global__ void __launch_bounds__(kCompThreads) deflate_size_kernel(const uint8_
   const uint8_t* src = x + (int64_t)bt * n_bytes + (int64_t)blk * b;
   for (int i = lane; i < b; i += 32) S.xs[i] = src[i];
   for (int i = lane; i < kNumSyms; i += 32) S.freq[i] = 0u;
-  S.skip[lane] = 0u;
+  for (int i = lane; i < 128; i += 32) S.skip[i] = 0u;  // skip, vis, mat, cand
   __syncwarp();
   // (three-byte key, position) of every position with three bytes left,
   // padded with the largest value; sorted ascending, an entry whose
@@ -314,6 +328,7 @@ __global__ void __launch_bounds__(kCompThreads) deflate_size_kernel(const uint8_
       __syncwarp();
     }
   }
+  // common prefix with the nearest same-key position (at least its 3 bytes)
   for (int t = 1 + lane; t < np2; t += 32) {
     const uint64_t cur = S.srt[t], prev = S.srt[t - 1];
     if (cur != ~0ull && (cur >> 32) == (prev >> 32)) {
@@ -325,56 +340,60 @@ __global__ void __launch_bounds__(kCompThreads) deflate_size_kernel(const uint8_
     }
   }
   __syncwarp();
-  // the parse (lane 0): the nearest same-key position q is the candidate
-  // unless it lies inside a long match; then the chain of same-key positions
-  // (each one's own nearest) is followed back to an entered one
+  for (int base = 0; base < b; base += 32) {
+    const uint32_t cb = __ballot_sync(0xffffffffu, base + lane < b && S.mlen[base + lane] >= 3);
+    if (lane == 0) S.cand[base >> 5] = cb;
+  }
+  __syncwarp();
+  // the parse (lane 0): a run of positions without a same-key position is a
+  // run of literals; elsewhere the nearest same-key position q is the
+  // candidate unless it lies inside a long match, and then the chain of
+  // same-key positions (each one's own nearest) is followed back to an
+  // entered one
   if (lane == 0) {
-    uint32_t vw = 0u, mw = 0u;  // bits of the current 32-position word
-    int word = 0;
-    auto flush_to = [&](int w) {
-      while (word < w) {
-        S.vis[word] = vw;
-        S.mat[word] = mw;
-        vw = mw = 0u;
-        ++word;
+    auto set_bits = [&](uint32_t* bm, int lo, int hi) {  // bits [lo, hi)
+      for (int i = lo; i < hi;) {
+        const int sh = i & 31, nbit = min(32 - sh, hi - i);
+        bm[i >> 5] |= (nbit == 32 ? 0xffffffffu : ((1u << nbit) - 1u)) << sh;
+        i += nbit;
       }
     };
+    const int nwords = (b + 31) >> 5;
     int p = 0;
     while (p < b) {
+      int w = p >> 5;
+      uint32_t c = S.cand[w] & (0xffffffffu << (p & 31));
+      while (c == 0u && ++w < nwords) c = S.cand[w];
+      const int nx = c ? (w << 5) + __ffs(c) - 1 : b;
+      if (nx > p) {  // literals p .. nx - 1
+        set_bits(S.vis, p, nx);
+        p = nx;
+        continue;
+      }
       int m = S.mlen[p];
-      if (m >= 3) {
-        int q = p - S.mdist[p];
-        if ((S.skip[q >> 5] >> (q & 31)) & 1u) {
-          do {
-            q = S.mlen[q] >= 3 ? q - S.mdist[q] : -1;
-          } while (q >= 0 && ((S.skip[q >> 5] >> (q & 31)) & 1u));
-          if (q < 0) {
-            m = 0;
-          } else {
-            m = 3;
-            while (p + m < b && m < 258 && S.xs[q + m] == S.xs[p + m]) ++m;
-            S.mlen[p] = (uint16_t)m;
-            S.mdist[p] = (uint16_t)(p - q);
-          }
+      int q = p - S.mdist[p];
+      if ((S.skip[q >> 5] >> (q & 31)) & 1u) {
+        do {
+          q = S.mlen[q] >= 3 ? q - S.mdist[q] : -1;
+        } while (q >= 0 && ((S.skip[q >> 5] >> (q & 31)) & 1u));
+        if (q < 0) {
+          m = 0;
+        } else {
+          m = 3;
+          while (p + m < b && m < 258 && S.xs[q + m] == S.xs[p + m]) ++m;
+          S.mlen[p] = (uint16_t)m;
+          S.mdist[p] = (uint16_t)(p - q);
         }
       }
-      flush_to(p >> 5);
-      vw |= 1u << (p & 31);
+      S.vis[p >> 5] |= 1u << (p & 31);
       if (m >= 3) {
-        mw |= 1u << (p & 31);
-        if (m > kMaxInsert) {  // positions p + 1 .. p + m - 1 are not entered
-          for (int i = p + 1; i < p + m;) {
-            const int sh = i & 31, nbit = min(32 - sh, p + m - i);
-            S.skip[i >> 5] |= (nbit == 32 ? 0xffffffffu : ((1u << nbit) - 1u)) << sh;
-            i += nbit;
-          }
-        }
+        S.mat[p >> 5] |= 1u << (p & 31);
+        if (m > kMaxInsert) set_bits(S.skip, p + 1, p + m);  // not entered
         p += m;
       } else {
         p += 1;
       }
     }
-    flush_to((b + 31) >> 5);
   }
   __syncwarp();
   // symbol counts; the fixed code's bits and the extra bits (same in both codes)
