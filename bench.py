@@ -292,6 +292,7 @@ class GistWorkload(GzipWorkload):
     def __init__(self, sa, torch, w, backward=False):
         self.sa, self.torch, self.backward = sa, torch, backward
         self.w = w
+        self.device_flags = False  # the gist layout has no a1 step
         N, H, Hkv, d = w["seq_len"], w["heads"], w["kv_heads"], w["head_dim"]
         self.h_in = {t: torch.from_numpy(W.qkv(w, t, 0)[None]).to(torch.bfloat16).pin_memory()
                      for t in ("q", "k", "v") + (("do",) if backward else ())}
