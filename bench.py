@@ -862,7 +862,9 @@ def main():
         if bwd_ms is not None:
             roof["forward_tflops"] = fwd_ach
             roof["backward_ms"] = bwd_ms
-    roof["traffic"] = recorded_traffic(args.workload if args.size == "full" else "", roof["kernel"])
+    # (the recorded rows are the default selection rule's, at full size)
+    roof["traffic"] = recorded_traffic(args.workload if args.size == "full" and not args.select else "",
+                                       roof["kernel"])
     if rank != 0:
         if world > 1:
             dist.destroy_process_group()
