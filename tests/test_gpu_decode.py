@@ -91,8 +91,15 @@ def valid_alternative(w, rule, top_p, q, gk, s, x, got, want_scores):
     assert prob[shorter].sum() < top_p + 1e-4
 
 
-def check(sa, w, seqs=None, rule=0, top_p=1.0):
+def check(sa, w, seqs=None, rule=0, top_p=1.0, edit=None, exact=()):
+    """edit(q, gk) may change the gist keys in place before the run; `exact`
+    lists (sequence, group) pairs whose selection must equal the oracle's
+    exactly (no near-tie allowance)."""
     q, gk, gv, tq, tgk, tgv, kc, vc = upload_workload(w)
+    if edit is not None:
+        edit(q, gk)
+        tgk.copy_(torch.from_numpy(gk).to(torch.bfloat16))
+        gk = tgk.float().cpu().numpy()  # the oracle sees the same bf16 gists
     sel, o, lse = sa.gist_decode(tq, tgk, tgv, kc, vc, w["chunk"], w["top_k"], w["window"],
                                  select_rule=rule, top_p=top_p)
     torch.cuda.synchronize()
@@ -108,6 +115,8 @@ def check(sa, w, seqs=None, rule=0, top_p=1.0):
                                             w["window"], w["top_k"], rule=rule, top_p=top_p)
         per_head = rule == D.PER_HEAD
         for x in range(w["heads"] if per_head else w["kv_heads"]):
+            if (s, x) in exact:
+                np.testing.assert_array_equal(sel[s, x], osel[x], err_msg=f"seq {s} group {x}")
             if not np.array_equal(sel[s, x], osel[x]):
                 # accept a different set only where float32 rounding can decide it
                 valid_alternative(w, rule, top_p, q, gk, s, x, sel[s, x], scores[x])
@@ -193,3 +202,50 @@ def test_decode_per_head_past_the_union_limit(sa):
 def test_decode_select_rules_full_size(sa, rule):
     r, p = RULES[rule]
     check(sa, W.WORKLOADS["gist_decode_128k"], seqs=[0, 15], rule=r, top_p=p)
+
+
+@pytest.mark.parametrize("top_k,G,chunk", [(64, 1024, 32), (1, 1500, 16), (128, 3000, 32), (129, 2000, 16)])
+def test_decode_list_selection_shapes(sa, top_k, G, chunk):
+    """8 to 32 candidates per thread: the selection ranks a short candidate list
+    (ragged last thread at G = 1500 and 3000; k = 1 and k = 128, the list's
+    limits); k = 129 takes the radix passes."""
+    w = W.scaled("gist_decode_128k", index=700 + top_k + G, n_seq=2, cache_len=chunk * G,
+                 chunk=chunk, n_gists=G, top_k=top_k, window=256, heads=8, kv_heads=2)
+    check(sa, w)
+    if top_k <= 128:
+        check(sa, w, rule=3)  # per head: one list selection per query head
+
+
+def _tie_edit(w, groups, rank, copies, seed):
+    """Copy the gist of the eligible chunk ranked `rank` (sum of logits) into
+    `copies` other eligible chunks of each listed (sequence, group): the
+    selection boundary then falls inside a run of exactly equal scores, which
+    both sides break toward the lower index."""
+    def edit(q, gk):
+        rng = np.random.default_rng(seed)
+        rep = w["heads"] // w["kv_heads"]
+        elig = np.nonzero(D.eligible_chunks(w["n_gists"], w["chunk"], w["cache_len"], w["window"]))[0]
+        for s, g in groups:
+            gb = gk[s, g].astype(np.float32)
+            sc = (q[s, g * rep:(g + 1) * rep].astype(np.float64) @ gb.T.astype(np.float64)).sum(0)
+            order = elig[np.argsort(-sc[elig], kind="stable")]
+            src = order[rank]
+            dst = rng.choice(np.setdiff1d(elig, [src]), copies, replace=False)
+            gk[s, g, dst] = gk[s, g, src]
+    return edit
+
+
+def test_decode_exact_ties_inside_the_list(sa):
+    """k = 64 with 40 copies of the 50th best gist: the list path takes the
+    lowest-index copies that fit, as the oracle does."""
+    w = W.scaled("gist_decode_128k", index=720, n_seq=1)
+    groups = [(0, 0), (0, 5)]
+    check(sa, w, edit=_tie_edit(w, groups, 50, 40, 1), exact=groups)
+
+
+def test_decode_exact_ties_past_the_list(sa):
+    """3000 copies of one gist: more than 128 keys reach the thread-maximum
+    bound, so the radix passes decide, with the same ties to the lower index."""
+    w = W.scaled("gist_decode_128k", index=721, n_seq=1)
+    groups = [(0, 2)]
+    check(sa, w, edit=_tie_edit(w, groups, 10, 3000, 2), exact=groups)
