@@ -146,7 +146,6 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------- workloads
-_host_out = {}
 
 
 # the kernels whose DRAM traffic profiles/traffic.json records, and their sources; the
@@ -184,16 +183,72 @@ def recorded_traffic(workload, kernel):
     return None
 
 
-def copy_out(tensors):
-    """Device -> pinned host copies of a step's results (reused buffers)."""
-    outs = []
-    for t in tensors:
-        key = (t.data_ptr(), t.numel(), t.dtype)
-        if key not in _host_out:
-            _host_out[key] = t.new_empty(t.shape, device="cpu").pin_memory()
-        _host_out[key].copy_(t, non_blocking=True)
-        outs.append(_host_out[key])
-    return outs
+def io_bytes(wl):
+    """Bytes a step copies host -> device and device -> host."""
+    ins, outs = wl.io_tensors()
+    nb = lambda t: t.numel() * t.element_size()
+    return sum(nb(h) for h, _ in ins), sum(nb(o) for o in outs)
+
+
+def e2e_run(wl, torch, steps):
+    """`steps` end-to-end steps through the public API, each copying its inputs
+    from pinned host memory and reading its results back, pipelined on three
+    streams with two staging sets: while step i computes, step i+1's inputs
+    come in and step i-1's results go out (PCIe both ways at once). Inputs land
+    in a staging buffer and are copied on the device into the workload's
+    tensors, results are copied out to a staging buffer before the next step
+    overwrites them. Returns the elapsed ms of all steps (CUDA events)."""
+    ins, outs = wl.io_tensors()
+    cur = torch.cuda.current_stream()
+    sh, sd = torch.cuda.Stream(), torch.cuda.Stream()
+    stg_in = [[d.new_empty(d.shape) for _, d in ins] for _ in range(2)]
+    stg_out = [[o.new_empty(o.shape) for o in outs] for _ in range(2)]
+    host_out = [[o.new_empty(o.shape, device="cpu").pin_memory() for o in outs] for _ in range(2)]
+    in_free, out_free, h2d_done = [None, None], [None, None], [None, None]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def h2d(i):
+        b = i & 1
+        with torch.cuda.stream(sh):
+            if in_free[b] is not None:
+                sh.wait_event(in_free[b])
+            for (h, _), st in zip(ins, stg_in[b]):
+                st.copy_(h, non_blocking=True)
+            h2d_done[b] = torch.cuda.Event()
+            h2d_done[b].record(sh)
+
+    t0.record(cur)
+    sh.wait_stream(cur)
+    sd.wait_stream(cur)
+    h2d(0)
+    for i in range(steps):
+        b = i & 1
+        if i + 1 < steps:
+            h2d(i + 1)
+        cur.wait_event(h2d_done[b])
+        for (_, d), st in zip(ins, stg_in[b]):
+            d.copy_(st, non_blocking=True)
+        in_free[b] = torch.cuda.Event()
+        in_free[b].record(cur)
+        wl.step()
+        if out_free[b] is not None:
+            cur.wait_event(out_free[b])
+        for o, st in zip(outs, stg_out[b]):
+            st.copy_(o, non_blocking=True)
+        done = torch.cuda.Event()
+        done.record(cur)
+        with torch.cuda.stream(sd):
+            sd.wait_event(done)
+            for st, h in zip(stg_out[b], host_out[b]):
+                h.copy_(st, non_blocking=True)
+            out_free[b] = torch.cuda.Event()
+            out_free[b].record(sd)
+    cur.wait_stream(sh)
+    cur.wait_stream(sd)
+    t1.record(cur)
+    torch.cuda.synchronize()
+    return t0.elapsed_time(t1)
+
 
 class GzipWorkload:
     def __init__(self, sa, torch, w, backward, device_flags=False):
@@ -277,25 +332,12 @@ class GzipWorkload:
             if ev is not None:
                 ev[2].record()
 
-    def e2e_step(self):
-        """Host buffers in, result out: the public API with H2D/D2H copies."""
-        for t, h in self.h_in.items():
-            getattr(self, t).copy_(h, non_blocking=True)
-        if self.device_flags:
-            self.x.copy_(self.h_bytes, non_blocking=True)
-        else:
-            self.flags.copy_(self.h_flags, non_blocking=True)
-        self.step()
-        out = [self.o, self.lse] + ([self.dq, self.dk, self.dv] if self.backward else [])
-        return copy_out(out)
-
-    def io_bytes(self):
-        h2d = sum(x.numel() * x.element_size() for x in self.h_in.values()) + \
-            (self.h_bytes.numel() if self.device_flags else self.h_flags.numel())
-        d2h = self.o.numel() * 2 + self.lse.numel() * 4
-        if self.backward:
-            d2h += 3 * self.dq.numel() * 4
-        return h2d, d2h
+    def io_tensors(self):
+        """(host input, device input) pairs a step copies in, and the device
+        results it reads back."""
+        ins = [(h, getattr(self, t)) for t, h in self.h_in.items()]
+        ins.append((self.h_bytes, self.x) if self.device_flags else (self.h_flags, self.flags))
+        return ins, [self.o, self.lse] + ([self.dq, self.dk, self.dv] if self.backward else [])
 
     def cpu_baseline(self, heads=None):
         """The oracle on batch row 0, one head of each class (whole heads)."""
@@ -372,16 +414,9 @@ class GistWorkload(GzipWorkload):
         self.kernel = "fwd_tc_kernel"
         self.unit = "TFLOP/s"
 
-    def e2e_step(self):
-        for t, h in self.h_in.items():
-            getattr(self, t).copy_(h, non_blocking=True)
-        self.step()
-        return copy_out([self.o, self.lse] + ([self.dq, self.dk, self.dv] if self.backward else []))
-
-    def io_bytes(self):
-        h2d = sum(x.numel() * x.element_size() for x in self.h_in.values())
-        outs = [self.o, self.lse] + ([self.dq, self.dk, self.dv] if self.backward else [])
-        return h2d, sum(x.numel() * x.element_size() for x in outs)
+    def io_tensors(self):
+        ins = [(h, getattr(self, t)) for t, h in self.h_in.items()]
+        return ins, [self.o, self.lse] + ([self.dq, self.dk, self.dv] if self.backward else [])
 
     def cpu_baseline(self):
         from oracle import attention as A
@@ -515,14 +550,9 @@ class DecodeWorkload:
         if ev is not None:
             ev[1].record()
 
-    def e2e_step(self):
+    def io_tensors(self):
         # a decode step's input is the new token's query; the caches are resident
-        self.q.copy_(self.h_q, non_blocking=True)
-        self.step()
-        return copy_out([self.o, self.lse, self.sel])
-
-    def io_bytes(self):
-        return self.h_q.numel() * 2, self.o.numel() * 2 + self.lse.numel() * 4 + self.sel.numel() * 4
+        return [(self.h_q, self.q)], [self.o, self.lse, self.sel]
 
     def cpu_baseline(self, budget_s=10.0):
         from oracle import decode as D
@@ -608,14 +638,8 @@ class HierDecodeWorkload(DecodeWorkload):
         if ev is not None:
             ev[1].record()
 
-    def e2e_step(self):
-        self.q.copy_(self.h_q, non_blocking=True)
-        self.step()
-        return copy_out([self.o, self.lse, self.sel2, self.sel])
-
-    def io_bytes(self):
-        return (self.h_q.numel() * 2,
-                self.o.numel() * 2 + self.lse.numel() * 4 + (self.sel.numel() + self.sel2.numel()) * 4)
+    def io_tensors(self):
+        return [(self.h_q, self.q)], [self.o, self.lse, self.sel2, self.sel]
 
     def cpu_baseline(self, budget_s=10.0):
         from oracle import decode as D
@@ -665,13 +689,8 @@ class FlagsWorkload:
         if ev is not None:
             ev[1].record()
 
-    def e2e_step(self):
-        self.x.copy_(self.h_x, non_blocking=True)
-        self.step()
-        return copy_out([self.flags])
-
-    def io_bytes(self):
-        return self.h_x.numel(), self.flags.numel()
+    def io_tensors(self):
+        return [(self.h_x, self.x)], [self.flags]
 
     def cpu_baseline(self, budget_s=10.0):
         from oracle import deflate_size as F
@@ -865,19 +884,11 @@ def main():
               if getattr(wl, "backward", False) else None)
 
     # ---- end-to-end through the public API with host buffers
-    for _ in range(2):
-        wl.e2e_step()
-    torch.cuda.synchronize()
+    e2e_run(wl, torch, 2)
     barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(args.steps):
-        outs = wl.e2e_step()
-    e1.record()
-    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e2e_run(wl, torch, args.steps)) / args.steps
     barrier()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1)) / args.steps
-    h2d, d2h = wl.io_bytes()
+    h2d, d2h = io_bytes(wl)
 
     hbm, bf16, src = peaks()
     if wl.unit == "GB/s":
