@@ -197,9 +197,24 @@ def e2e_run(wl, torch, steps):
     come in and step i-1's results go out (PCIe both ways at once). Inputs land
     in a staging buffer and are copied on the device into the workload's
     tensors, results are copied out to a staging buffer before the next step
-    overwrites them. Returns the elapsed ms of all steps (CUDA events)."""
+    overwrites them. Steps that move under 16 MB run the copies in line on the
+    compute stream. Returns the elapsed ms of all steps (CUDA events)."""
     ins, outs = wl.io_tensors()
     cur = torch.cuda.current_stream()
+    if sum(io_bytes(wl)) < (16 << 20):
+        # a few KB per step (a decode token): staging would only add copies
+        host_out = [o.new_empty(o.shape, device="cpu").pin_memory() for o in outs]
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(cur)
+        for _ in range(steps):
+            for h, d in ins:
+                d.copy_(h, non_blocking=True)
+            wl.step()
+            for o, h in zip(outs, host_out):
+                h.copy_(o, non_blocking=True)
+        t1.record(cur)
+        torch.cuda.synchronize()
+        return t0.elapsed_time(t1)
     sh, sd = torch.cuda.Stream(), torch.cuda.Stream()
     stg_in = [[d.new_empty(d.shape) for _, d in ins] for _ in range(2)]
     stg_out = [[o.new_empty(o.shape) for o in outs] for _ in range(2)]

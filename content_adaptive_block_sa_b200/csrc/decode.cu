@@ -24,6 +24,8 @@
 //      tokens.
 //   4. combine the partials of every slice into O (bf16) and LSE (fp32).
 // Keys and values are read with 16-byte loads, 16 lanes per 256-byte row.
+#include <cuda.h>
+
 #include <mutex>
 
 #include "sa_common.cuh"
@@ -671,21 +673,43 @@ static __device__ __align__(256) unsigned char g_decode_scratch[kStaticDecodeScr
 constexpr int kMaxDevices = 64;
 static std::mutex g_scratch_mutex;
 static void* g_scratch_addr[kMaxDevices];
+static CUcontext g_scratch_ctx[kMaxDevices];
+
+// cuCtxGetCurrent through the runtime's driver entry point (no link to libcuda)
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+static CtxGetCurrentFn ctx_get_current() {
+  static const CtxGetCurrentFn fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      p = nullptr;
+    return reinterpret_cast<CtxGetCurrentFn>(p);
+  }();
+  return fn;
+}
 
 // Device address of the array on the current device. In host code the
-// array's name is only a stand-in, so the address is looked up once per
-// device (with that device current) and cached.
+// array's name is only a stand-in, so the address is looked up once per device
+// and context (with that device current) and cached; a new context on the
+// device (after cudaDeviceReset, for one) is looked up again.
 cudaError_t decode_scratch_address(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  CtxGetCurrentFn get = ctx_get_current();
+  if (get == nullptr) return cudaErrorNotSupported;
   std::lock_guard<std::mutex> lock(g_scratch_mutex);
-  if (g_scratch_addr[dev] == nullptr) {
+  CUcontext ctx = nullptr;
+  if (get(&ctx) != CUDA_SUCCESS) return cudaErrorUnknown;
+  if (ctx == nullptr || g_scratch_addr[dev] == nullptr || g_scratch_ctx[dev] != ctx) {
     void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_decode_scratch);
+    e = cudaGetSymbolAddress(&p, g_decode_scratch);  // (makes the device's context current)
     if (e != cudaSuccess) return e;
+    if (get(&ctx) != CUDA_SUCCESS) return cudaErrorUnknown;
     g_scratch_addr[dev] = p;
+    g_scratch_ctx[dev] = ctx;
   }
   *out = g_scratch_addr[dev];
   return cudaSuccess;

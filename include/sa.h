@@ -487,9 +487,9 @@ sa_status sa_gist_decode(const sa_decode_desc* desc, const void* q,
  *    return SA_ERR_WORKSPACE; use sa_gist_decode for them.
  *  - The first call on a device looks up the array's device address (with
  *    that device current) and caches it; make that first call before any
- *    stream capture. The cached address belongs to the device's context of
- *    that time: after cudaDeviceReset it is stale, so do not call this entry
- *    point again in a process that has reset the device.
+ *    stream capture. The address is cached per device and context: after
+ *    cudaDeviceReset (a new context) the next call looks it up again, so
+ *    that call, too, belongs outside a stream capture.
  *  - Every call on a device shares the one array, which keeps the last call's
  *    contents (its status word is cleared by each call). Calls that overlap on
  *    the GPU - on different streams, or from different host threads without
