@@ -769,10 +769,55 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
         };
         // top_k of scores[] into sel_s (ascending, -1 padded); returns the
         // number of eligible chunks taken
+        // top_k of at most 256 candidates (one or two per thread: the
+        // gist-of-gists selections, small flat decodes): every key goes to
+        // shared memory and each thread ranks its own by (key descending,
+        // index ascending) against all of them. Four group barriers, where
+        // the radix passes take about twenty; same result.
+        auto small_select = [&]() __attribute__((always_inline)) -> uint32_t {
+          uint32_t kk[2] = {0u, 0u};
+#pragma unroll
+          for (int t = 0; t < 2; ++t)
+            if (t < per && j0 + t < j1) {
+              kk[t] = key_of(j0 + t);
+              hist[j0 + t] = kk[t];
+            }
+          const int n4 = (sel_n + 3) >> 2;
+          for (int x = sel_n + r; x < 4 * n4; x += 128) hist[x] = 0u;  // zero keys rank nothing
+          ok = ok && gs(53);
+          const uint4* h4 = reinterpret_cast<const uint4*>(hist);
+          uint32_t take = 0u, cnt = 0u;
+#pragma unroll
+          for (int t = 0; t < 2; ++t) {
+            const uint32_t key = kk[t];
+            if (key == 0u) continue;
+            const int j = j0 + t;
+            uint32_t rank = 0u;
+#pragma unroll 4
+            for (int c = 0; c < n4; ++c) {
+              const uint4 v = h4[c];
+              rank += (v.x > key || (v.x == key && 4 * c < j)) ? 1u : 0u;
+              rank += (v.y > key || (v.y == key && 4 * c + 1 < j)) ? 1u : 0u;
+              rank += (v.z > key || (v.z == key && 4 * c + 2 < j)) ? 1u : 0u;
+              rank += (v.w > key || (v.w == key && 4 * c + 3 < j)) ? 1u : 0u;
+            }
+            if (rank < (uint32_t)sel_k) {
+              take |= 1u << t;
+              ++cnt;
+            }
+          }
+          uint32_t sel_total = 0u;
+          uint32_t off = group_exclusive_scan(cnt, r, scan, gs, ok, &sel_total);
+#pragma unroll
+          for (int t = 0; t < 2; ++t)
+            if ((take >> t) & 1u) sel_dst[off++] = value_of(j0 + t);
+          for (int x = r; x < sel_k; x += 128)
+            if (x >= (int)sel_total) sel_dst[x] = -1;
+          ok = ok && gs(35);  // (also orders hist's reads before its next writes)
+          return sel_total;
+        };
         auto radix_select = [&]() __attribute__((always_inline)) -> uint32_t {
-        // (with a few candidates per thread the radix passes are cheaper; the
-        // gist-of-gists selections have 1 or 2, and leave the list path out of
-        // that kernel's register budget)
+        if (per <= 2) return small_select();
         if constexpr (!HIER) {
           if (per >= 8 && per <= 32 && sel_k <= 128) {
             uint32_t total = 0u;
