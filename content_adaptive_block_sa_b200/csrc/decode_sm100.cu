@@ -122,7 +122,8 @@ constexpr uint32_t OFF_RED = OFF_SEL + kMaxTopK * 4;     // float [2][4 warps][k
 constexpr uint32_t OFF_SCAN = OFF_RED + 2 * 4 * kN * 4;  // uint32 [8] + misc
 constexpr uint32_t OFF_HMASK = OFF_SCAN + 64;            // uint8 [kMaxTopK]: heads per slot
 constexpr uint32_t OFF_SEL2 = OFF_HMASK + kMaxTopK;      // int32 [kMaxTopK]: kept groups
-constexpr uint32_t OFF_BARS = OFF_SEL2 + kMaxTopK * 4;
+constexpr uint32_t OFF_SIDX = OFF_SEL2 + kMaxTopK * 4;    // uint8 [256]: sorted candidate indices
+constexpr uint32_t OFF_BARS = OFF_SIDX + 256;
 constexpr uint32_t kSmemBytes = OFF_BARS + 256 + 1024;
 
 enum {
@@ -770,38 +771,91 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
         // top_k of scores[] into sel_s (ascending, -1 padded); returns the
         // number of eligible chunks taken
         // top_k of at most 256 candidates (one or two per thread: the
-        // gist-of-gists selections, small flat decodes): every key goes to
-        // shared memory and each thread ranks its own by (key descending,
-        // index ascending) against all of them. Four group barriers, where
-        // the radix passes take about twenty; same result.
+        // gist-of-gists selections, small flat decodes). Each warp sorts its
+        // 64 candidates in registers (bitonic, descending by key, ties to the
+        // lower index) into shared memory; a candidate's rank is its position
+        // in its warp's list plus a binary search in each other warp's list.
+        // Five group barriers, where the radix passes take about twenty; same
+        // result.
         auto small_select = [&]() __attribute__((always_inline)) -> uint32_t {
-          uint32_t kk[2] = {0u, 0u};
+          uint8_t* sidx = smem + OFF_SIDX;
+          uint32_t* flags = scan + 8;  // 256 bits: the taken candidates
+          // (key, 255 - index) packed: descending order is key descending,
+          // then index ascending; absent or ineligible candidates are 0
+          uint64_t x[2];
 #pragma unroll
-          for (int t = 0; t < 2; ++t)
-            if (t < per && j0 + t < j1) {
-              kk[t] = key_of(j0 + t);
-              hist[j0 + t] = kk[t];
+          for (int t = 0; t < 2; ++t) {
+            const int j = j0 + t;
+            const uint32_t key = (t < per && j < j1) ? key_of(j) : 0u;
+            x[t] = key ? ((uint64_t)key << 32) | (uint32_t)(255 - j) : 0ull;
+          }
+#pragma unroll
+          for (int size = 2; size <= 64; size <<= 1) {
+#pragma unroll
+            for (int stride = size >> 1; stride > 0; stride >>= 1) {
+              if (stride == 1) {  // both elements of the pair are this lane's
+                const bool desc = ((2 * lane) & size) == 0;
+                const uint64_t hi = x[0] > x[1] ? x[0] : x[1], lo = x[0] > x[1] ? x[1] : x[0];
+                x[0] = desc ? hi : lo;
+                x[1] = desc ? lo : hi;
+              } else {
+#pragma unroll
+                for (int t = 0; t < 2; ++t) {
+                  const int e = 2 * lane + t;
+                  const uint32_t yl = __shfl_xor_sync(0xffffffffu, (uint32_t)x[t], stride >> 1);
+                  const uint32_t yh = __shfl_xor_sync(0xffffffffu, (uint32_t)(x[t] >> 32), stride >> 1);
+                  const uint64_t y = ((uint64_t)yh << 32) | yl;
+                  const bool keep_max = ((e & stride) == 0) == ((e & size) == 0);
+                  x[t] = keep_max ? (x[t] > y ? x[t] : y) : (x[t] > y ? y : x[t]);
+                }
+              }
             }
-          const int n4 = (sel_n + 3) >> 2;
-          for (int x = sel_n + r; x < 4 * n4; x += 128) hist[x] = 0u;  // zero keys rank nothing
+          }
+#pragma unroll
+          for (int t = 0; t < 2; ++t) {
+            hist[sw * 64 + 2 * lane + t] = (uint32_t)(x[t] >> 32);
+            sidx[sw * 64 + 2 * lane + t] = (uint8_t)(uint32_t)x[t];
+          }
+          if (r < 8) flags[r] = 0u;
           ok = ok && gs(53);
-          const uint4* h4 = reinterpret_cast<const uint4*>(hist);
+          // entries of list w2 ranked above x[t]: a prefix of the descending
+          // list, found a bit at a time; the six searches (two elements, three
+          // other lists) advance together so that their loads overlap
+          auto above = [&](int w2, int i, uint64_t v) -> bool {
+            const uint32_t k2 = hist[w2 * 64 + i];
+            return k2 != 0u && (((uint64_t)k2 << 32) | sidx[w2 * 64 + i]) > v;
+          };
+          int pos[2][3] = {{0, 0, 0}, {0, 0, 0}};
+#pragma unroll
+          for (int step = 32; step >= 1; step >>= 1) {
+#pragma unroll
+            for (int t = 0; t < 2; ++t)
+#pragma unroll
+              for (int u = 0; u < 3; ++u) {
+                const int w2 = u + (u >= sw ? 1 : 0);
+                if (above(w2, pos[t][u] + step - 1, x[t])) pos[t][u] += step;
+              }
+          }
+#pragma unroll
+          for (int t = 0; t < 2; ++t) {
+            if (x[t] == 0ull) continue;
+            uint32_t rank = (uint32_t)(2 * lane + t);
+#pragma unroll
+            for (int u = 0; u < 3; ++u) {
+              const int w2 = u + (u >= sw ? 1 : 0);
+              rank += (uint32_t)(pos[t][u] == 63 && above(w2, 63, x[t]) ? 64 : pos[t][u]);
+            }
+            if (rank < (uint32_t)sel_k) {
+              const int j = 255 - (int)(uint32_t)(x[t] & 0xffu);
+              atomicOr(&flags[j >> 5], 1u << (j & 31));
+            }
+          }
+          ok = ok && gs(54);
           uint32_t take = 0u, cnt = 0u;
 #pragma unroll
           for (int t = 0; t < 2; ++t) {
-            const uint32_t key = kk[t];
-            if (key == 0u) continue;
             const int j = j0 + t;
-            uint32_t rank = 0u;
-#pragma unroll 4
-            for (int c = 0; c < n4; ++c) {
-              const uint4 v = h4[c];
-              rank += (v.x > key || (v.x == key && 4 * c < j)) ? 1u : 0u;
-              rank += (v.y > key || (v.y == key && 4 * c + 1 < j)) ? 1u : 0u;
-              rank += (v.z > key || (v.z == key && 4 * c + 2 < j)) ? 1u : 0u;
-              rank += (v.w > key || (v.w == key && 4 * c + 3 < j)) ? 1u : 0u;
-            }
-            if (rank < (uint32_t)sel_k) {
+            if (t < per && j < j1 && ((flags[j >> 5] >> (j & 31)) & 1u)) {
               take |= 1u << t;
               ++cnt;
             }
@@ -811,9 +865,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
 #pragma unroll
           for (int t = 0; t < 2; ++t)
             if ((take >> t) & 1u) sel_dst[off++] = value_of(j0 + t);
-          for (int x = r; x < sel_k; x += 128)
-            if (x >= (int)sel_total) sel_dst[x] = -1;
-          ok = ok && gs(35);  // (also orders hist's reads before its next writes)
+          for (int x2 = r; x2 < sel_k; x2 += 128)
+            if (x2 >= (int)sel_total) sel_dst[x2] = -1;
+          ok = ok && gs(35);  // (also orders hist's and the flags' reads before their next writes)
           return sel_total;
         };
         auto radix_select = [&]() __attribute__((always_inline)) -> uint32_t {
