@@ -125,7 +125,8 @@ struct Item {
 // tiles start at or below J (I = J .. J + c - 1: the start is non-decreasing
 // in I and at most nt - 1 tiles below it); gist far items, the query tiles
 // whose far-key prefix reaches past 128 J (a suffix of the query tiles, found
-// by bisection: far_ptr and the near start are non-decreasing).
+// by bisection: far_ptr and the near start are non-decreasing), visited from
+// the last tile down.
 struct Visits {
   int n, cnt, i0;
   __device__ void init(const MaskArgs& m, const Item& itm, int rep, int nt) {
@@ -158,8 +159,17 @@ struct Visits {
   __device__ void entry(const MaskArgs& m, const Item& itm, int rep, int it, int& h, int& I,
                         int& kind) const {
     if (m.kind == SA_MASK_GIST) {
-      h = itm.hk * rep + it / cnt;
-      I = i0 + it % cnt;
+      if (itm.far) {
+        // far items: query tiles from the last one down, the group's heads
+        // per tile. Every far item's suffix ends at the last query tile, so
+        // the far items that run together start on the same tiles and read
+        // their Q and dO rows from L2 while they stay in step.
+        I = m.T - 1 - it / rep;
+        h = itm.hk * rep + it % rep;
+      } else {
+        h = itm.hk * rep + it / cnt;
+        I = i0 + it % cnt;
+      }
       kind = SA_TILE_MASKED;
       return;
     }
