@@ -53,7 +53,7 @@ struct BwdTcParams {
 
 namespace bwd {
 
-constexpr int kSlots = 2;             // mask ring depth
+constexpr int kSlots = 8;             // mask ring depth (visits the mask warp may run ahead)
 constexpr uint32_t kSlotBytes = 2048;  // [4 words][128 key rows]
 constexpr int kCompute = 256;          // compute threads
 constexpr int kThreads = 64 + kCompute + 32;
@@ -67,24 +67,23 @@ struct Layout {
   static constexpr uint32_t k = 0;
   static constexpr uint32_t v = kT;
   static constexpr uint32_t q = 2 * kT;           // 2 stages
-  static constexpr uint32_t dO = 4 * kT;
-  static constexpr uint32_t dst = 5 * kT;         // dS^T [keys][queries]
-  static constexpr uint32_t rowv = 5 * kT + kP;   // [2 stages][lse2 128 | delta 128] fp32
+  static constexpr uint32_t dO = 4 * kT;          // 2 stages
+  static constexpr uint32_t rowv = 6 * kT;        // [2 stages][lse2 128 | delta 128] fp32
   static constexpr uint32_t mask = rowv + 2 * 1024;
-  static constexpr uint32_t hdr = mask + kSlots * kSlotBytes;  // [slot] {h, I}
+  static constexpr uint32_t hdr = mask + kSlots * kSlotBytes;  // the item ring's slots
   static constexpr uint32_t bars = hdr + 64;
   static constexpr uint32_t bytes = bars + 512 + 1024;
 };
 
 // mbarriers. KVF/KVE: K, V of the item loaded / no longer read. QF/QE: Q
-// stage (with its LSE and D rows) full / free. DOF/DOE: dO full / free. SF,
-// DPF: S^T, dP^T in TMEM. PF1: P^T written to TMEM; PF2: dS^T written to
-// shared memory. MF/ME: mask slot full / read. OI: every MMA of the item done.
-// OF: dV and dK of the item read out. DRAIN: all MMAs done.
+// stage (with its LSE and D rows) full / free. DOF/DOE: dO stage full / free.
+// SF, DPF: S^T, dP^T in TMEM. PF1: P^T written to TMEM over S^T; PF2: dS^T
+// written to TMEM over dP^T. MF/ME: mask slot full / read. OI: every MMA of
+// the item done. OF: dV and dK of the item read out. DRAIN: all MMAs done.
 enum {
-  B_KVF = 0, B_KVE = 1, B_QF = 2, B_QE = 4, B_DOF = 6, B_DOE = 7, B_SF = 8, B_DPF = 9, B_PF1 = 10,
-  B_PF2 = 11, B_OI = 12, B_MF = 14, B_ME = 16, B_OF = 18, B_DRAIN = 21, B_IQF = 22,
-  B_IQE = B_IQF + kItemRing, kNumBars = B_IQE + kItemRing
+  B_KVF = 0, B_KVE = 1, B_QF = 2, B_QE = 4, B_DOF = 6, B_DOE = 8, B_SF = 10, B_DPF = 11,
+  B_PF1 = 12, B_PF2 = 13, B_OI = 14, B_MF = 16, B_ME = B_MF + kSlots, B_OF = B_ME + kSlots,
+  B_DRAIN = B_OF + 1, B_IQF = B_DRAIN + 1, B_IQE = B_IQF + kItemRing, kNumBars = B_IQE + kItemRing
 };
 // consumers of each item of the run-time queue: the MMA thread, the mask warp
 // and the eight compute warps
@@ -252,11 +251,15 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bar[B_QF + s], 1);
       mbar_init(&bar[B_QE + s], 1);
+    }
+    for (int s = 0; s < kSlots; ++s) {
       mbar_init(&bar[B_MF + s], 32);
       mbar_init(&bar[B_ME + s], kCompute);
     }
-    mbar_init(&bar[B_DOF], 1);
-    mbar_init(&bar[B_DOE], 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bar[B_DOF + s], 1);
+      mbar_init(&bar[B_DOE + s], 1);
+    }
     mbar_init(&bar[B_SF], 1);
     mbar_init(&bar[B_DPF], 1);
     mbar_init(&bar[B_PF1], kCompute);
@@ -334,14 +337,14 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
           bulk_load(rowv + s * 256, P.lse2 + ro, 512, &bar[B_QF + s]);
           bulk_load(rowv + s * 256 + 128, P.delta + ro, 512, &bar[B_QF + s]);
           last_q = gt;
-          if (!mbar_wait(&bar[B_DOE], (gt & 1) ^ 1, abort, st, 102)) {
+          if (!mbar_wait(&bar[B_DOE + s], ((gt >> 1) & 1) ^ 1, abort, st, 102)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&bar[B_DOF], L::kT);
+          mbar_arrive_expect_tx(&bar[B_DOF + s], L::kT);
           for (int at = 0; at < D / 64; ++at)
-            tma_load_4d(smem + L::dO + at * L::kAtom, &P.tmdo, &bar[B_DOF], at * 64, h, I * kTile,
-                        itm.bt);
+            tma_load_4d(smem + L::dO + s * L::kT + at * L::kAtom, &P.tmdo, &bar[B_DOF + s], at * 64, h,
+                        I * kTile, itm.bt);
           last_do = gt;
         }
         if (ok) count_tiles(st, CNT_DKDV_VISITS, vis.n);
@@ -356,7 +359,11 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
           const int gs = last_q - ((last_q - s) & 1);
           mbar_wait(&bar[B_QF + s], (gs >> 1) & 1, &no_abort, nullptr, 104);
         }
-      if (last_do >= 0) mbar_wait(&bar[B_DOF], last_do & 1, &no_abort, nullptr, 105);
+      for (int s = 0; s < 2; ++s)
+        if (last_do >= s) {
+          const int gs = last_do - ((last_do - s) & 1);
+          mbar_wait(&bar[B_DOF + s], (gs >> 1) & 1, &no_abort, nullptr, 105);
+        }
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -368,7 +375,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
       // Per visit gt the order is: dV(gt) once P^T is written, then S^T(gt + 1)
       // (its S columns held P^T(gt), read by the dV just issued: tcgen05.mma ops
       // of one thread run in order), dK(gt) once dS^T is written, then
-      // dP^T(gt + 1) (dS^T(gt) being written means dP^T(gt) has been read).
+      // dP^T(gt + 1) (its columns held dS^T(gt), read by the dK just issued).
+      // dO has two stages, so dO(gt + 1) loads while visit gt runs.
       auto issue_s = [&](int gt) -> bool {  // S^T = K Q^T
         const int s = gt & 1;
         if (!mbar_wait(&bar[B_QF + s], (gt >> 1) & 1, abort, st, 111)) return false;
@@ -384,13 +392,14 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
         return true;
       };
       auto issue_dp = [&](int gt) -> bool {  // dP^T = V dO^T
-        if (!mbar_wait(&bar[B_DOF], gt & 1, abort, st, 112)) return false;
+        const int d = gt & 1;
+        if (!mbar_wait(&bar[B_DOF + d], (gt >> 1) & 1, abort, st, 112)) return false;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * L::kAtom + (kk & 3) * 32;
           mma_bf16(tmem + kColDP, smem_desc_sw128(sb + L::v + off, 16, 1024),
-                   smem_desc_sw128(sb + L::dO + off, 16, 1024), kIdS, kk > 0);
+                   smem_desc_sw128(sb + L::dO + d * L::kT + off, 16, 1024), kIdS, kk > 0);
         }
         mma_commit(&bar[B_DPF]);
         return true;
@@ -420,15 +429,16 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {  // K = 128 queries
             const uint32_t pa = tmem + kColS + (kk >> 2) * 64 + (kk & 3) * 8;
-            mma_bf16_ts(tmem + kColDV, pa, smem_desc_sw128(sb + L::dO + kk * 2048, L::kAtom, 1024),
-                        kIdAcc, (it > 0 || kk > 0) ? 1u : 0u);
+            mma_bf16_ts(tmem + kColDV, pa,
+                        smem_desc_sw128(sb + L::dO + s * L::kT + kk * 2048, L::kAtom, 1024), kIdAcc,
+                        (it > 0 || kk > 0) ? 1u : 0u);
           }
-          mma_commit(&bar[B_DOE]);
+          mma_commit(&bar[B_DOE + s]);
           if (more && !issue_s(gt + 1)) {
             ok = false;
             break;
           }
-          // dS^T in shared memory: dK += dS^T Q
+          // dS^T in TMEM (over dP^T): dK += dS^T Q
           if (!mbar_wait(&bar[B_PF2], gt & 1, abort, st, 117)) {
             ok = false;
             break;
@@ -436,11 +446,10 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
           tc_fence_after();
           const uint32_t qb = sb + L::q + s * L::kT;
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t aoff = (kk >> 2) * L::kAtom + (kk & 3) * 32;
-            mma_bf16(tmem + kColDV + D, smem_desc_sw128(sb + L::dst + aoff, 16, 1024),
-                     smem_desc_sw128(qb + kk * 2048, L::kAtom, 1024), kIdAcc,
-                     (it > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < 8; ++kk) {  // K = 128 queries
+            const uint32_t da = tmem + kColDP + (kk >> 2) * 64 + (kk & 3) * 8;
+            mma_bf16_ts(tmem + kColDV + D, da, smem_desc_sw128(qb + kk * 2048, L::kAtom, 1024),
+                        kIdAcc, (it > 0 || kk > 0) ? 1u : 0u);
           }
           mma_commit(&bar[B_QE + s]);
           if (more && !issue_dp(gt + 1)) {
@@ -475,18 +484,15 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
       vis.init(m, itm, rep, P.near_nt);
       bool ok = true;
       for (int it = 0; it < vis.n; ++it) {
-        const int gt = g + it, s = gt & 1;
-        if (!__all_sync(0xffffffffu, mbar_wait(&bar[B_ME + s], ((gt >> 1) & 1) ^ 1, abort, st, 130))) {
+        const int gt = g + it, s = gt % kSlots;
+        if (!__all_sync(0xffffffffu,
+                        mbar_wait(&bar[B_ME + s], ((gt / kSlots) & 1) ^ 1, abort, st, 130))) {
           ok = false;
           break;
         }
         int h, I, kind;
         vis.entry(m, itm, rep, it, h, I, kind);
         const int list = list_of(m, itm.bt, h);
-        if (lane == 0) {
-          hdr[2 * s] = h;
-          hdr[2 * s + 1] = I;
-        }
         uint32_t* words = mwords + s * (kSlotBytes / 4);
         const int q0 = I * kTile;
         if (gist && !itm.far) {
@@ -567,17 +573,17 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
       vis.init(m, itm, rep, P.near_nt);
       const int kq = itm.J * kTile + r;  // this thread's key row
       for (int it = 0; it < vis.n; ++it) {
-        const int gt = g + it, s = gt & 1;
+        const int gt = g + it, s = gt & 1, ms = gt % kSlots;
         // phase 1: P from S^T (needs only S^T and the stored LSE)
-        if (!__all_sync(0xffffffffu, mbar_wait(&bar[B_SF], gt & 1, abort, st, 120) &&
-                                         mbar_wait(&bar[B_MF + s], (gt >> 1) & 1, abort, st, 121))) {
+        if (!__all_sync(0xffffffffu,
+                        mbar_wait(&bar[B_SF], gt & 1, abort, st, 120) &&
+                            mbar_wait(&bar[B_MF + ms], (gt / kSlots) & 1, abort, st, 121))) {
           ok = false;
           break;
         }
-        const uint32_t* words = mwords + s * (kSlotBytes / 4);
+        const uint32_t* words = mwords + ms * (kSlotBytes / 4);
         const uint32_t mw[2] = {words[(2 * half) * 128 + r], words[(2 * half + 1) * 128 + r]};
-        const int h = hdr[2 * s], I = hdr[2 * s + 1];
-        mbar_arrive(&bar[B_ME + s]);
+        mbar_arrive(&bar[B_ME + ms]);
         const float* lse2 = rowv + s * 256 + half * 64;
         const float* dlt = lse2 + 128;
         tc_fence_after();
@@ -619,20 +625,20 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
         tc_fence_before();
         mbar_arrive(&bar[B_PF1]);
         // phase 2: dS = P (dP - D) into dS^T (key row r, this half's 64 query
-        // columns); the previous dS^T was read by MMAs that finished before
-        // dP^T of this visit
+        // columns), bf16 pairs over the first 32 of this half's dP^T columns
+        // once all 64 are read
         if (!__all_sync(0xffffffffu, mbar_wait(&bar[B_DPF], gt & 1, abort, st, 122))) {
           ok = false;
           break;
         }
         tc_fence_after();
         __syncwarp();
+        uint32_t dsk[32];
 #pragma unroll
         for (int c2 = 0; c2 < 2; ++c2) {  // 32 query columns at a time
           float dv[32];
           tmem_ld32(lane_addr + kColDP + half * 64 + c2 * 32, dv);
           tmem_wait_ld();
-          uint32_t dk[16];
 #pragma unroll
           for (int c = 0; c < 32; c += 4) {
             const int i = c2 * 32 + c;
@@ -641,16 +647,13 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
                                     fadd2(make_float2(dv[c], dv[c + 1]), make_float2(-d4.x, -d4.y)));
             const float2 s1 = fmul2(make_float2(pv[i + 2], pv[i + 3]),
                                     fadd2(make_float2(dv[c + 2], dv[c + 3]), make_float2(-d4.z, -d4.w)));
-            dk[c >> 1] = pack_bf16(s0.x, s0.y);
-            dk[(c >> 1) + 1] = pack_bf16(s1.x, s1.y);
+            dsk[i >> 1] = pack_bf16(s0.x, s0.y);
+            dsk[(i >> 1) + 1] = pack_bf16(s1.x, s1.y);
           }
-          const uint32_t base = sb + L::dst + half * L::kAtom;
-#pragma unroll
-          for (int ch = 0; ch < 4; ++ch)
-            st_shared_v4(base + sw128_offset(r, c2 * 32 + ch * 8), dk[ch * 4], dk[ch * 4 + 1],
-                         dk[ch * 4 + 2], dk[ch * 4 + 3]);
         }
-        fence_async_shared();
+        __syncwarp();
+        tmem_st32(lane_addr + kColDP + half * 64, reinterpret_cast<const float*>(dsk));
+        tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&bar[B_PF2]);
       }
