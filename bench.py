@@ -679,8 +679,9 @@ class HierDecodeWorkload(DecodeWorkload):
 
 
 class FlagsWorkload:
-    """On-device literal flags (fixed-Huffman DEFLATE size estimate per block,
-    then the mean rule) over rows of bytes already in HBM."""
+    """On-device literal flags (each block's DEFLATE size, the smallest of a
+    fixed, dynamic or stored block, then the mean rule) over rows of bytes
+    already in HBM."""
 
     def __init__(self, sa, torch, w):
         self.sa, self.torch, self.w = sa, torch, w
