@@ -58,3 +58,34 @@ def test_random_text_and_degenerate_blocks(sa, b):
             (b"the cat sat on the mat. " * (n // 24 + 1))[:n],         # periodic text
             rng.integers(0, 3, n, dtype=np.uint8).tobytes()]           # three symbols
     check(sa, rows, b)
+
+
+def _zipf_rows(b, n_rows=2, seed=0):
+    """Bytes drawn from a Zipf law over a shuffled alphabet: few matches and a
+    wide spread of literal counts, so the code-length code of some blocks is
+    deeper than 7 bits and needs package-merge."""
+    rng = np.random.default_rng(seed)
+    rows = []
+    for a in np.linspace(0.75, 1.6, n_rows):
+        p = 1.0 / np.arange(1, 257) ** a
+        perm = rng.permutation(256)
+        rows.append(perm[rng.choice(256, b * 24, p=p / p.sum())].astype(np.uint8).tobytes())
+    return rows
+
+
+def _code_length_code_depth(block):
+    # the unlimited Huffman depth of the block's code-length code
+    _, _, _, _, _, runs, _, _ = F.dynamic_code(block)
+    cf = [0] * 19
+    for sym, _, _ in runs:
+        cf[sym] += 1
+    return max(F.huffman_lengths(cf, 99))
+
+
+@pytest.mark.parametrize("b", [256, 1000, 1024])
+def test_zipf_bytes_package_merge(sa, b):
+    rows = _zipf_rows(b, seed=b)
+    depths = [_code_length_code_depth(r[i:i + b]) for r in rows for i in range(0, len(r), b)]
+    if b >= 1000:
+        assert max(depths) > 7  # the limited code-length code is reached
+    check(sa, rows, b)
