@@ -66,7 +66,7 @@ def test_nvml_samples(monkeypatch):
     assert out["reasons"] == ["hw_slowdown", "sw_power_cap"]  # idle is not a reason kept
     assert out["samples"] >= len(samples)
     assert out["source"].startswith("nvml")
-    # the repeated last sample (1700) can only pull the median down to 1800 or 1700
+    # the five samples' median is 1900; repeats of the last one (1700) pull it to 1800 or 1700
     assert out["sm_mhz"] in (1700.0, 1800.0, 1900.0)
 
 
